@@ -1,0 +1,415 @@
+"""CPU oracle of the TTT-E2E inner loop (prefill and decode).
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path imports this module:
+only the tests, the package's smoke check and the benchmark's CPU-baseline leg
+call it. It shares no code with the CUDA library.
+
+What it computes follows the pages describing End-to-End Test-Time Training
+(TTT-E2E) for long context:
+  * per-token loss l_t(W) = CE(f(x_{t-1}; W), x_t)
+      - b-lab.team summary, "Test-Time Training (Inner Loop)", loss equation;
+      - technical review §3, eq. (3);
+  * mini-batch GD W_i = W_{i-1} - eta * (1/b) * sum_k grad l_k(W_{i-1}), every
+    target of chunk i scored with W_{i-1} before the update
+      - summary, "Mini-Batch Gradient Descent"; review §5, eq. (9);
+  * sliding-window attention with k >= b, causal inside the chunk
+      - summary, "Integration with Sliding-Window Attention"; review §5;
+  * only the MLPs of the last quarter of the blocks update; a static second MLP
+    follows the adaptive one in those blocks; embeddings, norms and attention
+    are frozen - summary, "Implementation Details for TTT"; review §6;
+  * Algorithm 1 (causal prefill with adaptation) and Algorithm 3 (generation
+    with periodic adaptation, update after a full mini-batch of generated
+    tokens) - review §7; per-sequence fresh copy of the fast weights -
+    review §7, Algorithm 1 step 1.
+
+Readings taken where the pages are silent (each also listed in the design doc):
+  R1 T+1 ids x_0..x_T in, T positions processed, out_losses[t-1] = l_t.
+  R2 query at position p attends to keys [p-k+1, p]; k >= T is full attention.
+  R3 K/V cached from earlier chunks are constants: gradients flow only through
+     the current chunk's K/V. They hold the values computed when their chunk
+     was processed (with that step's weights) and are never recomputed.
+  R4 both TTT-MLP matrices (W1t, W2t) update; no biases anywhere.
+  R5 pre-norm blocks; adaptive block = attention, TTT-MLP, static MLP, each
+     with its own RMSNorm gain and residual.
+  R6 final RMSNorm then the tied LM head z = E r.
+  R7 exact GELU 0.5u(1+erf(u/sqrt2)); RMSNorm y = g x / sqrt(mean(x^2)+eps).
+  R8 RoPE rotate-half pairing (i, i+hd/2), theta_i = base^(-2i/hd), absolute
+     positions; scale 1/sqrt(hd); softmax without bias or dropout.
+  R9 one constant eta for every adaptive block; the chunk loss is the mean
+     over its b positions; sequences are independent (no 1/B).
+  R10 a trailing partial chunk is scored but not used for an update; its
+     positions stay pending until later positions (decode) complete it.
+  R11 greedy decode takes the lowest id among equal maxima; decode's loss
+     output is -log p(chosen token) under the weights in force.
+
+Arithmetic is float64 throughout. Matrix products use numpy's matmul as the
+library primitive. Queries are processed in groups only to bound memory; each
+row is the plain definition. This oracle is pinned by the tests in
+tests/test_oracle_pins.py (finite differences, an independent whole-sequence
+forward and autograd, and the special cases eta=0, k>=T, b=T, b=1).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy.special import erf
+
+__all__ = ["Oracle", "rms_norm", "rms_norm_backward", "gelu", "gelu_prime", "rope",
+           "rope_backward", "rope_tables", "window_attention", "window_attention_backward"]
+
+
+# ----------------------------------------------------------------------------- primitives
+
+def rms_norm(x, g, eps):
+    """RMSNorm (reading R7): y = g * x / sqrt(mean(x^2) + eps). Returns (y, rstd)."""
+    rstd = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return g * x * rstd, rstd
+
+
+def rms_norm_backward(x, g, rstd, dy):
+    """Derivative of rms_norm w.r.t. x for upstream dy (g and eps are frozen)."""
+    n = x.shape[-1]
+    gdy = g * dy
+    dot = np.sum(gdy * x, axis=-1, keepdims=True)
+    return rstd * gdy - x * (rstd ** 3) * dot / n
+
+
+def gelu(u):
+    """Exact GELU (reading R7)."""
+    return 0.5 * u * (1.0 + erf(u / math.sqrt(2.0)))
+
+
+def gelu_prime(u):
+    """d gelu / du = Phi(u) + u * phi(u)."""
+    return 0.5 * (1.0 + erf(u / math.sqrt(2.0))) + u * np.exp(-0.5 * u * u) / math.sqrt(2.0 * math.pi)
+
+
+def rope_tables(positions, hd, base):
+    """cos/sin [n, hd/2] of angle p * base^(-2i/hd) (reading R8)."""
+    i = np.arange(hd // 2, dtype=np.float64)
+    theta = base ** (-2.0 * i / hd)
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * theta[None, :]
+    return np.cos(ang), np.sin(ang)
+
+
+def rope(x, cos, sin):
+    """Rotate pairs (i, i+hd/2) of x [n, H, hd] by the per-position angles."""
+    h = x.shape[-1] // 2
+    x1, x2 = x[..., :h], x[..., h:]
+    c, s = cos[:, None, :], sin[:, None, :]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def rope_backward(dy, cos, sin):
+    """Transpose (= inverse) of the rotation applied by rope()."""
+    h = dy.shape[-1] // 2
+    d1, d2 = dy[..., :h], dy[..., h:]
+    c, s = cos[:, None, :], sin[:, None, :]
+    return np.concatenate([d1 * c + d2 * s, d2 * c - d1 * s], axis=-1)
+
+
+def _window_mask(q_pos, k_pos, window):
+    qp = np.asarray(q_pos)[:, None]
+    kp = np.asarray(k_pos)[None, :]
+    return (kp <= qp) & (kp >= qp - window + 1)
+
+
+def window_attention(q, keys, vals, q_pos, k_pos, window, keep_probs=False, group=512):
+    """Causal sliding-window softmax attention (reading R2, R8).
+
+    q [n, H, hd] at positions q_pos; keys/vals [m, H, hd] at positions k_pos.
+    Query p uses the keys with p-window+1 <= position <= p; k_pos is ascending.
+    Returns o [n, H, hd]
+    and, if keep_probs, the probabilities [H, n, m].
+    """
+    n, H, hd = q.shape
+    scale = 1.0 / math.sqrt(hd)
+    o = np.empty_like(q)
+    probs = np.empty((H, n, keys.shape[0])) if keep_probs else None
+    k_pos = np.asarray(k_pos)
+    for g0 in range(0, n, group):
+        g1 = min(n, g0 + group)
+        # keys outside [first query - window + 1, last query] are masked for every
+        # query of the group, so they are skipped (their probability is exactly 0)
+        lo = int(np.searchsorted(k_pos, q_pos[g0] - window + 1, side="left"))
+        hi = int(np.searchsorted(k_pos, q_pos[g1 - 1], side="right"))
+        mask = _window_mask(q_pos[g0:g1], k_pos[lo:hi], window)
+        for h in range(H):
+            s = (q[g0:g1, h, :] @ keys[lo:hi, h, :].T) * scale
+            s = np.where(mask, s, -np.inf)
+            s = s - s.max(axis=1, keepdims=True)
+            p = np.exp(s)
+            p /= p.sum(axis=1, keepdims=True)
+            o[g0:g1, h, :] = p @ vals[lo:hi, h, :]
+            if keep_probs:
+                probs[h, g0:g1, :] = 0.0
+                probs[h, g0:g1, lo:hi] = p
+    return o, probs
+
+
+def window_attention_backward(q, keys, vals, o, probs, do):
+    """Gradients of window_attention w.r.t. q, keys and vals (all keys given)."""
+    n, H, hd = q.shape
+    scale = 1.0 / math.sqrt(hd)
+    dq = np.empty_like(q)
+    dk = np.empty_like(keys)
+    dv = np.empty_like(vals)
+    for h in range(H):
+        p = probs[h]
+        dp = do[:, h, :] @ vals[:, h, :].T
+        dsum = np.sum(do[:, h, :] * o[:, h, :], axis=1, keepdims=True)
+        ds = p * (dp - dsum)
+        dq[:, h, :] = (ds @ keys[:, h, :]) * scale
+        dk[:, h, :] = (ds.T @ q[:, h, :]) * scale
+        dv[:, h, :] = p.T @ do[:, h, :]
+    return dq, dk, dv
+
+
+def _logsumexp(z):
+    m = z.max(axis=-1, keepdims=True)
+    return (m + np.log(np.sum(np.exp(z - m), axis=-1, keepdims=True)))[..., 0]
+
+
+# ----------------------------------------------------------------------------- state
+
+class _History:
+    """Post-RoPE keys and values of every processed position of one layer."""
+
+    def __init__(self, H, hd):
+        self.K = np.empty((0, H, hd))
+        self.V = np.empty((0, H, hd))
+
+    def append(self, k, v):
+        self.K = np.concatenate([self.K, k], axis=0)
+        self.V = np.concatenate([self.V, v], axis=0)
+
+
+class _Seq:
+    """Per-sequence state: a fresh copy of the fast weights (review §7, Alg. 1 step 1)."""
+
+    def __init__(self, cfg, w0):
+        self.fast = [{"W1t": w0[f"layers.{l}.W1t"].copy(), "W2t": w0[f"layers.{l}.W2t"].copy()}
+                     for l in range(cfg.first_ttt, cfg.n_layers)]
+        self.hist = [_History(cfg.n_heads, cfg.head_dim) for _ in range(cfg.n_layers)]
+        self.n_pos = 0
+        self.pending_token = None
+        self.pend_inputs = []
+        self.pend_targets = []
+
+
+class Oracle:
+    """Plain implementation of Algorithms 1 and 3 for B independent sequences."""
+
+    def __init__(self, cfg, weights):
+        self.cfg = cfg
+        self.w = {k: np.asarray(v, dtype=np.float64) for k, v in weights.items()}
+        self.reset()
+
+    def reset(self):
+        self.seqs = [_Seq(self.cfg, self.w) for _ in range(self.cfg.batch)]
+
+    # --------------------------------------------------------------- blocks
+    def _attn(self, seq, l, x, s, commit, keep):
+        """Pre-norm attention sub-block of layer l for positions [s, s+n)."""
+        cfg, w, p = self.cfg, self.w, f"layers.{l}."
+        n, H, hd = x.shape[0], cfg.n_heads, cfg.head_dim
+        r1, rstd1 = rms_norm(x, w[p + "attn_norm"], cfg.rms_eps)
+        pos = np.arange(s, s + n)
+        cos, sin = rope_tables(pos, hd, cfg.rope_base)
+        q = rope((r1 @ w[p + "Wq"].T).reshape(n, H, hd), cos, sin)
+        k = rope((r1 @ w[p + "Wk"].T).reshape(n, H, hd), cos, sin)
+        v = (r1 @ w[p + "Wv"].T).reshape(n, H, hd)
+        hist = seq.hist[l]
+        lo = max(0, s - cfg.window_k + 1)
+        keys = np.concatenate([hist.K[lo:s], k], axis=0)
+        vals = np.concatenate([hist.V[lo:s], v], axis=0)
+        k_pos = np.arange(lo, s + n)
+        o, probs = window_attention(q, keys, vals, pos, k_pos, cfg.window_k, keep_probs=keep)
+        a = x + o.reshape(n, -1) @ w[p + "Wo"].T
+        if commit:
+            hist.append(k, v)
+        cache = dict(x=x, rstd1=rstd1, q=q, keys=keys, vals=vals, o=o, probs=probs,
+                     n_cached=s - lo, cos=cos, sin=sin) if keep else None
+        return a, cache
+
+    def _frozen_block(self, seq, l, x, s, commit):
+        cfg, w, p = self.cfg, self.w, f"layers.{l}."
+        a, _ = self._attn(seq, l, x, s, commit, keep=False)
+        r2, _ = rms_norm(a, w[p + "mlp_norm"], cfg.rms_eps)
+        return a + gelu(r2 @ w[p + "W1"].T) @ w[p + "W2"].T
+
+    def _ttt_block(self, seq, j, x, s, commit, keep):
+        """Adaptive block j: attention, TTT-MLP with fast weights, static MLP (reading R5)."""
+        cfg, w = self.cfg, self.w
+        l = cfg.first_ttt + j
+        p = f"layers.{l}."
+        fw = seq.fast[j]
+        a, c = self._attn(seq, l, x, s, commit, keep)
+        r2, rstd2 = rms_norm(a, w[p + "ttt_norm"], cfg.rms_eps)
+        u = r2 @ fw["W1t"].T
+        g = gelu(u)
+        m = a + g @ fw["W2t"].T
+        r3, rstd3 = rms_norm(m, w[p + "static_norm"], cfg.rms_eps)
+        us = r3 @ w[p + "W1s"].T
+        y = m + gelu(us) @ w[p + "W2s"].T
+        if keep:
+            c.update(a=a, rstd2=rstd2, r2=r2, u=u, g=g, m=m, rstd3=rstd3, us=us)
+        return y, c
+
+    def _head(self, y):
+        """Final RMSNorm and tied LM head (reading R6)."""
+        rf, rstdf = rms_norm(y, self.w["final_norm"], self.cfg.rms_eps)
+        return rf @ self.w["E"].T, rf, rstdf
+
+    def _frozen_forward(self, seq, tokens_in, s, commit):
+        x = self.w["E"][np.asarray(tokens_in)]
+        for l in range(self.cfg.first_ttt):
+            x = self._frozen_block(seq, l, x, s, commit)
+        return x
+
+    # --------------------------------------------------------------- one chunk
+    def _chunk(self, seq, h_in, s, targets, need_grad, commit):
+        """Forward the adaptive blocks for positions [s, s+n) with the weights in force.
+
+        Returns the per-position losses, the fast-weight gradients of the chunk's
+        mean loss (if need_grad) and nothing else; commits K/V when asked.
+        """
+        cfg, w = self.cfg, self.w
+        n = h_in.shape[0]
+        y = h_in
+        caches = []
+        for j in range(cfg.n_ttt):
+            y, c = self._ttt_block(seq, j, y, s, commit, keep=need_grad)
+            caches.append(c)
+        z, rf, rstdf = self._head(y)
+        t = np.asarray(targets)
+        lse = _logsumexp(z)
+        losses = lse - z[np.arange(n), t]
+        if not need_grad:
+            return losses, None
+        # mean over the b positions of the chunk (reading R9)
+        pz = np.exp(z - lse[:, None])
+        pz[np.arange(n), t] -= 1.0
+        dz = pz / cfg.minibatch_b
+        dy = rms_norm_backward(y, w["final_norm"], rstdf, dz @ w["E"])
+        grads = [None] * cfg.n_ttt
+        for j in reversed(range(cfg.n_ttt)):
+            c = caches[j]
+            l = cfg.first_ttt + j
+            p = f"layers.{l}."
+            fw = seq.fast[j]
+            # static MLP (frozen): only the data gradient
+            dus = (dy @ w[p + "W2s"]) * gelu_prime(c["us"])
+            dm = dy + rms_norm_backward(c["m"], w[p + "static_norm"], c["rstd3"], dus @ w[p + "W1s"])
+            # TTT-MLP: weight gradients and data gradient, all at W_{i-1}
+            dW2t = dm.T @ c["g"]
+            du = (dm @ fw["W2t"]) * gelu_prime(c["u"])
+            dW1t = du.T @ c["r2"]
+            grads[j] = {"W1t": dW1t, "W2t": dW2t}
+            if j == 0:
+                break  # upstream of the first adaptive MLP does not depend on W
+            da = dm + rms_norm_backward(c["a"], w[p + "ttt_norm"], c["rstd2"], du @ fw["W1t"])
+            # frozen attention: data gradients; cached keys are constants (reading R3)
+            do = (da @ w[p + "Wo"]).reshape(n, cfg.n_heads, cfg.head_dim)
+            dq, dk_all, dv_all = window_attention_backward(c["q"], c["keys"], c["vals"], c["o"], c["probs"], do)
+            nc = c["n_cached"]
+            dq = rope_backward(dq, c["cos"], c["sin"]).reshape(n, -1)
+            dk = rope_backward(dk_all[nc:], c["cos"], c["sin"]).reshape(n, -1)
+            dv = dv_all[nc:].reshape(n, -1)
+            dr1 = dq @ w[p + "Wq"] + dk @ w[p + "Wk"] + dv @ w[p + "Wv"]
+            dy = da + rms_norm_backward(c["x"], w[p + "attn_norm"], c["rstd1"], dr1)
+        return losses, grads
+
+    def _sgd(self, seq, grads):
+        """W_i = W_{i-1} - eta * mean-gradient (summary, mini-batch GD equation)."""
+        for j, g in enumerate(grads):
+            for name in ("W1t", "W2t"):
+                seq.fast[j][name] = seq.fast[j][name] - self.cfg.eta * g[name]
+
+    # --------------------------------------------------------------- Algorithm 1
+    def prefill(self, tokens):
+        """tokens [B][T+1] -> losses [B][T] (reading R1). Updates the state."""
+        cfg = self.cfg
+        tokens = np.asarray(tokens)
+        assert tokens.shape[0] == cfg.batch
+        T = tokens.shape[1] - 1
+        out = np.zeros((cfg.batch, T))
+        b = cfg.minibatch_b
+        for si, seq in enumerate(self.seqs):
+            tok = tokens[si]
+            if seq.pend_inputs:
+                raise ValueError("prefill while a decode chunk is pending")
+            if seq.n_pos > 0 and tok[0] != seq.pending_token:
+                raise ValueError("stream continuity: first id must be the pending token")
+            s0 = seq.n_pos
+            h = self._frozen_forward(seq, tok[:T], s0, commit=True)
+            for c0 in range(0, T, b):
+                c1 = min(T, c0 + b)
+                full = (c1 - c0) == b
+                losses, grads = self._chunk(seq, h[c0:c1], s0 + c0, tok[c0 + 1:c1 + 1],
+                                            need_grad=full, commit=True)
+                out[si, c0:c1] = losses
+                if full:
+                    self._sgd(seq, grads)
+                else:  # reading R10
+                    seq.pend_inputs = list(h[c0:c1])
+                    seq.pend_targets = list(tok[c0 + 1:c1 + 1])
+            seq.n_pos = s0 + T
+            seq.pending_token = int(tok[T])
+        return out
+
+    # --------------------------------------------------------------- Algorithm 3
+    def decode(self, n, forced=None):
+        """Generate n tokens per sequence (greedy unless forced [B][n] is given).
+
+        Returns dict(tokens, losses, z_chosen, z_max), each [B][n].
+        """
+        cfg = self.cfg
+        b = cfg.minibatch_b
+        res = {k: np.zeros((cfg.batch, n)) for k in ("losses", "z_chosen", "z_max")}
+        res["tokens"] = np.zeros((cfg.batch, n), dtype=np.int64)
+        for si, seq in enumerate(self.seqs):
+            for t in range(n):
+                p = seq.n_pos
+                h = self._frozen_forward(seq, [seq.pending_token], p, commit=True)
+                y = h
+                for j in range(cfg.n_ttt):
+                    y, _ = self._ttt_block(seq, j, y, p, commit=True, keep=False)
+                z = self._head(y)[0][0]
+                zmax = z.max()
+                tok = int(np.argmax(z)) if forced is None else int(forced[si][t])  # reading R11
+                res["tokens"][si, t] = tok
+                res["losses"][si, t] = _logsumexp(z[None])[0] - z[tok]
+                res["z_chosen"][si, t] = z[tok]
+                res["z_max"][si, t] = zmax
+                seq.pend_inputs.append(h[0])
+                seq.pend_targets.append(tok)
+                seq.n_pos = p + 1
+                seq.pending_token = tok
+                if seq.n_pos % b == 0:
+                    s = seq.n_pos - b
+                    _, grads = self._chunk(seq, np.stack(seq.pend_inputs), s, seq.pend_targets,
+                                           need_grad=True, commit=False)
+                    self._sgd(seq, grads)
+                    seq.pend_inputs, seq.pend_targets = [], []
+        return res
+
+    # --------------------------------------------------------------- inspection
+    def fast_weights(self, seq, j):
+        """(W1t [h_t][d], W2t [d][h_t]) of adaptive block j of sequence seq."""
+        f = self.seqs[seq].fast[j]
+        return f["W1t"].copy(), f["W2t"].copy()
+
+    def chunk_loss_and_grad(self, seq, tokens_chunk):
+        """Mean loss and gradient of the next full chunk, without changing any state.
+
+        tokens_chunk holds b+1 ids: the pending token followed by the chunk's b
+        targets. Used by the finite-difference pins.
+        """
+        st = self.seqs[seq]
+        cfg = self.cfg
+        assert len(tokens_chunk) == cfg.minibatch_b + 1 and not st.pend_inputs
+        h = self._frozen_forward(st, tokens_chunk[:-1], st.n_pos, commit=False)
+        losses, grads = self._chunk(st, h, st.n_pos, tokens_chunk[1:], need_grad=True, commit=False)
+        return float(np.mean(losses)), grads
