@@ -1,0 +1,70 @@
+/*
+ * ttt_kernels.h — per-kernel C ABI of the TTT-E2E library (sm_100a).
+ *
+ * The same kernels that ttt_prefill/ttt_decode run, exposed one at a time so
+ * that each can be checked against the CPU reference and timed against its
+ * roofline. All pointers are DEVICE pointers; `stream` is a cudaStream_t (NULL
+ * = legacy default stream). Calls are asynchronous: they only enqueue work.
+ * ttt_k_status() synchronises the stream and reports launch or device-side
+ * errors (bounded waits that expired). Return codes are the TTT_* codes of ttt.h.
+ * elem_dtype: TTT_FP32 (float operands) or TTT_BF16 (bf16 operands).
+ */
+#ifndef TTT_KERNELS_H
+#define TTT_KERNELS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Epilogues of ttt_k_gemm (acc = alpha * sum_k A[m][k] B[n][k], fp32):
+ *   TTT_EPI_STORE: D = acc (D float if d_f32, else elem type)
+ *   TTT_EPI_RESID: D(float) = acc + X(float)             (X may equal D: residual add in place)
+ *   TTT_EPI_GELU:  Y = acc (if Y), D = gelu(acc)          (exact erf GELU; elem type)
+ *   TTT_EPI_DGELU: D = acc * gelu'(X)                     (X, D elem type)
+ *   TTT_EPI_SGD:   D(float) += acc; Y = D (if Y, elem type)  (alpha = -eta: fused SGD step,
+ *                  summary of the TTT-E2E paper, mini-batch gradient-descent equation) */
+enum { TTT_EPI_STORE = 0, TTT_EPI_RESID = 1, TTT_EPI_GELU = 2, TTT_EPI_DGELU = 3, TTT_EPI_SGD = 4 };
+
+/* Engines: 0 = automatic (tcgen05 tensor cores for bf16 shapes with N % 128 == 0 and K % 64 == 0,
+ * else SIMT), 1 = SIMT fp32-FFMA only. */
+enum { TTT_ENGINE_AUTO = 0, TTT_ENGINE_SIMT = 1 };
+
+/* Batched GEMM D[z][m][n] = epilogue(alpha * sum_k A[z](m,k) * B[z](n,k)).
+ * A(m,k) = a_mn ? A[k*lda + m] : A[m*lda + k]   (batch stride sA elements)
+ * B(n,k) = b_mn ? B[k*ldb + n] : B[n*ldb + k]   (batch stride sB)
+ * D, X, Y row-major with leading dims ldd, ldx, ldy and batch strides sD, sX, sY.
+ * Forward products use (a_mn, b_mn) = (0, 0), data gradients (0, 1), weight gradients (1, 1). */
+int ttt_k_gemm(int32_t elem_dtype, int32_t M, int32_t N, int32_t K, int32_t batch, const void* A, int64_t lda,
+               int64_t sA, int32_t a_mn, const void* B, int64_t ldb, int64_t sB, int32_t b_mn, void* D, int64_t ldd,
+               int64_t sD, int32_t d_f32, const void* X, int64_t ldx, int64_t sX, void* Y, int64_t ldy, int64_t sY,
+               float alpha, int32_t epi, int32_t engine, void* stream);
+
+/* Causal sliding-window attention forward (technical review §5: window k >= b,
+ * causal inside the chunk). Rows [B][n] of qkv ([B*n][3*H*hd]: q | k | v per row,
+ * q and k already rotated) are positions q0..q0+n-1; query P attends to keys
+ * [max(0, P-window+1), P], taking positions < q0 from the rings ring_k/ring_v
+ * ([B][C][H*hd], slot = pos % C) and the others from qkv.
+ * out [B*n][H*hd]; lse [B][H][n] (may be NULL). */
+int ttt_k_attention_fwd(int32_t elem_dtype, int32_t B, int32_t H, int32_t hd, int32_t n, int64_t q0,
+                        int32_t window, const void* qkv, const void* ring_k, const void* ring_v, int32_t C, void* out,
+                        float* lse, int32_t engine, void* stream);
+
+/* Backward of ttt_k_attention_fwd for dout [B*n][H*hd]: dq for every row over its
+ * whole window, dk and dv only for the current rows (cached keys are constants).
+ * dqkv [B*n][3*H*hd] receives dq | dk | dv; dsum [B][H][n] is scratch. */
+int ttt_k_attention_bwd(int32_t elem_dtype, int32_t B, int32_t H, int32_t hd, int32_t n, int64_t q0,
+                        int32_t window, const void* qkv, const void* ring_k, const void* ring_v, int32_t C,
+                        const void* out, const float* lse, const void* dout, void* dqkv, float* dsum,
+                        int32_t engine, void* stream);
+
+/* Synchronise `stream` and return TTT_OK, TTT_ERR_CUDA or TTT_ERR_TIMEOUT (a
+ * bounded device wait expired). Clears the device status word. */
+int ttt_k_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_KERNELS_H */

@@ -1,0 +1,329 @@
+"""Python binding of the TTT-E2E inner-loop library (B200, sm_100a).
+
+Argument marshalling only: every step of prefill and decode runs in the CUDA
+library libttt_b200.so through its C ABI (include/ttt.h, include/ttt_kernels.h).
+PyTorch supplies device memory and the CUDA stream. There is no fallback: if
+the library is missing, importing the binding raises.
+
+    h = ttt_create(cfg, weights)            # cfg: object/dict with the ttt_config fields
+    losses = ttt_prefill(h, tokens)         # tokens [B][T+1] int32 (torch or numpy)
+    toks, losses = ttt_decode(h, n)
+    w1, w2 = ttt_get_weights(h, seq, block)
+    ttt_destroy(h)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libttt_b200.so")
+
+TTT_OK, TTT_ERR_INVALID_ARG, TTT_ERR_OOM, TTT_ERR_CUDA = 0, -1, -2, -3
+TTT_ERR_TIMEOUT, TTT_ERR_STREAM, TTT_ERR_POISONED, TTT_ERR_UNSUPPORTED = -4, -5, -6, -7
+TTT_FP32, TTT_BF16 = 0, 1
+TTT_PTR_HOST, TTT_PTR_DEVICE = 0, 1
+EPI_STORE, EPI_RESID, EPI_GELU, EPI_DGELU, EPI_SGD = 0, 1, 2, 3, 4
+ENGINE_AUTO, ENGINE_SIMT = 0, 1
+
+_ERRNAMES = {0: "OK", -1: "INVALID_ARG", -2: "OOM", -3: "CUDA", -4: "TIMEOUT", -5: "STREAM", -6: "POISONED",
+             -7: "UNSUPPORTED"}
+
+
+class TTTError(RuntimeError):
+    def __init__(self, code, msg=""):
+        super().__init__(f"TTT_ERR_{_ERRNAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+class ttt_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("vocab", "d", "n_layers", "n_heads", "n_ttt", "mlp_hidden",
+                                              "ttt_hidden", "static_hidden", "window_k", "minibatch_b", "batch")] + \
+               [("eta", ctypes.c_float), ("rms_eps", ctypes.c_float), ("rope_base", ctypes.c_float),
+                ("dtype", ctypes.c_int32), ("max_segment", ctypes.c_int32), ("cuda_stream", ctypes.c_void_p)]
+
+
+class ttt_weights(ctypes.Structure):
+    _fields_ = [("tensors", ctypes.POINTER(ctypes.c_void_p)), ("n_tensors", ctypes.c_int32),
+                ("values_dtype", ctypes.c_int32), ("ptr_kind", ctypes.c_int32)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m long_context_prefill_ttt_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, F, VP = ctypes.POINTER, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p
+    sigs = {
+        "ttt_num_weight_tensors": (I32, [P(ttt_config)]),
+        "ttt_create": (ctypes.c_int, [P(ttt_config), P(ttt_weights), P(VP)]),
+        "ttt_prefill": (ctypes.c_int, [VP, VP, I64, VP, I32]),
+        "ttt_decode": (ctypes.c_int, [VP, I64, VP, VP, VP, I32]),
+        "ttt_get_weights": (ctypes.c_int, [VP, I32, I32, VP, VP, I32]),
+        "ttt_reset": (ctypes.c_int, [VP]),
+        "ttt_position": (I64, [VP]),
+        "ttt_device_bytes": (I64, [VP]),
+        "ttt_last_launch_count": (I64, [VP]),
+        "ttt_destroy": (None, [VP]),
+        "ttt_last_error": (ctypes.c_char_p, [VP]),
+        "ttt_version": (ctypes.c_char_p, []),
+        "ttt_k_gemm": (ctypes.c_int, [I32, I32, I32, I32, I32, VP, I64, I64, I32, VP, I64, I64, I32, VP, I64, I64,
+                                      I32, VP, I64, I64, VP, I64, I64, F, I32, I32, VP]),
+        "ttt_k_attention_fwd": (ctypes.c_int, [I32, I32, I32, I32, I32, I64, I32, VP, VP, VP, I32, VP, VP, I32, VP]),
+        "ttt_k_attention_bwd": (ctypes.c_int, [I32, I32, I32, I32, I32, I64, I32, VP, VP, VP, I32, VP, VP, VP, VP,
+                                               VP, I32, VP]),
+        "ttt_k_status": (ctypes.c_int, [VP]),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_ptr(stream=None):
+    torch = _torch()
+    if stream is not None:
+        return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+    if torch.cuda.is_available():
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return ctypes.c_void_p(0)
+
+
+def _ptr(x):
+    """(address, ptr_kind) of a contiguous torch tensor or numpy array."""
+    if x is None:
+        return None, TTT_PTR_HOST
+    if isinstance(x, np.ndarray):
+        assert x.flags["C_CONTIGUOUS"], "arrays must be contiguous"
+        return x.ctypes.data, TTT_PTR_HOST
+    assert x.is_contiguous(), "tensors must be contiguous"
+    return x.data_ptr(), (TTT_PTR_DEVICE if x.is_cuda else TTT_PTR_HOST)
+
+
+def _get(cfg, name, default=None):
+    if isinstance(cfg, dict):
+        return cfg.get(name, default)
+    return getattr(cfg, name, default)
+
+
+def make_config(cfg, stream=None, max_segment=0) -> ttt_config:
+    """Fill the C struct from any object or dict carrying the fields of ttt_config."""
+    c = ttt_config()
+    for n in ("vocab", "d", "n_layers", "n_heads", "n_ttt", "mlp_hidden", "ttt_hidden", "static_hidden",
+              "window_k", "minibatch_b", "batch"):
+        setattr(c, n, int(_get(cfg, n)))
+    c.eta = float(_get(cfg, "eta"))
+    c.rms_eps = float(_get(cfg, "rms_eps", 1e-6))
+    c.rope_base = float(_get(cfg, "rope_base", 10000.0))
+    dt = _get(cfg, "dtype", "bf16")
+    c.dtype = TTT_BF16 if dt in ("bf16", TTT_BF16) else TTT_FP32
+    c.max_segment = int(max_segment or _get(cfg, "max_segment", 0) or 0)
+    c.cuda_stream = _stream_ptr(stream).value
+    return c
+
+
+def weight_names(cfg):
+    """Tensor order of ttt_weights (include/ttt.h)."""
+    names = ["E", "final_norm"]
+    L, Lt = int(_get(cfg, "n_layers")), int(_get(cfg, "n_ttt"))
+    for l in range(L):
+        p = f"layers.{l}."
+        names += [p + n for n in ("attn_norm", "Wq", "Wk", "Wv", "Wo")]
+        if l >= L - Lt:
+            names += [p + n for n in ("ttt_norm", "W1t", "W2t", "static_norm", "W1s", "W2s")]
+        else:
+            names += [p + n for n in ("mlp_norm", "W1", "W2")]
+    return names
+
+
+class Handle:
+    """Owns a ttt_handle*; keeps the config and stream it was created with."""
+
+    def __init__(self, ptr, cfg, cstruct):
+        self.ptr = ptr
+        self.cfg = cfg
+        self.c = cstruct
+
+    @property
+    def batch(self):
+        return self.c.batch
+
+    def error(self):
+        return lib.ttt_last_error(self.ptr).decode()
+
+    def check(self, rc):
+        if rc != TTT_OK:
+            raise TTTError(rc, self.error())
+
+    def __del__(self):
+        if getattr(self, "ptr", None):
+            lib.ttt_destroy(self.ptr)
+            self.ptr = None
+
+
+# ----------------------------------------------------------------------------- C ABI, same names
+
+def ttt_create(cfg, weights, stream=None, max_segment=0) -> Handle:
+    """weights: dict name -> float32 array/tensor (values exactly representable in cfg's dtype)."""
+    c = make_config(cfg, stream, max_segment)
+    names = weight_names(cfg)
+    ptrs, kinds, keep = [], set(), []
+    for n in names:
+        t = weights[n]
+        if isinstance(t, np.ndarray):
+            t = np.ascontiguousarray(t, dtype=np.float32)
+        keep.append(t)
+        p, k = _ptr(t)
+        ptrs.append(p)
+        kinds.add(k)
+    if len(kinds) != 1:
+        raise ValueError("weights must be all host or all device")
+    arr = (ctypes.c_void_p * len(ptrs))(*ptrs)
+    w = ttt_weights(ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)), len(ptrs), TTT_FP32, kinds.pop())
+    out = ctypes.c_void_p()
+    rc = lib.ttt_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(out))
+    if rc != TTT_OK:
+        raise TTTError(rc, "ttt_create failed")
+    return Handle(out, cfg, c)
+
+
+def ttt_prefill(h: Handle, tokens, out_losses=None):
+    """tokens [B][T+1] int32; returns losses [B][T] (float32, same kind as tokens)."""
+    B, n1 = tokens.shape
+    T = n1 - 1
+    if out_losses is None:
+        if isinstance(tokens, np.ndarray):
+            out_losses = np.empty((B, T), dtype=np.float32)
+        else:
+            out_losses = _torch().empty((B, T), dtype=_torch().float32, device=tokens.device)
+    tp, kind = _ptr(tokens)
+    lp, kind2 = _ptr(out_losses)
+    assert kind == kind2
+    h.check(lib.ttt_prefill(h.ptr, ctypes.c_void_p(tp), T, ctypes.c_void_p(lp), kind))
+    return out_losses
+
+
+def ttt_decode(h: Handle, n: int, forced=None, device=None):
+    """Generate n tokens per sequence; returns (tokens [B][n] int32, losses [B][n] float32)."""
+    B = h.batch
+    if device is not None and str(device).startswith("cuda"):
+        torch = _torch()
+        toks = torch.empty((B, n), dtype=torch.int32, device=device)
+        losses = torch.empty((B, n), dtype=torch.float32, device=device)
+        kind = TTT_PTR_DEVICE
+        fp = forced.data_ptr() if forced is not None else None
+        tp, lp = toks.data_ptr(), losses.data_ptr()
+    else:
+        toks = np.empty((B, n), dtype=np.int32)
+        losses = np.empty((B, n), dtype=np.float32)
+        kind = TTT_PTR_HOST
+        if forced is not None:
+            forced = np.ascontiguousarray(forced, dtype=np.int32)
+        fp = forced.ctypes.data if forced is not None else None
+        tp, lp = toks.ctypes.data, losses.ctypes.data
+    h.check(lib.ttt_decode(h.ptr, n, ctypes.c_void_p(fp) if fp else None, ctypes.c_void_p(tp),
+                           ctypes.c_void_p(lp), kind))
+    return toks, losses
+
+
+def ttt_get_weights(h: Handle, seq: int, block: int):
+    """fp32 fast weights (W1t [h_t][d], W2t [d][h_t]) of sequence seq, adaptive block `block`."""
+    d, ht = h.c.d, h.c.ttt_hidden
+    w1 = np.empty((ht, d), dtype=np.float32)
+    w2 = np.empty((d, ht), dtype=np.float32)
+    h.check(lib.ttt_get_weights(h.ptr, seq, block, ctypes.c_void_p(w1.ctypes.data), ctypes.c_void_p(w2.ctypes.data),
+                                TTT_PTR_HOST))
+    return w1, w2
+
+
+def ttt_reset(h: Handle):
+    h.check(lib.ttt_reset(h.ptr))
+
+
+def ttt_destroy(h: Handle):
+    if h.ptr:
+        lib.ttt_destroy(h.ptr)
+        h.ptr = None
+
+
+def ttt_last_error(h: Handle) -> str:
+    return h.error()
+
+
+def ttt_position(h: Handle) -> int:
+    return int(lib.ttt_position(h.ptr))
+
+
+def ttt_device_bytes(h: Handle) -> int:
+    return int(lib.ttt_device_bytes(h.ptr))
+
+
+def ttt_last_launch_count(h: Handle) -> int:
+    return int(lib.ttt_last_launch_count(h.ptr))
+
+
+def ttt_version() -> str:
+    return lib.ttt_version().decode()
+
+
+# ----------------------------------------------------------------------------- per-kernel ABI
+
+def _dtype_code(t):
+    torch = _torch()
+    return TTT_BF16 if t.dtype == torch.bfloat16 else TTT_FP32
+
+
+def ttt_k_gemm(A, B, D, M, N, K, *, batch=1, lda=None, sA=0, a_mn=False, ldb=None, sB=0, b_mn=False, ldd=None,
+               sD=0, X=None, ldx=0, sX=0, Y=None, ldy=0, sY=0, alpha=1.0, epi=EPI_STORE, engine=ENGINE_AUTO,
+               stream=None):
+    """Enqueue one contraction on device tensors (see include/ttt_kernels.h)."""
+    torch = _torch()
+    lda = lda if lda is not None else (M if a_mn else K)
+    ldb = ldb if ldb is not None else (N if b_mn else K)
+    ldd = ldd if ldd is not None else N
+    rc = lib.ttt_k_gemm(_dtype_code(A), M, N, K, batch, A.data_ptr(), lda, sA, int(a_mn), B.data_ptr(), ldb, sB,
+                        int(b_mn), D.data_ptr(), ldd, sD, int(D.dtype == torch.float32),
+                        X.data_ptr() if X is not None else None, ldx, sX,
+                        Y.data_ptr() if Y is not None else None, ldy, sY, float(alpha), epi, engine,
+                        _stream_ptr(stream))
+    if rc != TTT_OK:
+        raise TTTError(rc, "ttt_k_gemm")
+
+
+def ttt_k_attention_fwd(qkv, out, lse, B, H, hd, n, q0, window, ring_k=None, ring_v=None, C=0,
+                        engine=ENGINE_AUTO, stream=None):
+    rc = lib.ttt_k_attention_fwd(_dtype_code(qkv), B, H, hd, n, q0, window, qkv.data_ptr(),
+                                 ring_k.data_ptr() if ring_k is not None else None,
+                                 ring_v.data_ptr() if ring_v is not None else None, C, out.data_ptr(),
+                                 lse.data_ptr() if lse is not None else None, engine, _stream_ptr(stream))
+    if rc != TTT_OK:
+        raise TTTError(rc, "ttt_k_attention_fwd")
+
+
+def ttt_k_attention_bwd(qkv, out, lse, dout, dqkv, dsum, B, H, hd, n, q0, window, ring_k=None, ring_v=None, C=0,
+                        engine=ENGINE_AUTO, stream=None):
+    rc = lib.ttt_k_attention_bwd(_dtype_code(qkv), B, H, hd, n, q0, window, qkv.data_ptr(),
+                                 ring_k.data_ptr() if ring_k is not None else None,
+                                 ring_v.data_ptr() if ring_v is not None else None, C, out.data_ptr(),
+                                 lse.data_ptr(), dout.data_ptr(), dqkv.data_ptr(), dsum.data_ptr(), engine,
+                                 _stream_ptr(stream))
+    if rc != TTT_OK:
+        raise TTTError(rc, "ttt_k_attention_bwd")
+
+
+def ttt_k_status(stream=None):
+    rc = lib.ttt_k_status(_stream_ptr(stream))
+    if rc != TTT_OK:
+        raise TTTError(rc, "device status")

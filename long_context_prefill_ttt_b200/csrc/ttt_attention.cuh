@@ -1,0 +1,230 @@
+// Causal sliding-window attention of the TTT-E2E path, forward and backward.
+//
+// Query row i of sequence b sits at absolute position P = q0 + i and attends to
+// keys at positions [max(0, P-k+1), P] (window k, causal), as the pages'
+// sliding-window attention with k >= b prescribes (b-lab.team summary,
+// "Integration with Sliding-Window Attention"; technical review §5).
+// Keys come from two places:
+//   * positions >= q0: the current rows (same rows as the queries),
+//   * positions <  q0: the per-sequence ring cache [B][C][d], slot = pos % C,
+//     holding K/V computed when their rows were processed. These cached K/V are
+//     constants: the backward produces dK/dV for current rows only.
+// Online softmax in fp32; lse = m + log(l) is kept for the backward.
+#pragma once
+
+#include "ttt_common.cuh"
+
+namespace ttt {
+
+struct AttnParams {
+  int B, H, hd, n, d;
+  int64_t q0;
+  int window;
+  const void* Q; int64_t ldq;          // [B*n][ldq], head h at column h*hd
+  const void* K; const void* V; int64_t ldkv;
+  const void* Kc; const void* Vc; int C;  // rings [B][C][d]
+  void* O; int64_t ldo;
+  float* lse;                          // [B][H][n]
+  float scale;
+  // backward
+  const void* dO; int64_t lddo;
+  float* Dsum;                         // [B][H][n] = rowsum(dO * O)
+  void* dQ; void* dK; void* dV; int64_t lddq;  // dQ/dK/dV rows [B*n][lddq]
+};
+
+template <typename T>
+__device__ __forceinline__ const T* key_row(const AttnParams& p, const T* cur, const T* ring, int b, int h,
+                                            int64_t pos) {
+  if (pos >= p.q0) return cur + ((int64_t)b * p.n + (pos - p.q0)) * p.ldkv + h * p.hd;
+  return ring + ((int64_t)b * p.C + pos % p.C) * p.d + h * p.hd;
+}
+
+// ---------------------------------------------------------------- SIMT forward
+// One warp per (row, head); lanes take 32 consecutive keys at a time.
+template <typename T>
+__global__ void __launch_bounds__(128) attn_fwd_simt_kernel(AttnParams p) {
+  __shared__ float qs[4][128];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t)blockIdx.x * 4 + warp;
+  if (gw >= (int64_t)p.B * p.n * p.H) return;
+  const int h = (int)(gw % p.H);
+  const int row = (int)(gw / p.H);
+  const int b = row / p.n, i = row % p.n;
+  const int64_t P = p.q0 + i;
+  const int64_t lo = P - p.window + 1 > 0 ? P - p.window + 1 : 0;
+  const T* Q = (const T*)p.Q + (int64_t)row * p.ldq + h * p.hd;
+  for (int c = lane; c < p.hd; c += 32) qs[warp][c] = to_f32(Q[c]) * p.scale;
+  __syncwarp();
+  const int nd = (p.hd + 31) / 32;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float m = -INFINITY, l = 0.f;
+  for (int64_t j0 = lo; j0 <= P; j0 += 32) {
+    const int64_t j = j0 + lane;
+    float s = -INFINITY;
+    if (j <= P) {
+      const T* kr = key_row<T>(p, (const T*)p.K, (const T*)p.Kc, b, h, j);
+      float dot = 0.f;
+      for (int c = 0; c < p.hd; ++c) dot = fmaf(qs[warp][c], to_f32(kr[c]), dot);
+      s = dot;
+    }
+    float mb = s;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+    const float mnew = fmaxf(m, mb);
+    const float pj = (j <= P) ? expf(s - mnew) : 0.f;
+    const float corr = expf(m - mnew);
+    float ps = pj;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+    l = l * corr + ps;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) acc[t] *= corr;
+    const int cnt = (int)((P - j0 + 1) < 32 ? (P - j0 + 1) : 32);
+    for (int jj = 0; jj < cnt; ++jj) {
+      const float pp = __shfl_sync(0xffffffffu, pj, jj);
+      const T* vr = key_row<T>(p, (const T*)p.V, (const T*)p.Vc, b, h, j0 + jj);
+      for (int t = 0; t < nd; ++t) {
+        const int c = lane + 32 * t;
+        if (c < p.hd) acc[t] = fmaf(pp, to_f32(vr[c]), acc[t]);
+      }
+    }
+    m = mnew;
+  }
+  T* O = (T*)p.O + (int64_t)row * p.ldo + h * p.hd;
+  const float inv = 1.f / l;
+  for (int t = 0; t < nd; ++t) {
+    const int c = lane + 32 * t;
+    if (c < p.hd) O[c] = from_f32<T>(acc[t] * inv);
+  }
+  if (lane == 0 && p.lse) p.lse[((int64_t)b * p.H + h) * p.n + i] = m + logf(l);
+}
+
+// ---------------------------------------------------------------- backward
+// Dsum[b][h][i] = sum_c dO[row][h*hd+c] * O[row][h*hd+c]
+template <typename T>
+__global__ void attn_bwd_prep_kernel(AttnParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + warp;
+  if (gw >= (int64_t)p.B * p.n * p.H) return;
+  const int h = (int)(gw % p.H);
+  const int row = (int)(gw / p.H);
+  const T* dO = (const T*)p.dO + (int64_t)row * p.lddo + h * p.hd;
+  const T* O = (const T*)p.O + (int64_t)row * p.ldo + h * p.hd;
+  float s = 0.f;
+  for (int c = lane; c < p.hd; c += 32) s += to_f32(dO[c]) * to_f32(O[c]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0) p.Dsum[((int64_t)(row / p.n) * p.H + h) * p.n + row % p.n] = s;
+}
+
+// dQ for every query over its whole window (cached and current keys).
+template <typename T>
+__global__ void __launch_bounds__(128) attn_bwd_dq_simt_kernel(AttnParams p) {
+  __shared__ float qs[4][128];
+  __shared__ float dos[4][128];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t)blockIdx.x * 4 + warp;
+  if (gw >= (int64_t)p.B * p.n * p.H) return;
+  const int h = (int)(gw % p.H);
+  const int row = (int)(gw / p.H);
+  const int b = row / p.n, i = row % p.n;
+  const int64_t P = p.q0 + i;
+  const int64_t lo = P - p.window + 1 > 0 ? P - p.window + 1 : 0;
+  const T* Q = (const T*)p.Q + (int64_t)row * p.ldq + h * p.hd;
+  const T* dO = (const T*)p.dO + (int64_t)row * p.lddo + h * p.hd;
+  for (int c = lane; c < p.hd; c += 32) { qs[warp][c] = to_f32(Q[c]) * p.scale; dos[warp][c] = to_f32(dO[c]); }
+  __syncwarp();
+  const int64_t si = ((int64_t)b * p.H + h) * p.n + i;
+  const float lse = p.lse[si], D = p.Dsum[si];
+  const int nd = (p.hd + 31) / 32;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int64_t j0 = lo; j0 <= P; j0 += 32) {
+    const int64_t j = j0 + lane;
+    float ds = 0.f;
+    if (j <= P) {
+      const T* kr = key_row<T>(p, (const T*)p.K, (const T*)p.Kc, b, h, j);
+      const T* vr = key_row<T>(p, (const T*)p.V, (const T*)p.Vc, b, h, j);
+      float s = 0.f, dp = 0.f;
+      for (int c = 0; c < p.hd; ++c) {
+        s = fmaf(qs[warp][c], to_f32(kr[c]), s);
+        dp = fmaf(dos[warp][c], to_f32(vr[c]), dp);
+      }
+      const float pr = expf(s - lse);
+      ds = pr * (dp - D);
+    }
+    const int cnt = (int)((P - j0 + 1) < 32 ? (P - j0 + 1) : 32);
+    for (int jj = 0; jj < cnt; ++jj) {
+      const float g = __shfl_sync(0xffffffffu, ds, jj);
+      const T* kr = key_row<T>(p, (const T*)p.K, (const T*)p.Kc, b, h, j0 + jj);
+      for (int t = 0; t < nd; ++t) {
+        const int c = lane + 32 * t;
+        if (c < p.hd) acc[t] = fmaf(g, to_f32(kr[c]), acc[t]);
+      }
+    }
+  }
+  T* dQ = (T*)p.dQ + (int64_t)row * p.lddq + h * p.hd;
+  for (int t = 0; t < nd; ++t) {
+    const int c = lane + 32 * t;
+    if (c < p.hd) dQ[c] = from_f32<T>(acc[t] * p.scale);
+  }
+}
+
+// dK, dV for the current rows only (cached keys are constants).
+template <typename T>
+__global__ void __launch_bounds__(128) attn_bwd_dkv_simt_kernel(AttnParams p) {
+  __shared__ float ks[4][128];
+  __shared__ float vs[4][128];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gw = (int64_t)blockIdx.x * 4 + warp;
+  if (gw >= (int64_t)p.B * p.n * p.H) return;
+  const int h = (int)(gw % p.H);
+  const int row = (int)(gw / p.H);
+  const int b = row / p.n, jr = row % p.n;
+  const T* K = (const T*)p.K + (int64_t)row * p.ldkv + h * p.hd;
+  const T* V = (const T*)p.V + (int64_t)row * p.ldkv + h * p.hd;
+  for (int c = lane; c < p.hd; c += 32) { ks[warp][c] = to_f32(K[c]) * p.scale; vs[warp][c] = to_f32(V[c]); }
+  __syncwarp();
+  const int iend = (jr + p.window < p.n) ? jr + p.window : p.n;  // queries i in [jr, iend)
+  const int nd = (p.hd + 31) / 32;
+  float dk[4] = {0.f, 0.f, 0.f, 0.f}, dv[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int i0 = jr; i0 < iend; i0 += 32) {
+    const int i = i0 + lane;
+    float pr = 0.f, ds = 0.f;
+    if (i < iend) {
+      const int qrow = b * p.n + i;
+      const T* Q = (const T*)p.Q + (int64_t)qrow * p.ldq + h * p.hd;
+      const T* dO = (const T*)p.dO + (int64_t)qrow * p.lddo + h * p.hd;
+      float s = 0.f, dp = 0.f;
+      for (int c = 0; c < p.hd; ++c) {
+        s = fmaf(ks[warp][c], to_f32(Q[c]), s);
+        dp = fmaf(vs[warp][c], to_f32(dO[c]), dp);
+      }
+      const int64_t si = ((int64_t)b * p.H + h) * p.n + i;
+      pr = expf(s - p.lse[si]);
+      ds = pr * (dp - p.Dsum[si]);
+    }
+    const int cnt = (iend - i0) < 32 ? (iend - i0) : 32;
+    for (int ii = 0; ii < cnt; ++ii) {
+      const float pp = __shfl_sync(0xffffffffu, pr, ii);
+      const float g = __shfl_sync(0xffffffffu, ds, ii);
+      const int qrow = b * p.n + i0 + ii;
+      const T* Q = (const T*)p.Q + (int64_t)qrow * p.ldq + h * p.hd;
+      const T* dO = (const T*)p.dO + (int64_t)qrow * p.lddo + h * p.hd;
+      for (int t = 0; t < nd; ++t) {
+        const int c = lane + 32 * t;
+        if (c < p.hd) {
+          dv[t] = fmaf(pp, to_f32(dO[c]), dv[t]);
+          dk[t] = fmaf(g, to_f32(Q[c]), dk[t]);
+        }
+      }
+    }
+  }
+  T* dK = (T*)p.dK + (int64_t)row * p.lddq + h * p.hd;
+  T* dV = (T*)p.dV + (int64_t)row * p.lddq + h * p.hd;
+  for (int t = 0; t < nd; ++t) {
+    const int c = lane + 32 * t;
+    if (c < p.hd) { dK[c] = from_f32<T>(dk[t] * p.scale); dV[c] = from_f32<T>(dv[t]); }
+  }
+}
+
+}  // namespace ttt

@@ -1,0 +1,355 @@
+// Dense contractions of the TTT-E2E path: D[m][n] = alpha * sum_k A[m][k] * B[n][k]
+// with fused epilogues.
+//
+// Two engines share one parameter block and one epilogue definition:
+//  * gemm_tc: tcgen05 tensor cores (bf16 operands, fp32 accumulation in TMEM),
+//    operands staged by TMA into 128-byte-swizzled shared memory, a 4-6 stage
+//    mbarrier ring, one elected thread issuing MMAs, double-buffered TMEM
+//    accumulators so that the epilogue of tile t overlaps the main loop of
+//    tile t+1 (persistent CTAs, one per SM).
+//  * gemm_simt: plain fp32 FFMA tiles for float operands (the fp32 workload
+//    needs fp32-exact products) and for shapes the tensor-core tiles do not fit.
+//
+// Operand "majors": A is logically [M][K]; stored K-major (A[m*lda+k]) or
+// MN-major (A[k*lda+m]). Same for B ([N][K]). Forward products use (K, K),
+// data gradients (K, MN), weight gradients (MN, MN).
+#pragma once
+
+#include "ttt_common.cuh"
+
+namespace ttt {
+
+enum EpiKind : int {
+  EPI_STORE = 0,   // D = acc                              (D f32 or element type)
+  EPI_RESID = 1,   // D(f32) = acc + X(f32)                (X may alias D)
+  EPI_GELU = 2,    // Y = acc (if Y), D = gelu(acc)        (element type)
+  EPI_DGELU = 3,   // D = acc * gelu'(X)                   (element type, X element type)
+  EPI_SGD = 4,     // D(f32) += acc, Y = D (if Y)          (alpha = -eta)
+};
+
+struct GemmParams {
+  int M, N, K, batch;
+  const void* A; int64_t lda, sA; int a_mn;
+  const void* B; int64_t ldb, sB; int b_mn;
+  void* D; int64_t ldd, sD; int d_f32;
+  const void* X; int64_t ldx, sX;
+  void* Y; int64_t ldy, sY;
+  float alpha;
+  int epi;
+};
+
+// ============================================================== epilogue (per element)
+template <typename T>
+__device__ __forceinline__ void epi_apply(const GemmParams& p, int z, int m, int n, float acc) {
+  acc *= p.alpha;
+  const int64_t od = (int64_t)z * p.sD + (int64_t)m * p.ldd + n;
+  switch (p.epi) {
+    case EPI_STORE:
+      if (p.d_f32) ((float*)p.D)[od] = acc; else ((T*)p.D)[od] = from_f32<T>(acc);
+      break;
+    case EPI_RESID: {
+      const float r = ((const float*)p.X)[(int64_t)z * p.sX + (int64_t)m * p.ldx + n];
+      ((float*)p.D)[od] = acc + r;
+      break;
+    }
+    case EPI_GELU:
+      if (p.Y) ((T*)p.Y)[(int64_t)z * p.sY + (int64_t)m * p.ldy + n] = from_f32<T>(acc);
+      ((T*)p.D)[od] = from_f32<T>(gelu_f(acc));
+      break;
+    case EPI_DGELU: {
+      const float u = to_f32(((const T*)p.X)[(int64_t)z * p.sX + (int64_t)m * p.ldx + n]);
+      ((T*)p.D)[od] = from_f32<T>(acc * gelu_prime_f(u));
+      break;
+    }
+    case EPI_SGD: {
+      float* w = (float*)p.D + od;
+      const float nw = *w + acc;
+      *w = nw;
+      if (p.Y) ((T*)p.Y)[(int64_t)z * p.sY + (int64_t)m * p.ldy + n] = from_f32<T>(nw);
+      break;
+    }
+  }
+}
+
+// ============================================================== SIMT engine
+// 64x64 output tile, K step 16, 256 threads with 4x4 outputs each.
+template <typename T>
+__global__ void __launch_bounds__(256) gemm_simt_kernel(GemmParams p) {
+  __shared__ float As[16][68];
+  __shared__ float Bs[16][68];
+  const int z = blockIdx.z;
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  const int t = threadIdx.x, tx = t & 15, ty = t >> 4;
+  const T* A = (const T*)p.A + (int64_t)z * p.sA;
+  const T* B = (const T*)p.B + (int64_t)z * p.sB;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < p.K; k0 += 16) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = t + i * 256;
+      int mm, kk;
+      if (p.a_mn) { kk = e >> 6; mm = e & 63; } else { mm = e >> 4; kk = e & 15; }
+      const int gm = m0 + mm, gk = k0 + kk;
+      float v = 0.f;
+      if (gm < p.M && gk < p.K) v = to_f32(p.a_mn ? A[(int64_t)gk * p.lda + gm] : A[(int64_t)gm * p.lda + gk]);
+      As[kk][mm] = v;
+      int nn;
+      if (p.b_mn) { kk = e >> 6; nn = e & 63; } else { nn = e >> 4; kk = e & 15; }
+      const int gn = n0 + nn;
+      const int gk2 = k0 + kk;
+      float w = 0.f;
+      if (gn < p.N && gk2 < p.K) w = to_f32(p.b_mn ? B[(int64_t)gk2 * p.ldb + gn] : B[(int64_t)gn * p.ldb + gk2]);
+      Bs[kk][nn] = w;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[4], b[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { a[i] = As[kk][ty * 4 + i]; b[i] = Bs[kk][tx * 4 + i]; }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int m = m0 + ty * 4 + i, n = n0 + tx * 4 + j;
+      if (m < p.M && n < p.N) epi_apply<T>(p, z, m, n, acc[i][j]);
+    }
+}
+
+// ============================================================== tcgen05 engine
+constexpr int TC_BM = 128;
+constexpr int TC_BK = 64;
+constexpr int TC_THREADS = 192;  // warp 0: TMA, warp 1: MMA + TMEM owner, warps 2-5: epilogue
+
+template <int BN> struct TcCfg {
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int A_BYTES = TC_BM * TC_BK * 2;
+  static constexpr int B_BYTES = BN * TC_BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int TMEM_COLS = 2 * BN;
+};
+
+// 32 consecutive accumulator columns of one row through the epilogue, vectorised.
+template <typename T>
+__device__ __forceinline__ void epi_row32(const GemmParams& p, int z, int m, int n, float* v) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] *= p.alpha;
+  const int64_t od = (int64_t)z * p.sD + (int64_t)m * p.ldd + n;
+  if (p.epi == EPI_STORE && p.d_f32) {
+    float4* d = (float4*)((float*)p.D + od);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  } else if (p.epi == EPI_STORE) {
+    uint4* d = (uint4*)((T*)p.D + od);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      d[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                        pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+  } else if (p.epi == EPI_RESID) {
+    const float4* x = (const float4*)((const float*)p.X + (int64_t)z * p.sX + (int64_t)m * p.ldx + n);
+    float4* d = (float4*)((float*)p.D + od);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 r = x[i];
+      d[i] = make_float4(v[4 * i] + r.x, v[4 * i + 1] + r.y, v[4 * i + 2] + r.z, v[4 * i + 3] + r.w);
+    }
+  } else if (p.epi == EPI_GELU) {
+    if (p.Y) {
+      uint4* y = (uint4*)((T*)p.Y + (int64_t)z * p.sY + (int64_t)m * p.ldy + n);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        y[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                          pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = gelu_f(v[i]);
+    uint4* d = (uint4*)((T*)p.D + od);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      d[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                        pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+  } else if (p.epi == EPI_DGELU) {
+    const uint4* x = (const uint4*)((const T*)p.X + (int64_t)z * p.sX + (int64_t)m * p.ldx + n);
+    uint4* d = (uint4*)((T*)p.D + od);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint4 u4 = x[i];
+      const bf16* u = reinterpret_cast<const bf16*>(&u4);
+      float o[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = v[8 * i + j] * gelu_prime_f(__bfloat162float(u[j]));
+      d[i] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                        pack_bf16x2(o[6], o[7]));
+    }
+  } else {  // EPI_SGD
+    float4* w = (float4*)((float*)p.D + od);
+    float nw[32];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float4 c = w[i];
+      c.x += v[4 * i]; c.y += v[4 * i + 1]; c.z += v[4 * i + 2]; c.w += v[4 * i + 3];
+      w[i] = c;
+      nw[4 * i] = c.x; nw[4 * i + 1] = c.y; nw[4 * i + 2] = c.z; nw[4 * i + 3] = c.w;
+    }
+    if (p.Y) {
+      uint4* y = (uint4*)((T*)p.Y + (int64_t)z * p.sY + (int64_t)m * p.ldy + n);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        y[i] = make_uint4(pack_bf16x2(nw[8 * i], nw[8 * i + 1]), pack_bf16x2(nw[8 * i + 2], nw[8 * i + 3]),
+                          pack_bf16x2(nw[8 * i + 4], nw[8 * i + 5]), pack_bf16x2(nw[8 * i + 6], nw[8 * i + 7]));
+    }
+  }
+}
+
+// Persistent warp-specialised tcgen05 GEMM. Requirements (checked on the host):
+// N % BN == 0, K % 64 == 0, 16-byte aligned rows; M may have a tail (TMA fills
+// out-of-range rows with zeros and the epilogue skips them).
+template <int BN, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmParams p, int* err) {
+  using C = TcCfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = (uint64_t*)(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = bars;                    // [STAGES]
+  uint64_t* empty = bars + C::STAGES;       // [STAGES]
+  uint64_t* acc_full = bars + 2 * C::STAGES;      // [2]
+  uint64_t* acc_empty = bars + 2 * C::STAGES + 2; // [2]
+  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * C::STAGES + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int m_tiles = (p.M + TC_BM - 1) / TC_BM;
+  const int n_tiles = p.N / BN;
+  const int tiles_per_batch = m_tiles * n_tiles;
+  const int num_tiles = tiles_per_batch * p.batch;
+  const int k_blocks = p.K / TC_BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 4); }
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (elect_lane0()) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int z = tile / tiles_per_batch;
+        const int r = tile % tiles_per_batch;
+        const int m0 = (r / n_tiles) * TC_BM;
+        const int n0 = (r % n_tiles) * BN;
+        for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t round = it / C::STAGES;
+          if (!mbar_wait(&empty[s], (round & 1) ^ 1, err, DEV_TIMEOUT_EMPTY)) { ok = false; break; }
+          uint8_t* sa = smem + s * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+          const int k0 = kb * TC_BK;
+          if (A_MN) {
+            tma_load_3d(sa, &tmA, &full[s], m0, k0, z);
+            tma_load_3d(sa + 8192, &tmA, &full[s], m0 + 64, k0, z);
+          } else {
+            tma_load_3d(sa, &tmA, &full[s], k0, m0, z);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tma_load_3d(sb + j * 8192, &tmB, &full[s], n0 + 64 * j, k0, z);
+          } else {
+            tma_load_3d(sb, &tmB, &full[s], k0, n0, z);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_lane0()) {
+      constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, BN, A_MN, B_MN);
+      int it = 0, lt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++lt) {
+        const int acc = lt & 1;
+        const uint32_t use = lt >> 1;
+        if (!mbar_wait(&acc_empty[acc], (use & 1) ^ 1, err, DEV_TIMEOUT_ACC)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t round = it / C::STAGES;
+          if (!mbar_wait(&full[s], round & 1, err, DEV_TIMEOUT_FULL)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < TC_BK / 16; ++kk) {
+            const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+                                     : smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                     : smem_desc_sw128(sb + kk * 32, 16, 1024);
+            tc_mma_f16(d_tmem, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[acc]);
+      }
+    }
+  } else {
+    // epilogue warps 2..5: TMEM lane quarter = warp % 4
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + (threadIdx.x & 31);
+    int lt = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
+      const int z = tile / tiles_per_batch;
+      const int r = tile % tiles_per_batch;
+      const int m0 = (r / n_tiles) * TC_BM;
+      const int n0 = (r % n_tiles) * BN;
+      const int acc = lt & 1;
+      const uint32_t use = lt >> 1;
+      if (!mbar_wait(&acc_full[acc], use & 1, err, DEV_TIMEOUT_ACC)) break;
+      tc_fence_after();
+      const int m = m0 + row_in_tile;
+      const uint32_t taddr = tmem_base + acc * BN + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(taddr + c * 32, v);
+        if (m < p.M) epi_row32<bf16>(p, z, m, n0 + c * 32, v);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (elect_lane0()) mbar_arrive(&acc_empty[acc]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ============================================================== host side
+int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t stream, int* err, int num_sms,
+                int force_simt);
+
+}  // namespace ttt

@@ -1,0 +1,135 @@
+// Per-kernel C ABI (include/ttt_kernels.h): one contraction or one attention
+// pass at a time, on caller-provided device buffers.
+#include <cmath>
+#include <cstring>
+
+#include "ttt.h"
+#include "ttt_attention.cuh"
+#include "ttt_common.cuh"
+#include "ttt_gemm.cuh"
+#include "ttt_kernels.h"
+
+namespace ttt {
+
+// Device status word shared by the per-kernel entry points (allocated once per process).
+static int* status_word() {
+  static int* p = nullptr;
+  if (!p) {
+    if (cudaMalloc(&p, sizeof(int)) != cudaSuccess) { cudaGetLastError(); p = nullptr; return nullptr; }
+    cudaMemset(p, 0, sizeof(int));
+  }
+  return p;
+}
+
+static int sm_count() {
+  int dev = 0, n = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+template <typename T>
+static int attn_fwd(const AttnParams& ap, int engine, cudaStream_t st) {
+  (void)engine;
+  const int64_t rows = (int64_t)ap.B * ap.n;
+  attn_fwd_simt_kernel<T><<<(unsigned)((rows * ap.H + 3) / 4), 128, 0, st>>>(ap);
+  return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
+template <typename T>
+static int attn_bwd(const AttnParams& ap, int engine, cudaStream_t st) {
+  (void)engine;
+  const int64_t rows = (int64_t)ap.B * ap.n;
+  attn_bwd_prep_kernel<T><<<(unsigned)((rows * ap.H + 7) / 8), 256, 0, st>>>(ap);
+  attn_bwd_dq_simt_kernel<T><<<(unsigned)((rows * ap.H + 3) / 4), 128, 0, st>>>(ap);
+  attn_bwd_dkv_simt_kernel<T><<<(unsigned)((rows * ap.H + 3) / 4), 128, 0, st>>>(ap);
+  return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+}
+
+static AttnParams attn_params(int B, int H, int hd, int n, int64_t q0, int window, const void* qkv, size_t esz,
+                              const void* rk, const void* rv, int C, void* out, float* lse) {
+  AttnParams ap;
+  memset(&ap, 0, sizeof(ap));
+  const int d = H * hd;
+  ap.B = B; ap.H = H; ap.hd = hd; ap.n = n; ap.d = d; ap.q0 = q0; ap.window = window;
+  ap.Q = qkv; ap.ldq = 3 * d;
+  ap.K = (const char*)qkv + (size_t)d * esz;
+  ap.V = (const char*)qkv + (size_t)2 * d * esz;
+  ap.ldkv = 3 * d;
+  ap.Kc = rk; ap.Vc = rv; ap.C = C;
+  ap.O = out; ap.ldo = d; ap.lse = lse;
+  ap.scale = 1.0f / sqrtf((float)hd);
+  return ap;
+}
+
+}  // namespace ttt
+
+using namespace ttt;
+
+extern "C" {
+
+int ttt_k_gemm(int32_t elem_dtype, int32_t M, int32_t N, int32_t K, int32_t batch, const void* A, int64_t lda,
+               int64_t sA, int32_t a_mn, const void* B, int64_t ldb, int64_t sB, int32_t b_mn, void* D, int64_t ldd,
+               int64_t sD, int32_t d_f32, const void* X, int64_t ldx, int64_t sX, void* Y, int64_t ldy, int64_t sY,
+               float alpha, int32_t epi, int32_t engine, void* stream) {
+  if (M < 0 || N < 0 || K < 0 || batch < 1 || !A || !B || !D || epi < 0 || epi > 4) return TTT_ERR_INVALID_ARG;
+  if ((epi == EPI_RESID || epi == EPI_DGELU) && !X) return TTT_ERR_INVALID_ARG;
+  if ((epi == EPI_RESID || epi == EPI_SGD) && !d_f32) return TTT_ERR_INVALID_ARG;
+  int* err = status_word();
+  if (!err) return TTT_ERR_OOM;
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.M = M; p.N = N; p.K = K; p.batch = batch;
+  p.A = A; p.lda = lda; p.sA = sA; p.a_mn = a_mn;
+  p.B = B; p.ldb = ldb; p.sB = sB; p.b_mn = b_mn;
+  p.D = D; p.ldd = ldd; p.sD = sD; p.d_f32 = d_f32;
+  p.X = X; p.ldx = ldx; p.sX = sX;
+  p.Y = Y; p.ldy = ldy; p.sY = sY;
+  p.alpha = alpha; p.epi = epi;
+  const int e = gemm_launch(p, elem_dtype == TTT_BF16 ? 1 : 0, (cudaStream_t)stream, err, sm_count(),
+                            engine == TTT_ENGINE_SIMT);
+  return e == 0 ? TTT_OK : TTT_ERR_CUDA;
+}
+
+int ttt_k_attention_fwd(int32_t elem_dtype, int32_t B, int32_t H, int32_t hd, int32_t n, int64_t q0,
+                        int32_t window, const void* qkv, const void* ring_k, const void* ring_v, int32_t C, void* out,
+                        float* lse, int32_t engine, void* stream) {
+  if (B < 1 || H < 1 || hd < 2 || hd > 128 || n < 1 || window < 1 || !qkv || !out) return TTT_ERR_INVALID_ARG;
+  if (q0 > 0 && (!ring_k || !ring_v || C < window)) return TTT_ERR_INVALID_ARG;
+  const size_t esz = elem_dtype == TTT_BF16 ? 2 : 4;
+  AttnParams ap = attn_params(B, H, hd, n, q0, window, qkv, esz, ring_k, ring_v, C, out, lse);
+  if (elem_dtype == TTT_BF16) return attn_fwd<bf16>(ap, engine, (cudaStream_t)stream);
+  return attn_fwd<float>(ap, engine, (cudaStream_t)stream);
+}
+
+int ttt_k_attention_bwd(int32_t elem_dtype, int32_t B, int32_t H, int32_t hd, int32_t n, int64_t q0,
+                        int32_t window, const void* qkv, const void* ring_k, const void* ring_v, int32_t C,
+                        const void* out, const float* lse, const void* dout, void* dqkv, float* dsum,
+                        int32_t engine, void* stream) {
+  if (B < 1 || H < 1 || hd < 2 || hd > 128 || n < 1 || window < 1 || !qkv || !out || !lse || !dout || !dqkv || !dsum)
+    return TTT_ERR_INVALID_ARG;
+  if (q0 > 0 && (!ring_k || !ring_v || C < window)) return TTT_ERR_INVALID_ARG;
+  const size_t esz = elem_dtype == TTT_BF16 ? 2 : 4;
+  AttnParams ap = attn_params(B, H, hd, n, q0, window, qkv, esz, ring_k, ring_v, C, const_cast<void*>(out),
+                              const_cast<float*>(lse));
+  const int d = H * hd;
+  ap.dO = dout; ap.lddo = d; ap.Dsum = dsum;
+  ap.dQ = dqkv;
+  ap.dK = (char*)dqkv + (size_t)d * esz;
+  ap.dV = (char*)dqkv + (size_t)2 * d * esz;
+  ap.lddq = 3 * d;
+  if (elem_dtype == TTT_BF16) return attn_bwd<bf16>(ap, engine, (cudaStream_t)stream);
+  return attn_bwd<float>(ap, engine, (cudaStream_t)stream);
+}
+
+int ttt_k_status(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) { cudaGetLastError(); return TTT_ERR_CUDA; }
+  int* err = status_word();
+  if (!err) return TTT_ERR_OOM;
+  int flag = 0;
+  if (cudaMemcpy(&flag, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TTT_ERR_CUDA;
+  if (flag) { cudaMemset(err, 0, sizeof(int)); return TTT_ERR_TIMEOUT; }
+  return TTT_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,294 @@
+// Row-wise and elementwise kernels of the TTT-E2E path (HBM-bound work).
+//
+// Rows of d elements, one warp per row, fp32 statistics. Residual streams are
+// fp32; normalised activations (GEMM operands) use the element type T.
+#pragma once
+
+#include "ttt_common.cuh"
+
+namespace ttt {
+
+// ---------------------------------------------------------------- embedding (frozen E)
+// x[row][:] = E[token][:] for rows of [B][n] positions, token = tok[b*tok_ld + tok_off + i].
+template <typename T>
+__global__ void embed_kernel(const int32_t* __restrict__ tok, int64_t tok_ld, int tok_off, int n, int rows,
+                             const T* __restrict__ E, int V, int d, float* __restrict__ x, int* err) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int b = row / n, i = row % n;
+  int t = tok[(int64_t)b * tok_ld + tok_off + i];
+  if (t < 0 || t >= V) {
+    if (lane == 0) set_error(err, DEV_BAD_TOKEN);
+    t = 0;
+  }
+  const T* e = E + (int64_t)t * d;
+  float* o = x + (int64_t)row * d;
+  for (int c = lane; c < d; c += 32) o[c] = to_f32(e[c]);
+}
+
+// ---------------------------------------------------------------- RMSNorm
+// y = g * x / sqrt(mean(x^2) + eps); rstd kept for the backward.
+template <typename T>
+__global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, int64_t ldx, const float* __restrict__ g,
+                                   float eps, int rows, int d, T* __restrict__ y, int64_t ldy,
+                                   float* __restrict__ rstd_out) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const float* xr = x + (int64_t)row * ldx;
+  float ss = 0.f;
+  for (int c = lane * 4; c < d; c += 128) {
+    const float4 v = *(const float4*)(xr + c);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float rs = rsqrtf(ss / d + eps);
+  if (lane == 0 && rstd_out) rstd_out[row] = rs;
+  T* yr = y + (int64_t)row * ldy;
+  for (int c = lane * 4; c < d; c += 128) {
+    const float4 v = *(const float4*)(xr + c);
+    const float4 gg = *(const float4*)(g + c);
+    yr[c] = from_f32<T>(v.x * rs * gg.x);
+    yr[c + 1] = from_f32<T>(v.y * rs * gg.y);
+    yr[c + 2] = from_f32<T>(v.z * rs * gg.z);
+    yr[c + 3] = from_f32<T>(v.w * rs * gg.w);
+  }
+}
+
+// dx = dres + rstd*(g*dy) - x*rstd^3*sum(g*dy*x)/d ; writes fp32 and (optionally) a T copy.
+template <typename T>
+__global__ void rmsnorm_bwd_kernel(const float* __restrict__ x, const float* __restrict__ g,
+                                   const float* __restrict__ rstd, const float* __restrict__ dy,
+                                   const float* dres, int rows, int d, float* dx, T* __restrict__ dx_t) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int64_t o = (int64_t)row * d;
+  float dot = 0.f;
+  for (int c = lane * 4; c < d; c += 128) {
+    const float4 xv = *(const float4*)(x + o + c);
+    const float4 dv = *(const float4*)(dy + o + c);
+    const float4 gv = *(const float4*)(g + c);
+    dot += gv.x * dv.x * xv.x + gv.y * dv.y * xv.y + gv.z * dv.z * xv.z + gv.w * dv.w * xv.w;
+  }
+#pragma unroll
+  for (int s = 16; s; s >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, s);
+  const float rs = rstd[row];
+  const float coef = rs * rs * rs * dot / d;
+  for (int c = lane * 4; c < d; c += 128) {
+    const float4 xv = *(const float4*)(x + o + c);
+    const float4 dv = *(const float4*)(dy + o + c);
+    const float4 gv = *(const float4*)(g + c);
+    float4 r = dres ? *(const float4*)(dres + o + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+    r.x += rs * gv.x * dv.x - xv.x * coef;
+    r.y += rs * gv.y * dv.y - xv.y * coef;
+    r.z += rs * gv.z * dv.z - xv.z * coef;
+    r.w += rs * gv.w * dv.w - xv.w * coef;
+    *(float4*)(dx + o + c) = r;
+    if (dx_t) {
+      dx_t[o + c] = from_f32<T>(r.x);
+      dx_t[o + c + 1] = from_f32<T>(r.y);
+      dx_t[o + c + 2] = from_f32<T>(r.z);
+      dx_t[o + c + 3] = from_f32<T>(r.w);
+    }
+  }
+}
+
+// ---------------------------------------------------------------- RoPE
+// Rotate pairs (i, i+hd/2) of every head in columns [0, ncols) of rows laid out
+// [B][n] at absolute positions pos0 + i. Angles pos * base^(-2i/hd) come from
+// two tables built in double precision on the host:
+//   cos/sin(p*t) from (p = 1024*hi + lo) by the angle-addition identities.
+// inverse != 0 applies the transpose rotation (backward of the forward map).
+template <typename T>
+__global__ void rope_kernel(T* __restrict__ qk, int64_t ld, int ncols, int rows, int n, int64_t pos0, int hd,
+                            const float2* __restrict__ lo_tab, const float2* __restrict__ hi_tab, int inverse) {
+  const int half = hd >> 1;
+  const int pairs_per_row = ncols >> 1;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)rows * pairs_per_row) return;
+  const int row = (int)(idx / pairs_per_row);
+  const int pr = (int)(idx % pairs_per_row);
+  const int head = pr / half, i = pr % half;
+  const int64_t pos = pos0 + (row % n);
+  const float2 a = lo_tab[(pos & 1023) * half + i];   // (cos, sin) of lo * theta_i
+  const float2 b = hi_tab[(pos >> 10) * half + i];    // of 1024*hi * theta_i
+  const float c = a.x * b.x - a.y * b.y;
+  float s = a.y * b.x + a.x * b.y;
+  if (inverse) s = -s;
+  T* base = qk + (int64_t)row * ld + head * hd;
+  const float x1 = to_f32(base[i]), x2 = to_f32(base[i + half]);
+  base[i] = from_f32<T>(x1 * c - x2 * s);
+  base[i + half] = from_f32<T>(x2 * c + x1 * s);
+}
+
+// ---------------------------------------------------------------- window ring
+// Append the K/V of rows [B][n] (positions pos0+i, columns [kcol, kcol+d) and
+// [vcol, vcol+d) of src) to the per-sequence rings [B][C][d] at slot pos % C.
+// Only the last min(n, C) positions are written.
+template <typename T>
+__global__ void kv_append_kernel(const T* __restrict__ src, int64_t ld, int kcol, int vcol, int n, int B,
+                                 int64_t pos0, int d, T* __restrict__ ring_k, T* __restrict__ ring_v, int C) {
+  const int first = n > C ? n - C : 0;
+  const int cnt = n - first;
+  const int per_row = d / 8;  // 16-byte chunks (d % 8 == 0 for bf16; float path uses scalar loop)
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (sizeof(T) == 2) {
+    if (idx >= (int64_t)B * cnt * per_row) return;
+    const int ch = (int)(idx % per_row);
+    const int64_t r = idx / per_row;
+    const int b = (int)(r / cnt), i = first + (int)(r % cnt);
+    const int64_t slot = (pos0 + i) % C;
+    const T* s = src + ((int64_t)b * n + i) * ld;
+    *(uint4*)(ring_k + ((int64_t)b * C + slot) * d + ch * 8) = *(const uint4*)(s + kcol + ch * 8);
+    *(uint4*)(ring_v + ((int64_t)b * C + slot) * d + ch * 8) = *(const uint4*)(s + vcol + ch * 8);
+  } else {
+    if (idx >= (int64_t)B * cnt * d) return;
+    const int c = (int)(idx % d);
+    const int64_t r = idx / d;
+    const int b = (int)(r / cnt), i = first + (int)(r % cnt);
+    const int64_t slot = (pos0 + i) % C;
+    const T* s = src + ((int64_t)b * n + i) * ld;
+    ring_k[((int64_t)b * C + slot) * d + c] = s[kcol + c];
+    ring_v[((int64_t)b * C + slot) * d + c] = s[vcol + c];
+  }
+}
+
+// ---------------------------------------------------------------- cross entropy
+// One CTA per row of logits z [rows][V]. loss = logsumexp(z) - z[target].
+// If grad_scale != 0, z is overwritten in place by dz = (softmax(z) - onehot) * grad_scale.
+// Row r belongs to sequence r / n at chunk offset r % n; its loss goes to
+// loss_out[(r / n) * loss_ld + loss_off + r % n] (skipped when loss_out is null).
+template <typename T>
+__global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ z, int V, const int32_t* __restrict__ targets,
+                                                 int n, float* loss_out, int64_t loss_ld, int64_t loss_off,
+                                                 float grad_scale, int* err) {
+  const int row = blockIdx.x;
+  T* zr = z + (int64_t)row * V;
+  __shared__ float red[32];
+  __shared__ float bc[2];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
+  float mx = -INFINITY;
+  for (int c = tid; c < V; c += blockDim.x) mx = fmaxf(mx, to_f32(zr[c]));
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red[w] = mx;
+  __syncthreads();
+  if (tid == 0) {
+    float m = red[0];
+    for (int i = 1; i < nw; ++i) m = fmaxf(m, red[i]);
+    bc[0] = m;
+  }
+  __syncthreads();
+  mx = bc[0];
+  float se = 0.f;
+  for (int c = tid; c < V; c += blockDim.x) se += expf(to_f32(zr[c]) - mx);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
+  __syncthreads();
+  if (lane == 0) red[w] = se;
+  __syncthreads();
+  if (tid == 0) {
+    float s = 0.f;
+    for (int i = 0; i < nw; ++i) s += red[i];
+    bc[1] = mx + logf(s);
+  }
+  __syncthreads();
+  const float lse = bc[1];
+  int t = targets[row];
+  if (t < 0 || t >= V) {  // ids are validated here too: the last target of a call is never embedded
+    if (tid == 0) set_error(err, DEV_BAD_TOKEN);
+    t = 0;
+  }
+  if (tid == 0 && loss_out) {
+    const int seq = row / n, i = row % n;
+    loss_out[(int64_t)seq * loss_ld + loss_off + i] = lse - to_f32(zr[t]);
+  }
+  if (grad_scale != 0.f) {
+    __syncthreads();  // every thread has read zr[t] before it is overwritten
+    for (int c = tid; c < V; c += blockDim.x) {
+      const float p = expf(to_f32(zr[c]) - lse);
+      zr[c] = from_f32<T>((p - (c == t ? 1.f : 0.f)) * grad_scale);
+    }
+  }
+}
+
+// Greedy choice for decode: argmax (lowest id on ties) unless forced[row] >= 0.
+// Writes chosen id, its loss -log p, and the row's max logit.
+template <typename T>
+__global__ void __launch_bounds__(256) argmax_kernel(const T* __restrict__ z, int V,
+                                                     const int32_t* __restrict__ forced, int32_t* chosen,
+                                                     float* loss, float* zmax_out) {
+  const int row = blockIdx.x;
+  const T* zr = z + (int64_t)row * V;
+  __shared__ float rv[32];
+  __shared__ int ri[32];
+  __shared__ float rs[32];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
+  float best = -INFINITY;
+  int bi = 0x7fffffff;
+  for (int c = tid; c < V; c += blockDim.x) {
+    const float v = to_f32(zr[c]);
+    if (v > best || (v == best && c < bi)) { best = v; bi = c; }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+    if (ov > best || (ov == best && oi < bi)) { best = ov; bi = oi; }
+  }
+  if (lane == 0) { rv[w] = best; ri[w] = bi; }
+  __syncthreads();
+  if (tid == 0) {
+    for (int i = 1; i < nw; ++i)
+      if (rv[i] > rv[0] || (rv[i] == rv[0] && ri[i] < ri[0])) { rv[0] = rv[i]; ri[0] = ri[i]; }
+  }
+  __syncthreads();
+  const float mx = rv[0];
+  float se = 0.f;
+  for (int c = tid; c < V; c += blockDim.x) se += expf(to_f32(zr[c]) - mx);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
+  if (lane == 0) rs[w] = se;
+  __syncthreads();
+  if (tid == 0) {
+    float s = 0.f;
+    for (int i = 0; i < nw; ++i) s += rs[i];
+    const int f = forced ? forced[row] : -1;
+    const int c = (f >= 0 && f < V) ? f : ri[0];
+    chosen[row] = c;
+    loss[row] = mx + logf(s) - to_f32(zr[c]);
+    if (zmax_out) zmax_out[row] = mx;
+  }
+}
+
+// ---------------------------------------------------------------- small copies
+template <typename S, typename D>
+__global__ void convert_kernel(const S* __restrict__ src, D* __restrict__ dst, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) dst[i] = from_f32<D>(to_f32(src[i]));
+}
+
+// Copy rows: dst[b][i][:] = src[b*src_bstride + (off + i)*ld ...] for i < n (fp32 rows of d).
+__global__ void gather_rows_kernel(const float* __restrict__ src, int64_t src_bstride, int64_t off, int n, int B,
+                                   int d, float* __restrict__ dst, int64_t dst_bstride, int64_t dst_off) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t per = (int64_t)n * d;
+  if (idx >= per * B) return;
+  const int b = (int)(idx / per);
+  const int64_t r = idx % per;
+  dst[b * dst_bstride + dst_off * d + r] = src[b * src_bstride + off * d + r];
+}
+
+// targets[b][i] = tok[b*tok_ld + off + i]
+__global__ void gather_tokens_kernel(const int32_t* __restrict__ tok, int64_t tok_ld, int64_t off, int n, int B,
+                                     int32_t* __restrict__ out, int64_t out_bstride, int64_t out_off) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n * B) return;
+  const int b = idx / n, i = idx % n;
+  out[b * out_bstride + out_off + i] = tok[(int64_t)b * tok_ld + off + i];
+}
+
+}  // namespace ttt

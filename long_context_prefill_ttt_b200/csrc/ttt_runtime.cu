@@ -1,0 +1,979 @@
+// Runtime of the TTT-E2E inner loop: device state, the prefill schedule
+// (Algorithm 1 of the technical review, §7) and the decode schedule
+// (Algorithm 3), behind the C ABI declared in include/ttt.h.
+//
+// Schedule of one prefill call over T positions of B sequences:
+//   for each segment of S positions (S a multiple of b):
+//     frozen phase: embedding, then every frozen block over all B*S rows at
+//       once (ordinary parallel sliding-window prefill; the frozen blocks do
+//       not depend on the fast weights);
+//     adaptive phase: for each chunk of b positions, in order (the chain
+//       W_{i-1} -> loss_i -> grad -> W_i is serial):
+//       forward of the adaptive blocks with W_{i-1}, LM head + cross-entropy
+//       (losses recorded before any update), backward into every adaptive
+//       MLP's weights, and the SGD update fused into the weight-gradient GEMM.
+// Window caches: per layer and sequence a ring of C = roundup(k + b, 128)
+// positions. Rows of the current segment/chunk are read directly; older
+// positions from the ring. K/V are appended after use and never recomputed.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "ttt.h"
+#include "ttt_attention.cuh"
+#include "ttt_common.cuh"
+#include "ttt_gemm.cuh"
+#include "ttt_ops.cuh"
+
+namespace ttt {
+
+// ============================================================== GEMM dispatch (host)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)ptr;
+  }
+  return fn;
+}
+
+// Operand map: logical [rows][K] (K-major, box {64, box_rows}) or logical [rows][K]
+// stored [K][rows] (MN-major, box {64, 64}). 128-byte swizzle, zero fill out of range.
+static bool make_operand_map(CUtensorMap* map, const void* base, int64_t rows, int64_t K, int64_t ld,
+                             int64_t batch, int64_t bstride, bool mn_major, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3], estr[3] = {1, 1, 1};
+  if (!mn_major) {
+    dims[0] = (cuuint64_t)K; dims[1] = (cuuint64_t)rows;
+    box[0] = 64; box[1] = (cuuint32_t)box_rows;
+  } else {
+    dims[0] = (cuuint64_t)rows; dims[1] = (cuuint64_t)K;
+    box[0] = 64; box[1] = 64;
+  }
+  dims[2] = (cuuint64_t)batch;
+  box[2] = 1;
+  strides[0] = (cuuint64_t)ld * 2;
+  strides[1] = (cuuint64_t)(batch > 1 ? bstride : (mn_major ? K : rows) * ld) * 2;
+  if (strides[1] == 0) strides[1] = strides[0];
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+template <int BN, bool AM, bool BM>
+static cudaError_t launch_tc(const GemmParams& p, cudaStream_t st, int* err, int num_sms, bool* ok) {
+  CUtensorMap ta, tb;
+  *ok = make_operand_map(&ta, p.A, p.M, p.K, p.lda, p.batch, p.sA, AM, TC_BM) &&
+        make_operand_map(&tb, p.B, p.N, p.K, p.ldb, p.batch, p.sB, BM, BN);
+  if (!*ok) return cudaSuccess;
+  using C = TcCfg<BN>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, AM, BM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int tiles = ((p.M + TC_BM - 1) / TC_BM) * (p.N / BN) * p.batch;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  gemm_tc_kernel<BN, AM, BM><<<grid, TC_THREADS, C::SMEM, st>>>(ta, tb, p, err);
+  return cudaGetLastError();
+}
+
+// Returns 0 on success, or a cudaError_t value.
+int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err, int num_sms, int force_simt) {
+  if (p.M <= 0 || p.N <= 0 || p.K <= 0 || p.batch <= 0) return 0;
+  bool use_tc = elem_is_bf16 && !force_simt && (p.K % TC_BK == 0) && (p.N % 128 == 0) && aligned16(p.A) &&
+                aligned16(p.B) && aligned16(p.D) && (p.lda % 8 == 0) && (p.ldb % 8 == 0) &&
+                (p.ldd % (p.d_f32 || p.epi == EPI_RESID || p.epi == EPI_SGD ? 4 : 8) == 0) &&
+                (p.batch == 1 || (p.sA % 8 == 0 && p.sB % 8 == 0)) && (!p.a_mn || p.b_mn) && p.M >= 1;
+  if (use_tc && p.X && !(aligned16(p.X) && p.ldx % (p.epi == EPI_DGELU ? 8 : 4) == 0 &&
+                         (p.batch == 1 || p.sX % 8 == 0)))
+    use_tc = false;
+  if (use_tc && p.batch > 1 && p.sD % 8 != 0) use_tc = false;
+  if (use_tc && p.Y && !(aligned16(p.Y) && p.ldy % 8 == 0 && (p.batch == 1 || p.sY % 8 == 0))) use_tc = false;
+  if (use_tc) {
+    const int m_tiles = (p.M + TC_BM - 1) / TC_BM;
+    const bool n256 = (p.N % 256 == 0) && (m_tiles * (p.N / 256) * p.batch >= (num_sms * 9) / 10);
+    bool ok = false;
+    cudaError_t e;
+    if (!p.a_mn && !p.b_mn)
+      e = n256 ? launch_tc<256, false, false>(p, st, err, num_sms, &ok) : launch_tc<128, false, false>(p, st, err, num_sms, &ok);
+    else if (!p.a_mn && p.b_mn)
+      e = n256 ? launch_tc<256, false, true>(p, st, err, num_sms, &ok) : launch_tc<128, false, true>(p, st, err, num_sms, &ok);
+    else
+      e = n256 ? launch_tc<256, true, true>(p, st, err, num_sms, &ok) : launch_tc<128, true, true>(p, st, err, num_sms, &ok);
+    if (e != cudaSuccess) return (int)e;
+    if (ok) return 0;
+  }
+  dim3 grid((p.N + 63) / 64, (p.M + 63) / 64, p.batch);
+  if (elem_is_bf16)
+    gemm_simt_kernel<bf16><<<grid, 256, 0, st>>>(p);
+  else
+    gemm_simt_kernel<float><<<grid, 256, 0, st>>>(p);
+  return (int)cudaGetLastError();
+}
+
+// ============================================================== device memory
+struct Arena {
+  std::vector<void*> ptrs;
+  int64_t bytes = 0;
+  bool failed = false;
+  void* alloc(size_t n) {
+    if (n == 0) n = 16;
+    n = (n + 255) & ~(size_t)255;
+    void* p = nullptr;
+    if (cudaMalloc(&p, n) != cudaSuccess) {
+      cudaGetLastError();
+      failed = true;
+      return nullptr;
+    }
+    ptrs.push_back(p);
+    bytes += (int64_t)n;
+    return p;
+  }
+  template <typename X> X* get(size_t count) { return (X*)alloc(count * sizeof(X)); }
+  void release() {
+    for (void* p : ptrs) cudaFree(p);
+    ptrs.clear();
+    bytes = 0;
+  }
+};
+
+}  // namespace ttt
+
+// ============================================================== handle
+struct ttt_handle {
+  virtual ~ttt_handle() {}
+  virtual int prefill(const int32_t* tokens, int64_t T, float* out, int32_t kind) = 0;
+  virtual int decode(int64_t n, const int32_t* forced, int32_t* out_tok, float* out_loss, int32_t kind) = 0;
+  virtual int get_weights(int32_t seq, int32_t blk, float* w1, float* w2, int32_t kind) = 0;
+  virtual int reset() = 0;
+  std::string err_msg;
+  bool poisoned = false;
+  int64_t n_pos = 0;
+  int64_t launches = 0;
+  int64_t dev_bytes = 0;
+};
+
+namespace ttt {
+
+static int fail(ttt_handle* h, int code, const std::string& msg) {
+  if (h) h->err_msg = msg;
+  return code;
+}
+
+#define TTT_CUDA(call)                                                                           \
+  do {                                                                                           \
+    cudaError_t _e = (call);                                                                     \
+    if (_e != cudaSuccess) {                                                                     \
+      poisoned = true;                                                                           \
+      return fail(this, TTT_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(_e));       \
+    }                                                                                            \
+  } while (0)
+
+#define TTT_LAUNCHED()                                                                           \
+  do {                                                                                           \
+    ++launches;                                                                                  \
+    cudaError_t _e = cudaGetLastError();                                                         \
+    if (_e != cudaSuccess) {                                                                     \
+      poisoned = true;                                                                           \
+      return fail(this, TTT_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(_e));         \
+    }                                                                                            \
+  } while (0)
+
+static inline unsigned nblk(int64_t n, int t) { return (unsigned)((n + t - 1) / t); }
+
+// Per-layer device weights and caches.
+template <typename T> struct LayerDev {
+  float* g_attn = nullptr;
+  T* Wqkv = nullptr;  // [3d][d]
+  T* Wo = nullptr;    // [d][d]
+  float* g_mlp = nullptr; T* W1 = nullptr; T* W2 = nullptr;           // frozen MLP
+  float* g_ttt = nullptr; float* g_static = nullptr;                   // adaptive block
+  T* W1s = nullptr; T* W2s = nullptr;
+  float* W1t32 = nullptr; float* W2t32 = nullptr;                      // [B][ht][d], [B][d][ht] master
+  T* W1t = nullptr; T* W2t = nullptr;                                  // shadows (alias master for fp32)
+  float* W1t_init = nullptr; float* W2t_init = nullptr;                // W_init (one copy)
+  T* ring_k = nullptr; T* ring_v = nullptr;                            // [B][C][d]
+};
+
+// Activations of one adaptive block kept for the backward (rows Mc = B*b).
+template <typename T> struct BlockAct {
+  float* x; float* rstd1; T* qkv; T* o; float* lse; float* a; float* rstd2; T* r2; T* u; T* g;
+  float* m; float* rstd3; T* r3; T* us; T* gs;
+};
+
+template <typename T> class Engine : public ttt_handle {
+ public:
+  ttt_config cfg;
+  cudaStream_t st = nullptr;
+  int num_sms = 148;
+  int B, d, V, L, Lt, H, hd, h, ht, hs, kwin, bsz, C, S;
+  int first_ttt;
+  bool is_bf16;
+  Arena arena;
+  int* dev_err = nullptr;
+  T* E = nullptr;
+  float* g_final = nullptr;
+  float2* rope_lo = nullptr;
+  float2* rope_hi = nullptr;
+  static constexpr int kRopeHi = 16384;  // positions < 16384 * 1024
+  std::vector<LayerDev<T>> layers;
+  // frozen-phase segment buffers (Ms = B*S rows)
+  float* xs = nullptr; T* rs = nullptr; T* qkvs = nullptr; T* os = nullptr; T* hids = nullptr;
+  // adaptive-phase buffers (Mc = B*b rows)
+  std::vector<BlockAct<T>> blk;
+  float* tin = nullptr; float* y = nullptr; float* rstdf = nullptr; T* rf = nullptr; T* z = nullptr;
+  int32_t* tgt = nullptr;
+  float* G = nullptr; T* GT = nullptr; T* dhid = nullptr; float* dr = nullptr; T* dqkv = nullptr;
+  T* dob = nullptr; float* Dsum = nullptr;
+  // pending (incomplete) chunk: inputs of the first adaptive block and targets
+  float* pend_in = nullptr; int32_t* pend_tgt = nullptr; int pend_cnt = 0;
+  int32_t* pend_tok_dev = nullptr;        // [B] pending input id of each sequence
+  std::vector<int32_t> pend_tok_host;
+  // decode scratch
+  int32_t* chosen = nullptr; float* dec_loss = nullptr; float* dec_zmax = nullptr; int32_t* forced_col = nullptr;
+  // per-call growable buffers
+  int64_t chunk_pos = 0;                  // absolute position of row 0 of the chunk in the adaptive buffers
+  int32_t* tok_dev = nullptr; int64_t tok_cap = 0;
+  float* loss_dev = nullptr; int64_t loss_cap = 0;
+  int32_t* otok_dev = nullptr; int64_t otok_cap = 0;
+  Arena call_arena;
+
+  ~Engine() override {
+    if (st) cudaStreamSynchronize(st);
+    call_arena.release();
+    arena.release();
+  }
+
+  int create(const ttt_config* c, const ttt_weights* w);
+  int prefill(const int32_t* tokens, int64_t T_, float* out, int32_t kind) override;
+  int decode(int64_t n, const int32_t* forced, int32_t* out_tok, float* out_loss, int32_t kind) override;
+  int get_weights(int32_t seq, int32_t blk, float* w1, float* w2, int32_t kind) override;
+  int reset() override;
+
+ private:
+  int gemm(GemmParams p) {
+    const int e = gemm_launch(p, is_bf16 ? 1 : 0, st, dev_err, num_sms, 0);
+    ++launches;
+    if (e != 0) {
+      poisoned = true;
+      return fail(this, TTT_ERR_CUDA, std::string("gemm: ") + cudaGetErrorString((cudaError_t)e));
+    }
+    return TTT_OK;
+  }
+  static GemmParams gp(int M, int N, int K, const void* A, int64_t lda, bool a_mn, const void* Bm, int64_t ldb,
+                       bool b_mn, void* D, int64_t ldd, bool d_f32, int epi) {
+    GemmParams p;
+    memset(&p, 0, sizeof(p));
+    p.M = M; p.N = N; p.K = K; p.batch = 1;
+    p.A = A; p.lda = lda; p.a_mn = a_mn;
+    p.B = Bm; p.ldb = ldb; p.b_mn = b_mn;
+    p.D = D; p.ldd = ldd; p.d_f32 = d_f32;
+    p.alpha = 1.f; p.epi = epi;
+    return p;
+  }
+  int attention_block(const LayerDev<T>& Lw, int layer, float* xin, float* xout, T* r, float* rstd, T* qkv, T* o,
+                      float* lse, int n, int64_t q0, bool commit);
+  int frozen_mlp(const LayerDev<T>& Lw, float* x, T* r, T* hid, int rows);
+  int ttt_forward(int cn, int64_t pos, bool commit);
+  int ttt_backward(int cn);
+  int ttt_step(const float* in, const int32_t* targets, int cn, int64_t pos, float* loss_out, int64_t loss_ld,
+               int64_t loss_off, bool grad, bool commit);
+  int sync_and_check();
+  int ensure(void** ptr, int64_t* cap, int64_t need, size_t elem);
+};
+
+template <typename T> int Engine<T>::ensure(void** ptr, int64_t* cap, int64_t need, size_t elem) {
+  if (need <= *cap) return TTT_OK;
+  void* p = call_arena.alloc((size_t)need * elem);
+  if (!p) return fail(this, TTT_ERR_OOM, "device allocation failed (call buffers)");
+  *ptr = p;
+  *cap = need;
+  dev_bytes = arena.bytes + call_arena.bytes;
+  return TTT_OK;
+}
+
+template <typename T> int Engine<T>::sync_and_check() {
+  TTT_CUDA(cudaStreamSynchronize(st));
+  int flag = 0;
+  TTT_CUDA(cudaMemcpy(&flag, dev_err, sizeof(int), cudaMemcpyDeviceToHost));
+  if (flag == DEV_BAD_TOKEN) {
+    TTT_CUDA(cudaMemset(dev_err, 0, sizeof(int)));
+    poisoned = true;  // the call ran with a clamped id; the state is no longer meaningful
+    return fail(this, TTT_ERR_INVALID_ARG, "token id outside [0, vocab)");
+  }
+  if (flag != 0) {
+    poisoned = true;
+    return fail(this, TTT_ERR_TIMEOUT, "device wait expired (code " + std::to_string(flag) + ")");
+  }
+  return TTT_OK;
+}
+
+// ------------------------------------------------------------------ create
+template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weights* w) {
+  cfg = *c;
+  st = (cudaStream_t)cfg.cuda_stream;
+  B = cfg.batch; d = cfg.d; V = cfg.vocab; L = cfg.n_layers; Lt = cfg.n_ttt; H = cfg.n_heads;
+  hd = d / H; h = cfg.mlp_hidden; ht = cfg.ttt_hidden; hs = cfg.static_hidden; kwin = cfg.window_k;
+  bsz = cfg.minibatch_b;
+  first_ttt = L - Lt;
+  is_bf16 = cfg.dtype == TTT_BF16;
+  C = ((kwin + bsz + 127) / 128) * 128;
+  int seg = cfg.max_segment > 0 ? cfg.max_segment : 32768;
+  S = ((seg + bsz - 1) / bsz) * bsz;
+  int dev = 0;
+  TTT_CUDA(cudaGetDevice(&dev));
+  TTT_CUDA(cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev));
+
+  const int64_t Ms = (int64_t)B * S, Mc = (int64_t)B * bsz;
+  dev_err = arena.get<int>(1);
+  E = arena.get<T>((size_t)V * d);
+  g_final = arena.get<float>(d);
+  rope_lo = arena.get<float2>((size_t)1024 * (hd / 2));
+  rope_hi = arena.get<float2>((size_t)kRopeHi * (hd / 2));
+  layers.resize(L);
+  for (int l = 0; l < L; ++l) {
+    LayerDev<T>& Lw = layers[l];
+    Lw.g_attn = arena.get<float>(d);
+    Lw.Wqkv = arena.get<T>((size_t)3 * d * d);
+    Lw.Wo = arena.get<T>((size_t)d * d);
+    Lw.ring_k = arena.get<T>((size_t)B * C * d);
+    Lw.ring_v = arena.get<T>((size_t)B * C * d);
+    if (l < first_ttt) {
+      Lw.g_mlp = arena.get<float>(d);
+      Lw.W1 = arena.get<T>((size_t)h * d);
+      Lw.W2 = arena.get<T>((size_t)d * h);
+    } else {
+      Lw.g_ttt = arena.get<float>(d);
+      Lw.g_static = arena.get<float>(d);
+      Lw.W1s = arena.get<T>((size_t)hs * d);
+      Lw.W2s = arena.get<T>((size_t)d * hs);
+      Lw.W1t32 = arena.get<float>((size_t)B * ht * d);
+      Lw.W2t32 = arena.get<float>((size_t)B * d * ht);
+      Lw.W1t_init = arena.get<float>((size_t)ht * d);
+      Lw.W2t_init = arena.get<float>((size_t)d * ht);
+      if (is_bf16) {
+        Lw.W1t = arena.get<T>((size_t)B * ht * d);
+        Lw.W2t = arena.get<T>((size_t)B * d * ht);
+      } else {
+        Lw.W1t = (T*)Lw.W1t32;
+        Lw.W2t = (T*)Lw.W2t32;
+      }
+    }
+  }
+  const int hmax = h > ht ? (h > hs ? h : hs) : (ht > hs ? ht : hs);
+  xs = arena.get<float>((size_t)Ms * d);
+  rs = arena.get<T>((size_t)Ms * d);
+  qkvs = arena.get<T>((size_t)Ms * 3 * d);
+  os = arena.get<T>((size_t)Ms * d);
+  hids = arena.get<T>((size_t)Ms * hmax);
+  blk.resize(Lt);
+  for (int j = 0; j < Lt; ++j) {
+    BlockAct<T>& A = blk[j];
+    A.x = arena.get<float>((size_t)Mc * d);
+    A.rstd1 = arena.get<float>(Mc);
+    A.qkv = arena.get<T>((size_t)Mc * 3 * d);
+    A.o = arena.get<T>((size_t)Mc * d);
+    A.lse = arena.get<float>((size_t)B * H * bsz);
+    A.a = arena.get<float>((size_t)Mc * d);
+    A.rstd2 = arena.get<float>(Mc);
+    A.r2 = arena.get<T>((size_t)Mc * d);
+    A.u = arena.get<T>((size_t)Mc * ht);
+    A.g = arena.get<T>((size_t)Mc * ht);
+    A.m = arena.get<float>((size_t)Mc * d);
+    A.rstd3 = arena.get<float>(Mc);
+    A.r3 = arena.get<T>((size_t)Mc * d);
+    A.us = arena.get<T>((size_t)Mc * hs);
+    A.gs = arena.get<T>((size_t)Mc * hs);
+  }
+  tin = blk.empty() ? nullptr : blk[0].x;
+  y = arena.get<float>((size_t)Mc * d);
+  rstdf = arena.get<float>(Mc);
+  rf = arena.get<T>((size_t)Mc * d);
+  z = arena.get<T>((size_t)Mc * V);
+  tgt = arena.get<int32_t>(Mc);
+  G = arena.get<float>((size_t)Mc * d);
+  GT = arena.get<T>((size_t)Mc * d);
+  dhid = arena.get<T>((size_t)Mc * (ht > hs ? ht : hs));
+  dr = arena.get<float>((size_t)Mc * d);
+  dqkv = arena.get<T>((size_t)Mc * 3 * d);
+  dob = arena.get<T>((size_t)Mc * d);
+  Dsum = arena.get<float>((size_t)B * H * bsz);
+  pend_in = arena.get<float>((size_t)Mc * d);
+  pend_tgt = arena.get<int32_t>(Mc);
+  pend_tok_dev = arena.get<int32_t>(B);
+  chosen = arena.get<int32_t>(B);
+  dec_loss = arena.get<float>(B);
+  dec_zmax = arena.get<float>(B);
+  forced_col = arena.get<int32_t>(B);
+  if (arena.failed) {
+    arena.release();
+    return fail(this, TTT_ERR_OOM, "device allocation failed");
+  }
+  dev_bytes = arena.bytes;
+  TTT_CUDA(cudaMemsetAsync(dev_err, 0, sizeof(int), st));
+
+  // RoPE tables in double precision: lo[p][i] = angle p*theta_i (p < 1024), hi[q][i] = angle 1024*q*theta_i
+  {
+    const int half = hd / 2;
+    std::vector<float2> lo((size_t)1024 * half), hi((size_t)kRopeHi * half);
+    for (int i = 0; i < half; ++i) {
+      const double theta = std::pow((double)cfg.rope_base, -2.0 * i / hd);
+      for (int p = 0; p < 1024; ++p) {
+        const double a = p * theta;
+        lo[(size_t)p * half + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+      }
+      for (int q = 0; q < kRopeHi; ++q) {
+        const double a = 1024.0 * q * theta;
+        hi[(size_t)q * half + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+      }
+    }
+    TTT_CUDA(cudaMemcpyAsync(rope_lo, lo.data(), lo.size() * sizeof(float2), cudaMemcpyHostToDevice, st));
+    TTT_CUDA(cudaMemcpyAsync(rope_hi, hi.data(), hi.size() * sizeof(float2), cudaMemcpyHostToDevice, st));
+    TTT_CUDA(cudaStreamSynchronize(st));
+  }
+
+  // weights: stage each tensor on the device, then convert into place
+  const bool src_bf16 = w->values_dtype == TTT_BF16;
+  const size_t src_elem = src_bf16 ? 2 : 4;
+  int64_t max_elems = (int64_t)V * d;
+  if ((int64_t)h * d > max_elems) max_elems = (int64_t)h * d;
+  if ((int64_t)ht * d > max_elems) max_elems = (int64_t)ht * d;
+  if ((int64_t)hs * d > max_elems) max_elems = (int64_t)hs * d;
+  void* stage = nullptr;
+  if (w->ptr_kind == TTT_PTR_HOST) {
+    TTT_CUDA(cudaMalloc(&stage, (size_t)max_elems * 4));
+  }
+  int ti = 0;
+  auto upload = [&](void* dst, bool dst_f32, int64_t count, bool gain) -> int {
+    const void* src = w->tensors[ti++];
+    if (!src) return fail(this, TTT_ERR_INVALID_ARG, "null weight tensor " + std::to_string(ti - 1));
+    const size_t es = gain ? 4 : src_elem;
+    const void* dsrc = src;
+    if (w->ptr_kind == TTT_PTR_HOST) {
+      TTT_CUDA(cudaMemcpyAsync(stage, src, (size_t)count * es, cudaMemcpyHostToDevice, st));
+      dsrc = stage;
+    }
+    const unsigned g = nblk(count, 256);
+    if (gain || !src_bf16) {
+      if (dst_f32) convert_kernel<float, float><<<g, 256, 0, st>>>((const float*)dsrc, (float*)dst, count);
+      else convert_kernel<float, T><<<g, 256, 0, st>>>((const float*)dsrc, (T*)dst, count);
+    } else {
+      if (dst_f32) convert_kernel<bf16, float><<<g, 256, 0, st>>>((const bf16*)dsrc, (float*)dst, count);
+      else convert_kernel<bf16, T><<<g, 256, 0, st>>>((const bf16*)dsrc, (T*)dst, count);
+    }
+    TTT_LAUNCHED();
+    if (w->ptr_kind == TTT_PTR_HOST) TTT_CUDA(cudaStreamSynchronize(st));  // stage reuse
+    return TTT_OK;
+  };
+  int rc;
+#define UP(dst, f32, cnt, gain) if ((rc = upload((dst), (f32), (cnt), (gain))) != TTT_OK) { if (stage) cudaFree(stage); return rc; }
+  UP(E, false, (int64_t)V * d, false);
+  UP(g_final, true, d, true);
+  const int64_t dd = (int64_t)d * d;
+  for (int l = 0; l < L; ++l) {
+    LayerDev<T>& Lw = layers[l];
+    UP(Lw.g_attn, true, d, true);
+    UP(Lw.Wqkv, false, dd, false);
+    UP(Lw.Wqkv + dd, false, dd, false);
+    UP(Lw.Wqkv + 2 * dd, false, dd, false);
+    UP(Lw.Wo, false, dd, false);
+    if (l < first_ttt) {
+      UP(Lw.g_mlp, true, d, true);
+      UP(Lw.W1, false, (int64_t)h * d, false);
+      UP(Lw.W2, false, (int64_t)d * h, false);
+    } else {
+      UP(Lw.g_ttt, true, d, true);
+      UP(Lw.W1t_init, true, (int64_t)ht * d, false);
+      UP(Lw.W2t_init, true, (int64_t)d * ht, false);
+      UP(Lw.g_static, true, d, true);
+      UP(Lw.W1s, false, (int64_t)hs * d, false);
+      UP(Lw.W2s, false, (int64_t)d * hs, false);
+    }
+  }
+#undef UP
+  if (stage) cudaFree(stage);
+  return reset();
+}
+
+template <typename T> int Engine<T>::reset() {
+  if (poisoned) return fail(this, TTT_ERR_POISONED, "handle poisoned by an earlier device error");
+  for (int l = first_ttt; l < L; ++l) {
+    LayerDev<T>& Lw = layers[l];
+    const int64_t n1 = (int64_t)ht * d;
+    for (int b = 0; b < B; ++b) {
+      TTT_CUDA(cudaMemcpyAsync(Lw.W1t32 + b * n1, Lw.W1t_init, n1 * 4, cudaMemcpyDeviceToDevice, st));
+      TTT_CUDA(cudaMemcpyAsync(Lw.W2t32 + b * n1, Lw.W2t_init, n1 * 4, cudaMemcpyDeviceToDevice, st));
+    }
+    if (is_bf16) {
+      convert_kernel<float, T><<<nblk(B * n1, 256), 256, 0, st>>>(Lw.W1t32, Lw.W1t, B * n1);
+      TTT_LAUNCHED();
+      convert_kernel<float, T><<<nblk(B * n1, 256), 256, 0, st>>>(Lw.W2t32, Lw.W2t, B * n1);
+      TTT_LAUNCHED();
+    }
+  }
+  for (int l = 0; l < L; ++l) {
+    TTT_CUDA(cudaMemsetAsync(layers[l].ring_k, 0, (size_t)B * C * d * sizeof(T), st));
+    TTT_CUDA(cudaMemsetAsync(layers[l].ring_v, 0, (size_t)B * C * d * sizeof(T), st));
+  }
+  n_pos = 0;
+  pend_cnt = 0;
+  pend_tok_host.assign(B, -1);
+  return sync_and_check();
+}
+
+// ------------------------------------------------------------------ blocks
+// Pre-norm attention sub-block over rows [B][n] at positions q0 + i:
+// xout = xin + Wo * Attn(RoPE(Wq r), RoPE(Wk r), Wv r), r = RMSNorm(xin).
+template <typename T>
+int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, float* xout, T* r, float* rstd, T* qkv,
+                               T* o, float* lse, int n, int64_t q0, bool commit) {
+  const int rows = B * n;
+  int rc;
+  rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(xin, d, Lw.g_attn, cfg.rms_eps, rows, d, r, d, rstd);
+  TTT_LAUNCHED();
+  if ((rc = gemm(gp(rows, 3 * d, d, r, d, false, Lw.Wqkv, d, false, qkv, 3 * d, false, EPI_STORE))) != TTT_OK)
+    return rc;
+  rope_kernel<T><<<nblk((int64_t)rows * d, 256), 256, 0, st>>>(qkv, 3 * d, 2 * d, rows, n, q0, hd, rope_lo, rope_hi,
+                                                                0);
+  TTT_LAUNCHED();
+  AttnParams ap;
+  memset(&ap, 0, sizeof(ap));
+  ap.B = B; ap.H = H; ap.hd = hd; ap.n = n; ap.d = d; ap.q0 = q0; ap.window = kwin;
+  ap.Q = qkv; ap.ldq = 3 * d; ap.K = qkv + d; ap.V = qkv + 2 * d; ap.ldkv = 3 * d;
+  ap.Kc = Lw.ring_k; ap.Vc = Lw.ring_v; ap.C = C;
+  ap.O = o; ap.ldo = d; ap.lse = lse; ap.scale = 1.0f / sqrtf((float)hd);
+  attn_fwd_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
+  TTT_LAUNCHED();
+  GemmParams p = gp(rows, d, d, o, d, false, Lw.Wo, d, false, xout, d, true, EPI_RESID);
+  p.X = xin; p.ldx = d;
+  if ((rc = gemm(p)) != TTT_OK) return rc;
+  if (commit) {
+    const int cnt = n > C ? C : n;
+    const int64_t work = sizeof(T) == 2 ? (int64_t)B * cnt * (d / 8) : (int64_t)B * cnt * d;
+    kv_append_kernel<T><<<nblk(work, 256), 256, 0, st>>>(qkv, 3 * d, d, 2 * d, n, B, q0, d, Lw.ring_k, Lw.ring_v,
+                                                         C);
+    TTT_LAUNCHED();
+  }
+  return TTT_OK;
+}
+
+// x += W2 gelu(W1 RMSNorm(x)) (frozen blocks)
+template <typename T> int Engine<T>::frozen_mlp(const LayerDev<T>& Lw, float* x, T* r, T* hid, int rows) {
+  int rc;
+  rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(x, d, Lw.g_mlp, cfg.rms_eps, rows, d, r, d, nullptr);
+  TTT_LAUNCHED();
+  if ((rc = gemm(gp(rows, h, d, r, d, false, Lw.W1, d, false, hid, h, false, EPI_GELU))) != TTT_OK) return rc;
+  GemmParams p = gp(rows, d, h, hid, h, false, Lw.W2, h, false, x, d, true, EPI_RESID);
+  p.X = x; p.ldx = d;
+  return gemm(p);
+}
+
+// Forward of the adaptive blocks for cn positions per sequence at pos..pos+cn-1.
+// Input in blk[0].x, output in y. Activations of each block stay in blk[j].
+template <typename T> int Engine<T>::ttt_forward(int cn, int64_t pos, bool commit) {
+  const int rows = B * cn;
+  int rc;
+  for (int j = 0; j < Lt; ++j) {
+    const int l = first_ttt + j;
+    const LayerDev<T>& Lw = layers[l];
+    BlockAct<T>& A = blk[j];
+    if ((rc = attention_block(Lw, l, A.x, A.a, A.r3 /*scratch for r1*/, A.rstd1, A.qkv, A.o, A.lse, cn, pos,
+                              commit)) != TTT_OK)
+      return rc;
+    // TTT-MLP with the fast weights of each sequence (batched over sequences)
+    rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(A.a, d, Lw.g_ttt, cfg.rms_eps, rows, d, A.r2, d, A.rstd2);
+    TTT_LAUNCHED();
+    GemmParams p = gp(cn, ht, d, A.r2, d, false, Lw.W1t, d, false, A.g, ht, false, EPI_GELU);
+    p.batch = B; p.sA = (int64_t)cn * d; p.sB = (int64_t)ht * d; p.sD = (int64_t)cn * ht;
+    p.Y = A.u; p.ldy = ht; p.sY = (int64_t)cn * ht;
+    if ((rc = gemm(p)) != TTT_OK) return rc;
+    p = gp(cn, d, ht, A.g, ht, false, Lw.W2t, ht, false, A.m, d, true, EPI_RESID);
+    p.batch = B; p.sA = (int64_t)cn * ht; p.sB = (int64_t)d * ht; p.sD = (int64_t)cn * d;
+    p.X = A.a; p.ldx = d; p.sX = (int64_t)cn * d;
+    if ((rc = gemm(p)) != TTT_OK) return rc;
+    // static MLP
+    rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(A.m, d, Lw.g_static, cfg.rms_eps, rows, d, A.r3, d,
+                                                         A.rstd3);
+    TTT_LAUNCHED();
+    p = gp(rows, hs, d, A.r3, d, false, Lw.W1s, d, false, A.gs, hs, false, EPI_GELU);
+    p.Y = A.us; p.ldy = hs;
+    if ((rc = gemm(p)) != TTT_OK) return rc;
+    float* xnext = (j + 1 < Lt) ? blk[j + 1].x : y;
+    p = gp(rows, d, hs, A.gs, hs, false, Lw.W2s, hs, false, xnext, d, true, EPI_RESID);
+    p.X = A.m; p.ldx = d;
+    if ((rc = gemm(p)) != TTT_OK) return rc;
+  }
+  return TTT_OK;
+}
+
+// Reverse mode from dz (in z) back to every adaptive MLP, with the SGD step
+// fused into the weight-gradient GEMMs (W <- W - eta * dW, dW already a mean).
+template <typename T> int Engine<T>::ttt_backward(int cn) {
+  const int rows = B * cn;
+  int rc;
+  // LM head: dr = dz E ; G = d loss / d y through the final RMSNorm
+  if ((rc = gemm(gp(rows, d, V, z, V, false, E, d, true, dr, d, true, EPI_STORE))) != TTT_OK) return rc;
+  rmsnorm_bwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(y, g_final, rstdf, dr, nullptr, rows, d, G, GT);
+  TTT_LAUNCHED();
+  for (int j = Lt - 1; j >= 0; --j) {
+    const int l = first_ttt + j;
+    const LayerDev<T>& Lw = layers[l];
+    BlockAct<T>& A = blk[j];
+    // static MLP (frozen): dm = G + RMSNorm_bwd(W1s^T (gelu'(us) * (W2s^T G)))
+    GemmParams p = gp(rows, hs, d, GT, d, false, Lw.W2s, hs, true, dhid, hs, false, EPI_DGELU);
+    p.X = A.us; p.ldx = hs;
+    if ((rc = gemm(p)) != TTT_OK) return rc;
+    if ((rc = gemm(gp(rows, d, hs, dhid, hs, false, Lw.W1s, d, true, dr, d, true, EPI_STORE))) != TTT_OK) return rc;
+    rmsnorm_bwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(A.m, Lw.g_static, A.rstd3, dr, G, rows, d, G, GT);
+    TTT_LAUNCHED();
+    // TTT-MLP data gradients (with W_{i-1}), then the fused weight gradient + SGD
+    p = gp(cn, ht, d, GT, d, false, Lw.W2t, ht, true, dhid, ht, false, EPI_DGELU);
+    p.batch = B; p.sA = (int64_t)cn * d; p.sB = (int64_t)d * ht; p.sD = (int64_t)cn * ht;
+    p.X = A.u; p.ldx = ht; p.sX = (int64_t)cn * ht;
+    if ((rc = gemm(p)) != TTT_OK) return rc;
+    if (j > 0) {
+      p = gp(cn, d, ht, dhid, ht, false, Lw.W1t, d, true, dr, d, true, EPI_STORE);
+      p.batch = B; p.sA = (int64_t)cn * ht; p.sB = (int64_t)ht * d; p.sD = (int64_t)cn * d;
+      if ((rc = gemm(p)) != TTT_OK) return rc;
+    }
+    // dW2t[o][i] = sum_t dm[t][o] g[t][i]  -> W2t32 += -eta * dW2t ; shadow refreshed
+    p = gp(d, ht, cn, GT, d, true, A.g, ht, true, Lw.W2t32, ht, true, EPI_SGD);
+    p.batch = B; p.sA = (int64_t)cn * d; p.sB = (int64_t)cn * ht; p.sD = (int64_t)d * ht;
+    p.alpha = -cfg.eta;
+    if (is_bf16) { p.Y = Lw.W2t; p.ldy = ht; p.sY = (int64_t)d * ht; }
+    if ((rc = gemm(p)) != TTT_OK) return rc;
+    // dW1t[o][i] = sum_t du[t][o] r2[t][i]
+    p = gp(ht, d, cn, dhid, ht, true, A.r2, d, true, Lw.W1t32, d, true, EPI_SGD);
+    p.batch = B; p.sA = (int64_t)cn * ht; p.sB = (int64_t)cn * d; p.sD = (int64_t)ht * d;
+    p.alpha = -cfg.eta;
+    if (is_bf16) { p.Y = Lw.W1t; p.ldy = d; p.sY = (int64_t)ht * d; }
+    if ((rc = gemm(p)) != TTT_OK) return rc;
+    if (j == 0) break;  // upstream of the first adaptive MLP does not depend on the fast weights
+    rmsnorm_bwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(A.a, Lw.g_ttt, A.rstd2, dr, G, rows, d, G, GT);
+    TTT_LAUNCHED();
+    // frozen attention: data gradients only; cached K/V are constants
+    if ((rc = gemm(gp(rows, d, d, GT, d, false, Lw.Wo, d, true, dob, d, false, EPI_STORE))) != TTT_OK) return rc;
+    AttnParams ap;
+    memset(&ap, 0, sizeof(ap));
+    ap.B = B; ap.H = H; ap.hd = hd; ap.n = cn; ap.d = d; ap.q0 = 0; ap.window = kwin;
+    ap.Q = A.qkv; ap.ldq = 3 * d; ap.K = A.qkv + d; ap.V = A.qkv + 2 * d; ap.ldkv = 3 * d;
+    ap.Kc = Lw.ring_k; ap.Vc = Lw.ring_v; ap.C = C;
+    ap.O = A.o; ap.ldo = d; ap.lse = A.lse; ap.scale = 1.0f / sqrtf((float)hd);
+    ap.dO = dob; ap.lddo = d; ap.Dsum = Dsum;
+    ap.dQ = dqkv; ap.dK = dqkv + d; ap.dV = dqkv + 2 * d; ap.lddq = 3 * d;
+    ap.q0 = chunk_pos;
+    attn_bwd_prep_kernel<T><<<nblk((int64_t)rows * H, 8), 256, 0, st>>>(ap);
+    TTT_LAUNCHED();
+    attn_bwd_dq_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
+    TTT_LAUNCHED();
+    attn_bwd_dkv_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
+    TTT_LAUNCHED();
+    rope_kernel<T><<<nblk((int64_t)rows * d, 256), 256, 0, st>>>(dqkv, 3 * d, 2 * d, rows, cn, chunk_pos, hd,
+                                                                  rope_lo, rope_hi, 1);
+    TTT_LAUNCHED();
+    if ((rc = gemm(gp(rows, d, 3 * d, dqkv, 3 * d, false, Lw.Wqkv, d, true, dr, d, true, EPI_STORE))) != TTT_OK)
+      return rc;
+    // G <- G + RMSNorm_bwd through the attention norm: gradient w.r.t. this block's input
+    rmsnorm_bwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(A.x, Lw.g_attn, A.rstd1, dr, G, rows, d, G, GT);
+    TTT_LAUNCHED();
+  }
+  return TTT_OK;
+}
+
+}  // namespace ttt
+
+namespace ttt {
+
+// One adaptive step over cn positions per sequence (rows [B][cn], pos..pos+cn-1):
+// forward with W_{i-1}, losses recorded, and (grad) backward + in-place SGD.
+template <typename T>
+int Engine<T>::ttt_step(const float* in, const int32_t* targets, int cn, int64_t pos, float* loss_out,
+                        int64_t loss_ld, int64_t loss_off, bool grad, bool commit) {
+  const int rows = B * cn;
+  int rc;
+  chunk_pos = pos;
+  if (in != blk[0].x) {
+    TTT_CUDA(cudaMemcpyAsync(blk[0].x, in, (size_t)rows * d * 4, cudaMemcpyDeviceToDevice, st));
+  }
+  if (targets != tgt) {
+    TTT_CUDA(cudaMemcpyAsync(tgt, targets, (size_t)rows * 4, cudaMemcpyDeviceToDevice, st));
+  }
+  if ((rc = ttt_forward(cn, pos, commit)) != TTT_OK) return rc;
+  rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf);
+  TTT_LAUNCHED();
+  if ((rc = gemm(gp(rows, V, d, rf, d, false, E, d, false, z, V, false, EPI_STORE))) != TTT_OK) return rc;
+  // mean over the b positions of the chunk (summary: mini-batch GD with 1/b)
+  ce_kernel<T><<<rows, 256, 0, st>>>(z, V, tgt, cn, loss_out, loss_ld, loss_off, grad ? 1.0f / bsz : 0.f,
+                                     dev_err);
+  TTT_LAUNCHED();
+  if (grad) {
+    if ((rc = ttt_backward(cn)) != TTT_OK) return rc;
+  }
+  return TTT_OK;
+}
+
+// ------------------------------------------------------------------ prefill (Algorithm 1)
+template <typename T> int Engine<T>::prefill(const int32_t* tokens, int64_t T_, float* out, int32_t kind) {
+  if (poisoned) return fail(this, TTT_ERR_POISONED, "handle poisoned by an earlier device error");
+  if (!tokens || !out || T_ <= 0) return fail(this, TTT_ERR_INVALID_ARG, "prefill: null buffer or T <= 0");
+  if (pend_cnt != 0) return fail(this, TTT_ERR_STREAM, "prefill: a partial chunk is pending; decode completes it");
+  if ((n_pos + T_) / 1024 >= kRopeHi) return fail(this, TTT_ERR_INVALID_ARG, "prefill: position limit exceeded");
+  launches = 0;
+  const int64_t ld = T_ + 1;
+  int rc;
+  if ((rc = ensure((void**)&tok_dev, &tok_cap, (int64_t)B * ld, 4)) != TTT_OK) return rc;
+  if ((rc = ensure((void**)&loss_dev, &loss_cap, (int64_t)B * T_, 4)) != TTT_OK) return rc;
+  std::vector<int32_t> first(B), last(B);
+  if (kind == TTT_PTR_HOST) {
+    for (int b = 0; b < B; ++b) { first[b] = tokens[b * ld]; last[b] = tokens[b * ld + T_]; }
+    TTT_CUDA(cudaMemcpyAsync(tok_dev, tokens, (size_t)B * ld * 4, cudaMemcpyHostToDevice, st));
+  } else {
+    TTT_CUDA(cudaMemcpyAsync(tok_dev, tokens, (size_t)B * ld * 4, cudaMemcpyDeviceToDevice, st));
+    for (int b = 0; b < B; ++b) {
+      TTT_CUDA(cudaMemcpyAsync(&first[b], tok_dev + b * ld, 4, cudaMemcpyDeviceToHost, st));
+      TTT_CUDA(cudaMemcpyAsync(&last[b], tok_dev + b * ld + T_, 4, cudaMemcpyDeviceToHost, st));
+    }
+    TTT_CUDA(cudaStreamSynchronize(st));
+  }
+  if (n_pos > 0)
+    for (int b = 0; b < B; ++b)
+      if (first[b] != pend_tok_host[b]) return fail(this, TTT_ERR_STREAM, "prefill: first id is not the pending token");
+  float* lout = kind == TTT_PTR_DEVICE ? out : loss_dev;
+  for (int64_t s0 = 0; s0 < T_; s0 += S) {
+    const int n = (int)((T_ - s0) < S ? (T_ - s0) : S);
+    const int64_t P0 = n_pos + s0;
+    const int rows = B * n;
+    embed_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(tok_dev, ld, (int)s0, n, rows, E, V, d, xs, dev_err);
+    TTT_LAUNCHED();
+    for (int l = 0; l < first_ttt; ++l) {
+      if ((rc = attention_block(layers[l], l, xs, xs, rs, nullptr, qkvs, os, nullptr, n, P0, true)) != TTT_OK)
+        return rc;
+      if ((rc = frozen_mlp(layers[l], xs, rs, hids, rows)) != TTT_OK) return rc;
+    }
+    for (int c0 = 0; c0 < n; c0 += bsz) {
+      const int cn = (n - c0) < bsz ? (n - c0) : bsz;
+      gather_rows_kernel<<<nblk((int64_t)B * cn * d, 256), 256, 0, st>>>(xs, (int64_t)n * d, c0, cn, B, d, blk[0].x,
+                                                                        (int64_t)cn * d, 0);
+      TTT_LAUNCHED();
+      gather_tokens_kernel<<<nblk(B * cn, 256), 256, 0, st>>>(tok_dev, ld, s0 + c0 + 1, cn, B, tgt, cn, 0);
+      TTT_LAUNCHED();
+      const bool full = cn == bsz;
+      if ((rc = ttt_step(blk[0].x, tgt, cn, P0 + c0, lout, T_, s0 + c0, full, true)) != TTT_OK) return rc;
+      if (!full) {  // trailing partial chunk: keep its inputs and targets pending
+        TTT_CUDA(cudaMemcpy2DAsync(pend_in, (size_t)bsz * d * 4, blk[0].x, (size_t)cn * d * 4, (size_t)cn * d * 4, B,
+                                   cudaMemcpyDeviceToDevice, st));
+        TTT_CUDA(cudaMemcpy2DAsync(pend_tgt, (size_t)bsz * 4, tgt, (size_t)cn * 4, (size_t)cn * 4, B,
+                                   cudaMemcpyDeviceToDevice, st));
+        pend_cnt = cn;
+      }
+    }
+  }
+  gather_tokens_kernel<<<nblk(B, 256), 256, 0, st>>>(tok_dev, ld, T_, 1, B, pend_tok_dev, 1, 0);
+  TTT_LAUNCHED();
+  if (kind == TTT_PTR_HOST) {
+    TTT_CUDA(cudaMemcpyAsync(out, loss_dev, (size_t)B * T_ * 4, cudaMemcpyDeviceToHost, st));
+  }
+  if ((rc = sync_and_check()) != TTT_OK) return rc;
+  n_pos += T_;
+  pend_tok_host = last;
+  return TTT_OK;
+}
+
+// ------------------------------------------------------------------ decode (Algorithm 3)
+__global__ void decode_record_kernel(const int32_t* chosen, const float* loss, int B, int64_t t, int64_t n,
+                                     int32_t* out_tok, float* out_loss, int32_t* pend_tgt, int bsz, int cnt) {
+  const int b = threadIdx.x;
+  if (b >= B) return;
+  out_tok[b * n + t] = chosen[b];
+  if (out_loss) out_loss[b * n + t] = loss[b];
+  pend_tgt[b * bsz + cnt] = chosen[b];
+}
+
+template <typename T>
+int Engine<T>::decode(int64_t n, const int32_t* forced, int32_t* out_tok, float* out_loss, int32_t kind) {
+  if (poisoned) return fail(this, TTT_ERR_POISONED, "handle poisoned by an earlier device error");
+  if (n <= 0 || !out_tok) return fail(this, TTT_ERR_INVALID_ARG, "decode: n <= 0 or null output");
+  if (n_pos == 0) return fail(this, TTT_ERR_STREAM, "decode: nothing prefilled (no pending token)");
+  if ((n_pos + n) / 1024 >= kRopeHi) return fail(this, TTT_ERR_INVALID_ARG, "decode: position limit exceeded");
+  launches = 0;
+  int rc;
+  int32_t* otok = out_tok;
+  float* oloss = out_loss;
+  int32_t* fdev = nullptr;
+  if ((rc = ensure((void**)&otok_dev, &otok_cap, (int64_t)B * n * 2, 4)) != TTT_OK) return rc;
+  if ((rc = ensure((void**)&loss_dev, &loss_cap, (int64_t)B * n, 4)) != TTT_OK) return rc;
+  if (kind == TTT_PTR_HOST) {
+    otok = otok_dev;
+    oloss = out_loss ? loss_dev : nullptr;
+    if (forced) {
+      fdev = otok_dev + (int64_t)B * n;
+      TTT_CUDA(cudaMemcpyAsync(fdev, forced, (size_t)B * n * 4, cudaMemcpyHostToDevice, st));
+    }
+  } else {
+    fdev = (int32_t*)forced;
+  }
+  const int rows = B;
+  for (int64_t t = 0; t < n; ++t) {
+    const int64_t p = n_pos;
+    embed_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(pend_tok_dev, 1, 0, 1, rows, E, V, d, xs, dev_err);
+    TTT_LAUNCHED();
+    for (int l = 0; l < first_ttt; ++l) {
+      if ((rc = attention_block(layers[l], l, xs, xs, rs, nullptr, qkvs, os, nullptr, 1, p, true)) != TTT_OK)
+        return rc;
+      if ((rc = frozen_mlp(layers[l], xs, rs, hids, rows)) != TTT_OK) return rc;
+    }
+    // keep the first adaptive block's input of this position for the chunk's update
+    gather_rows_kernel<<<nblk((int64_t)B * d, 256), 256, 0, st>>>(xs, d, 0, 1, B, d, pend_in, (int64_t)bsz * d,
+                                                                 pend_cnt);
+    TTT_LAUNCHED();
+    TTT_CUDA(cudaMemcpyAsync(blk[0].x, xs, (size_t)B * d * 4, cudaMemcpyDeviceToDevice, st));
+    chunk_pos = p;
+    if ((rc = ttt_forward(1, p, true)) != TTT_OK) return rc;
+    rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf);
+    TTT_LAUNCHED();
+    if ((rc = gemm(gp(rows, V, d, rf, d, false, E, d, false, z, V, false, EPI_STORE))) != TTT_OK) return rc;
+    const int32_t* fcol = nullptr;
+    if (fdev) {
+      gather_tokens_kernel<<<1, 256, 0, st>>>(fdev, n, t, 1, B, forced_col, 1, 0);
+      TTT_LAUNCHED();
+      fcol = forced_col;
+    }
+    argmax_kernel<T><<<rows, 256, 0, st>>>(z, V, fcol, pend_tok_dev, dec_loss, dec_zmax);
+    TTT_LAUNCHED();
+    decode_record_kernel<<<1, 32 * ((B + 31) / 32), 0, st>>>(pend_tok_dev, dec_loss, B, t, n, otok, oloss, pend_tgt,
+                                                             bsz, pend_cnt);
+    TTT_LAUNCHED();
+    ++pend_cnt;
+    ++n_pos;
+    if (pend_cnt == bsz) {  // a full chunk of decoded positions: differentiate and update
+      if ((rc = ttt_step(pend_in, pend_tgt, bsz, n_pos - bsz, nullptr, 0, 0, true, false)) != TTT_OK) return rc;
+      pend_cnt = 0;
+    }
+  }
+  if (kind == TTT_PTR_HOST) {
+    TTT_CUDA(cudaMemcpyAsync(out_tok, otok_dev, (size_t)B * n * 4, cudaMemcpyDeviceToHost, st));
+    if (out_loss) TTT_CUDA(cudaMemcpyAsync(out_loss, loss_dev, (size_t)B * n * 4, cudaMemcpyDeviceToHost, st));
+  }
+  TTT_CUDA(cudaMemcpyAsync(pend_tok_host.data(), pend_tok_dev, (size_t)B * 4, cudaMemcpyDeviceToHost, st));
+  return sync_and_check();
+}
+
+template <typename T> int Engine<T>::get_weights(int32_t seq, int32_t j, float* w1, float* w2, int32_t kind) {
+  if (poisoned) return fail(this, TTT_ERR_POISONED, "handle poisoned by an earlier device error");
+  if (seq < 0 || seq >= B || j < 0 || j >= Lt) return fail(this, TTT_ERR_INVALID_ARG, "get_weights: bad index");
+  const LayerDev<T>& Lw = layers[first_ttt + j];
+  const int64_t n1 = (int64_t)ht * d;
+  const cudaMemcpyKind k = kind == TTT_PTR_HOST ? cudaMemcpyDeviceToHost : cudaMemcpyDeviceToDevice;
+  if (w1) TTT_CUDA(cudaMemcpyAsync(w1, Lw.W1t32 + seq * n1, n1 * 4, k, st));
+  if (w2) TTT_CUDA(cudaMemcpyAsync(w2, Lw.W2t32 + seq * n1, n1 * 4, k, st));
+  return sync_and_check();
+}
+
+static int validate(const ttt_config* c, std::string* why) {
+  auto bad = [&](const char* m) { *why = m; return TTT_ERR_INVALID_ARG; };
+  if (!c) return bad("null config");
+  if (c->vocab <= 0 || c->d <= 0 || c->n_layers <= 0 || c->n_heads <= 0 || c->batch <= 0) return bad("non-positive size");
+  if (c->n_ttt < 1 || c->n_ttt > c->n_layers) return bad("n_ttt must be in [1, n_layers]");
+  if (c->d % c->n_heads) return bad("d must be a multiple of n_heads");
+  const int hd = c->d / c->n_heads;
+  if (hd % 2 || hd > 128) return bad("head dim must be even and <= 128");
+  if (c->minibatch_b <= 0 || c->window_k < c->minibatch_b) return bad("need window_k >= minibatch_b > 0");
+  if (c->d % 8 || c->mlp_hidden % 8 || c->ttt_hidden % 8 || c->static_hidden % 8 || c->vocab % 8)
+    return bad("widths and vocab must be multiples of 8");
+  if (c->mlp_hidden <= 0 || c->ttt_hidden <= 0 || c->static_hidden <= 0) return bad("non-positive hidden width");
+  if (c->dtype != TTT_FP32 && c->dtype != TTT_BF16) return bad("dtype must be TTT_FP32 or TTT_BF16");
+  if (!(c->rms_eps > 0.f) || !(c->rope_base > 1.f) || !std::isfinite(c->eta)) return bad("bad eps, rope base or eta");
+  return TTT_OK;
+}
+
+}  // namespace ttt
+
+// ============================================================== C ABI
+using namespace ttt;
+
+extern "C" {
+
+int32_t ttt_num_weight_tensors(const ttt_config* c) {
+  if (!c) return -1;
+  return 2 + (c->n_layers - c->n_ttt) * 8 + c->n_ttt * 11;
+}
+
+int ttt_create(const ttt_config* cfg, const ttt_weights* w, ttt_handle** out) {
+  if (!out) return TTT_ERR_INVALID_ARG;
+  *out = nullptr;
+  std::string why;
+  if (validate(cfg, &why) != TTT_OK) return TTT_ERR_INVALID_ARG;
+  if (!w || !w->tensors || w->n_tensors != ttt_num_weight_tensors(cfg)) return TTT_ERR_INVALID_ARG;
+  ttt_handle* h = nullptr;
+  int rc;
+  try {
+    if (cfg->dtype == TTT_BF16) {
+      auto* e = new Engine<bf16>();
+      h = e;
+      rc = e->create(cfg, w);
+    } else {
+      auto* e = new Engine<float>();
+      h = e;
+      rc = e->create(cfg, w);
+    }
+  } catch (...) {
+    delete h;
+    return TTT_ERR_OOM;
+  }
+  if (rc != TTT_OK) {
+    delete h;
+    return rc;
+  }
+  *out = h;
+  return TTT_OK;
+}
+
+int ttt_prefill(ttt_handle* h, const int32_t* tokens, int64_t T, float* out_losses, int32_t ptr_kind) {
+  if (!h) return TTT_ERR_INVALID_ARG;
+  try { return h->prefill(tokens, T, out_losses, ptr_kind); } catch (...) { return TTT_ERR_OOM; }
+}
+
+int ttt_decode(ttt_handle* h, int64_t n, const int32_t* forced, int32_t* out_tokens, float* out_losses,
+               int32_t ptr_kind) {
+  if (!h) return TTT_ERR_INVALID_ARG;
+  try { return h->decode(n, forced, out_tokens, out_losses, ptr_kind); } catch (...) { return TTT_ERR_OOM; }
+}
+
+int ttt_get_weights(ttt_handle* h, int32_t seq, int32_t ttt_block, float* w1, float* w2, int32_t ptr_kind) {
+  if (!h) return TTT_ERR_INVALID_ARG;
+  return h->get_weights(seq, ttt_block, w1, w2, ptr_kind);
+}
+
+int ttt_reset(ttt_handle* h) {
+  if (!h) return TTT_ERR_INVALID_ARG;
+  return h->reset();
+}
+
+int64_t ttt_position(const ttt_handle* h) { return h ? h->n_pos : -1; }
+int64_t ttt_device_bytes(const ttt_handle* h) { return h ? h->dev_bytes : -1; }
+int64_t ttt_last_launch_count(const ttt_handle* h) { return h ? h->launches : -1; }
+
+void ttt_destroy(ttt_handle* h) { delete h; }
+
+const char* ttt_last_error(const ttt_handle* h) { return h ? h->err_msg.c_str() : "null handle"; }
+
+const char* ttt_version(void) { return "ttt-e2e-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,162 @@
+"""Kernel-level checks through the per-kernel C ABI (include/ttt_kernels.h) on a GPU.
+
+Each kernel is compared with a float64 PyTorch computation of the same
+operation on the same (bf16- or fp32-valued) inputs.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def T():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import long_context_prefill_ttt_b200 as T
+    return T
+
+
+def _rand(shape, dtype, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g, dtype=torch.float32) * scale).to(dtype).cuda()
+
+
+def _store(x_log, mn):
+    """x_log [batch][rows][K] -> storage [batch][K][rows] when MN-major."""
+    return x_log.transpose(1, 2).contiguous() if mn else x_log.contiguous()
+
+
+SHAPES = [(256, 256, 128, 1), (200, 384, 192, 2), (1024, 512, 64, 1), (128, 2048, 256, 1), (384, 128, 1024, 3)]
+
+
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 1)])
+@pytest.mark.parametrize("M,N,K,batch", SHAPES)
+@pytest.mark.parametrize("engine", [0, 1])
+def test_gemm_store_f32(T, a_mn, b_mn, M, N, K, batch, engine):
+    A = _rand((batch, M, K), torch.bfloat16, 1)
+    B = _rand((batch, N, K), torch.bfloat16, 2)
+    ref = A.double() @ B.double().transpose(1, 2)
+    D = torch.full((batch, M, N), float("nan"), dtype=torch.float32, device="cuda")
+    T.ttt_k_gemm(_store(A, a_mn), _store(B, b_mn), D, M, N, K, batch=batch, sA=M * K, a_mn=a_mn, sB=N * K,
+                 b_mn=b_mn, sD=M * N, engine=engine)
+    T.ttt_k_status()
+    err = (D.double() - ref).abs().max().item() / ref.abs().max().item()
+    assert err < 2e-6, err
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 512, 256), (130, 256, 64)])
+def test_gemm_store_bf16_and_fp32_simt(T, M, N, K):
+    A = _rand((1, M, K), torch.bfloat16, 3)
+    B = _rand((1, N, K), torch.bfloat16, 4)
+    ref = A.double() @ B.double().transpose(1, 2)
+    D = torch.empty((1, M, N), dtype=torch.bfloat16, device="cuda")
+    T.ttt_k_gemm(A, B, D, M, N, K)
+    T.ttt_k_status()
+    assert torch.allclose(D.double(), ref, rtol=1e-2, atol=1e-2 * ref.abs().max().item())
+    # fp32 operands (SIMT engine) against float64
+    A32, B32 = A.float(), B.float() + 1e-3
+    D32 = torch.empty((1, M, N), dtype=torch.float32, device="cuda")
+    T.ttt_k_gemm(A32, B32, D32, M, N, K)
+    T.ttt_k_status()
+    ref32 = A32.double() @ B32.double().transpose(1, 2)
+    assert ((D32.double() - ref32).abs().max() / ref32.abs().max()).item() < 1e-6
+
+
+@pytest.mark.parametrize("engine", [0, 1])
+def test_gemm_epilogues(T, engine):
+    M, N, K = 256, 384, 128
+    A = _rand((1, M, K), torch.bfloat16, 5, 0.5)
+    B = _rand((1, N, K), torch.bfloat16, 6, 0.5)
+    acc = (A.double() @ B.double().transpose(1, 2))[0]
+    # residual, in place
+    R = _rand((M, N), torch.float32, 7)
+    D = R.clone()
+    T.ttt_k_gemm(A, B, D, M, N, K, X=D, ldx=N, epi=T.EPI_RESID, engine=engine)
+    T.ttt_k_status()
+    assert (D.double() - (acc + R.double())).abs().max().item() < 1e-4
+    # gelu pair
+    U = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    G = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    T.ttt_k_gemm(A, B, G, M, N, K, Y=U, ldy=N, epi=T.EPI_GELU, engine=engine)
+    T.ttt_k_status()
+    gelu = torch.nn.functional.gelu(acc, approximate="none")
+    assert torch.allclose(U.double(), acc, rtol=1e-2, atol=1e-2)
+    assert torch.allclose(G.double(), gelu, rtol=1e-2, atol=1e-2)
+    # gelu' gate
+    Xu = _rand((M, N), torch.bfloat16, 8)
+    Dg = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    T.ttt_k_gemm(A, B, Dg, M, N, K, X=Xu, ldx=N, epi=T.EPI_DGELU, engine=engine)
+    T.ttt_k_status()
+    x = Xu.double()
+    gp = 0.5 * (1 + torch.erf(x / math.sqrt(2))) + x * torch.exp(-0.5 * x * x) / math.sqrt(2 * math.pi)
+    assert torch.allclose(Dg.double(), acc * gp, rtol=2e-2, atol=2e-2)
+    # fused SGD: W += alpha * acc, shadow refreshed
+    W = _rand((M, N), torch.float32, 9)
+    W0 = W.double().clone()
+    Sh = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    T.ttt_k_gemm(A, B, W, M, N, K, Y=Sh, ldy=N, alpha=-0.05, epi=T.EPI_SGD, engine=engine)
+    T.ttt_k_status()
+    assert (W.double() - (W0 - 0.05 * acc)).abs().max().item() < 1e-5
+    assert torch.equal(Sh, W.to(torch.bfloat16))
+
+
+def _attn_reference(qkv, ring_k, ring_v, B, H, hd, n, q0, window, C):
+    """float64 keys/values at absolute positions, explicit window mask."""
+    d = H * hd
+    q = qkv[..., :d].double().view(B, n, H, hd)
+    kc = qkv[..., d:2 * d].double().view(B, n, H, hd)
+    vc = qkv[..., 2 * d:].double().view(B, n, H, hd)
+    lo = max(0, q0 - window + 1)
+    pos = torch.arange(lo, q0 + n)
+    ks, vs = [], []
+    for p in pos.tolist():
+        if p >= q0:
+            ks.append(kc[:, p - q0]); vs.append(vc[:, p - q0])
+        else:
+            ks.append(ring_k.double().view(B, C, H, hd)[:, p % C]); vs.append(ring_v.double().view(B, C, H, hd)[:, p % C])
+    K = torch.stack(ks, 1)
+    V = torch.stack(vs, 1)
+    qp = torch.arange(q0, q0 + n)[:, None]
+    mask = (pos[None, :] <= qp) & (pos[None, :] >= qp - window + 1)
+    return q, kc, vc, K, V, mask.cuda(), lo
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("B,H,hd,n,q0,window,C", [(2, 2, 64, 96, 160, 128, 256), (1, 4, 16, 48, 0, 16, 32),
+                                                  (1, 2, 128, 64, 300, 200, 384), (3, 1, 64, 1, 777, 64, 128)])
+def test_attention_forward_and_backward(T, dtype, B, H, hd, n, q0, window, C):
+    d = H * hd
+    qkv = _rand((B * n, 3 * d), dtype, 11)
+    ring_k = _rand((B, C, d), dtype, 12)
+    ring_v = _rand((B, C, d), dtype, 13)
+    out = torch.empty((B * n, d), dtype=dtype, device="cuda")
+    lse = torch.empty((B, H, n), dtype=torch.float32, device="cuda")
+    T.ttt_k_attention_fwd(qkv, out, lse, B, H, hd, n, q0, window, ring_k, ring_v, C)
+    T.ttt_k_status()
+    q, kc, vc, K, V, mask, lo = _attn_reference(qkv, ring_k, ring_v, B, H, hd, n, q0, window, C)
+    q.requires_grad_(True); kc.requires_grad_(True); vc.requires_grad_(True)
+    # rebuild keys so autograd sees the current part
+    ncached = q0 - lo
+    Kf = torch.cat([K[:, :ncached], kc], 1)
+    Vf = torch.cat([V[:, :ncached], vc], 1)
+    s = torch.einsum("bqhd,bkhd->bhqk", q, Kf) / math.sqrt(hd)
+    s = s.masked_fill(~mask, float("-inf"))
+    ref_lse = torch.logsumexp(s, -1)
+    o = torch.einsum("bhqk,bkhd->bqhd", torch.softmax(s, -1), Vf)
+    tol = 1e-5 if dtype == torch.float32 else 2e-2
+    assert (out.double().view(B, n, H, hd) - o).abs().max().item() < tol
+    assert (lse.double() - ref_lse).abs().max().item() < tol
+    dout = _rand((B * n, d), dtype, 14)
+    o.backward(dout.double().view(B, n, H, hd))
+    dqkv = torch.zeros((B * n, 3 * d), dtype=dtype, device="cuda")
+    dsum = torch.empty((B, H, n), dtype=torch.float32, device="cuda")
+    T.ttt_k_attention_bwd(qkv, out, lse, dout, dqkv, dsum, B, H, hd, n, q0, window, ring_k, ring_v, C)
+    T.ttt_k_status()
+    for got, ref in ((dqkv[:, :d], q.grad), (dqkv[:, d:2 * d], kc.grad), (dqkv[:, 2 * d:], vc.grad)):
+        scale = ref.abs().max().item() + 1e-12
+        err = (got.double().view(B, n, H, hd) - ref).abs().max().item() / scale
+        assert err < (1e-5 if dtype == torch.float32 else 3e-2), err
