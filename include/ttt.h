@@ -135,6 +135,19 @@ int64_t ttt_device_bytes(const ttt_handle* h);
 /* Kernel launches issued by the most recent prefill or decode call. */
 int64_t ttt_last_launch_count(const ttt_handle* h);
 
+/* Kernel-class timing. When enabled, CUDA events are recorded on the handle's
+ * stream around every launch of these classes, and the algorithmic work of each
+ * launch is counted: 0 frozen-phase GEMMs, 1 adaptive-phase GEMMs, 2 attention
+ * forward, 3 attention backward. FLOPs: 2*M*N*K per GEMM; attention 4*hd*H per
+ * query-key pair of the window forward (review eq. (1) counts the pairs), and
+ * 2*hd*H*(2 window pairs + 2 current-chunk pairs) backward (no recompute counted). Bytes: operands read
+ * once plus the output written once. ttt_profile(h, 1) clears the counters.
+ * ttt_profile_read fills up to n_classes entries (any pointer may be NULL) and
+ * returns the number of classes. Accumulates over calls until cleared. */
+int ttt_profile(ttt_handle* h, int32_t enable);
+int ttt_profile_read(const ttt_handle* h, int32_t n_classes, double* ms, int64_t* launches, double* flops,
+                     double* bytes);
+
 void ttt_destroy(ttt_handle* h);
 
 const char* ttt_last_error(const ttt_handle* h);

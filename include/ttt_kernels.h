@@ -27,17 +27,23 @@ extern "C" {
  *                  summary of the TTT-E2E paper, mini-batch gradient-descent equation) */
 enum { TTT_EPI_STORE = 0, TTT_EPI_RESID = 1, TTT_EPI_GELU = 2, TTT_EPI_DGELU = 3, TTT_EPI_SGD = 4 };
 
-/* Engines: 0 = automatic (tcgen05 tensor cores for bf16 shapes with N % 128 == 0 and K % 64 == 0,
- * else SIMT), 1 = SIMT fp32-FFMA only. */
+/* Engines: 0 = automatic: GEMMs on tcgen05 tensor cores for bf16 shapes with N % 128 == 0 and
+ * K % 64 == 0; attention on tensor cores (mma.sync m16n8k16) for bf16 with head dim 64 or 128 and
+ * q0 % 64 == 0 (and C % 64 == 0); otherwise, and for fp32, SIMT FFMA kernels.
+ * 1 = SIMT only. */
 enum { TTT_ENGINE_AUTO = 0, TTT_ENGINE_SIMT = 1 };
 
-/* Batched GEMM D[z][m][n] = epilogue(alpha * sum_k A[z](m,k) * B[z](n,k)).
+/* Batched GEMM D[z][m][n] = epilogue(alpha * sum_k A[z](m,k) * (B[z](n,k) + B2[z](n,k))).
  * A(m,k) = a_mn ? A[k*lda + m] : A[m*lda + k]   (batch stride sA elements)
- * B(n,k) = b_mn ? B[k*ldb + n] : B[n*ldb + k]   (batch stride sB)
+ * B(n,k) = b_mn ? B[k*ldb + n] : B[n*ldb + k]   (batch stride sB; 0 = one matrix shared by all z)
+ * B2: optional (NULL), same layout and ldb as B, batch stride sB2. The adaptive MLPs use
+ *     B = W_init (shared) and B2 = dW (per sequence): the fast weights W_init + dW without
+ *     rounding a small dW against W_init into one bf16 value.
  * D, X, Y row-major with leading dims ldd, ldx, ldy and batch strides sD, sX, sY.
  * Forward products use (a_mn, b_mn) = (0, 0), data gradients (0, 1), weight gradients (1, 1). */
 int ttt_k_gemm(int32_t elem_dtype, int32_t M, int32_t N, int32_t K, int32_t batch, const void* A, int64_t lda,
-               int64_t sA, int32_t a_mn, const void* B, int64_t ldb, int64_t sB, int32_t b_mn, void* D, int64_t ldd,
+               int64_t sA, int32_t a_mn, const void* B, int64_t ldb, int64_t sB, int32_t b_mn, const void* B2,
+               int64_t sB2, void* D, int64_t ldd,
                int64_t sD, int32_t d_f32, const void* X, int64_t ldx, int64_t sX, void* Y, int64_t ldy, int64_t sY,
                float alpha, int32_t epi, int32_t engine, void* stream);
 

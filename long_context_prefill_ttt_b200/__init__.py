@@ -66,10 +66,12 @@ def _load():
         "ttt_device_bytes": (I64, [VP]),
         "ttt_last_launch_count": (I64, [VP]),
         "ttt_destroy": (None, [VP]),
+        "ttt_profile": (ctypes.c_int, [VP, I32]),
+        "ttt_profile_read": (ctypes.c_int, [VP, I32, VP, VP, VP, VP]),
         "ttt_last_error": (ctypes.c_char_p, [VP]),
         "ttt_version": (ctypes.c_char_p, []),
-        "ttt_k_gemm": (ctypes.c_int, [I32, I32, I32, I32, I32, VP, I64, I64, I32, VP, I64, I64, I32, VP, I64, I64,
-                                      I32, VP, I64, I64, VP, I64, I64, F, I32, I32, VP]),
+        "ttt_k_gemm": (ctypes.c_int, [I32, I32, I32, I32, I32, VP, I64, I64, I32, VP, I64, I64, I32, VP, I64, VP,
+                                      I64, I64, I32, VP, I64, I64, VP, I64, I64, F, I32, I32, VP]),
         "ttt_k_attention_fwd": (ctypes.c_int, [I32, I32, I32, I32, I32, I64, I32, VP, VP, VP, I32, VP, VP, I32, VP]),
         "ttt_k_attention_bwd": (ctypes.c_int, [I32, I32, I32, I32, I32, I64, I32, VP, VP, VP, I32, VP, VP, VP, VP,
                                                VP, I32, VP]),
@@ -274,6 +276,24 @@ def ttt_last_launch_count(h: Handle) -> int:
     return int(lib.ttt_last_launch_count(h.ptr))
 
 
+PROFILE_CLASSES = ("gemm_frozen", "gemm_adaptive", "attention_fwd", "attention_bwd")
+
+
+def ttt_profile(h: Handle, enable: bool = True):
+    h.check(lib.ttt_profile(h.ptr, int(enable)))
+
+
+def ttt_profile_read(h: Handle):
+    """{class: dict(ms, launches, flops, bytes)} accumulated since ttt_profile(h, True)."""
+    n = len(PROFILE_CLASSES)
+    ms = (ctypes.c_double * n)()
+    la = (ctypes.c_int64 * n)()
+    fl = (ctypes.c_double * n)()
+    by = (ctypes.c_double * n)()
+    lib.ttt_profile_read(h.ptr, n, ms, la, fl, by)
+    return {c: dict(ms=ms[i], launches=la[i], flops=fl[i], bytes=by[i]) for i, c in enumerate(PROFILE_CLASSES)}
+
+
 def ttt_version() -> str:
     return lib.ttt_version().decode()
 
@@ -285,16 +305,17 @@ def _dtype_code(t):
     return TTT_BF16 if t.dtype == torch.bfloat16 else TTT_FP32
 
 
-def ttt_k_gemm(A, B, D, M, N, K, *, batch=1, lda=None, sA=0, a_mn=False, ldb=None, sB=0, b_mn=False, ldd=None,
-               sD=0, X=None, ldx=0, sX=0, Y=None, ldy=0, sY=0, alpha=1.0, epi=EPI_STORE, engine=ENGINE_AUTO,
-               stream=None):
+def ttt_k_gemm(A, B, D, M, N, K, *, batch=1, lda=None, sA=0, a_mn=False, ldb=None, sB=0, b_mn=False, B2=None,
+               sB2=0, ldd=None, sD=0, X=None, ldx=0, sX=0, Y=None, ldy=0, sY=0, alpha=1.0, epi=EPI_STORE,
+               engine=ENGINE_AUTO, stream=None):
     """Enqueue one contraction on device tensors (see include/ttt_kernels.h)."""
     torch = _torch()
     lda = lda if lda is not None else (M if a_mn else K)
     ldb = ldb if ldb is not None else (N if b_mn else K)
     ldd = ldd if ldd is not None else N
     rc = lib.ttt_k_gemm(_dtype_code(A), M, N, K, batch, A.data_ptr(), lda, sA, int(a_mn), B.data_ptr(), ldb, sB,
-                        int(b_mn), D.data_ptr(), ldd, sD, int(D.dtype == torch.float32),
+                        int(b_mn), B2.data_ptr() if B2 is not None else None, sB2, D.data_ptr(), ldd, sD,
+                        int(D.dtype == torch.float32),
                         X.data_ptr() if X is not None else None, ldx, sX,
                         Y.data_ptr() if Y is not None else None, ldy, sY, float(alpha), epi, engine,
                         _stream_ptr(stream))

@@ -31,6 +31,11 @@ struct GemmParams {
   int M, N, K, batch;
   const void* A; int64_t lda, sA; int a_mn;
   const void* B; int64_t ldb, sB; int b_mn;
+  // Optional second B of the same shape and layout, accumulated over the same A:
+  // acc = sum_k A(m,k) (B(n,k) + B2(n,k)). Used for fast weights held as
+  // W_init (shared, sB = 0) + dW (per sequence), so that a bf16 copy of the
+  // small update dW is not rounded away against W_init.
+  const void* B2; int64_t sB2;
   void* D; int64_t ldd, sD; int d_f32;
   const void* X; int64_t ldx, sX;
   void* Y; int64_t ldy, sY;
@@ -83,6 +88,9 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmParams p) {
   const T* A = (const T*)p.A + (int64_t)z * p.sA;
   const T* B = (const T*)p.B + (int64_t)z * p.sB;
   float acc[4][4] = {};
+  const int passes = p.B2 ? 2 : 1;
+  for (int pass = 0; pass < passes; ++pass) {
+  if (pass == 1) B = (const T*)p.B2 + (int64_t)z * p.sB2;
   for (int k0 = 0; k0 < p.K; k0 += 16) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -113,6 +121,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmParams p) {
         for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
     }
     __syncthreads();
+  }
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i)
@@ -215,7 +224,7 @@ __device__ __forceinline__ void epi_row32(const GemmParams& p, int z, int m, int
 template <int BN, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const GemmParams p, int* err) {
+                   const __grid_constant__ CUtensorMap tmB2, const GemmParams p, int* err) {
   using C = TcCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -231,7 +240,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int n_tiles = p.N / BN;
   const int tiles_per_batch = m_tiles * n_tiles;
   const int num_tiles = tiles_per_batch * p.batch;
-  const int k_blocks = p.K / TC_BK;
+  const int kb_one = p.K / TC_BK;
+  const int k_blocks = p.B2 ? 2 * kb_one : kb_one;
+  const int zb_scale = p.sB ? 1 : 0;    // shared B (batch stride 0): always batch slice 0
+  const int zb2_scale = p.sB2 ? 1 : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -239,6 +251,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     fence_mbar_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    if (p.B2) prefetch_tmap(&tmB2);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -265,7 +278,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           uint8_t* sa = smem + s * C::STAGE_BYTES;
           uint8_t* sb = sa + C::A_BYTES;
           mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-          const int k0 = kb * TC_BK;
+          const bool second = kb >= kb_one;
+          const int k0 = (second ? kb - kb_one : kb) * TC_BK;
+          const CUtensorMap* mb = second ? &tmB2 : &tmB;
+          const int zb = z * (second ? zb2_scale : zb_scale);
           if (A_MN) {
             tma_load_3d(sa, &tmA, &full[s], m0, k0, z);
             tma_load_3d(sa + 8192, &tmA, &full[s], m0 + 64, k0, z);
@@ -274,9 +290,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           if (B_MN) {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j) tma_load_3d(sb + j * 8192, &tmB, &full[s], n0 + 64 * j, k0, z);
+            for (int j = 0; j < BN / 64; ++j) tma_load_3d(sb + j * 8192, mb, &full[s], n0 + 64 * j, k0, zb);
           } else {
-            tma_load_3d(sb, &tmB, &full[s], k0, n0, z);
+            tma_load_3d(sb, mb, &full[s], k0, n0, zb);
           }
         }
       }

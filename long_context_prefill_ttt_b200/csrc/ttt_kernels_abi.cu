@@ -5,6 +5,7 @@
 
 #include "ttt.h"
 #include "ttt_attention.cuh"
+#include "ttt_attention_mma.cuh"
 #include "ttt_common.cuh"
 #include "ttt_gemm.cuh"
 #include "ttt_kernels.h"
@@ -30,17 +31,23 @@ static int sm_count() {
 
 template <typename T>
 static int attn_fwd(const AttnParams& ap, int engine, cudaStream_t st) {
-  (void)engine;
   const int64_t rows = (int64_t)ap.B * ap.n;
+  if (sizeof(T) == 2 && engine != TTT_ENGINE_SIMT && attn_mma_ok(ap)) {
+    const cudaError_t e = ap.hd == 128 ? attn_fwd_mma_launch<128>(ap, st) : attn_fwd_mma_launch<64>(ap, st);
+    return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+  }
   attn_fwd_simt_kernel<T><<<(unsigned)((rows * ap.H + 3) / 4), 128, 0, st>>>(ap);
   return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 
 template <typename T>
 static int attn_bwd(const AttnParams& ap, int engine, cudaStream_t st) {
-  (void)engine;
   const int64_t rows = (int64_t)ap.B * ap.n;
   attn_bwd_prep_kernel<T><<<(unsigned)((rows * ap.H + 7) / 8), 256, 0, st>>>(ap);
+  if (sizeof(T) == 2 && engine != TTT_ENGINE_SIMT && attn_mma_ok(ap)) {
+    const cudaError_t e = ap.hd == 128 ? attn_bwd_mma_launch<128>(ap, st) : attn_bwd_mma_launch<64>(ap, st);
+    return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
+  }
   attn_bwd_dq_simt_kernel<T><<<(unsigned)((rows * ap.H + 3) / 4), 128, 0, st>>>(ap);
   attn_bwd_dkv_simt_kernel<T><<<(unsigned)((rows * ap.H + 3) / 4), 128, 0, st>>>(ap);
   return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
@@ -69,7 +76,8 @@ using namespace ttt;
 extern "C" {
 
 int ttt_k_gemm(int32_t elem_dtype, int32_t M, int32_t N, int32_t K, int32_t batch, const void* A, int64_t lda,
-               int64_t sA, int32_t a_mn, const void* B, int64_t ldb, int64_t sB, int32_t b_mn, void* D, int64_t ldd,
+               int64_t sA, int32_t a_mn, const void* B, int64_t ldb, int64_t sB, int32_t b_mn, const void* B2,
+               int64_t sB2, void* D, int64_t ldd,
                int64_t sD, int32_t d_f32, const void* X, int64_t ldx, int64_t sX, void* Y, int64_t ldy, int64_t sY,
                float alpha, int32_t epi, int32_t engine, void* stream) {
   if (M < 0 || N < 0 || K < 0 || batch < 1 || !A || !B || !D || epi < 0 || epi > 4) return TTT_ERR_INVALID_ARG;
@@ -82,6 +90,7 @@ int ttt_k_gemm(int32_t elem_dtype, int32_t M, int32_t N, int32_t K, int32_t batc
   p.M = M; p.N = N; p.K = K; p.batch = batch;
   p.A = A; p.lda = lda; p.sA = sA; p.a_mn = a_mn;
   p.B = B; p.ldb = ldb; p.sB = sB; p.b_mn = b_mn;
+  p.B2 = B2; p.sB2 = sB2;
   p.D = D; p.ldd = ldd; p.sD = sD; p.d_f32 = d_f32;
   p.X = X; p.ldx = ldx; p.sX = sX;
   p.Y = Y; p.ldy = ldy; p.sY = sY;

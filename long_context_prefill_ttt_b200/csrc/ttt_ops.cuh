@@ -271,6 +271,14 @@ __global__ void convert_kernel(const S* __restrict__ src, D* __restrict__ dst, i
   if (i < n) dst[i] = from_f32<D>(to_f32(src[i]));
 }
 
+// out = init + delta (fast weights W_init + dW exported in fp32)
+template <typename T>
+__global__ void add_init_kernel(const T* __restrict__ init, const float* __restrict__ delta, float* __restrict__ out,
+                                int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = to_f32(init[i]) + delta[i];
+}
+
 // Copy rows: dst[b][i][:] = src[b*src_bstride + (off + i)*ld ...] for i < n (fp32 rows of d).
 __global__ void gather_rows_kernel(const float* __restrict__ src, int64_t src_bstride, int64_t off, int n, int B,
                                    int d, float* __restrict__ dst, int64_t dst_bstride, int64_t dst_off) {

@@ -23,6 +23,7 @@
 
 #include "ttt.h"
 #include "ttt_attention.cuh"
+#include "ttt_attention_mma.cuh"
 #include "ttt_common.cuh"
 #include "ttt_gemm.cuh"
 #include "ttt_ops.cuh"
@@ -63,9 +64,10 @@ static bool make_operand_map(CUtensorMap* map, const void* base, int64_t rows, i
   }
   dims[2] = (cuuint64_t)batch;
   box[2] = 1;
+  if (bstride == 0) batch = 1;  // shared operand: one slice, always read at batch index 0
+  dims[2] = (cuuint64_t)batch;
   strides[0] = (cuuint64_t)ld * 2;
   strides[1] = (cuuint64_t)(batch > 1 ? bstride : (mn_major ? K : rows) * ld) * 2;
-  if (strides[1] == 0) strides[1] = strides[0];
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -76,9 +78,11 @@ static bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
 template <int BN, bool AM, bool BM>
 static cudaError_t launch_tc(const GemmParams& p, cudaStream_t st, int* err, int num_sms, bool* ok) {
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tb2;
   *ok = make_operand_map(&ta, p.A, p.M, p.K, p.lda, p.batch, p.sA, AM, TC_BM) &&
         make_operand_map(&tb, p.B, p.N, p.K, p.ldb, p.batch, p.sB, BM, BN);
+  if (*ok && p.B2) *ok = make_operand_map(&tb2, p.B2, p.N, p.K, p.ldb, p.batch, p.sB2, BM, BN);
+  else tb2 = tb;
   if (!*ok) return cudaSuccess;
   using C = TcCfg<BN>;
   static bool attr_set = false;
@@ -90,7 +94,7 @@ static cudaError_t launch_tc(const GemmParams& p, cudaStream_t st, int* err, int
   }
   const int tiles = ((p.M + TC_BM - 1) / TC_BM) * (p.N / BN) * p.batch;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  gemm_tc_kernel<BN, AM, BM><<<grid, TC_THREADS, C::SMEM, st>>>(ta, tb, p, err);
+  gemm_tc_kernel<BN, AM, BM><<<grid, TC_THREADS, C::SMEM, st>>>(ta, tb, tb2, p, err);
   return cudaGetLastError();
 }
 
@@ -100,7 +104,8 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
   bool use_tc = elem_is_bf16 && !force_simt && (p.K % TC_BK == 0) && (p.N % 128 == 0) && aligned16(p.A) &&
                 aligned16(p.B) && aligned16(p.D) && (p.lda % 8 == 0) && (p.ldb % 8 == 0) &&
                 (p.ldd % (p.d_f32 || p.epi == EPI_RESID || p.epi == EPI_SGD ? 4 : 8) == 0) &&
-                (p.batch == 1 || (p.sA % 8 == 0 && p.sB % 8 == 0)) && (!p.a_mn || p.b_mn) && p.M >= 1;
+                (p.batch == 1 || (p.sA % 8 == 0 && p.sB % 8 == 0 && p.sB2 % 8 == 0)) && (!p.a_mn || p.b_mn) &&
+                p.M >= 1 && (!p.B2 || aligned16(p.B2));
   if (use_tc && p.X && !(aligned16(p.X) && p.ldx % (p.epi == EPI_DGELU ? 8 : 4) == 0 &&
                          (p.batch == 1 || p.sX % 8 == 0)))
     use_tc = false;
@@ -154,6 +159,49 @@ struct Arena {
   }
 };
 
+// Kernel-class timer: CUDA events recorded on the launching stream around each
+// launch of a class, plus the algorithmic FLOPs and bytes of that launch.
+enum ProfClass : int { PC_GEMM_FROZEN = 0, PC_GEMM_TTT = 1, PC_ATTN_FWD = 2, PC_ATTN_BWD = 3, PC_COUNT = 4 };
+struct Profiler {
+  bool on = false;
+  std::vector<cudaEvent_t> ev;     // pairs
+  std::vector<int> cls;
+  std::vector<double> fl, by;
+  size_t used = 0;
+  double ms[PC_COUNT] = {}, flops[PC_COUNT] = {}, bytes[PC_COUNT] = {};
+  int64_t n[PC_COUNT] = {};
+  void begin(cudaStream_t st, int c, double f, double b) {
+    if (!on) return;
+    if (used * 2 + 2 > ev.size()) {
+      for (int i = 0; i < 256; ++i) {
+        cudaEvent_t e;
+        cudaEventCreate(&e);
+        ev.push_back(e);
+      }
+    }
+    cls.resize(used + 1); fl.resize(used + 1); by.resize(used + 1);
+    cls[used] = c; fl[used] = f; by[used] = b;
+    cudaEventRecord(ev[2 * used], st);
+  }
+  void end(cudaStream_t st) {
+    if (!on) return;
+    cudaEventRecord(ev[2 * used + 1], st);
+    ++used;
+  }
+  void collect() {  // after the stream has synchronised
+    for (size_t i = 0; i < used; ++i) {
+      float t = 0.f;
+      cudaEventElapsedTime(&t, ev[2 * i], ev[2 * i + 1]);
+      ms[cls[i]] += t; flops[cls[i]] += fl[i]; bytes[cls[i]] += by[i]; n[cls[i]] += 1;
+    }
+    used = 0;
+  }
+  void clear() {
+    for (int c = 0; c < PC_COUNT; ++c) { ms[c] = flops[c] = bytes[c] = 0; n[c] = 0; }
+  }
+  ~Profiler() { for (auto e : ev) cudaEventDestroy(e); }
+};
+
 }  // namespace ttt
 
 // ============================================================== handle
@@ -168,6 +216,7 @@ struct ttt_handle {
   int64_t n_pos = 0;
   int64_t launches = 0;
   int64_t dev_bytes = 0;
+  ttt::Profiler prof;
 };
 
 namespace ttt {
@@ -206,9 +255,14 @@ template <typename T> struct LayerDev {
   float* g_mlp = nullptr; T* W1 = nullptr; T* W2 = nullptr;           // frozen MLP
   float* g_ttt = nullptr; float* g_static = nullptr;                   // adaptive block
   T* W1s = nullptr; T* W2s = nullptr;
-  float* W1t32 = nullptr; float* W2t32 = nullptr;                      // [B][ht][d], [B][d][ht] master
-  T* W1t = nullptr; T* W2t = nullptr;                                  // shadows (alias master for fp32)
-  float* W1t_init = nullptr; float* W2t_init = nullptr;                // W_init (one copy)
+  // Fast weights of the adaptive MLP, per sequence. fp32 path: W itself (W1t32/W2t32,
+  // shadows alias them). bf16 path: W = W_init + dW with W_init held once in bf16
+  // (shared by all sequences) and the per-sequence update dW as an fp32 master
+  // (W1t32/W2t32) plus a bf16 copy for the GEMMs (W1t/W2t): a bf16 copy of
+  // W_init + dW would round most of a small update away.
+  float* W1t32 = nullptr; float* W2t32 = nullptr;                      // [B][ht][d], [B][d][ht]
+  T* W1t = nullptr; T* W2t = nullptr;
+  T* W1t_init = nullptr; T* W2t_init = nullptr;                        // [ht][d], [d][ht]
   T* ring_k = nullptr; T* ring_v = nullptr;                            // [B][C][d]
 };
 
@@ -253,6 +307,7 @@ template <typename T> class Engine : public ttt_handle {
   int32_t* tok_dev = nullptr; int64_t tok_cap = 0;
   float* loss_dev = nullptr; int64_t loss_cap = 0;
   int32_t* otok_dev = nullptr; int64_t otok_cap = 0;
+  float* wexp = nullptr; int64_t wexp_cap = 0;
   Arena call_arena;
 
   ~Engine() override {
@@ -268,8 +323,14 @@ template <typename T> class Engine : public ttt_handle {
   int reset() override;
 
  private:
+  int gemm_class = PC_GEMM_FROZEN;
   int gemm(GemmParams p) {
+    const size_t es = is_bf16 ? 2 : 4;
+    prof.begin(st, gemm_class, 2.0 * p.M * p.N * (double)p.K * p.batch,
+               (double)p.batch * ((double)p.M * p.K * es + (double)p.N * p.K * es +
+                                  (double)p.M * p.N * (p.d_f32 ? 4 : es)));
     const int e = gemm_launch(p, is_bf16 ? 1 : 0, st, dev_err, num_sms, 0);
+    prof.end(st);
     ++launches;
     if (e != 0) {
       poisoned = true;
@@ -287,6 +348,27 @@ template <typename T> class Engine : public ttt_handle {
     p.D = D; p.ldd = ldd; p.d_f32 = d_f32;
     p.alpha = 1.f; p.epi = epi;
     return p;
+  }
+  // sum over queries P = q0..q0+n-1 of min(P+1, k): query-key pairs of the window (review eq. (1))
+  double attn_pairs(int64_t n, int64_t q0) const {
+    double s = 0;
+    const int64_t k = kwin;
+    // positions below k contribute P+1, the rest k
+    const int64_t a = q0, b = q0 + n;  // [a, b)
+    const int64_t m = b < k ? b : (a > k ? a : k);  // split point clamp
+    if (a < m) s += (double)(m - a) * (a + 1 + m) / 2.0;  // sum_{P=a}^{m-1} (P+1)
+    if (m < b) s += (double)(b - (a > m ? a : m)) * k;
+    return s;
+  }
+  // B operand of a product with the fast weights W (per sequence): fp32 path reads W
+  // directly; bf16 path accumulates W_init (shared) and dW (per sequence).
+  void fast_operand(GemmParams& p, const T* init, const T* delta, int64_t per_seq) const {
+    if (is_bf16) {
+      p.B = init; p.sB = 0;
+      p.B2 = delta; p.sB2 = per_seq;
+    } else {
+      p.B = delta; p.sB = per_seq;
+    }
   }
   int attention_block(const LayerDev<T>& Lw, int layer, float* xin, float* xout, T* r, float* rstd, T* qkv, T* o,
                       float* lse, int n, int64_t q0, bool commit);
@@ -311,6 +393,7 @@ template <typename T> int Engine<T>::ensure(void** ptr, int64_t* cap, int64_t ne
 
 template <typename T> int Engine<T>::sync_and_check() {
   TTT_CUDA(cudaStreamSynchronize(st));
+  prof.collect();
   int flag = 0;
   TTT_CUDA(cudaMemcpy(&flag, dev_err, sizeof(int), cudaMemcpyDeviceToHost));
   if (flag == DEV_BAD_TOKEN) {
@@ -366,8 +449,8 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
       Lw.W2s = arena.get<T>((size_t)d * hs);
       Lw.W1t32 = arena.get<float>((size_t)B * ht * d);
       Lw.W2t32 = arena.get<float>((size_t)B * d * ht);
-      Lw.W1t_init = arena.get<float>((size_t)ht * d);
-      Lw.W2t_init = arena.get<float>((size_t)d * ht);
+      Lw.W1t_init = arena.get<T>((size_t)ht * d);
+      Lw.W2t_init = arena.get<T>((size_t)d * ht);
       if (is_bf16) {
         Lw.W1t = arena.get<T>((size_t)B * ht * d);
         Lw.W2t = arena.get<T>((size_t)B * d * ht);
@@ -500,8 +583,8 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
       UP(Lw.W2, false, (int64_t)d * h, false);
     } else {
       UP(Lw.g_ttt, true, d, true);
-      UP(Lw.W1t_init, true, (int64_t)ht * d, false);
-      UP(Lw.W2t_init, true, (int64_t)d * ht, false);
+      UP(Lw.W1t_init, !is_bf16, (int64_t)ht * d, false);
+      UP(Lw.W2t_init, !is_bf16, (int64_t)d * ht, false);
       UP(Lw.g_static, true, d, true);
       UP(Lw.W1s, false, (int64_t)hs * d, false);
       UP(Lw.W2s, false, (int64_t)d * hs, false);
@@ -517,15 +600,16 @@ template <typename T> int Engine<T>::reset() {
   for (int l = first_ttt; l < L; ++l) {
     LayerDev<T>& Lw = layers[l];
     const int64_t n1 = (int64_t)ht * d;
-    for (int b = 0; b < B; ++b) {
-      TTT_CUDA(cudaMemcpyAsync(Lw.W1t32 + b * n1, Lw.W1t_init, n1 * 4, cudaMemcpyDeviceToDevice, st));
-      TTT_CUDA(cudaMemcpyAsync(Lw.W2t32 + b * n1, Lw.W2t_init, n1 * 4, cudaMemcpyDeviceToDevice, st));
-    }
-    if (is_bf16) {
-      convert_kernel<float, T><<<nblk(B * n1, 256), 256, 0, st>>>(Lw.W1t32, Lw.W1t, B * n1);
-      TTT_LAUNCHED();
-      convert_kernel<float, T><<<nblk(B * n1, 256), 256, 0, st>>>(Lw.W2t32, Lw.W2t, B * n1);
-      TTT_LAUNCHED();
+    if (is_bf16) {  // dW = 0
+      TTT_CUDA(cudaMemsetAsync(Lw.W1t32, 0, (size_t)B * n1 * 4, st));
+      TTT_CUDA(cudaMemsetAsync(Lw.W2t32, 0, (size_t)B * n1 * 4, st));
+      TTT_CUDA(cudaMemsetAsync(Lw.W1t, 0, (size_t)B * n1 * sizeof(T), st));
+      TTT_CUDA(cudaMemsetAsync(Lw.W2t, 0, (size_t)B * n1 * sizeof(T), st));
+    } else {  // W = W_init
+      for (int b = 0; b < B; ++b) {
+        TTT_CUDA(cudaMemcpyAsync(Lw.W1t32 + b * n1, Lw.W1t_init, n1 * 4, cudaMemcpyDeviceToDevice, st));
+        TTT_CUDA(cudaMemcpyAsync(Lw.W2t32 + b * n1, Lw.W2t_init, n1 * 4, cudaMemcpyDeviceToDevice, st));
+      }
     }
   }
   for (int l = 0; l < L; ++l) {
@@ -559,7 +643,14 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
   ap.Q = qkv; ap.ldq = 3 * d; ap.K = qkv + d; ap.V = qkv + 2 * d; ap.ldkv = 3 * d;
   ap.Kc = Lw.ring_k; ap.Vc = Lw.ring_v; ap.C = C;
   ap.O = o; ap.ldo = d; ap.lse = lse; ap.scale = 1.0f / sqrtf((float)hd);
-  attn_fwd_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
+  prof.begin(st, PC_ATTN_FWD, 4.0 * hd * H * (double)B * attn_pairs(n, q0), 0.0);
+  if (is_bf16 && attn_mma_ok(ap)) {
+    const cudaError_t e = hd == 128 ? attn_fwd_mma_launch<128>(ap, st) : attn_fwd_mma_launch<64>(ap, st);
+    (void)e;
+  } else {
+    attn_fwd_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
+  }
+  prof.end(st);
   TTT_LAUNCHED();
   GemmParams p = gp(rows, d, d, o, d, false, Lw.Wo, d, false, xout, d, true, EPI_RESID);
   p.X = xin; p.ldx = d;
@@ -601,11 +692,13 @@ template <typename T> int Engine<T>::ttt_forward(int cn, int64_t pos, bool commi
     rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(A.a, d, Lw.g_ttt, cfg.rms_eps, rows, d, A.r2, d, A.rstd2);
     TTT_LAUNCHED();
     GemmParams p = gp(cn, ht, d, A.r2, d, false, Lw.W1t, d, false, A.g, ht, false, EPI_GELU);
-    p.batch = B; p.sA = (int64_t)cn * d; p.sB = (int64_t)ht * d; p.sD = (int64_t)cn * ht;
+    p.batch = B; p.sA = (int64_t)cn * d; p.sD = (int64_t)cn * ht;
+    fast_operand(p, Lw.W1t_init, Lw.W1t, (int64_t)ht * d);
     p.Y = A.u; p.ldy = ht; p.sY = (int64_t)cn * ht;
     if ((rc = gemm(p)) != TTT_OK) return rc;
     p = gp(cn, d, ht, A.g, ht, false, Lw.W2t, ht, false, A.m, d, true, EPI_RESID);
-    p.batch = B; p.sA = (int64_t)cn * ht; p.sB = (int64_t)d * ht; p.sD = (int64_t)cn * d;
+    p.batch = B; p.sA = (int64_t)cn * ht; p.sD = (int64_t)cn * d;
+    fast_operand(p, Lw.W2t_init, Lw.W2t, (int64_t)d * ht);
     p.X = A.a; p.ldx = d; p.sX = (int64_t)cn * d;
     if ((rc = gemm(p)) != TTT_OK) return rc;
     // static MLP
@@ -645,15 +738,18 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
     TTT_LAUNCHED();
     // TTT-MLP data gradients (with W_{i-1}), then the fused weight gradient + SGD
     p = gp(cn, ht, d, GT, d, false, Lw.W2t, ht, true, dhid, ht, false, EPI_DGELU);
-    p.batch = B; p.sA = (int64_t)cn * d; p.sB = (int64_t)d * ht; p.sD = (int64_t)cn * ht;
+    p.batch = B; p.sA = (int64_t)cn * d; p.sD = (int64_t)cn * ht;
+    fast_operand(p, Lw.W2t_init, Lw.W2t, (int64_t)d * ht);
     p.X = A.u; p.ldx = ht; p.sX = (int64_t)cn * ht;
     if ((rc = gemm(p)) != TTT_OK) return rc;
     if (j > 0) {
       p = gp(cn, d, ht, dhid, ht, false, Lw.W1t, d, true, dr, d, true, EPI_STORE);
-      p.batch = B; p.sA = (int64_t)cn * ht; p.sB = (int64_t)ht * d; p.sD = (int64_t)cn * d;
+      p.batch = B; p.sA = (int64_t)cn * ht; p.sD = (int64_t)cn * d;
+      fast_operand(p, Lw.W1t_init, Lw.W1t, (int64_t)ht * d);
       if ((rc = gemm(p)) != TTT_OK) return rc;
     }
-    // dW2t[o][i] = sum_t dm[t][o] g[t][i]  -> W2t32 += -eta * dW2t ; shadow refreshed
+    // dW2t[o][i] = sum_t dm[t][o] g[t][i]  -> W2t32 += -eta * dW2t ; bf16 copy refreshed
+    // (bf16 path: W2t32 holds the accumulated update dW, so the copy keeps its precision)
     p = gp(d, ht, cn, GT, d, true, A.g, ht, true, Lw.W2t32, ht, true, EPI_SGD);
     p.batch = B; p.sA = (int64_t)cn * d; p.sB = (int64_t)cn * ht; p.sD = (int64_t)d * ht;
     p.alpha = -cfg.eta;
@@ -679,11 +775,22 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
     ap.dO = dob; ap.lddo = d; ap.Dsum = Dsum;
     ap.dQ = dqkv; ap.dK = dqkv + d; ap.dV = dqkv + 2 * d; ap.lddq = 3 * d;
     ap.q0 = chunk_pos;
+    // algorithmic (recompute of QK^T not counted): dQ over the window (dO V^T, dS K) and
+    // dK, dV over current-chunk keys only (dS^T Q, P^T dO)
+    prof.begin(st, PC_ATTN_BWD,
+               2.0 * hd * H * (double)B * (2.0 * attn_pairs(cn, chunk_pos) + 2.0 * attn_pairs(cn, 0)), 0.0);
     attn_bwd_prep_kernel<T><<<nblk((int64_t)rows * H, 8), 256, 0, st>>>(ap);
     TTT_LAUNCHED();
-    attn_bwd_dq_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
-    TTT_LAUNCHED();
-    attn_bwd_dkv_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
+    if (is_bf16 && attn_mma_ok(ap)) {
+      const cudaError_t e = hd == 128 ? attn_bwd_mma_launch<128>(ap, st) : attn_bwd_mma_launch<64>(ap, st);
+      (void)e;
+      launches += 1;
+    } else {
+      attn_bwd_dq_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
+      TTT_LAUNCHED();
+      attn_bwd_dkv_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
+    }
+    prof.end(st);
     TTT_LAUNCHED();
     rope_kernel<T><<<nblk((int64_t)rows * d, 256), 256, 0, st>>>(dqkv, 3 * d, 2 * d, rows, cn, chunk_pos, hd,
                                                                   rope_lo, rope_hi, 1);
@@ -709,6 +816,7 @@ int Engine<T>::ttt_step(const float* in, const int32_t* targets, int cn, int64_t
   const int rows = B * cn;
   int rc;
   chunk_pos = pos;
+  gemm_class = PC_GEMM_TTT;
   if (in != blk[0].x) {
     TTT_CUDA(cudaMemcpyAsync(blk[0].x, in, (size_t)rows * d * 4, cudaMemcpyDeviceToDevice, st));
   }
@@ -762,6 +870,7 @@ template <typename T> int Engine<T>::prefill(const int32_t* tokens, int64_t T_, 
     const int rows = B * n;
     embed_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(tok_dev, ld, (int)s0, n, rows, E, V, d, xs, dev_err);
     TTT_LAUNCHED();
+    gemm_class = PC_GEMM_FROZEN;
     for (int l = 0; l < first_ttt; ++l) {
       if ((rc = attention_block(layers[l], l, xs, xs, rs, nullptr, qkvs, os, nullptr, n, P0, true)) != TTT_OK)
         return rc;
@@ -881,8 +990,27 @@ template <typename T> int Engine<T>::get_weights(int32_t seq, int32_t j, float* 
   const LayerDev<T>& Lw = layers[first_ttt + j];
   const int64_t n1 = (int64_t)ht * d;
   const cudaMemcpyKind k = kind == TTT_PTR_HOST ? cudaMemcpyDeviceToHost : cudaMemcpyDeviceToDevice;
-  if (w1) TTT_CUDA(cudaMemcpyAsync(w1, Lw.W1t32 + seq * n1, n1 * 4, k, st));
-  if (w2) TTT_CUDA(cudaMemcpyAsync(w2, Lw.W2t32 + seq * n1, n1 * 4, k, st));
+  if (!is_bf16) {
+    if (w1) TTT_CUDA(cudaMemcpyAsync(w1, Lw.W1t32 + seq * n1, n1 * 4, k, st));
+    if (w2) TTT_CUDA(cudaMemcpyAsync(w2, Lw.W2t32 + seq * n1, n1 * 4, k, st));
+    return sync_and_check();
+  }
+  // W = W_init + dW, formed in fp32 on the device
+  float* stage = nullptr;
+  int64_t cap = 0;
+  int rc;
+  if ((rc = ensure((void**)&wexp, &wexp_cap, n1, 4)) != TTT_OK) return rc;
+  stage = wexp;
+  (void)cap;
+  for (int m = 0; m < 2; ++m) {
+    float* dst = m == 0 ? w1 : w2;
+    if (!dst) continue;
+    add_init_kernel<T><<<nblk(n1, 256), 256, 0, st>>>(m == 0 ? Lw.W1t_init : Lw.W2t_init,
+                                                      (m == 0 ? Lw.W1t32 : Lw.W2t32) + seq * n1, stage, n1);
+    TTT_LAUNCHED();
+    TTT_CUDA(cudaMemcpyAsync(dst, stage, n1 * 4, k, st));
+    TTT_CUDA(cudaStreamSynchronize(st));
+  }
   return sync_and_check();
 }
 
@@ -969,6 +1097,25 @@ int ttt_reset(ttt_handle* h) {
 int64_t ttt_position(const ttt_handle* h) { return h ? h->n_pos : -1; }
 int64_t ttt_device_bytes(const ttt_handle* h) { return h ? h->dev_bytes : -1; }
 int64_t ttt_last_launch_count(const ttt_handle* h) { return h ? h->launches : -1; }
+
+int ttt_profile(ttt_handle* h, int32_t enable) {
+  if (!h) return TTT_ERR_INVALID_ARG;
+  h->prof.on = enable != 0;
+  h->prof.clear();
+  return TTT_OK;
+}
+
+int ttt_profile_read(const ttt_handle* h, int32_t n_classes, double* ms, int64_t* launches, double* flops,
+                     double* bytes) {
+  if (!h || n_classes < 0) return TTT_ERR_INVALID_ARG;
+  for (int c = 0; c < n_classes && c < PC_COUNT; ++c) {
+    if (ms) ms[c] = h->prof.ms[c];
+    if (launches) launches[c] = h->prof.n[c];
+    if (flops) flops[c] = h->prof.flops[c];
+    if (bytes) bytes[c] = h->prof.bytes[c];
+  }
+  return PC_COUNT;
+}
 
 void ttt_destroy(ttt_handle* h) { delete h; }
 

@@ -48,6 +48,24 @@ def test_gemm_store_f32(T, a_mn, b_mn, M, N, K, batch, engine):
     assert err < 2e-6, err
 
 
+@pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1)])
+@pytest.mark.parametrize("engine", [0, 1])
+def test_gemm_shared_plus_per_batch_operand(T, a_mn, b_mn, engine):
+    """acc = A (B_shared + B2[z]): a small per-batch B2 must survive next to a large shared B."""
+    M, N, K, batch = 200, 256, 192, 3
+    A = _rand((batch, M, K), torch.bfloat16, 21)
+    Bs = _rand((1, N, K), torch.bfloat16, 22)
+    B2 = _rand((batch, N, K), torch.bfloat16, 23, 1e-3)
+    ref = A.double() @ (Bs.double() + B2.double()).transpose(1, 2)
+    D = torch.empty((batch, M, N), dtype=torch.float32, device="cuda")
+    T.ttt_k_gemm(_store(A, a_mn), _store(Bs, b_mn), D, M, N, K, batch=batch, sA=M * K, a_mn=a_mn, sB=0,
+                 b_mn=b_mn, B2=_store(B2, b_mn), sB2=N * K, sD=M * N, engine=engine)
+    T.ttt_k_status()
+    small = A.double() @ B2.double().transpose(1, 2)
+    err = (D.double() - ref).abs().max().item()
+    assert err < 1e-3 * small.abs().max().item(), (err, small.abs().max().item())
+
+
 @pytest.mark.parametrize("M,N,K", [(256, 512, 256), (130, 256, 64)])
 def test_gemm_store_bf16_and_fp32_simt(T, M, N, K):
     A = _rand((1, M, K), torch.bfloat16, 3)
@@ -125,17 +143,27 @@ def _attn_reference(qkv, ring_k, ring_v, B, H, hd, n, q0, window, C):
     return q, kc, vc, K, V, mask.cuda(), lo
 
 
+ATTN_CASES = [
+    # SIMT engine (q0 not 64-aligned, head dim 16, single query)
+    (2, 2, 64, 96, 160, 128, 256), (1, 4, 16, 48, 0, 16, 32), (1, 2, 128, 64, 300, 200, 384),
+    (3, 1, 64, 1, 777, 64, 128),
+    # tensor-core engine for bf16 (q0 % 64 == 0): ragged rows, windows off the tile grid, window < tile
+    (2, 2, 64, 96, 128, 128, 256), (1, 2, 128, 200, 256, 300, 640), (2, 3, 128, 64, 0, 64, 128),
+    (1, 2, 64, 130, 64, 40, 128), (1, 1, 128, 256, 1024, 1024, 2048),
+]
+
+
+@pytest.mark.parametrize("engine", [0, 1])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("B,H,hd,n,q0,window,C", [(2, 2, 64, 96, 160, 128, 256), (1, 4, 16, 48, 0, 16, 32),
-                                                  (1, 2, 128, 64, 300, 200, 384), (3, 1, 64, 1, 777, 64, 128)])
-def test_attention_forward_and_backward(T, dtype, B, H, hd, n, q0, window, C):
+@pytest.mark.parametrize("B,H,hd,n,q0,window,C", ATTN_CASES)
+def test_attention_forward_and_backward(T, engine, dtype, B, H, hd, n, q0, window, C):
     d = H * hd
     qkv = _rand((B * n, 3 * d), dtype, 11)
     ring_k = _rand((B, C, d), dtype, 12)
     ring_v = _rand((B, C, d), dtype, 13)
     out = torch.empty((B * n, d), dtype=dtype, device="cuda")
     lse = torch.empty((B, H, n), dtype=torch.float32, device="cuda")
-    T.ttt_k_attention_fwd(qkv, out, lse, B, H, hd, n, q0, window, ring_k, ring_v, C)
+    T.ttt_k_attention_fwd(qkv, out, lse, B, H, hd, n, q0, window, ring_k, ring_v, C, engine=engine)
     T.ttt_k_status()
     q, kc, vc, K, V, mask, lo = _attn_reference(qkv, ring_k, ring_v, B, H, hd, n, q0, window, C)
     q.requires_grad_(True); kc.requires_grad_(True); vc.requires_grad_(True)
@@ -154,7 +182,8 @@ def test_attention_forward_and_backward(T, dtype, B, H, hd, n, q0, window, C):
     o.backward(dout.double().view(B, n, H, hd))
     dqkv = torch.zeros((B * n, 3 * d), dtype=dtype, device="cuda")
     dsum = torch.empty((B, H, n), dtype=torch.float32, device="cuda")
-    T.ttt_k_attention_bwd(qkv, out, lse, dout, dqkv, dsum, B, H, hd, n, q0, window, ring_k, ring_v, C)
+    T.ttt_k_attention_bwd(qkv, out, lse, dout, dqkv, dsum, B, H, hd, n, q0, window, ring_k, ring_v, C,
+                          engine=engine)
     T.ttt_k_status()
     for got, ref in ((dqkv[:, :d], q.grad), (dqkv[:, d:2 * d], kc.grad), (dqkv[:, 2 * d:], vc.grad)):
         scale = ref.abs().max().item() + 1e-12

@@ -146,6 +146,19 @@ def test_small_bf16_matches_oracle(T):
     assert rep["dw"] <= 5e-2
 
 
+def test_bf16_update_effect_matches_oracle(T):
+    """The update moves the next chunks' losses; in bf16 that move must match the
+    oracle's (a bf16 copy of W_init + dW would round a small dW away)."""
+    cfg = syn.config("small_bf16", T=1024)
+    r = P.prefill_both(T, cfg)
+    static = Oracle(cfg.replace(eta=0.0), r["w"]).prefill(r["toks"])[0]
+    b = cfg.minibatch_b
+    want = float(np.mean(r["orc_losses"][0][b:] - static[b:]))
+    got = float(np.mean(r["gpu_losses"][0][b:] - static[b:]))
+    assert abs(want) > 1e-3
+    assert abs(got - want) <= 0.1 * abs(want), (got, want)
+
+
 def test_small_bf16_device_buffers_match_host_buffers(T):
     cfg = syn.config("small_bf16", T=1024)
     w = syn.make_weights(cfg)
