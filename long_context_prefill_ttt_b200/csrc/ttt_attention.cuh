@@ -227,4 +227,80 @@ __global__ void __launch_bounds__(128) attn_bwd_dkv_simt_kernel(AttnParams p) {
   }
 }
 
+// ---------------------------------------------------------------- decode (one query)
+// One query per sequence at position P = *pos (the token's own K/V already in the
+// ring); keys [max(0, P-k+1), P] all read from the ring. One CTA per (head,
+// sequence), 8 warps splitting the window, lanes over keys for the scores and over
+// head dims for P·V, merged across warps at the end. HBM-bound: each key and value
+// row of the window is read once.
+template <typename T>
+__global__ void __launch_bounds__(256) attn_decode_kernel(const T* __restrict__ q, int64_t ldq,
+                                                          const T* __restrict__ ring_k, const T* __restrict__ ring_v,
+                                                          int C, int d, int hd, int window,
+                                                          const int64_t* __restrict__ pos, float scale,
+                                                          T* __restrict__ out, int64_t ldo) {
+  __shared__ float qs[128];
+  __shared__ float wm[8], wl[8];
+  __shared__ float wo[8][128];
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t P = *pos;
+  const int64_t lo = P - window + 1 > 0 ? P - window + 1 : 0;
+  for (int c = threadIdx.x; c < hd; c += 256) qs[c] = to_f32(q[(int64_t)b * ldq + h * hd + c]) * scale;
+  __syncthreads();
+  const T* Kb = ring_k + (int64_t)b * C * d + h * hd;
+  const T* Vb = ring_v + (int64_t)b * C * d + h * hd;
+  const int nd = (hd + 31) / 32;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float m = -INFINITY, l = 0.f;
+  for (int64_t j0 = lo + warp * 32; j0 <= P; j0 += 256) {
+    const int64_t j = j0 + lane;
+    float s = -INFINITY;
+    if (j <= P) {
+      const T* kr = Kb + (j % C) * d;
+      float dot = 0.f;
+      for (int c = 0; c < hd; ++c) dot = fmaf(qs[c], to_f32(kr[c]), dot);
+      s = dot;
+    }
+    float mb = s;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+    const float mnew = fmaxf(m, mb);
+    const float pj = (j <= P) ? expf(s - mnew) : 0.f;
+    const float corr = expf(m - mnew);
+    float ps = pj;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+    l = l * corr + ps;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) acc[t] *= corr;
+    const int cnt = (int)((P - j0 + 1) < 32 ? (P - j0 + 1) : 32);
+    for (int jj = 0; jj < cnt; ++jj) {
+      const float pp = __shfl_sync(0xffffffffu, pj, jj);
+      const T* vr = Vb + ((j0 + jj) % C) * d;
+      for (int t = 0; t < nd; ++t) {
+        const int c = lane + 32 * t;
+        if (c < hd) acc[t] = fmaf(pp, to_f32(vr[c]), acc[t]);
+      }
+    }
+    m = mnew;
+  }
+  if (lane == 0) { wm[warp] = m; wl[warp] = l; }
+  for (int t = 0; t < nd; ++t) {
+    const int c = lane + 32 * t;
+    if (c < hd) wo[warp][c] = acc[t];
+  }
+  __syncthreads();
+  float M = -INFINITY;
+  for (int w = 0; w < 8; ++w) M = fmaxf(M, wm[w]);
+  float Lsum = 0.f;
+  for (int w = 0; w < 8; ++w) Lsum += wm[w] == -INFINITY ? 0.f : wl[w] * expf(wm[w] - M);
+  for (int c = threadIdx.x; c < hd; c += 256) {
+    float o = 0.f;
+    for (int w = 0; w < 8; ++w)
+      if (wm[w] != -INFINITY) o += wo[w][c] * expf(wm[w] - M);
+    out[(int64_t)b * ldo + h * hd + c] = from_f32<T>(o / Lsum);
+  }
+}
+
 }  // namespace ttt

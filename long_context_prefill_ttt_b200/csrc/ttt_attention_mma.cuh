@@ -488,29 +488,28 @@ inline bool attn_mma_ok(const AttnParams& p) {
          p.ldkv % 8 == 0 && p.d % 8 == 0 && p.n >= 1;
 }
 
+template <int HD> inline cudaError_t attn_mma_attributes() {
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_mma_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       attn_fwd_mma_smem<HD>());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_bwd_dq_mma_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             attn_bwd_mma_smem<HD>());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(attn_bwd_dkv_mma_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             attn_bwd_mma_smem<HD>());
+  return e;
+}
+
+// (attributes are set by prime_kernel_attributes() before the first launch)
 template <int HD> inline cudaError_t attn_fwd_mma_launch(const AttnParams& p, cudaStream_t st) {
-  static bool set = false;
   constexpr int smem = attn_fwd_mma_smem<HD>();
-  if (!set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_mma_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    set = true;
-  }
   dim3 grid((p.n + AM_BM - 1) / AM_BM, p.H, p.B);
   attn_fwd_mma_kernel<HD><<<grid, 128, smem, st>>>(p);
   return cudaGetLastError();
 }
 
 template <int HD> inline cudaError_t attn_bwd_mma_launch(const AttnParams& p, cudaStream_t st) {
-  static bool set = false;
   constexpr int smem = attn_bwd_mma_smem<HD>();
-  if (!set) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_dq_mma_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(attn_bwd_dkv_mma_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    set = true;
-  }
   dim3 grid((p.n + AM_BM - 1) / AM_BM, p.H, p.B);
   attn_bwd_dq_mma_kernel<HD><<<grid, 128, smem, st>>>(p);
   attn_bwd_dkv_mma_kernel<HD><<<grid, 128, smem, st>>>(p);

@@ -367,5 +367,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 // ============================================================== host side
 int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t stream, int* err, int num_sms,
                 int force_simt);
+// Sets the dynamic shared-memory limits of all large-smem kernels; 0 or a cudaError_t.
+int prime_kernel_attributes();
 
 }  // namespace ttt

@@ -23,6 +23,7 @@ static int* status_word() {
 }
 
 static int sm_count() {
+  prime_kernel_attributes();
   int dev = 0, n = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -31,6 +32,7 @@ static int sm_count() {
 
 template <typename T>
 static int attn_fwd(const AttnParams& ap, int engine, cudaStream_t st) {
+  if (prime_kernel_attributes() != 0) return TTT_ERR_CUDA;
   const int64_t rows = (int64_t)ap.B * ap.n;
   if (sizeof(T) == 2 && engine != TTT_ENGINE_SIMT && attn_mma_ok(ap)) {
     const cudaError_t e = ap.hd == 128 ? attn_fwd_mma_launch<128>(ap, st) : attn_fwd_mma_launch<64>(ap, st);
@@ -42,6 +44,7 @@ static int attn_fwd(const AttnParams& ap, int engine, cudaStream_t st) {
 
 template <typename T>
 static int attn_bwd(const AttnParams& ap, int engine, cudaStream_t st) {
+  if (prime_kernel_attributes() != 0) return TTT_ERR_CUDA;
   const int64_t rows = (int64_t)ap.B * ap.n;
   attn_bwd_prep_kernel<T><<<(unsigned)((rows * ap.H + 7) / 8), 256, 0, st>>>(ap);
   if (sizeof(T) == 2 && engine != TTT_ENGINE_SIMT && attn_mma_ok(ap)) {

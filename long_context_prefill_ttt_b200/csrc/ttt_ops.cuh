@@ -104,7 +104,9 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ x, const float* __r
 // inverse != 0 applies the transpose rotation (backward of the forward map).
 template <typename T>
 __global__ void rope_kernel(T* __restrict__ qk, int64_t ld, int ncols, int rows, int n, int64_t pos0, int hd,
-                            const float2* __restrict__ lo_tab, const float2* __restrict__ hi_tab, int inverse) {
+                            const float2* __restrict__ lo_tab, const float2* __restrict__ hi_tab, int inverse,
+                            const int64_t* pos_dev = nullptr) {
+  if (pos_dev) pos0 = *pos_dev;  // position held on the device (graph-captured decode step)
   const int half = hd >> 1;
   const int pairs_per_row = ncols >> 1;
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -130,7 +132,9 @@ __global__ void rope_kernel(T* __restrict__ qk, int64_t ld, int ncols, int rows,
 // Only the last min(n, C) positions are written.
 template <typename T>
 __global__ void kv_append_kernel(const T* __restrict__ src, int64_t ld, int kcol, int vcol, int n, int B,
-                                 int64_t pos0, int d, T* __restrict__ ring_k, T* __restrict__ ring_v, int C) {
+                                 int64_t pos0, int d, T* __restrict__ ring_k, T* __restrict__ ring_v, int C,
+                                 const int64_t* pos_dev = nullptr) {
+  if (pos_dev) pos0 = *pos_dev;
   const int first = n > C ? n - C : 0;
   const int cnt = n - first;
   const int per_row = d / 8;  // 16-byte chunks (d % 8 == 0 for bf16; float path uses scalar loop)
@@ -278,6 +282,42 @@ __global__ void add_init_kernel(const T* __restrict__ init, const float* __restr
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) out[i] = to_f32(init[i]) + delta[i];
 }
+
+// ---------------------------------------------------------------- decode step helpers
+// The decode step runs as one captured CUDA graph per call; what changes from token
+// to token is read from the device: the absolute position *pos (advanced by
+// decode_advance_kernel at the end of the step) and the call's first position base.
+
+// pend_in[b][pos % bsz][:] = x[b][:] (input of the first adaptive block of this position)
+__global__ void pend_store_kernel(const float* __restrict__ x, int B, int d, float* __restrict__ pend_in, int bsz,
+                                  const int64_t* __restrict__ pos) {
+  const int64_t slot = *pos % bsz;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)B * d) return;
+  const int b = (int)(idx / d), c = (int)(idx % d);
+  pend_in[((int64_t)b * bsz + slot) * d + c] = x[idx];
+}
+
+// forced_col[b] = forced[b][t] with t = *pos - base (or -1 without forcing)
+__global__ void forced_gather_kernel(const int32_t* __restrict__ forced, int64_t n, int B, int32_t* forced_col,
+                                     const int64_t* __restrict__ pos, int64_t base) {
+  const int b = threadIdx.x;
+  if (b < B) forced_col[b] = forced[b * n + (*pos - base)];
+}
+
+// out_tok[b][t] = chosen[b]; out_loss[b][t] = loss[b]; pend_tgt[b][pos % bsz] = chosen[b]; t = *pos - base
+__global__ void decode_record_kernel(const int32_t* chosen, const float* loss, int B, int64_t n, int32_t* out_tok,
+                                     float* out_loss, int32_t* pend_tgt, int bsz, const int64_t* __restrict__ pos,
+                                     int64_t base) {
+  const int b = threadIdx.x;
+  if (b >= B) return;
+  const int64_t t = *pos - base;
+  out_tok[b * n + t] = chosen[b];
+  if (out_loss) out_loss[b * n + t] = loss[b];
+  pend_tgt[(int64_t)b * bsz + *pos % bsz] = chosen[b];
+}
+
+__global__ void decode_advance_kernel(int64_t* pos) { *pos += 1; }
 
 // Copy rows: dst[b][i][:] = src[b*src_bstride + (off + i)*ld ...] for i < n (fp32 rows of d).
 __global__ void gather_rows_kernel(const float* __restrict__ src, int64_t src_bstride, int64_t off, int n, int B,

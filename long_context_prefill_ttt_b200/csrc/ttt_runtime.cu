@@ -85,17 +85,30 @@ static cudaError_t launch_tc(const GemmParams& p, cudaStream_t st, int* err, int
   else tb2 = tb;
   if (!*ok) return cudaSuccess;
   using C = TcCfg<BN>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, AM, BM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
   const int tiles = ((p.M + TC_BM - 1) / TC_BM) * (p.N / BN) * p.batch;
   const int grid = tiles < num_sms ? tiles : num_sms;
   gemm_tc_kernel<BN, AM, BM><<<grid, TC_THREADS, C::SMEM, st>>>(ta, tb, tb2, p, err);
   return cudaGetLastError();
+}
+
+// Dynamic shared-memory limits of every large-smem kernel, set once per process
+// before any launch (and so never inside a CUDA graph capture).
+template <int BN, bool AM, bool BM> static cudaError_t tc_attr() {
+  return cudaFuncSetAttribute(gemm_tc_kernel<BN, AM, BM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              TcCfg<BN>::SMEM);
+}
+int prime_kernel_attributes() {
+  static int done = 0;
+  if (done) return 0;
+  cudaError_t e = cudaSuccess;
+  const cudaError_t r[] = {tc_attr<128, false, false>(), tc_attr<256, false, false>(), tc_attr<128, false, true>(),
+                           tc_attr<256, false, true>(),  tc_attr<128, true, true>(),   tc_attr<256, true, true>(),
+                           attn_mma_attributes<64>(),    attn_mma_attributes<128>()};
+  for (cudaError_t x : r)
+    if (x != cudaSuccess) e = x;
+  if (e != cudaSuccess) return (int)e;
+  done = 1;
+  return 0;
 }
 
 // Returns 0 on success, or a cudaError_t value.
@@ -304,6 +317,8 @@ template <typename T> class Engine : public ttt_handle {
   int32_t* chosen = nullptr; float* dec_loss = nullptr; float* dec_zmax = nullptr; int32_t* forced_col = nullptr;
   // per-call growable buffers
   int64_t chunk_pos = 0;                  // absolute position of row 0 of the chunk in the adaptive buffers
+  bool decode_mode = false;               // set while a decode token step is being captured
+  int64_t* pos_dev = nullptr;             // device copy of the position of the token being decoded
   int32_t* tok_dev = nullptr; int64_t tok_cap = 0;
   float* loss_dev = nullptr; int64_t loss_cap = 0;
   int32_t* otok_dev = nullptr; int64_t otok_cap = 0;
@@ -375,6 +390,7 @@ template <typename T> class Engine : public ttt_handle {
   int frozen_mlp(const LayerDev<T>& Lw, float* x, T* r, T* hid, int rows);
   int ttt_forward(int cn, int64_t pos, bool commit);
   int ttt_backward(int cn);
+  int decode_token_launches(int64_t n, int32_t* otok, float* oloss, const int32_t* fdev, int64_t base);
   int ttt_step(const float* in, const int32_t* targets, int cn, int64_t pos, float* loss_out, int64_t loss_ld,
                int64_t loss_off, bool grad, bool commit);
   int sync_and_check();
@@ -422,6 +438,7 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
   S = ((seg + bsz - 1) / bsz) * bsz;
   int dev = 0;
   TTT_CUDA(cudaGetDevice(&dev));
+  TTT_CUDA((cudaError_t)prime_kernel_attributes());
   TTT_CUDA(cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev));
 
   const int64_t Ms = (int64_t)B * S, Mc = (int64_t)B * bsz;
@@ -505,6 +522,7 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
   dec_loss = arena.get<float>(B);
   dec_zmax = arena.get<float>(B);
   forced_col = arena.get<int32_t>(B);
+  pos_dev = arena.get<int64_t>(1);
   if (arena.failed) {
     arena.release();
     return fail(this, TTT_ERR_OOM, "device allocation failed");
@@ -634,6 +652,23 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
   TTT_LAUNCHED();
   if ((rc = gemm(gp(rows, 3 * d, d, r, d, false, Lw.Wqkv, d, false, qkv, 3 * d, false, EPI_STORE))) != TTT_OK)
     return rc;
+  if (decode_mode) {
+    // one position per sequence, position on the device: append its K/V to the ring
+    // first, then attend over the window entirely from the ring
+    rope_kernel<T><<<nblk((int64_t)rows * d, 256), 256, 0, st>>>(qkv, 3 * d, 2 * d, rows, 1, 0, hd, rope_lo,
+                                                                  rope_hi, 0, pos_dev);
+    TTT_LAUNCHED();
+    const int64_t work = sizeof(T) == 2 ? (int64_t)B * (d / 8) : (int64_t)B * d;
+    kv_append_kernel<T><<<nblk(work, 256), 256, 0, st>>>(qkv, 3 * d, d, 2 * d, 1, B, 0, d, Lw.ring_k, Lw.ring_v, C,
+                                                         pos_dev);
+    TTT_LAUNCHED();
+    attn_decode_kernel<T><<<dim3(H, B), 256, 0, st>>>(qkv, 3 * d, Lw.ring_k, Lw.ring_v, C, d, hd, kwin, pos_dev,
+                                                      1.0f / sqrtf((float)hd), o, d);
+    TTT_LAUNCHED();
+    GemmParams pd = gp(rows, d, d, o, d, false, Lw.Wo, d, false, xout, d, true, EPI_RESID);
+    pd.X = xin; pd.ldx = d;
+    return gemm(pd);
+  }
   rope_kernel<T><<<nblk((int64_t)rows * d, 256), 256, 0, st>>>(qkv, 3 * d, 2 * d, rows, n, q0, hd, rope_lo, rope_hi,
                                                                 0);
   TTT_LAUNCHED();
@@ -906,13 +941,45 @@ template <typename T> int Engine<T>::prefill(const int32_t* tokens, int64_t T_, 
 }
 
 // ------------------------------------------------------------------ decode (Algorithm 3)
-__global__ void decode_record_kernel(const int32_t* chosen, const float* loss, int B, int64_t t, int64_t n,
-                                     int32_t* out_tok, float* out_loss, int32_t* pend_tgt, int bsz, int cnt) {
-  const int b = threadIdx.x;
-  if (b >= B) return;
-  out_tok[b * n + t] = chosen[b];
-  if (out_loss) out_loss[b * n + t] = loss[b];
-  pend_tgt[b * bsz + cnt] = chosen[b];
+// One generated token per sequence = one replay of a CUDA graph captured at the
+// start of the call: embedding of the pending id, every block for one position
+// (window attention read from the rings), LM head, greedy (or forced) choice,
+// bookkeeping, position advance. Every b decoded positions the completed chunk is
+// re-forwarded with W_{i-1}, differentiated and the fast weights updated.
+template <typename T> int Engine<T>::decode_token_launches(int64_t n, int32_t* otok, float* oloss, const int32_t* fdev,
+                                                           int64_t base) {
+  const int rows = B;
+  int rc;
+  embed_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(pend_tok_dev, 1, 0, 1, rows, E, V, d, xs, dev_err);
+  TTT_LAUNCHED();
+  gemm_class = PC_GEMM_FROZEN;
+  for (int l = 0; l < first_ttt; ++l) {
+    if ((rc = attention_block(layers[l], l, xs, xs, rs, nullptr, qkvs, os, nullptr, 1, 0, true)) != TTT_OK) return rc;
+    if ((rc = frozen_mlp(layers[l], xs, rs, hids, rows)) != TTT_OK) return rc;
+  }
+  // keep the first adaptive block's input of this position for the chunk's update
+  pend_store_kernel<<<nblk((int64_t)B * d, 256), 256, 0, st>>>(xs, B, d, pend_in, bsz, pos_dev);
+  TTT_LAUNCHED();
+  TTT_CUDA(cudaMemcpyAsync(blk[0].x, xs, (size_t)B * d * 4, cudaMemcpyDeviceToDevice, st));
+  gemm_class = PC_GEMM_TTT;
+  if ((rc = ttt_forward(1, 0, true)) != TTT_OK) return rc;
+  rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf);
+  TTT_LAUNCHED();
+  if ((rc = gemm(gp(rows, V, d, rf, d, false, E, d, false, z, V, false, EPI_STORE))) != TTT_OK) return rc;
+  const int32_t* fcol = nullptr;
+  if (fdev) {
+    forced_gather_kernel<<<1, 32 * ((B + 31) / 32), 0, st>>>(fdev, n, B, forced_col, pos_dev, base);
+    TTT_LAUNCHED();
+    fcol = forced_col;
+  }
+  argmax_kernel<T><<<rows, 256, 0, st>>>(z, V, fcol, pend_tok_dev, dec_loss, dec_zmax);
+  TTT_LAUNCHED();
+  decode_record_kernel<<<1, 32 * ((B + 31) / 32), 0, st>>>(pend_tok_dev, dec_loss, B, n, otok, oloss, pend_tgt, bsz,
+                                                           pos_dev, base);
+  TTT_LAUNCHED();
+  decode_advance_kernel<<<1, 1, 0, st>>>(pos_dev);
+  TTT_LAUNCHED();
+  return TTT_OK;
 }
 
 template <typename T>
@@ -925,63 +992,74 @@ int Engine<T>::decode(int64_t n, const int32_t* forced, int32_t* out_tok, float*
   int rc;
   int32_t* otok = out_tok;
   float* oloss = out_loss;
-  int32_t* fdev = nullptr;
+  const int32_t* fdev = nullptr;
   if ((rc = ensure((void**)&otok_dev, &otok_cap, (int64_t)B * n * 2, 4)) != TTT_OK) return rc;
   if ((rc = ensure((void**)&loss_dev, &loss_cap, (int64_t)B * n, 4)) != TTT_OK) return rc;
   if (kind == TTT_PTR_HOST) {
     otok = otok_dev;
     oloss = out_loss ? loss_dev : nullptr;
     if (forced) {
-      fdev = otok_dev + (int64_t)B * n;
-      TTT_CUDA(cudaMemcpyAsync(fdev, forced, (size_t)B * n * 4, cudaMemcpyHostToDevice, st));
+      int32_t* f = otok_dev + (int64_t)B * n;
+      TTT_CUDA(cudaMemcpyAsync(f, forced, (size_t)B * n * 4, cudaMemcpyHostToDevice, st));
+      fdev = f;
     }
   } else {
-    fdev = (int32_t*)forced;
+    fdev = forced;
   }
-  const int rows = B;
+  const int64_t base = n_pos;
+  TTT_CUDA(cudaMemcpyAsync(pos_dev, &base, sizeof(int64_t), cudaMemcpyHostToDevice, st));
+  TTT_CUDA(cudaStreamSynchronize(st));  // the source lives on the host stack
+  // capture one token step
+  const bool prof_on = prof.on;
+  prof.on = false;
+  decode_mode = true;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  TTT_CUDA(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
+  const int64_t before = launches;
+  rc = decode_token_launches(n, otok, oloss, fdev, base);
+  const int64_t per_token = launches - before;
+  cudaError_t ce = cudaStreamEndCapture(st, &graph);
+  decode_mode = false;
+  prof.on = prof_on;
+  if (rc != TTT_OK) {
+    if (graph) cudaGraphDestroy(graph);
+    return rc;
+  }
+  if (ce == cudaSuccess) ce = cudaGraphInstantiate(&exec, graph, 0);
+  if (graph) cudaGraphDestroy(graph);
+  if (ce != cudaSuccess) {
+    poisoned = true;
+    return fail(this, TTT_ERR_CUDA, std::string("decode graph: ") + cudaGetErrorString(ce));
+  }
+  launches = 0;
   for (int64_t t = 0; t < n; ++t) {
-    const int64_t p = n_pos;
-    embed_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(pend_tok_dev, 1, 0, 1, rows, E, V, d, xs, dev_err);
-    TTT_LAUNCHED();
-    for (int l = 0; l < first_ttt; ++l) {
-      if ((rc = attention_block(layers[l], l, xs, xs, rs, nullptr, qkvs, os, nullptr, 1, p, true)) != TTT_OK)
-        return rc;
-      if ((rc = frozen_mlp(layers[l], xs, rs, hids, rows)) != TTT_OK) return rc;
-    }
-    // keep the first adaptive block's input of this position for the chunk's update
-    gather_rows_kernel<<<nblk((int64_t)B * d, 256), 256, 0, st>>>(xs, d, 0, 1, B, d, pend_in, (int64_t)bsz * d,
-                                                                 pend_cnt);
-    TTT_LAUNCHED();
-    TTT_CUDA(cudaMemcpyAsync(blk[0].x, xs, (size_t)B * d * 4, cudaMemcpyDeviceToDevice, st));
-    chunk_pos = p;
-    if ((rc = ttt_forward(1, p, true)) != TTT_OK) return rc;
-    rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf);
-    TTT_LAUNCHED();
-    if ((rc = gemm(gp(rows, V, d, rf, d, false, E, d, false, z, V, false, EPI_STORE))) != TTT_OK) return rc;
-    const int32_t* fcol = nullptr;
-    if (fdev) {
-      gather_tokens_kernel<<<1, 256, 0, st>>>(fdev, n, t, 1, B, forced_col, 1, 0);
-      TTT_LAUNCHED();
-      fcol = forced_col;
-    }
-    argmax_kernel<T><<<rows, 256, 0, st>>>(z, V, fcol, pend_tok_dev, dec_loss, dec_zmax);
-    TTT_LAUNCHED();
-    decode_record_kernel<<<1, 32 * ((B + 31) / 32), 0, st>>>(pend_tok_dev, dec_loss, B, t, n, otok, oloss, pend_tgt,
-                                                             bsz, pend_cnt);
-    TTT_LAUNCHED();
+    ce = cudaGraphLaunch(exec, st);
+    if (ce != cudaSuccess) break;
+    launches += per_token;
     ++pend_cnt;
     ++n_pos;
     if (pend_cnt == bsz) {  // a full chunk of decoded positions: differentiate and update
-      if ((rc = ttt_step(pend_in, pend_tgt, bsz, n_pos - bsz, nullptr, 0, 0, true, false)) != TTT_OK) return rc;
+      if ((rc = ttt_step(pend_in, pend_tgt, bsz, n_pos - bsz, nullptr, 0, 0, true, false)) != TTT_OK) {
+        cudaGraphExecDestroy(exec);
+        return rc;
+      }
       pend_cnt = 0;
     }
+  }
+  if (ce != cudaSuccess) {
+    cudaGraphExecDestroy(exec);
+    poisoned = true;
+    return fail(this, TTT_ERR_CUDA, std::string("decode graph launch: ") + cudaGetErrorString(ce));
   }
   if (kind == TTT_PTR_HOST) {
     TTT_CUDA(cudaMemcpyAsync(out_tok, otok_dev, (size_t)B * n * 4, cudaMemcpyDeviceToHost, st));
     if (out_loss) TTT_CUDA(cudaMemcpyAsync(out_loss, loss_dev, (size_t)B * n * 4, cudaMemcpyDeviceToHost, st));
   }
   TTT_CUDA(cudaMemcpyAsync(pend_tok_host.data(), pend_tok_dev, (size_t)B * 4, cudaMemcpyDeviceToHost, st));
-  return sync_and_check();
+  rc = sync_and_check();
+  cudaGraphExecDestroy(exec);
+  return rc;
 }
 
 template <typename T> int Engine<T>::get_weights(int32_t seq, int32_t j, float* w1, float* w2, int32_t kind) {

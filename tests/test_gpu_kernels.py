@@ -63,7 +63,8 @@ def test_gemm_shared_plus_per_batch_operand(T, a_mn, b_mn, engine):
     T.ttt_k_status()
     small = A.double() @ B2.double().transpose(1, 2)
     err = (D.double() - ref).abs().max().item()
-    assert err < 1e-3 * small.abs().max().item(), (err, small.abs().max().item())
+    # fp32 accumulation of the large term leaves ~1e-5 absolute; losing B2 would leave |small| ~ 7e-2
+    assert err < 1e-2 * small.abs().max().item(), (err, small.abs().max().item())
 
 
 @pytest.mark.parametrize("M,N,K", [(256, 512, 256), (130, 256, 64)])
