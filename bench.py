@@ -238,7 +238,7 @@ def run_ours(args):
     loss_dev = torch.empty((cfg.batch, cfg.T), dtype=torch.float32, device=device)
     tok_host = torch.from_numpy(toks_np).pin_memory()
     loss_host = torch.empty((cfg.batch, cfg.T), dtype=torch.float32).pin_memory()
-    h = T.ttt_create(cfg, wd)
+    h = T.ttt_create(cfg, wd, max_segment=args.segment)
     del wd
     torch.cuda.synchronize()
 
@@ -309,6 +309,7 @@ def run_ours(args):
                                f"H{cfg.n_heads} h{cfg.mlp_hidden} ({cfg.ttt_hidden}+{cfg.static_hidden}) "
                                f"k{cfg.window_k} b{cfg.minibatch_b} T{cfg.T} B{cfg.batch}",
                    "tokens_per_step_per_gpu": cfg.batch * cfg.T, "parallelism": f"replicas x{ws}",
+                   "device_bytes": T.ttt_device_bytes(h),
                    "l2": "no flush: every step streams > 2.5 GB of weights and GBs of activations (L2 126 MB)"},
         "model_flops": {"tflop_per_step": flops_step / 1e12, "achieved_tflops": achieved_model,
                         "frac_of_peak": achieved_model / peaks["bf16"], "peak_tflops": peaks["bf16"],
@@ -346,6 +347,7 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD)
     ap.add_argument("--T", type=int, default=0, help="override positions per sequence (quick runs)")
     ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--segment", type=int, default=0, help="frozen-phase segment length (0 = library default)")
     ap.add_argument("--ref-tokens", type=int, default=1024)
     ap.add_argument("--no-decode", dest="decode", action="store_false")
     ap.add_argument("--decode-prefix", type=int, default=0)

@@ -28,10 +28,11 @@ extern "C" {
 enum { TTT_EPI_STORE = 0, TTT_EPI_RESID = 1, TTT_EPI_GELU = 2, TTT_EPI_DGELU = 3, TTT_EPI_SGD = 4 };
 
 /* Engines: 0 = automatic: GEMMs on tcgen05 tensor cores for bf16 shapes with N % 128 == 0 and
- * K % 64 == 0; attention on tensor cores (mma.sync m16n8k16) for bf16 with head dim 64 or 128 and
- * q0 % 64 == 0 (and C % 64 == 0); otherwise, and for fp32, SIMT FFMA kernels.
- * 1 = SIMT only. */
-enum { TTT_ENGINE_AUTO = 0, TTT_ENGINE_SIMT = 1 };
+ * K % 64 == 0; attention forward on tcgen05 for bf16 with head dim 64 or 128, q0 % 128 == 0 and
+ * C % 128 == 0; attention on warp-level tensor cores (mma.sync m16n8k16) for bf16 with head dim
+ * 64 or 128 and q0 % 64 == 0 (and C % 64 == 0); otherwise, and for fp32, SIMT FFMA kernels.
+ * 1 = SIMT only. 2 = attention on the mma.sync kernels (tests compare engines). */
+enum { TTT_ENGINE_AUTO = 0, TTT_ENGINE_SIMT = 1, TTT_ENGINE_MMA = 2 };
 
 /* Batched GEMM D[z][m][n] = epilogue(alpha * sum_k A[z](m,k) * (B[z](n,k) + B2[z](n,k))).
  * A(m,k) = a_mn ? A[k*lda + m] : A[m*lda + k]   (batch stride sA elements)

@@ -1,0 +1,274 @@
+// Sliding-window attention forward on tcgen05 tensor cores (bf16 in, fp32 softmax
+// and accumulation), for the frozen-phase prefill and the adaptive chunks.
+//
+// One CTA = 128 queries of one (sequence, head); key tiles of 128 positions,
+// 128-aligned in absolute position, each taken whole from the ring (positions
+// < q0) or from the current rows (the q|k|v buffer). Warp roles:
+//   warp 0     TMA: Q once, then K and V tiles into a 2-stage ring;
+//   warp 1     MMA issue (one thread): S_j = Q K_j^T into one of two TMEM S
+//              buffers, then O += P_{j-1} V_{j-1} (P from shared memory, V as an
+//              MN-major operand) into the TMEM O accumulator;
+//   warps 2-5  softmax, one thread per query row (TMEM lane): read S_j, mask on
+//              diagonal / window-edge tiles, online softmax in the log2 domain,
+//              write P_j (bf16) to shared memory in the 128-byte-swizzled layout
+//              the MMA reads. The running maximum is raised only when a row's
+//              maximum grows by more than 8 (a factor 256): then the thread's O
+//              row is rescaled in TMEM after the previous P·V has completed.
+//              Exponents stay below 2^8, so bf16 P and fp32 sums stay exact
+//              enough, and O and l always share the same reference maximum.
+// TMEM: S0 columns [0,128), S1 [128,256), O [256, 256+HD); 512 allocated.
+// Every mbarrier wait is time-bounded and records an error instead of hanging.
+#pragma once
+
+#include "ttt_attention.cuh"
+#include "ttt_common.cuh"
+
+namespace ttt {
+
+template <int HD> struct AttnTcCfg {
+  static constexpr int BM = 128, BN = 128;
+  static constexpr int QB = BM * HD * 2;      // Q tile bytes
+  static constexpr int KVB = BN * HD * 2;     // K (and V) tile bytes
+  static constexpr int PB = BM * BN * 2;      // P tile bytes
+  static constexpr int OFF_K0 = QB;
+  static constexpr int OFF_P0 = QB + 2 * 2 * KVB;
+  static constexpr int OFF_BAR = OFF_P0 + 2 * PB;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr uint32_t S_COL = 0, O_COL = 256;
+};
+
+__device__ __forceinline__ bool warp_any(bool v) { return __any_sync(0xffffffffu, v); }
+__device__ __forceinline__ float ex2_tc(float x) {
+  float y;
+  asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <int HD>
+__global__ void __launch_bounds__(192, 1)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_rk,
+                       const __grid_constant__ CUtensorMap tm_rv, const AttnParams p, int* err) {
+  using Cf = AttnTcCfg<HD>;
+  constexpr int KB = HD / 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = (uint64_t*)(sm + Cf::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;    // [2]
+  uint64_t* kv_empty = bars + 3;   // [2]
+  uint64_t* s_full = bars + 5;     // [2]
+  uint64_t* s_free = bars + 7;     // [2]
+  uint64_t* p_full = bars + 9;     // [2]
+  uint64_t* pv_done = bars + 11;   // [2]
+  uint64_t* o_done = bars + 13;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 14);
+
+  const int warp = threadIdx.x >> 5;
+  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int i0 = qb * Cf::BM;
+  const int64_t P0 = p.q0 + i0;
+  const int nq = min(Cf::BM, p.n - i0);
+  const int64_t Plast = P0 + nq - 1;
+  const int64_t jlo = max((int64_t)0, P0 - p.window + 1);
+  const int64_t jt0 = (jlo / Cf::BN) * Cf::BN;
+  const int ntiles = (int)((Plast / Cf::BN) * Cf::BN - jt0) / Cf::BN + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1);
+      mbar_init(&s_full[s], 1);  mbar_init(&s_free[s], 4);
+      mbar_init(&p_full[s], 4);  mbar_init(&pv_done[s], 1);
+    }
+    mbar_init(o_done, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tm_qkv);
+    prefetch_tmap(&tm_rk);
+    prefetch_tmap(&tm_rv);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (elect_lane0()) {
+      const int qrow = b * p.n + i0;
+      mbar_arrive_expect_tx(q_full, Cf::QB);
+      for (int kb = 0; kb < KB; ++kb) tma_load_3d(sm + kb * Cf::BM * 128, &tm_qkv, q_full, h * HD + kb * 64, qrow, 0);
+      for (int j = 0; j < ntiles; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(&kv_empty[s], ((j >> 1) & 1) ^ 1, err, DEV_TIMEOUT_EMPTY)) break;
+        uint8_t* sk = sm + Cf::OFF_K0 + s * 2 * Cf::KVB;
+        uint8_t* sv = sk + Cf::KVB;
+        mbar_arrive_expect_tx(&kv_full[s], 2 * Cf::KVB);
+        const int64_t j0 = jt0 + (int64_t)j * Cf::BN;
+        if (j0 >= p.q0) {
+          const int y = b * p.n + (int)(j0 - p.q0);
+          for (int kb = 0; kb < KB; ++kb) {
+            tma_load_3d(sk + kb * Cf::BN * 128, &tm_qkv, &kv_full[s], p.d + h * HD + kb * 64, y, 0);
+            tma_load_3d(sv + kb * Cf::BN * 128, &tm_qkv, &kv_full[s], 2 * p.d + h * HD + kb * 64, y, 0);
+          }
+        } else {
+          const int y = b * p.C + (int)(j0 % p.C);
+          for (int kb = 0; kb < KB; ++kb) {
+            tma_load_3d(sk + kb * Cf::BN * 128, &tm_rk, &kv_full[s], h * HD + kb * 64, y, 0);
+            tma_load_3d(sv + kb * Cf::BN * 128, &tm_rv, &kv_full[s], h * HD + kb * 64, y, 0);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_lane0()) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, Cf::BN, false, false);
+      constexpr uint32_t idO = idesc_bf16_f32(128, HD, false, true);
+      const uint32_t sQ = smem_u32(sm);
+      bool ok = mbar_wait(q_full, 0, err, DEV_TIMEOUT_FULL);
+      auto issue_pv = [&](int i) -> bool {
+        const int s = i & 1;
+        if (!mbar_wait(&p_full[s], (i >> 1) & 1, err, DEV_TIMEOUT_FULL)) return false;
+        tc_fence_after();
+        const uint32_t sP = smem_u32(sm + Cf::OFF_P0 + s * Cf::PB);
+        const uint32_t sV = smem_u32(sm + Cf::OFF_K0 + s * 2 * Cf::KVB + Cf::KVB);
+#pragma unroll
+        for (int kk = 0; kk < Cf::BN / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(sP + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sV + kk * 2048, Cf::BN * 128, 1024);
+          tc_mma_f16(tmem + Cf::O_COL, ad, bd, idO, (i | kk) ? 1u : 0u);
+        }
+        tc_commit(&pv_done[s]);
+        tc_commit(&kv_empty[s]);
+        return true;
+      };
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const int s = j & 1;
+        if (!mbar_wait(&kv_full[s], (j >> 1) & 1, err, DEV_TIMEOUT_FULL)) { ok = false; break; }
+        if (!mbar_wait(&s_free[s], ((j >> 1) & 1) ^ 1, err, DEV_TIMEOUT_ACC)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sK = smem_u32(sm + Cf::OFF_K0 + s * 2 * Cf::KVB);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(sQ + (kk >> 2) * (Cf::BM * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sK + (kk >> 2) * (Cf::BN * 128) + (kk & 3) * 32, 16, 1024);
+          tc_mma_f16(tmem + Cf::S_COL + s * Cf::BN, ad, bd, idS, kk ? 1u : 0u);
+        }
+        tc_commit(&s_full[s]);
+        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok) ok = issue_pv(ntiles - 1);
+      if (ok) tc_commit(o_done);
+    }
+  } else {
+    // softmax warps: TMEM lane quarter = warp % 4, one query row per thread
+    const int quarter = warp & 3;
+    const int lane = threadIdx.x & 31;
+    const int r = quarter * 32 + lane;
+    const int64_t P = P0 + r;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const float sc = p.scale * 1.4426950408889634f;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int s = j & 1;
+      const int64_t j0 = jt0 + (int64_t)j * Cf::BN;
+      if (!mbar_wait(&s_full[s], (j >> 1) & 1, err, DEV_TIMEOUT_ACC)) { ok = false; break; }
+      tc_fence_after();
+      float v[Cf::BN];
+#pragma unroll
+      for (int c = 0; c < Cf::BN / 32; ++c) tmem_ld32(tmem + lane_base + Cf::S_COL + s * Cf::BN + c * 32, v + c * 32);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[s]);
+      const bool need_mask = (j0 + Cf::BN - 1 > P0) || (j0 < Plast - p.window + 1);
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < Cf::BN; ++c) {
+        float x = v[c] * sc;
+        if (need_mask) {
+          const int64_t key = j0 + c;
+          if (key > P || key < P - p.window + 1) x = -INFINITY;
+        }
+        v[c] = x;
+        mt = fmaxf(mt, x);
+      }
+      // lazily raised reference maximum
+      const bool first = m_used == -INFINITY;
+      const bool raise = mt > m_used + 8.f;
+      float factor = 1.f;
+      if (raise) {
+        if (!first) factor = ex2_tc(m_used - mt);
+        m_used = mt;
+      }
+      if (j >= 1 && warp_any(raise && !first)) {
+        // O holds P_0..P_{j-1} V: wait for the last of them, then rescale this warp's rows
+        if (!mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, err, DEV_TIMEOUT_ACC)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < HD / 32; ++c) {
+          float o[32];
+          tmem_ld32(tmem + lane_base + Cf::O_COL + c * 32, o);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] *= factor;
+          tmem_st32(tmem + lane_base + Cf::O_COL + c * 32, o);
+        }
+      }
+      l *= factor;
+      // the P buffer s was last read by P_{j-2} V_{j-2}
+      if (j >= 2 && !mbar_wait(&pv_done[s], ((j - 2) >> 1) & 1, err, DEV_TIMEOUT_ACC)) { ok = false; break; }
+      const float base = m_used == -INFINITY ? 0.f : m_used;
+      uint8_t* prow = sm + Cf::OFF_P0 + s * Cf::PB + r * 128;
+      float lsum = 0.f;
+#pragma unroll
+      for (int kb = 0; kb < Cf::BN / 64; ++kb) {
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          float e8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            e8[e] = ex2_tc(v[kb * 64 + cc * 8 + e] - base);
+            lsum += e8[e];
+          }
+          const uint4 pk = make_uint4(pack_bf16x2(e8[0], e8[1]), pack_bf16x2(e8[2], e8[3]),
+                                      pack_bf16x2(e8[4], e8[5]), pack_bf16x2(e8[6], e8[7]));
+          *(uint4*)(prow + kb * (Cf::BM * 128) + ((cc ^ (r & 7)) << 4)) = pk;
+        }
+      }
+      l += lsum;
+      fence_proxy_async();  // P (generic-proxy stores) visible to the tensor core
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[s]);
+    }
+    if (ok && mbar_wait(o_done, 0, err, DEV_TIMEOUT_ACC)) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      bf16* O = (bf16*)p.O + ((int64_t)b * p.n + i0 + r) * p.ldo + h * HD;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        float o[32];
+        tmem_ld32(tmem + lane_base + Cf::O_COL + c * 32, o);
+        if (r < nq) {
+          uint4* dst = (uint4*)(O + c * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv), pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+        }
+      }
+      if (r < nq && p.lse) p.lse[((int64_t)b * p.H + h) * p.n + i0 + r] = (m_used + __log2f(l)) * 0.6931471805599453f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace ttt

@@ -369,5 +369,8 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t stream, int*
                 int force_simt);
 // Sets the dynamic shared-memory limits of all large-smem kernels; 0 or a cudaError_t.
 int prime_kernel_attributes();
+struct AttnParams;
+bool attn_tc_ok(const AttnParams& p);
+cudaError_t attn_fwd_tc_launch(const AttnParams& p, cudaStream_t st, int* err, bool* ok);
 
 }  // namespace ttt

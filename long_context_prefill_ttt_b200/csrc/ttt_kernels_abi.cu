@@ -34,6 +34,13 @@ template <typename T>
 static int attn_fwd(const AttnParams& ap, int engine, cudaStream_t st) {
   if (prime_kernel_attributes() != 0) return TTT_ERR_CUDA;
   const int64_t rows = (int64_t)ap.B * ap.n;
+  if (sizeof(T) == 2 && engine == TTT_ENGINE_AUTO && attn_tc_ok(ap)) {
+    int* err = status_word();
+    bool ok = false;
+    const cudaError_t e = attn_fwd_tc_launch(ap, st, err, &ok);
+    if (e != cudaSuccess) return TTT_ERR_CUDA;
+    if (ok) return TTT_OK;
+  }
   if (sizeof(T) == 2 && engine != TTT_ENGINE_SIMT && attn_mma_ok(ap)) {
     const cudaError_t e = ap.hd == 128 ? attn_fwd_mma_launch<128>(ap, st) : attn_fwd_mma_launch<64>(ap, st);
     return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;

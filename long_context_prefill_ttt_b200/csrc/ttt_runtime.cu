@@ -24,6 +24,7 @@
 #include "ttt.h"
 #include "ttt_attention.cuh"
 #include "ttt_attention_mma.cuh"
+#include "ttt_attention_tc.cuh"
 #include "ttt_common.cuh"
 #include "ttt_gemm.cuh"
 #include "ttt_ops.cuh"
@@ -91,6 +92,44 @@ static cudaError_t launch_tc(const GemmParams& p, cudaStream_t st, int* err, int
   return cudaGetLastError();
 }
 
+// ============================================================== tcgen05 attention (host)
+bool attn_tc_ok(const AttnParams& p) {
+  return (p.hd == 64 || p.hd == 128) && p.q0 % 128 == 0 && (p.q0 == 0 || p.C % 128 == 0) && p.d % 64 == 0 &&
+         p.ldq == 3 * p.d && p.ldkv == 3 * p.d && (const char*)p.K == (const char*)p.Q + 2 * p.d &&
+         aligned16(p.Q) && (p.q0 == 0 || (aligned16(p.Kc) && aligned16(p.Vc))) && p.n >= 1;
+}
+
+// Rows of 'inner' bf16 elements, 'rows' rows, box {64, 128}, 128-byte swizzle.
+static bool make_rows_map(CUtensorMap* map, const void* base, int64_t inner, int64_t rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)(inner * rows * 2)};
+  cuuint32_t box[3] = {64, 128, 1}, estr[3] = {1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Returns cudaSuccess and sets *ok = false when the maps cannot be built (caller falls back).
+cudaError_t attn_fwd_tc_launch(const AttnParams& p, cudaStream_t st, int* err, bool* ok) {
+  CUtensorMap tq, tk, tv;
+  *ok = make_rows_map(&tq, p.Q, 3 * p.d, (int64_t)p.B * p.n);
+  if (*ok && p.q0 > 0) {
+    *ok = make_rows_map(&tk, p.Kc, p.d, (int64_t)p.B * p.C) && make_rows_map(&tv, p.Vc, p.d, (int64_t)p.B * p.C);
+  } else {
+    tk = tq;
+    tv = tq;
+  }
+  if (!*ok) return cudaSuccess;
+  dim3 grid((p.n + 127) / 128, p.H, p.B);
+  if (p.hd == 128)
+    attn_fwd_tc_kernel<128><<<grid, 192, AttnTcCfg<128>::SMEM, st>>>(tq, tk, tv, p, err);
+  else
+    attn_fwd_tc_kernel<64><<<grid, 192, AttnTcCfg<64>::SMEM, st>>>(tq, tk, tv, p, err);
+  return cudaGetLastError();
+}
+
 // Dynamic shared-memory limits of every large-smem kernel, set once per process
 // before any launch (and so never inside a CUDA graph capture).
 template <int BN, bool AM, bool BM> static cudaError_t tc_attr() {
@@ -103,7 +142,11 @@ int prime_kernel_attributes() {
   cudaError_t e = cudaSuccess;
   const cudaError_t r[] = {tc_attr<128, false, false>(), tc_attr<256, false, false>(), tc_attr<128, false, true>(),
                            tc_attr<256, false, true>(),  tc_attr<128, true, true>(),   tc_attr<256, true, true>(),
-                           attn_mma_attributes<64>(),    attn_mma_attributes<128>()};
+                           attn_mma_attributes<64>(),    attn_mma_attributes<128>(),
+                           cudaFuncSetAttribute(attn_fwd_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                AttnTcCfg<64>::SMEM),
+                           cudaFuncSetAttribute(attn_fwd_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                AttnTcCfg<128>::SMEM)};
   for (cudaError_t x : r)
     if (x != cudaSuccess) e = x;
   if (e != cudaSuccess) return (int)e;
@@ -318,6 +361,8 @@ template <typename T> class Engine : public ttt_handle {
   // per-call growable buffers
   int64_t chunk_pos = 0;                  // absolute position of row 0 of the chunk in the adaptive buffers
   bool decode_mode = false;               // set while a decode token step is being captured
+  cudaStream_t cap_st = nullptr;          // private stream the decode step is captured on (the caller's
+                                          // stream may be the legacy default stream, which cannot capture)
   int64_t* pos_dev = nullptr;             // device copy of the position of the token being decoded
   int32_t* tok_dev = nullptr; int64_t tok_cap = 0;
   float* loss_dev = nullptr; int64_t loss_cap = 0;
@@ -327,6 +372,7 @@ template <typename T> class Engine : public ttt_handle {
 
   ~Engine() override {
     if (st) cudaStreamSynchronize(st);
+    if (cap_st) cudaStreamDestroy(cap_st);
     call_arena.release();
     arena.release();
   }
@@ -439,6 +485,7 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
   int dev = 0;
   TTT_CUDA(cudaGetDevice(&dev));
   TTT_CUDA((cudaError_t)prime_kernel_attributes());
+  TTT_CUDA(cudaStreamCreateWithFlags(&cap_st, cudaStreamNonBlocking));
   TTT_CUDA(cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev));
 
   const int64_t Ms = (int64_t)B * S, Mc = (int64_t)B * bsz;
@@ -679,11 +726,21 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
   ap.Kc = Lw.ring_k; ap.Vc = Lw.ring_v; ap.C = C;
   ap.O = o; ap.ldo = d; ap.lse = lse; ap.scale = 1.0f / sqrtf((float)hd);
   prof.begin(st, PC_ATTN_FWD, 4.0 * hd * H * (double)B * attn_pairs(n, q0), 0.0);
-  if (is_bf16 && attn_mma_ok(ap)) {
-    const cudaError_t e = hd == 128 ? attn_fwd_mma_launch<128>(ap, st) : attn_fwd_mma_launch<64>(ap, st);
-    (void)e;
-  } else {
-    attn_fwd_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
+  bool done = false;
+  if (is_bf16 && attn_tc_ok(ap)) {
+    const cudaError_t e = attn_fwd_tc_launch(ap, st, dev_err, &done);
+    if (e != cudaSuccess) {
+      poisoned = true;
+      return fail(this, TTT_ERR_CUDA, std::string("attention: ") + cudaGetErrorString(e));
+    }
+  }
+  if (!done) {
+    if (is_bf16 && attn_mma_ok(ap)) {
+      const cudaError_t e = hd == 128 ? attn_fwd_mma_launch<128>(ap, st) : attn_fwd_mma_launch<64>(ap, st);
+      (void)e;
+    } else {
+      attn_fwd_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
+    }
   }
   prof.end(st);
   TTT_LAUNCHED();
@@ -1015,11 +1072,21 @@ int Engine<T>::decode(int64_t n, const int32_t* forced, int32_t* out_tok, float*
   decode_mode = true;
   cudaGraph_t graph = nullptr;
   cudaGraphExec_t exec = nullptr;
-  TTT_CUDA(cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal));
+  cudaStream_t user_st = st;
+  st = cap_st;  // capture only records: nothing runs on cap_st; the graph runs on the caller's stream
+  cudaError_t ce = cudaStreamBeginCapture(st, cudaStreamCaptureModeThreadLocal);
+  if (ce != cudaSuccess) {
+    st = user_st;
+    decode_mode = false;
+    prof.on = prof_on;
+    poisoned = true;
+    return fail(this, TTT_ERR_CUDA, std::string("decode capture: ") + cudaGetErrorString(ce));
+  }
   const int64_t before = launches;
   rc = decode_token_launches(n, otok, oloss, fdev, base);
   const int64_t per_token = launches - before;
-  cudaError_t ce = cudaStreamEndCapture(st, &graph);
+  ce = cudaStreamEndCapture(st, &graph);
+  st = user_st;
   decode_mode = false;
   prof.on = prof_on;
   if (rc != TTT_OK) {

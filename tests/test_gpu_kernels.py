@@ -151,10 +151,12 @@ ATTN_CASES = [
     # tensor-core engine for bf16 (q0 % 64 == 0): ragged rows, windows off the tile grid, window < tile
     (2, 2, 64, 96, 128, 128, 256), (1, 2, 128, 200, 256, 300, 640), (2, 3, 128, 64, 0, 64, 128),
     (1, 2, 64, 130, 64, 40, 128), (1, 1, 128, 256, 1024, 1024, 2048),
+    # tcgen05 forward (q0 % 128 == 0, C % 128 == 0): many ring tiles, partial last query tile
+    (2, 2, 128, 384, 512, 700, 1280), (1, 4, 64, 300, 1024, 1000, 2048),
 ]
 
 
-@pytest.mark.parametrize("engine", [0, 1])
+@pytest.mark.parametrize("engine", [0, 1, 2])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("B,H,hd,n,q0,window,C", ATTN_CASES)
 def test_attention_forward_and_backward(T, engine, dtype, B, H, hd, n, q0, window, C):
