@@ -66,6 +66,24 @@ int ttt_k_attention_bwd(int32_t elem_dtype, int32_t B, int32_t H, int32_t hd, in
                         const void* out, const float* lse, const void* dout, void* dqkv, float* dsum,
                         int32_t engine, void* stream);
 
+/* Same as ttt_k_attention_bwd without the dsum argument, for callers that may not
+ * allocate device memory: for example a host application that reserved the GPU's
+ * memory for its own pool and hands this code only pointers, or a latency-bound
+ * thread that must not call cudaMalloc, which can block and synchronise the device.
+ * This entry point allocates nothing. Its scratch (one float per sequence, head and
+ * row) is a fixed 4 MiB array inside the library that every GPU loading the library
+ * keeps until exit. Limit: B*H*n <= 1048576, else TTT_ERR_INVALID_ARG.
+ * The first call on each device looks up that array's device address
+ * (cudaGetSymbolAddress) with the device current; make that first call before
+ * any stream capture. All calls share the one array: calls whose work overlaps on
+ * the GPU (other streams, other host threads) race on it and must be serialised by
+ * the caller. Nothing in it needs clearing: each call writes every element it reads.
+ * The pages have no counterpart of this entry point: it is an interface variant. */
+int ttt_k_attention_bwd_noalloc(int32_t elem_dtype, int32_t B, int32_t H, int32_t hd, int32_t n, int64_t q0,
+                                int32_t window, const void* qkv, const void* ring_k, const void* ring_v, int32_t C,
+                                const void* out, const float* lse, const void* dout, void* dqkv, int32_t engine,
+                                void* stream);
+
 /* Synchronise `stream` and return TTT_OK, TTT_ERR_CUDA or TTT_ERR_TIMEOUT (a
  * bounded device wait expired). Clears the device status word. */
 int ttt_k_status(void* stream);

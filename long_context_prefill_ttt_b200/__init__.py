@@ -75,6 +75,8 @@ def _load():
         "ttt_k_attention_fwd": (ctypes.c_int, [I32, I32, I32, I32, I32, I64, I32, VP, VP, VP, I32, VP, VP, I32, VP]),
         "ttt_k_attention_bwd": (ctypes.c_int, [I32, I32, I32, I32, I32, I64, I32, VP, VP, VP, I32, VP, VP, VP, VP,
                                                VP, I32, VP]),
+        "ttt_k_attention_bwd_noalloc": (ctypes.c_int, [I32, I32, I32, I32, I32, I64, I32, VP, VP, VP, I32, VP, VP,
+                                                       VP, VP, I32, VP]),
         "ttt_k_status": (ctypes.c_int, [VP]),
     }
     for name, (res, args) in sigs.items():
@@ -342,6 +344,18 @@ def ttt_k_attention_bwd(qkv, out, lse, dout, dqkv, dsum, B, H, hd, n, q0, window
                                  _stream_ptr(stream))
     if rc != TTT_OK:
         raise TTTError(rc, "ttt_k_attention_bwd")
+
+
+def ttt_k_attention_bwd_noalloc(qkv, out, lse, dout, dqkv, B, H, hd, n, q0, window, ring_k=None, ring_v=None, C=0,
+                                engine=ENGINE_AUTO, stream=None):
+    """Attention backward that allocates nothing (its scratch is a fixed array inside the library)."""
+    rc = lib.ttt_k_attention_bwd_noalloc(_dtype_code(qkv), B, H, hd, n, q0, window, qkv.data_ptr(),
+                                         ring_k.data_ptr() if ring_k is not None else None,
+                                         ring_v.data_ptr() if ring_v is not None else None, C, out.data_ptr(),
+                                         lse.data_ptr(), dout.data_ptr(), dqkv.data_ptr(), engine,
+                                         _stream_ptr(stream))
+    if rc != TTT_OK:
+        raise TTTError(rc, "ttt_k_attention_bwd_noalloc")
 
 
 def ttt_k_status(stream=None):

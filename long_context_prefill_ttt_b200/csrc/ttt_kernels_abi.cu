@@ -2,6 +2,7 @@
 // pass at a time, on caller-provided device buffers.
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "ttt.h"
 #include "ttt_attention.cuh"
@@ -79,6 +80,40 @@ static AttnParams attn_params(int B, int H, int hd, int n, int64_t q0, int windo
   return ap;
 }
 
+// ---------------------------------------------------------------- allocation-free backward
+// Scratch of ttt_k_attention_bwd_noalloc: the per-row sums D = rowsum(dO * O),
+// one float per (sequence, head, row). It lives in this library's own device
+// image, so every GPU that loads the library holds these 4 MiB until the process
+// exits, and no call ever allocates. The host must not pass the symbol itself to
+// a kernel (in host code it names a host-side stand-in); it passes the device
+// address that cudaGetSymbolAddress returns for the current device.
+constexpr int64_t kNoAllocDsumFloats = int64_t(1) << 20;
+static __device__ __align__(256) float g_noalloc_dsum[kNoAllocDsumFloats];
+
+// Device address of g_noalloc_dsum on the current device, looked up once per device.
+static float* noalloc_dsum_ptr(int* rc) {
+  static std::mutex mu;
+  static float* ptrs[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    *rc = TTT_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_dsum) != cudaSuccess || !p) {
+      cudaGetLastError();
+      *rc = TTT_ERR_CUDA;
+      return nullptr;
+    }
+    ptrs[dev] = (float*)p;
+  }
+  *rc = TTT_OK;
+  return ptrs[dev];
+}
+
 }  // namespace ttt
 
 using namespace ttt;
@@ -128,6 +163,31 @@ int ttt_k_attention_bwd(int32_t elem_dtype, int32_t B, int32_t H, int32_t hd, in
   if (B < 1 || H < 1 || hd < 2 || hd > 128 || n < 1 || window < 1 || !qkv || !out || !lse || !dout || !dqkv || !dsum)
     return TTT_ERR_INVALID_ARG;
   if (q0 > 0 && (!ring_k || !ring_v || C < window)) return TTT_ERR_INVALID_ARG;
+  const size_t esz = elem_dtype == TTT_BF16 ? 2 : 4;
+  AttnParams ap = attn_params(B, H, hd, n, q0, window, qkv, esz, ring_k, ring_v, C, const_cast<void*>(out),
+                              const_cast<float*>(lse));
+  const int d = H * hd;
+  ap.dO = dout; ap.lddo = d; ap.Dsum = dsum;
+  ap.dQ = dqkv;
+  ap.dK = (char*)dqkv + (size_t)d * esz;
+  ap.dV = (char*)dqkv + (size_t)2 * d * esz;
+  ap.lddq = 3 * d;
+  if (elem_dtype == TTT_BF16) return attn_bwd<bf16>(ap, engine, (cudaStream_t)stream);
+  return attn_bwd<float>(ap, engine, (cudaStream_t)stream);
+}
+
+int ttt_k_attention_bwd_noalloc(int32_t elem_dtype, int32_t B, int32_t H, int32_t hd, int32_t n, int64_t q0,
+                                int32_t window, const void* qkv, const void* ring_k, const void* ring_v, int32_t C,
+                                const void* out, const float* lse, const void* dout, void* dqkv, int32_t engine,
+                                void* stream) {
+  if (B < 1 || H < 1 || hd < 2 || hd > 128 || n < 1 || window < 1 || !qkv || !out || !lse || !dout || !dqkv)
+    return TTT_ERR_INVALID_ARG;
+  if (q0 > 0 && (!ring_k || !ring_v || C < window)) return TTT_ERR_INVALID_ARG;
+  if ((int64_t)B * H * n > kNoAllocDsumFloats) return TTT_ERR_INVALID_ARG;  // B*H*n above the fixed scratch
+  int rc = TTT_OK;
+  float* dsum = noalloc_dsum_ptr(&rc);
+  if (!dsum) return rc;
+  // Nothing needs clearing: the first kernel of the call writes every D it later reads.
   const size_t esz = elem_dtype == TTT_BF16 ? 2 : 4;
   AttnParams ap = attn_params(B, H, hd, n, q0, window, qkv, esz, ring_k, ring_v, C, const_cast<void*>(out),
                               const_cast<float*>(lse));
