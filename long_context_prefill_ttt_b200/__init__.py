@@ -171,9 +171,10 @@ class Handle:
         if rc != TTT_OK:
             raise TTTError(rc, self.error())
 
-    def __del__(self):
-        if getattr(self, "ptr", None):
-            lib.ttt_destroy(self.ptr)
+    def __del__(self, _lib=lib):
+        # _lib is bound at class creation: module globals may already be gone at interpreter exit
+        if getattr(self, "ptr", None) and _lib is not None:
+            _lib.ttt_destroy(self.ptr)
             self.ptr = None
 
 

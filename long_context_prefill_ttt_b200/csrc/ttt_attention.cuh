@@ -230,76 +230,105 @@ __global__ void __launch_bounds__(128) attn_bwd_dkv_simt_kernel(AttnParams p) {
 // ---------------------------------------------------------------- decode (one query)
 // One query per sequence at position P = *pos (the token's own K/V already in the
 // ring); keys [max(0, P-k+1), P] all read from the ring. One CTA per (head,
-// sequence), 8 warps splitting the window, lanes over keys for the scores and over
-// head dims for P·V, merged across warps at the end. HBM-bound: each key and value
-// row of the window is read once.
-template <typename T>
+// sequence), 8 warps splitting the window: lanes over keys for the scores (each
+// key row read with 16-byte loads issued together), lanes over head dims for P·V,
+// merged across warps at the end. HBM-bound: each K and V row of the window is
+// read once.
+template <typename T> __device__ __forceinline__ void load_row_f32(const T* src, float* dst, int n);
+template <> __device__ __forceinline__ void load_row_f32<bf16>(const bf16* src, float* dst, int n) {
+  for (int v = 0; v < n / 8; ++v) {
+    const uint4 u = reinterpret_cast<const uint4*>(src)[v];
+    const bf16* e = reinterpret_cast<const bf16*>(&u);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) dst[v * 8 + k] = __bfloat162float(e[k]);
+  }
+}
+template <> __device__ __forceinline__ void load_row_f32<float>(const float* src, float* dst, int n) {
+  for (int v = 0; v < n / 4; ++v) {
+    const float4 u = reinterpret_cast<const float4*>(src)[v];
+    dst[v * 4] = u.x; dst[v * 4 + 1] = u.y; dst[v * 4 + 2] = u.z; dst[v * 4 + 3] = u.w;
+  }
+}
+
+template <typename T, int HD>
 __global__ void __launch_bounds__(256) attn_decode_kernel(const T* __restrict__ q, int64_t ldq,
                                                           const T* __restrict__ ring_k, const T* __restrict__ ring_v,
-                                                          int C, int d, int hd, int window,
-                                                          const int64_t* __restrict__ pos, float scale,
-                                                          T* __restrict__ out, int64_t ldo) {
-  __shared__ float qs[128];
+                                                          int C, int d, int window, const int64_t* __restrict__ pos,
+                                                          float scale, T* __restrict__ out, int64_t ldo) {
+  // Each lane owns one key per step: its K row gives the score, its V row is
+  // accumulated into the lane's partial output (all row loads independent); the
+  // 32 partial outputs of a warp are summed once at the end.
+  constexpr int CH = HD < 32 ? HD : (HD == 128 ? 16 : 32);  // row chunk held in registers
+  __shared__ float qs[HD];
   __shared__ float wm[8], wl[8];
-  __shared__ float wo[8][128];
+  __shared__ float wo[8][HD];
   const int h = blockIdx.x, b = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t P = *pos;
   const int64_t lo = P - window + 1 > 0 ? P - window + 1 : 0;
-  for (int c = threadIdx.x; c < hd; c += 256) qs[c] = to_f32(q[(int64_t)b * ldq + h * hd + c]) * scale;
+  for (int c = threadIdx.x; c < HD; c += 256) qs[c] = to_f32(q[(int64_t)b * ldq + h * HD + c]) * scale;
   __syncthreads();
-  const T* Kb = ring_k + (int64_t)b * C * d + h * hd;
-  const T* Vb = ring_v + (int64_t)b * C * d + h * hd;
-  const int nd = (hd + 31) / 32;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  float m = -INFINITY, l = 0.f;
+  const T* Kb = ring_k + (int64_t)b * C * d + h * HD;
+  const T* Vb = ring_v + (int64_t)b * C * d + h * HD;
+  float acc[HD];
+#pragma unroll
+  for (int c = 0; c < HD; ++c) acc[c] = 0.f;
+  float m = -INFINITY, l = 0.f;  // warp-uniform running max, lane-partial sum
   for (int64_t j0 = lo + warp * 32; j0 <= P; j0 += 256) {
     const int64_t j = j0 + lane;
-    float s = -INFINITY;
-    if (j <= P) {
-      const T* kr = Kb + (j % C) * d;
-      float dot = 0.f;
-      for (int c = 0; c < hd; ++c) dot = fmaf(qs[c], to_f32(kr[c]), dot);
-      s = dot;
+    const bool valid = j <= P;
+    const int64_t slot = (valid ? j : P) % C;
+    float s = 0.f;
+#pragma unroll
+    for (int c0 = 0; c0 < HD; c0 += CH) {
+      float kr[CH];
+      load_row_f32<T>(Kb + slot * d + c0, kr, CH);
+#pragma unroll
+      for (int c = 0; c < CH; ++c) s = fmaf(qs[c0 + c], kr[c], s);
     }
+    s = valid ? s : -INFINITY;
     float mb = s;
 #pragma unroll
     for (int o = 16; o; o >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, o));
     const float mnew = fmaxf(m, mb);
-    const float pj = (j <= P) ? expf(s - mnew) : 0.f;
-    const float corr = expf(m - mnew);
-    float ps = pj;
+    const float corr = expf(m - mnew);  // 0 on the first step (m = -inf)
+    const float pj = valid ? expf(s - mnew) : 0.f;
+    l = l * corr + pj;
 #pragma unroll
-    for (int o = 16; o; o >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-    l = l * corr + ps;
+    for (int c0 = 0; c0 < HD; c0 += CH) {
+      float vr[CH];
+      load_row_f32<T>(Vb + slot * d + c0, vr, CH);
 #pragma unroll
-    for (int t = 0; t < 4; ++t) acc[t] *= corr;
-    const int cnt = (int)((P - j0 + 1) < 32 ? (P - j0 + 1) : 32);
-    for (int jj = 0; jj < cnt; ++jj) {
-      const float pp = __shfl_sync(0xffffffffu, pj, jj);
-      const T* vr = Vb + ((j0 + jj) % C) * d;
-      for (int t = 0; t < nd; ++t) {
-        const int c = lane + 32 * t;
-        if (c < hd) acc[t] = fmaf(pp, to_f32(vr[c]), acc[t]);
-      }
+      for (int c = 0; c < CH; ++c) acc[c0 + c] = fmaf(pj, vr[c], acc[c0 + c] * corr);
     }
     m = mnew;
   }
-  if (lane == 0) { wm[warp] = m; wl[warp] = l; }
-  for (int t = 0; t < nd; ++t) {
-    const int c = lane + 32 * t;
-    if (c < hd) wo[warp][c] = acc[t];
+  // warp sums of the lane partials
+#pragma unroll
+  for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+#pragma unroll
+  for (int c = 0; c < HD; ++c) {
+    float v = acc[c];
+#pragma unroll
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    acc[c] = v;
+  }
+  if (lane == 0) {
+    wm[warp] = m;
+    wl[warp] = l;
+#pragma unroll
+    for (int c = 0; c < HD; ++c) wo[warp][c] = acc[c];
   }
   __syncthreads();
   float M = -INFINITY;
   for (int w = 0; w < 8; ++w) M = fmaxf(M, wm[w]);
   float Lsum = 0.f;
   for (int w = 0; w < 8; ++w) Lsum += wm[w] == -INFINITY ? 0.f : wl[w] * expf(wm[w] - M);
-  for (int c = threadIdx.x; c < hd; c += 256) {
+  for (int c = threadIdx.x; c < HD; c += 256) {
     float o = 0.f;
     for (int w = 0; w < 8; ++w)
       if (wm[w] != -INFINITY) o += wo[w][c] * expf(wm[w] - M);
-    out[(int64_t)b * ldo + h * hd + c] = from_f32<T>(o / Lsum);
+    out[(int64_t)b * ldo + h * HD + c] = from_f32<T>(o / Lsum);
   }
 }
 

@@ -4,7 +4,8 @@
 // One CTA = 128 queries of one (sequence, head); key tiles of 128 positions,
 // 128-aligned in absolute position, each taken whole from the ring (positions
 // < q0) or from the current rows (the q|k|v buffer). Warp roles:
-//   warp 0     TMA: Q once, then K and V tiles into a 2-stage ring;
+//   warp 0     TMA: Q once, then K and V tiles into separate rings (a K stage is
+//              freed as soon as its Q K^T is done, a V stage after its P V);
 //   warp 1     MMA issue (one thread): S_j = Q K_j^T into one of two TMEM S
 //              buffers, then O += P_{j-1} V_{j-1} (P from shared memory, V as an
 //              MN-major operand) into the TMEM O accumulator;
@@ -27,11 +28,14 @@ namespace ttt {
 
 template <int HD> struct AttnTcCfg {
   static constexpr int BM = 128, BN = 128;
+  static constexpr int KST = HD == 64 ? 3 : 2;  // K stages
+  static constexpr int VST = HD == 64 ? 3 : 2;  // V stages
   static constexpr int QB = BM * HD * 2;      // Q tile bytes
   static constexpr int KVB = BN * HD * 2;     // K (and V) tile bytes
   static constexpr int PB = BM * BN * 2;      // P tile bytes
   static constexpr int OFF_K0 = QB;
-  static constexpr int OFF_P0 = QB + 2 * 2 * KVB;
+  static constexpr int OFF_V0 = OFF_K0 + KST * KVB;
+  static constexpr int OFF_P0 = OFF_V0 + VST * KVB;
   static constexpr int OFF_BAR = OFF_P0 + 2 * PB;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr uint32_t S_COL = 0, O_COL = 256;
@@ -54,14 +58,16 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(sm + Cf::OFF_BAR);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;    // [2]
-  uint64_t* kv_empty = bars + 3;   // [2]
-  uint64_t* s_full = bars + 5;     // [2]
-  uint64_t* s_free = bars + 7;     // [2]
-  uint64_t* p_full = bars + 9;     // [2]
-  uint64_t* pv_done = bars + 11;   // [2]
-  uint64_t* o_done = bars + 13;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 14);
+  uint64_t* k_full = bars + 1;     // [3]
+  uint64_t* k_empty = bars + 4;    // [3]
+  uint64_t* v_full = bars + 7;     // [3]
+  uint64_t* v_empty = bars + 10;   // [3]
+  uint64_t* s_full = bars + 13;    // [2]
+  uint64_t* s_free = bars + 15;    // [2]
+  uint64_t* p_full = bars + 17;    // [2]
+  uint64_t* pv_done = bars + 19;   // [2]
+  uint64_t* o_done = bars + 21;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 22);
 
   const int warp = threadIdx.x >> 5;
   const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -75,8 +81,11 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1);
       mbar_init(&s_full[s], 1);  mbar_init(&s_free[s], 4);
       mbar_init(&p_full[s], 4);  mbar_init(&pv_done[s], 1);
     }
@@ -100,25 +109,36 @@ __global__ void __launch_bounds__(192, 1)
       const int qrow = b * p.n + i0;
       mbar_arrive_expect_tx(q_full, Cf::QB);
       for (int kb = 0; kb < KB; ++kb) tma_load_3d(sm + kb * Cf::BM * 128, &tm_qkv, q_full, h * HD + kb * 64, qrow, 0);
-      for (int j = 0; j < ntiles; ++j) {
-        const int s = j & 1;
-        if (!mbar_wait(&kv_empty[s], ((j >> 1) & 1) ^ 1, err, DEV_TIMEOUT_EMPTY)) break;
-        uint8_t* sk = sm + Cf::OFF_K0 + s * 2 * Cf::KVB;
-        uint8_t* sv = sk + Cf::KVB;
-        mbar_arrive_expect_tx(&kv_full[s], 2 * Cf::KVB);
+      // K runs up to KST tiles ahead of its use; V up to VST tiles. K_j is issued
+      // before V_j, and K_{j+1} before V_j when its stage is free, so that the
+      // next Q K^T never waits behind a P V.
+      int jk = 0, jv = 0;
+      bool ok = true;
+      auto load = [&](bool isK, int j) -> bool {
+        const int st = isK ? j % Cf::KST : j % Cf::VST;
+        const int use = isK ? j / Cf::KST : j / Cf::VST;
+        uint64_t* emp = isK ? &k_empty[st] : &v_empty[st];
+        uint64_t* ful = isK ? &k_full[st] : &v_full[st];
+        if (!mbar_wait(emp, (use & 1) ^ 1, err, DEV_TIMEOUT_EMPTY)) return false;
+        uint8_t* dst = sm + (isK ? Cf::OFF_K0 : Cf::OFF_V0) + st * Cf::KVB;
+        mbar_arrive_expect_tx(ful, Cf::KVB);
         const int64_t j0 = jt0 + (int64_t)j * Cf::BN;
         if (j0 >= p.q0) {
           const int y = b * p.n + (int)(j0 - p.q0);
-          for (int kb = 0; kb < KB; ++kb) {
-            tma_load_3d(sk + kb * Cf::BN * 128, &tm_qkv, &kv_full[s], p.d + h * HD + kb * 64, y, 0);
-            tma_load_3d(sv + kb * Cf::BN * 128, &tm_qkv, &kv_full[s], 2 * p.d + h * HD + kb * 64, y, 0);
-          }
+          const int x0 = (isK ? p.d : 2 * p.d) + h * HD;
+          for (int kb = 0; kb < KB; ++kb) tma_load_3d(dst + kb * Cf::BN * 128, &tm_qkv, ful, x0 + kb * 64, y, 0);
         } else {
           const int y = b * p.C + (int)(j0 % p.C);
-          for (int kb = 0; kb < KB; ++kb) {
-            tma_load_3d(sk + kb * Cf::BN * 128, &tm_rk, &kv_full[s], h * HD + kb * 64, y, 0);
-            tma_load_3d(sv + kb * Cf::BN * 128, &tm_rv, &kv_full[s], h * HD + kb * 64, y, 0);
-          }
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_3d(dst + kb * Cf::BN * 128, isK ? &tm_rk : &tm_rv, ful, h * HD + kb * 64, y, 0);
+        }
+        return true;
+      };
+      while (ok && (jk < ntiles || jv < ntiles)) {
+        if (jk < ntiles && jk <= jv + 1) {
+          ok = load(true, jk++);
+        } else {
+          ok = load(false, jv++);
         }
       }
     }
@@ -130,10 +150,12 @@ __global__ void __launch_bounds__(192, 1)
       bool ok = mbar_wait(q_full, 0, err, DEV_TIMEOUT_FULL);
       auto issue_pv = [&](int i) -> bool {
         const int s = i & 1;
+        const int vs = i % Cf::VST;
+        if (!mbar_wait(&v_full[vs], (i / Cf::VST) & 1, err, DEV_TIMEOUT_FULL)) return false;
         if (!mbar_wait(&p_full[s], (i >> 1) & 1, err, DEV_TIMEOUT_FULL)) return false;
         tc_fence_after();
         const uint32_t sP = smem_u32(sm + Cf::OFF_P0 + s * Cf::PB);
-        const uint32_t sV = smem_u32(sm + Cf::OFF_K0 + s * 2 * Cf::KVB + Cf::KVB);
+        const uint32_t sV = smem_u32(sm + Cf::OFF_V0 + vs * Cf::KVB);
 #pragma unroll
         for (int kk = 0; kk < Cf::BN / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(sP + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
@@ -141,15 +163,16 @@ __global__ void __launch_bounds__(192, 1)
           tc_mma_f16(tmem + Cf::O_COL, ad, bd, idO, (i | kk) ? 1u : 0u);
         }
         tc_commit(&pv_done[s]);
-        tc_commit(&kv_empty[s]);
+        tc_commit(&v_empty[vs]);
         return true;
       };
       for (int j = 0; j < ntiles && ok; ++j) {
         const int s = j & 1;
-        if (!mbar_wait(&kv_full[s], (j >> 1) & 1, err, DEV_TIMEOUT_FULL)) { ok = false; break; }
+        const int ks = j % Cf::KST;
+        if (!mbar_wait(&k_full[ks], (j / Cf::KST) & 1, err, DEV_TIMEOUT_FULL)) { ok = false; break; }
         if (!mbar_wait(&s_free[s], ((j >> 1) & 1) ^ 1, err, DEV_TIMEOUT_ACC)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t sK = smem_u32(sm + Cf::OFF_K0 + s * 2 * Cf::KVB);
+        const uint32_t sK = smem_u32(sm + Cf::OFF_K0 + ks * Cf::KVB);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint64_t ad = smem_desc_sw128(sQ + (kk >> 2) * (Cf::BM * 128) + (kk & 3) * 32, 16, 1024);
@@ -157,6 +180,7 @@ __global__ void __launch_bounds__(192, 1)
           tc_mma_f16(tmem + Cf::S_COL + s * Cf::BN, ad, bd, idS, kk ? 1u : 0u);
         }
         tc_commit(&s_full[s]);
+        tc_commit(&k_empty[ks]);
         if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
       }
       if (ok) ok = issue_pv(ntiles - 1);
@@ -178,23 +202,35 @@ __global__ void __launch_bounds__(192, 1)
       if (!mbar_wait(&s_full[s], (j >> 1) & 1, err, DEV_TIMEOUT_ACC)) { ok = false; break; }
       tc_fence_after();
       float v[Cf::BN];
+      {
+        uint32_t* vr = reinterpret_cast<uint32_t*>(v);
 #pragma unroll
-      for (int c = 0; c < Cf::BN / 32; ++c) tmem_ld32(tmem + lane_base + Cf::S_COL + s * Cf::BN + c * 32, v + c * 32);
+        for (int c = 0; c < Cf::BN / 32; ++c)
+          tmem_ld32_nowait(tmem + lane_base + Cf::S_COL + s * Cf::BN + c * 32, vr + c * 32);
+        tmem_ld_wait();
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s_free[s]);
       const bool need_mask = (j0 + Cf::BN - 1 > P0) || (j0 < Plast - p.window + 1);
-      float mt = -INFINITY;
+      if (need_mask) {  // diagonal / window-edge tile: branch-free per-element mask
+        const int64_t lo_key = P - p.window + 1;
+        const uint32_t span = (uint32_t)(P - lo_key);
 #pragma unroll
-      for (int c = 0; c < Cf::BN; ++c) {
-        float x = v[c] * sc;
-        if (need_mask) {
-          const int64_t key = j0 + c;
-          if (key > P || key < P - p.window + 1) x = -INFINITY;
+        for (int c = 0; c < Cf::BN; ++c) {
+          const uint32_t off = (uint32_t)(j0 + c - lo_key);
+          v[c] = off <= span ? v[c] : -INFINITY;
         }
-        v[c] = x;
-        mt = fmaxf(mt, x);
       }
+      // row maximum of the raw scores, eight independent chains
+      float mx8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx8[e] = v[e];
+#pragma unroll
+      for (int c = 8; c < Cf::BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], v[c]);
+      float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      mt *= sc;  // scores are compared in the scaled log2 domain (sc > 0 keeps the order)
       // lazily raised reference maximum
       const bool first = m_used == -INFINITY;
       const bool raise = mt > m_used + 8.f;
@@ -219,9 +255,9 @@ __global__ void __launch_bounds__(192, 1)
       l *= factor;
       // the P buffer s was last read by P_{j-2} V_{j-2}
       if (j >= 2 && !mbar_wait(&pv_done[s], ((j - 2) >> 1) & 1, err, DEV_TIMEOUT_ACC)) { ok = false; break; }
-      const float base = m_used == -INFINITY ? 0.f : m_used;
+      const float nbase = m_used == -INFINITY ? 0.f : -m_used;
       uint8_t* prow = sm + Cf::OFF_P0 + s * Cf::PB + r * 128;
-      float lsum = 0.f;
+      float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int kb = 0; kb < Cf::BN / 64; ++kb) {
 #pragma unroll
@@ -229,15 +265,15 @@ __global__ void __launch_bounds__(192, 1)
           float e8[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            e8[e] = ex2_tc(v[kb * 64 + cc * 8 + e] - base);
-            lsum += e8[e];
+            e8[e] = ex2_tc(fmaf(v[kb * 64 + cc * 8 + e], sc, nbase));  // exp2(s*sc - m): masked -inf -> 0
+            ls8[e] += e8[e];
           }
           const uint4 pk = make_uint4(pack_bf16x2(e8[0], e8[1]), pack_bf16x2(e8[2], e8[3]),
                                       pack_bf16x2(e8[4], e8[5]), pack_bf16x2(e8[6], e8[7]));
           *(uint4*)(prow + kb * (Cf::BM * 128) + ((cc ^ (r & 7)) << 4)) = pk;
         }
       }
-      l += lsum;
+      l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       fence_proxy_async();  // P (generic-proxy stores) visible to the tensor core
       tc_fence_before();
       __syncwarp();
@@ -261,6 +297,244 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       if (r < nq && p.lse) p.lse[((int64_t)b * p.H + h) * p.n + i0 + r] = (m_used + __log2f(l)) * 0.6931471805599453f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- backward dQ on tcgen05
+// One CTA = 128 query rows of one (sequence, head), key tiles of 128 positions over
+// each row's whole window (ring and current rows). Per tile: S = Q K^T and
+// dP = dO V^T into TMEM (MMA warp), then four warps form dS = P (dP - D) with
+// P = exp(S*scale - lse) from the forward's log-sum-exp, write dS (bf16) to
+// shared memory, and the MMA warp accumulates dQ += dS K in TMEM (the K tile read
+// again as an MN-major operand). dQ is scaled by 1/sqrt(hd) on the way out.
+template <int HD> struct AttnDqCfg {
+  static constexpr int BM = 128, BN = 128;
+  static constexpr int KST = HD == 64 ? 3 : 2;
+  static constexpr int VST = HD == 64 ? 3 : 2;
+  static constexpr int QB = BM * HD * 2;
+  static constexpr int KVB = BN * HD * 2;
+  static constexpr int DSB = BM * BN * 2;
+  static constexpr int OFF_DO = QB;
+  static constexpr int OFF_K0 = 2 * QB;
+  static constexpr int OFF_V0 = OFF_K0 + KST * KVB;
+  static constexpr int OFF_DS = OFF_V0 + VST * KVB;
+  static constexpr int OFF_BAR = OFF_DS + DSB;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr uint32_t S_COL = 0, DP_COL = 128, DQ_COL = 256;
+};
+
+template <int HD>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_rk,
+                          const __grid_constant__ CUtensorMap tm_rv, const __grid_constant__ CUtensorMap tm_do,
+                          const AttnParams p, int* err) {
+  using Cf = AttnDqCfg<HD>;
+  constexpr int KB = HD / 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = (uint64_t*)(sm + Cf::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;     // [3]
+  uint64_t* k_empty = bars + 4;    // [3]
+  uint64_t* v_full = bars + 7;     // [3]
+  uint64_t* v_empty = bars + 10;   // [3]
+  uint64_t* sp_full = bars + 13;
+  uint64_t* st_free = bars + 14;
+  uint64_t* ds_full = bars + 15;
+  uint64_t* ds_free = bars + 16;
+  uint64_t* dq_done = bars + 17;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 18);
+
+  const int warp = threadIdx.x >> 5;
+  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int i0 = qb * Cf::BM;
+  const int64_t P0 = p.q0 + i0;
+  const int nq = min(Cf::BM, p.n - i0);
+  const int64_t Plast = P0 + nq - 1;
+  const int64_t jlo = max((int64_t)0, P0 - p.window + 1);
+  const int64_t jt0 = (jlo / Cf::BN) * Cf::BN;
+  const int ntiles = (int)((Plast / Cf::BN) * Cf::BN - jt0) / Cf::BN + 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < 3; ++s) {
+      mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
+    }
+    mbar_init(sp_full, 1); mbar_init(st_free, 4);
+    mbar_init(ds_full, 4); mbar_init(ds_free, 1);
+    mbar_init(dq_done, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tm_qkv); prefetch_tmap(&tm_rk); prefetch_tmap(&tm_rv); prefetch_tmap(&tm_do);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (elect_lane0()) {
+      const int qrow = b * p.n + i0;
+      mbar_arrive_expect_tx(q_full, 2 * Cf::QB);
+      for (int kb = 0; kb < KB; ++kb) {
+        tma_load_3d(sm + kb * Cf::BM * 128, &tm_qkv, q_full, h * HD + kb * 64, qrow, 0);
+        tma_load_3d(sm + Cf::OFF_DO + kb * Cf::BM * 128, &tm_do, q_full, h * HD + kb * 64, qrow, 0);
+      }
+      int jk = 0, jv = 0;
+      bool ok = true;
+      auto load = [&](bool isK, int j) -> bool {
+        const int st = isK ? j % Cf::KST : j % Cf::VST;
+        const int use = isK ? j / Cf::KST : j / Cf::VST;
+        uint64_t* emp = isK ? &k_empty[st] : &v_empty[st];
+        uint64_t* ful = isK ? &k_full[st] : &v_full[st];
+        if (!mbar_wait(emp, (use & 1) ^ 1, err, DEV_TIMEOUT_EMPTY)) return false;
+        uint8_t* dst = sm + (isK ? Cf::OFF_K0 : Cf::OFF_V0) + st * Cf::KVB;
+        mbar_arrive_expect_tx(ful, Cf::KVB);
+        const int64_t j0 = jt0 + (int64_t)j * Cf::BN;
+        if (j0 >= p.q0) {
+          const int y = b * p.n + (int)(j0 - p.q0);
+          const int x0 = (isK ? p.d : 2 * p.d) + h * HD;
+          for (int kb = 0; kb < KB; ++kb) tma_load_3d(dst + kb * Cf::BN * 128, &tm_qkv, ful, x0 + kb * 64, y, 0);
+        } else {
+          const int y = b * p.C + (int)(j0 % p.C);
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_3d(dst + kb * Cf::BN * 128, isK ? &tm_rk : &tm_rv, ful, h * HD + kb * 64, y, 0);
+        }
+        return true;
+      };
+      // V_j is consumed first (dP_j), K_j last (dQ_j): keep V one tile ahead of K
+      while (ok && (jk < ntiles || jv < ntiles)) {
+        if (jv < ntiles && jv <= jk) ok = load(false, jv++);
+        else ok = load(true, jk++);
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_lane0()) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, Cf::BN, false, false);
+      constexpr uint32_t idQ = idesc_bf16_f32(128, HD, false, true);
+      const uint32_t sQ = smem_u32(sm), sdO = smem_u32(sm + Cf::OFF_DO), sdS = smem_u32(sm + Cf::OFF_DS);
+      bool ok = mbar_wait(q_full, 0, err, DEV_TIMEOUT_FULL);
+      for (int j = 0; j < ntiles && ok; ++j) {
+        const int ks = j % Cf::KST, vs = j % Cf::VST;
+        if (!mbar_wait(&k_full[ks], (j / Cf::KST) & 1, err, DEV_TIMEOUT_FULL) ||
+            !mbar_wait(&v_full[vs], (j / Cf::VST) & 1, err, DEV_TIMEOUT_FULL) ||
+            !mbar_wait(st_free, (j & 1) ^ 1, err, DEV_TIMEOUT_ACC)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sK = smem_u32(sm + Cf::OFF_K0 + ks * Cf::KVB);
+        const uint32_t sV = smem_u32(sm + Cf::OFF_V0 + vs * Cf::KVB);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          tc_mma_f16(tmem + Cf::S_COL, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(sK + off, 16, 1024), idS,
+                     kk ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          tc_mma_f16(tmem + Cf::DP_COL, smem_desc_sw128(sdO + off, 16, 1024), smem_desc_sw128(sV + off, 16, 1024),
+                     idS, kk ? 1u : 0u);
+        }
+        tc_commit(sp_full);
+        tc_commit(&v_empty[vs]);
+        if (!mbar_wait(ds_full, j & 1, err, DEV_TIMEOUT_FULL)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < Cf::BN / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(sdS + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sK + kk * 2048, Cf::BN * 128, 1024);
+          tc_mma_f16(tmem + Cf::DQ_COL, ad, bd, idQ, (j | kk) ? 1u : 0u);
+        }
+        tc_commit(ds_free);
+        tc_commit(&k_empty[ks]);
+      }
+      if (ok) tc_commit(dq_done);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int lane = threadIdx.x & 31;
+    const int r = quarter * 32 + lane;
+    const int64_t P = P0 + r;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const float sc = p.scale * 1.4426950408889634f;
+    const int64_t si = ((int64_t)b * p.H + h) * p.n + i0 + r;
+    const float nL = r < nq ? -p.lse[si] * 1.4426950408889634f : -INFINITY;  // exp2(s*sc - lse*log2e)
+    const float Dr = r < nq ? p.Dsum[si] : 0.f;
+    const int64_t lo_key = P - p.window + 1;
+    const uint32_t span = (uint32_t)(P - lo_key);
+    uint8_t* drow = sm + Cf::OFF_DS + r * 128;
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      const int64_t j0 = jt0 + (int64_t)j * Cf::BN;
+      const bool need_mask = (j0 + Cf::BN - 1 > P0) || (j0 < Plast - p.window + 1);
+      if (!mbar_wait(sp_full, j & 1, err, DEV_TIMEOUT_ACC) || !mbar_wait(ds_free, (j & 1) ^ 1, err, DEV_TIMEOUT_ACC)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < Cf::BN / 32; ++c) {
+        uint32_t sr[32], dr[32];
+        tmem_ld32_nowait(tmem + lane_base + Cf::S_COL + c * 32, sr);
+        tmem_ld32_nowait(tmem + lane_base + Cf::DP_COL + c * 32, dr);
+        tmem_ld_wait();
+        float ds[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float pr = ex2_tc(fmaf(__uint_as_float(sr[e]), sc, nL));
+          if (need_mask) {
+            const uint32_t off = (uint32_t)(j0 + c * 32 + e - lo_key);
+            pr = off <= span ? pr : 0.f;
+          }
+          ds[e] = pr * (__uint_as_float(dr[e]) - Dr);
+        }
+        const int kb = c >> 1;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int cc = (c & 1) * 4 + q;
+          *(uint4*)(drow + kb * (Cf::BM * 128) + ((cc ^ (r & 7)) << 4)) =
+              make_uint4(pack_bf16x2(ds[8 * q], ds[8 * q + 1]), pack_bf16x2(ds[8 * q + 2], ds[8 * q + 3]),
+                         pack_bf16x2(ds[8 * q + 4], ds[8 * q + 5]), pack_bf16x2(ds[8 * q + 6], ds[8 * q + 7]));
+        }
+      }
+      tc_fence_before();
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(st_free);
+        mbar_arrive(ds_full);
+      }
+    }
+    if (ok && mbar_wait(dq_done, 0, err, DEV_TIMEOUT_ACC)) {
+      tc_fence_after();
+      bf16* dQ = (bf16*)p.dQ + ((int64_t)b * p.n + i0 + r) * p.lddq + h * HD;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        float o[32];
+        tmem_ld32(tmem + lane_base + Cf::DQ_COL + c * 32, o);
+        if (r < nq) {
+          uint4* dst = (uint4*)(dQ + c * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack_bf16x2(o[8 * q] * p.scale, o[8 * q + 1] * p.scale),
+                                pack_bf16x2(o[8 * q + 2] * p.scale, o[8 * q + 3] * p.scale),
+                                pack_bf16x2(o[8 * q + 4] * p.scale, o[8 * q + 5] * p.scale),
+                                pack_bf16x2(o[8 * q + 6] * p.scale, o[8 * q + 7] * p.scale));
+        }
+      }
     }
   }
   tc_fence_before();

@@ -25,6 +25,7 @@ enum EpiKind : int {
   EPI_GELU = 2,    // Y = acc (if Y), D = gelu(acc)        (element type)
   EPI_DGELU = 3,   // D = acc * gelu'(X)                   (element type, X element type)
   EPI_SGD = 4,     // D(f32) += acc, Y = D (if Y)          (alpha = -eta)
+  EPI_QKV_ROPE = 5,  // D = acc (element type) with RoPE applied to columns [0, rope_cols)
 };
 
 struct GemmParams {
@@ -41,6 +42,12 @@ struct GemmParams {
   void* Y; int64_t ldy, sY;
   float alpha;
   int epi;
+  // EPI_QKV_ROPE: rotate pairs (i, i + hd/2) of each head in columns [0, rope_cols) of row m at
+  // position rope_pos0 + (m % rope_n) (rope_pos0 read from *rope_pos_dev when given), angles
+  // pos * base^(-2i/hd) from the double-precision tables lo[p & 1023][i], hi[p >> 10][i].
+  const float2* rope_lo; const float2* rope_hi;
+  int64_t rope_pos0; const int64_t* rope_pos_dev;
+  int rope_n, rope_hd, rope_cols;
 };
 
 // ============================================================== epilogue (per element)
@@ -345,11 +352,50 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_after();
       const int m = m0 + row_in_tile;
       const uint32_t taddr = tmem_base + acc * BN + ((uint32_t)(quarter * 32) << 16);
+      if (p.epi == EPI_QKV_ROPE && n0 < p.rope_cols) {
+        // chunks come in pairs (c, c + hd/64): the two halves of each head
+        const int half_chunks = p.rope_hd / 64;
+        const int64_t pos = (p.rope_pos_dev ? *p.rope_pos_dev : p.rope_pos0) + (m % p.rope_n);
+        const int hh = p.rope_hd / 2;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        tmem_ld32(taddr + c * 32, v);
-        if (m < p.M) epi_row32<bf16>(p, z, m, n0 + c * 32, v);
+        for (int c = 0; c < BN / 32; ++c) {
+          if ((c / half_chunks) & 1) continue;  // second half of a head: done with its partner
+          float v1[32], v2[32];
+          tmem_ld32(taddr + c * 32, v1);
+          tmem_ld32(taddr + (c + half_chunks) * 32, v2);
+          if (m < p.M) {
+            const int i0 = (c % half_chunks) * 32;  // pair index of v1[0] within the head
+#pragma unroll 4
+            for (int e = 0; e < 32; ++e) {
+              const float2 a = p.rope_lo[(pos & 1023) * hh + i0 + e];
+              const float2 bq = p.rope_hi[(pos >> 10) * hh + i0 + e];
+              const float cs = a.x * bq.x - a.y * bq.y, sn = a.y * bq.x + a.x * bq.y;
+              const float x1 = v1[e] * p.alpha, x2 = v2[e] * p.alpha;
+              v1[e] = x1 * cs - x2 * sn;
+              v2[e] = x2 * cs + x1 * sn;
+            }
+            GemmParams q = p;
+            q.epi = EPI_STORE;
+            q.alpha = 1.f;
+            epi_row32<bf16>(q, z, m, n0 + c * 32, v1);
+            epi_row32<bf16>(q, z, m, n0 + (c + half_chunks) * 32, v2);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(taddr + c * 32, v);
+          if (m < p.M) {
+            if (p.epi == EPI_QKV_ROPE) {
+              GemmParams q = p;
+              q.epi = EPI_STORE;
+              epi_row32<bf16>(q, z, m, n0 + c * 32, v);
+            } else {
+              epi_row32<bf16>(p, z, m, n0 + c * 32, v);
+            }
+          }
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -372,5 +418,7 @@ int prime_kernel_attributes();
 struct AttnParams;
 bool attn_tc_ok(const AttnParams& p);
 cudaError_t attn_fwd_tc_launch(const AttnParams& p, cudaStream_t st, int* err, bool* ok);
+bool attn_dq_tc_ok(const AttnParams& p);
+cudaError_t attn_bwd_dq_tc_launch(const AttnParams& p, cudaStream_t st, int* err, bool* ok);
 
 }  // namespace ttt

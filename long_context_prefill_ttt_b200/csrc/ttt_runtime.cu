@@ -130,6 +130,28 @@ cudaError_t attn_fwd_tc_launch(const AttnParams& p, cudaStream_t st, int* err, b
   return cudaGetLastError();
 }
 
+bool attn_dq_tc_ok(const AttnParams& p) {
+  return attn_tc_ok(p) && p.lddo == p.d && aligned16(p.dO) && aligned16(p.dQ) && p.lddq % 8 == 0;
+}
+
+cudaError_t attn_bwd_dq_tc_launch(const AttnParams& p, cudaStream_t st, int* err, bool* ok) {
+  CUtensorMap tq, tk, tv, tdo;
+  *ok = make_rows_map(&tq, p.Q, 3 * p.d, (int64_t)p.B * p.n) && make_rows_map(&tdo, p.dO, p.d, (int64_t)p.B * p.n);
+  if (*ok && p.q0 > 0) {
+    *ok = make_rows_map(&tk, p.Kc, p.d, (int64_t)p.B * p.C) && make_rows_map(&tv, p.Vc, p.d, (int64_t)p.B * p.C);
+  } else {
+    tk = tq;
+    tv = tq;
+  }
+  if (!*ok) return cudaSuccess;
+  dim3 grid((p.n + 127) / 128, p.H, p.B);
+  if (p.hd == 128)
+    attn_bwd_dq_tc_kernel<128><<<grid, 192, AttnDqCfg<128>::SMEM, st>>>(tq, tk, tv, tdo, p, err);
+  else
+    attn_bwd_dq_tc_kernel<64><<<grid, 192, AttnDqCfg<64>::SMEM, st>>>(tq, tk, tv, tdo, p, err);
+  return cudaGetLastError();
+}
+
 // Dynamic shared-memory limits of every large-smem kernel, set once per process
 // before any launch (and so never inside a CUDA graph capture).
 template <int BN, bool AM, bool BM> static cudaError_t tc_attr() {
@@ -146,7 +168,11 @@ int prime_kernel_attributes() {
                            cudaFuncSetAttribute(attn_fwd_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 AttnTcCfg<64>::SMEM),
                            cudaFuncSetAttribute(attn_fwd_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                AttnTcCfg<128>::SMEM)};
+                                                AttnTcCfg<128>::SMEM),
+                           cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                AttnDqCfg<64>::SMEM),
+                           cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<128>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, AttnDqCfg<128>::SMEM)};
   for (cudaError_t x : r)
     if (x != cudaSuccess) e = x;
   if (e != cudaSuccess) return (int)e;
@@ -167,9 +193,20 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
     use_tc = false;
   if (use_tc && p.batch > 1 && p.sD % 8 != 0) use_tc = false;
   if (use_tc && p.Y && !(aligned16(p.Y) && p.ldy % 8 == 0 && (p.batch == 1 || p.sY % 8 == 0))) use_tc = false;
+  if (p.epi == EPI_QKV_ROPE &&
+      !(p.rope_hd == 64 || p.rope_hd == 128) ) use_tc = false;
+  // no tile may straddle the end of the rotated columns: rope_cols a multiple of the widest tile
+  if (use_tc && p.epi == EPI_QKV_ROPE && (p.batch != 1 || p.rope_cols % 256 != 0)) use_tc = false;
   if (use_tc) {
+    // tile width: the one whose tile count fills the persistent grid's waves best
+    // (fraction of CTA slots busy over ceil(tiles / SMs) waves); ties go to 256
     const int m_tiles = (p.M + TC_BM - 1) / TC_BM;
-    const bool n256 = (p.N % 256 == 0) && (m_tiles * (p.N / 256) * p.batch >= (num_sms * 9) / 10);
+    auto wave_eff = [&](int bn) {
+      const double t = (double)m_tiles * (p.N / bn) * p.batch;
+      const double waves = std::ceil(t / num_sms);
+      return t / (waves * num_sms);
+    };
+    const bool n256 = (p.N % 256 == 0) && wave_eff(256) >= wave_eff(128) - 1e-9;
     bool ok = false;
     cudaError_t e;
     if (!p.a_mn && !p.b_mn)
@@ -182,10 +219,22 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
     if (ok) return 0;
   }
   dim3 grid((p.N + 63) / 64, (p.M + 63) / 64, p.batch);
+  GemmParams q = p;
+  if (p.epi == EPI_QKV_ROPE) q.epi = EPI_STORE;  // rotation as a separate pass below
   if (elem_is_bf16)
-    gemm_simt_kernel<bf16><<<grid, 256, 0, st>>>(p);
+    gemm_simt_kernel<bf16><<<grid, 256, 0, st>>>(q);
   else
-    gemm_simt_kernel<float><<<grid, 256, 0, st>>>(p);
+    gemm_simt_kernel<float><<<grid, 256, 0, st>>>(q);
+  if (p.epi == EPI_QKV_ROPE) {
+    const int64_t work = (int64_t)p.M * (p.rope_cols / 2);
+    const unsigned blocks = (unsigned)((work + 255) / 256);
+    if (elem_is_bf16)
+      rope_kernel<bf16><<<blocks, 256, 0, st>>>((bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0,
+                                                 p.rope_hd, p.rope_lo, p.rope_hi, 0, p.rope_pos_dev);
+    else
+      rope_kernel<float><<<blocks, 256, 0, st>>>((float*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0,
+                                                  p.rope_hd, p.rope_lo, p.rope_hi, 0, p.rope_pos_dev);
+  }
   return (int)cudaGetLastError();
 }
 
@@ -697,28 +746,35 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
   int rc;
   rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(xin, d, Lw.g_attn, cfg.rms_eps, rows, d, r, d, rstd);
   TTT_LAUNCHED();
-  if ((rc = gemm(gp(rows, 3 * d, d, r, d, false, Lw.Wqkv, d, false, qkv, 3 * d, false, EPI_STORE))) != TTT_OK)
-    return rc;
+  {  // q|k|v = r Wqkv^T with RoPE applied to q and k in the GEMM epilogue
+    GemmParams pq = gp(rows, 3 * d, d, r, d, false, Lw.Wqkv, d, false, qkv, 3 * d, false, EPI_QKV_ROPE);
+    pq.rope_lo = rope_lo; pq.rope_hi = rope_hi; pq.rope_hd = hd; pq.rope_cols = 2 * d;
+    pq.rope_n = decode_mode ? 1 : n;
+    pq.rope_pos0 = decode_mode ? 0 : q0;
+    pq.rope_pos_dev = decode_mode ? pos_dev : nullptr;
+    if ((rc = gemm(pq)) != TTT_OK) return rc;
+  }
   if (decode_mode) {
     // one position per sequence, position on the device: append its K/V to the ring
     // first, then attend over the window entirely from the ring
-    rope_kernel<T><<<nblk((int64_t)rows * d, 256), 256, 0, st>>>(qkv, 3 * d, 2 * d, rows, 1, 0, hd, rope_lo,
-                                                                  rope_hi, 0, pos_dev);
-    TTT_LAUNCHED();
     const int64_t work = sizeof(T) == 2 ? (int64_t)B * (d / 8) : (int64_t)B * d;
     kv_append_kernel<T><<<nblk(work, 256), 256, 0, st>>>(qkv, 3 * d, d, 2 * d, 1, B, 0, d, Lw.ring_k, Lw.ring_v, C,
                                                          pos_dev);
     TTT_LAUNCHED();
-    attn_decode_kernel<T><<<dim3(H, B), 256, 0, st>>>(qkv, 3 * d, Lw.ring_k, Lw.ring_v, C, d, hd, kwin, pos_dev,
-                                                      1.0f / sqrtf((float)hd), o, d);
+    const float scale = 1.0f / sqrtf((float)hd);
+    const dim3 dg(H, B);
+    switch (hd) {
+      case 16: attn_decode_kernel<T, 16><<<dg, 256, 0, st>>>(qkv, 3 * d, Lw.ring_k, Lw.ring_v, C, d, kwin, pos_dev, scale, o, d); break;
+      case 32: attn_decode_kernel<T, 32><<<dg, 256, 0, st>>>(qkv, 3 * d, Lw.ring_k, Lw.ring_v, C, d, kwin, pos_dev, scale, o, d); break;
+      case 64: attn_decode_kernel<T, 64><<<dg, 256, 0, st>>>(qkv, 3 * d, Lw.ring_k, Lw.ring_v, C, d, kwin, pos_dev, scale, o, d); break;
+      case 128: attn_decode_kernel<T, 128><<<dg, 256, 0, st>>>(qkv, 3 * d, Lw.ring_k, Lw.ring_v, C, d, kwin, pos_dev, scale, o, d); break;
+      default: poisoned = true; return fail(this, TTT_ERR_UNSUPPORTED, "decode: head dim must be 16, 32, 64 or 128");
+    }
     TTT_LAUNCHED();
     GemmParams pd = gp(rows, d, d, o, d, false, Lw.Wo, d, false, xout, d, true, EPI_RESID);
     pd.X = xin; pd.ldx = d;
     return gemm(pd);
   }
-  rope_kernel<T><<<nblk((int64_t)rows * d, 256), 256, 0, st>>>(qkv, 3 * d, 2 * d, rows, n, q0, hd, rope_lo, rope_hi,
-                                                                0);
-  TTT_LAUNCHED();
   AttnParams ap;
   memset(&ap, 0, sizeof(ap));
   ap.B = B; ap.H = H; ap.hd = hd; ap.n = n; ap.d = d; ap.q0 = q0; ap.window = kwin;
@@ -873,8 +929,17 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
                2.0 * hd * H * (double)B * (2.0 * attn_pairs(cn, chunk_pos) + 2.0 * attn_pairs(cn, 0)), 0.0);
     attn_bwd_prep_kernel<T><<<nblk((int64_t)rows * H, 8), 256, 0, st>>>(ap);
     TTT_LAUNCHED();
+    bool dq_done = false;
+    if (is_bf16 && attn_dq_tc_ok(ap)) {
+      const cudaError_t e = attn_bwd_dq_tc_launch(ap, st, dev_err, &dq_done);
+      if (e != cudaSuccess) {
+        poisoned = true;
+        return fail(this, TTT_ERR_CUDA, std::string("attention backward: ") + cudaGetErrorString(e));
+      }
+    }
     if (is_bf16 && attn_mma_ok(ap)) {
-      const cudaError_t e = hd == 128 ? attn_bwd_mma_launch<128>(ap, st) : attn_bwd_mma_launch<64>(ap, st);
+      const cudaError_t e =
+          hd == 128 ? attn_bwd_mma_launch<128>(ap, st, !dq_done) : attn_bwd_mma_launch<64>(ap, st, !dq_done);
       (void)e;
       launches += 1;
     } else {
@@ -1166,7 +1231,7 @@ static int validate(const ttt_config* c, std::string* why) {
   if (c->n_ttt < 1 || c->n_ttt > c->n_layers) return bad("n_ttt must be in [1, n_layers]");
   if (c->d % c->n_heads) return bad("d must be a multiple of n_heads");
   const int hd = c->d / c->n_heads;
-  if (hd % 2 || hd > 128) return bad("head dim must be even and <= 128");
+  if (hd != 16 && hd != 32 && hd != 64 && hd != 128) return bad("head dim must be 16, 32, 64 or 128");
   if (c->minibatch_b <= 0 || c->window_k < c->minibatch_b) return bad("need window_k >= minibatch_b > 0");
   if (c->d % 8 || c->mlp_hidden % 8 || c->ttt_hidden % 8 || c->static_hidden % 8 || c->vocab % 8)
     return bad("widths and vocab must be multiples of 8");
