@@ -103,6 +103,8 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     if (elect_lane0()) {
@@ -308,16 +310,18 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // ---------------------------------------------------------------- backward dQ on tcgen05
-// One CTA = 128 query rows of one (sequence, head), key tiles of 128 positions over
-// each row's whole window (ring and current rows). Per tile: S = Q K^T and
-// dP = dO V^T into TMEM (MMA warp), then four warps form dS = P (dP - D) with
-// P = exp(S*scale - lse) from the forward's log-sum-exp, write dS (bf16) to
-// shared memory, and the MMA warp accumulates dQ += dS K in TMEM (the K tile read
-// again as an MN-major operand). dQ is scaled by 1/sqrt(hd) on the way out.
+// One CTA = 128 query rows of one (sequence, head), key tiles of 64 positions over
+// each row's whole window (ring and current rows). Per tile j: S = Q K^T and
+// dP = dO V^T into one of two TMEM buffers (MMA warp); four warps form
+// dS = P (dP - D) with P = exp(S*scale - lse) from the forward's log-sum-exp and
+// write dS (bf16) to one of two shared-memory buffers; the MMA warp accumulates
+// dQ += dS K in TMEM (the K tile read again as an MN-major operand). With S/dP and
+// dS double-buffered, S_{j+1} and dP_{j+1} run on the tensor cores while the
+// warps form dS_j. dQ is scaled by 1/sqrt(hd) on the way out.
+// TMEM: S0 [0,64), dP0 [64,128), S1 [128,192), dP1 [192,256), dQ [256, 256+HD).
 template <int HD> struct AttnDqCfg {
-  static constexpr int BM = 128, BN = 128;
-  static constexpr int KST = HD == 64 ? 3 : 2;
-  static constexpr int VST = HD == 64 ? 3 : 2;
+  static constexpr int BM = 128, BN = 64;
+  static constexpr int KST = 3, VST = 3;
   static constexpr int QB = BM * HD * 2;
   static constexpr int KVB = BN * HD * 2;
   static constexpr int DSB = BM * BN * 2;
@@ -325,16 +329,18 @@ template <int HD> struct AttnDqCfg {
   static constexpr int OFF_K0 = 2 * QB;
   static constexpr int OFF_V0 = OFF_K0 + KST * KVB;
   static constexpr int OFF_DS = OFF_V0 + VST * KVB;
-  static constexpr int OFF_BAR = OFF_DS + DSB;
+  static constexpr int OFF_BAR = OFF_DS + 2 * DSB;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
-  static constexpr uint32_t S_COL = 0, DP_COL = 128, DQ_COL = 256;
+  static constexpr uint32_t DQ_COL = 256;
+  static __device__ __forceinline__ uint32_t s_col(int b) { return b * 128; }
+  static __device__ __forceinline__ uint32_t dp_col(int b) { return b * 128 + 64; }
 };
 
 template <int HD>
 __global__ void __launch_bounds__(192, 1)
-    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_rk,
-                          const __grid_constant__ CUtensorMap tm_rv, const __grid_constant__ CUtensorMap tm_do,
-                          const AttnParams p, int* err) {
+    attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                          const __grid_constant__ CUtensorMap tm_rk, const __grid_constant__ CUtensorMap tm_rv,
+                          const __grid_constant__ CUtensorMap tm_do, const AttnParams p, int* err) {
   using Cf = AttnDqCfg<HD>;
   constexpr int KB = HD / 64;
   extern __shared__ uint8_t smem_raw[];
@@ -345,12 +351,12 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* k_empty = bars + 4;    // [3]
   uint64_t* v_full = bars + 7;     // [3]
   uint64_t* v_empty = bars + 10;   // [3]
-  uint64_t* sp_full = bars + 13;
-  uint64_t* st_free = bars + 14;
-  uint64_t* ds_full = bars + 15;
-  uint64_t* ds_free = bars + 16;
-  uint64_t* dq_done = bars + 17;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 18);
+  uint64_t* sp_full = bars + 13;   // [2]
+  uint64_t* sp_free = bars + 15;   // [2]
+  uint64_t* ds_full = bars + 17;   // [2]
+  uint64_t* ds_free = bars + 19;   // [2]
+  uint64_t* dq_done = bars + 21;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 22);
 
   const int warp = threadIdx.x >> 5;
   const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -368,11 +374,13 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
       mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
     }
-    mbar_init(sp_full, 1); mbar_init(st_free, 4);
-    mbar_init(ds_full, 4); mbar_init(ds_free, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sp_full[s], 1); mbar_init(&sp_free[s], 4);
+      mbar_init(&ds_full[s], 4); mbar_init(&ds_free[s], 1);
+    }
     mbar_init(dq_done, 1);
     fence_mbar_init();
-    prefetch_tmap(&tm_qkv); prefetch_tmap(&tm_rk); prefetch_tmap(&tm_rv); prefetch_tmap(&tm_do);
+    prefetch_tmap(&tm_q); prefetch_tmap(&tm_kv); prefetch_tmap(&tm_rk); prefetch_tmap(&tm_rv); prefetch_tmap(&tm_do);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -382,20 +390,20 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
 
   if (warp == 0) {
     if (elect_lane0()) {
       const int qrow = b * p.n + i0;
       mbar_arrive_expect_tx(q_full, 2 * Cf::QB);
       for (int kb = 0; kb < KB; ++kb) {
-        tma_load_3d(sm + kb * Cf::BM * 128, &tm_qkv, q_full, h * HD + kb * 64, qrow, 0);
+        tma_load_3d(sm + kb * Cf::BM * 128, &tm_q, q_full, h * HD + kb * 64, qrow, 0);
         tma_load_3d(sm + Cf::OFF_DO + kb * Cf::BM * 128, &tm_do, q_full, h * HD + kb * 64, qrow, 0);
       }
-      int jk = 0, jv = 0;
-      bool ok = true;
       auto load = [&](bool isK, int j) -> bool {
-        const int st = isK ? j % Cf::KST : j % Cf::VST;
-        const int use = isK ? j / Cf::KST : j / Cf::VST;
+        const int st = j % 3;
+        const int use = j / 3;
         uint64_t* emp = isK ? &k_empty[st] : &v_empty[st];
         uint64_t* ful = isK ? &k_full[st] : &v_full[st];
         if (!mbar_wait(emp, (use & 1) ^ 1, err, DEV_TIMEOUT_EMPTY)) return false;
@@ -405,7 +413,7 @@ __global__ void __launch_bounds__(192, 1)
         if (j0 >= p.q0) {
           const int y = b * p.n + (int)(j0 - p.q0);
           const int x0 = (isK ? p.d : 2 * p.d) + h * HD;
-          for (int kb = 0; kb < KB; ++kb) tma_load_3d(dst + kb * Cf::BN * 128, &tm_qkv, ful, x0 + kb * 64, y, 0);
+          for (int kb = 0; kb < KB; ++kb) tma_load_3d(dst + kb * Cf::BN * 128, &tm_kv, ful, x0 + kb * 64, y, 0);
         } else {
           const int y = b * p.C + (int)(j0 % p.C);
           for (int kb = 0; kb < KB; ++kb)
@@ -413,23 +421,36 @@ __global__ void __launch_bounds__(192, 1)
         }
         return true;
       };
-      // V_j is consumed first (dP_j), K_j last (dQ_j): keep V one tile ahead of K
-      while (ok && (jk < ntiles || jv < ntiles)) {
-        if (jv < ntiles && jv <= jk) ok = load(false, jv++);
-        else ok = load(true, jk++);
-      }
+      for (int j = 0; j < ntiles; ++j)
+        if (!load(true, j) || !load(false, j)) break;
     }
   } else if (warp == 1) {
     if (elect_lane0()) {
       constexpr uint32_t idS = idesc_bf16_f32(128, Cf::BN, false, false);
       constexpr uint32_t idQ = idesc_bf16_f32(128, HD, false, true);
-      const uint32_t sQ = smem_u32(sm), sdO = smem_u32(sm + Cf::OFF_DO), sdS = smem_u32(sm + Cf::OFF_DS);
+      const uint32_t sQ = smem_u32(sm), sdO = smem_u32(sm + Cf::OFF_DO);
       bool ok = mbar_wait(q_full, 0, err, DEV_TIMEOUT_FULL);
+      auto issue_dq = [&](int i) -> bool {
+        const int s = i & 1, ks = i % 3;
+        if (!mbar_wait(&ds_full[s], (i >> 1) & 1, err, DEV_TIMEOUT_FULL)) return false;
+        tc_fence_after();
+        const uint32_t sdS = smem_u32(sm + Cf::OFF_DS + s * Cf::DSB);
+        const uint32_t sK = smem_u32(sm + Cf::OFF_K0 + ks * Cf::KVB);
+#pragma unroll
+        for (int kk = 0; kk < Cf::BN / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(sdS + kk * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(sK + kk * 2048, Cf::BN * 128, 1024);
+          tc_mma_f16(tmem + Cf::DQ_COL, ad, bd, idQ, (i | kk) ? 1u : 0u);
+        }
+        tc_commit(&ds_free[s]);
+        tc_commit(&k_empty[ks]);
+        return true;
+      };
       for (int j = 0; j < ntiles && ok; ++j) {
-        const int ks = j % Cf::KST, vs = j % Cf::VST;
-        if (!mbar_wait(&k_full[ks], (j / Cf::KST) & 1, err, DEV_TIMEOUT_FULL) ||
-            !mbar_wait(&v_full[vs], (j / Cf::VST) & 1, err, DEV_TIMEOUT_FULL) ||
-            !mbar_wait(st_free, (j & 1) ^ 1, err, DEV_TIMEOUT_ACC)) {
+        const int s = j & 1, ks = j % 3, vs = j % 3;
+        if (!mbar_wait(&k_full[ks], (j / 3) & 1, err, DEV_TIMEOUT_FULL) ||
+            !mbar_wait(&v_full[vs], (j / 3) & 1, err, DEV_TIMEOUT_FULL) ||
+            !mbar_wait(&sp_free[s], ((j >> 1) & 1) ^ 1, err, DEV_TIMEOUT_ACC)) {
           ok = false;
           break;
         }
@@ -438,29 +459,23 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t sV = smem_u32(sm + Cf::OFF_V0 + vs * Cf::KVB);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          tc_mma_f16(tmem + Cf::S_COL, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(sK + off, 16, 1024), idS,
-                     kk ? 1u : 0u);
+          const uint32_t offa = (kk >> 2) * (Cf::BM * 128) + (kk & 3) * 32;
+          const uint32_t offb = (kk >> 2) * (Cf::BN * 128) + (kk & 3) * 32;
+          tc_mma_f16(tmem + Cf::s_col(s), smem_desc_sw128(sQ + offa, 16, 1024), smem_desc_sw128(sK + offb, 16, 1024),
+                     idS, kk ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          tc_mma_f16(tmem + Cf::DP_COL, smem_desc_sw128(sdO + off, 16, 1024), smem_desc_sw128(sV + off, 16, 1024),
-                     idS, kk ? 1u : 0u);
+          const uint32_t offa = (kk >> 2) * (Cf::BM * 128) + (kk & 3) * 32;
+          const uint32_t offb = (kk >> 2) * (Cf::BN * 128) + (kk & 3) * 32;
+          tc_mma_f16(tmem + Cf::dp_col(s), smem_desc_sw128(sdO + offa, 16, 1024),
+                     smem_desc_sw128(sV + offb, 16, 1024), idS, kk ? 1u : 0u);
         }
-        tc_commit(sp_full);
+        tc_commit(&sp_full[s]);
         tc_commit(&v_empty[vs]);
-        if (!mbar_wait(ds_full, j & 1, err, DEV_TIMEOUT_FULL)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < Cf::BN / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(sdS + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(sK + kk * 2048, Cf::BN * 128, 1024);
-          tc_mma_f16(tmem + Cf::DQ_COL, ad, bd, idQ, (j | kk) ? 1u : 0u);
-        }
-        tc_commit(ds_free);
-        tc_commit(&k_empty[ks]);
+        if (j >= 1 && !issue_dq(j - 1)) { ok = false; break; }
       }
+      if (ok) ok = issue_dq(ntiles - 1);
       if (ok) tc_commit(dq_done);
     }
   } else {
@@ -475,48 +490,47 @@ __global__ void __launch_bounds__(192, 1)
     const float Dr = r < nq ? p.Dsum[si] : 0.f;
     const int64_t lo_key = P - p.window + 1;
     const uint32_t span = (uint32_t)(P - lo_key);
-    uint8_t* drow = sm + Cf::OFF_DS + r * 128;
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
+      const int s = j & 1;
       const int64_t j0 = jt0 + (int64_t)j * Cf::BN;
       const bool need_mask = (j0 + Cf::BN - 1 > P0) || (j0 < Plast - p.window + 1);
-      if (!mbar_wait(sp_full, j & 1, err, DEV_TIMEOUT_ACC) || !mbar_wait(ds_free, (j & 1) ^ 1, err, DEV_TIMEOUT_ACC)) {
+      if (!mbar_wait(&sp_full[s], (j >> 1) & 1, err, DEV_TIMEOUT_ACC) ||
+          !mbar_wait(&ds_free[s], ((j >> 1) & 1) ^ 1, err, DEV_TIMEOUT_ACC)) {
         ok = false;
         break;
       }
       tc_fence_after();
+      uint32_t sr[64], dr[64];
+      tmem_ld32_nowait(tmem + lane_base + Cf::s_col(s), sr);
+      tmem_ld32_nowait(tmem + lane_base + Cf::s_col(s) + 32, sr + 32);
+      tmem_ld32_nowait(tmem + lane_base + Cf::dp_col(s), dr);
+      tmem_ld32_nowait(tmem + lane_base + Cf::dp_col(s) + 32, dr + 32);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sp_free[s]);  // S/dP buffer s may be overwritten by tile j+2
+      uint8_t* drow = sm + Cf::OFF_DS + s * Cf::DSB + r * 128;
 #pragma unroll
-      for (int c = 0; c < Cf::BN / 32; ++c) {
-        uint32_t sr[32], dr[32];
-        tmem_ld32_nowait(tmem + lane_base + Cf::S_COL + c * 32, sr);
-        tmem_ld32_nowait(tmem + lane_base + Cf::DP_COL + c * 32, dr);
-        tmem_ld_wait();
-        float ds[32];
+      for (int cc = 0; cc < 8; ++cc) {
+        float ds[8];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float pr = ex2_tc(fmaf(__uint_as_float(sr[e]), sc, nL));
+        for (int e = 0; e < 8; ++e) {
+          const int c = cc * 8 + e;
+          float pr = ex2_tc(fmaf(__uint_as_float(sr[c]), sc, nL));
           if (need_mask) {
-            const uint32_t off = (uint32_t)(j0 + c * 32 + e - lo_key);
+            const uint32_t off = (uint32_t)(j0 + c - lo_key);
             pr = off <= span ? pr : 0.f;
           }
-          ds[e] = pr * (__uint_as_float(dr[e]) - Dr);
+          ds[e] = pr * (__uint_as_float(dr[c]) - Dr);
         }
-        const int kb = c >> 1;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int cc = (c & 1) * 4 + q;
-          *(uint4*)(drow + kb * (Cf::BM * 128) + ((cc ^ (r & 7)) << 4)) =
-              make_uint4(pack_bf16x2(ds[8 * q], ds[8 * q + 1]), pack_bf16x2(ds[8 * q + 2], ds[8 * q + 3]),
-                         pack_bf16x2(ds[8 * q + 4], ds[8 * q + 5]), pack_bf16x2(ds[8 * q + 6], ds[8 * q + 7]));
-        }
+        *(uint4*)(drow + ((cc ^ (r & 7)) << 4)) =
+            make_uint4(pack_bf16x2(ds[0], ds[1]), pack_bf16x2(ds[2], ds[3]), pack_bf16x2(ds[4], ds[5]),
+                       pack_bf16x2(ds[6], ds[7]));
       }
-      tc_fence_before();
       fence_proxy_async();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(st_free);
-        mbar_arrive(ds_full);
-      }
+      if (lane == 0) mbar_arrive(&ds_full[s]);
     }
     if (ok && mbar_wait(dq_done, 0, err, DEV_TIMEOUT_ACC)) {
       tc_fence_after();

@@ -219,4 +219,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
 
 __device__ __forceinline__ int elect_lane0() { return (threadIdx.x & 31) == 0; }
 
+// Programmatic dependent launch. A kernel launched with the programmatic
+// stream-serialisation attribute may start before its predecessor in the stream
+// has finished; pdl_wait() blocks until that predecessor grid has completed and
+// its memory is visible (a no-op for a normally launched kernel), so every thread
+// calls it before its first global-memory access. pdl_trigger() lets the next
+// such kernel in the stream begin launching (its blocks then wait in pdl_wait).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 }  // namespace ttt

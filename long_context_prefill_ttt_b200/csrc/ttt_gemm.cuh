@@ -25,7 +25,7 @@ enum EpiKind : int {
   EPI_GELU = 2,    // Y = acc (if Y), D = gelu(acc)        (element type)
   EPI_DGELU = 3,   // D = acc * gelu'(X)                   (element type, X element type)
   EPI_SGD = 4,     // D(f32) += acc, Y = D (if Y)          (alpha = -eta)
-  EPI_QKV_ROPE = 5,  // D = acc (element type) with RoPE applied to columns [0, rope_cols)
+  EPI_QKV_ROPE = 5,  // D = acc (element type), then RoPE on columns [0, rope_cols) by a separate pass
 };
 
 struct GemmParams {
@@ -42,7 +42,7 @@ struct GemmParams {
   void* Y; int64_t ldy, sY;
   float alpha;
   int epi;
-  // EPI_QKV_ROPE: rotate pairs (i, i + hd/2) of each head in columns [0, rope_cols) of row m at
+  // EPI_QKV_ROPE: after the product, rotate pairs (i, i + hd/2) of each head in columns [0, rope_cols) of row m at
   // position rope_pos0 + (m % rope_n) (rope_pos0 read from *rope_pos_dev when given), angles
   // pos * base^(-2i/hd) from the double-precision tables lo[p & 1023][i], hi[p >> 10][i].
   const float2* rope_lo; const float2* rope_hi;
@@ -137,6 +137,61 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmParams p) {
       const int m = m0 + ty * 4 + i, n = n0 + tx * 4 + j;
       if (m < p.M && n < p.N) epi_apply<T>(p, z, m, n, acc[i][j]);
     }
+}
+
+// ============================================================== skinny engine (decode)
+// At most 16 rows per batch slice (one row per sequence in decode): the work is
+// reading the weight matrix once, so one warp per output column streams its
+// weight row (and the per-sequence update row for the W_init + dW operand) with
+// 16-byte loads across all SMs; the few activation rows come from L1. K-major
+// operands only; the epilogue is the shared per-element one.
+constexpr int SK_MAXM = 16;
+template <typename T>
+__global__ void __launch_bounds__(256) gemm_skinny_kernel(GemmParams p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = blockIdx.x * 8 + warp;
+  const int z = blockIdx.y;
+  if (n >= p.N) return;
+  constexpr int VEC = 16 / sizeof(T);
+  const T* A = (const T*)p.A + (int64_t)z * p.sA;
+  const T* Bw = (const T*)p.B + (int64_t)z * p.sB + (int64_t)n * p.ldb;
+  const T* B2w = p.B2 ? (const T*)p.B2 + (int64_t)z * p.sB2 + (int64_t)n * p.ldb : nullptr;
+  float acc[SK_MAXM];
+#pragma unroll
+  for (int m = 0; m < SK_MAXM; ++m) acc[m] = 0.f;
+  for (int k0 = lane * VEC; k0 < p.K; k0 += 32 * VEC) {
+    float w[VEC];
+    {
+      const uint4 u = *reinterpret_cast<const uint4*>(Bw + k0);
+      const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) w[i] = to_f32(e[i]);
+    }
+    if (B2w) {
+      const uint4 u = *reinterpret_cast<const uint4*>(B2w + k0);
+      const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) w[i] += to_f32(e[i]);
+    }
+#pragma unroll
+    for (int m = 0; m < SK_MAXM; ++m) {
+      if (m < p.M) {
+        const uint4 u = *reinterpret_cast<const uint4*>(A + (int64_t)m * p.lda + k0);
+        const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) acc[m] = fmaf(to_f32(e[i]), w[i], acc[m]);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < SK_MAXM; ++m) {
+    if (m < p.M) {
+      float v = acc[m];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0) epi_apply<T>(p, z, m, n, v);
+    }
+  }
 }
 
 // ============================================================== tcgen05 engine
@@ -268,6 +323,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();     // operands and epilogue inputs come from the previous kernel
+  pdl_trigger();
 
   if (warp == 0) {
     if (elect_lane0()) {
@@ -352,50 +409,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_after();
       const int m = m0 + row_in_tile;
       const uint32_t taddr = tmem_base + acc * BN + ((uint32_t)(quarter * 32) << 16);
-      if (p.epi == EPI_QKV_ROPE && n0 < p.rope_cols) {
-        // chunks come in pairs (c, c + hd/64): the two halves of each head
-        const int half_chunks = p.rope_hd / 64;
-        const int64_t pos = (p.rope_pos_dev ? *p.rope_pos_dev : p.rope_pos0) + (m % p.rope_n);
-        const int hh = p.rope_hd / 2;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          if ((c / half_chunks) & 1) continue;  // second half of a head: done with its partner
-          float v1[32], v2[32];
-          tmem_ld32(taddr + c * 32, v1);
-          tmem_ld32(taddr + (c + half_chunks) * 32, v2);
-          if (m < p.M) {
-            const int i0 = (c % half_chunks) * 32;  // pair index of v1[0] within the head
-#pragma unroll 4
-            for (int e = 0; e < 32; ++e) {
-              const float2 a = p.rope_lo[(pos & 1023) * hh + i0 + e];
-              const float2 bq = p.rope_hi[(pos >> 10) * hh + i0 + e];
-              const float cs = a.x * bq.x - a.y * bq.y, sn = a.y * bq.x + a.x * bq.y;
-              const float x1 = v1[e] * p.alpha, x2 = v2[e] * p.alpha;
-              v1[e] = x1 * cs - x2 * sn;
-              v2[e] = x2 * cs + x1 * sn;
-            }
-            GemmParams q = p;
-            q.epi = EPI_STORE;
-            q.alpha = 1.f;
-            epi_row32<bf16>(q, z, m, n0 + c * 32, v1);
-            epi_row32<bf16>(q, z, m, n0 + (c + half_chunks) * 32, v2);
-          }
-        }
-      } else {
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          float v[32];
-          tmem_ld32(taddr + c * 32, v);
-          if (m < p.M) {
-            if (p.epi == EPI_QKV_ROPE) {
-              GemmParams q = p;
-              q.epi = EPI_STORE;
-              epi_row32<bf16>(q, z, m, n0 + c * 32, v);
-            } else {
-              epi_row32<bf16>(p, z, m, n0 + c * 32, v);
-            }
-          }
-        }
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(taddr + c * 32, v);
+        if (m < p.M) epi_row32<bf16>(p, z, m, n0 + c * 32, v);
       }
       tc_fence_before();
       __syncwarp();

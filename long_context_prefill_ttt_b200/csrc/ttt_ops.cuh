@@ -33,6 +33,8 @@ template <typename T>
 __global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, int64_t ldx, const float* __restrict__ g,
                                    float eps, int rows, int d, T* __restrict__ y, int64_t ldy,
                                    float* __restrict__ rstd_out) {
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -62,6 +64,8 @@ template <typename T>
 __global__ void rmsnorm_bwd_kernel(const float* __restrict__ x, const float* __restrict__ g,
                                    const float* __restrict__ rstd, const float* __restrict__ dy,
                                    const float* dres, int rows, int d, float* dx, T* __restrict__ dx_t) {
+  pdl_wait();
+  pdl_trigger();
   const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -161,46 +165,58 @@ __global__ void kv_append_kernel(const T* __restrict__ src, int64_t ld, int kcol
 }
 
 // ---------------------------------------------------------------- cross entropy
-// One CTA per row of logits z [rows][V]. loss = logsumexp(z) - z[target].
-// If grad_scale != 0, z is overwritten in place by dz = (softmax(z) - onehot) * grad_scale.
-// Row r belongs to sequence r / n at chunk offset r % n; its loss goes to
-// loss_out[(r / n) * loss_ld + loss_off + r % n] (skipped when loss_out is null).
+// One CTA per row of logits z [rows][V] (V % (16 / sizeof(T)) == 0).
+// loss = logsumexp(z) - z[target], from one pass of 16-byte loads keeping a
+// running (max, sum of exp) per thread, merged across the block. If
+// grad_scale != 0, z is overwritten in place by dz = (softmax(z) - onehot) *
+// grad_scale in a second vectorised pass. Row r belongs to sequence r / n at
+// chunk offset r % n; its loss goes to loss_out[(r / n) * loss_ld + loss_off + r % n]
+// (skipped when loss_out is null).
+__device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2) {
+  const float M = fmaxf(m, m2);
+  if (M == -INFINITY) return;
+  s = s * expf(m - M) + s2 * expf(m2 - M);
+  m = M;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ z, int V, const int32_t* __restrict__ targets,
                                                  int n, float* loss_out, int64_t loss_ld, int64_t loss_off,
                                                  float grad_scale, int* err) {
+  constexpr int VEC = 16 / sizeof(T);
   const int row = blockIdx.x;
   T* zr = z + (int64_t)row * V;
-  __shared__ float red[32];
-  __shared__ float bc[2];
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
-  float mx = -INFINITY;
-  for (int c = tid; c < V; c += blockDim.x) mx = fmaxf(mx, to_f32(zr[c]));
+  __shared__ float sm_m[8], sm_s[8];
+  __shared__ float bc[1];
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  float m = -INFINITY, sum = 0.f;
+  for (int c = tid * VEC; c < V; c += 256 * VEC) {
+    const uint4 u = *reinterpret_cast<const uint4*>(zr + c);
+    const T* e = reinterpret_cast<const T*>(&u);
+    float x[VEC], mv = -INFINITY;
 #pragma unroll
-  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) red[w] = mx;
+    for (int i = 0; i < VEC; ++i) { x[i] = to_f32(e[i]); mv = fmaxf(mv, x[i]); }
+    const float M = fmaxf(m, mv);
+    float add = 0.f;
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) add += expf(x[i] - M);
+    sum = (m == -INFINITY ? 0.f : sum * expf(m - M)) + add;
+    m = M;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, sum, o);
+    lse_merge(m, sum, m2, s2);
+  }
+  if (lane == 0) { sm_m[w] = m; sm_s[w] = sum; }
   __syncthreads();
   if (tid == 0) {
-    float m = red[0];
-    for (int i = 1; i < nw; ++i) m = fmaxf(m, red[i]);
-    bc[0] = m;
+    float M = sm_m[0], S = sm_s[0];
+    for (int i = 1; i < 8; ++i) lse_merge(M, S, sm_m[i], sm_s[i]);
+    bc[0] = M + logf(S);
   }
   __syncthreads();
-  mx = bc[0];
-  float se = 0.f;
-  for (int c = tid; c < V; c += blockDim.x) se += expf(to_f32(zr[c]) - mx);
-#pragma unroll
-  for (int o = 16; o; o >>= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
-  __syncthreads();
-  if (lane == 0) red[w] = se;
-  __syncthreads();
-  if (tid == 0) {
-    float s = 0.f;
-    for (int i = 0; i < nw; ++i) s += red[i];
-    bc[1] = mx + logf(s);
-  }
-  __syncthreads();
-  const float lse = bc[1];
+  const float lse = bc[0];
   int t = targets[row];
   if (t < 0 || t >= V) {  // ids are validated here too: the last target of a call is never embedded
     if (tid == 0) set_error(err, DEV_BAD_TOKEN);
@@ -212,9 +228,15 @@ __global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ z, int V, const
   }
   if (grad_scale != 0.f) {
     __syncthreads();  // every thread has read zr[t] before it is overwritten
-    for (int c = tid; c < V; c += blockDim.x) {
-      const float p = expf(to_f32(zr[c]) - lse);
-      zr[c] = from_f32<T>((p - (c == t ? 1.f : 0.f)) * grad_scale);
+    for (int c = tid * VEC; c < V; c += 256 * VEC) {
+      uint4 u = *reinterpret_cast<const uint4*>(zr + c);
+      T* e = reinterpret_cast<T*>(&u);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) {
+        const float p = expf(to_f32(e[i]) - lse);
+        e[i] = from_f32<T>((p - (c + i == t ? 1.f : 0.f)) * grad_scale);
+      }
+      *reinterpret_cast<uint4*>(zr + c) = u;
     }
   }
 }

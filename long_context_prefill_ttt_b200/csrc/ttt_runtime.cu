@@ -31,6 +31,25 @@
 
 namespace ttt {
 
+// ============================================================== launch helper
+// Launch with programmatic stream serialisation (the kernel must call pdl_wait()
+// before touching global memory; see ttt_common.cuh).
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // ============================================================== GEMM dispatch (host)
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -88,8 +107,7 @@ static cudaError_t launch_tc(const GemmParams& p, cudaStream_t st, int* err, int
   using C = TcCfg<BN>;
   const int tiles = ((p.M + TC_BM - 1) / TC_BM) * (p.N / BN) * p.batch;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  gemm_tc_kernel<BN, AM, BM><<<grid, TC_THREADS, C::SMEM, st>>>(ta, tb, tb2, p, err);
-  return cudaGetLastError();
+  return launch_pdl(gemm_tc_kernel<BN, AM, BM>, dim3(grid), dim3(TC_THREADS), C::SMEM, st, ta, tb, tb2, p, err);
 }
 
 // ============================================================== tcgen05 attention (host)
@@ -99,13 +117,13 @@ bool attn_tc_ok(const AttnParams& p) {
          aligned16(p.Q) && (p.q0 == 0 || (aligned16(p.Kc) && aligned16(p.Vc))) && p.n >= 1;
 }
 
-// Rows of 'inner' bf16 elements, 'rows' rows, box {64, 128}, 128-byte swizzle.
-static bool make_rows_map(CUtensorMap* map, const void* base, int64_t inner, int64_t rows) {
+// Rows of 'inner' bf16 elements, 'rows' rows, box {64, box_rows}, 128-byte swizzle.
+static bool make_rows_map(CUtensorMap* map, const void* base, int64_t inner, int64_t rows, int box_rows = 128) {
   EncodeTiledFn enc = get_encode();
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, 1};
   cuuint64_t strides[2] = {(cuuint64_t)inner * 2, (cuuint64_t)(inner * rows * 2)};
-  cuuint32_t box[3] = {64, 128, 1}, estr[3] = {1, 1, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1}, estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -123,11 +141,8 @@ cudaError_t attn_fwd_tc_launch(const AttnParams& p, cudaStream_t st, int* err, b
   }
   if (!*ok) return cudaSuccess;
   dim3 grid((p.n + 127) / 128, p.H, p.B);
-  if (p.hd == 128)
-    attn_fwd_tc_kernel<128><<<grid, 192, AttnTcCfg<128>::SMEM, st>>>(tq, tk, tv, p, err);
-  else
-    attn_fwd_tc_kernel<64><<<grid, 192, AttnTcCfg<64>::SMEM, st>>>(tq, tk, tv, p, err);
-  return cudaGetLastError();
+  if (p.hd == 128) return launch_pdl(attn_fwd_tc_kernel<128>, grid, dim3(192), AttnTcCfg<128>::SMEM, st, tq, tk, tv, p, err);
+  return launch_pdl(attn_fwd_tc_kernel<64>, grid, dim3(192), AttnTcCfg<64>::SMEM, st, tq, tk, tv, p, err);
 }
 
 bool attn_dq_tc_ok(const AttnParams& p) {
@@ -135,21 +150,24 @@ bool attn_dq_tc_ok(const AttnParams& p) {
 }
 
 cudaError_t attn_bwd_dq_tc_launch(const AttnParams& p, cudaStream_t st, int* err, bool* ok) {
-  CUtensorMap tq, tk, tv, tdo;
-  *ok = make_rows_map(&tq, p.Q, 3 * p.d, (int64_t)p.B * p.n) && make_rows_map(&tdo, p.dO, p.d, (int64_t)p.B * p.n);
+  CUtensorMap tq, tkv, tk, tv, tdo;  // Q and dO in 128-row boxes, K and V in 64-row boxes
+  *ok = make_rows_map(&tq, p.Q, 3 * p.d, (int64_t)p.B * p.n) &&
+        make_rows_map(&tkv, p.Q, 3 * p.d, (int64_t)p.B * p.n, 64) &&
+        make_rows_map(&tdo, p.dO, p.d, (int64_t)p.B * p.n);
   if (*ok && p.q0 > 0) {
-    *ok = make_rows_map(&tk, p.Kc, p.d, (int64_t)p.B * p.C) && make_rows_map(&tv, p.Vc, p.d, (int64_t)p.B * p.C);
+    *ok = make_rows_map(&tk, p.Kc, p.d, (int64_t)p.B * p.C, 64) &&
+          make_rows_map(&tv, p.Vc, p.d, (int64_t)p.B * p.C, 64);
   } else {
-    tk = tq;
-    tv = tq;
+    tk = tkv;
+    tv = tkv;
   }
   if (!*ok) return cudaSuccess;
   dim3 grid((p.n + 127) / 128, p.H, p.B);
   if (p.hd == 128)
-    attn_bwd_dq_tc_kernel<128><<<grid, 192, AttnDqCfg<128>::SMEM, st>>>(tq, tk, tv, tdo, p, err);
-  else
-    attn_bwd_dq_tc_kernel<64><<<grid, 192, AttnDqCfg<64>::SMEM, st>>>(tq, tk, tv, tdo, p, err);
-  return cudaGetLastError();
+    return launch_pdl(attn_bwd_dq_tc_kernel<128>, grid, dim3(192), AttnDqCfg<128>::SMEM, st, tq, tkv, tk, tv, tdo,
+                      p, err);
+  return launch_pdl(attn_bwd_dq_tc_kernel<64>, grid, dim3(192), AttnDqCfg<64>::SMEM, st, tq, tkv, tk, tv, tdo, p,
+                    err);
 }
 
 // Dynamic shared-memory limits of every large-smem kernel, set once per process
@@ -183,6 +201,32 @@ int prime_kernel_attributes() {
 // Returns 0 on success, or a cudaError_t value.
 int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err, int num_sms, int force_simt) {
   if (p.M <= 0 || p.N <= 0 || p.K <= 0 || p.batch <= 0) return 0;
+  // few rows per slice (decode): skinny kernel, all SMs streaming the weight rows
+  const size_t vec = elem_is_bf16 ? 8 : 4;
+  if (!force_simt && p.M <= SK_MAXM && !p.a_mn && !p.b_mn && p.K % vec == 0 && p.lda % vec == 0 &&
+      p.ldb % vec == 0 && aligned16(p.A) && aligned16(p.B) && (!p.B2 || aligned16(p.B2)) &&
+      (p.batch == 1 || (p.sA % vec == 0 && p.sB % vec == 0 && p.sB2 % vec == 0))) {
+    GemmParams q = p;
+    if (p.epi == EPI_QKV_ROPE) q.epi = EPI_STORE;
+    dim3 grid((p.N + 7) / 8, p.batch);
+    if (elem_is_bf16)
+      gemm_skinny_kernel<bf16><<<grid, 256, 0, st>>>(q);
+    else
+      gemm_skinny_kernel<float><<<grid, 256, 0, st>>>(q);
+    if (p.epi == EPI_QKV_ROPE) {
+      const int64_t work = (int64_t)p.M * (p.rope_cols / 2);
+      const unsigned blocks = (unsigned)((work + 255) / 256);
+      if (elem_is_bf16)
+        rope_kernel<bf16><<<blocks, 256, 0, st>>>((bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0,
+                                                   p.rope_hd, p.rope_lo, p.rope_hi, 0, p.rope_pos_dev);
+      else
+        rope_kernel<float><<<blocks, 256, 0, st>>>((float*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0,
+                                                    p.rope_hd, p.rope_lo, p.rope_hi, 0, p.rope_pos_dev);
+    }
+    return (int)cudaGetLastError();
+  }
+  GemmParams pt = p;  // tensor-core launch: the rotation of EPI_QKV_ROPE runs as a separate pass
+  if (p.epi == EPI_QKV_ROPE) pt.epi = EPI_STORE;
   bool use_tc = elem_is_bf16 && !force_simt && (p.K % TC_BK == 0) && (p.N % 128 == 0) && aligned16(p.A) &&
                 aligned16(p.B) && aligned16(p.D) && (p.lda % 8 == 0) && (p.ldb % 8 == 0) &&
                 (p.ldd % (p.d_f32 || p.epi == EPI_RESID || p.epi == EPI_SGD ? 4 : 8) == 0) &&
@@ -193,30 +237,36 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
     use_tc = false;
   if (use_tc && p.batch > 1 && p.sD % 8 != 0) use_tc = false;
   if (use_tc && p.Y && !(aligned16(p.Y) && p.ldy % 8 == 0 && (p.batch == 1 || p.sY % 8 == 0))) use_tc = false;
-  if (p.epi == EPI_QKV_ROPE &&
-      !(p.rope_hd == 64 || p.rope_hd == 128) ) use_tc = false;
-  // no tile may straddle the end of the rotated columns: rope_cols a multiple of the widest tile
-  if (use_tc && p.epi == EPI_QKV_ROPE && (p.batch != 1 || p.rope_cols % 256 != 0)) use_tc = false;
   if (use_tc) {
-    // tile width: the one whose tile count fills the persistent grid's waves best
-    // (fraction of CTA slots busy over ceil(tiles / SMs) waves); ties go to 256
+    // tile width: 256 (fewer A re-reads, longer MMAs) unless 128-wide tiles fill the
+    // persistent grid's waves clearly better (fraction of CTA slots busy over
+    // ceil(tiles / SMs) waves, by more than 5 points: small-M shapes)
     const int m_tiles = (p.M + TC_BM - 1) / TC_BM;
     auto wave_eff = [&](int bn) {
       const double t = (double)m_tiles * (p.N / bn) * p.batch;
       const double waves = std::ceil(t / num_sms);
       return t / (waves * num_sms);
     };
-    const bool n256 = (p.N % 256 == 0) && wave_eff(256) >= wave_eff(128) - 1e-9;
+    const bool n256 = (p.N % 256 == 0) && wave_eff(256) + 0.05 >= wave_eff(128);
     bool ok = false;
     cudaError_t e;
     if (!p.a_mn && !p.b_mn)
-      e = n256 ? launch_tc<256, false, false>(p, st, err, num_sms, &ok) : launch_tc<128, false, false>(p, st, err, num_sms, &ok);
+      e = n256 ? launch_tc<256, false, false>(pt, st, err, num_sms, &ok) : launch_tc<128, false, false>(pt, st, err, num_sms, &ok);
     else if (!p.a_mn && p.b_mn)
-      e = n256 ? launch_tc<256, false, true>(p, st, err, num_sms, &ok) : launch_tc<128, false, true>(p, st, err, num_sms, &ok);
+      e = n256 ? launch_tc<256, false, true>(pt, st, err, num_sms, &ok) : launch_tc<128, false, true>(pt, st, err, num_sms, &ok);
     else
-      e = n256 ? launch_tc<256, true, true>(p, st, err, num_sms, &ok) : launch_tc<128, true, true>(p, st, err, num_sms, &ok);
+      e = n256 ? launch_tc<256, true, true>(pt, st, err, num_sms, &ok) : launch_tc<128, true, true>(pt, st, err, num_sms, &ok);
     if (e != cudaSuccess) return (int)e;
-    if (ok) return 0;
+    if (ok) {
+      if (p.epi == EPI_QKV_ROPE) {
+        const int64_t work = (int64_t)p.M * (p.rope_cols / 2);
+        rope_kernel<bf16><<<(unsigned)((work + 255) / 256), 256, 0, st>>>(
+            (bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd, p.rope_lo, p.rope_hi, 0,
+            p.rope_pos_dev);
+        return (int)cudaGetLastError();
+      }
+      return 0;
+    }
   }
   dim3 grid((p.N + 63) / 64, (p.M + 63) / 64, p.batch);
   GemmParams q = p;
@@ -744,7 +794,7 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
                                T* o, float* lse, int n, int64_t q0, bool commit) {
   const int rows = B * n;
   int rc;
-  rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(xin, d, Lw.g_attn, cfg.rms_eps, rows, d, r, d, rstd);
+  launch_pdl(rmsnorm_fwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)xin, d, Lw.g_attn, cfg.rms_eps, rows, d, r, d, rstd);
   TTT_LAUNCHED();
   {  // q|k|v = r Wqkv^T with RoPE applied to q and k in the GEMM epilogue
     GemmParams pq = gp(rows, 3 * d, d, r, d, false, Lw.Wqkv, d, false, qkv, 3 * d, false, EPI_QKV_ROPE);
@@ -816,7 +866,7 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
 // x += W2 gelu(W1 RMSNorm(x)) (frozen blocks)
 template <typename T> int Engine<T>::frozen_mlp(const LayerDev<T>& Lw, float* x, T* r, T* hid, int rows) {
   int rc;
-  rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(x, d, Lw.g_mlp, cfg.rms_eps, rows, d, r, d, nullptr);
+  launch_pdl(rmsnorm_fwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)x, d, Lw.g_mlp, cfg.rms_eps, rows, d, r, d, nullptr);
   TTT_LAUNCHED();
   if ((rc = gemm(gp(rows, h, d, r, d, false, Lw.W1, d, false, hid, h, false, EPI_GELU))) != TTT_OK) return rc;
   GemmParams p = gp(rows, d, h, hid, h, false, Lw.W2, h, false, x, d, true, EPI_RESID);
@@ -837,7 +887,7 @@ template <typename T> int Engine<T>::ttt_forward(int cn, int64_t pos, bool commi
                               commit)) != TTT_OK)
       return rc;
     // TTT-MLP with the fast weights of each sequence (batched over sequences)
-    rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(A.a, d, Lw.g_ttt, cfg.rms_eps, rows, d, A.r2, d, A.rstd2);
+    launch_pdl(rmsnorm_fwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)A.a, d, Lw.g_ttt, cfg.rms_eps, rows, d, A.r2, d, A.rstd2);
     TTT_LAUNCHED();
     GemmParams p = gp(cn, ht, d, A.r2, d, false, Lw.W1t, d, false, A.g, ht, false, EPI_GELU);
     p.batch = B; p.sA = (int64_t)cn * d; p.sD = (int64_t)cn * ht;
@@ -850,7 +900,7 @@ template <typename T> int Engine<T>::ttt_forward(int cn, int64_t pos, bool commi
     p.X = A.a; p.ldx = d; p.sX = (int64_t)cn * d;
     if ((rc = gemm(p)) != TTT_OK) return rc;
     // static MLP
-    rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(A.m, d, Lw.g_static, cfg.rms_eps, rows, d, A.r3, d,
+    launch_pdl(rmsnorm_fwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)A.m, d, Lw.g_static, cfg.rms_eps, rows, d, A.r3, d,
                                                          A.rstd3);
     TTT_LAUNCHED();
     p = gp(rows, hs, d, A.r3, d, false, Lw.W1s, d, false, A.gs, hs, false, EPI_GELU);
@@ -871,7 +921,7 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
   int rc;
   // LM head: dr = dz E ; G = d loss / d y through the final RMSNorm
   if ((rc = gemm(gp(rows, d, V, z, V, false, E, d, true, dr, d, true, EPI_STORE))) != TTT_OK) return rc;
-  rmsnorm_bwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(y, g_final, rstdf, dr, nullptr, rows, d, G, GT);
+  launch_pdl(rmsnorm_bwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)y, g_final, rstdf, dr, nullptr, rows, d, G, GT);
   TTT_LAUNCHED();
   for (int j = Lt - 1; j >= 0; --j) {
     const int l = first_ttt + j;
@@ -882,7 +932,7 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
     p.X = A.us; p.ldx = hs;
     if ((rc = gemm(p)) != TTT_OK) return rc;
     if ((rc = gemm(gp(rows, d, hs, dhid, hs, false, Lw.W1s, d, true, dr, d, true, EPI_STORE))) != TTT_OK) return rc;
-    rmsnorm_bwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(A.m, Lw.g_static, A.rstd3, dr, G, rows, d, G, GT);
+    launch_pdl(rmsnorm_bwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)A.m, Lw.g_static, A.rstd3, dr, G, rows, d, G, GT);
     TTT_LAUNCHED();
     // TTT-MLP data gradients (with W_{i-1}), then the fused weight gradient + SGD
     p = gp(cn, ht, d, GT, d, false, Lw.W2t, ht, true, dhid, ht, false, EPI_DGELU);
@@ -910,7 +960,7 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
     if (is_bf16) { p.Y = Lw.W1t; p.ldy = d; p.sY = (int64_t)ht * d; }
     if ((rc = gemm(p)) != TTT_OK) return rc;
     if (j == 0) break;  // upstream of the first adaptive MLP does not depend on the fast weights
-    rmsnorm_bwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(A.a, Lw.g_ttt, A.rstd2, dr, G, rows, d, G, GT);
+    launch_pdl(rmsnorm_bwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)A.a, Lw.g_ttt, A.rstd2, dr, G, rows, d, G, GT);
     TTT_LAUNCHED();
     // frozen attention: data gradients only; cached K/V are constants
     if ((rc = gemm(gp(rows, d, d, GT, d, false, Lw.Wo, d, true, dob, d, false, EPI_STORE))) != TTT_OK) return rc;
@@ -955,7 +1005,7 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
     if ((rc = gemm(gp(rows, d, 3 * d, dqkv, 3 * d, false, Lw.Wqkv, d, true, dr, d, true, EPI_STORE))) != TTT_OK)
       return rc;
     // G <- G + RMSNorm_bwd through the attention norm: gradient w.r.t. this block's input
-    rmsnorm_bwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(A.x, Lw.g_attn, A.rstd1, dr, G, rows, d, G, GT);
+    launch_pdl(rmsnorm_bwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)A.x, Lw.g_attn, A.rstd1, dr, G, rows, d, G, GT);
     TTT_LAUNCHED();
   }
   return TTT_OK;
@@ -981,7 +1031,7 @@ int Engine<T>::ttt_step(const float* in, const int32_t* targets, int cn, int64_t
     TTT_CUDA(cudaMemcpyAsync(tgt, targets, (size_t)rows * 4, cudaMemcpyDeviceToDevice, st));
   }
   if ((rc = ttt_forward(cn, pos, commit)) != TTT_OK) return rc;
-  rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf);
+  launch_pdl(rmsnorm_fwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf);
   TTT_LAUNCHED();
   if ((rc = gemm(gp(rows, V, d, rf, d, false, E, d, false, z, V, false, EPI_STORE))) != TTT_OK) return rc;
   // mean over the b positions of the chunk (summary: mini-batch GD with 1/b)
@@ -1085,7 +1135,7 @@ template <typename T> int Engine<T>::decode_token_launches(int64_t n, int32_t* o
   TTT_CUDA(cudaMemcpyAsync(blk[0].x, xs, (size_t)B * d * 4, cudaMemcpyDeviceToDevice, st));
   gemm_class = PC_GEMM_TTT;
   if ((rc = ttt_forward(1, 0, true)) != TTT_OK) return rc;
-  rmsnorm_fwd_kernel<T><<<nblk(rows, 4), 128, 0, st>>>(y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf);
+  launch_pdl(rmsnorm_fwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf);
   TTT_LAUNCHED();
   if ((rc = gemm(gp(rows, V, d, rf, d, false, E, d, false, z, V, false, EPI_STORE))) != TTT_OK) return rc;
   const int32_t* fcol = nullptr;

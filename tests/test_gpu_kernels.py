@@ -192,3 +192,28 @@ def test_attention_forward_and_backward(T, engine, dtype, B, H, hd, n, q0, windo
         scale = ref.abs().max().item() + 1e-12
         err = (got.double().view(B, n, H, hd) - ref).abs().max().item() / scale
         assert err < (1e-5 if dtype == torch.float32 else 3e-2), err
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("M,N,K,batch", [(1, 768, 768, 8), (8, 2304, 768, 1), (16, 384, 3072, 2), (8, 32000, 768, 1)])
+def test_skinny_gemm_rows_per_sequence(T, dtype, M, N, K, batch):
+    """Decode-sized products (<= 16 rows per slice): shared W plus per-slice dW, residual and GELU epilogues."""
+    A = _rand((batch, M, K), dtype, 31)
+    Bs = _rand((1, N, K), dtype, 32, 0.05)
+    B2 = _rand((batch, N, K), dtype, 33, 1e-3)
+    ref = A.double() @ (Bs.double() + B2.double()).transpose(1, 2)
+    tol = 1e-5 if dtype == torch.float32 else 1e-2
+    R = _rand((batch, M, N), torch.float32, 34)
+    D = R.clone()
+    T.ttt_k_gemm(A, Bs, D, M, N, K, batch=batch, sA=M * K, sB=0, B2=B2, sB2=N * K, sD=M * N, X=D, ldx=N, sX=M * N,
+                 epi=T.EPI_RESID)
+    T.ttt_k_status()
+    assert (D.double() - (ref + R.double())).abs().max().item() <= tol * ref.abs().max().item()
+    G = torch.empty((batch, M, N), dtype=dtype, device="cuda")
+    U = torch.empty((batch, M, N), dtype=dtype, device="cuda")
+    T.ttt_k_gemm(A, Bs, G, M, N, K, batch=batch, sA=M * K, sB=0, B2=B2, sB2=N * K, sD=M * N, Y=U, ldy=N, sY=M * N,
+                 epi=T.EPI_GELU)
+    T.ttt_k_status()
+    assert torch.allclose(U.double(), ref, rtol=2 * tol, atol=2 * tol * ref.abs().max().item())
+    assert torch.allclose(G.double(), torch.nn.functional.gelu(ref, approximate="none"), rtol=2 * tol,
+                          atol=2 * tol * ref.abs().max().item())
