@@ -508,11 +508,12 @@ template <int HD> inline cudaError_t attn_fwd_mma_launch(const AttnParams& p, cu
   return cudaGetLastError();
 }
 
-template <int HD> inline cudaError_t attn_bwd_mma_launch(const AttnParams& p, cudaStream_t st, bool with_dq = true) {
+template <int HD>
+inline cudaError_t attn_bwd_mma_launch(const AttnParams& p, cudaStream_t st, bool with_dq = true, bool with_dkv = true) {
   constexpr int smem = attn_bwd_mma_smem<HD>();
   dim3 grid((p.n + AM_BM - 1) / AM_BM, p.H, p.B);
   if (with_dq) attn_bwd_dq_mma_kernel<HD><<<grid, 128, smem, st>>>(p);
-  attn_bwd_dkv_mma_kernel<HD><<<grid, 128, smem, st>>>(p);
+  if (with_dkv) attn_bwd_dkv_mma_kernel<HD><<<grid, 128, smem, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -559,4 +559,274 @@ __global__ void __launch_bounds__(192, 1)
   }
 }
 
+
+// ---------------------------------------------------------------- backward dK, dV on tcgen05
+// Keys of the current rows only (cached ring keys are constants of the chunk
+// step): one CTA = 128 keys of one (sequence, head) at row offsets [k0, k0+128),
+// over the query blocks of 64 rows that can see them (query i sees key j when
+// 0 <= i - j < window). The roles mirror the dQ kernel with keys as the MMA's M
+// dimension. Per query block j: S^T = K Q_j^T and dP^T = V dO_j^T into one of two
+// TMEM buffers (MMA warp); four warps (one key row each) form P^T = exp(S^T*scale
+// - lse) and dS^T = P^T (dP^T - D) with the per-query lse and D read from shared
+// memory, and write both (bf16) to one of two shared-memory buffers; the MMA warp
+// accumulates dV += P^T dO_j and dK += dS^T Q_j in TMEM (Q_j and dO_j read again as
+// MN-major operands). Query rows past the sequence end get lse = +inf, so their
+// P and dS vanish. dK is scaled by 1/sqrt(hd) on the way out.
+// TMEM: dV [0,HD), dK [128,128+HD), S^T_b [256+128b, 256+128b+64), dP^T_b next 64.
+template <int HD> struct AttnDkvCfg {
+  static constexpr int BK = 128, BQ = 64;
+  static constexpr int QST = 3;                 // Q / dO stages
+  static constexpr int KVB = BK * HD * 2;       // K (and V) tile bytes
+  static constexpr int QB = BQ * HD * 2;        // Q (and dO) block bytes
+  static constexpr int PB = BK * BQ * 2;        // P^T (and dS^T) tile bytes
+  static constexpr int OFF_V = KVB;
+  static constexpr int OFF_Q0 = 2 * KVB;
+  static constexpr int OFF_DO0 = OFF_Q0 + QST * QB;
+  static constexpr int OFF_P0 = OFF_DO0 + QST * QB;
+  static constexpr int OFF_DS0 = OFF_P0 + 2 * PB;
+  static constexpr int OFF_LD = OFF_DS0 + 2 * PB;  // [2][ -lse*log2e (64) | D (64) ] floats
+  static constexpr int OFF_BAR = OFF_LD + 2 * 2 * BQ * 4;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
+  static constexpr uint32_t DV_COL = 0, DK_COL = 128;
+  static __device__ __forceinline__ uint32_t s_col(int b) { return 256 + b * 128; }
+  static __device__ __forceinline__ uint32_t dp_col(int b) { return 256 + b * 128 + 64; }
+};
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+template <int HD>
+__global__ void __launch_bounds__(192, 1)
+    attn_bwd_dkv_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_q,
+                           const __grid_constant__ CUtensorMap tm_do, const AttnParams p, int* err) {
+  using Cf = AttnDkvCfg<HD>;
+  constexpr int KB = HD / 64;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = (uint64_t*)(sm + Cf::OFF_BAR);
+  uint64_t* kv_full = bars;
+  uint64_t* q_full = bars + 1;     // [3]
+  uint64_t* q_empty = bars + 4;    // [3]
+  uint64_t* sp_full = bars + 7;    // [2]
+  uint64_t* sp_free = bars + 9;    // [2]
+  uint64_t* pd_full = bars + 11;   // [2]
+  uint64_t* pd_free = bars + 13;   // [2]
+  uint64_t* acc_done = bars + 15;
+  uint32_t* tmem_slot = (uint32_t*)(bars + 16);
+  float* ldbuf = (float*)(sm + Cf::OFF_LD);
+
+  const int warp = threadIdx.x >> 5;
+  const int kblk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int k0 = kblk * Cf::BK;                       // first key row (offset within the rows)
+  const int nk = min(Cf::BK, p.n - k0);
+  const int qlast = (int)min((int64_t)p.n - 1, (int64_t)k0 + Cf::BK - 1 + p.window - 1);
+  const int qb0 = k0 / Cf::BQ;
+  const int nqb = qlast / Cf::BQ - qb0 + 1;           // >= 1: the key block's own rows see it
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < Cf::QST; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&sp_full[s], 1); mbar_init(&sp_free[s], 4);
+      mbar_init(&pd_full[s], 4); mbar_init(&pd_free[s], 1);
+    }
+    mbar_init(acc_done, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tm_k); prefetch_tmap(&tm_q); prefetch_tmap(&tm_do);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
+
+  if (warp == 0) {
+    if (elect_lane0()) {
+      const int krow = b * p.n + k0;
+      mbar_arrive_expect_tx(kv_full, 2 * Cf::KVB);
+      for (int kb = 0; kb < KB; ++kb) {
+        tma_load_3d(sm + kb * Cf::BK * 128, &tm_k, kv_full, p.d + h * HD + kb * 64, krow, 0);
+        tma_load_3d(sm + Cf::OFF_V + kb * Cf::BK * 128, &tm_k, kv_full, 2 * p.d + h * HD + kb * 64, krow, 0);
+      }
+      for (int j = 0; j < nqb; ++j) {
+        const int st = j % Cf::QST, use = j / Cf::QST;
+        if (!mbar_wait(&q_empty[st], (use & 1) ^ 1, err, DEV_TIMEOUT_EMPTY)) break;
+        mbar_arrive_expect_tx(&q_full[st], 2 * Cf::QB);
+        const int qrow = b * p.n + (qb0 + j) * Cf::BQ;
+        for (int kb = 0; kb < KB; ++kb) {
+          tma_load_3d(sm + Cf::OFF_Q0 + st * Cf::QB + kb * Cf::BQ * 128, &tm_q, &q_full[st], h * HD + kb * 64, qrow, 0);
+          tma_load_3d(sm + Cf::OFF_DO0 + st * Cf::QB + kb * Cf::BQ * 128, &tm_do, &q_full[st], h * HD + kb * 64, qrow,
+                      0);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_lane0()) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, Cf::BQ, false, false);
+      constexpr uint32_t idA = idesc_bf16_f32(128, HD, false, true);
+      const uint32_t sK = smem_u32(sm), sV = smem_u32(sm + Cf::OFF_V);
+      bool ok = mbar_wait(kv_full, 0, err, DEV_TIMEOUT_FULL);
+      auto issue_acc = [&](int i) -> bool {
+        const int s = i & 1, qs = i % Cf::QST;
+        if (!mbar_wait(&pd_full[s], (i >> 1) & 1, err, DEV_TIMEOUT_FULL)) return false;
+        tc_fence_after();
+        const uint32_t sP = smem_u32(sm + Cf::OFF_P0 + s * Cf::PB), sdS = smem_u32(sm + Cf::OFF_DS0 + s * Cf::PB);
+        const uint32_t sQ = smem_u32(sm + Cf::OFF_Q0 + qs * Cf::QB), sdO = smem_u32(sm + Cf::OFF_DO0 + qs * Cf::QB);
+#pragma unroll
+        for (int kk = 0; kk < Cf::BQ / 16; ++kk) {
+          tc_mma_f16(tmem + Cf::DV_COL, smem_desc_sw128(sP + kk * 32, 16, 1024),
+                     smem_desc_sw128(sdO + kk * 2048, Cf::BQ * 128, 1024), idA, (i | kk) ? 1u : 0u);
+          tc_mma_f16(tmem + Cf::DK_COL, smem_desc_sw128(sdS + kk * 32, 16, 1024),
+                     smem_desc_sw128(sQ + kk * 2048, Cf::BQ * 128, 1024), idA, (i | kk) ? 1u : 0u);
+        }
+        tc_commit(&pd_free[s]);
+        tc_commit(&q_empty[qs]);
+        return true;
+      };
+      for (int j = 0; j < nqb && ok; ++j) {
+        const int s = j & 1, qs = j % Cf::QST;
+        if (!mbar_wait(&q_full[qs], (j / Cf::QST) & 1, err, DEV_TIMEOUT_FULL) ||
+            !mbar_wait(&sp_free[s], ((j >> 1) & 1) ^ 1, err, DEV_TIMEOUT_ACC)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sQ = smem_u32(sm + Cf::OFF_Q0 + qs * Cf::QB), sdO = smem_u32(sm + Cf::OFF_DO0 + qs * Cf::QB);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t offa = (kk >> 2) * (Cf::BK * 128) + (kk & 3) * 32;
+          const uint32_t offb = (kk >> 2) * (Cf::BQ * 128) + (kk & 3) * 32;
+          tc_mma_f16(tmem + Cf::s_col(s), smem_desc_sw128(sK + offa, 16, 1024), smem_desc_sw128(sQ + offb, 16, 1024),
+                     idS, kk ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t offa = (kk >> 2) * (Cf::BK * 128) + (kk & 3) * 32;
+          const uint32_t offb = (kk >> 2) * (Cf::BQ * 128) + (kk & 3) * 32;
+          tc_mma_f16(tmem + Cf::dp_col(s), smem_desc_sw128(sV + offa, 16, 1024),
+                     smem_desc_sw128(sdO + offb, 16, 1024), idS, kk ? 1u : 0u);
+        }
+        tc_commit(&sp_full[s]);
+        if (j >= 1 && !issue_acc(j - 1)) { ok = false; break; }
+      }
+      if (ok) ok = issue_acc(nqb - 1);
+      if (ok) tc_commit(acc_done);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int lane = threadIdx.x & 31;
+    const int r = quarter * 32 + lane;              // key row of this thread (TMEM lane)
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const float sc = p.scale * 1.4426950408889634f;
+    const int64_t sbase = ((int64_t)b * p.H + h) * p.n;
+    const int kidx = k0 + r;
+    // per-query values of block j: threads r < 64 fetch -lse*log2e of query r, the
+    // others D of query r - 64 (rows past the end: +inf lse, zero D)
+    auto fetch = [&](int j) -> float {
+      const int i = (qb0 + j) * Cf::BQ + (r & 63);
+      if (i >= p.n) return r < 64 ? -INFINITY : 0.f;
+      return r < 64 ? -p.lse[sbase + i] * 1.4426950408889634f : p.Dsum[sbase + i];
+    };
+    ldbuf[r] = fetch(0);
+    named_bar_sync(1, 128);
+    bool ok = true;
+    for (int j = 0; j < nqb; ++j) {
+      const int s = j & 1;
+      const int i0 = (qb0 + j) * Cf::BQ;
+      const float nxt = j + 1 < nqb ? fetch(j + 1) : 0.f;
+      const bool need_mask = (i0 < k0 + Cf::BK - 1) || (i0 + Cf::BQ - 1 - k0 > p.window - 1);
+      // after a timed-out wait the loop still runs to its end (without waiting or
+      // computing) so that all four warps meet at every named barrier
+      if (ok) ok = mbar_wait(&sp_full[s], (j >> 1) & 1, err, DEV_TIMEOUT_ACC) &&
+                   mbar_wait(&pd_free[s], ((j >> 1) & 1) ^ 1, err, DEV_TIMEOUT_ACC);
+      if (ok) {
+        tc_fence_after();
+        uint32_t sr[64], dr[64];
+        tmem_ld32_nowait(tmem + lane_base + Cf::s_col(s), sr);
+        tmem_ld32_nowait(tmem + lane_base + Cf::s_col(s) + 32, sr + 32);
+        tmem_ld32_nowait(tmem + lane_base + Cf::dp_col(s), dr);
+        tmem_ld32_nowait(tmem + lane_base + Cf::dp_col(s) + 32, dr + 32);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sp_free[s]);  // S^T/dP^T buffer s may be overwritten by block j+2
+        const float* nl = ldbuf + s * 2 * Cf::BQ;
+        const float* dd = nl + Cf::BQ;
+        uint8_t* prow = sm + Cf::OFF_P0 + s * Cf::PB + r * 128;
+        uint8_t* drow = sm + Cf::OFF_DS0 + s * Cf::PB + r * 128;
+  #pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          const float4 nl0 = *(const float4*)(nl + cc * 8), nl1 = *(const float4*)(nl + cc * 8 + 4);
+          const float4 d0 = *(const float4*)(dd + cc * 8), d1 = *(const float4*)(dd + cc * 8 + 4);
+          const float nlv[8] = {nl0.x, nl0.y, nl0.z, nl0.w, nl1.x, nl1.y, nl1.z, nl1.w};
+          const float dv[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
+          float pv[8], ds[8];
+  #pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int c = cc * 8 + e;
+            float pr = ex2_tc(fmaf(__uint_as_float(sr[c]), sc, nlv[e]));
+            if (need_mask) {
+              const uint32_t off = (uint32_t)(i0 + c - kidx);
+              pr = off <= (uint32_t)(p.window - 1) ? pr : 0.f;
+            }
+            pv[e] = pr;
+            ds[e] = pr * (__uint_as_float(dr[c]) - dv[e]);
+          }
+          const int sw = (cc ^ (r & 7)) << 4;
+          *(uint4*)(prow + sw) = make_uint4(pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]),
+                                            pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
+          *(uint4*)(drow + sw) = make_uint4(pack_bf16x2(ds[0], ds[1]), pack_bf16x2(ds[2], ds[3]),
+                                            pack_bf16x2(ds[4], ds[5]), pack_bf16x2(ds[6], ds[7]));
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&pd_full[s]);
+      }
+      // block j+1's values go to the other half; every thread is past its reads of it
+      ldbuf[((j + 1) & 1) * 2 * Cf::BQ + r] = nxt;
+      named_bar_sync(1, 128);
+    }
+    if (ok && mbar_wait(acc_done, 0, err, DEV_TIMEOUT_ACC)) {
+      tc_fence_after();
+      const int64_t orow = ((int64_t)b * p.n + kidx) * p.lddq + h * HD;
+      bf16* dV = (bf16*)p.dV + orow;
+      bf16* dK = (bf16*)p.dK + orow;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        float o[32];
+        tmem_ld32(tmem + lane_base + Cf::DV_COL + c * 32, o);
+        if (r < nk) {
+          uint4* dst = (uint4*)(dV + c * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack_bf16x2(o[8 * q], o[8 * q + 1]), pack_bf16x2(o[8 * q + 2], o[8 * q + 3]),
+                                pack_bf16x2(o[8 * q + 4], o[8 * q + 5]), pack_bf16x2(o[8 * q + 6], o[8 * q + 7]));
+        }
+        tmem_ld32(tmem + lane_base + Cf::DK_COL + c * 32, o);
+        if (r < nk) {
+          uint4* dst = (uint4*)(dK + c * 32);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(pack_bf16x2(o[8 * q] * p.scale, o[8 * q + 1] * p.scale),
+                                pack_bf16x2(o[8 * q + 2] * p.scale, o[8 * q + 3] * p.scale),
+                                pack_bf16x2(o[8 * q + 4] * p.scale, o[8 * q + 5] * p.scale),
+                                pack_bf16x2(o[8 * q + 6] * p.scale, o[8 * q + 7] * p.scale));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 }  // namespace ttt

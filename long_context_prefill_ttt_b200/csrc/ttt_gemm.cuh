@@ -141,47 +141,58 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmParams p) {
 
 // ============================================================== skinny engine (decode)
 // At most 16 rows per batch slice (one row per sequence in decode): the work is
-// reading the weight matrix once, so one warp per output column streams its
-// weight row (and the per-sequence update row for the W_init + dW operand) with
-// 16-byte loads across all SMs; the few activation rows come from L1. K-major
-// operands only; the epilogue is the shared per-element one.
+// reading the weight matrix once. A CTA owns two output columns; four warps per
+// column split K into 16-byte-per-lane slabs, two slabs in flight per warp, so
+// every SM keeps many weight loads outstanding. Partial sums meet in shared
+// memory and the first lanes of each column apply the shared epilogue, one row
+// each. The few activation rows come from L1. K-major operands only.
 constexpr int SK_MAXM = 16;
 template <typename T>
 __global__ void __launch_bounds__(256) gemm_skinny_kernel(GemmParams p) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n = blockIdx.x * 8 + warp;
-  const int z = blockIdx.y;
-  if (n >= p.N) return;
   constexpr int VEC = 16 / sizeof(T);
-  const T* A = (const T*)p.A + (int64_t)z * p.sA;
-  const T* Bw = (const T*)p.B + (int64_t)z * p.sB + (int64_t)n * p.ldb;
-  const T* B2w = p.B2 ? (const T*)p.B2 + (int64_t)z * p.sB2 + (int64_t)n * p.ldb : nullptr;
+  constexpr int SLAB = 32 * VEC;  // elements of K per warp-iteration
+  __shared__ float part[8][SK_MAXM];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int col = warp >> 2, kw = warp & 3;  // column within the CTA, K quarter
+  const int n = blockIdx.x * 2 + col;
+  const int z = blockIdx.y;
   float acc[SK_MAXM];
 #pragma unroll
   for (int m = 0; m < SK_MAXM; ++m) acc[m] = 0.f;
-  for (int k0 = lane * VEC; k0 < p.K; k0 += 32 * VEC) {
-    float w[VEC];
-    {
-      const uint4 u = *reinterpret_cast<const uint4*>(Bw + k0);
-      const T* e = reinterpret_cast<const T*>(&u);
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) w[i] = to_f32(e[i]);
-    }
-    if (B2w) {
-      const uint4 u = *reinterpret_cast<const uint4*>(B2w + k0);
-      const T* e = reinterpret_cast<const T*>(&u);
-#pragma unroll
-      for (int i = 0; i < VEC; ++i) w[i] += to_f32(e[i]);
-    }
-#pragma unroll
-    for (int m = 0; m < SK_MAXM; ++m) {
-      if (m < p.M) {
-        const uint4 u = *reinterpret_cast<const uint4*>(A + (int64_t)m * p.lda + k0);
+  if (n < p.N) {
+    const T* A = (const T*)p.A + (int64_t)z * p.sA;
+    const T* Bw = (const T*)p.B + (int64_t)z * p.sB + (int64_t)n * p.ldb;
+    const T* B2w = p.B2 ? (const T*)p.B2 + (int64_t)z * p.sB2 + (int64_t)n * p.ldb : nullptr;
+    auto slab = [&](int k0) {
+      float w[VEC];
+      {
+        const uint4 u = *reinterpret_cast<const uint4*>(Bw + k0);
         const T* e = reinterpret_cast<const T*>(&u);
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) acc[m] = fmaf(to_f32(e[i]), w[i], acc[m]);
+        for (int i = 0; i < VEC; ++i) w[i] = to_f32(e[i]);
       }
+      if (B2w) {
+        const uint4 u = *reinterpret_cast<const uint4*>(B2w + k0);
+        const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) w[i] += to_f32(e[i]);
+      }
+#pragma unroll
+      for (int m = 0; m < SK_MAXM; ++m) {
+        if (m < p.M) {
+          const uint4 u = *reinterpret_cast<const uint4*>(A + (int64_t)m * p.lda + k0);
+          const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+          for (int i = 0; i < VEC; ++i) acc[m] = fmaf(to_f32(e[i]), w[i], acc[m]);
+        }
+      }
+    };
+    int k0 = (kw * 32 + lane) * VEC;
+    for (; k0 + 4 * SLAB < p.K; k0 += 8 * SLAB) {  // two slabs per iteration (this warp's and +4 warps')
+      slab(k0);
+      slab(k0 + 4 * SLAB);
     }
+    for (; k0 < p.K; k0 += 4 * SLAB) slab(k0);
   }
 #pragma unroll
   for (int m = 0; m < SK_MAXM; ++m) {
@@ -189,8 +200,14 @@ __global__ void __launch_bounds__(256) gemm_skinny_kernel(GemmParams p) {
       float v = acc[m];
 #pragma unroll
       for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) epi_apply<T>(p, z, m, n, v);
+      if (lane == 0) part[warp][m] = v;
     }
+  }
+  __syncthreads();
+  if (kw == 0 && lane < p.M && n < p.N) {
+    const int m = lane;
+    const float v = part[col * 4][m] + part[col * 4 + 1][m] + part[col * 4 + 2][m] + part[col * 4 + 3][m];
+    epi_apply<T>(p, z, m, n, v);
   }
 }
 
@@ -438,5 +455,7 @@ bool attn_tc_ok(const AttnParams& p);
 cudaError_t attn_fwd_tc_launch(const AttnParams& p, cudaStream_t st, int* err, bool* ok);
 bool attn_dq_tc_ok(const AttnParams& p);
 cudaError_t attn_bwd_dq_tc_launch(const AttnParams& p, cudaStream_t st, int* err, bool* ok);
+bool attn_dkv_tc_ok(const AttnParams& p);
+cudaError_t attn_bwd_dkv_tc_launch(const AttnParams& p, cudaStream_t st, int* err, bool* ok);
 
 }  // namespace ttt

@@ -55,19 +55,21 @@ static int attn_bwd(const AttnParams& ap, int engine, cudaStream_t st) {
   if (prime_kernel_attributes() != 0) return TTT_ERR_CUDA;
   const int64_t rows = (int64_t)ap.B * ap.n;
   attn_bwd_prep_kernel<T><<<(unsigned)((rows * ap.H + 7) / 8), 256, 0, st>>>(ap);
-  bool dq_done = false;
+  bool dq_done = false, dkv_done = false;
   if (sizeof(T) == 2 && engine == TTT_ENGINE_AUTO && attn_dq_tc_ok(ap)) {
     int* err = status_word();
-    const cudaError_t e = attn_bwd_dq_tc_launch(ap, st, err, &dq_done);
+    cudaError_t e = attn_bwd_dq_tc_launch(ap, st, err, &dq_done);
+    if (e == cudaSuccess && attn_dkv_tc_ok(ap)) e = attn_bwd_dkv_tc_launch(ap, st, err, &dkv_done);
     if (e != cudaSuccess) return TTT_ERR_CUDA;
   }
+  if (dq_done && dkv_done) return TTT_OK;
   if (sizeof(T) == 2 && engine != TTT_ENGINE_SIMT && attn_mma_ok(ap)) {
-    const cudaError_t e =
-        ap.hd == 128 ? attn_bwd_mma_launch<128>(ap, st, !dq_done) : attn_bwd_mma_launch<64>(ap, st, !dq_done);
+    const cudaError_t e = ap.hd == 128 ? attn_bwd_mma_launch<128>(ap, st, !dq_done, !dkv_done)
+                                       : attn_bwd_mma_launch<64>(ap, st, !dq_done, !dkv_done);
     return e == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
   }
-  attn_bwd_dq_simt_kernel<T><<<(unsigned)((rows * ap.H + 3) / 4), 128, 0, st>>>(ap);
-  attn_bwd_dkv_simt_kernel<T><<<(unsigned)((rows * ap.H + 3) / 4), 128, 0, st>>>(ap);
+  if (!dq_done) attn_bwd_dq_simt_kernel<T><<<(unsigned)((rows * ap.H + 3) / 4), 128, 0, st>>>(ap);
+  if (!dkv_done) attn_bwd_dkv_simt_kernel<T><<<(unsigned)((rows * ap.H + 3) / 4), 128, 0, st>>>(ap);
   return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 

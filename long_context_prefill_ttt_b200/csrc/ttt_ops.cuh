@@ -27,76 +27,198 @@ __global__ void embed_kernel(const int32_t* __restrict__ tok, int64_t tok_ld, in
   for (int c = lane; c < d; c += 32) o[c] = to_f32(e[c]);
 }
 
+// ---------------------------------------------------------------- 8-element vectors
+// Eight consecutive elements <-> fp32 registers: one 16-byte access for bf16,
+// two for fp32. The address must be 16-byte aligned.
+__device__ __forceinline__ void ld8(const float* p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ void ld8(const bf16* p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x; v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void st8(float* p, const float (&v)[8]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+  *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+__device__ __forceinline__ void st8(bf16* p, const float (&v)[8]) {
+  uint4 u;
+  u.x = pack_bf16x2(v[0], v[1]); u.y = pack_bf16x2(v[2], v[3]);
+  u.z = pack_bf16x2(v[4], v[5]); u.w = pack_bf16x2(v[6], v[7]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+
+// Sum over the TPR threads that share a row (TPR a power of two <= 256; the
+// block holds 256 / TPR rows). Every thread of the block must call it.
+template <int TPR> __device__ __forceinline__ float row_sum(float v, float* red) {
+#pragma unroll
+  for (int o = (TPR < 32 ? TPR : 32) >> 1; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if constexpr (TPR > 32) {
+    constexpr int W = TPR / 32;
+    const int w = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) red[w] = v;
+    __syncthreads();
+    const int w0 = w & ~(W - 1);
+    v = 0.f;
+#pragma unroll
+    for (int i = 0; i < W; ++i) v += red[w0 + i];
+  }
+  return v;
+}
+
+// Threads per row of d elements: each thread owns 8-element chunks
+// c = (k * TPR + t) * 8, k = 0, 1, ...; the first RC_CACHE chunks stay in
+// registers between the two passes of a row kernel.
+constexpr int RC_CACHE = 2;
+inline int row_threads(int d) {  // two chunks per thread where the row is long enough
+  const int ch = d / 16;
+  return ch >= 256 ? 256 : ch >= 128 ? 128 : ch >= 64 ? 64 : 32;
+}
+
 // ---------------------------------------------------------------- RMSNorm
 // y = g * x / sqrt(mean(x^2) + eps); rstd kept for the backward.
-template <typename T>
-__global__ void rmsnorm_fwd_kernel(const float* __restrict__ x, int64_t ldx, const float* __restrict__ g,
-                                   float eps, int rows, int d, T* __restrict__ y, int64_t ldy,
-                                   float* __restrict__ rstd_out) {
+// Blocks of 256 threads, TPR threads per row (d % 8 == 0, ldx % 4 == 0, ldy % 8 == 0).
+template <typename T, int TPR>
+__global__ void __launch_bounds__(256, 4) rmsnorm_fwd_kernel(const float* __restrict__ x, int64_t ldx,
+                                                          const float* __restrict__ g, float eps, int rows, int d,
+                                                          T* __restrict__ y, int64_t ldy,
+                                                          float* __restrict__ rstd_out) {
+  __shared__ float red[8];
   pdl_wait();
   pdl_trigger();
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const float* xr = x + (int64_t)row * ldx;
+  const int t = threadIdx.x % TPR;
+  const int row = blockIdx.x * (256 / TPR) + threadIdx.x / TPR;
+  const bool live = row < rows;
+  const int nch = (d / 8 + TPR - 1) / TPR;
+  const float* xr = x + (int64_t)(live ? row : 0) * ldx;
+  float cache[RC_CACHE][8];
   float ss = 0.f;
-  for (int c = lane * 4; c < d; c += 128) {
-    const float4 v = *(const float4*)(xr + c);
-    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-  }
 #pragma unroll
-  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  for (int k = 0; k < RC_CACHE; ++k) {
+    const int c = (k * TPR + t) * 8;
+    if (k < nch && live && c < d) {
+      ld8(xr + c, cache[k]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ss += cache[k][i] * cache[k][i];
+    }
+  }
+  for (int k = RC_CACHE; k < nch; ++k) {
+    const int c = (k * TPR + t) * 8;
+    if (live && c < d) {
+      float v[8];
+      ld8(xr + c, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) ss += v[i] * v[i];
+    }
+  }
+  ss = row_sum<TPR>(ss, red);
+  if (!live) return;
   const float rs = rsqrtf(ss / d + eps);
-  if (lane == 0 && rstd_out) rstd_out[row] = rs;
+  if (t == 0 && rstd_out) rstd_out[row] = rs;
   T* yr = y + (int64_t)row * ldy;
-  for (int c = lane * 4; c < d; c += 128) {
-    const float4 v = *(const float4*)(xr + c);
-    const float4 gg = *(const float4*)(g + c);
-    yr[c] = from_f32<T>(v.x * rs * gg.x);
-    yr[c + 1] = from_f32<T>(v.y * rs * gg.y);
-    yr[c + 2] = from_f32<T>(v.z * rs * gg.z);
-    yr[c + 3] = from_f32<T>(v.w * rs * gg.w);
+  for (int k = 0; k < nch; ++k) {
+    const int c = (k * TPR + t) * 8;
+    if (c >= d) continue;
+    float v[8], gg[8];
+    if (k < RC_CACHE) {
+#pragma unroll
+      for (int kk = 0; kk < RC_CACHE; ++kk)
+        if (kk == k) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[i] = cache[kk][i];
+        }
+    } else {
+      ld8(xr + c, v);
+    }
+    ld8(g + c, gg);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = v[i] * rs * gg[i];
+    st8(yr + c, v);
   }
 }
 
 // dx = dres + rstd*(g*dy) - x*rstd^3*sum(g*dy*x)/d ; writes fp32 and (optionally) a T copy.
-template <typename T>
-__global__ void rmsnorm_bwd_kernel(const float* __restrict__ x, const float* __restrict__ g,
-                                   const float* __restrict__ rstd, const float* __restrict__ dy,
-                                   const float* dres, int rows, int d, float* dx, T* __restrict__ dx_t) {
+// dres may alias dx (each element is read before it is written, by the same thread).
+template <typename T, int TPR>
+__global__ void __launch_bounds__(256, 3) rmsnorm_bwd_kernel(const float* __restrict__ x, const float* __restrict__ g,
+                                                          const float* __restrict__ rstd,
+                                                          const float* __restrict__ dy, const float* dres, int rows,
+                                                          int d, float* dx, T* __restrict__ dx_t) {
+  __shared__ float red[8];
   pdl_wait();
   pdl_trigger();
-  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  const int64_t o = (int64_t)row * d;
+  const int t = threadIdx.x % TPR;
+  const int row = blockIdx.x * (256 / TPR) + threadIdx.x / TPR;
+  const bool live = row < rows;
+  const int nch = (d / 8 + TPR - 1) / TPR;
+  const int64_t o = (int64_t)(live ? row : 0) * d;
+  float cx[RC_CACHE][8], cgd[RC_CACHE][8];  // x and g * dy of the cached chunks
   float dot = 0.f;
-  for (int c = lane * 4; c < d; c += 128) {
-    const float4 xv = *(const float4*)(x + o + c);
-    const float4 dv = *(const float4*)(dy + o + c);
-    const float4 gv = *(const float4*)(g + c);
-    dot += gv.x * dv.x * xv.x + gv.y * dv.y * xv.y + gv.z * dv.z * xv.z + gv.w * dv.w * xv.w;
-  }
 #pragma unroll
-  for (int s = 16; s; s >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, s);
+  for (int k = 0; k < RC_CACHE; ++k) {
+    const int c = (k * TPR + t) * 8;
+    if (k < nch && live && c < d) {
+      float gg[8];
+      ld8(x + o + c, cx[k]);
+      ld8(dy + o + c, cgd[k]);
+      ld8(g + c, gg);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        cgd[k][i] *= gg[i];
+        dot += cgd[k][i] * cx[k][i];
+      }
+    }
+  }
+  for (int k = RC_CACHE; k < nch; ++k) {
+    const int c = (k * TPR + t) * 8;
+    if (live && c < d) {
+      float xv[8], dv[8], gg[8];
+      ld8(x + o + c, xv);
+      ld8(dy + o + c, dv);
+      ld8(g + c, gg);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dot += gg[i] * dv[i] * xv[i];
+    }
+  }
+  dot = row_sum<TPR>(dot, red);
+  if (!live) return;
   const float rs = rstd[row];
   const float coef = rs * rs * rs * dot / d;
-  for (int c = lane * 4; c < d; c += 128) {
-    const float4 xv = *(const float4*)(x + o + c);
-    const float4 dv = *(const float4*)(dy + o + c);
-    const float4 gv = *(const float4*)(g + c);
-    float4 r = dres ? *(const float4*)(dres + o + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-    r.x += rs * gv.x * dv.x - xv.x * coef;
-    r.y += rs * gv.y * dv.y - xv.y * coef;
-    r.z += rs * gv.z * dv.z - xv.z * coef;
-    r.w += rs * gv.w * dv.w - xv.w * coef;
-    *(float4*)(dx + o + c) = r;
-    if (dx_t) {
-      dx_t[o + c] = from_f32<T>(r.x);
-      dx_t[o + c + 1] = from_f32<T>(r.y);
-      dx_t[o + c + 2] = from_f32<T>(r.z);
-      dx_t[o + c + 3] = from_f32<T>(r.w);
+  for (int k = 0; k < nch; ++k) {
+    const int c = (k * TPR + t) * 8;
+    if (c >= d) continue;
+    float xv[8], gd[8];
+    if (k < RC_CACHE) {
+#pragma unroll
+      for (int kk = 0; kk < RC_CACHE; ++kk)
+        if (kk == k) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) { xv[i] = cx[kk][i]; gd[i] = cgd[kk][i]; }
+        }
+    } else {
+      float dv[8], gg[8];
+      ld8(x + o + c, xv);
+      ld8(dy + o + c, dv);
+      ld8(g + c, gg);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) gd[i] = gg[i] * dv[i];
     }
+    float r[8];
+    if (dres) ld8(dres + o + c, r);
+    else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) r[i] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) r[i] += rs * gd[i] - xv[i] * coef;
+    st8(dx + o + c, r);
+    if (dx_t) st8(dx_t + o + c, r);
   }
 }
 
@@ -106,28 +228,69 @@ __global__ void rmsnorm_bwd_kernel(const float* __restrict__ x, const float* __r
 // two tables built in double precision on the host:
 //   cos/sin(p*t) from (p = 1024*hi + lo) by the angle-addition identities.
 // inverse != 0 applies the transpose rotation (backward of the forward map).
+// The rotation depends on (position, pair index) only, so one thread takes 8
+// consecutive pairs of RP_HEADS heads of one row and forms their (cos, sin) once
+// (hd % 16 == 0, ncols % hd == 0, ld % 8 == 0).
+constexpr int RP_HEADS = 4;
 template <typename T>
-__global__ void rope_kernel(T* __restrict__ qk, int64_t ld, int ncols, int rows, int n, int64_t pos0, int hd,
-                            const float2* __restrict__ lo_tab, const float2* __restrict__ hi_tab, int inverse,
-                            const int64_t* pos_dev = nullptr) {
+__global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ qk, int64_t ld, int ncols, int rows, int n,
+                                                   int64_t pos0, int hd, const float2* __restrict__ lo_tab,
+                                                   const float2* __restrict__ hi_tab, int inverse,
+                                                   const int64_t* pos_dev = nullptr) {
+  pdl_wait();
+  pdl_trigger();
   if (pos_dev) pos0 = *pos_dev;  // position held on the device (graph-captured decode step)
   const int half = hd >> 1;
-  const int pairs_per_row = ncols >> 1;
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (int64_t)rows * pairs_per_row) return;
-  const int row = (int)(idx / pairs_per_row);
-  const int pr = (int)(idx % pairs_per_row);
-  const int head = pr / half, i = pr % half;
+  const int ng = half >> 3;                                  // 8-pair groups per head
+  const int nheads = ncols / hd;
+  const int per_row = ng * ((nheads + RP_HEADS - 1) / RP_HEADS);
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows * per_row) return;
+  const int row = idx / per_row;
+  const int rem = idx - row * per_row;
+  const int hc = rem / ng;
+  const int i = (rem - hc * ng) * 8;
   const int64_t pos = pos0 + (row % n);
-  const float2 a = lo_tab[(pos & 1023) * half + i];   // (cos, sin) of lo * theta_i
-  const float2 b = hi_tab[(pos >> 10) * half + i];    // of 1024*hi * theta_i
-  const float c = a.x * b.x - a.y * b.y;
-  float s = a.y * b.x + a.x * b.y;
-  if (inverse) s = -s;
-  T* base = qk + (int64_t)row * ld + head * hd;
-  const float x1 = to_f32(base[i]), x2 = to_f32(base[i + half]);
-  base[i] = from_f32<T>(x1 * c - x2 * s);
-  base[i + half] = from_f32<T>(x2 * c + x1 * s);
+  const float4* a4 = reinterpret_cast<const float4*>(lo_tab + (pos & 1023) * half + i);  // (cos, sin) of lo * theta
+  const float4* b4 = reinterpret_cast<const float4*>(hi_tab + (pos >> 10) * half + i);   // of 1024*hi * theta
+  float cs[8], sn[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float4 a = a4[j], b = b4[j];  // two pairs: (a.x, a.y) and (a.z, a.w)
+    cs[2 * j] = a.x * b.x - a.y * b.y;
+    sn[2 * j] = a.y * b.x + a.x * b.y;
+    cs[2 * j + 1] = a.z * b.z - a.w * b.w;
+    sn[2 * j + 1] = a.w * b.z + a.z * b.w;
+  }
+  if (inverse) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) sn[q] = -sn[q];
+  }
+  T* rowp = qk + (int64_t)row * ld + i;
+#pragma unroll
+  for (int t = 0; t < RP_HEADS; ++t) {
+    const int head = hc * RP_HEADS + t;
+    if (head < nheads) {
+      T* base = rowp + head * hd;
+      float x1[8], x2[8];
+      ld8(base, x1);
+      ld8(base + half, x2);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float u = x1[q], v = x2[q];
+        x1[q] = u * cs[q] - v * sn[q];
+        x2[q] = v * cs[q] + u * sn[q];
+      }
+      st8(base, x1);
+      st8(base + half, x2);
+    }
+  }
+}
+
+// Grid of rope_kernel for rows x ncols (head dim hd).
+inline int64_t rope_threads(int rows, int ncols, int hd) {
+  const int nheads = ncols / hd;
+  return (int64_t)rows * (hd >> 4) * ((nheads + RP_HEADS - 1) / RP_HEADS);
 }
 
 // ---------------------------------------------------------------- window ring

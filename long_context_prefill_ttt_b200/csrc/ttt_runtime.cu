@@ -50,6 +50,44 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// Row-kernel launches (PDL): RMSNorm with row_threads(d) threads per row in
+// blocks of 256; RoPE with one thread per 8 pairs.
+template <typename T>
+static cudaError_t rmsnorm_fwd_launch(const float* x, int64_t ldx, const float* g, float eps, int rows, int d, T* y,
+                                      int64_t ldy, float* rstd, cudaStream_t st) {
+  const int tpr = row_threads(d), rpb = 256 / tpr;
+  const dim3 grid((unsigned)((rows + rpb - 1) / rpb)), blk(256);
+  switch (tpr) {
+    case 256: return launch_pdl(rmsnorm_fwd_kernel<T, 256>, grid, blk, 0, st, x, ldx, g, eps, rows, d, y, ldy, rstd);
+    case 128: return launch_pdl(rmsnorm_fwd_kernel<T, 128>, grid, blk, 0, st, x, ldx, g, eps, rows, d, y, ldy, rstd);
+    case 64: return launch_pdl(rmsnorm_fwd_kernel<T, 64>, grid, blk, 0, st, x, ldx, g, eps, rows, d, y, ldy, rstd);
+    default: return launch_pdl(rmsnorm_fwd_kernel<T, 32>, grid, blk, 0, st, x, ldx, g, eps, rows, d, y, ldy, rstd);
+  }
+}
+
+template <typename T>
+static cudaError_t rmsnorm_bwd_launch(const float* x, const float* g, const float* rstd, const float* dy,
+                                      const float* dres, int rows, int d, float* dx, T* dx_t, cudaStream_t st) {
+  const int tpr = row_threads(d), rpb = 256 / tpr;
+  const dim3 grid((unsigned)((rows + rpb - 1) / rpb)), blk(256);
+  switch (tpr) {
+    case 256: return launch_pdl(rmsnorm_bwd_kernel<T, 256>, grid, blk, 0, st, x, g, rstd, dy, dres, rows, d, dx, dx_t);
+    case 128: return launch_pdl(rmsnorm_bwd_kernel<T, 128>, grid, blk, 0, st, x, g, rstd, dy, dres, rows, d, dx, dx_t);
+    case 64: return launch_pdl(rmsnorm_bwd_kernel<T, 64>, grid, blk, 0, st, x, g, rstd, dy, dres, rows, d, dx, dx_t);
+    default: return launch_pdl(rmsnorm_bwd_kernel<T, 32>, grid, blk, 0, st, x, g, rstd, dy, dres, rows, d, dx, dx_t);
+  }
+}
+
+template <typename T>
+static cudaError_t rope_launch(T* qk, int64_t ld, int ncols, int rows, int n, int64_t pos0, int hd,
+                               const float2* lo, const float2* hi, int inverse, const int64_t* pos_dev,
+                               cudaStream_t st) {
+  const int64_t threads = rope_threads(rows, ncols, hd);
+  if (threads >= (int64_t)INT32_MAX || ncols % hd) return cudaErrorInvalidValue;
+  return launch_pdl(rope_kernel<T>, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, st, qk, ld, ncols, rows,
+                    n, pos0, hd, lo, hi, inverse, pos_dev);
+}
+
 // ============================================================== GEMM dispatch (host)
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -170,6 +208,22 @@ cudaError_t attn_bwd_dq_tc_launch(const AttnParams& p, cudaStream_t st, int* err
                     err);
 }
 
+bool attn_dkv_tc_ok(const AttnParams& p) {
+  return attn_dq_tc_ok(p) && aligned16(p.dK) && aligned16(p.dV) && p.window >= 1;
+}
+
+cudaError_t attn_bwd_dkv_tc_launch(const AttnParams& p, cudaStream_t st, int* err, bool* ok) {
+  CUtensorMap tk, tq, tdo;  // K and V in 128-row boxes, Q and dO in 64-row boxes
+  *ok = make_rows_map(&tk, p.Q, 3 * p.d, (int64_t)p.B * p.n) &&
+        make_rows_map(&tq, p.Q, 3 * p.d, (int64_t)p.B * p.n, 64) &&
+        make_rows_map(&tdo, p.dO, p.d, (int64_t)p.B * p.n, 64);
+  if (!*ok) return cudaSuccess;
+  dim3 grid((p.n + 127) / 128, p.H, p.B);
+  if (p.hd == 128)
+    return launch_pdl(attn_bwd_dkv_tc_kernel<128>, grid, dim3(192), AttnDkvCfg<128>::SMEM, st, tk, tq, tdo, p, err);
+  return launch_pdl(attn_bwd_dkv_tc_kernel<64>, grid, dim3(192), AttnDkvCfg<64>::SMEM, st, tk, tq, tdo, p, err);
+}
+
 // Dynamic shared-memory limits of every large-smem kernel, set once per process
 // before any launch (and so never inside a CUDA graph capture).
 template <int BN, bool AM, bool BM> static cudaError_t tc_attr() {
@@ -190,7 +244,11 @@ int prime_kernel_attributes() {
                            cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 AttnDqCfg<64>::SMEM),
                            cudaFuncSetAttribute(attn_bwd_dq_tc_kernel<128>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, AttnDqCfg<128>::SMEM)};
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, AttnDqCfg<128>::SMEM),
+                           cudaFuncSetAttribute(attn_bwd_dkv_tc_kernel<64>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, AttnDkvCfg<64>::SMEM),
+                           cudaFuncSetAttribute(attn_bwd_dkv_tc_kernel<128>,
+                                                cudaFuncAttributeMaxDynamicSharedMemorySize, AttnDkvCfg<128>::SMEM)};
   for (cudaError_t x : r)
     if (x != cudaSuccess) e = x;
   if (e != cudaSuccess) return (int)e;
@@ -208,20 +266,18 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
       (p.batch == 1 || (p.sA % vec == 0 && p.sB % vec == 0 && p.sB2 % vec == 0))) {
     GemmParams q = p;
     if (p.epi == EPI_QKV_ROPE) q.epi = EPI_STORE;
-    dim3 grid((p.N + 7) / 8, p.batch);
+    dim3 grid((p.N + 1) / 2, p.batch);
     if (elem_is_bf16)
       gemm_skinny_kernel<bf16><<<grid, 256, 0, st>>>(q);
     else
       gemm_skinny_kernel<float><<<grid, 256, 0, st>>>(q);
     if (p.epi == EPI_QKV_ROPE) {
-      const int64_t work = (int64_t)p.M * (p.rope_cols / 2);
-      const unsigned blocks = (unsigned)((work + 255) / 256);
-      if (elem_is_bf16)
-        rope_kernel<bf16><<<blocks, 256, 0, st>>>((bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0,
-                                                   p.rope_hd, p.rope_lo, p.rope_hi, 0, p.rope_pos_dev);
-      else
-        rope_kernel<float><<<blocks, 256, 0, st>>>((float*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0,
-                                                    p.rope_hd, p.rope_lo, p.rope_hi, 0, p.rope_pos_dev);
+      const cudaError_t re =
+        elem_is_bf16 ? rope_launch<bf16>((bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd,
+                                         p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st)
+                     : rope_launch<float>((float*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd,
+                                          p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st);
+    if (re != cudaSuccess) return (int)re;
     }
     return (int)cudaGetLastError();
   }
@@ -259,11 +315,8 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
     if (e != cudaSuccess) return (int)e;
     if (ok) {
       if (p.epi == EPI_QKV_ROPE) {
-        const int64_t work = (int64_t)p.M * (p.rope_cols / 2);
-        rope_kernel<bf16><<<(unsigned)((work + 255) / 256), 256, 0, st>>>(
-            (bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd, p.rope_lo, p.rope_hi, 0,
-            p.rope_pos_dev);
-        return (int)cudaGetLastError();
+        return (int)rope_launch<bf16>((bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd,
+                                      p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st);
       }
       return 0;
     }
@@ -276,14 +329,12 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
   else
     gemm_simt_kernel<float><<<grid, 256, 0, st>>>(q);
   if (p.epi == EPI_QKV_ROPE) {
-    const int64_t work = (int64_t)p.M * (p.rope_cols / 2);
-    const unsigned blocks = (unsigned)((work + 255) / 256);
-    if (elem_is_bf16)
-      rope_kernel<bf16><<<blocks, 256, 0, st>>>((bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0,
-                                                 p.rope_hd, p.rope_lo, p.rope_hi, 0, p.rope_pos_dev);
-    else
-      rope_kernel<float><<<blocks, 256, 0, st>>>((float*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0,
-                                                  p.rope_hd, p.rope_lo, p.rope_hi, 0, p.rope_pos_dev);
+    const cudaError_t re =
+        elem_is_bf16 ? rope_launch<bf16>((bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd,
+                                         p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st)
+                     : rope_launch<float>((float*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd,
+                                          p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st);
+    if (re != cudaSuccess) return (int)re;
   }
   return (int)cudaGetLastError();
 }
@@ -794,7 +845,7 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
                                T* o, float* lse, int n, int64_t q0, bool commit) {
   const int rows = B * n;
   int rc;
-  launch_pdl(rmsnorm_fwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)xin, d, Lw.g_attn, cfg.rms_eps, rows, d, r, d, rstd);
+  rmsnorm_fwd_launch<T>((const float*)xin, d, Lw.g_attn, cfg.rms_eps, rows, d, r, d, rstd, st);
   TTT_LAUNCHED();
   {  // q|k|v = r Wqkv^T with RoPE applied to q and k in the GEMM epilogue
     GemmParams pq = gp(rows, 3 * d, d, r, d, false, Lw.Wqkv, d, false, qkv, 3 * d, false, EPI_QKV_ROPE);
@@ -866,7 +917,7 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
 // x += W2 gelu(W1 RMSNorm(x)) (frozen blocks)
 template <typename T> int Engine<T>::frozen_mlp(const LayerDev<T>& Lw, float* x, T* r, T* hid, int rows) {
   int rc;
-  launch_pdl(rmsnorm_fwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)x, d, Lw.g_mlp, cfg.rms_eps, rows, d, r, d, nullptr);
+  rmsnorm_fwd_launch<T>((const float*)x, d, Lw.g_mlp, cfg.rms_eps, rows, d, r, d, nullptr, st);
   TTT_LAUNCHED();
   if ((rc = gemm(gp(rows, h, d, r, d, false, Lw.W1, d, false, hid, h, false, EPI_GELU))) != TTT_OK) return rc;
   GemmParams p = gp(rows, d, h, hid, h, false, Lw.W2, h, false, x, d, true, EPI_RESID);
@@ -887,7 +938,7 @@ template <typename T> int Engine<T>::ttt_forward(int cn, int64_t pos, bool commi
                               commit)) != TTT_OK)
       return rc;
     // TTT-MLP with the fast weights of each sequence (batched over sequences)
-    launch_pdl(rmsnorm_fwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)A.a, d, Lw.g_ttt, cfg.rms_eps, rows, d, A.r2, d, A.rstd2);
+    rmsnorm_fwd_launch<T>((const float*)A.a, d, Lw.g_ttt, cfg.rms_eps, rows, d, A.r2, d, A.rstd2, st);
     TTT_LAUNCHED();
     GemmParams p = gp(cn, ht, d, A.r2, d, false, Lw.W1t, d, false, A.g, ht, false, EPI_GELU);
     p.batch = B; p.sA = (int64_t)cn * d; p.sD = (int64_t)cn * ht;
@@ -900,8 +951,8 @@ template <typename T> int Engine<T>::ttt_forward(int cn, int64_t pos, bool commi
     p.X = A.a; p.ldx = d; p.sX = (int64_t)cn * d;
     if ((rc = gemm(p)) != TTT_OK) return rc;
     // static MLP
-    launch_pdl(rmsnorm_fwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)A.m, d, Lw.g_static, cfg.rms_eps, rows, d, A.r3, d,
-                                                         A.rstd3);
+    rmsnorm_fwd_launch<T>((const float*)A.m, d, Lw.g_static, cfg.rms_eps, rows, d, A.r3, d,
+                                                         A.rstd3, st);
     TTT_LAUNCHED();
     p = gp(rows, hs, d, A.r3, d, false, Lw.W1s, d, false, A.gs, hs, false, EPI_GELU);
     p.Y = A.us; p.ldy = hs;
@@ -921,7 +972,7 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
   int rc;
   // LM head: dr = dz E ; G = d loss / d y through the final RMSNorm
   if ((rc = gemm(gp(rows, d, V, z, V, false, E, d, true, dr, d, true, EPI_STORE))) != TTT_OK) return rc;
-  launch_pdl(rmsnorm_bwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)y, g_final, rstdf, dr, nullptr, rows, d, G, GT);
+  rmsnorm_bwd_launch<T>((const float*)y, g_final, rstdf, dr, nullptr, rows, d, G, GT, st);
   TTT_LAUNCHED();
   for (int j = Lt - 1; j >= 0; --j) {
     const int l = first_ttt + j;
@@ -932,7 +983,7 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
     p.X = A.us; p.ldx = hs;
     if ((rc = gemm(p)) != TTT_OK) return rc;
     if ((rc = gemm(gp(rows, d, hs, dhid, hs, false, Lw.W1s, d, true, dr, d, true, EPI_STORE))) != TTT_OK) return rc;
-    launch_pdl(rmsnorm_bwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)A.m, Lw.g_static, A.rstd3, dr, G, rows, d, G, GT);
+    rmsnorm_bwd_launch<T>((const float*)A.m, Lw.g_static, A.rstd3, dr, G, rows, d, G, GT, st);
     TTT_LAUNCHED();
     // TTT-MLP data gradients (with W_{i-1}), then the fused weight gradient + SGD
     p = gp(cn, ht, d, GT, d, false, Lw.W2t, ht, true, dhid, ht, false, EPI_DGELU);
@@ -960,7 +1011,7 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
     if (is_bf16) { p.Y = Lw.W1t; p.ldy = d; p.sY = (int64_t)ht * d; }
     if ((rc = gemm(p)) != TTT_OK) return rc;
     if (j == 0) break;  // upstream of the first adaptive MLP does not depend on the fast weights
-    launch_pdl(rmsnorm_bwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)A.a, Lw.g_ttt, A.rstd2, dr, G, rows, d, G, GT);
+    rmsnorm_bwd_launch<T>((const float*)A.a, Lw.g_ttt, A.rstd2, dr, G, rows, d, G, GT, st);
     TTT_LAUNCHED();
     // frozen attention: data gradients only; cached K/V are constants
     if ((rc = gemm(gp(rows, d, d, GT, d, false, Lw.Wo, d, true, dob, d, false, EPI_STORE))) != TTT_OK) return rc;
@@ -979,33 +1030,35 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
                2.0 * hd * H * (double)B * (2.0 * attn_pairs(cn, chunk_pos) + 2.0 * attn_pairs(cn, 0)), 0.0);
     attn_bwd_prep_kernel<T><<<nblk((int64_t)rows * H, 8), 256, 0, st>>>(ap);
     TTT_LAUNCHED();
-    bool dq_done = false;
+    // dQ and dK/dV: tcgen05 kernels where they apply, else mma.sync, else SIMT
+    bool dq_done = false, dkv_done = false;
     if (is_bf16 && attn_dq_tc_ok(ap)) {
-      const cudaError_t e = attn_bwd_dq_tc_launch(ap, st, dev_err, &dq_done);
+      cudaError_t e = attn_bwd_dq_tc_launch(ap, st, dev_err, &dq_done);
+      if (e == cudaSuccess && attn_dkv_tc_ok(ap)) e = attn_bwd_dkv_tc_launch(ap, st, dev_err, &dkv_done);
       if (e != cudaSuccess) {
         poisoned = true;
         return fail(this, TTT_ERR_CUDA, std::string("attention backward: ") + cudaGetErrorString(e));
       }
     }
-    if (is_bf16 && attn_mma_ok(ap)) {
-      const cudaError_t e =
-          hd == 128 ? attn_bwd_mma_launch<128>(ap, st, !dq_done) : attn_bwd_mma_launch<64>(ap, st, !dq_done);
-      (void)e;
-      launches += 1;
-    } else {
-      attn_bwd_dq_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
-      TTT_LAUNCHED();
-      attn_bwd_dkv_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
+    if (!(dq_done && dkv_done)) {
+      if (is_bf16 && attn_mma_ok(ap)) {
+        const cudaError_t e = hd == 128 ? attn_bwd_mma_launch<128>(ap, st, !dq_done, !dkv_done)
+                                        : attn_bwd_mma_launch<64>(ap, st, !dq_done, !dkv_done);
+        (void)e;  // checked by the launch accounting below
+      } else {
+        if (!dq_done) attn_bwd_dq_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
+        if (!dkv_done) attn_bwd_dkv_simt_kernel<T><<<nblk((int64_t)rows * H, 4), 128, 0, st>>>(ap);
+      }
     }
+    launches += 1;  // dQ and dK/dV are two launches whichever engine ran them; one more below
     prof.end(st);
     TTT_LAUNCHED();
-    rope_kernel<T><<<nblk((int64_t)rows * d, 256), 256, 0, st>>>(dqkv, 3 * d, 2 * d, rows, cn, chunk_pos, hd,
-                                                                  rope_lo, rope_hi, 1);
+    rope_launch<T>(dqkv, 3 * d, 2 * d, rows, cn, chunk_pos, hd, rope_lo, rope_hi, 1, nullptr, st);
     TTT_LAUNCHED();
     if ((rc = gemm(gp(rows, d, 3 * d, dqkv, 3 * d, false, Lw.Wqkv, d, true, dr, d, true, EPI_STORE))) != TTT_OK)
       return rc;
     // G <- G + RMSNorm_bwd through the attention norm: gradient w.r.t. this block's input
-    launch_pdl(rmsnorm_bwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)A.x, Lw.g_attn, A.rstd1, dr, G, rows, d, G, GT);
+    rmsnorm_bwd_launch<T>((const float*)A.x, Lw.g_attn, A.rstd1, dr, G, rows, d, G, GT, st);
     TTT_LAUNCHED();
   }
   return TTT_OK;
@@ -1031,7 +1084,7 @@ int Engine<T>::ttt_step(const float* in, const int32_t* targets, int cn, int64_t
     TTT_CUDA(cudaMemcpyAsync(tgt, targets, (size_t)rows * 4, cudaMemcpyDeviceToDevice, st));
   }
   if ((rc = ttt_forward(cn, pos, commit)) != TTT_OK) return rc;
-  launch_pdl(rmsnorm_fwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf);
+  rmsnorm_fwd_launch<T>((const float*)y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf, st);
   TTT_LAUNCHED();
   if ((rc = gemm(gp(rows, V, d, rf, d, false, E, d, false, z, V, false, EPI_STORE))) != TTT_OK) return rc;
   // mean over the b positions of the chunk (summary: mini-batch GD with 1/b)
@@ -1135,7 +1188,7 @@ template <typename T> int Engine<T>::decode_token_launches(int64_t n, int32_t* o
   TTT_CUDA(cudaMemcpyAsync(blk[0].x, xs, (size_t)B * d * 4, cudaMemcpyDeviceToDevice, st));
   gemm_class = PC_GEMM_TTT;
   if ((rc = ttt_forward(1, 0, true)) != TTT_OK) return rc;
-  launch_pdl(rmsnorm_fwd_kernel<T>, dim3(nblk(rows, 4)), dim3(128), 0, st, (const float*)y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf);
+  rmsnorm_fwd_launch<T>((const float*)y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf, st);
   TTT_LAUNCHED();
   if ((rc = gemm(gp(rows, V, d, rf, d, false, E, d, false, z, V, false, EPI_STORE))) != TTT_OK) return rc;
   const int32_t* fcol = nullptr;

@@ -153,6 +153,14 @@ ATTN_CASES = [
     (1, 2, 64, 130, 64, 40, 128), (1, 1, 128, 256, 1024, 1024, 2048),
     # tcgen05 forward (q0 % 128 == 0, C % 128 == 0): many ring tiles, partial last query tile
     (2, 2, 128, 384, 512, 700, 1280), (1, 4, 64, 300, 1024, 1000, 2048),
+    # tcgen05 dK/dV: window shorter than the rows (key blocks that some query blocks no
+    # longer see), ragged last key block with the next sequence's rows behind it, no ring
+    # (q0 = 0), window shorter than one query block
+    (2, 2, 128, 520, 256, 200, 768), (1, 3, 64, 330, 0, 150, 384), (2, 2, 128, 256, 128, 40, 256),
+    # enough (sequence, head) pairs that the forward gives each CTA two query tiles sharing
+    # K/V: ragged rows with a short window, the second tile's keys one tile further on
+    # (window a multiple of 128), and no ring with a window longer than the rows
+    (2, 40, 64, 520, 256, 300, 768), (1, 80, 128, 384, 1024, 512, 1536), (1, 150, 64, 300, 0, 4096, 4224),
 ]
 
 
