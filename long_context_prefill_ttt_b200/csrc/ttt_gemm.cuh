@@ -48,6 +48,10 @@ struct GemmParams {
   const float2* rope_lo; const float2* rope_hi;
   int64_t rope_pos0; const int64_t* rope_pos_dev;
   int rope_n, rope_hd, rope_cols;
+  // Tile order of the tensor-core engine within a batch slice: 0 = row blocks outer
+  // (consecutive tiles share A rows), 1 = column blocks outer (consecutive tiles share
+  // B rows, so a B larger than L2 streams from DRAM once). Set by the host.
+  int m_fast;
 };
 
 // ============================================================== epilogue (per element)
@@ -350,8 +354,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
         const int z = tile / tiles_per_batch;
         const int r = tile % tiles_per_batch;
-        const int m0 = (r / n_tiles) * TC_BM;
-        const int n0 = (r % n_tiles) * BN;
+        const int m0 = (p.m_fast ? r % m_tiles : r / n_tiles) * TC_BM;
+        const int n0 = (p.m_fast ? r / m_tiles : r % n_tiles) * BN;
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
           const int s = it % C::STAGES;
           const uint32_t round = it / C::STAGES;
@@ -418,8 +422,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
       const int z = tile / tiles_per_batch;
       const int r = tile % tiles_per_batch;
-      const int m0 = (r / n_tiles) * TC_BM;
-      const int n0 = (r % n_tiles) * BN;
+      const int m0 = (p.m_fast ? r % m_tiles : r / n_tiles) * TC_BM;
+      const int n0 = (p.m_fast ? r / m_tiles : r % n_tiles) * BN;
       const int acc = lt & 1;
       const uint32_t use = lt >> 1;
       if (!mbar_wait(&acc_full[acc], use & 1, err, DEV_TIMEOUT_ACC)) break;

@@ -294,16 +294,15 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
   if (use_tc && p.batch > 1 && p.sD % 8 != 0) use_tc = false;
   if (use_tc && p.Y && !(aligned16(p.Y) && p.ldy % 8 == 0 && (p.batch == 1 || p.sY % 8 == 0))) use_tc = false;
   if (use_tc) {
-    // tile width: 256 (fewer A re-reads, longer MMAs) unless 128-wide tiles fill the
-    // persistent grid's waves clearly better (fraction of CTA slots busy over
-    // ceil(tiles / SMs) waves, by more than 5 points: small-M shapes)
+    // Tile width. A 128x256 tile does twice the work of a 128x128 one in about 1.32
+    // times its time (tensor pipe 68% vs 45% busy on the same frozen-block GEMMs), so
+    // 256 wins unless 128-wide tiles need fewer than 1.32x the persistent-grid waves
+    // (ceil(tiles / SMs)): the small-M shapes with N = 2048.
     const int m_tiles = (p.M + TC_BM - 1) / TC_BM;
-    auto wave_eff = [&](int bn) {
-      const double t = (double)m_tiles * (p.N / bn) * p.batch;
-      const double waves = std::ceil(t / num_sms);
-      return t / (waves * num_sms);
-    };
-    const bool n256 = (p.N % 256 == 0) && wave_eff(256) + 0.05 >= wave_eff(128);
+    auto waves = [&](int bn) { return std::ceil((double)m_tiles * (p.N / bn) * p.batch / num_sms); };
+    const bool n256 = (p.N % 256 == 0) && waves(128) >= 1.32 * waves(256);
+    // walk the larger operand once: column blocks outer when B is the larger matrix
+    pt.m_fast = p.N > p.M ? 1 : 0;
     bool ok = false;
     cudaError_t e;
     if (!p.a_mn && !p.b_mn)
