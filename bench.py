@@ -290,6 +290,11 @@ def run_ours(args):
         ms_e2e = _max_over_ranks(dist, e0.elapsed_time(e1), device)
         e2e_value = _sum_over_ranks(dist, float(cfg.batch * cfg.T * args.e2e_steps), device) / (ms_e2e / 1e3)
 
+    # Mean DRAM bytes (read + write) per launch of a kernel class, from one ncu capture of
+    # the current kernels (profiles/gemm_adaptive_chunk_b1_T8192.md: the 83 GEMM launches of
+    # one adaptive step, whose shapes do not depend on T). Classes without such a capture
+    # report null.
+    traffic_per_launch = {"gemm_adaptive": 38.05e6} if cfg.name == "b1_128k_bf16" and cfg.batch == 1 else {}
     peaks = measured_peaks()
     flops_step = model_flops(cfg)
     achieved_model = flops_step * args.steps / (ms / 1e3) / 1e12
@@ -318,7 +323,7 @@ def run_ours(args):
                 "d2h_bytes_per_step": int(loss_host.numel() * 4)},
         "gpu_launches": launches,
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                     "frac": ach / peak, "traffic": None,
+                     "frac": ach / peak, "traffic": traffic_per_launch.get(dom),
                      "peak_source": f"{peaks['source']} bf16 sustained (kernel timed inside a long step)"},
         "profile": {c: {"ms_per_step": v["ms"] / args.steps, "share": v["ms"] / ms,
                         "launches_per_step": v["launches"] / args.steps,
