@@ -218,6 +218,41 @@ def run_decode(T, args, device):
             "gpu_launches": launches}
 
 
+def run_full_attention(cfg, tok_dev, args, device):
+    """Comparator of the pages' speed claim (summary "Results": TTT-E2E prefill 2.7x
+    faster than full attention at 128K on one H100): the same architecture with no
+    adaptive block and full causal attention (window >= T), same tokens, same
+    kernels; prefill records the per-position losses. Reported beside the metric."""
+    import torch
+    import long_context_prefill_ttt_b200 as T
+    fcfg = cfg.replace(n_ttt=0, window_k=max(cfg.T, cfg.window_k))
+    w = syn.make_weights(fcfg)
+    wd = {k: torch.from_numpy(v).to(device) for k, v in w.items()}
+    del w
+    loss = torch.empty((fcfg.batch, fcfg.T), dtype=torch.float32, device=device)
+    h = T.ttt_create(fcfg, wd)
+    del wd
+    steps = args.comparator_steps
+    for _ in range(1):
+        T.ttt_reset(h)
+        T.ttt_prefill(h, tok_dev, loss)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        T.ttt_reset(h)
+        T.ttt_prefill(h, tok_dev, loss)
+    e1.record()
+    torch.cuda.synchronize()
+    assert torch.isfinite(loss).all().item(), "non-finite comparator loss"
+    ms = e0.elapsed_time(e1) / steps
+    del h
+    torch.cuda.empty_cache()
+    return {"workload": f"{fcfg.name} without adaptive blocks, full causal attention (k = {fcfg.window_k})",
+            "tokens_per_s": fcfg.batch * fcfg.T / (ms / 1e3), "ms_per_step": ms, "steps": steps, "warmup": 1,
+            "model_tflop_per_step": model_flops(fcfg) / 1e12}
+
+
 def run_ours(args):
     import torch
 
@@ -303,9 +338,17 @@ def run_ours(args):
     dp = prof[dom]
     ach = dp["flops"] / (dp["ms"] / 1e3) / 1e12 if dp["ms"] > 0 else 0.0
     peak = peaks["bf16_sustained"]
+    dev_bytes = T.ttt_device_bytes(h)
     decode = None
     if args.decode and rank == 0 and ws == 1:
         decode = run_decode(T, args, device)
+    comparator = None
+    if args.comparator and rank == 0 and ws == 1:
+        del h
+        torch.cuda.empty_cache()
+        h = None
+        comparator = run_full_attention(cfg, tok_dev, args, device)
+        comparator["ttt_e2e_speedup"] = value / comparator["tokens_per_s"]
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -314,7 +357,7 @@ def run_ours(args):
                                f"H{cfg.n_heads} h{cfg.mlp_hidden} ({cfg.ttt_hidden}+{cfg.static_hidden}) "
                                f"k{cfg.window_k} b{cfg.minibatch_b} T{cfg.T} B{cfg.batch}",
                    "tokens_per_step_per_gpu": cfg.batch * cfg.T, "parallelism": f"replicas x{ws}",
-                   "device_bytes": T.ttt_device_bytes(h),
+                   "device_bytes": dev_bytes,
                    "l2": "no flush: every step streams > 2.5 GB of weights and GBs of activations (L2 126 MB)"},
         "model_flops": {"tflop_per_step": flops_step / 1e12, "achieved_tflops": achieved_model,
                         "frac_of_peak": achieved_model / peaks["bf16"], "peak_tflops": peaks["bf16"],
@@ -332,6 +375,8 @@ def run_ours(args):
     }
     if decode is not None:
         line["decode"] = decode
+    if comparator is not None:
+        line["full_attention_comparator"] = comparator
     if rank == 0 and ws == 1 and args.cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, n_tokens=args.ref_tokens)
     if rank == 0:
@@ -358,6 +403,9 @@ def main():
     ap.add_argument("--decode-prefix", type=int, default=0)
     ap.add_argument("--decode-n", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-comparator", dest="comparator", action="store_false",
+                    help="skip the full-attention comparator (same architecture, no adaptive blocks, k >= T)")
+    ap.add_argument("--comparator-steps", type=int, default=2)
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -52,7 +52,11 @@ enum { TTT_PTR_HOST = 0, TTT_PTR_DEVICE = 1 };
 typedef struct ttt_handle ttt_handle;
 
 /* Model and inner-loop hyper-parameters. Notation: V vocab, d width, L layers,
- * L_t adaptive (last) layers, H heads (head dim d/H), k window, b mini-batch. */
+ * L_t adaptive (last) layers, H heads (head dim d/H), k window, b mini-batch.
+ * n_ttt = L_t may be 0: no block adapts, and the handle is the plain SWA
+ * Transformer (full causal attention when window_k >= T), whose prefill records
+ * the per-position losses only. It is the comparator the summary's speed claim
+ * is made against (TTT-E2E vs full attention at 128K, "Results"). */
 typedef struct {
   int32_t vocab, d, n_layers, n_heads, n_ttt;
   int32_t mlp_hidden;     /* frozen blocks' MLP hidden width h */

@@ -698,7 +698,8 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
     A.us = arena.get<T>((size_t)Mc * hs);
     A.gs = arena.get<T>((size_t)Mc * hs);
   }
-  tin = blk.empty() ? nullptr : blk[0].x;
+  // chunk input: the first adaptive block's input buffer, or its own buffer without adaptive blocks
+  tin = blk.empty() ? arena.get<float>((size_t)Mc * d) : blk[0].x;
   y = arena.get<float>((size_t)Mc * d);
   rstdf = arena.get<float>(Mc);
   rf = arena.get<T>((size_t)Mc * d);
@@ -925,10 +926,14 @@ template <typename T> int Engine<T>::frozen_mlp(const LayerDev<T>& Lw, float* x,
 }
 
 // Forward of the adaptive blocks for cn positions per sequence at pos..pos+cn-1.
-// Input in blk[0].x, output in y. Activations of each block stay in blk[j].
+// Input in tin, output in y. Activations of each block stay in blk[j].
 template <typename T> int Engine<T>::ttt_forward(int cn, int64_t pos, bool commit) {
   const int rows = B * cn;
   int rc;
+  if (Lt == 0) {  // no adaptive block: the head reads the frozen stack's output
+    TTT_CUDA(cudaMemcpyAsync(y, tin, (size_t)rows * d * 4, cudaMemcpyDeviceToDevice, st));
+    return TTT_OK;
+  }
   for (int j = 0; j < Lt; ++j) {
     const int l = first_ttt + j;
     const LayerDev<T>& Lw = layers[l];
@@ -1076,8 +1081,9 @@ int Engine<T>::ttt_step(const float* in, const int32_t* targets, int cn, int64_t
   int rc;
   chunk_pos = pos;
   gemm_class = PC_GEMM_TTT;
-  if (in != blk[0].x) {
-    TTT_CUDA(cudaMemcpyAsync(blk[0].x, in, (size_t)rows * d * 4, cudaMemcpyDeviceToDevice, st));
+  grad = grad && Lt > 0;  // without adaptive blocks there is nothing to update
+  if (in != tin) {
+    TTT_CUDA(cudaMemcpyAsync(tin, in, (size_t)rows * d * 4, cudaMemcpyDeviceToDevice, st));
   }
   if (targets != tgt) {
     TTT_CUDA(cudaMemcpyAsync(tgt, targets, (size_t)rows * 4, cudaMemcpyDeviceToDevice, st));
@@ -1137,15 +1143,15 @@ template <typename T> int Engine<T>::prefill(const int32_t* tokens, int64_t T_, 
     }
     for (int c0 = 0; c0 < n; c0 += bsz) {
       const int cn = (n - c0) < bsz ? (n - c0) : bsz;
-      gather_rows_kernel<<<nblk((int64_t)B * cn * d, 256), 256, 0, st>>>(xs, (int64_t)n * d, c0, cn, B, d, blk[0].x,
+      gather_rows_kernel<<<nblk((int64_t)B * cn * d, 256), 256, 0, st>>>(xs, (int64_t)n * d, c0, cn, B, d, tin,
                                                                         (int64_t)cn * d, 0);
       TTT_LAUNCHED();
       gather_tokens_kernel<<<nblk(B * cn, 256), 256, 0, st>>>(tok_dev, ld, s0 + c0 + 1, cn, B, tgt, cn, 0);
       TTT_LAUNCHED();
       const bool full = cn == bsz;
-      if ((rc = ttt_step(blk[0].x, tgt, cn, P0 + c0, lout, T_, s0 + c0, full, true)) != TTT_OK) return rc;
+      if ((rc = ttt_step(tin, tgt, cn, P0 + c0, lout, T_, s0 + c0, full, true)) != TTT_OK) return rc;
       if (!full) {  // trailing partial chunk: keep its inputs and targets pending
-        TTT_CUDA(cudaMemcpy2DAsync(pend_in, (size_t)bsz * d * 4, blk[0].x, (size_t)cn * d * 4, (size_t)cn * d * 4, B,
+        TTT_CUDA(cudaMemcpy2DAsync(pend_in, (size_t)bsz * d * 4, tin, (size_t)cn * d * 4, (size_t)cn * d * 4, B,
                                    cudaMemcpyDeviceToDevice, st));
         TTT_CUDA(cudaMemcpy2DAsync(pend_tgt, (size_t)bsz * 4, tgt, (size_t)cn * 4, (size_t)cn * 4, B,
                                    cudaMemcpyDeviceToDevice, st));
@@ -1184,7 +1190,7 @@ template <typename T> int Engine<T>::decode_token_launches(int64_t n, int32_t* o
   // keep the first adaptive block's input of this position for the chunk's update
   pend_store_kernel<<<nblk((int64_t)B * d, 256), 256, 0, st>>>(xs, B, d, pend_in, bsz, pos_dev);
   TTT_LAUNCHED();
-  TTT_CUDA(cudaMemcpyAsync(blk[0].x, xs, (size_t)B * d * 4, cudaMemcpyDeviceToDevice, st));
+  TTT_CUDA(cudaMemcpyAsync(tin, xs, (size_t)B * d * 4, cudaMemcpyDeviceToDevice, st));
   gemm_class = PC_GEMM_TTT;
   if ((rc = ttt_forward(1, 0, true)) != TTT_OK) return rc;
   rmsnorm_fwd_launch<T>((const float*)y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf, st);
@@ -1274,7 +1280,7 @@ int Engine<T>::decode(int64_t n, const int32_t* forced, int32_t* out_tok, float*
     ++pend_cnt;
     ++n_pos;
     if (pend_cnt == bsz) {  // a full chunk of decoded positions: differentiate and update
-      if ((rc = ttt_step(pend_in, pend_tgt, bsz, n_pos - bsz, nullptr, 0, 0, true, false)) != TTT_OK) {
+      if (Lt > 0 && (rc = ttt_step(pend_in, pend_tgt, bsz, n_pos - bsz, nullptr, 0, 0, true, false)) != TTT_OK) {
         cudaGraphExecDestroy(exec);
         return rc;
       }
@@ -1330,7 +1336,7 @@ static int validate(const ttt_config* c, std::string* why) {
   auto bad = [&](const char* m) { *why = m; return TTT_ERR_INVALID_ARG; };
   if (!c) return bad("null config");
   if (c->vocab <= 0 || c->d <= 0 || c->n_layers <= 0 || c->n_heads <= 0 || c->batch <= 0) return bad("non-positive size");
-  if (c->n_ttt < 1 || c->n_ttt > c->n_layers) return bad("n_ttt must be in [1, n_layers]");
+  if (c->n_ttt < 0 || c->n_ttt > c->n_layers) return bad("n_ttt must be in [0, n_layers]");
   if (c->d % c->n_heads) return bad("d must be a multiple of n_heads");
   const int hd = c->d / c->n_heads;
   if (hd != 16 && hd != 32 && hd != 64 && hd != 128) return bad("head dim must be 16, 32, 64 or 128");

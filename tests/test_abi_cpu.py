@@ -47,7 +47,7 @@ def test_weight_tensor_count_and_order_match_the_generator():
         assert T.weight_names(cfg) == [n for n, _ in syn.weight_shapes(cfg)]
 
 
-@pytest.mark.parametrize("field,value", [("window_k", 8), ("n_ttt", 0), ("n_ttt", 9), ("d", 63),
+@pytest.mark.parametrize("field,value", [("window_k", 8), ("n_ttt", -1), ("n_ttt", 9), ("d", 63),
                                          ("minibatch_b", 0), ("vocab", 0), ("n_heads", 5)])
 def test_create_rejects_invalid_configs_without_touching_the_device(field, value):
     import long_context_prefill_ttt_b200 as T

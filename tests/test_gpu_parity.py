@@ -34,6 +34,8 @@ def T():
     (dict(n_ttt=2), 0),                                   # attention backward inside the adaptive blocks
     (dict(n_ttt=2, batch=3, window_k=40, T=200), 48),     # batch, window > b, ragged tail chunk pending
     (dict(n_ttt=4, T=96, minibatch_b=32, window_k=32), 0),  # every block adaptive
+    (dict(n_ttt=0), 0),                                   # no adaptive block: the plain SWA model
+    (dict(n_ttt=0, window_k=512), 64),                    # ... with full causal attention (k >= T), 4 segments
 ])
 def test_tiny_fp32_matches_oracle(T, overrides, seg):
     cfg = syn.config("tiny_fp32", **overrides)
@@ -88,8 +90,9 @@ def test_sequences_are_independent(T):
         assert P.max_rel(together[s], alone[0]) <= 1e-6
 
 
-def test_decode_fp32_greedy_and_teacher_forced(T):
-    cfg = syn.config("tiny_fp32", n_ttt=2, T=40)
+@pytest.mark.parametrize("n_ttt", [2, 0])
+def test_decode_fp32_greedy_and_teacher_forced(T, n_ttt):
+    cfg = syn.config("tiny_fp32", n_ttt=n_ttt, T=40)
     w = syn.make_weights(cfg)
     toks = syn.make_token_batch(cfg)
     h = T.ttt_create(cfg, w)
@@ -144,6 +147,13 @@ def test_small_bf16_matches_oracle(T):
     P.compare(cfg, r["w"], r["gpu_losses"], r["orc_losses"], r["gpu_w"], r["orc_w"], report=rep)
     print("small_bf16", rep)
     assert rep["dw"] <= 5e-2
+
+
+def test_small_bf16_full_attention_without_adaptive_blocks_matches_oracle(T):
+    """The comparator model of the speed claim: no adaptive block, window >= T."""
+    cfg = syn.config("small_bf16", n_ttt=0, T=2048, window_k=4096)
+    r = P.prefill_both(T, cfg)
+    P.compare(cfg, r["w"], r["gpu_losses"], r["orc_losses"], r["gpu_w"], r["orc_w"])
 
 
 def test_bf16_update_effect_matches_oracle(T):

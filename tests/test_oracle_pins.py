@@ -172,7 +172,7 @@ def test_chunk_gradient_matches_finite_differences_with_constant_cache(n_ttt):
             np.testing.assert_allclose(grads[j][name], num, rtol=1e-5, atol=1e-9)
 
 
-@pytest.mark.parametrize("n_ttt", [1, 2])
+@pytest.mark.parametrize("n_ttt", [0, 1, 2])
 def test_eta_zero_reproduces_static_swa_model(n_ttt):
     cfg = tiny(n_ttt=n_ttt, eta=0.0, T=24)
     w = weights(cfg)
@@ -188,7 +188,7 @@ def test_eta_zero_reproduces_static_swa_model(n_ttt):
         assert np.array_equal(W2, w[f"layers.{l}.W2t"].astype(np.float64))
 
 
-@pytest.mark.parametrize("n_ttt", [1, 2])
+@pytest.mark.parametrize("n_ttt", [0, 1, 2])
 def test_full_window_reproduces_full_causal_attention_model(n_ttt):
     cfg = tiny(n_ttt=n_ttt, eta=0.0, window_k=64, minibatch_b=8, T=24)
     w = weights(cfg)
