@@ -3,8 +3,8 @@
 
 One step = one ttt_prefill call over the whole 128K-token sequence of the ~1B
 workload (V32000 d2048 L24, last 6 blocks adaptive, H16, k8192, b1024, T131072,
-B1), after ttt_reset (a fresh per-sequence copy of W_init: review §7 Alg. 1
-step 1). The step runs every row of the hot path: embedding, the frozen blocks
+B1), after ttt_reset (a fresh per-sequence copy of W_init: review §7,
+Algorithm 1). The step runs every row of the hot path: embedding, the frozen blocks
 over all positions, then 128 sequential mini-batch steps of adaptive-block
 forward, fused LM-head cross-entropy forward/backward, backward into the
 adaptive MLPs and the fused SGD update. Inputs are synthetic (seeded Zipf +
@@ -233,9 +233,8 @@ def run_full_attention(cfg, tok_dev, args, device):
     h = T.ttt_create(fcfg, wd)
     del wd
     steps = args.comparator_steps
-    for _ in range(1):
-        T.ttt_reset(h)
-        T.ttt_prefill(h, tok_dev, loss)
+    T.ttt_reset(h)
+    T.ttt_prefill(h, tok_dev, loss)  # warm-up
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()

@@ -96,7 +96,7 @@ int32_t ttt_num_weight_tensors(const ttt_config* cfg);
 /* Validate cfg (k >= b, d % H == 0, widths multiples of 8, ...), allocate
  * device state (frozen weights, B copies of the fast weights W_init as fp32
  * master + bf16 shadow, window caches of roundup(k + b, 128) positions per
- * layer and sequence, workspace) and copy the weights (review Alg. 1 step 1:
+ * layer and sequence, workspace) and copy the weights (review §7, Algorithm 1:
  * every sequence starts from a fresh copy of W_init). *out receives the handle
  * (NULL on failure). On failure nothing is leaked. */
 int ttt_create(const ttt_config* cfg, const ttt_weights* w, ttt_handle** out);
@@ -104,8 +104,8 @@ int ttt_create(const ttt_config* cfg, const ttt_weights* w, ttt_handle** out);
 /* Algorithm 1 over T positions of each of the B sequences.
  * tokens [B][T+1] int32 (x_0..x_T per sequence, row stride T+1): positions 0..T-1
  * are processed and out_losses[b][t-1] = l_t = -log p(x_t | x_<t) for t = 1..T,
- * every loss of chunk i scored with W_{i-1} before the update (review §5,
- * Alg. 1 step 3.3). Chunks are the global grid [(i-1)b, ib) of positions since
+ * every loss of chunk i scored with W_{i-1} before the update (review §5 and
+ * Algorithm 1). Chunks are the global grid [(i-1)b, ib) of positions since
  * creation/reset; a chunk updates W only when complete; a trailing partial
  * chunk stays pending (decode completes it). x_T becomes the pending input.
  * A continuing call must start with the pending id (else TTT_ERR_STREAM) and
@@ -126,8 +126,8 @@ int ttt_decode(ttt_handle* h, int64_t n, const int32_t* forced, int32_t* out_tok
  * w1 [h_t][d] and w2 [d][h_t] (either may be NULL). */
 int ttt_get_weights(ttt_handle* h, int32_t seq, int32_t ttt_block, float* w1, float* w2, int32_t ptr_kind);
 
-/* Fast weights <- W_init, window caches and pending state cleared (review
- * Alg. 2 step 7: adapted state is discarded between documents). */
+/* Fast weights <- W_init, window caches and pending state cleared (review §7,
+ * Algorithm 2: adapted state is discarded between documents). */
 int ttt_reset(ttt_handle* h);
 
 /* Positions processed so far (per sequence). */

@@ -20,9 +20,9 @@ What it computes follows the pages describing End-to-End Test-Time Training
   * Algorithm 1 (causal prefill with adaptation) and Algorithm 3 (generation
     with periodic adaptation, update after a full mini-batch of generated
     tokens) - review §7; per-sequence fresh copy of the fast weights -
-    review §7, Algorithm 1 step 1.
+    review §7, Algorithm 1.
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   R1 T+1 ids x_0..x_T in, T positions processed, out_losses[t-1] = l_t.
   R2 query at position p attends to keys [p-k+1, p]; k >= T is full attention.
   R3 K/V cached from earlier chunks are constants: gradients flow only through
@@ -186,7 +186,7 @@ class _History:
 
 
 class _Seq:
-    """Per-sequence state: a fresh copy of the fast weights (review §7, Alg. 1 step 1)."""
+    """Per-sequence state: a fresh copy of the fast weights (review §7, Algorithm 1)."""
 
     def __init__(self, cfg, w0):
         self.fast = [{"W1t": w0[f"layers.{l}.W1t"].copy(), "W2t": w0[f"layers.{l}.W2t"].copy()}

@@ -11,9 +11,9 @@ Each test names what it pins:
     review eq. (9)); b=1 is online GD (review eq. (3));
   * k >= T equals textbook causal softmax attention (review §9.2: an 8K window
     at 8K length is full attention);
-  * causality of scoring (review §2.2 and §7, Alg. 1 step 3.3), only the
+  * causality of scoring (review §2.2 and §7, Algorithm 1), only the
     adaptive MLPs change (summary, "Selective Parameter Update"), sequences are
-    independent (review §7, Alg. 1 step 1, Alg. 2 step 7), decode updates only
+    independent (review §7, Algorithms 1 and 2), decode updates only
     after a full chunk (summary, "Decoding Multiple Tokens"; review Alg. 3).
 """
 import math
