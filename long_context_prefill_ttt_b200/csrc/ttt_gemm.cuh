@@ -218,7 +218,10 @@ __global__ void __launch_bounds__(256) gemm_skinny_kernel(GemmParams p) {
 // ============================================================== tcgen05 engine
 constexpr int TC_BM = 128;
 constexpr int TC_BK = 64;
-constexpr int TC_THREADS = 192;  // warp 0: TMA, warp 1: MMA + TMEM owner, warps 2-5: epilogue
+// warp 0: TMA, warp 1: MMA + TMEM owner, warps 2-9: epilogue (two warps per TMEM lane
+// quarter, each taking half of the tile's columns)
+constexpr int TC_THREADS = 320;
+constexpr int TC_EPI_WARPS = 8;
 
 template <int BN> struct TcCfg {
   static constexpr int STAGES = (BN == 256) ? 4 : 6;
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 4); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], TC_EPI_WARPS); }
     fence_mbar_init();
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
@@ -415,8 +418,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
     }
   } else {
-    // epilogue warps 2..5: TMEM lane quarter = warp % 4
+    // epilogue warps 2..9: TMEM lane quarter = warp % 4; warps 2-5 take columns
+    // [0, BN/2) of the tile, warps 6-9 columns [BN/2, BN)
     const int quarter = warp & 3;
+    const int c_first = (warp >= 6 ? 1 : 0) * (BN / 64);
     const int row_in_tile = quarter * 32 + (threadIdx.x & 31);
     int lt = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
@@ -431,14 +436,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int m = m0 + row_in_tile;
       const uint32_t taddr = tmem_base + acc * BN + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = c_first; c < c_first + BN / 64; ++c) {
         float v[32];
         tmem_ld32(taddr + c * 32, v);
+        if (c == c_first + BN / 64 - 1) {  // this warp's columns are read: its share of the accumulator is free
+          tc_fence_before();
+          __syncwarp();
+          if (elect_lane0()) mbar_arrive(&acc_empty[acc]);
+        }
         if (m < p.M) epi_row32<bf16>(p, z, m, n0 + c * 32, v);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (elect_lane0()) mbar_arrive(&acc_empty[acc]);
     }
   }
   tc_fence_before();
