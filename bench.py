@@ -328,7 +328,7 @@ def run_ours(args):
     # the current kernels (profiles/gemm_adaptive_chunk_b1_T8192.md: the 83 GEMM launches of
     # one adaptive step, whose shapes do not depend on T). Classes without such a capture
     # report null.
-    traffic_per_launch = {"gemm_adaptive": 38.05e6} if cfg.name == "b1_128k_bf16" and cfg.batch == 1 else {}
+    traffic_per_launch = {"gemm_adaptive": 38.03e6} if cfg.name == "b1_128k_bf16" and cfg.batch == 1 else {}
     peaks = measured_peaks()
     flops_step = model_flops(cfg)
     achieved_model = flops_step * args.steps / (ms / 1e3) / 1e12
