@@ -116,6 +116,53 @@ def _ptr(x):
     return x.data_ptr(), (TTT_PTR_DEVICE if x.is_cuda else TTT_PTR_HOST)
 
 
+def _is_torch(x):
+    return not isinstance(x, np.ndarray) and hasattr(x, "data_ptr")
+
+
+def _elem_name(x):
+    if isinstance(x, np.ndarray):
+        return str(x.dtype)
+    return str(x.dtype).replace("torch.", "")
+
+
+def _check(x, name, dtypes, min_elems=None, shape=None, cuda=None):
+    """Validate a buffer handed to the library, which only sees its address: element
+    type in dtypes (names such as "int32", "float32", "bfloat16"), contiguous, and
+    covering min_elems elements (or exactly `shape`). cuda=True/False requires a
+    device/host buffer. Raises ValueError before anything reaches the device."""
+    if x is None:
+        raise ValueError(f"{name}: missing buffer")
+    if _elem_name(x) not in dtypes:
+        raise ValueError(f"{name}: element type {_elem_name(x)}, expected {' or '.join(dtypes)}")
+    contiguous = x.flags["C_CONTIGUOUS"] if isinstance(x, np.ndarray) else x.is_contiguous()
+    if not contiguous:
+        raise ValueError(f"{name}: must be contiguous")
+    if shape is not None and tuple(x.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(x.shape)}, expected {tuple(shape)}")
+    numel = x.size if isinstance(x, np.ndarray) else x.numel()
+    if min_elems is not None and numel < min_elems:
+        raise ValueError(f"{name}: {numel} elements, the call reads or writes {min_elems}")
+    if cuda is not None:
+        on_cuda = _is_torch(x) and x.is_cuda
+        if on_cuda != cuda:
+            raise ValueError(f"{name}: must be a {'device' if cuda else 'host'} buffer")
+
+
+def _on_device(**bufs):
+    for name, x in bufs.items():
+        if x is not None and not (_is_torch(x) and x.is_cuda):
+            raise ValueError(f"{name}: must be a device buffer")
+
+
+def _extent(rows, cols, ld, stride, batch):
+    """Elements spanned by `batch` row-major [rows][cols] slices with leading dimension
+    ld, `stride` apart (stride 0: one slice shared by all)."""
+    if rows <= 0 or cols <= 0:
+        return 0
+    return (batch - 1) * stride + (rows - 1) * ld + cols
+
+
 def _get(cfg, name, default=None):
     if isinstance(cfg, dict):
         return cfg.get(name, default)
@@ -180,15 +227,34 @@ class Handle:
 
 # ----------------------------------------------------------------------------- C ABI, same names
 
+def weight_shapes(cfg):
+    """Element counts of the weight tensors, in weight_names order (include/ttt.h)."""
+    V, d = _get(cfg, "vocab"), _get(cfg, "d")
+    L, Lt = _get(cfg, "n_layers"), _get(cfg, "n_ttt")
+    h, ht, hs = _get(cfg, "mlp_hidden"), _get(cfg, "ttt_hidden"), _get(cfg, "static_hidden")
+    out = [V * d, d]
+    for l in range(L):
+        out += [d, d * d, d * d, d * d, d * d]
+        if l >= L - Lt:
+            out += [d, ht * d, d * ht, d, hs * d, d * hs]
+        else:
+            out += [d, h * d, d * h]
+    return out
+
+
 def ttt_create(cfg, weights, stream=None, max_segment=0) -> Handle:
     """weights: dict name -> float32 array/tensor (values exactly representable in cfg's dtype)."""
     c = make_config(cfg, stream, max_segment)
     names = weight_names(cfg)
     ptrs, kinds, keep = [], set(), []
-    for n in names:
+    for n, numel in zip(names, weight_shapes(cfg)):
         t = weights[n]
         if isinstance(t, np.ndarray):
             t = np.ascontiguousarray(t, dtype=np.float32)
+        _check(t, n, ("float32",))
+        tn = t.size if isinstance(t, np.ndarray) else t.numel()
+        if tn != numel:
+            raise ValueError(f"{n}: {tn} elements, the model has {numel}")
         keep.append(t)
         p, k = _ptr(t)
         ptrs.append(p)
@@ -206,16 +272,20 @@ def ttt_create(cfg, weights, stream=None, max_segment=0) -> Handle:
 
 def ttt_prefill(h: Handle, tokens, out_losses=None):
     """tokens [B][T+1] int32; returns losses [B][T] (float32, same kind as tokens)."""
+    if len(tokens.shape) != 2 or tokens.shape[0] != h.batch or tokens.shape[1] < 2:
+        raise ValueError(f"tokens: shape {tuple(tokens.shape)}, expected [B={h.batch}][T+1] with T >= 1")
     B, n1 = tokens.shape
     T = n1 - 1
+    on_cuda = _is_torch(tokens) and tokens.is_cuda
+    _check(tokens, "tokens", ("int32",))
     if out_losses is None:
         if isinstance(tokens, np.ndarray):
             out_losses = np.empty((B, T), dtype=np.float32)
         else:
             out_losses = _torch().empty((B, T), dtype=_torch().float32, device=tokens.device)
+    _check(out_losses, "out_losses", ("float32",), shape=(B, T), cuda=on_cuda)
     tp, kind = _ptr(tokens)
-    lp, kind2 = _ptr(out_losses)
-    assert kind == kind2
+    lp, _ = _ptr(out_losses)
     h.check(lib.ttt_prefill(h.ptr, ctypes.c_void_p(tp), T, ctypes.c_void_p(lp), kind))
     return out_losses
 
@@ -228,6 +298,8 @@ def ttt_decode(h: Handle, n: int, forced=None, device=None):
         toks = torch.empty((B, n), dtype=torch.int32, device=device)
         losses = torch.empty((B, n), dtype=torch.float32, device=device)
         kind = TTT_PTR_DEVICE
+        if forced is not None:
+            _check(forced, "forced", ("int32",), shape=(B, n), cuda=True)
         fp = forced.data_ptr() if forced is not None else None
         tp, lp = toks.data_ptr(), losses.data_ptr()
     else:
@@ -236,6 +308,7 @@ def ttt_decode(h: Handle, n: int, forced=None, device=None):
         kind = TTT_PTR_HOST
         if forced is not None:
             forced = np.ascontiguousarray(forced, dtype=np.int32)
+            _check(forced, "forced", ("int32",), shape=(B, n))
         fp = forced.ctypes.data if forced is not None else None
         tp, lp = toks.ctypes.data, losses.ctypes.data
     h.check(lib.ttt_decode(h.ptr, n, ctypes.c_void_p(fp) if fp else None, ctypes.c_void_p(tp),
@@ -316,6 +389,23 @@ def ttt_k_gemm(A, B, D, M, N, K, *, batch=1, lda=None, sA=0, a_mn=False, ldb=Non
     lda = lda if lda is not None else (M if a_mn else K)
     ldb = ldb if ldb is not None else (N if b_mn else K)
     ldd = ldd if ldd is not None else N
+    el = (_elem_name(A),)
+    if el[0] not in ("bfloat16", "float32"):
+        raise ValueError(f"A: element type {el[0]}, expected bfloat16 or float32")
+    a_rows, a_cols = (K, M) if a_mn else (M, K)
+    b_rows, b_cols = (K, N) if b_mn else (N, K)
+    if lda < a_cols or ldb < b_cols or ldd < N:
+        raise ValueError("leading dimensions must cover a row")
+    _check(A, "A", el, _extent(a_rows, a_cols, lda, sA, batch))
+    _check(B, "B", el, _extent(b_rows, b_cols, ldb, sB, batch))
+    if B2 is not None:
+        _check(B2, "B2", el, _extent(b_rows, b_cols, ldb, sB2, batch))
+    _check(D, "D", ("float32",) + el, _extent(M, N, ldd, sD, batch))
+    if X is not None:
+        _check(X, "X", ("float32",) if epi == EPI_RESID else el, _extent(M, N, ldx, sX, batch))
+    if Y is not None:
+        _check(Y, "Y", el, _extent(M, N, ldy, sY, batch))
+    _on_device(A=A, B=B, B2=B2, D=D, X=X, Y=Y)
     rc = lib.ttt_k_gemm(_dtype_code(A), M, N, K, batch, A.data_ptr(), lda, sA, int(a_mn), B.data_ptr(), ldb, sB,
                         int(b_mn), B2.data_ptr() if B2 is not None else None, sB2, D.data_ptr(), ldd, sD,
                         int(D.dtype == torch.float32),
@@ -326,8 +416,29 @@ def ttt_k_gemm(A, B, D, M, N, K, *, batch=1, lda=None, sA=0, a_mn=False, ldb=Non
         raise TTTError(rc, "ttt_k_gemm")
 
 
+def _check_attention(qkv, out, lse, B, H, hd, n, q0, ring_k, ring_v, C, dout=None, dqkv=None, dsum=None):
+    el = (_elem_name(qkv),)
+    d = H * hd
+    _check(qkv, "qkv", el, B * n * 3 * d)
+    _check(out, "out", el, B * n * d)
+    if lse is not None:
+        _check(lse, "lse", ("float32",), B * H * n)
+    if q0 > 0:
+        _check(ring_k, "ring_k", el, B * C * d)
+        _check(ring_v, "ring_v", el, B * C * d)
+    if dout is not None:
+        _check(dout, "dout", el, B * n * d)
+    if dqkv is not None:
+        _check(dqkv, "dqkv", el, B * n * 3 * d)
+    if dsum is not None:
+        _check(dsum, "dsum", ("float32",), B * H * n)
+    _on_device(qkv=qkv, out=out, lse=lse, ring_k=ring_k if q0 > 0 else None, ring_v=ring_v if q0 > 0 else None,
+               dout=dout, dqkv=dqkv, dsum=dsum)
+
+
 def ttt_k_attention_fwd(qkv, out, lse, B, H, hd, n, q0, window, ring_k=None, ring_v=None, C=0,
                         engine=ENGINE_AUTO, stream=None):
+    _check_attention(qkv, out, lse, B, H, hd, n, q0, ring_k, ring_v, C)
     rc = lib.ttt_k_attention_fwd(_dtype_code(qkv), B, H, hd, n, q0, window, qkv.data_ptr(),
                                  ring_k.data_ptr() if ring_k is not None else None,
                                  ring_v.data_ptr() if ring_v is not None else None, C, out.data_ptr(),
@@ -338,6 +449,9 @@ def ttt_k_attention_fwd(qkv, out, lse, B, H, hd, n, q0, window, ring_k=None, rin
 
 def ttt_k_attention_bwd(qkv, out, lse, dout, dqkv, dsum, B, H, hd, n, q0, window, ring_k=None, ring_v=None, C=0,
                         engine=ENGINE_AUTO, stream=None):
+    if lse is None:
+        raise ValueError("lse: missing buffer")
+    _check_attention(qkv, out, lse, B, H, hd, n, q0, ring_k, ring_v, C, dout=dout, dqkv=dqkv, dsum=dsum)
     rc = lib.ttt_k_attention_bwd(_dtype_code(qkv), B, H, hd, n, q0, window, qkv.data_ptr(),
                                  ring_k.data_ptr() if ring_k is not None else None,
                                  ring_v.data_ptr() if ring_v is not None else None, C, out.data_ptr(),
@@ -350,6 +464,9 @@ def ttt_k_attention_bwd(qkv, out, lse, dout, dqkv, dsum, B, H, hd, n, q0, window
 def ttt_k_attention_bwd_noalloc(qkv, out, lse, dout, dqkv, B, H, hd, n, q0, window, ring_k=None, ring_v=None, C=0,
                                 engine=ENGINE_AUTO, stream=None):
     """Attention backward that allocates nothing (its scratch is a fixed array inside the library)."""
+    if lse is None:
+        raise ValueError("lse: missing buffer")
+    _check_attention(qkv, out, lse, B, H, hd, n, q0, ring_k, ring_v, C, dout=dout, dqkv=dqkv)
     rc = lib.ttt_k_attention_bwd_noalloc(_dtype_code(qkv), B, H, hd, n, q0, window, qkv.data_ptr(),
                                          ring_k.data_ptr() if ring_k is not None else None,
                                          ring_v.data_ptr() if ring_v is not None else None, C, out.data_ptr(),

@@ -4,7 +4,9 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
+import torch
 
 import synthetic as syn
 
@@ -69,3 +71,47 @@ def test_null_handle_calls_return_invalid_arg():
     assert T.lib.ttt_reset(None) == T.TTT_ERR_INVALID_ARG
     assert T.lib.ttt_position(None) == -1
     T.lib.ttt_destroy(None)
+
+
+def test_binding_refuses_buffers_that_do_not_cover_the_call():
+    """The library sees only addresses, so the binding checks element types and extents
+    first: nothing undersized or mistyped reaches a kernel."""
+    import long_context_prefill_ttt_b200 as T
+    bf = torch.bfloat16
+    M, N, K = 64, 128, 64
+    A, B, D = torch.zeros(M, K, dtype=bf), torch.zeros(N, K, dtype=bf), torch.zeros(M, N)
+    with pytest.raises(ValueError, match="A: .* elements"):
+        T.ttt_k_gemm(A[:10], B, D, M, N, K)
+    with pytest.raises(ValueError, match="D: .* elements"):
+        T.ttt_k_gemm(A, B, D[:5], M, N, K)
+    with pytest.raises(ValueError, match="X: element type"):
+        T.ttt_k_gemm(A, B, D, M, N, K, X=torch.zeros(M, N, dtype=bf), ldx=N, epi=T.EPI_RESID)
+    with pytest.raises(ValueError, match="B2: .* elements"):
+        T.ttt_k_gemm(A, B, D, M, N, K, batch=2, sA=0, sB=0, B2=B, sB2=N * K, sD=0)
+    with pytest.raises(ValueError, match="must be a device buffer"):
+        T.ttt_k_gemm(A, B, D, M, N, K)       # right sizes, but host memory
+    qkv, out, lse = torch.zeros(4 * 3 * 64, dtype=bf), torch.zeros(4 * 64, dtype=bf), torch.zeros(4)
+    with pytest.raises(ValueError, match="ring_k"):
+        T.ttt_k_attention_fwd(qkv, out, lse, 1, 1, 64, 4, 128, 64, None, None, 256)
+    with pytest.raises(ValueError, match="qkv: .* elements"):
+        T.ttt_k_attention_fwd(qkv, out, lse, 1, 2, 64, 4, 0, 64)
+
+
+def test_binding_checks_prefill_and_create_inputs():
+    import long_context_prefill_ttt_b200 as T
+    cfg = syn.config("tiny_fp32", T=32)
+    h = T.Handle(None, cfg, T.make_config(cfg))   # never reaches the library: inputs are refused first
+    toks = syn.make_token_batch(cfg)
+    with pytest.raises(ValueError, match="int32"):
+        T.ttt_prefill(h, toks.astype(np.int64))
+    with pytest.raises(ValueError, match="shape"):
+        T.ttt_prefill(h, np.ascontiguousarray(np.concatenate([toks, toks])))
+    with pytest.raises(ValueError, match="out_losses"):
+        T.ttt_prefill(h, toks, np.zeros((1, 31), dtype=np.float32))
+    with pytest.raises(ValueError, match="forced"):
+        T.ttt_decode(h, 4, forced=np.zeros((1, 3), dtype=np.int32))
+    w = syn.make_weights(cfg)
+    w["layers.0.Wq"] = w["layers.0.Wq"][:-1]
+    with pytest.raises(ValueError, match="layers.0.Wq"):
+        T.ttt_create(cfg, w)
+    assert T.weight_shapes(cfg) == [int(np.prod(s)) for _, s in syn.weight_shapes(cfg)]

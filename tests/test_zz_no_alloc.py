@@ -53,7 +53,10 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(T):
     out = torch.empty((8, 64), dtype=torch.bfloat16, device="cuda")
     lse = torch.empty((1, 1, 8), dtype=torch.float32, device="cuda")
     dq = torch.empty((8, 192), dtype=torch.bfloat16, device="cuda")
-    # B*H*n = 1 * 16 * 65537 > 1048576 rows of scratch: rejected before any launch
-    with pytest.raises(T.TTTError) as e:
+    # B*H*n = 1 * 16 * 65537 > 1048576 rows of scratch: the library rejects the call before any
+    # launch (called directly: the binding would already refuse the buffers as too small)
+    rc = T.lib.ttt_k_attention_bwd_noalloc(T.TTT_BF16, 1, 16, 64, 65537, 0, 64, qkv.data_ptr(), None, None, 0,
+                                           out.data_ptr(), lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), 0, None)
+    assert rc == T.TTT_ERR_INVALID_ARG
+    with pytest.raises(ValueError):
         T.ttt_k_attention_bwd_noalloc(qkv, out, lse, dout, dq, 1, 16, 64, 65537, 0, 64)
-    assert e.value.code == T.TTT_ERR_INVALID_ARG
