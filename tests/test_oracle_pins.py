@@ -362,3 +362,46 @@ def test_cross_entropy_gradient_rows_sum_to_zero():
     p = np.exp(z - lse[:, None])
     np.testing.assert_allclose(p.sum(axis=1), 1.0, rtol=1e-14)
     assert np.all(lse - z.max(axis=1) >= 0)
+
+
+# ----------------------------------------------------------------------------- window cache of later adaptive blocks
+
+@pytest.mark.parametrize("n_ttt,b,k,T", [(2, 4, 6, 16), (3, 4, 9, 18), (2, 3, 5, 14)])
+def test_multi_block_trajectory_matches_chunkwise_autograd_with_cache_as_computed(n_ttt, b, k, T):
+    """With two or more adaptive blocks the keys/values that a later adaptive block caches
+    depend on W. Reading R4: a cached key/value keeps the value computed when its chunk ran
+    (with that chunk's W_{i-1}) and is a constant afterwards (technical review §7,
+    Algorithm 1, attention state carried across chunks; §5, eq. (9)). An independent
+    chunk-wise loop (library SDPA and autograd, tests/torch_static.py) must reproduce the
+    oracle's losses and final fast weights; the two plausible misreadings must not."""
+    cfg = tiny(n_ttt=n_ttt, minibatch_b=b, window_k=k, T=T, eta=0.5)
+    w = weights(cfg)
+    toks = tokens(cfg)
+    orc = Oracle(cfg, w)
+    losses = orc.prefill(toks)
+    ref_losses, ref_fast = TS.mini_batch_ttt_chunked(cfg, w, toks[0], "as_computed")
+    np.testing.assert_allclose(losses[0], ref_losses.numpy(), rtol=1e-10, atol=1e-12)
+    for j in range(n_ttt):
+        W1, W2 = orc.fast_weights(0, j)
+        np.testing.assert_allclose(W1, ref_fast[j]["W1t"].numpy(), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(W2, ref_fast[j]["W2t"].numpy(), rtol=1e-10, atol=1e-12)
+    # negative controls, far outside the tolerance above: recomputing the cache with the
+    # current W changes chunk 2 on (chunk 1's K/V would carry W_1 instead of W_0); keeping
+    # the K/V of W_0 agrees through chunk 2 (chunk 1 ran with W_0) and changes chunk 3 on
+    for rule, same in (("recompute_current", b), ("initial_weights", 2 * b)):
+        alt, _ = TS.mini_batch_ttt_chunked(cfg, w, toks[0], rule)
+        np.testing.assert_allclose(alt[:same].numpy(), losses[0, :same], rtol=1e-10, atol=1e-12)
+        assert np.max(np.abs(alt[same:same + b].numpy() - losses[0, same:same + b])) > 1e-6, rule
+
+
+def test_chunkwise_autograd_reduces_to_the_static_loop_with_one_adaptive_block():
+    """Cross-check of the two autograd references: with one adaptive block nothing cached
+    depends on W, so every cache rule gives the whole-sequence loop's trajectory."""
+    cfg = tiny(n_ttt=1, minibatch_b=4, window_k=6, T=14)
+    w = weights(cfg)
+    toks = tokens(cfg)
+    ref_losses, ref_fast = TS.mini_batch_ttt_single_adaptive_block(cfg, w, toks[0])
+    for rule in ("as_computed", "recompute_current", "initial_weights"):
+        got, fast = TS.mini_batch_ttt_chunked(cfg, w, toks[0], rule)
+        np.testing.assert_allclose(got.numpy(), ref_losses.numpy(), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(fast[0]["W1t"].numpy(), ref_fast[0]["W1t"].numpy(), rtol=1e-10, atol=1e-12)

@@ -3,10 +3,12 @@
 Test-only. It is written separately from the oracle (no shared code) and uses
 library routines where they exist (rms_norm, scaled_dot_product_attention with
 an explicit window mask, exact gelu, cross_entropy); RoPE is written as a
-complex rotation of the pairs (i, i + hd/2). It processes all positions at once
-with fixed weights, so it is the static sliding-window model; with autograd it
-also gives the gradient of a chunk's mean loss w.r.t. the fast weights when
-nothing cached depends on them.
+complex rotation of the pairs (i, i + hd/2). static_forward processes all
+positions at once with fixed weights, so it is the static sliding-window model;
+with autograd it also gives the gradient of a chunk's mean loss w.r.t. the fast
+weights when nothing cached depends on them. mini_batch_ttt_chunked runs the
+method chunk by chunk with an explicit key/value cache for any number of
+adaptive blocks, under a selectable rule for what the cache holds.
 """
 import torch
 import torch.nn.functional as F
@@ -100,4 +102,132 @@ def mini_batch_ttt_single_adaptive_block(cfg, weights, tokens):
         if c1 - c0 == b:
             (chunk.sum() / b).backward()
             fast = [{n: (t - cfg.eta * t.grad).detach() for n, t in f.items()} for f in cur]
+    return losses, fast
+
+
+# ----------------------------------------------------------------------------- chunk-wise loop with a K/V cache
+
+def _attend(q, keys, vals, q_pos, k_pos, window):
+    """Windowed causal attention of q [n,H,hd] over keys/vals [m,H,hd] (library SDPA, boolean mask)."""
+    mask = (k_pos[None, :] <= q_pos[:, None]) & (k_pos[None, :] >= q_pos[:, None] - window + 1)
+    o = F.scaled_dot_product_attention(q.transpose(0, 1), keys.transpose(0, 1), vals.transpose(0, 1),
+                                       attn_mask=mask)
+    return o.transpose(0, 1)
+
+
+def _adaptive_layer(cfg, w, l, fast_j, x, pos, k_hist, v_hist, hist_pos):
+    """One adaptive block over rows x at positions pos; attention sees the given
+    earlier keys/values (constants) and the rows' own keys/values.
+    Returns (output, post-RoPE keys of the rows, values of the rows)."""
+    d, H = cfg.d, cfg.n_heads
+    hd = d // H
+    n = x.shape[0]
+    p = f"layers.{l}."
+    r = F.rms_norm(x, (d,), weight=w[p + "attn_norm"], eps=cfg.rms_eps)
+    q = _rope_complex((r @ w[p + "Wq"].T).view(n, H, hd), pos, cfg.rope_base)
+    k = _rope_complex((r @ w[p + "Wk"].T).view(n, H, hd), pos, cfg.rope_base)
+    v = (r @ w[p + "Wv"].T).view(n, H, hd)
+    keys = torch.cat([k_hist.detach(), k], dim=0)
+    vals = torch.cat([v_hist.detach(), v], dim=0)
+    o = _attend(q, keys, vals, pos, torch.cat([hist_pos, pos]), cfg.window_k)
+    x = x + o.reshape(n, d) @ w[p + "Wo"].T
+    r2 = F.rms_norm(x, (d,), weight=w[p + "ttt_norm"], eps=cfg.rms_eps)
+    x = x + F.gelu(r2 @ fast_j["W1t"].T, approximate="none") @ fast_j["W2t"].T
+    r3 = F.rms_norm(x, (d,), weight=w[p + "static_norm"], eps=cfg.rms_eps)
+    x = x + F.gelu(r3 @ w[p + "W1s"].T, approximate="none") @ w[p + "W2s"].T
+    return x, k, v
+
+
+def _frozen_stack(cfg, w, tok_in, pos):
+    """Embedding and every frozen block over all positions at once (they do not depend on W)."""
+    d, H = cfg.d, cfg.n_heads
+    hd = d // H
+    T = tok_in.shape[0]
+    x = w["E"][tok_in]
+    for l in range(cfg.n_layers - cfg.n_ttt):
+        p = f"layers.{l}."
+        r = F.rms_norm(x, (d,), weight=w[p + "attn_norm"], eps=cfg.rms_eps)
+        q = _rope_complex((r @ w[p + "Wq"].T).view(T, H, hd), pos, cfg.rope_base)
+        k = _rope_complex((r @ w[p + "Wk"].T).view(T, H, hd), pos, cfg.rope_base)
+        v = (r @ w[p + "Wv"].T).view(T, H, hd)
+        x = x + _attend(q, k, v, pos, pos, cfg.window_k).reshape(T, d) @ w[p + "Wo"].T
+        r2 = F.rms_norm(x, (d,), weight=w[p + "mlp_norm"], eps=cfg.rms_eps)
+        x = x + F.gelu(r2 @ w[p + "W1"].T, approximate="none") @ w[p + "W2"].T
+    return x
+
+
+def _static_adaptive_kv(cfg, w, x, pos, fast):
+    """Keys/values of every adaptive block over the rows x, all computed with the one set
+    of fast weights `fast` (a static pass of the adaptive stack). Used by the negative controls."""
+    H, hd = cfg.n_heads, cfg.d // cfg.n_heads
+    empty = torch.zeros(0, H, hd, dtype=torch.float64)
+    none = torch.zeros(0, dtype=torch.long)
+    ks, vs = [], []
+    with torch.no_grad():
+        for j in range(cfg.n_ttt):
+            l = cfg.n_layers - cfg.n_ttt + j
+            x, k, v = _adaptive_layer(cfg, w, l, fast[j], x, pos, empty, empty, none)
+            ks.append(k)
+            vs.append(v)
+    return ks, vs
+
+
+def mini_batch_ttt_chunked(cfg, weights, tokens, cache_rule="as_computed"):
+    """Mini-batch TTT by autograd, chunk by chunk, for any number of adaptive blocks.
+
+    Chunk i (positions [(i-1)b, ib)) runs the adaptive blocks with W_{i-1}; its
+    attention reads earlier positions' keys/values as constants (no gradient)
+    and its own rows' keys/values with gradient; its losses are recorded, and
+    W_i = W_{i-1} - eta * autograd gradient of the chunk's mean loss.
+
+    cache_rule decides what the earlier positions' keys/values of the adaptive
+    blocks are:
+      "as_computed"       - the values computed when their own chunk ran, i.e.
+                            with the weights in force then (W_{j-1} for chunk j),
+                            never recomputed;
+      "recompute_current" - recomputed for every chunk with the current W_{i-1};
+      "initial_weights"   - computed with the initial fast weights W_0.
+    The frozen blocks' keys/values do not depend on W under any rule.
+    Returns (losses [T], fast weights after the last full chunk).
+    """
+    w = {k: _t(v) for k, v in weights.items()}
+    tok = torch.as_tensor(tokens, dtype=torch.long)
+    T = tok.shape[0] - 1
+    H, hd = cfg.n_heads, cfg.d // cfg.n_heads
+    b, first = cfg.minibatch_b, cfg.n_layers - cfg.n_ttt
+    x0 = _frozen_stack(cfg, w, tok[:T], torch.arange(T))
+    fast = initial_fast(cfg, weights)
+    init = [{n: t.clone() for n, t in f.items()} for f in fast]
+    k_cache = [torch.zeros(0, H, hd, dtype=torch.float64) for _ in range(cfg.n_ttt)]
+    v_cache = [torch.zeros(0, H, hd, dtype=torch.float64) for _ in range(cfg.n_ttt)]
+    losses = torch.zeros(T, dtype=torch.float64)
+    for c0 in range(0, T, b):
+        c1 = min(T, c0 + b)
+        cur = [{n: t.detach().clone().requires_grad_(True) for n, t in f.items()} for f in fast]
+        lo = max(0, c0 - cfg.window_k + 1)
+        if cache_rule == "as_computed":
+            ks, vs = k_cache, v_cache
+        elif cache_rule == "recompute_current":
+            ks, vs = _static_adaptive_kv(cfg, w, x0[:c0], torch.arange(c0), [
+                {n: t.detach() for n, t in f.items()} for f in cur])
+        elif cache_rule == "initial_weights":
+            ks, vs = _static_adaptive_kv(cfg, w, x0[:c0], torch.arange(c0), init)
+        else:
+            raise ValueError(cache_rule)
+        x = x0[c0:c1]
+        pos = torch.arange(c0, c1)
+        new = []
+        for j in range(cfg.n_ttt):
+            x, k, v = _adaptive_layer(cfg, w, first + j, cur[j], x, pos, ks[j][lo:c0], vs[j][lo:c0],
+                                      torch.arange(lo, c0))
+            new.append((k.detach(), v.detach()))
+        rf = F.rms_norm(x, (cfg.d,), weight=w["final_norm"], eps=cfg.rms_eps)
+        ell = F.cross_entropy(rf @ w["E"].T, tok[c0 + 1:c1 + 1], reduction="none")
+        losses[c0:c1] = ell.detach()
+        if c1 - c0 == b:
+            (ell.sum() / b).backward()
+            fast = [{n: (t - cfg.eta * t.grad).detach() for n, t in f.items()} for f in cur]
+        for j in range(cfg.n_ttt):
+            k_cache[j] = torch.cat([k_cache[j], new[j][0]])
+            v_cache[j] = torch.cat([v_cache[j], new[j][1]])
     return losses, fast
