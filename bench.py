@@ -218,6 +218,80 @@ def run_decode(T, args, device):
             "gpu_launches": launches}
 
 
+def _time_prefill(T, h, tok, loss, steps, warmup):
+    """Device time (ms) of `steps` reset+prefill calls after `warmup` untimed ones."""
+    import torch
+    for _ in range(warmup):
+        T.ttt_reset(h)
+        T.ttt_prefill(h, tok, loss)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        T.ttt_reset(h)
+        T.ttt_prefill(h, tok, loss)
+    e1.record()
+    torch.cuda.synchronize()
+    assert torch.isfinite(loss).all().item(), "non-finite loss"
+    return e0.elapsed_time(e1) / steps
+
+
+def run_batched_prefill(T, args, device, peaks):
+    """Prefill of the ~125M model on B = 4 independent sequences of T = 32768 positions,
+    each with its own fast weights (review §7, Algorithm 1: a fresh copy of W per
+    sequence). Reported beside the metric: the only batched prefill workload."""
+    import torch
+    cfg = syn.config("m125_bf16")
+    w = syn.make_weights(cfg)
+    wd = {k: torch.from_numpy(v).to(device) for k, v in w.items()}
+    del w
+    tok = torch.from_numpy(syn.make_token_batch(cfg)).to(device)
+    loss = torch.empty((cfg.batch, cfg.T), dtype=torch.float32, device=device)
+    h = T.ttt_create(cfg, wd)
+    del wd
+    ms = _time_prefill(T, h, tok, loss, args.batched_steps, 1)
+    del h
+    torch.cuda.empty_cache()
+    fl = model_flops(cfg)
+    return {"workload": f"{cfg.name}: V{cfg.vocab} d{cfg.d} L{cfg.n_layers} (last {cfg.n_ttt} adaptive) "
+                        f"H{cfg.n_heads} k{cfg.window_k} b{cfg.minibatch_b} T{cfg.T} B{cfg.batch}",
+            "tokens_per_s": cfg.batch * cfg.T / (ms / 1e3), "ms_per_step": ms, "steps": args.batched_steps,
+            "warmup": 1, "model_tflop_per_step": fl / 1e12,
+            "frac_of_peak": fl / (ms / 1e3) / 1e12 / peaks["bf16"]}
+
+
+def run_sweep(T, cfg, args, device, peaks):
+    """Fixed 128K tokens per batch, split as 8K x 16, 16K x 8, 32K x 4, 64K x 2 and
+    128K x 1 sequences of the ~1B model (technical review Fig. 1 and §11.1 eq. (11):
+    prefill seconds per 1K tokens against context length, nearly flat for TTT-E2E).
+    Every sequence carries its own fast weights; each point is one prefill call."""
+    import torch
+    total = cfg.batch * cfg.T
+    w = syn.make_weights(cfg)
+    wd = {k: torch.from_numpy(v).to(device) for k, v in w.items()}
+    del w
+    points = []
+    for Tp in args.sweep_lengths:
+        if total % Tp:
+            continue
+        B = total // Tp
+        pcfg = cfg.replace(T=Tp, batch=B)
+        tok = torch.from_numpy(syn.make_token_batch(pcfg)).to(device)
+        loss = torch.empty((B, Tp), dtype=torch.float32, device=device)
+        h = T.ttt_create(pcfg, wd, max_segment=min(Tp, 32768))
+        ms = _time_prefill(T, h, tok, loss, args.sweep_steps, 1)
+        fl = model_flops(pcfg)
+        points.append({"T": Tp, "B": B, "ms_per_step": ms, "s_per_1k_tokens": ms / 1e3 / (total / 1e3),
+                       "tokens_per_s": total / (ms / 1e3), "model_tflop_per_step": fl / 1e12,
+                       "frac_of_peak": fl / (ms / 1e3) / 1e12 / peaks["bf16"],
+                       "device_bytes": T.ttt_device_bytes(h)})
+        del h, tok, loss
+        torch.cuda.empty_cache()
+    del wd
+    torch.cuda.empty_cache()
+    return {"tokens_per_step": total, "steps": args.sweep_steps, "warmup": 1, "points": points}
+
+
 def run_full_attention(cfg, tok_dev, args, device):
     """Comparator of the pages' speed claim (summary "Results": TTT-E2E prefill 2.7x
     faster than full attention at 128K on one H100): the same architecture with no
@@ -289,19 +363,17 @@ def run_ours(args):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
+    # timed region of `value`: no instrumentation inside it
     sampler = ClockSampler(local)
     sampler.start()
-    T.ttt_profile(h, True)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches = 0
     e0.record()
     for _ in range(args.steps):
-        launches += step() + 2 * cfg.n_ttt  # + shadow refresh kernels of ttt_reset
+        launches += step()
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
-    prof = T.ttt_profile_read(h)
-    T.ttt_profile(h, False)
     clocks = sampler.stop()
     if dist is not None:
         dist.barrier()
@@ -309,6 +381,18 @@ def run_ours(args):
     tokens = _sum_over_ranks(dist, float(cfg.batch * cfg.T * args.steps), device)
     value = tokens / (ms_max / 1e3)
     assert torch.isfinite(loss_dev).all().item(), "non-finite loss"
+
+    # per-class kernel timing in a separate pass: CUDA events around every launch of a
+    # class on the library's stream (their recording would slow the step above)
+    T.ttt_profile(h, True)
+    e0.record()
+    for _ in range(args.profile_steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    ms_prof = e0.elapsed_time(e1)
+    prof = T.ttt_profile_read(h)
+    T.ttt_profile(h, False)
 
     # end to end through the same call with pinned host buffers
     e2e_value = None
@@ -325,10 +409,10 @@ def run_ours(args):
         e2e_value = _sum_over_ranks(dist, float(cfg.batch * cfg.T * args.e2e_steps), device) / (ms_e2e / 1e3)
 
     # Mean DRAM bytes (read + write) per launch of a kernel class, from one ncu capture of
-    # the current kernels (profiles/gemm_adaptive_chunk_b1_T8192.md: the 83 GEMM launches of
-    # one adaptive step, whose shapes do not depend on T). Classes without such a capture
-    # report null.
-    traffic_per_launch = {"gemm_adaptive": 38.03e6} if cfg.name == "b1_128k_bf16" and cfg.batch == 1 else {}
+    # the current kernels (the GEMM launches of one adaptive step, whose shapes do not depend
+    # on T; the profile summary under profiles/ names the command). Classes without such a
+    # capture, or whose kernels changed since it was taken, report null.
+    traffic_per_launch = dict(args.traffic) if cfg.name == "b1_128k_bf16" and cfg.batch == 1 else {}
     peaks = measured_peaks()
     flops_step = model_flops(cfg)
     achieved_model = flops_step * args.steps / (ms / 1e3) / 1e12
@@ -341,6 +425,15 @@ def run_ours(args):
     decode = None
     if args.decode and rank == 0 and ws == 1:
         decode = run_decode(T, args, device)
+    batched = None
+    if args.batched and rank == 0 and ws == 1:
+        batched = run_batched_prefill(T, args, device, peaks)
+    sweep = None
+    if args.sweep and rank == 0 and ws == 1:
+        del h
+        torch.cuda.empty_cache()
+        h = None
+        sweep = run_sweep(T, cfg, args, device, peaks)
     comparator = None
     if args.comparator and rank == 0 and ws == 1:
         del h
@@ -367,13 +460,20 @@ def run_ours(args):
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                      "frac": ach / peak, "traffic": traffic_per_launch.get(dom),
                      "peak_source": f"{peaks['source']} bf16 sustained (kernel timed inside a long step)"},
-        "profile": {c: {"ms_per_step": v["ms"] / args.steps, "share": v["ms"] / ms,
-                        "launches_per_step": v["launches"] / args.steps,
-                        "tflops": (v["flops"] / (v["ms"] / 1e3) / 1e12) if v["ms"] else 0.0} for c, v in prof.items()},
+        "profile": {"steps": args.profile_steps, "ms_per_step": ms_prof / args.profile_steps,
+                    "note": "separate instrumented pass (CUDA events around every launch of a class)",
+                    "classes": {c: {"ms_per_step": v["ms"] / args.profile_steps, "share": v["ms"] / ms_prof,
+                                    "launches_per_step": v["launches"] / args.profile_steps,
+                                    "tflops": (v["flops"] / (v["ms"] / 1e3) / 1e12) if v["ms"] else 0.0}
+                                for c, v in prof.items()}},
         "clocks": clocks,
     }
     if decode is not None:
         line["decode"] = decode
+    if batched is not None:
+        line["batched_prefill"] = batched
+    if sweep is not None:
+        line["fixed_128k_tokens_sweep"] = sweep
     if comparator is not None:
         line["full_attention_comparator"] = comparator
     if rank == 0 and ws == 1 and args.cpu_baseline:
@@ -405,6 +505,18 @@ def main():
     ap.add_argument("--no-comparator", dest="comparator", action="store_false",
                     help="skip the full-attention comparator (same architecture, no adaptive blocks, k >= T)")
     ap.add_argument("--comparator-steps", type=int, default=2)
+    ap.add_argument("--profile-steps", type=int, default=1,
+                    help="steps of the separate instrumented pass that gives the per-class profile")
+    ap.add_argument("--no-batched", dest="batched", action="store_false",
+                    help="skip the ~125M B=4 T=32768 batched prefill line")
+    ap.add_argument("--batched-steps", type=int, default=3)
+    ap.add_argument("--no-sweep", dest="sweep", action="store_false",
+                    help="skip the fixed-128K-tokens-per-batch sweep (8K x 16 ... 128K x 1)")
+    ap.add_argument("--sweep-steps", type=int, default=2)
+    ap.add_argument("--sweep-lengths", type=lambda s: [int(x) for x in s.split(",")],
+                    default=[8192, 16384, 32768, 65536, 131072])
+    ap.add_argument("--traffic", type=lambda s: [(k, float(v)) for k, v in (x.split("=") for x in s.split(","))],
+                    default=[], help="class=bytes per launch from an ncu capture of the current kernels")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

@@ -78,6 +78,10 @@ def _load():
         "ttt_k_attention_bwd_noalloc": (ctypes.c_int, [I32, I32, I32, I32, I32, I64, I32, VP, VP, VP, I32, VP, VP,
                                                        VP, VP, I32, VP]),
         "ttt_k_status": (ctypes.c_int, [VP]),
+        "ttt_test_fail_allocation": (None, [I64]),
+        "ttt_test_allocation_count": (I64, []),
+        "ttt_test_set_device_status": (ctypes.c_int, [VP, I32]),
+        "ttt_k_test_set_status": (ctypes.c_int, [I32]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -480,3 +484,24 @@ def ttt_k_status(stream=None):
     rc = lib.ttt_k_status(_stream_ptr(stream))
     if rc != TTT_OK:
         raise TTTError(rc, "device status")
+
+
+# ----------------------------------------------------------------------------- host-side fault injection (tests)
+
+def ttt_test_fail_allocation(n: int):
+    """Make the library's n-th device allocation from now fail (include/ttt_testing.h); n < 0 cancels."""
+    lib.ttt_test_fail_allocation(int(n))
+
+
+def ttt_test_allocation_count() -> int:
+    return int(lib.ttt_test_allocation_count())
+
+
+def ttt_test_set_device_status(h: Handle, code: int):
+    h.check(lib.ttt_test_set_device_status(h.ptr, int(code)))
+
+
+def ttt_k_test_set_status(code: int):
+    rc = lib.ttt_k_test_set_status(int(code))
+    if rc != TTT_OK:
+        raise TTTError(rc, "ttt_k_test_set_status")

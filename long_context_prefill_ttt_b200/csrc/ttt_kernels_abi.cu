@@ -10,17 +10,59 @@
 #include "ttt_common.cuh"
 #include "ttt_gemm.cuh"
 #include "ttt_kernels.h"
+#include "ttt_testing.h"
 
 namespace ttt {
 
-// Device status word shared by the per-kernel entry points (allocated once per process).
-static int* status_word() {
-  static int* p = nullptr;
-  if (!p) {
-    if (cudaMalloc(&p, sizeof(int)) != cudaSuccess) { cudaGetLastError(); p = nullptr; return nullptr; }
-    cudaMemset(p, 0, sizeof(int));
+// ---------------------------------------------------------------- library-resident device words
+// Status word of the per-kernel entry points: kernels whose bounded wait runs out
+// record a code here (see ttt_common.cuh); ttt_k_status reads and clears it. It
+// lives in this library's own device image (zero at load), so no entry point
+// allocates it.
+static __device__ int g_kernel_status;
+
+// Scratch of ttt_k_attention_bwd_noalloc: the per-row sums D = rowsum(dO * O),
+// one float per (sequence, head, row). It lives in this library's own device
+// image, so every GPU that loads the library holds these 4 MiB until the process
+// exits, and no call ever allocates. The host must not pass the symbol itself to
+// a kernel (in host code it names a host-side stand-in); it passes the device
+// address that cudaGetSymbolAddress returns for the current device.
+constexpr int64_t kNoAllocDsumFloats = int64_t(1) << 20;
+static __device__ __align__(256) float g_noalloc_dsum[kNoAllocDsumFloats];
+
+// Device addresses of the two words above on the current device, looked up once
+// per device (with that device current) under one lock.
+struct ResidentPtrs {
+  int* status;
+  float* dsum;
+};
+static const ResidentPtrs* resident_ptrs() {
+  static std::mutex mu;
+  static ResidentPtrs table[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return nullptr;
   }
-  return p;
+  std::lock_guard<std::mutex> lock(mu);
+  ResidentPtrs& r = table[dev];
+  if (!r.status) {
+    void* ps = nullptr;
+    void* pd = nullptr;
+    if (cudaGetSymbolAddress(&ps, g_kernel_status) != cudaSuccess || !ps ||
+        cudaGetSymbolAddress(&pd, g_noalloc_dsum) != cudaSuccess || !pd) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    r.dsum = (float*)pd;
+    r.status = (int*)ps;
+  }
+  return &r;
+}
+
+static int* status_word() {
+  const ResidentPtrs* r = resident_ptrs();
+  return r ? r->status : nullptr;
 }
 
 static int sm_count() {
@@ -37,6 +79,7 @@ static int attn_fwd(const AttnParams& ap, int engine, cudaStream_t st) {
   const int64_t rows = (int64_t)ap.B * ap.n;
   if (sizeof(T) == 2 && engine == TTT_ENGINE_AUTO && attn_tc_ok(ap)) {
     int* err = status_word();
+    if (!err) return TTT_ERR_CUDA;
     bool ok = false;
     const cudaError_t e = attn_fwd_tc_launch(ap, st, err, &ok);
     if (e != cudaSuccess) return TTT_ERR_CUDA;
@@ -58,6 +101,7 @@ static int attn_bwd(const AttnParams& ap, int engine, cudaStream_t st) {
   bool dq_done = false, dkv_done = false;
   if (sizeof(T) == 2 && engine == TTT_ENGINE_AUTO && attn_dq_tc_ok(ap)) {
     int* err = status_word();
+    if (!err) return TTT_ERR_CUDA;
     cudaError_t e = attn_bwd_dq_tc_launch(ap, st, err, &dq_done);
     if (e == cudaSuccess && attn_dkv_tc_ok(ap)) e = attn_bwd_dkv_tc_launch(ap, st, err, &dkv_done);
     if (e != cudaSuccess) return TTT_ERR_CUDA;
@@ -89,40 +133,6 @@ static AttnParams attn_params(int B, int H, int hd, int n, int64_t q0, int windo
   return ap;
 }
 
-// ---------------------------------------------------------------- allocation-free backward
-// Scratch of ttt_k_attention_bwd_noalloc: the per-row sums D = rowsum(dO * O),
-// one float per (sequence, head, row). It lives in this library's own device
-// image, so every GPU that loads the library holds these 4 MiB until the process
-// exits, and no call ever allocates. The host must not pass the symbol itself to
-// a kernel (in host code it names a host-side stand-in); it passes the device
-// address that cudaGetSymbolAddress returns for the current device.
-constexpr int64_t kNoAllocDsumFloats = int64_t(1) << 20;
-static __device__ __align__(256) float g_noalloc_dsum[kNoAllocDsumFloats];
-
-// Device address of g_noalloc_dsum on the current device, looked up once per device.
-static float* noalloc_dsum_ptr(int* rc) {
-  static std::mutex mu;
-  static float* ptrs[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
-    cudaGetLastError();
-    *rc = TTT_ERR_CUDA;
-    return nullptr;
-  }
-  std::lock_guard<std::mutex> lock(mu);
-  if (!ptrs[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_dsum) != cudaSuccess || !p) {
-      cudaGetLastError();
-      *rc = TTT_ERR_CUDA;
-      return nullptr;
-    }
-    ptrs[dev] = (float*)p;
-  }
-  *rc = TTT_OK;
-  return ptrs[dev];
-}
-
 }  // namespace ttt
 
 using namespace ttt;
@@ -138,7 +148,7 @@ int ttt_k_gemm(int32_t elem_dtype, int32_t M, int32_t N, int32_t K, int32_t batc
   if ((epi == EPI_RESID || epi == EPI_DGELU) && !X) return TTT_ERR_INVALID_ARG;
   if ((epi == EPI_RESID || epi == EPI_SGD) && !d_f32) return TTT_ERR_INVALID_ARG;
   int* err = status_word();
-  if (!err) return TTT_ERR_OOM;
+  if (!err) return TTT_ERR_CUDA;
   GemmParams p;
   memset(&p, 0, sizeof(p));
   p.M = M; p.N = N; p.K = K; p.batch = batch;
@@ -193,9 +203,9 @@ int ttt_k_attention_bwd_noalloc(int32_t elem_dtype, int32_t B, int32_t H, int32_
     return TTT_ERR_INVALID_ARG;
   if (q0 > 0 && (!ring_k || !ring_v || C < window)) return TTT_ERR_INVALID_ARG;
   if ((int64_t)B * H * n > kNoAllocDsumFloats) return TTT_ERR_INVALID_ARG;  // B*H*n above the fixed scratch
-  int rc = TTT_OK;
-  float* dsum = noalloc_dsum_ptr(&rc);
-  if (!dsum) return rc;
+  const ResidentPtrs* res = resident_ptrs();
+  if (!res) return TTT_ERR_CUDA;
+  float* dsum = res->dsum;
   // Nothing needs clearing: the first kernel of the call writes every D it later reads.
   const size_t esz = elem_dtype == TTT_BF16 ? 2 : 4;
   AttnParams ap = attn_params(B, H, hd, n, q0, window, qkv, esz, ring_k, ring_v, C, const_cast<void*>(out),
@@ -213,10 +223,18 @@ int ttt_k_attention_bwd_noalloc(int32_t elem_dtype, int32_t B, int32_t H, int32_
 int ttt_k_status(void* stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) { cudaGetLastError(); return TTT_ERR_CUDA; }
   int* err = status_word();
-  if (!err) return TTT_ERR_OOM;
+  if (!err) return TTT_ERR_CUDA;
   int flag = 0;
   if (cudaMemcpy(&flag, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TTT_ERR_CUDA;
   if (flag) { cudaMemset(err, 0, sizeof(int)); return TTT_ERR_TIMEOUT; }
+  return TTT_OK;
+}
+
+int ttt_k_test_set_status(int32_t code) {
+  if (cudaDeviceSynchronize() != cudaSuccess) { cudaGetLastError(); return TTT_ERR_CUDA; }
+  int* err = status_word();
+  if (!err) return TTT_ERR_CUDA;
+  if (cudaMemcpy(err, &code, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return TTT_ERR_CUDA;
   return TTT_OK;
 }
 

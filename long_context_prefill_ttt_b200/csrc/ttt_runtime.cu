@@ -15,6 +15,7 @@
 // Window caches: per layer and sequence a ring of C = roundup(k + b, 128)
 // positions. Rows of the current segment/chunk are read directly; older
 // positions from the ring. K/V are appended after use and never recomputed.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -22,6 +23,8 @@
 #include <vector>
 
 #include "ttt.h"
+#include "ttt_devmem.h"
+#include "ttt_testing.h"
 #include "ttt_attention.cuh"
 #include "ttt_attention_mma.cuh"
 #include "ttt_attention_tc.cuh"
@@ -339,6 +342,26 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
 }
 
 // ============================================================== device memory
+// Injected allocation failure: the request with this index (counted from the
+// moment it was set) fails; -1 = none. Requests made so far: g_alloc_count.
+static std::atomic<int64_t> g_fail_countdown{-1};
+static std::atomic<int64_t> g_alloc_count{0};
+
+cudaError_t device_alloc(void** p, size_t bytes) {
+  *p = nullptr;
+  int64_t c = g_fail_countdown.load();
+  while (c >= 0 && !g_fail_countdown.compare_exchange_weak(c, c - 1)) {
+  }
+  if (c == 0) return cudaErrorMemoryAllocation;
+  const cudaError_t e = cudaMalloc(p, bytes);
+  if (e == cudaSuccess) g_alloc_count.fetch_add(1);
+  return e;
+}
+
+void device_free(void* p) {
+  if (p) cudaFree(p);
+}
+
 struct Arena {
   std::vector<void*> ptrs;
   int64_t bytes = 0;
@@ -347,7 +370,7 @@ struct Arena {
     if (n == 0) n = 16;
     n = (n + 255) & ~(size_t)255;
     void* p = nullptr;
-    if (cudaMalloc(&p, n) != cudaSuccess) {
+    if (device_alloc(&p, n) != cudaSuccess) {
       cudaGetLastError();
       failed = true;
       return nullptr;
@@ -358,7 +381,7 @@ struct Arena {
   }
   template <typename X> X* get(size_t count) { return (X*)alloc(count * sizeof(X)); }
   void release() {
-    for (void* p : ptrs) cudaFree(p);
+    for (void* p : ptrs) device_free(p);
     ptrs.clear();
     bytes = 0;
   }
@@ -416,6 +439,7 @@ struct ttt_handle {
   virtual int decode(int64_t n, const int32_t* forced, int32_t* out_tok, float* out_loss, int32_t kind) = 0;
   virtual int get_weights(int32_t seq, int32_t blk, float* w1, float* w2, int32_t kind) = 0;
   virtual int reset() = 0;
+  virtual int set_device_status(int32_t code) = 0;
   std::string err_msg;
   bool poisoned = false;
   int64_t n_pos = 0;
@@ -531,6 +555,14 @@ template <typename T> class Engine : public ttt_handle {
   int decode(int64_t n, const int32_t* forced, int32_t* out_tok, float* out_loss, int32_t kind) override;
   int get_weights(int32_t seq, int32_t blk, float* w1, float* w2, int32_t kind) override;
   int reset() override;
+  // Test hook: with the stream idle, write `code` into the device status word, as a
+  // kernel whose bounded wait ran out would. The next call that checks the word
+  // reports it.
+  int set_device_status(int32_t code) override {
+    TTT_CUDA(cudaStreamSynchronize(st));
+    TTT_CUDA(cudaMemcpy(dev_err, &code, sizeof(int), cudaMemcpyHostToDevice));
+    return TTT_OK;
+  }
 
  private:
   int gemm_class = PC_GEMM_FROZEN;
@@ -756,7 +788,11 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
   if ((int64_t)hs * d > max_elems) max_elems = (int64_t)hs * d;
   void* stage = nullptr;
   if (w->ptr_kind == TTT_PTR_HOST) {
-    TTT_CUDA(cudaMalloc(&stage, (size_t)max_elems * 4));
+    if (device_alloc(&stage, (size_t)max_elems * 4) != cudaSuccess) {
+      cudaGetLastError();
+      arena.release();
+      return fail(this, TTT_ERR_OOM, "device allocation failed (weight staging buffer)");
+    }
   }
   int ti = 0;
   auto upload = [&](void* dst, bool dst_f32, int64_t count, bool gain) -> int {
@@ -781,7 +817,7 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
     return TTT_OK;
   };
   int rc;
-#define UP(dst, f32, cnt, gain) if ((rc = upload((dst), (f32), (cnt), (gain))) != TTT_OK) { if (stage) cudaFree(stage); return rc; }
+#define UP(dst, f32, cnt, gain) if ((rc = upload((dst), (f32), (cnt), (gain))) != TTT_OK) { device_free(stage); return rc; }
   UP(E, false, (int64_t)V * d, false);
   UP(g_final, true, d, true);
   const int64_t dd = (int64_t)d * d;
@@ -806,7 +842,7 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
     }
   }
 #undef UP
-  if (stage) cudaFree(stage);
+  device_free(stage);
   return reset();
 }
 
@@ -1436,6 +1472,15 @@ int ttt_profile_read(const ttt_handle* h, int32_t n_classes, double* ms, int64_t
 }
 
 void ttt_destroy(ttt_handle* h) { delete h; }
+
+void ttt_test_fail_allocation(int64_t n) { g_fail_countdown.store(n < 0 ? -1 : n); }
+
+int64_t ttt_test_allocation_count(void) { return g_alloc_count.load(); }
+
+int ttt_test_set_device_status(ttt_handle* h, int32_t code) {
+  if (!h) return TTT_ERR_INVALID_ARG;
+  return h->set_device_status(code);
+}
 
 const char* ttt_last_error(const ttt_handle* h) { return h ? h->err_msg.c_str() : "null handle"; }
 

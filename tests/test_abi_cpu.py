@@ -115,3 +115,19 @@ def test_binding_checks_prefill_and_create_inputs():
     with pytest.raises(ValueError, match="layers.0.Wq"):
         T.ttt_create(cfg, w)
     assert T.weight_shapes(cfg) == [int(np.prod(s)) for _, s in syn.weight_shapes(cfg)]
+
+
+def test_every_device_allocation_goes_through_the_one_allocation_routine():
+    """The allocation-failure hook (include/ttt_testing.h) and the allocation-free entry
+    point rely on this: the library calls cudaMalloc in exactly one place."""
+    csrc = os.path.join(ROOT, "long_context_prefill_ttt_b200", "csrc")
+    sites = []
+    for f in sorted(os.listdir(csrc)):
+        for i, line in enumerate(open(os.path.join(csrc, f)), 1):
+            code = line.split("//")[0]
+            if re.search(r"\bcu(da)?Mem(Alloc|alloc)\w*\s*\(|\bcudaMalloc\w*\s*\(", code):
+                sites.append((f, i))
+    assert len(sites) == 1 and sites[0][0] == "ttt_runtime.cu", sites
+    src = open(os.path.join(csrc, "ttt_runtime.cu")).read()
+    body = src[src.index("cudaError_t device_alloc("):]
+    assert "cudaMalloc(p, bytes)" in body[:body.index("\n}\n")]

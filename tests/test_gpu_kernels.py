@@ -161,6 +161,11 @@ ATTN_CASES = [
     # K/V: ragged rows with a short window, the second tile's keys one tile further on
     # (window a multiple of 128), and no ring with a window longer than the rows
     (2, 40, 64, 520, 256, 300, 768), (1, 80, 128, 384, 1024, 512, 1536), (1, 150, 64, 300, 0, 4096, 4224),
+    # the ring has wrapped (q0 > C): the window's cached keys cross slot C-1 -> 0, with the
+    # window's first key inside a ring tile, at head dims 128 and 64, ragged rows, and the
+    # ~1B workload's geometry (k = 8192, b = 1024, C = 9216) one chunk after the first wrap
+    (1, 2, 128, 256, 3072, 1000, 1280), (2, 4, 64, 300, 5120, 1500, 1664), (1, 3, 128, 200, 2816, 768, 896),
+    (1, 2, 128, 1024, 10240, 8192, 9216),
 ]
 
 

@@ -180,6 +180,32 @@ def test_small_bf16_device_buffers_match_host_buffers(T):
     assert np.array_equal(lh, ld.cpu().numpy())
 
 
+def test_hd128_ring_wrap_and_segments_bf16_matches_oracle(T):
+    """The ~1B workload's head geometry (head dim 128) at a width the oracle runs in
+    seconds, long enough that the paths of the 128K run are all taken: the frozen
+    phase runs in 4 segments, each reading the previous segment's keys from the ring;
+    the window fills; the ring (C = 768 positions) wraps five times."""
+    cfg = syn.config("b1_128k_bf16", vocab=8192, d=512, n_layers=8, n_heads=4, n_ttt=2, mlp_hidden=2048,
+                     ttt_hidden=1024, static_hidden=1024, window_k=512, minibatch_b=256, T=4096)
+    r = P.prefill_both(T, cfg, max_segment=1024)
+    rep = {}
+    P.compare(cfg, r["w"], r["gpu_losses"], r["orc_losses"], r["gpu_w"], r["orc_w"], report=rep)
+    print("hd128 ring wrap", rep)
+    assert rep["dw"] <= 5e-2
+
+
+def test_batched_bf16_window_shorter_than_sequence_matches_oracle(T):
+    """Four sequences with their own fast weights (the per-sequence W_init + dW GEMM
+    operands) and a window shorter than the sequence: the batched path of the
+    fixed-128K-tokens sweep."""
+    cfg = syn.config("small_bf16", batch=4, T=2048)
+    r = P.prefill_both(T, cfg)
+    rep = {}
+    P.compare(cfg, r["w"], r["gpu_losses"], r["orc_losses"], r["gpu_w"], r["orc_w"], report=rep)
+    print("small_bf16 B=4", rep)
+    assert rep["dw"] <= 5e-2
+
+
 def test_m125_bf16_prefix_matches_oracle(T):
     cfg = syn.config("m125_bf16", T=2048, batch=2)
     r = P.prefill_both(T, cfg)
@@ -215,8 +241,7 @@ def test_m125_decode_bf16_greedy_matches_oracle(T):
     r = orc.decode(n, forced=gtok)
     delta = 2e-2 * np.maximum(1.0, np.abs(r["z_max"]))
     assert np.all(r["z_chosen"] >= r["z_max"] - delta)
-    assert float(np.max(np.abs(gloss - r["losses"]) / np.abs(r["losses"]))) <= 2e-2 or \
-        float(np.max(np.abs(gloss - r["losses"]))) <= 2e-2
+    assert float(np.max(np.abs(gloss - r["losses"]) / np.abs(r["losses"]))) <= 2e-2
     for s in range(cfg.batch):
         for j in range(cfg.n_ttt):
             g1, g2 = T.ttt_get_weights(h, s, j)

@@ -3,14 +3,23 @@
 ttt_k_attention_bwd_noalloc serves callers that may not allocate device memory:
 its scratch is a fixed array inside the library instead of a caller buffer. This
 test calls it through the C ABI twice in a row (the second time on new inputs,
-so the shared scratch is reused) and compares each result with
-ttt_k_attention_bwd on the same inputs. It lives in its own file, collected
-last, and passes both alone in a fresh process and after the other tests.
+so the shared scratch is reused), checks the device status after each call, and
+compares each result with ttt_k_attention_bwd on the same inputs. A second test
+makes it the very first call into the library in a fresh process, with every
+device allocation of the library set to fail. It lives in its own file,
+collected last, and passes both alone in a fresh process and after the other
+tests.
 """
+import os
+import subprocess
+import sys
+
 import pytest
 import torch
 
 pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 @pytest.fixture(scope="module")
@@ -29,7 +38,8 @@ def _inputs(dtype, seed, B, H, hd, n, C):
 
 
 @pytest.mark.parametrize("dtype,tol", [(torch.float32, 1e-5), (torch.bfloat16, 3e-2)])
-@pytest.mark.parametrize("B,H,hd,n,q0,window,C", [(2, 2, 64, 96, 128, 128, 256), (1, 2, 128, 200, 300, 200, 384)])
+@pytest.mark.parametrize("B,H,hd,n,q0,window,C", [(2, 2, 64, 96, 128, 128, 256), (1, 2, 128, 200, 300, 200, 384),
+                                                  (1, 2, 128, 256, 1024, 512, 640)])
 def test_noalloc_backward_matches_allocating_backward_twice(T, dtype, tol, B, H, hd, n, q0, window, C):
     d = H * hd
     for call, seed in enumerate((101, 202)):
@@ -40,9 +50,10 @@ def test_noalloc_backward_matches_allocating_backward_twice(T, dtype, tol, B, H,
         ref = torch.zeros((B * n, 3 * d), dtype=dtype, device="cuda")
         dsum = torch.empty((B, H, n), dtype=torch.float32, device="cuda")
         T.ttt_k_attention_bwd(qkv, out, lse, dout, ref, dsum, B, H, hd, n, q0, window, ring_k, ring_v, C)
+        T.ttt_k_status()
         got = torch.zeros_like(ref)
         T.ttt_k_attention_bwd_noalloc(qkv, out, lse, dout, got, B, H, hd, n, q0, window, ring_k, ring_v, C)
-        torch.cuda.synchronize()
+        T.ttt_k_status()  # raises unless the call's kernels finished without an expired wait
         scale = ref.float().abs().max().item()
         err = (got.float() - ref.float()).abs().max().item() / scale
         assert err <= tol, (call, err)
@@ -60,3 +71,39 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(T):
     assert rc == T.TTT_ERR_INVALID_ARG
     with pytest.raises(ValueError):
         T.ttt_k_attention_bwd_noalloc(qkv, out, lse, dout, dq, 1, 16, 64, 65537, 0, 64)
+
+
+_FIRST_CALL = r"""
+import sys, torch
+sys.path.insert(0, sys.argv[1])
+B, H, hd, n, q0, window, C = 1, 4, 128, 256, 1024, 512, 640
+d = H * hd
+g = torch.Generator().manual_seed(5)
+r = lambda *s: torch.randn(*s, generator=g).to(torch.bfloat16).cuda()
+qkv, ring_k, ring_v, dout = r(B * n, 3 * d), r(B, C, d), r(B, C, d), r(B * n, d)
+out = r(B * n, d)
+lse = torch.randn(B, H, n, generator=g).cuda() + 6.0
+got = torch.zeros(B * n, 3 * d, dtype=torch.bfloat16, device="cuda")
+torch.cuda.synchronize()
+import long_context_prefill_ttt_b200 as T
+T.ttt_test_fail_allocation(0)          # every device allocation of the library would now fail
+T.ttt_k_attention_bwd_noalloc(qkv, out, lse, dout, got, B, H, hd, n, q0, window, ring_k, ring_v, C)
+T.ttt_k_status()
+T.ttt_test_fail_allocation(-1)
+assert T.ttt_test_allocation_count() == 0, T.ttt_test_allocation_count()
+ref = torch.zeros_like(got)
+dsum = torch.empty(B, H, n, device="cuda")
+T.ttt_k_attention_bwd(qkv, out, lse, dout, ref, dsum, B, H, hd, n, q0, window, ring_k, ring_v, C)
+T.ttt_k_status()
+err = (got.float() - ref.float()).abs().max().item() / ref.float().abs().max().item()
+assert err <= 3e-2, err
+print("first-call ok", err)
+"""
+
+
+def test_noalloc_as_the_first_library_call_of_a_fresh_process(T):
+    """A caller that cannot allocate may call this entry point before anything else:
+    no earlier call has set anything up for it, and no allocation may happen."""
+    r = subprocess.run([sys.executable, "-c", _FIRST_CALL, ROOT], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "first-call ok" in r.stdout
