@@ -28,11 +28,13 @@ extern "C" {
 enum { TTT_EPI_STORE = 0, TTT_EPI_RESID = 1, TTT_EPI_GELU = 2, TTT_EPI_DGELU = 3, TTT_EPI_SGD = 4 };
 
 /* Engines: 0 = automatic: GEMMs on tcgen05 tensor cores for bf16 shapes with N % 128 == 0 and
- * K % 64 == 0; attention forward on tcgen05 for bf16 with head dim 64 or 128, q0 % 128 == 0 and
- * C % 128 == 0; attention on warp-level tensor cores (mma.sync m16n8k16) for bf16 with head dim
- * 64 or 128 and q0 % 64 == 0 (and C % 64 == 0); otherwise, and for fp32, SIMT FFMA kernels.
- * 1 = SIMT only. 2 = attention on the mma.sync kernels (tests compare engines). */
-enum { TTT_ENGINE_AUTO = 0, TTT_ENGINE_SIMT = 1, TTT_ENGINE_MMA = 2 };
+ * K % 64 == 0 (pairs of CTAs on two SMs sharing 256-row tiles when M > 128, one CTA per
+ * 128-row tile otherwise); attention forward on tcgen05 for bf16 with head dim 64 or 128,
+ * q0 % 128 == 0 and C % 128 == 0; attention on warp-level tensor cores (mma.sync m16n8k16)
+ * for bf16 with head dim 64 or 128 and q0 % 64 == 0 (and C % 64 == 0); otherwise, and for
+ * fp32, SIMT FFMA kernels. 1 = SIMT only. 2 = attention on the mma.sync kernels. 3 = GEMMs
+ * on single-CTA tcgen05 tiles only (tests compare engines). */
+enum { TTT_ENGINE_AUTO = 0, TTT_ENGINE_SIMT = 1, TTT_ENGINE_MMA = 2, TTT_ENGINE_TC1 = 3 };
 
 /* Batched GEMM D[z][m][n] = epilogue(alpha * sum_k A[z](m,k) * (B[z](n,k) + B2[z](n,k))).
  * A(m,k) = a_mn ? A[k*lda + m] : A[m*lda + k]   (batch stride sA elements)
@@ -47,6 +49,20 @@ int ttt_k_gemm(int32_t elem_dtype, int32_t M, int32_t N, int32_t K, int32_t batc
                int64_t sB2, void* D, int64_t ldd,
                int64_t sD, int32_t d_f32, const void* X, int64_t ldx, int64_t sX, void* Y, int64_t ldy, int64_t sY,
                float alpha, int32_t epi, int32_t engine, void* stream);
+
+/* LM head and softmax cross-entropy, chunked over the vocabulary (summary, loss l_t;
+ * technical review §3, eq. (3)), bf16 on tcgen05. r [M][d] (final-norm output rows),
+ * E [V][d] (tied embedding), targets [M] int32 in [0, V).
+ * One GEMM z = r E^T whose epilogue keeps, per row and 64-column vocabulary chunk,
+ * the fp32 maximum and sum of exponentials and the target's fp32 logit; then one pass
+ * per row merges the chunks into the log-sum-exp, writes loss[m] = lse - z[m][t],
+ * and, when grad_scale != 0, overwrites z with dz = (softmax(z) - onehot(t)) * grad_scale.
+ * z [M][V] bf16 receives the logits (grad_scale == 0) or dz. scratch: float buffer of
+ * 2*M*(V/64) + M elements (device). V % 128 == 0, d % 64 == 0, else
+ * TTT_ERR_UNSUPPORTED. An id outside [0, V) gives that row loss 0 and sets the device
+ * status, which the next ttt_k_status() reports as TTT_ERR_INVALID_ARG. */
+int ttt_k_lm_head_ce(int32_t M, int32_t V, int32_t d, const void* r, const void* E, const int32_t* targets,
+                     void* z, float* loss, float* scratch, float grad_scale, void* stream);
 
 /* Causal sliding-window attention forward (technical review §5: window k >= b,
  * causal inside the chunk). Rows [B][n] of qkv ([B*n][3*H*hd]: q | k | v per row,
@@ -73,9 +89,9 @@ int ttt_k_attention_bwd(int32_t elem_dtype, int32_t B, int32_t H, int32_t hd, in
  * This entry point allocates nothing. Its scratch (one float per sequence, head and
  * row) is a fixed 4 MiB array inside the library that every GPU loading the library
  * keeps until exit. Limit: B*H*n <= 1048576, else TTT_ERR_INVALID_ARG.
- * The first call on each device looks up that array's device address
- * (cudaGetSymbolAddress) with the device current; make that first call before
- * any stream capture. All calls share the one array: calls whose work overlaps on
+ * The first per-kernel call on each device (this entry point or any other of this
+ * header) looks up that array's device address (cudaGetSymbolAddress) with the
+ * device current; make that first call before any stream capture. All calls share the one array: calls whose work overlaps on
  * the GPU (other streams, other host threads) race on it and must be serialised by
  * the caller. Nothing in it needs clearing: each call writes every element it reads.
  * The pages have no counterpart of this entry point: it is an interface variant. */
@@ -84,8 +100,10 @@ int ttt_k_attention_bwd_noalloc(int32_t elem_dtype, int32_t B, int32_t H, int32_
                                 const void* out, const float* lse, const void* dout, void* dqkv, int32_t engine,
                                 void* stream);
 
-/* Synchronise `stream` and return TTT_OK, TTT_ERR_CUDA or TTT_ERR_TIMEOUT (a
- * bounded device wait expired). Clears the device status word. */
+/* Synchronise `stream` and return TTT_OK, TTT_ERR_CUDA, TTT_ERR_TIMEOUT (a
+ * bounded device wait expired) or TTT_ERR_INVALID_ARG (a token id outside the
+ * vocabulary reached ttt_k_lm_head_ce). Clears the device status word. The word is
+ * one per device, shared by all per-kernel calls on it. */
 int ttt_k_status(void* stream);
 
 #ifdef __cplusplus

@@ -26,7 +26,7 @@ TTT_ERR_TIMEOUT, TTT_ERR_STREAM, TTT_ERR_POISONED, TTT_ERR_UNSUPPORTED = -4, -5,
 TTT_FP32, TTT_BF16 = 0, 1
 TTT_PTR_HOST, TTT_PTR_DEVICE = 0, 1
 EPI_STORE, EPI_RESID, EPI_GELU, EPI_DGELU, EPI_SGD = 0, 1, 2, 3, 4
-ENGINE_AUTO, ENGINE_SIMT = 0, 1
+ENGINE_AUTO, ENGINE_SIMT, ENGINE_MMA, ENGINE_TC1 = 0, 1, 2, 3
 
 _ERRNAMES = {0: "OK", -1: "INVALID_ARG", -2: "OOM", -3: "CUDA", -4: "TIMEOUT", -5: "STREAM", -6: "POISONED",
              -7: "UNSUPPORTED"}
@@ -78,6 +78,7 @@ def _load():
         "ttt_k_attention_bwd_noalloc": (ctypes.c_int, [I32, I32, I32, I32, I32, I64, I32, VP, VP, VP, I32, VP, VP,
                                                        VP, VP, I32, VP]),
         "ttt_k_status": (ctypes.c_int, [VP]),
+        "ttt_k_lm_head_ce": (ctypes.c_int, [I32, I32, I32, VP, VP, VP, VP, VP, VP, F, VP]),
         "ttt_test_fail_allocation": (None, [I64]),
         "ttt_test_allocation_count": (I64, []),
         "ttt_test_set_device_status": (ctypes.c_int, [VP, I32]),
@@ -478,6 +479,21 @@ def ttt_k_attention_bwd_noalloc(qkv, out, lse, dout, dqkv, B, H, hd, n, q0, wind
                                          _stream_ptr(stream))
     if rc != TTT_OK:
         raise TTTError(rc, "ttt_k_attention_bwd_noalloc")
+
+
+def ttt_k_lm_head_ce(r, E, targets, z, loss, scratch, M, V, d, grad_scale=0.0, stream=None):
+    """Fused LM head + cross-entropy (include/ttt_kernels.h): z [M][V] gets the logits or dz."""
+    _check(r, "r", ("bfloat16",), M * d)
+    _check(E, "E", ("bfloat16",), V * d)
+    _check(targets, "targets", ("int32",), M)
+    _check(z, "z", ("bfloat16",), M * V)
+    _check(loss, "loss", ("float32",), M)
+    _check(scratch, "scratch", ("float32",), 2 * M * (V // 64) + M)
+    _on_device(r=r, E=E, targets=targets, z=z, loss=loss, scratch=scratch)
+    rc = lib.ttt_k_lm_head_ce(M, V, d, r.data_ptr(), E.data_ptr(), targets.data_ptr(), z.data_ptr(),
+                              loss.data_ptr(), scratch.data_ptr(), float(grad_scale), _stream_ptr(stream))
+    if rc != TTT_OK:
+        raise TTTError(rc, "ttt_k_lm_head_ce")
 
 
 def ttt_k_status(stream=None):

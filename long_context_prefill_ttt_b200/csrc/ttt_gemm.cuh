@@ -26,6 +26,9 @@ enum EpiKind : int {
   EPI_DGELU = 3,   // D = acc * gelu'(X)                   (element type, X element type)
   EPI_SGD = 4,     // D(f32) += acc, Y = D (if Y)          (alpha = -eta)
   EPI_QKV_ROPE = 5,  // D = acc (element type), then RoPE on columns [0, rope_cols) by a separate pass
+  EPI_CE = 6,      // LM head + cross-entropy statistics: D = acc (element type); per row and per
+                   // 64-column vocabulary chunk k, ce_part[row][k] = (max, sum exp(acc - max)) in
+                   // fp32; ce_zt[row] = acc at column ce_tgt[row] (fp32). tcgen05 engine only.
 };
 
 struct GemmParams {
@@ -48,6 +51,8 @@ struct GemmParams {
   const float2* rope_lo; const float2* rope_hi;
   int64_t rope_pos0; const int64_t* rope_pos_dev;
   int rope_n, rope_hd, rope_cols;
+  // EPI_CE: targets [M] (batch 1), partials [M][N / 64], target logits [M]
+  const int32_t* ce_tgt; float2* ce_part; float* ce_zt;
   // Tile order of the tensor-core engine within a batch slice: 0 = row blocks outer
   // (consecutive tiles share A rows), 1 = column blocks outer (consecutive tiles share
   // B rows, so a B larger than L2 streams from DRAM once). Set by the host.
@@ -304,6 +309,70 @@ __device__ __forceinline__ void epi_row32(const GemmParams& p, int z, int m, int
   }
 }
 
+// EPI_CE on 32 consecutive columns [n, n+32) of row m: store the logits (element
+// type), fold them into the running (max, sum-exp) of the current 64-column
+// vocabulary chunk, and keep the target's logit in fp32 when it lies here. The
+// caller writes (cm, cs) to ce_part after every second call (a chunk is complete).
+__device__ __forceinline__ void epi_ce32(const GemmParams& p, int m, int n, float* v, int tgt, float& cm,
+                                         float& cs) {
+  float mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    v[i] *= p.alpha;
+    mx = fmaxf(mx, v[i]);
+  }
+  uint4* d = (uint4*)((bf16*)p.D + (int64_t)m * p.ldd + n);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    d[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                      pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+  if (tgt >= n && tgt < n + 32) {
+    float zt = v[0];
+#pragma unroll
+    for (int i = 1; i < 32; ++i) zt = (tgt - n == i) ? v[i] : zt;
+    p.ce_zt[m] = zt;
+  }
+  const float M = fmaxf(cm, mx);
+  float add = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) add += __expf(v[i] - M);
+  cs = (cm == -INFINITY ? 0.f : cs * __expf(cm - M)) + add;
+  cm = M;
+}
+
+// Epilogue of one accumulator tile for one epilogue warp: the warp reads its TMEM
+// lane quarter (one output row per thread, row m) over its half of the tile's
+// columns [c_first*32, c_first*32 + BN/2), calls release() once those columns are
+// read (the accumulator may then be overwritten), and applies the epilogue.
+template <int BN, typename Release>
+__device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t taddr, int z, int m, int n0, int c_first,
+                                              Release release) {
+  const int tgt = (p.epi == EPI_CE && m < p.M) ? p.ce_tgt[m] : -1;
+  float cm = -INFINITY, cs = 0.f;
+#pragma unroll 1
+  for (int c = c_first; c < c_first + BN / 64; ++c) {
+    float v[32];
+    tmem_ld32(taddr + c * 32, v);
+    if (c == c_first + BN / 64 - 1) {  // this warp's columns are read: its share of the accumulator is free
+      tc_fence_before();
+      __syncwarp();
+      release();
+    }
+    if (m < p.M) {
+      if (p.epi == EPI_CE) {
+        epi_ce32(p, m, n0 + c * 32, v, tgt, cm, cs);
+        if (c & 1) {  // a 64-column vocabulary chunk is complete
+          p.ce_part[(int64_t)m * (p.N / 64) + (n0 + c * 32) / 64] = make_float2(cm, cs);
+          cm = -INFINITY;
+          cs = 0.f;
+        }
+      } else {
+        epi_row32<bf16>(p, z, m, n0 + c * 32, v);
+      }
+    }
+  }
+}
+
 // Persistent warp-specialised tcgen05 GEMM. Requirements (checked on the host):
 // N % BN == 0, K % 64 == 0, 16-byte aligned rows; M may have a tail (TMA fills
 // out-of-range rows with zeros and the epilogue skips them).
@@ -433,19 +502,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const uint32_t use = lt >> 1;
       if (!mbar_wait(&acc_full[acc], use & 1, err, DEV_TIMEOUT_ACC)) break;
       tc_fence_after();
-      const int m = m0 + row_in_tile;
       const uint32_t taddr = tmem_base + acc * BN + ((uint32_t)(quarter * 32) << 16);
-#pragma unroll 1
-      for (int c = c_first; c < c_first + BN / 64; ++c) {
-        float v[32];
-        tmem_ld32(taddr + c * 32, v);
-        if (c == c_first + BN / 64 - 1) {  // this warp's columns are read: its share of the accumulator is free
-          tc_fence_before();
-          __syncwarp();
-          if (elect_lane0()) mbar_arrive(&acc_empty[acc]);
-        }
-        if (m < p.M) epi_row32<bf16>(p, z, m, n0 + c * 32, v);
-      }
+      epilogue_tile<BN>(p, taddr, z, m0 + row_in_tile, n0, c_first, [&] {
+        if (elect_lane0()) mbar_arrive(&acc_empty[acc]);
+      });
     }
   }
   tc_fence_before();
@@ -456,9 +516,178 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
 }
 
+// ============================================================== tcgen05 engine, CTA pairs
+// Pair tile: 256 rows x BN columns, computed by a cluster of two CTAs on two SMs
+// with one cta_group::2 MMA stream issued by the even CTA. CTA r of the pair loads
+// A rows [m0 + 128 r, +128) and B rows [n0 + r BN/2, +BN/2) into its own shared
+// memory; the MMA (M = 256, N = BN) reads both halves and leaves rows [m0 + 128 r,
+// +128) of the accumulator, all BN columns, in CTA r's TMEM. Per SM and K step
+// that is 128 + BN/2 operand rows for 128 x BN outputs, against 128 + BN for the
+// single-CTA tile: 25% (BN = 128) to 33% (BN = 256) less shared-memory and L2
+// traffic per FLOP, which the small-M adaptive GEMMs are bound by.
+// Barriers: the even CTA's full[s] counts the bytes of both CTAs' loads (their TMA
+// completion is signalled there); each MMA commit arrives on empty[s] and acc_full
+// of both CTAs; both CTAs' epilogue warps arrive on the even CTA's acc_empty.
+template <int BN> struct Tc2Cfg {
+  static constexpr int BH = BN / 2;  // B rows loaded per CTA
+  static constexpr int A_BYTES = TC_BM * TC_BK * 2;
+  static constexpr int B_BYTES = BH * TC_BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (BN == 256) ? 6 : 8;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int TMEM_COLS = 2 * BN;
+};
+
+template <int BN, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmB2, const GemmParams p, int* err) {
+  using C = Tc2Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = (uint64_t*)(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = bars;                          // [STAGES] (used on the even CTA)
+  uint64_t* empty = bars + C::STAGES;             // [STAGES]
+  uint64_t* acc_full = bars + 2 * C::STAGES;      // [2]
+  uint64_t* acc_empty = bars + 2 * C::STAGES + 2; // [2]   (used on the even CTA)
+  uint32_t* tmem_slot = (uint32_t*)(bars + 2 * C::STAGES + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = (int)cluster_id_x(), npairs = (int)cluster_count_x();
+  const int m_tiles = (p.M + 2 * TC_BM - 1) / (2 * TC_BM);
+  const int n_tiles = p.N / BN;
+  const int tiles_per_batch = m_tiles * n_tiles;
+  const int num_tiles = tiles_per_batch * p.batch;
+  const int kb_one = p.K / TC_BK;
+  const int k_blocks = p.B2 ? 2 * kb_one : kb_one;
+  const int zb_scale = p.sB ? 1 : 0;
+  const int zb2_scale = p.sB2 ? 1 : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], 2 * TC_EPI_WARPS); }
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    if (p.B2) prefetch_tmap(&tmB2);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before either signals the other's
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t full0 = mapa_shared(smem_u32(full), 0);
+  const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
+  pdl_wait();
+  pdl_trigger();
+
+  if (warp == 0) {
+    if (elect_lane0()) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs) {
+        const int z = tile / tiles_per_batch;
+        const int r = tile % tiles_per_batch;
+        const int m0 = (p.m_fast ? r % m_tiles : r / n_tiles) * 2 * TC_BM + (int)rank * TC_BM;
+        const int n0 = (p.m_fast ? r / m_tiles : r % n_tiles) * BN + (int)rank * C::BH;
+        for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t round = it / C::STAGES;
+          if (!mbar_wait(&empty[s], (round & 1) ^ 1, err, DEV_TIMEOUT_EMPTY)) { ok = false; break; }
+          uint8_t* sa = smem + s * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * C::STAGE_BYTES);
+          const uint32_t bar = full0 + 8u * s;
+          const bool second = kb >= kb_one;
+          const int k0 = (second ? kb - kb_one : kb) * TC_BK;
+          const CUtensorMap* mb = second ? &tmB2 : &tmB;
+          const int zb = z * (second ? zb2_scale : zb_scale);
+          if (A_MN) {
+            tma_load_3d_pair(sa, &tmA, bar, m0, k0, z);
+            tma_load_3d_pair(sa + 8192, &tmA, bar, m0 + 64, k0, z);
+          } else {
+            tma_load_3d_pair(sa, &tmA, bar, k0, m0, z);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int j = 0; j < C::BH / 64; ++j) tma_load_3d_pair(sb + j * 8192, mb, bar, n0 + 64 * j, k0, zb);
+          } else {
+            tma_load_3d_pair(sb, mb, bar, k0, n0, zb);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (rank == 0 && elect_lane0()) {
+      constexpr uint32_t idesc = idesc_bf16_f32(2 * TC_BM, BN, A_MN, B_MN);
+      int it = 0, lt = 0;
+      bool ok = true;
+      for (int tile = pair; tile < num_tiles && ok; tile += npairs, ++lt) {
+        const int acc = lt & 1;
+        const uint32_t use = lt >> 1;
+        if (!mbar_wait(&acc_empty[acc], (use & 1) ^ 1, err, DEV_TIMEOUT_ACC)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+          const int s = it % C::STAGES;
+          const uint32_t round = it / C::STAGES;
+          if (!mbar_wait(&full[s], round & 1, err, DEV_TIMEOUT_FULL)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < TC_BK / 16; ++kk) {
+            const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+                                     : smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                     : smem_desc_sw128(sb + kk * 32, 16, 1024);
+            tc_mma_pair_f16(d_tmem, ad, bd, idesc, (kb | kk) ? 1u : 0u);
+          }
+          tc_commit_pair(&empty[s], 3);
+        }
+        if (!ok) break;
+        tc_commit_pair(&acc_full[acc], 3);
+      }
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int c_first = (warp >= 6 ? 1 : 0) * (BN / 64);
+    const int row_in_tile = quarter * 32 + (threadIdx.x & 31);
+    int lt = 0;
+    for (int tile = pair; tile < num_tiles; tile += npairs, ++lt) {
+      const int z = tile / tiles_per_batch;
+      const int r = tile % tiles_per_batch;
+      const int m0 = (p.m_fast ? r % m_tiles : r / n_tiles) * 2 * TC_BM + (int)rank * TC_BM;
+      const int n0 = (p.m_fast ? r / m_tiles : r % n_tiles) * BN;
+      const int acc = lt & 1;
+      const uint32_t use = lt >> 1;
+      if (!mbar_wait(&acc_full[acc], use & 1, err, DEV_TIMEOUT_ACC)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + acc * BN + ((uint32_t)(quarter * 32) << 16);
+      epilogue_tile<BN>(p, taddr, z, m0 + row_in_tile, n0, c_first, [&] {
+        if (elect_lane0()) mbar_arrive_cluster(acc_empty0 + 8u * acc);
+      });
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while the pair's MMAs or arrivals may still touch it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
 // ============================================================== host side
-int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t stream, int* err, int num_sms,
-                int force_simt);
+enum GemmEngine : int { GEMM_AUTO = 0, GEMM_SIMT = 1, GEMM_TC1 = 3 };
+int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t stream, int* err, int num_sms, int engine);
+// Whether gemm_launch would run p on the tcgen05 engine (EPI_CE requires it).
+bool gemm_uses_tc(const GemmParams& p, int elem_is_bf16);
 // Sets the dynamic shared-memory limits of all large-smem kernels; 0 or a cudaError_t.
 int prime_kernel_attributes();
 struct AttnParams;

@@ -10,6 +10,7 @@
 #include "ttt_common.cuh"
 #include "ttt_gemm.cuh"
 #include "ttt_kernels.h"
+#include "ttt_ce.cuh"
 #include "ttt_testing.h"
 
 namespace ttt {
@@ -160,8 +161,31 @@ int ttt_k_gemm(int32_t elem_dtype, int32_t M, int32_t N, int32_t K, int32_t batc
   p.Y = Y; p.ldy = ldy; p.sY = sY;
   p.alpha = alpha; p.epi = epi;
   const int e = gemm_launch(p, elem_dtype == TTT_BF16 ? 1 : 0, (cudaStream_t)stream, err, sm_count(),
-                            engine == TTT_ENGINE_SIMT);
+                            engine == TTT_ENGINE_SIMT ? GEMM_SIMT : engine == TTT_ENGINE_TC1 ? GEMM_TC1 : GEMM_AUTO);
   return e == 0 ? TTT_OK : TTT_ERR_CUDA;
+}
+
+int ttt_k_lm_head_ce(int32_t M, int32_t V, int32_t d, const void* r, const void* E, const int32_t* targets,
+                     void* z, float* loss, float* scratch, float grad_scale, void* stream) {
+  if (M < 1 || V < 64 || d < 1 || V % 64 || !r || !E || !targets || !z || !loss || !scratch)
+    return TTT_ERR_INVALID_ARG;
+  int* err = status_word();
+  if (!err) return TTT_ERR_CUDA;
+  if (prime_kernel_attributes() != 0) return TTT_ERR_CUDA;
+  GemmParams p;
+  memset(&p, 0, sizeof(p));
+  p.M = M; p.N = V; p.K = d; p.batch = 1;
+  p.A = r; p.lda = d; p.B = E; p.ldb = d;
+  p.D = z; p.ldd = V; p.alpha = 1.f; p.epi = EPI_CE;
+  p.ce_tgt = targets;
+  p.ce_part = (float2*)scratch;
+  p.ce_zt = scratch + (int64_t)2 * M * (V / 64);
+  if (!gemm_uses_tc(p, 1)) return TTT_ERR_UNSUPPORTED;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (gemm_launch(p, 1, st, err, sm_count(), GEMM_AUTO) != 0) return TTT_ERR_CUDA;
+  ce_finish_kernel<bf16><<<M, 256, 0, st>>>((bf16*)z, V, (const float2*)p.ce_part, p.ce_zt, targets, M, loss, M, 0,
+                                           grad_scale, err);
+  return cudaGetLastError() == cudaSuccess ? TTT_OK : TTT_ERR_CUDA;
 }
 
 int ttt_k_attention_fwd(int32_t elem_dtype, int32_t B, int32_t H, int32_t hd, int32_t n, int64_t q0,
@@ -226,7 +250,10 @@ int ttt_k_status(void* stream) {
   if (!err) return TTT_ERR_CUDA;
   int flag = 0;
   if (cudaMemcpy(&flag, err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TTT_ERR_CUDA;
-  if (flag) { cudaMemset(err, 0, sizeof(int)); return TTT_ERR_TIMEOUT; }
+  if (flag) {
+    cudaMemset(err, 0, sizeof(int));
+    return flag == DEV_BAD_TOKEN ? TTT_ERR_INVALID_ARG : TTT_ERR_TIMEOUT;
+  }
   return TTT_OK;
 }
 

@@ -4,6 +4,7 @@
 // fp32; normalised activations (GEMM operands) use the element type T.
 #pragma once
 
+#include "ttt_ce.cuh"
 #include "ttt_common.cuh"
 
 namespace ttt {
@@ -335,12 +336,6 @@ __global__ void kv_append_kernel(const T* __restrict__ src, int64_t ld, int kcol
 // grad_scale in a second vectorised pass. Row r belongs to sequence r / n at
 // chunk offset r % n; its loss goes to loss_out[(r / n) * loss_ld + loss_off + r % n]
 // (skipped when loss_out is null).
-__device__ __forceinline__ void lse_merge(float& m, float& s, float m2, float s2) {
-  const float M = fmaxf(m, m2);
-  if (M == -INFINITY) return;
-  s = s * expf(m - M) + s2 * expf(m2 - M);
-  m = M;
-}
 
 template <typename T>
 __global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ z, int V, const int32_t* __restrict__ targets,

@@ -151,6 +151,64 @@ static cudaError_t launch_tc(const GemmParams& p, cudaStream_t st, int* err, int
   return launch_pdl(gemm_tc_kernel<BN, AM, BM>, dim3(grid), dim3(TC_THREADS), C::SMEM, st, ta, tb, tb2, p, err);
 }
 
+// Pairs of CTAs that can be resident at once for one paired-GEMM variant (0 = the
+// device cannot place them; then the single-CTA kernel runs). Queried once.
+template <int BN, bool AM, bool BM> static int pair_capacity() {
+  static int cap = -1;
+  if (cap < 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = Tc2Cfg<BN>::SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc2_kernel<BN, AM, BM>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    cap = n;
+  }
+  return cap;
+}
+
+template <int BN, bool AM, bool BM>
+static cudaError_t launch_tc2(const GemmParams& p, cudaStream_t st, int* err, bool* ok) {
+  CUtensorMap ta, tb, tb2;
+  *ok = make_operand_map(&ta, p.A, p.M, p.K, p.lda, p.batch, p.sA, AM, TC_BM) &&
+        make_operand_map(&tb, p.B, p.N, p.K, p.ldb, p.batch, p.sB, BM, BN / 2);
+  if (*ok && p.B2) *ok = make_operand_map(&tb2, p.B2, p.N, p.K, p.ldb, p.batch, p.sB2, BM, BN / 2);
+  else tb2 = tb;
+  if (!*ok) return cudaSuccess;
+  const int cap = pair_capacity<BN, AM, BM>();
+  if (cap <= 0) {
+    *ok = false;
+    return cudaSuccess;
+  }
+  const int tiles = ((p.M + 2 * TC_BM - 1) / (2 * TC_BM)) * (p.N / BN) * p.batch;
+  const int pairs = tiles < cap ? tiles : cap;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(TC_THREADS);
+  cfg.dynamicSmemBytes = Tc2Cfg<BN>::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, AM, BM>, ta, tb, tb2, p, err);
+}
+
 // ============================================================== tcgen05 attention (host)
 bool attn_tc_ok(const AttnParams& p) {
   return (p.hd == 64 || p.hd == 128) && p.q0 % 128 == 0 && (p.q0 == 0 || p.C % 128 == 0) && p.d % 64 == 0 &&
@@ -230,8 +288,11 @@ cudaError_t attn_bwd_dkv_tc_launch(const AttnParams& p, cudaStream_t st, int* er
 // Dynamic shared-memory limits of every large-smem kernel, set once per process
 // before any launch (and so never inside a CUDA graph capture).
 template <int BN, bool AM, bool BM> static cudaError_t tc_attr() {
-  return cudaFuncSetAttribute(gemm_tc_kernel<BN, AM, BM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              TcCfg<BN>::SMEM);
+  const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, AM, BM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             TcCfg<BN>::SMEM);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(gemm_tc2_kernel<BN, AM, BM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Tc2Cfg<BN>::SMEM);
 }
 int prime_kernel_attributes() {
   static int done = 0;
@@ -255,18 +316,49 @@ int prime_kernel_attributes() {
   for (cudaError_t x : r)
     if (x != cudaSuccess) e = x;
   if (e != cudaSuccess) return (int)e;
+  // resident-pair counts of the paired GEMMs, queried now rather than at a first launch
+  pair_capacity<128, false, false>(); pair_capacity<256, false, false>(); pair_capacity<128, false, true>();
+  pair_capacity<256, false, true>();  pair_capacity<128, true, true>();   pair_capacity<256, true, true>();
   done = 1;
   return 0;
 }
 
-// Returns 0 on success, or a cudaError_t value.
-int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err, int num_sms, int force_simt) {
-  if (p.M <= 0 || p.N <= 0 || p.K <= 0 || p.batch <= 0) return 0;
-  // few rows per slice (decode): skinny kernel, all SMs streaming the weight rows
+// Few rows per slice (decode): skinny kernel, all SMs streaming the weight rows.
+static bool skinny_ok(const GemmParams& p, int elem_is_bf16) {
   const size_t vec = elem_is_bf16 ? 8 : 4;
-  if (!force_simt && p.M <= SK_MAXM && !p.a_mn && !p.b_mn && p.K % vec == 0 && p.lda % vec == 0 &&
-      p.ldb % vec == 0 && aligned16(p.A) && aligned16(p.B) && (!p.B2 || aligned16(p.B2)) &&
-      (p.batch == 1 || (p.sA % vec == 0 && p.sB % vec == 0 && p.sB2 % vec == 0))) {
+  return p.M <= SK_MAXM && p.epi != EPI_CE && !p.a_mn && !p.b_mn && p.K % vec == 0 && p.lda % vec == 0 &&
+         p.ldb % vec == 0 && aligned16(p.A) && aligned16(p.B) && (!p.B2 || aligned16(p.B2)) &&
+         (p.batch == 1 || (p.sA % vec == 0 && p.sB % vec == 0 && p.sB2 % vec == 0));
+}
+
+// Shapes, layouts and alignments the tcgen05 engine takes.
+static bool tc_ok(const GemmParams& p, int elem_is_bf16) {
+  bool ok = elem_is_bf16 && (p.K % TC_BK == 0) && (p.N % 128 == 0) && aligned16(p.A) && aligned16(p.B) &&
+            aligned16(p.D) && (p.lda % 8 == 0) && (p.ldb % 8 == 0) &&
+            (p.ldd % (p.d_f32 || p.epi == EPI_RESID || p.epi == EPI_SGD ? 4 : 8) == 0) &&
+            (p.batch == 1 || (p.sA % 8 == 0 && p.sB % 8 == 0 && p.sB2 % 8 == 0)) && (!p.a_mn || p.b_mn) &&
+            p.M >= 1 && (!p.B2 || aligned16(p.B2));
+  if (ok && p.X && !(aligned16(p.X) && p.ldx % (p.epi == EPI_DGELU ? 8 : 4) == 0 && (p.batch == 1 || p.sX % 8 == 0)))
+    ok = false;
+  if (ok && p.batch > 1 && p.sD % 8 != 0) ok = false;
+  if (ok && p.Y && !(aligned16(p.Y) && p.ldy % 8 == 0 && (p.batch == 1 || p.sY % 8 == 0))) ok = false;
+  if (ok && p.epi == EPI_CE && !(p.batch == 1 && !p.d_f32 && p.ce_tgt && p.ce_part && p.ce_zt)) ok = false;
+  return ok;
+}
+
+bool gemm_uses_tc(const GemmParams& p, int elem_is_bf16) {
+  if (p.M <= 0 || p.N <= 0 || p.K <= 0 || p.batch <= 0) return false;
+  return !skinny_ok(p, elem_is_bf16) && tc_ok(p, elem_is_bf16);
+}
+
+// Returns 0 on success, or a cudaError_t value. engine: GEMM_AUTO (tcgen05 CTA pairs
+// for M > 128, single-CTA tcgen05 otherwise, SIMT where tensor cores do not fit),
+// GEMM_SIMT, or GEMM_TC1 (no CTA pairs).
+int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err, int num_sms, int engine) {
+  if (p.M <= 0 || p.N <= 0 || p.K <= 0 || p.batch <= 0) return 0;
+  const bool force_simt = engine == GEMM_SIMT;
+  if (p.epi == EPI_CE && (force_simt || !gemm_uses_tc(p, elem_is_bf16))) return (int)cudaErrorInvalidValue;
+  if (!force_simt && skinny_ok(p, elem_is_bf16)) {
     GemmParams q = p;
     if (p.epi == EPI_QKV_ROPE) q.epi = EPI_STORE;
     dim3 grid((p.N + 1) / 2, p.batch);
@@ -286,16 +378,7 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
   }
   GemmParams pt = p;  // tensor-core launch: the rotation of EPI_QKV_ROPE runs as a separate pass
   if (p.epi == EPI_QKV_ROPE) pt.epi = EPI_STORE;
-  bool use_tc = elem_is_bf16 && !force_simt && (p.K % TC_BK == 0) && (p.N % 128 == 0) && aligned16(p.A) &&
-                aligned16(p.B) && aligned16(p.D) && (p.lda % 8 == 0) && (p.ldb % 8 == 0) &&
-                (p.ldd % (p.d_f32 || p.epi == EPI_RESID || p.epi == EPI_SGD ? 4 : 8) == 0) &&
-                (p.batch == 1 || (p.sA % 8 == 0 && p.sB % 8 == 0 && p.sB2 % 8 == 0)) && (!p.a_mn || p.b_mn) &&
-                p.M >= 1 && (!p.B2 || aligned16(p.B2));
-  if (use_tc && p.X && !(aligned16(p.X) && p.ldx % (p.epi == EPI_DGELU ? 8 : 4) == 0 &&
-                         (p.batch == 1 || p.sX % 8 == 0)))
-    use_tc = false;
-  if (use_tc && p.batch > 1 && p.sD % 8 != 0) use_tc = false;
-  if (use_tc && p.Y && !(aligned16(p.Y) && p.ldy % 8 == 0 && (p.batch == 1 || p.sY % 8 == 0))) use_tc = false;
+  const bool use_tc = !force_simt && tc_ok(p, elem_is_bf16);
   if (use_tc) {
     // Tile width. A 128x256 tile does twice the work of a 128x128 one in about 1.32
     // times its time (tensor pipe 68% vs 45% busy on the same frozen-block GEMMs), so
@@ -307,7 +390,30 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
     // walk the larger operand once: column blocks outer when B is the larger matrix
     pt.m_fast = p.N > p.M ? 1 : 0;
     bool ok = false;
-    cudaError_t e;
+    cudaError_t e = cudaSuccess;
+    if (engine != GEMM_TC1 && p.M > TC_BM) {
+      // CTA pairs: 256-row tiles, waves counted in resident pairs
+      const int cap = pair_capacity<128, false, false>();
+      if (cap > 0) {
+        const int m2 = (p.M + 2 * TC_BM - 1) / (2 * TC_BM);
+        auto waves2 = [&](int bn) { return std::ceil((double)m2 * (p.N / bn) * p.batch / cap); };
+        const bool w256 = (p.N % 256 == 0) && waves2(128) >= 1.32 * waves2(256);
+        if (!p.a_mn && !p.b_mn)
+          e = w256 ? launch_tc2<256, false, false>(pt, st, err, &ok) : launch_tc2<128, false, false>(pt, st, err, &ok);
+        else if (!p.a_mn && p.b_mn)
+          e = w256 ? launch_tc2<256, false, true>(pt, st, err, &ok) : launch_tc2<128, false, true>(pt, st, err, &ok);
+        else
+          e = w256 ? launch_tc2<256, true, true>(pt, st, err, &ok) : launch_tc2<128, true, true>(pt, st, err, &ok);
+        if (e != cudaSuccess) return (int)e;
+      }
+    }
+    if (ok) {
+      if (p.epi == EPI_QKV_ROPE) {
+        return (int)rope_launch<bf16>((bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd,
+                                      p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st);
+      }
+      return 0;
+    }
     if (!p.a_mn && !p.b_mn)
       e = n256 ? launch_tc<256, false, false>(pt, st, err, num_sms, &ok) : launch_tc<128, false, false>(pt, st, err, num_sms, &ok);
     else if (!p.a_mn && p.b_mn)
@@ -323,6 +429,7 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
       return 0;
     }
   }
+  if (p.epi == EPI_CE) return (int)cudaErrorInvalidValue;  // the statistics epilogue exists on tcgen05 only
   dim3 grid((p.N + 63) / 64, (p.M + 63) / 64, p.batch);
   GemmParams q = p;
   if (p.epi == EPI_QKV_ROPE) q.epi = EPI_STORE;  // rotation as a separate pass below
@@ -523,6 +630,7 @@ template <typename T> class Engine : public ttt_handle {
   std::vector<BlockAct<T>> blk;
   float* tin = nullptr; float* y = nullptr; float* rstdf = nullptr; T* rf = nullptr; T* z = nullptr;
   int32_t* tgt = nullptr;
+  float2* ce_part = nullptr; float* ce_zt = nullptr;  // fused LM-head cross-entropy statistics (bf16 path)
   float* G = nullptr; T* GT = nullptr; T* dhid = nullptr; float* dr = nullptr; T* dqkv = nullptr;
   T* dob = nullptr; float* Dsum = nullptr;
   // pending (incomplete) chunk: inputs of the first adaptive block and targets
@@ -571,7 +679,7 @@ template <typename T> class Engine : public ttt_handle {
     prof.begin(st, gemm_class, 2.0 * p.M * p.N * (double)p.K * p.batch,
                (double)p.batch * ((double)p.M * p.K * es + (double)p.N * p.K * es +
                                   (double)p.M * p.N * (p.d_f32 ? 4 : es)));
-    const int e = gemm_launch(p, is_bf16 ? 1 : 0, st, dev_err, num_sms, 0);
+    const int e = gemm_launch(p, is_bf16 ? 1 : 0, st, dev_err, num_sms, GEMM_AUTO);
     prof.end(st);
     ++launches;
     if (e != 0) {
@@ -737,6 +845,10 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
   rf = arena.get<T>((size_t)Mc * d);
   z = arena.get<T>((size_t)Mc * V);
   tgt = arena.get<int32_t>(Mc);
+  if (is_bf16 && V % 64 == 0) {
+    ce_part = arena.get<float2>((size_t)Mc * (V / 64));
+    ce_zt = arena.get<float>(Mc);
+  }
   G = arena.get<float>((size_t)Mc * d);
   GT = arena.get<T>((size_t)Mc * d);
   dhid = arena.get<T>((size_t)Mc * (ht > hs ? ht : hs));
@@ -1127,10 +1239,26 @@ int Engine<T>::ttt_step(const float* in, const int32_t* targets, int cn, int64_t
   if ((rc = ttt_forward(cn, pos, commit)) != TTT_OK) return rc;
   rmsnorm_fwd_launch<T>((const float*)y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf, st);
   TTT_LAUNCHED();
-  if ((rc = gemm(gp(rows, V, d, rf, d, false, E, d, false, z, V, false, EPI_STORE))) != TTT_OK) return rc;
-  // mean over the b positions of the chunk (summary: mini-batch GD with 1/b)
-  ce_kernel<T><<<rows, 256, 0, st>>>(z, V, tgt, cn, loss_out, loss_ld, loss_off, grad ? 1.0f / bsz : 0.f,
-                                     dev_err);
+  // LM head + cross-entropy, chunked over the vocabulary: the tcgen05 GEMM epilogue
+  // keeps an fp32 (max, sum-exp) per row and 64-column chunk and the target's fp32
+  // logit; ce_finish merges the chunks, records the loss and writes dz in place of
+  // the logits. The gradient is the mean over the b positions of the chunk
+  // (summary: mini-batch GD with 1/b).
+  GemmParams ph = gp(rows, V, d, rf, d, false, E, d, false, z, V, false, EPI_STORE);
+  const float gscale = grad ? 1.0f / bsz : 0.f;
+  bool fused = false;
+  if (ce_part) {
+    GemmParams pc = ph;
+    pc.epi = EPI_CE; pc.ce_tgt = tgt; pc.ce_part = ce_part; pc.ce_zt = ce_zt;
+    if (gemm_uses_tc(pc, 1)) { ph = pc; fused = true; }
+  }
+  if ((rc = gemm(ph)) != TTT_OK) return rc;
+  if (fused) {
+    launch_pdl(ce_finish_kernel<T>, dim3(rows), dim3(256), 0, st, z, V, (const float2*)ce_part,
+               (const float*)ce_zt, (const int32_t*)tgt, cn, loss_out, loss_ld, loss_off, gscale, dev_err);
+  } else {
+    ce_kernel<T><<<rows, 256, 0, st>>>(z, V, tgt, cn, loss_out, loss_ld, loss_off, gscale, dev_err);
+  }
   TTT_LAUNCHED();
   if (grad) {
     if ((rc = ttt_backward(cn)) != TTT_OK) return rc;

@@ -30,12 +30,15 @@ def _store(x_log, mn):
     return x_log.transpose(1, 2).contiguous() if mn else x_log.contiguous()
 
 
-SHAPES = [(256, 256, 128, 1), (200, 384, 192, 2), (1024, 512, 64, 1), (128, 2048, 256, 1), (384, 128, 1024, 3)]
+# engine 0 runs M > 128 on CTA pairs (256-row tiles, ragged M tails and batches included),
+# engine 3 on single-CTA tiles, engine 1 on SIMT
+SHAPES = [(256, 256, 128, 1), (200, 384, 192, 2), (1024, 512, 64, 1), (128, 2048, 256, 1), (384, 128, 1024, 3),
+          (1024, 2048, 512, 1), (640, 4096, 128, 1), (100, 256, 64, 2)]
 
 
 @pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1), (1, 1)])
 @pytest.mark.parametrize("M,N,K,batch", SHAPES)
-@pytest.mark.parametrize("engine", [0, 1])
+@pytest.mark.parametrize("engine", [0, 1, 3])
 def test_gemm_store_f32(T, a_mn, b_mn, M, N, K, batch, engine):
     A = _rand((batch, M, K), torch.bfloat16, 1)
     B = _rand((batch, N, K), torch.bfloat16, 2)
@@ -49,7 +52,7 @@ def test_gemm_store_f32(T, a_mn, b_mn, M, N, K, batch, engine):
 
 
 @pytest.mark.parametrize("a_mn,b_mn", [(0, 0), (0, 1)])
-@pytest.mark.parametrize("engine", [0, 1])
+@pytest.mark.parametrize("engine", [0, 1, 3])
 def test_gemm_shared_plus_per_batch_operand(T, a_mn, b_mn, engine):
     """acc = A (B_shared + B2[z]): a small per-batch B2 must survive next to a large shared B."""
     M, N, K, batch = 200, 256, 192, 3
@@ -85,7 +88,7 @@ def test_gemm_store_bf16_and_fp32_simt(T, M, N, K):
     assert ((D32.double() - ref32).abs().max() / ref32.abs().max()).item() < 1e-6
 
 
-@pytest.mark.parametrize("engine", [0, 1])
+@pytest.mark.parametrize("engine", [0, 1, 3])
 def test_gemm_epilogues(T, engine):
     M, N, K = 256, 384, 128
     A = _rand((1, M, K), torch.bfloat16, 5, 0.5)
@@ -131,14 +134,11 @@ def _attn_reference(qkv, ring_k, ring_v, B, H, hd, n, q0, window, C):
     vc = qkv[..., 2 * d:].double().view(B, n, H, hd)
     lo = max(0, q0 - window + 1)
     pos = torch.arange(lo, q0 + n)
-    ks, vs = [], []
-    for p in pos.tolist():
-        if p >= q0:
-            ks.append(kc[:, p - q0]); vs.append(vc[:, p - q0])
-        else:
-            ks.append(ring_k.double().view(B, C, H, hd)[:, p % C]); vs.append(ring_v.double().view(B, C, H, hd)[:, p % C])
-    K = torch.stack(ks, 1)
-    V = torch.stack(vs, 1)
+    rk = ring_k.double().view(B, C, H, hd)
+    rv = ring_v.double().view(B, C, H, hd)
+    cached = torch.arange(lo, q0)
+    K = torch.cat([rk[:, (cached % C).cuda()], kc], 1)  # position p < q0 sits in ring slot p % C
+    V = torch.cat([rv[:, (cached % C).cuda()], vc], 1)
     qp = torch.arange(q0, q0 + n)[:, None]
     mask = (pos[None, :] <= qp) & (pos[None, :] >= qp - window + 1)
     return q, kc, vc, K, V, mask.cuda(), lo
@@ -230,3 +230,39 @@ def test_skinny_gemm_rows_per_sequence(T, dtype, M, N, K, batch):
     assert torch.allclose(U.double(), ref, rtol=2 * tol, atol=2 * tol * ref.abs().max().item())
     assert torch.allclose(G.double(), torch.nn.functional.gelu(ref, approximate="none"), rtol=2 * tol,
                           atol=2 * tol * ref.abs().max().item())
+
+
+@pytest.mark.parametrize("M,V,d", [(1024, 32000, 2048), (200, 8192, 512), (77, 256, 128)])
+def test_fused_lm_head_cross_entropy(T, M, V, d):
+    """LM head + softmax cross-entropy chunked over the vocabulary, against float64:
+    loss = logsumexp(z) - z[target] from the fp32 accumulators, dz = (softmax - onehot) * s."""
+    r = _rand((M, d), torch.bfloat16, 41)
+    E = _rand((V, d), torch.bfloat16, 42, 0.5)
+    g = torch.Generator().manual_seed(43)
+    tgt = torch.randint(0, V, (M,), generator=g, dtype=torch.int32)
+    tgt[0], tgt[-1] = 0, V - 1  # first and last vocabulary chunks
+    tgt = tgt.cuda()
+    zref = r.double() @ E.double().t()
+    lref = torch.logsumexp(zref, 1) - zref[torch.arange(M), tgt.long()]
+    z = torch.empty((M, V), dtype=torch.bfloat16, device="cuda")
+    loss = torch.empty(M, dtype=torch.float32, device="cuda")
+    scratch = torch.empty(2 * M * (V // 64) + M, dtype=torch.float32, device="cuda")
+    T.ttt_k_lm_head_ce(r, E, tgt, z, loss, scratch, M, V, d)
+    T.ttt_k_status()
+    assert (loss.double() - lref).abs().max().item() <= 1e-4 * lref.abs().max().item() + 1e-4
+    assert (z.double() - zref).abs().max().item() <= 1e-2 * zref.abs().max().item()
+    s = 1.0 / 256
+    T.ttt_k_lm_head_ce(r, E, tgt, z, loss, scratch, M, V, d, grad_scale=s)
+    T.ttt_k_status()
+    pref = torch.softmax(zref, 1)
+    pref[torch.arange(M), tgt.long()] -= 1.0
+    dref = pref * s
+    assert (z.double() - dref).abs().max().item() <= 2e-2 * dref.abs().max().item()
+    assert (z.double().sum(1)).abs().max().item() <= 1e-2 * s  # softmax rows sum to one
+    # an id outside the vocabulary is reported, not read
+    bad = tgt.clone()
+    bad[3] = V + 5
+    T.ttt_k_lm_head_ce(r, E, bad, z, loss, scratch, M, V, d)
+    with pytest.raises(T.TTTError) as e:
+        T.ttt_k_status()
+    assert e.value.code == T.TTT_ERR_INVALID_ARG
