@@ -384,15 +384,17 @@ def run_ours(args):
 
     # per-class kernel timing in a separate pass: CUDA events around every launch of a
     # class on the library's stream (their recording would slow the step above)
-    T.ttt_profile(h, True)
-    e0.record()
-    for _ in range(args.profile_steps):
-        step()
-    e1.record()
-    torch.cuda.synchronize()
-    ms_prof = e0.elapsed_time(e1)
-    prof = T.ttt_profile_read(h)
-    T.ttt_profile(h, False)
+    prof, ms_prof = {}, 0.0
+    if args.profile_steps > 0:
+        T.ttt_profile(h, True)
+        e0.record()
+        for _ in range(args.profile_steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+        ms_prof = e0.elapsed_time(e1)
+        prof = T.ttt_profile_read(h)
+        T.ttt_profile(h, False)
 
     # end to end through the same call with pinned host buffers
     e2e_value = None
@@ -417,8 +419,8 @@ def run_ours(args):
     flops_step = model_flops(cfg)
     achieved_model = flops_step * args.steps / (ms / 1e3) / 1e12
     # dominant kernel class by device time
-    dom = max(prof, key=lambda c: prof[c]["ms"])
-    dp = prof[dom]
+    dom = max(prof, key=lambda c: prof[c]["ms"]) if prof else None
+    dp = prof[dom] if prof else {"flops": 0.0, "ms": 0.0}
     ach = dp["flops"] / (dp["ms"] / 1e3) / 1e12 if dp["ms"] > 0 else 0.0
     peak = peaks["bf16_sustained"]
     dev_bytes = T.ttt_device_bytes(h)
@@ -460,7 +462,7 @@ def run_ours(args):
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                      "frac": ach / peak, "traffic": traffic_per_launch.get(dom),
                      "peak_source": f"{peaks['source']} bf16 sustained (kernel timed inside a long step)"},
-        "profile": {"steps": args.profile_steps, "ms_per_step": ms_prof / args.profile_steps,
+        "profile": {"steps": args.profile_steps, "ms_per_step": ms_prof / max(1, args.profile_steps),
                     "note": "separate instrumented pass (CUDA events around every launch of a class)",
                     "classes": {c: {"ms_per_step": v["ms"] / args.profile_steps, "share": v["ms"] / ms_prof,
                                     "launches_per_step": v["launches"] / args.profile_steps,
