@@ -123,7 +123,9 @@ int ttt_decode(ttt_handle* h, int64_t n, const int32_t* forced, int32_t* out_tok
                int32_t ptr_kind);
 
 /* Copy the fp32 fast weights of sequence seq, adaptive block j (0 = first TTT block):
- * w1 [h_t][d] and w2 [d][h_t] (either may be NULL). */
+ * w1 [h_t][d] and w2 [d][h_t] (either may be NULL). These are the adapted W that
+ * Algorithm 1 of the technical review (§7) returns beside the attention state: W_init
+ * after every completed chunk's update so far. ptr_kind: host or device buffers. */
 int ttt_get_weights(ttt_handle* h, int32_t seq, int32_t ttt_block, float* w1, float* w2, int32_t ptr_kind);
 
 /* Fast weights <- W_init, window caches and pending state cleared (review §7,
@@ -142,7 +144,9 @@ int64_t ttt_last_launch_count(const ttt_handle* h);
 /* Kernel-class timing. When enabled, CUDA events are recorded on the handle's
  * stream around every launch of these classes, and the algorithmic work of each
  * launch is counted: 0 frozen-phase GEMMs, 1 adaptive-phase GEMMs, 2 attention
- * forward, 3 attention backward. FLOPs: 2*M*N*K per GEMM; attention 4*hd*H per
+ * forward, 3 attention backward, 4 the adaptive weight-gradient + SGD GEMMs when they
+ * run on the handle's side stream beside the backward (events on that stream; their
+ * time overlaps the other classes'). FLOPs: 2*M*N*K per GEMM; attention 4*hd*H per
  * query-key pair of the window forward (review eq. (1) counts the pairs), and
  * 2*hd*H*(2 window pairs + 2 current-chunk pairs) backward (no recompute counted). Bytes: operands read
  * once plus the output written once. ttt_profile(h, 1) clears the counters.

@@ -236,8 +236,10 @@ def test_skinny_gemm_rows_per_sequence(T, dtype, M, N, K, batch):
 def test_fused_lm_head_cross_entropy(T, M, V, d):
     """LM head + softmax cross-entropy chunked over the vocabulary, against float64:
     loss = logsumexp(z) - z[target] from the fp32 accumulators, dz = (softmax - onehot) * s."""
+    # the model's scales: normalised rows, embedding ~ N(0, 0.02) (logits of a few units;
+    # dz is formed from bf16 logits, whose rounding grows with their magnitude)
     r = _rand((M, d), torch.bfloat16, 41)
-    E = _rand((V, d), torch.bfloat16, 42, 0.5)
+    E = _rand((V, d), torch.bfloat16, 42, 0.02)
     g = torch.Generator().manual_seed(43)
     tgt = torch.randint(0, V, (M,), generator=g, dtype=torch.int32)
     tgt[0], tgt[-1] = 0, V - 1  # first and last vocabulary chunks
