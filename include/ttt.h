@@ -144,9 +144,7 @@ int64_t ttt_last_launch_count(const ttt_handle* h);
 /* Kernel-class timing. When enabled, CUDA events are recorded on the handle's
  * stream around every launch of these classes, and the algorithmic work of each
  * launch is counted: 0 frozen-phase GEMMs, 1 adaptive-phase GEMMs, 2 attention
- * forward, 3 attention backward, 4 the adaptive weight-gradient + SGD GEMMs when they
- * run on the handle's side stream beside the backward (events on that stream; their
- * time overlaps the other classes'). FLOPs: 2*M*N*K per GEMM; attention 4*hd*H per
+ * forward, 3 attention backward. FLOPs: 2*M*N*K per GEMM; attention 4*hd*H per
  * query-key pair of the window forward (review eq. (1) counts the pairs), and
  * 2*hd*H*(2 window pairs + 2 current-chunk pairs) backward (no recompute counted). Bytes: operands read
  * once plus the output written once. ttt_profile(h, 1) clears the counters.

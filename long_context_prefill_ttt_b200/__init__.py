@@ -357,7 +357,7 @@ def ttt_last_launch_count(h: Handle) -> int:
     return int(lib.ttt_last_launch_count(h.ptr))
 
 
-PROFILE_CLASSES = ("gemm_frozen", "gemm_adaptive", "attention_fwd", "attention_bwd", "gemm_wgrad_side")
+PROFILE_CLASSES = ("gemm_frozen", "gemm_adaptive", "attention_fwd", "attention_bwd")
 
 
 def ttt_profile(h: Handle, enable: bool = True):

@@ -9,18 +9,14 @@
 //   warp 1     MMA issue (one thread): S_j = Q K_j^T into one of two TMEM S
 //              buffers, then O += P_{j-1} V_{j-1} (P from shared memory, V as an
 //              MN-major operand) into the TMEM O accumulator;
-//   warps 2-9  softmax, two warps per TMEM lane quarter (one query row per
-//              thread), each on 64 of the tile's 128 key columns and half of the
-//              O columns: read S_j, mask on diagonal / window-edge tiles, exchange
-//              the partial row maximum with the partner warp (named barrier per
-//              quarter), online softmax in the log2 domain, write P_j (bf16) to
-//              shared memory in the 128-byte-swizzled layout the MMA reads. The
-//              running maximum is raised only when a row's maximum grows by more
-//              than 8 (a factor 256): then O is rescaled in TMEM after the previous
-//              P·V has completed. Exponents stay below 2^8, so bf16 P and fp32 sums
-//              stay exact enough, and O and l always share the same reference
-//              maximum. Eight warps give each scheduler two independent softmax
-//              warps, so the exponentials of one hide the latencies of the other.
+//   warps 2-5  softmax, one thread per query row (TMEM lane): read S_j, mask on
+//              diagonal / window-edge tiles, online softmax in the log2 domain,
+//              write P_j (bf16) to shared memory in the 128-byte-swizzled layout
+//              the MMA reads. The running maximum is raised only when a row's
+//              maximum grows by more than 8 (a factor 256): then the thread's O
+//              row is rescaled in TMEM after the previous P·V has completed.
+//              Exponents stay below 2^8, so bf16 P and fp32 sums stay exact
+//              enough, and O and l always share the same reference maximum.
 // TMEM: S0 columns [0,128), S1 [128,256), O [256, 256+HD); 512 allocated.
 // Every mbarrier wait is time-bounded and records an error instead of hanging.
 #pragma once
@@ -41,18 +37,9 @@ template <int HD> struct AttnTcCfg {
   static constexpr int OFF_V0 = OFF_K0 + KST * KVB;
   static constexpr int OFF_P0 = OFF_V0 + VST * KVB;
   static constexpr int OFF_BAR = OFF_P0 + 2 * PB;
-  // exchange between the two softmax warps of a TMEM lane quarter: per key-tile parity,
-  // half and row, the partial row maximum (bf16, rounded up); after the loop, reused
-  // for the partial row sums (fp32, [half][row])
-  static constexpr int OFF_X = OFF_BAR + 256;
-  static constexpr int SMEM = OFF_X + 2 * 2 * BM * 2 + 1024;
+  static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr uint32_t S_COL = 0, O_COL = 256;
 };
-static_assert(AttnTcCfg<128>::SMEM <= 232448, "attention forward exceeds the shared memory of one CTA");
-
-__device__ __forceinline__ void named_bar_sync(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
 
 __device__ __forceinline__ bool warp_any(bool v) { return __any_sync(0xffffffffu, v); }
 __device__ __forceinline__ float ex2_tc(float x) {
@@ -62,7 +49,7 @@ __device__ __forceinline__ float ex2_tc(float x) {
 }
 
 template <int HD>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(192, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_rk,
                        const __grid_constant__ CUtensorMap tm_rv, const AttnParams p, int* err) {
   using Cf = AttnTcCfg<HD>;
@@ -99,8 +86,8 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);  mbar_init(&s_free[s], 8);
-      mbar_init(&p_full[s], 8);  mbar_init(&pv_done[s], 1);
+      mbar_init(&s_full[s], 1);  mbar_init(&s_free[s], 4);
+      mbar_init(&p_full[s], 4);  mbar_init(&pv_done[s], 1);
     }
     mbar_init(o_done, 1);
     fence_mbar_init();
@@ -202,64 +189,50 @@ __global__ void __launch_bounds__(320, 1)
       if (ok) tc_commit(o_done);
     }
   } else {
-    // softmax warps 2..9: TMEM lane quarter = warp % 4, one query row per thread;
-    // warps 2-5 take key columns [0, 64) of each tile and O columns [0, HD/2),
-    // warps 6-9 the other halves
+    // softmax warps: TMEM lane quarter = warp % 4, one query row per thread
     const int quarter = warp & 3;
-    const int half = warp >= 6 ? 1 : 0;
     const int lane = threadIdx.x & 31;
     const int r = quarter * 32 + lane;
     const int64_t P = P0 + r;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const float sc = p.scale * 1.4426950408889634f;
-    bf16* xmax = (bf16*)(sm + Cf::OFF_X);  // [parity][half][row]
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
       const int s = j & 1;
-      const int64_t j0 = jt0 + (int64_t)j * Cf::BN + half * 64;  // first key of this warp's columns
-      // after a timed-out wait the loop still runs to its end (without waiting or
-      // computing) so that both warps of the quarter meet at every named barrier
-      if (ok) ok = mbar_wait(&s_full[s], (j >> 1) & 1, err, DEV_TIMEOUT_ACC);
-      float v[64];
-      if (ok) {
-        tc_fence_after();
+      const int64_t j0 = jt0 + (int64_t)j * Cf::BN;
+      if (!mbar_wait(&s_full[s], (j >> 1) & 1, err, DEV_TIMEOUT_ACC)) { ok = false; break; }
+      tc_fence_after();
+      float v[Cf::BN];
+      {
         uint32_t* vr = reinterpret_cast<uint32_t*>(v);
-        tmem_ld32_nowait(tmem + lane_base + Cf::S_COL + s * Cf::BN + half * 64, vr);
-        tmem_ld32_nowait(tmem + lane_base + Cf::S_COL + s * Cf::BN + half * 64 + 32, vr + 32);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[s]);
-      } else {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) v[c] = -INFINITY;
+        for (int c = 0; c < Cf::BN / 32; ++c)
+          tmem_ld32_nowait(tmem + lane_base + Cf::S_COL + s * Cf::BN + c * 32, vr + c * 32);
+        tmem_ld_wait();
       }
-      const bool need_mask = (j0 + 63 > P0) || (j0 < Plast - p.window + 1);
-      if (need_mask) {  // diagonal / window-edge columns: branch-free per-element mask
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[s]);
+      const bool need_mask = (j0 + Cf::BN - 1 > P0) || (j0 < Plast - p.window + 1);
+      if (need_mask) {  // diagonal / window-edge tile: branch-free per-element mask
         const int64_t lo_key = P - p.window + 1;
         const uint32_t span = (uint32_t)(P - lo_key);
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < Cf::BN; ++c) {
           const uint32_t off = (uint32_t)(j0 + c - lo_key);
           v[c] = off <= span ? v[c] : -INFINITY;
         }
       }
-      // partial row maximum of the raw scores, eight independent chains
+      // row maximum of the raw scores, eight independent chains
       float mx8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mx8[e] = v[e];
 #pragma unroll
-      for (int c = 8; c < 64; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], v[c]);
-      float mp = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+      for (int c = 8; c < Cf::BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], v[c]);
+      float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                        fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      // both warps of the quarter take the maximum of the two bf16-rounded-up
-      // partials (scaled log2 domain, sc > 0 keeps the order): identical in both
-      const bf16 own = __float2bfloat16_ru(mp * sc);
-      xmax[(s * 2 + half) * Cf::BM + r] = own;
-      named_bar_sync(1 + quarter, 64);
-      const float mt = fmaxf(__bfloat162float(own), __bfloat162float(xmax[(s * 2 + (half ^ 1)) * Cf::BM + r]));
-      if (!ok) continue;
+      mt *= sc;  // scores are compared in the scaled log2 domain (sc > 0 keeps the order)
       // lazily raised reference maximum
       const bool first = m_used == -INFINITY;
       const bool raise = mt > m_used + 8.f;
@@ -270,10 +243,10 @@ __global__ void __launch_bounds__(320, 1)
       }
       if (j >= 1 && warp_any(raise && !first)) {
         // O holds P_0..P_{j-1} V: wait for the last of them, then rescale this warp's rows
-        if (!mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, err, DEV_TIMEOUT_ACC)) { ok = false; continue; }
+        if (!mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, err, DEV_TIMEOUT_ACC)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
-        for (int c = half * (HD / 64); c < (half + 1) * (HD / 64); ++c) {
+        for (int c = 0; c < HD / 32; ++c) {
           float o[32];
           tmem_ld32(tmem + lane_base + Cf::O_COL + c * 32, o);
 #pragma unroll
@@ -283,21 +256,24 @@ __global__ void __launch_bounds__(320, 1)
       }
       l *= factor;
       // the P buffer s was last read by P_{j-2} V_{j-2}
-      if (j >= 2 && !mbar_wait(&pv_done[s], ((j - 2) >> 1) & 1, err, DEV_TIMEOUT_ACC)) { ok = false; continue; }
+      if (j >= 2 && !mbar_wait(&pv_done[s], ((j - 2) >> 1) & 1, err, DEV_TIMEOUT_ACC)) { ok = false; break; }
       const float nbase = m_used == -INFINITY ? 0.f : -m_used;
-      uint8_t* prow = sm + Cf::OFF_P0 + s * Cf::PB + half * (Cf::BM * 128) + r * 128;
+      uint8_t* prow = sm + Cf::OFF_P0 + s * Cf::PB + r * 128;
       float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc) {
-        float e8[8];
+      for (int kb = 0; kb < Cf::BN / 64; ++kb) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          e8[e] = ex2_tc(fmaf(v[cc * 8 + e], sc, nbase));  // exp2(s*sc - m): masked -inf -> 0
-          ls8[e] += e8[e];
+        for (int cc = 0; cc < 8; ++cc) {
+          float e8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            e8[e] = ex2_tc(fmaf(v[kb * 64 + cc * 8 + e], sc, nbase));  // exp2(s*sc - m): masked -inf -> 0
+            ls8[e] += e8[e];
+          }
+          const uint4 pk = make_uint4(pack_bf16x2(e8[0], e8[1]), pack_bf16x2(e8[2], e8[3]),
+                                      pack_bf16x2(e8[4], e8[5]), pack_bf16x2(e8[6], e8[7]));
+          *(uint4*)(prow + kb * (Cf::BM * 128) + ((cc ^ (r & 7)) << 4)) = pk;
         }
-        const uint4 pk = make_uint4(pack_bf16x2(e8[0], e8[1]), pack_bf16x2(e8[2], e8[3]),
-                                    pack_bf16x2(e8[4], e8[5]), pack_bf16x2(e8[6], e8[7]));
-        *(uint4*)(prow + ((cc ^ (r & 7)) << 4)) = pk;
       }
       l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
       fence_proxy_async();  // P (generic-proxy stores) visible to the tensor core
@@ -305,19 +281,12 @@ __global__ void __launch_bounds__(320, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[s]);
     }
-    // row sum = both warps' partial sums (the exchange buffer is free once both have
-    // passed the loop: its last reads precede the barrier below)
-    float* xsum = (float*)(sm + Cf::OFF_X);  // [half][row]
-    named_bar_sync(1 + quarter, 64);
-    xsum[half * Cf::BM + r] = l;
-    named_bar_sync(1 + quarter, 64);
-    const float lt = l + xsum[(half ^ 1) * Cf::BM + r];
     if (ok && mbar_wait(o_done, 0, err, DEV_TIMEOUT_ACC)) {
       tc_fence_after();
-      const float inv = 1.f / lt;
+      const float inv = 1.f / l;
       bf16* O = (bf16*)p.O + ((int64_t)b * p.n + i0 + r) * p.ldo + h * HD;
 #pragma unroll 1
-      for (int c = half * (HD / 64); c < (half + 1) * (HD / 64); ++c) {
+      for (int c = 0; c < HD / 32; ++c) {
         float o[32];
         tmem_ld32(tmem + lane_base + Cf::O_COL + c * 32, o);
         if (r < nq) {
@@ -329,8 +298,7 @@ __global__ void __launch_bounds__(320, 1)
                                 pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
         }
       }
-      if (half == 0 && r < nq && p.lse)
-        p.lse[((int64_t)b * p.H + h) * p.n + i0 + r] = (m_used + __log2f(lt)) * 0.6931471805599453f;
+      if (r < nq && p.lse) p.lse[((int64_t)b * p.H + h) * p.n + i0 + r] = (m_used + __log2f(l)) * 0.6931471805599453f;
     }
   }
   tc_fence_before();
@@ -344,8 +312,7 @@ __global__ void __launch_bounds__(320, 1)
 // ---------------------------------------------------------------- backward dQ on tcgen05
 // One CTA = 128 query rows of one (sequence, head), key tiles of 64 positions over
 // each row's whole window (ring and current rows). Per tile j: S = Q K^T and
-// dP = dO V^T into one of two TMEM buffers (MMA warp); eight warps, two per TMEM
-// lane quarter each taking 32 of the tile's 64 columns, form
+// dP = dO V^T into one of two TMEM buffers (MMA warp); four warps form
 // dS = P (dP - D) with P = exp(S*scale - lse) from the forward's log-sum-exp and
 // write dS (bf16) to one of two shared-memory buffers; the MMA warp accumulates
 // dQ += dS K in TMEM (the K tile read again as an MN-major operand). With S/dP and
@@ -370,7 +337,7 @@ template <int HD> struct AttnDqCfg {
 };
 
 template <int HD>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(192, 1)
     attn_bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
                           const __grid_constant__ CUtensorMap tm_rk, const __grid_constant__ CUtensorMap tm_rv,
                           const __grid_constant__ CUtensorMap tm_do, const AttnParams p, int* err) {
@@ -408,8 +375,8 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&sp_full[s], 1); mbar_init(&sp_free[s], 8);
-      mbar_init(&ds_full[s], 8); mbar_init(&ds_free[s], 1);
+      mbar_init(&sp_full[s], 1); mbar_init(&sp_free[s], 4);
+      mbar_init(&ds_full[s], 4); mbar_init(&ds_free[s], 1);
     }
     mbar_init(dq_done, 1);
     fence_mbar_init();
@@ -512,10 +479,7 @@ __global__ void __launch_bounds__(320, 1)
       if (ok) tc_commit(dq_done);
     }
   } else {
-    // warps 2..9: TMEM lane quarter = warp % 4; warps 2-5 take columns [0, 32) of each
-    // key tile and dQ columns [0, HD/2), warps 6-9 the other halves
     const int quarter = warp & 3;
-    const int half = warp >= 6 ? 1 : 0;
     const int lane = threadIdx.x & 31;
     const int r = quarter * 32 + lane;
     const int64_t P = P0 + r;
@@ -523,36 +487,11 @@ __global__ void __launch_bounds__(320, 1)
     const float sc = p.scale * 1.4426950408889634f;
     const int64_t si = ((int64_t)b * p.H + h) * p.n + i0 + r;
     const float nL = r < nq ? -p.lse[si] * 1.4426950408889634f : -INFINITY;  // exp2(s*sc - lse*log2e)
+    const float Dr = r < nq ? p.Dsum[si] : 0.f;
     const int64_t lo_key = P - p.window + 1;
     const uint32_t span = (uint32_t)(P - lo_key);
     bool ok = true;
-    float Dr = 0.f;
-    if (p.dsum_in_dq) {
-      // D = rowsum(dO * O) for this row and head, from the staged dO tile and O; the
-      // dK/dV kernel that follows reads it from Dsum
-      ok = mbar_wait(q_full, 0, err, DEV_TIMEOUT_FULL);
-      if (ok && r < nq) {
-        const bf16* Orow = (const bf16*)p.O + ((int64_t)b * p.n + i0 + r) * p.ldo + h * HD;
-        float acc = 0.f;
-#pragma unroll
-        for (int kb = 0; kb < KB; ++kb) {
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 a = *(const uint4*)(sm + Cf::OFF_DO + kb * Cf::BM * 128 + r * 128 + ((c ^ (r & 7)) << 4));
-            const uint4 o = *(const uint4*)(Orow + kb * 64 + c * 8);
-            const bf16* ae = reinterpret_cast<const bf16*>(&a);
-            const bf16* oe = reinterpret_cast<const bf16*>(&o);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc = fmaf(__bfloat162float(ae[e]), __bfloat162float(oe[e]), acc);
-          }
-        }
-        Dr = acc;
-        if (half == 0) p.Dsum[si] = Dr;
-      }
-    } else {
-      Dr = r < nq ? p.Dsum[si] : 0.f;
-    }
-    for (int j = 0; j < ntiles && ok; ++j) {
+    for (int j = 0; j < ntiles; ++j) {
       const int s = j & 1;
       const int64_t j0 = jt0 + (int64_t)j * Cf::BN;
       const bool need_mask = (j0 + Cf::BN - 1 > P0) || (j0 < Plast - p.window + 1);
@@ -562,28 +501,30 @@ __global__ void __launch_bounds__(320, 1)
         break;
       }
       tc_fence_after();
-      uint32_t sr[32], dr[32];
-      tmem_ld32_nowait(tmem + lane_base + Cf::s_col(s) + half * 32, sr);
-      tmem_ld32_nowait(tmem + lane_base + Cf::dp_col(s) + half * 32, dr);
+      uint32_t sr[64], dr[64];
+      tmem_ld32_nowait(tmem + lane_base + Cf::s_col(s), sr);
+      tmem_ld32_nowait(tmem + lane_base + Cf::s_col(s) + 32, sr + 32);
+      tmem_ld32_nowait(tmem + lane_base + Cf::dp_col(s), dr);
+      tmem_ld32_nowait(tmem + lane_base + Cf::dp_col(s) + 32, dr + 32);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sp_free[s]);  // S/dP buffer s may be overwritten by tile j+2
       uint8_t* drow = sm + Cf::OFF_DS + s * Cf::DSB + r * 128;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 8; ++cc) {
         float ds[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int c = cc * 8 + e;
           float pr = ex2_tc(fmaf(__uint_as_float(sr[c]), sc, nL));
           if (need_mask) {
-            const uint32_t off = (uint32_t)(j0 + half * 32 + c - lo_key);
+            const uint32_t off = (uint32_t)(j0 + c - lo_key);
             pr = off <= span ? pr : 0.f;
           }
           ds[e] = pr * (__uint_as_float(dr[c]) - Dr);
         }
-        *(uint4*)(drow + (((half * 4 + cc) ^ (r & 7)) << 4)) =
+        *(uint4*)(drow + ((cc ^ (r & 7)) << 4)) =
             make_uint4(pack_bf16x2(ds[0], ds[1]), pack_bf16x2(ds[2], ds[3]), pack_bf16x2(ds[4], ds[5]),
                        pack_bf16x2(ds[6], ds[7]));
       }
@@ -595,7 +536,7 @@ __global__ void __launch_bounds__(320, 1)
       tc_fence_after();
       bf16* dQ = (bf16*)p.dQ + ((int64_t)b * p.n + i0 + r) * p.lddq + h * HD;
 #pragma unroll 1
-      for (int c = half * (HD / 64); c < (half + 1) * (HD / 64); ++c) {
+      for (int c = 0; c < HD / 32; ++c) {
         float o[32];
         tmem_ld32(tmem + lane_base + Cf::DQ_COL + c * 32, o);
         if (r < nq) {
@@ -650,6 +591,10 @@ template <int HD> struct AttnDkvCfg {
   static __device__ __forceinline__ uint32_t s_col(int b) { return 256 + b * 128; }
   static __device__ __forceinline__ uint32_t dp_col(int b) { return 256 + b * 128 + 64; }
 };
+
+__device__ __forceinline__ void named_bar_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 template <int HD>
 __global__ void __launch_bounds__(192, 1)

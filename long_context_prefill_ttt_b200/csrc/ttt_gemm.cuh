@@ -57,12 +57,6 @@ struct GemmParams {
   // (consecutive tiles share A rows), 1 = column blocks outer (consecutive tiles share
   // B rows, so a B larger than L2 streams from DRAM once). Set by the host.
   int m_fast;
-  // Upper bound on the CTAs of a tensor-core launch (0 = one per SM). A GEMM that runs
-  // beside another stream's work on the SMs that work leaves idle is capped this way.
-  int max_ctas;
-  // 1: launch without programmatic dependent launch. Kernels on the side stream use it:
-  // an early-launched successor would hold SMs the other stream needs while it waits.
-  int no_pdl;
 };
 
 // ============================================================== epilogue (per element)

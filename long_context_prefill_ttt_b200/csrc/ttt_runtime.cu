@@ -53,20 +53,6 @@ static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
-// Same launch, with programmatic dependent launch only when `pdl` (the kernel's
-// pdl_wait is then a no-op).
-template <typename... KArgs, typename... Args>
-static cudaError_t launch_maybe_pdl(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                                    cudaStream_t st, Args... args) {
-  if (pdl) return launch_pdl(kern, grid, block, smem, st, args...);
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  return cudaLaunchKernelEx(&cfg, kern, args...);
-}
-
 // Row-kernel launches (PDL): RMSNorm with row_threads(d) threads per row in
 // blocks of 256; RoPE with one thread per 8 pairs.
 template <typename T>
@@ -161,10 +147,8 @@ static cudaError_t launch_tc(const GemmParams& p, cudaStream_t st, int* err, int
   if (!*ok) return cudaSuccess;
   using C = TcCfg<BN>;
   const int tiles = ((p.M + TC_BM - 1) / TC_BM) * (p.N / BN) * p.batch;
-  int grid = tiles < num_sms ? tiles : num_sms;
-  if (p.max_ctas > 0 && grid > p.max_ctas) grid = p.max_ctas;
-  return launch_maybe_pdl(!p.no_pdl, gemm_tc_kernel<BN, AM, BM>, dim3(grid), dim3(TC_THREADS), C::SMEM, st, ta, tb,
-                          tb2, p, err);
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  return launch_pdl(gemm_tc_kernel<BN, AM, BM>, dim3(grid), dim3(TC_THREADS), C::SMEM, st, ta, tb, tb2, p, err);
 }
 
 // Pairs of CTAs that can be resident at once for one paired-GEMM variant (0 = the
@@ -207,8 +191,7 @@ static cudaError_t launch_tc2(const GemmParams& p, cudaStream_t st, int* err, bo
     return cudaSuccess;
   }
   const int tiles = ((p.M + 2 * TC_BM - 1) / (2 * TC_BM)) * (p.N / BN) * p.batch;
-  int pairs = tiles < cap ? tiles : cap;
-  if (p.max_ctas > 0 && pairs > p.max_ctas / 2) pairs = p.max_ctas / 2 > 0 ? p.max_ctas / 2 : 1;
+  const int pairs = tiles < cap ? tiles : cap;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
   cfg.blockDim = dim3(TC_THREADS);
@@ -222,7 +205,7 @@ static cudaError_t launch_tc2(const GemmParams& p, cudaStream_t st, int* err, bo
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = p.no_pdl ? 1 : 2;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel<BN, AM, BM>, ta, tb, tb2, p, err);
 }
 
@@ -257,8 +240,8 @@ cudaError_t attn_fwd_tc_launch(const AttnParams& p, cudaStream_t st, int* err, b
   }
   if (!*ok) return cudaSuccess;
   dim3 grid((p.n + 127) / 128, p.H, p.B);
-  if (p.hd == 128) return launch_pdl(attn_fwd_tc_kernel<128>, grid, dim3(320), AttnTcCfg<128>::SMEM, st, tq, tk, tv, p, err);
-  return launch_pdl(attn_fwd_tc_kernel<64>, grid, dim3(320), AttnTcCfg<64>::SMEM, st, tq, tk, tv, p, err);
+  if (p.hd == 128) return launch_pdl(attn_fwd_tc_kernel<128>, grid, dim3(192), AttnTcCfg<128>::SMEM, st, tq, tk, tv, p, err);
+  return launch_pdl(attn_fwd_tc_kernel<64>, grid, dim3(192), AttnTcCfg<64>::SMEM, st, tq, tk, tv, p, err);
 }
 
 bool attn_dq_tc_ok(const AttnParams& p) {
@@ -280,9 +263,9 @@ cudaError_t attn_bwd_dq_tc_launch(const AttnParams& p, cudaStream_t st, int* err
   if (!*ok) return cudaSuccess;
   dim3 grid((p.n + 127) / 128, p.H, p.B);
   if (p.hd == 128)
-    return launch_pdl(attn_bwd_dq_tc_kernel<128>, grid, dim3(320), AttnDqCfg<128>::SMEM, st, tq, tkv, tk, tv, tdo,
+    return launch_pdl(attn_bwd_dq_tc_kernel<128>, grid, dim3(192), AttnDqCfg<128>::SMEM, st, tq, tkv, tk, tv, tdo,
                       p, err);
-  return launch_pdl(attn_bwd_dq_tc_kernel<64>, grid, dim3(320), AttnDqCfg<64>::SMEM, st, tq, tkv, tk, tv, tdo, p,
+  return launch_pdl(attn_bwd_dq_tc_kernel<64>, grid, dim3(192), AttnDqCfg<64>::SMEM, st, tq, tkv, tk, tv, tdo, p,
                     err);
 }
 
@@ -402,17 +385,19 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
     // 256 wins unless 128-wide tiles need fewer than 1.32x the persistent-grid waves
     // (ceil(tiles / SMs)): the small-M shapes with N = 2048.
     const int m_tiles = (p.M + TC_BM - 1) / TC_BM;
-    const int ctas = p.max_ctas > 0 && p.max_ctas < num_sms ? p.max_ctas : num_sms;
-    auto waves = [&](int bn) { return std::ceil((double)m_tiles * (p.N / bn) * p.batch / ctas); };
+    auto waves = [&](int bn) { return std::ceil((double)m_tiles * (p.N / bn) * p.batch / num_sms); };
     const bool n256 = (p.N % 256 == 0) && waves(128) >= 1.32 * waves(256);
     // walk the larger operand once: column blocks outer when B is the larger matrix
     pt.m_fast = p.N > p.M ? 1 : 0;
     bool ok = false;
     cudaError_t e = cudaSuccess;
-    if (engine != GEMM_TC1 && p.M > TC_BM) {
+    // CTA pairs pay where the tile count is large: the frozen blocks' GEMMs over a whole
+    // segment (11% faster at 32768 rows) and the wide LM head (13% faster); on the
+    // 1024-row products of an adaptive step they are 2-20% slower than single-CTA tiles
+    // (measured per shape on B200), so those keep the single-CTA kernel.
+    if (engine != GEMM_TC1 && p.M > TC_BM && (p.M >= 4096 || p.N >= 16384)) {
       // CTA pairs: 256-row tiles, waves counted in resident pairs
-      int cap = pair_capacity<128, false, false>();
-      if (p.max_ctas > 0 && cap > p.max_ctas / 2) cap = p.max_ctas / 2 > 0 ? p.max_ctas / 2 : 1;
+      const int cap = pair_capacity<128, false, false>();
       if (cap > 0) {
         const int m2 = (p.M + 2 * TC_BM - 1) / (2 * TC_BM);
         auto waves2 = [&](int bn) { return std::ceil((double)m2 * (p.N / bn) * p.batch / cap); };
@@ -515,10 +500,7 @@ struct Arena {
 
 // Kernel-class timer: CUDA events recorded on the launching stream around each
 // launch of a class, plus the algorithmic FLOPs and bytes of that launch.
-// PC_GEMM_WGRAD: the adaptive weight-gradient + SGD GEMMs when they run on the side
-// stream beside the backward chain (their time overlaps the other classes').
-enum ProfClass : int { PC_GEMM_FROZEN = 0, PC_GEMM_TTT = 1, PC_ATTN_FWD = 2, PC_ATTN_BWD = 3, PC_GEMM_WGRAD = 4,
-                       PC_COUNT = 5 };
+enum ProfClass : int { PC_GEMM_FROZEN = 0, PC_GEMM_TTT = 1, PC_ATTN_FWD = 2, PC_ATTN_BWD = 3, PC_COUNT = 4 };
 struct Profiler {
   bool on = false;
   std::vector<cudaEvent_t> ev;     // pairs
@@ -664,15 +646,6 @@ template <typename T> class Engine : public ttt_handle {
   // per-call growable buffers
   int64_t chunk_pos = 0;                  // absolute position of row 0 of the chunk in the adaptive buffers
   bool decode_mode = false;               // set while a decode token step is being captured
-  // Side stream of the adaptive weight-gradient + SGD GEMMs: during the backward every
-  // kernel of the chain occupies at most 128 SMs, so these GEMMs, which nothing in the
-  // chain waits for, run beside it on the remaining side_ctas SMs. ev_chain[j]: block
-  // j's inputs of those GEMMs are ready and its W1t dgrad has read W1t; ev_side[j]:
-  // block j's fast weights are updated and its activations may be overwritten.
-  cudaStream_t side_st = nullptr;
-  int side_ctas = 0;
-  std::vector<cudaEvent_t> ev_chain, ev_side;
-  std::vector<T*> GTm, dhidt;             // per adaptive block: dL/d(m) (bf16) and dL/d(u) rows
   cudaStream_t cap_st = nullptr;          // private stream the decode step is captured on (the caller's
                                           // stream may be the legacy default stream, which cannot capture)
   int64_t* pos_dev = nullptr;             // device copy of the position of the token being decoded
@@ -684,10 +657,6 @@ template <typename T> class Engine : public ttt_handle {
 
   ~Engine() override {
     if (st) cudaStreamSynchronize(st);
-    if (side_st) cudaStreamSynchronize(side_st);
-    for (cudaEvent_t e : ev_chain) cudaEventDestroy(e);
-    for (cudaEvent_t e : ev_side) cudaEventDestroy(e);
-    if (side_st) cudaStreamDestroy(side_st);
     if (cap_st) cudaStreamDestroy(cap_st);
     call_arena.release();
     arena.release();
@@ -709,14 +678,13 @@ template <typename T> class Engine : public ttt_handle {
 
  private:
   int gemm_class = PC_GEMM_FROZEN;
-  int gemm(GemmParams p, cudaStream_t on = nullptr, int cls = -1) {
+  int gemm(GemmParams p) {
     const size_t es = is_bf16 ? 2 : 4;
-    if (!on) on = st;
-    prof.begin(on, cls >= 0 ? cls : gemm_class, 2.0 * p.M * p.N * (double)p.K * p.batch,
+    prof.begin(st, gemm_class, 2.0 * p.M * p.N * (double)p.K * p.batch,
                (double)p.batch * ((double)p.M * p.K * es + (double)p.N * p.K * es +
                                   (double)p.M * p.N * (p.d_f32 ? 4 : es)));
-    const int e = gemm_launch(p, is_bf16 ? 1 : 0, on, dev_err, num_sms, GEMM_AUTO);
-    prof.end(on);
+    const int e = gemm_launch(p, is_bf16 ? 1 : 0, st, dev_err, num_sms, GEMM_AUTO);
+    prof.end(st);
     ++launches;
     if (e != 0) {
       poisoned = true;
@@ -766,12 +734,6 @@ template <typename T> class Engine : public ttt_handle {
                int64_t loss_off, bool grad, bool commit);
   int sync_and_check();
   int ensure(void** ptr, int64_t* cap, int64_t need, size_t elem);
-  // The caller's stream waits for all work on the side stream.
-  int join_side() {
-    if (!side_st) return TTT_OK;
-    for (int j = 0; j < Lt; ++j) TTT_CUDA(cudaStreamWaitEvent(st, ev_side[j], 0));
-    return TTT_OK;
-  }
 };
 
 template <typename T> int Engine<T>::ensure(void** ptr, int64_t* cap, int64_t need, size_t elem) {
@@ -818,19 +780,6 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
   TTT_CUDA((cudaError_t)prime_kernel_attributes());
   TTT_CUDA(cudaStreamCreateWithFlags(&cap_st, cudaStreamNonBlocking));
   TTT_CUDA(cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev));
-  // the backward chain's kernels use at most 128 SMs (64 CTA pairs or 128 CTAs)
-  side_ctas = is_bf16 && Lt > 0 && num_sms >= 136 ? ((num_sms - 128) & ~1) : 0;
-  if (side_ctas > 0) {
-    int lo = 0, hi = 0;
-    TTT_CUDA(cudaDeviceGetStreamPriorityRange(&lo, &hi));
-    TTT_CUDA(cudaStreamCreateWithPriority(&side_st, cudaStreamNonBlocking, lo));
-    ev_chain.resize(Lt);
-    ev_side.resize(Lt);
-    for (int j = 0; j < Lt; ++j) {
-      TTT_CUDA(cudaEventCreateWithFlags(&ev_chain[j], cudaEventDisableTiming));
-      TTT_CUDA(cudaEventCreateWithFlags(&ev_side[j], cudaEventDisableTiming));
-    }
-  }
 
   const int64_t Ms = (int64_t)B * S, Mc = (int64_t)B * bsz;
   dev_err = arena.get<int>(1);
@@ -907,12 +856,6 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
   G = arena.get<float>((size_t)Mc * d);
   GT = arena.get<T>((size_t)Mc * d);
   dhid = arena.get<T>((size_t)Mc * (ht > hs ? ht : hs));
-  GTm.resize(Lt);
-  dhidt.resize(Lt);
-  for (int j = 0; j < Lt; ++j) {
-    GTm[j] = side_st ? arena.get<T>((size_t)Mc * d) : nullptr;
-    dhidt[j] = side_st ? arena.get<T>((size_t)Mc * ht) : nullptr;
-  }
   dr = arena.get<float>((size_t)Mc * d);
   dqkv = arena.get<T>((size_t)Mc * 3 * d);
   dob = arena.get<T>((size_t)Mc * d);
@@ -1021,7 +964,6 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
 
 template <typename T> int Engine<T>::reset() {
   if (poisoned) return fail(this, TTT_ERR_POISONED, "handle poisoned by an earlier device error");
-  if (int rc = join_side()) return rc;
   for (int l = first_ttt; l < L; ++l) {
     LayerDev<T>& Lw = layers[l];
     const int64_t n1 = (int64_t)ht * d;
@@ -1151,9 +1093,7 @@ template <typename T> int Engine<T>::ttt_forward(int cn, int64_t pos, bool commi
     if ((rc = attention_block(Lw, l, A.x, A.a, A.r3 /*scratch for r1*/, A.rstd1, A.qkv, A.o, A.lse, cn, pos,
                               commit)) != TTT_OK)
       return rc;
-    // TTT-MLP with the fast weights of each sequence (batched over sequences), after the
-    // previous chunk's update of this block (side stream) has landed and released A.r2, A.g
-    if (side_st && !decode_mode) TTT_CUDA(cudaStreamWaitEvent(st, ev_side[j], 0));
+    // TTT-MLP with the fast weights of each sequence (batched over sequences)
     rmsnorm_fwd_launch<T>((const float*)A.a, d, Lw.g_ttt, cfg.rms_eps, rows, d, A.r2, d, A.rstd2, st);
     TTT_LAUNCHED();
     GemmParams p = gp(cn, ht, d, A.r2, d, false, Lw.W1t, d, false, A.g, ht, false, EPI_GELU);
@@ -1199,52 +1139,33 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
     p.X = A.us; p.ldx = hs;
     if ((rc = gemm(p)) != TTT_OK) return rc;
     if ((rc = gemm(gp(rows, d, hs, dhid, hs, false, Lw.W1s, d, true, dr, d, true, EPI_STORE))) != TTT_OK) return rc;
-    // gradient at m (the TTT-MLP's output); with the side stream its bf16 copy is this
-    // block's own buffer, read later by the weight gradient of W2t
-    T* gm = side_st ? GTm[j] : GT;
-    T* du = side_st ? dhidt[j] : dhid;
-    rmsnorm_bwd_launch<T>((const float*)A.m, Lw.g_static, A.rstd3, dr, G, rows, d, G, gm, st);
+    rmsnorm_bwd_launch<T>((const float*)A.m, Lw.g_static, A.rstd3, dr, G, rows, d, G, GT, st);
     TTT_LAUNCHED();
     // TTT-MLP data gradients (with W_{i-1}), then the fused weight gradient + SGD
-    p = gp(cn, ht, d, gm, d, false, Lw.W2t, ht, true, du, ht, false, EPI_DGELU);
+    p = gp(cn, ht, d, GT, d, false, Lw.W2t, ht, true, dhid, ht, false, EPI_DGELU);
     p.batch = B; p.sA = (int64_t)cn * d; p.sD = (int64_t)cn * ht;
     fast_operand(p, Lw.W2t_init, Lw.W2t, (int64_t)d * ht);
     p.X = A.u; p.ldx = ht; p.sX = (int64_t)cn * ht;
     if ((rc = gemm(p)) != TTT_OK) return rc;
     if (j > 0) {
-      p = gp(cn, d, ht, du, ht, false, Lw.W1t, d, true, dr, d, true, EPI_STORE);
+      p = gp(cn, d, ht, dhid, ht, false, Lw.W1t, d, true, dr, d, true, EPI_STORE);
       p.batch = B; p.sA = (int64_t)cn * ht; p.sD = (int64_t)cn * d;
       fast_operand(p, Lw.W1t_init, Lw.W1t, (int64_t)ht * d);
       if ((rc = gemm(p)) != TTT_OK) return rc;
     }
-    // Both data gradients have read W_{i-1}; the weight gradients + SGD may now run. With
-    // the side stream they start on it here and overlap the rest of the backward.
-    cudaStream_t wst = st;
-    int wcls = -1;
-    if (side_st) {
-      TTT_CUDA(cudaEventRecord(ev_chain[j], st));
-      TTT_CUDA(cudaStreamWaitEvent(side_st, ev_chain[j], 0));
-      wst = side_st;
-      wcls = PC_GEMM_WGRAD;
-    }
     // dW2t[o][i] = sum_t dm[t][o] g[t][i]  -> W2t32 += -eta * dW2t ; bf16 copy refreshed
     // (bf16 path: W2t32 holds the accumulated update dW, so the copy keeps its precision)
-    p = gp(d, ht, cn, gm, d, true, A.g, ht, true, Lw.W2t32, ht, true, EPI_SGD);
+    p = gp(d, ht, cn, GT, d, true, A.g, ht, true, Lw.W2t32, ht, true, EPI_SGD);
     p.batch = B; p.sA = (int64_t)cn * d; p.sB = (int64_t)cn * ht; p.sD = (int64_t)d * ht;
     p.alpha = -cfg.eta;
-    p.max_ctas = side_st ? side_ctas : 0;
-    p.no_pdl = side_st ? 1 : 0;
     if (is_bf16) { p.Y = Lw.W2t; p.ldy = ht; p.sY = (int64_t)d * ht; }
-    if ((rc = gemm(p, wst, wcls)) != TTT_OK) return rc;
+    if ((rc = gemm(p)) != TTT_OK) return rc;
     // dW1t[o][i] = sum_t du[t][o] r2[t][i]
-    p = gp(ht, d, cn, du, ht, true, A.r2, d, true, Lw.W1t32, d, true, EPI_SGD);
+    p = gp(ht, d, cn, dhid, ht, true, A.r2, d, true, Lw.W1t32, d, true, EPI_SGD);
     p.batch = B; p.sA = (int64_t)cn * ht; p.sB = (int64_t)cn * d; p.sD = (int64_t)ht * d;
     p.alpha = -cfg.eta;
-    p.max_ctas = side_st ? side_ctas : 0;
-    p.no_pdl = side_st ? 1 : 0;
     if (is_bf16) { p.Y = Lw.W1t; p.ldy = d; p.sY = (int64_t)ht * d; }
-    if ((rc = gemm(p, wst, wcls)) != TTT_OK) return rc;
-    if (side_st) TTT_CUDA(cudaEventRecord(ev_side[j], side_st));
+    if ((rc = gemm(p)) != TTT_OK) return rc;
     if (j == 0) break;  // upstream of the first adaptive MLP does not depend on the fast weights
     rmsnorm_bwd_launch<T>((const float*)A.a, Lw.g_ttt, A.rstd2, dr, G, rows, d, G, GT, st);
     TTT_LAUNCHED();
@@ -1263,22 +1184,17 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
     // dK, dV over current-chunk keys only (dS^T Q, P^T dO)
     prof.begin(st, PC_ATTN_BWD,
                2.0 * hd * H * (double)B * (2.0 * attn_pairs(cn, chunk_pos) + 2.0 * attn_pairs(cn, 0)), 0.0);
-    // dQ and dK/dV: tcgen05 kernels where they apply (the dQ kernel forms D = rowsum(dO * O)
-    // itself), else a separate D pass and the mma.sync or SIMT kernels
+    attn_bwd_prep_kernel<T><<<nblk((int64_t)rows * H, 8), 256, 0, st>>>(ap);
+    TTT_LAUNCHED();
+    // dQ and dK/dV: tcgen05 kernels where they apply, else mma.sync, else SIMT
     bool dq_done = false, dkv_done = false;
     if (is_bf16 && attn_dq_tc_ok(ap)) {
-      ap.dsum_in_dq = 1;
       cudaError_t e = attn_bwd_dq_tc_launch(ap, st, dev_err, &dq_done);
-      ap.dsum_in_dq = 0;
-      if (e == cudaSuccess && dq_done && attn_dkv_tc_ok(ap)) e = attn_bwd_dkv_tc_launch(ap, st, dev_err, &dkv_done);
+      if (e == cudaSuccess && attn_dkv_tc_ok(ap)) e = attn_bwd_dkv_tc_launch(ap, st, dev_err, &dkv_done);
       if (e != cudaSuccess) {
         poisoned = true;
         return fail(this, TTT_ERR_CUDA, std::string("attention backward: ") + cudaGetErrorString(e));
       }
-    }
-    if (!dq_done) {
-      attn_bwd_prep_kernel<T><<<nblk((int64_t)rows * H, 8), 256, 0, st>>>(ap);
-      TTT_LAUNCHED();
     }
     if (!(dq_done && dkv_done)) {
       if (is_bf16 && attn_mma_ok(ap)) {
@@ -1413,7 +1329,6 @@ template <typename T> int Engine<T>::prefill(const int32_t* tokens, int64_t T_, 
   }
   gather_tokens_kernel<<<nblk(B, 256), 256, 0, st>>>(tok_dev, ld, T_, 1, B, pend_tok_dev, 1, 0);
   TTT_LAUNCHED();
-  if ((rc = join_side()) != TTT_OK) return rc;
   if (kind == TTT_PTR_HOST) {
     TTT_CUDA(cudaMemcpyAsync(out, loss_dev, (size_t)B * T_ * 4, cudaMemcpyDeviceToHost, st));
   }
@@ -1490,7 +1405,6 @@ int Engine<T>::decode(int64_t n, const int32_t* forced, int32_t* out_tok, float*
     fdev = forced;
   }
   const int64_t base = n_pos;
-  if ((rc = join_side()) != TTT_OK) return rc;
   TTT_CUDA(cudaMemcpyAsync(pos_dev, &base, sizeof(int64_t), cudaMemcpyHostToDevice, st));
   TTT_CUDA(cudaStreamSynchronize(st));  // the source lives on the host stack
   // capture one token step
@@ -1534,8 +1448,7 @@ int Engine<T>::decode(int64_t n, const int32_t* forced, int32_t* out_tok, float*
     ++pend_cnt;
     ++n_pos;
     if (pend_cnt == bsz) {  // a full chunk of decoded positions: differentiate and update
-      if (Lt > 0 && ((rc = ttt_step(pend_in, pend_tgt, bsz, n_pos - bsz, nullptr, 0, 0, true, false)) != TTT_OK ||
-                     (rc = join_side()) != TTT_OK)) {
+      if (Lt > 0 && (rc = ttt_step(pend_in, pend_tgt, bsz, n_pos - bsz, nullptr, 0, 0, true, false)) != TTT_OK) {
         cudaGraphExecDestroy(exec);
         return rc;
       }
@@ -1560,7 +1473,6 @@ int Engine<T>::decode(int64_t n, const int32_t* forced, int32_t* out_tok, float*
 template <typename T> int Engine<T>::get_weights(int32_t seq, int32_t j, float* w1, float* w2, int32_t kind) {
   if (poisoned) return fail(this, TTT_ERR_POISONED, "handle poisoned by an earlier device error");
   if (seq < 0 || seq >= B || j < 0 || j >= Lt) return fail(this, TTT_ERR_INVALID_ARG, "get_weights: bad index");
-  if (int rc = join_side()) return rc;
   const LayerDev<T>& Lw = layers[first_ttt + j];
   const int64_t n1 = (int64_t)ht * d;
   const cudaMemcpyKind k = kind == TTT_PTR_HOST ? cudaMemcpyDeviceToHost : cudaMemcpyDeviceToDevice;

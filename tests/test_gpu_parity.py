@@ -247,3 +247,27 @@ def test_m125_decode_bf16_greedy_matches_oracle(T):
             g1, g2 = T.ttt_get_weights(h, s, j)
             o1, o2 = orc.fast_weights(s, j)
             assert P.rel_fro(g1, o1) <= 5e-3 and P.rel_fro(g2, o2) <= 5e-3
+
+
+@pytest.mark.slow
+def test_b1_128k_bf16_past_window_fill_matches_stored_oracle(T):
+    """The ~1B workload on 16384 positions (16 chunks; chunks 9-16 see a full 8192-key
+    window), run as the 128K benchmark runs it but in 4 frozen segments of 4096 so
+    that every segment reads its predecessor's keys from the ring, whose 9216 slots
+    wrap. The oracle's results come from tests/golden/make_b1_prefix_T16384.py."""
+    import os
+    g = np.load(os.path.join(os.path.dirname(__file__), "golden", "b1_128k_bf16_T16384.npz"))
+    cfg = syn.config("b1_128k_bf16", T=int(g["T"]))
+    w = syn.make_weights(cfg)
+    toks = syn.make_token_batch(cfg)
+    h = T.ttt_create(cfg, w, max_segment=4096)
+    gl = T.ttt_prefill(h, np.ascontiguousarray(toks, dtype=np.int32))[0]
+    ol = g["losses"]
+    assert np.all(np.isfinite(gl))
+    assert float(np.max(np.abs(gl - ol) / np.abs(ol))) <= 2e-2
+    for j in range(cfg.n_ttt):
+        w1, w2 = T.ttt_get_weights(h, 0, j)
+        for W, r, ref, ref0 in ((w1, g["r1"], g["w1r"][j], g["w1r0"][j]), (w2, g["r2"], g["w2r"][j], g["w2r0"][j])):
+            got = W.astype(np.float64) @ r
+            assert P.rel_fro(got, ref) <= 5e-3
+            assert P.rel_fro(got - ref0, ref - ref0) <= 5e-2
