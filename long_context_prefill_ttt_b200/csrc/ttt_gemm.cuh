@@ -327,9 +327,14 @@ __device__ __forceinline__ void epi_ce32(const GemmParams& p, int m, int n, floa
     d[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
                       pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
   if (tgt >= n && tgt < n + 32) {
-    float zt = v[0];
+    // v[tgt - n] by predicated selects: an indexed read would move v to local memory
+    const int k = tgt - n;
+    float zt = 0.f;
 #pragma unroll
-    for (int i = 1; i < 32; ++i) zt = (tgt - n == i) ? v[i] : zt;
+    for (int i = 0; i < 32; ++i)
+      asm("{\n\t.reg .pred q;\n\tsetp.eq.s32 q, %2, %3;\n\tselp.f32 %0, %1, %0, q;\n\t}"
+          : "+f"(zt)
+          : "f"(v[i]), "r"(k), "r"(i));
     p.ce_zt[m] = zt;
   }
   const float M = fmaxf(cm, mx);
