@@ -51,6 +51,9 @@ struct GemmParams {
   const float2* rope_lo; const float2* rope_hi;
   int64_t rope_pos0; const int64_t* rope_pos_dev;
   int rope_n, rope_hd, rope_cols;
+  // Optional: the same pass appends the rotated keys and the values of the rows to the
+  // window ring [batch][rope_C][rope_cols/2] at slot (position mod rope_C).
+  void* rope_ring_k; void* rope_ring_v; int rope_C;
   // EPI_CE: targets [M] (batch 1), partials [M][N / 64], target logits [M]
   const int32_t* ce_tgt; float2* ce_part; float* ce_zt;
   // Tile order of the tensor-core engine within a batch slice: 0 = row blocks outer

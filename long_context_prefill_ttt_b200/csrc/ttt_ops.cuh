@@ -237,7 +237,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ qk, int64_t ld, int ncols, int rows, int n,
                                                    int64_t pos0, int hd, const float2* __restrict__ lo_tab,
                                                    const float2* __restrict__ hi_tab, int inverse,
-                                                   const int64_t* pos_dev = nullptr) {
+                                                   const int64_t* pos_dev = nullptr, T* __restrict__ ring_k = nullptr,
+                                                   T* __restrict__ ring_v = nullptr, int C = 0) {
   pdl_wait();
   pdl_trigger();
   if (pos_dev) pos0 = *pos_dev;  // position held on the device (graph-captured decode step)
@@ -284,11 +285,26 @@ __global__ void __launch_bounds__(256) rope_kernel(T* __restrict__ qk, int64_t l
       }
       st8(base, x1);
       st8(base + half, x2);
+      // window ring: a key head's rotated pairs and the same elements of its value head
+      // go to the row's slot (position mod C) of sequence row / n
+      const int dq = ncols >> 1;  // columns [0, dq) are q, [dq, 2 dq) k, [2 dq, 3 dq) v
+      if (ring_k && head * hd >= dq) {
+        const int64_t off = ((int64_t)(row / n) * C + pos % C) * dq + (head * hd - dq) + i;
+        st8(ring_k + off, x1);
+        st8(ring_k + off + half, x2);
+        float v1[8], v2[8];
+        ld8(base + dq, v1);
+        ld8(base + dq + half, v2);
+        st8(ring_v + off, v1);
+        st8(ring_v + off + half, v2);
+      }
     }
   }
 }
 
-// Grid of rope_kernel for rows x ncols (head dim hd).
+// Grid of rope_kernel for rows x ncols (head dim hd). With ring_k/ring_v the kernel
+// also appends each row's rotated key and its value (columns [ncols/2, 3 ncols/2) of
+// the q|k|v row) to the window ring [B][C][ncols/2] at slot (position mod C).
 inline int64_t rope_threads(int rows, int ncols, int hd) {
   const int nheads = ncols / hd;
   return (int64_t)rows * (hd >> 4) * ((nheads + RP_HEADS - 1) / RP_HEADS);

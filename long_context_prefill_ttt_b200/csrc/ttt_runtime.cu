@@ -84,11 +84,11 @@ static cudaError_t rmsnorm_bwd_launch(const float* x, const float* g, const floa
 template <typename T>
 static cudaError_t rope_launch(T* qk, int64_t ld, int ncols, int rows, int n, int64_t pos0, int hd,
                                const float2* lo, const float2* hi, int inverse, const int64_t* pos_dev,
-                               cudaStream_t st) {
+                               cudaStream_t st, void* ring_k = nullptr, void* ring_v = nullptr, int C = 0) {
   const int64_t threads = rope_threads(rows, ncols, hd);
   if (threads >= (int64_t)INT32_MAX || ncols % hd) return cudaErrorInvalidValue;
   return launch_pdl(rope_kernel<T>, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, st, qk, ld, ncols, rows,
-                    n, pos0, hd, lo, hi, inverse, pos_dev);
+                    n, pos0, hd, lo, hi, inverse, pos_dev, (T*)ring_k, (T*)ring_v, C);
 }
 
 // ============================================================== GEMM dispatch (host)
@@ -369,9 +369,9 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
     if (p.epi == EPI_QKV_ROPE) {
       const cudaError_t re =
         elem_is_bf16 ? rope_launch<bf16>((bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd,
-                                         p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st)
+                                         p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st, p.rope_ring_k, p.rope_ring_v, p.rope_C)
                      : rope_launch<float>((float*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd,
-                                          p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st);
+                                          p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st, p.rope_ring_k, p.rope_ring_v, p.rope_C);
     if (re != cudaSuccess) return (int)re;
     }
     return (int)cudaGetLastError();
@@ -414,7 +414,7 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
     if (ok) {
       if (p.epi == EPI_QKV_ROPE) {
         return (int)rope_launch<bf16>((bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd,
-                                      p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st);
+                                      p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st, p.rope_ring_k, p.rope_ring_v, p.rope_C);
       }
       return 0;
     }
@@ -428,7 +428,7 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
     if (ok) {
       if (p.epi == EPI_QKV_ROPE) {
         return (int)rope_launch<bf16>((bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd,
-                                      p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st);
+                                      p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st, p.rope_ring_k, p.rope_ring_v, p.rope_C);
       }
       return 0;
     }
@@ -444,9 +444,9 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
   if (p.epi == EPI_QKV_ROPE) {
     const cudaError_t re =
         elem_is_bf16 ? rope_launch<bf16>((bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd,
-                                         p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st)
+                                         p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st, p.rope_ring_k, p.rope_ring_v, p.rope_C)
                      : rope_launch<float>((float*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd,
-                                          p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st);
+                                          p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st, p.rope_ring_k, p.rope_ring_v, p.rope_C);
     if (re != cudaSuccess) return (int)re;
   }
   return (int)cudaGetLastError();
@@ -999,21 +999,22 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
   int rc;
   rmsnorm_fwd_launch<T>((const float*)xin, d, Lw.g_attn, cfg.rms_eps, rows, d, r, d, rstd, st);
   TTT_LAUNCHED();
+  // The chunk's keys and values go to the ring in the RoPE pass when that cannot
+  // overwrite a slot this attention still reads: rows of a chunk of n <= b positions
+  // and the window before them span n + k - 1 < C positions. (A frozen segment is
+  // longer than the ring and appends after its attention.) Decode appends its one
+  // position there too, then attends over the window entirely from the ring.
+  const bool append_in_rope = commit && (decode_mode || n <= bsz);
   {  // q|k|v = r Wqkv^T with RoPE applied to q and k in the GEMM epilogue
     GemmParams pq = gp(rows, 3 * d, d, r, d, false, Lw.Wqkv, d, false, qkv, 3 * d, false, EPI_QKV_ROPE);
     pq.rope_lo = rope_lo; pq.rope_hi = rope_hi; pq.rope_hd = hd; pq.rope_cols = 2 * d;
     pq.rope_n = decode_mode ? 1 : n;
     pq.rope_pos0 = decode_mode ? 0 : q0;
     pq.rope_pos_dev = decode_mode ? pos_dev : nullptr;
+    if (append_in_rope) { pq.rope_ring_k = Lw.ring_k; pq.rope_ring_v = Lw.ring_v; pq.rope_C = C; }
     if ((rc = gemm(pq)) != TTT_OK) return rc;
   }
   if (decode_mode) {
-    // one position per sequence, position on the device: append its K/V to the ring
-    // first, then attend over the window entirely from the ring
-    const int64_t work = sizeof(T) == 2 ? (int64_t)B * (d / 8) : (int64_t)B * d;
-    kv_append_kernel<T><<<nblk(work, 256), 256, 0, st>>>(qkv, 3 * d, d, 2 * d, 1, B, 0, d, Lw.ring_k, Lw.ring_v, C,
-                                                         pos_dev);
-    TTT_LAUNCHED();
     const float scale = 1.0f / sqrtf((float)hd);
     const dim3 dg(H, B);
     switch (hd) {
@@ -1056,7 +1057,7 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
   GemmParams p = gp(rows, d, d, o, d, false, Lw.Wo, d, false, xout, d, true, EPI_RESID);
   p.X = xin; p.ldx = d;
   if ((rc = gemm(p)) != TTT_OK) return rc;
-  if (commit) {
+  if (commit && !append_in_rope) {
     const int cnt = n > C ? C : n;
     const int64_t work = sizeof(T) == 2 ? (int64_t)B * cnt * (d / 8) : (int64_t)B * cnt * d;
     kv_append_kernel<T><<<nblk(work, 256), 256, 0, st>>>(qkv, 3 * d, d, 2 * d, n, B, q0, d, Lw.ring_k, Lw.ring_v,
