@@ -29,6 +29,7 @@ struct AttnParams {
   // backward
   const void* dO; int64_t lddo;
   float* Dsum;                         // [B][H][n] = rowsum(dO * O)
+  int dsum_in_dq;                      // 1: the tcgen05 dQ kernel forms Dsum itself (no separate pass)
   void* dQ; void* dK; void* dV; int64_t lddq;  // dQ/dK/dV rows [B*n][lddq]
 };
 

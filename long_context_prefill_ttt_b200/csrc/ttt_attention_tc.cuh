@@ -487,11 +487,36 @@ __global__ void __launch_bounds__(192, 1)
     const float sc = p.scale * 1.4426950408889634f;
     const int64_t si = ((int64_t)b * p.H + h) * p.n + i0 + r;
     const float nL = r < nq ? -p.lse[si] * 1.4426950408889634f : -INFINITY;  // exp2(s*sc - lse*log2e)
-    const float Dr = r < nq ? p.Dsum[si] : 0.f;
     const int64_t lo_key = P - p.window + 1;
     const uint32_t span = (uint32_t)(P - lo_key);
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
+    float Dr = 0.f;
+    if (p.dsum_in_dq) {
+      // D = rowsum(dO * O) of this row and head, from the staged dO tile and O; the
+      // dK/dV kernel that follows reads it from Dsum
+      ok = mbar_wait(q_full, 0, err, DEV_TIMEOUT_FULL);
+      if (ok && r < nq) {
+        const bf16* Orow = (const bf16*)p.O + ((int64_t)b * p.n + i0 + r) * p.ldo + h * HD;
+        float acc = 0.f;
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 a = *(const uint4*)(sm + Cf::OFF_DO + kb * Cf::BM * 128 + r * 128 + ((c ^ (r & 7)) << 4));
+            const uint4 o = *(const uint4*)(Orow + kb * 64 + c * 8);
+            const bf16* ae = reinterpret_cast<const bf16*>(&a);
+            const bf16* oe = reinterpret_cast<const bf16*>(&o);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc = fmaf(__bfloat162float(ae[e]), __bfloat162float(oe[e]), acc);
+          }
+        }
+        Dr = acc;
+        p.Dsum[si] = Dr;
+      }
+    } else {
+      Dr = r < nq ? p.Dsum[si] : 0.f;
+    }
+    for (int j = 0; j < ntiles && ok; ++j) {
       const int s = j & 1;
       const int64_t j0 = jt0 + (int64_t)j * Cf::BN;
       const bool need_mask = (j0 + Cf::BN - 1 > P0) || (j0 < Plast - p.window + 1);

@@ -240,6 +240,39 @@ template <int BN> struct TcCfg {
   static constexpr int TMEM_COLS = 2 * BN;
 };
 
+// GELU for the bf16 tensor-core epilogues. erf by the rational approximation of
+// Abramowitz & Stegun, Handbook of Mathematical Functions, eq. 7.1.28:
+// erf(x) = 1 - (1 + a1 x + ... + a6 x^6)^-16 for x >= 0 (|error| <= 3e-7 in exact
+// arithmetic, about 2e-6 in fp32 near 0), odd extension for x < 0. Branch-free, one
+// reciprocal; its error is far below the bf16 rounding of the outputs. (The fp32 path
+// keeps the library erff.)
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));  // rcp(+inf) = +0
+  return y;
+}
+__device__ __forceinline__ float erf_as7128(float x) {
+  const float ax = fabsf(x);
+  float t = fmaf(ax, 4.30638e-5f, 2.765672e-4f);
+  t = fmaf(ax, t, 1.520143e-4f);
+  t = fmaf(ax, t, 9.2705272e-3f);
+  t = fmaf(ax, t, 4.22820123e-2f);
+  t = fmaf(ax, t, 7.05230784e-2f);
+  t = fmaf(ax, t, 1.0f);
+  t *= t;
+  t *= t;
+  t *= t;
+  t *= t;  // t^16
+  return copysignf(1.0f - rcp_approx(t), x);
+}
+__device__ __forceinline__ float gelu_tc(float u) { return 0.5f * u * (1.0f + erf_as7128(u * 0.70710678118654752f)); }
+// d gelu / du = Phi(u) + u phi(u); exp(-u^2/2) as exp2 of (-u^2/2) log2(e)
+__device__ __forceinline__ float gelu_prime_tc(float u) {
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-0.72134752044448170f * u * u));
+  return 0.5f * (1.0f + erf_as7128(u * 0.70710678118654752f)) + u * e * 0.39894228040143268f;
+}
+
 // 32 consecutive accumulator columns of one row through the epilogue, vectorised.
 template <typename T>
 __device__ __forceinline__ void epi_row32(const GemmParams& p, int z, int m, int n, float* v) {
@@ -273,7 +306,7 @@ __device__ __forceinline__ void epi_row32(const GemmParams& p, int z, int m, int
                           pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
     }
 #pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = gelu_f(v[i]);
+    for (int i = 0; i < 32; ++i) v[i] = gelu_tc(v[i]);
     uint4* d = (uint4*)((T*)p.D + od);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -288,7 +321,7 @@ __device__ __forceinline__ void epi_row32(const GemmParams& p, int z, int m, int
       const bf16* u = reinterpret_cast<const bf16*>(&u4);
       float o[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) o[j] = v[8 * i + j] * gelu_prime_f(__bfloat162float(u[j]));
+      for (int j = 0; j < 8; ++j) o[j] = v[8 * i + j] * gelu_prime_tc(__bfloat162float(u[j]));
       d[i] = make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
                         pack_bf16x2(o[6], o[7]));
     }

@@ -98,15 +98,17 @@ template <typename T>
 static int attn_bwd(const AttnParams& ap, int engine, cudaStream_t st) {
   if (prime_kernel_attributes() != 0) return TTT_ERR_CUDA;
   const int64_t rows = (int64_t)ap.B * ap.n;
-  attn_bwd_prep_kernel<T><<<(unsigned)((rows * ap.H + 7) / 8), 256, 0, st>>>(ap);
   bool dq_done = false, dkv_done = false;
   if (sizeof(T) == 2 && engine == TTT_ENGINE_AUTO && attn_dq_tc_ok(ap)) {
     int* err = status_word();
     if (!err) return TTT_ERR_CUDA;
-    cudaError_t e = attn_bwd_dq_tc_launch(ap, st, err, &dq_done);
-    if (e == cudaSuccess && attn_dkv_tc_ok(ap)) e = attn_bwd_dkv_tc_launch(ap, st, err, &dkv_done);
+    AttnParams aq = ap;
+    aq.dsum_in_dq = 1;  // the tcgen05 dQ kernel forms D = rowsum(dO * O) and stores it for dK/dV
+    cudaError_t e = attn_bwd_dq_tc_launch(aq, st, err, &dq_done);
+    if (e == cudaSuccess && dq_done && attn_dkv_tc_ok(ap)) e = attn_bwd_dkv_tc_launch(ap, st, err, &dkv_done);
     if (e != cudaSuccess) return TTT_ERR_CUDA;
   }
+  if (!dq_done) attn_bwd_prep_kernel<T><<<(unsigned)((rows * ap.H + 7) / 8), 256, 0, st>>>(ap);
   if (dq_done && dkv_done) return TTT_OK;
   if (sizeof(T) == 2 && engine != TTT_ENGINE_SIMT && attn_mma_ok(ap)) {
     const cudaError_t e = ap.hd == 128 ? attn_bwd_mma_launch<128>(ap, st, !dq_done, !dkv_done)

@@ -515,16 +515,6 @@ __global__ void decode_record_kernel(const int32_t* chosen, const float* loss, i
 
 __global__ void decode_advance_kernel(int64_t* pos) { *pos += 1; }
 
-// Copy rows: dst[b][i][:] = src[b*src_bstride + (off + i)*ld ...] for i < n (fp32 rows of d).
-__global__ void gather_rows_kernel(const float* __restrict__ src, int64_t src_bstride, int64_t off, int n, int B,
-                                   int d, float* __restrict__ dst, int64_t dst_bstride, int64_t dst_off) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t per = (int64_t)n * d;
-  if (idx >= per * B) return;
-  const int b = (int)(idx / per);
-  const int64_t r = idx % per;
-  dst[b * dst_bstride + dst_off * d + r] = src[b * src_bstride + off * d + r];
-}
 
 // targets[b][i] = tok[b*tok_ld + off + i]
 __global__ void gather_tokens_kernel(const int32_t* __restrict__ tok, int64_t tok_ld, int64_t off, int n, int B,
@@ -533,6 +523,25 @@ __global__ void gather_tokens_kernel(const int32_t* __restrict__ tok, int64_t to
   if (idx >= n * B) return;
   const int b = idx / n, i = idx % n;
   out[b * out_bstride + out_off + i] = tok[(int64_t)b * tok_ld + off + i];
+}
+
+// One chunk's inputs, in one launch: rows [b][off, off+n) of the frozen stack's
+// output src [B][src rows][d] -> dst [B][n][d] (16-byte copies, d % 4 == 0), and the
+// chunk's targets tgt[b][i] = tok[b*tok_ld + tok_off + i].
+__global__ void gather_chunk_kernel(const float* __restrict__ src, int64_t src_bstride, int64_t off, int n, int B,
+                                    int d, float* __restrict__ dst, const int32_t* __restrict__ tok, int64_t tok_ld,
+                                    int64_t tok_off, int32_t* __restrict__ tgt) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t per = (int64_t)n * (d / 4);
+  if (idx < (int64_t)n * B) {
+    const int b = (int)(idx / n), i = (int)(idx % n);
+    tgt[idx] = tok[(int64_t)b * tok_ld + tok_off + i];
+  }
+  if (idx >= per * B) return;
+  const int b = (int)(idx / per);
+  const int64_t r = idx % per;
+  reinterpret_cast<float4*>(dst + (int64_t)b * n * d)[r] =
+      reinterpret_cast<const float4*>(src + b * src_bstride + off * d)[r];
 }
 
 }  // namespace ttt

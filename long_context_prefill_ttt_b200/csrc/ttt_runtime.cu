@@ -1185,17 +1185,22 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
     // dK, dV over current-chunk keys only (dS^T Q, P^T dO)
     prof.begin(st, PC_ATTN_BWD,
                2.0 * hd * H * (double)B * (2.0 * attn_pairs(cn, chunk_pos) + 2.0 * attn_pairs(cn, 0)), 0.0);
-    attn_bwd_prep_kernel<T><<<nblk((int64_t)rows * H, 8), 256, 0, st>>>(ap);
-    TTT_LAUNCHED();
-    // dQ and dK/dV: tcgen05 kernels where they apply, else mma.sync, else SIMT
+    // dQ and dK/dV: tcgen05 kernels where they apply (the dQ kernel forms D = rowsum(dO * O)
+    // itself), else a separate D pass and the mma.sync or SIMT kernels
     bool dq_done = false, dkv_done = false;
     if (is_bf16 && attn_dq_tc_ok(ap)) {
+      ap.dsum_in_dq = 1;
       cudaError_t e = attn_bwd_dq_tc_launch(ap, st, dev_err, &dq_done);
-      if (e == cudaSuccess && attn_dkv_tc_ok(ap)) e = attn_bwd_dkv_tc_launch(ap, st, dev_err, &dkv_done);
+      ap.dsum_in_dq = 0;
+      if (e == cudaSuccess && dq_done && attn_dkv_tc_ok(ap)) e = attn_bwd_dkv_tc_launch(ap, st, dev_err, &dkv_done);
       if (e != cudaSuccess) {
         poisoned = true;
         return fail(this, TTT_ERR_CUDA, std::string("attention backward: ") + cudaGetErrorString(e));
       }
+    }
+    if (!dq_done) {
+      attn_bwd_prep_kernel<T><<<nblk((int64_t)rows * H, 8), 256, 0, st>>>(ap);
+      TTT_LAUNCHED();
     }
     if (!(dq_done && dkv_done)) {
       if (is_bf16 && attn_mma_ok(ap)) {
@@ -1312,10 +1317,8 @@ template <typename T> int Engine<T>::prefill(const int32_t* tokens, int64_t T_, 
     }
     for (int c0 = 0; c0 < n; c0 += bsz) {
       const int cn = (n - c0) < bsz ? (n - c0) : bsz;
-      gather_rows_kernel<<<nblk((int64_t)B * cn * d, 256), 256, 0, st>>>(xs, (int64_t)n * d, c0, cn, B, d, tin,
-                                                                        (int64_t)cn * d, 0);
-      TTT_LAUNCHED();
-      gather_tokens_kernel<<<nblk(B * cn, 256), 256, 0, st>>>(tok_dev, ld, s0 + c0 + 1, cn, B, tgt, cn, 0);
+      gather_chunk_kernel<<<nblk((int64_t)B * cn * (d / 4), 256), 256, 0, st>>>(xs, (int64_t)n * d, c0, cn, B, d, tin,
+                                                                                tok_dev, ld, s0 + c0 + 1, tgt);
       TTT_LAUNCHED();
       const bool full = cn == bsz;
       if ((rc = ttt_step(tin, tgt, cn, P0 + c0, lout, T_, s0 + c0, full, true)) != TTT_OK) return rc;
