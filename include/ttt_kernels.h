@@ -28,8 +28,9 @@ extern "C" {
 enum { TTT_EPI_STORE = 0, TTT_EPI_RESID = 1, TTT_EPI_GELU = 2, TTT_EPI_DGELU = 3, TTT_EPI_SGD = 4 };
 
 /* Engines: 0 = automatic: GEMMs on tcgen05 tensor cores for bf16 shapes with N % 128 == 0 and
- * K % 64 == 0 (pairs of CTAs on two SMs sharing 256-row tiles when M > 128, one CTA per
- * 128-row tile otherwise); attention forward on tcgen05 for bf16 with head dim 64 or 128,
+ * K % 64 == 0 (pairs of CTAs on two SMs sharing 256-row tiles for large products; for thin
+ * products whose 128 x 256 tiles fill at most half the SMs, pairs of CTAs splitting K of one
+ * 128 x 256 tile, summed in a fixed order; one CTA per 128-row tile otherwise); attention forward on tcgen05 for bf16 with head dim 64 or 128,
  * q0 % 128 == 0 and C % 128 == 0; attention on warp-level tensor cores (mma.sync m16n8k16)
  * for bf16 with head dim 64 or 128 and q0 % 64 == 0 (and C % 64 == 0); otherwise, and for
  * fp32, SIMT FFMA kernels. 1 = SIMT only. 2 = attention on the mma.sync kernels. 3 = GEMMs

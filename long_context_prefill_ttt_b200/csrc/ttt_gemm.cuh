@@ -273,9 +273,35 @@ __device__ __forceinline__ float gelu_prime_tc(float u) {
   return 0.5f * (1.0f + erf_as7128(u * 0.70710678118654752f)) + u * e * 0.39894228040143268f;
 }
 
-// 32 consecutive accumulator columns of one row through the epilogue, vectorised.
+// Global inputs of the epilogue for 32 columns of one row, as raw 16-byte words: the
+// fp32 residual (EPI_RESID) or fp32 master weights (EPI_SGD) in all eight, the bf16
+// pre-activations (EPI_DGELU) in the first four. They are fetched one 32-column chunk
+// ahead of their use (the first chunk before the accumulator is waited for), so each
+// thread has a whole chunk of loads in flight instead of one load per store.
+struct EpiIn {
+  uint4 w[8];
+};
+__device__ __forceinline__ void epi_fetch32(const GemmParams& p, int z, int m, int n, EpiIn& in) {
+  if (m >= p.M) return;
+  if (p.epi == EPI_RESID) {
+    const uint4* x = (const uint4*)((const float*)p.X + (int64_t)z * p.sX + (int64_t)m * p.ldx + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) in.w[i] = x[i];
+  } else if (p.epi == EPI_SGD) {
+    const uint4* w = (const uint4*)((const float*)p.D + (int64_t)z * p.sD + (int64_t)m * p.ldd + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) in.w[i] = w[i];
+  } else if (p.epi == EPI_DGELU) {
+    const uint4* x = (const uint4*)((const bf16*)p.X + (int64_t)z * p.sX + (int64_t)m * p.ldx + n);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) in.w[i] = x[i];
+  }
+}
+
+// 32 consecutive accumulator columns of one row through the epilogue, vectorised;
+// `in` holds what epi_fetch32 read for the same columns.
 template <typename T>
-__device__ __forceinline__ void epi_row32(const GemmParams& p, int z, int m, int n, float* v) {
+__device__ __forceinline__ void epi_row32(const GemmParams& p, int z, int m, int n, float* v, const EpiIn& in) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] *= p.alpha;
   const int64_t od = (int64_t)z * p.sD + (int64_t)m * p.ldd + n;
@@ -290,11 +316,10 @@ __device__ __forceinline__ void epi_row32(const GemmParams& p, int z, int m, int
       d[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
                         pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
   } else if (p.epi == EPI_RESID) {
-    const float4* x = (const float4*)((const float*)p.X + (int64_t)z * p.sX + (int64_t)m * p.ldx + n);
     float4* d = (float4*)((float*)p.D + od);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float4 r = x[i];
+      const float4 r = *reinterpret_cast<const float4*>(&in.w[i]);
       d[i] = make_float4(v[4 * i] + r.x, v[4 * i + 1] + r.y, v[4 * i + 2] + r.z, v[4 * i + 3] + r.w);
     }
   } else if (p.epi == EPI_GELU) {
@@ -313,12 +338,10 @@ __device__ __forceinline__ void epi_row32(const GemmParams& p, int z, int m, int
       d[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
                         pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
   } else if (p.epi == EPI_DGELU) {
-    const uint4* x = (const uint4*)((const T*)p.X + (int64_t)z * p.sX + (int64_t)m * p.ldx + n);
     uint4* d = (uint4*)((T*)p.D + od);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      uint4 u4 = x[i];
-      const bf16* u = reinterpret_cast<const bf16*>(&u4);
+      const bf16* u = reinterpret_cast<const bf16*>(&in.w[i]);
       float o[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) o[j] = v[8 * i + j] * gelu_prime_tc(__bfloat162float(u[j]));
@@ -330,7 +353,7 @@ __device__ __forceinline__ void epi_row32(const GemmParams& p, int z, int m, int
     float nw[32];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      float4 c = w[i];
+      float4 c = *reinterpret_cast<const float4*>(&in.w[i]);
       c.x += v[4 * i]; c.y += v[4 * i + 1]; c.z += v[4 * i + 2]; c.w += v[4 * i + 3];
       w[i] = c;
       nw[4 * i] = c.x; nw[4 * i + 1] = c.y; nw[4 * i + 2] = c.z; nw[4 * i + 3] = c.w;
@@ -381,13 +404,28 @@ __device__ __forceinline__ void epi_ce32(const GemmParams& p, int m, int n, floa
   cm = M;
 }
 
-// Epilogue of one accumulator tile for one epilogue warp: the warp reads its TMEM
-// lane quarter (one output row per thread, row m) over its half of the tile's
-// columns [c_first*32, c_first*32 + BN/2), calls release() once those columns are
-// read (the accumulator may then be overwritten), and applies the epilogue.
-template <int BN, typename Release>
-__device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t taddr, int z, int m, int n0, int c_first,
-                                              Release release) {
+// Epilogue of one accumulator tile for one epilogue warp: the warp fetches the global
+// inputs of its first 32 columns, waits for the accumulator (wait_acc() false: the
+// wait timed out), then reads its TMEM lane quarter (one output row per thread, row m)
+// over its half of the tile's columns [c_first*32, c_first*32 + BN/2), calls release()
+// once those columns are read (the accumulator may then be overwritten), and applies
+// the epilogue, each chunk's inputs fetched while the previous chunk is stored.
+// Split-K partial tile in shared memory: fp32 [128 rows][BN], the 16-byte word q of a
+// row stored at q ^ (row & 7), so that eight consecutive rows writing or reading the
+// same columns hit distinct banks.
+template <int BN>
+__device__ __forceinline__ uint32_t part_addr(uint32_t base, int row, int q) {
+  return base + (uint32_t)(row * BN + ((q ^ (row & 7)) << 2)) * 4u;
+}
+
+// part: shared address of a split-K partial tile to add to the accumulator (0: none).
+template <int BN, typename Wait, typename Release>
+__device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint32_t taddr, int z, int m, int n0, int c_first,
+                                              Wait wait_acc, Release release, uint32_t part = 0, int row = 0) {
+  EpiIn nxt;
+  epi_fetch32(p, z, m, n0 + c_first * 32, nxt);
+  if (!wait_acc()) return false;
+  tc_fence_after();
   const int tgt = (p.epi == EPI_CE && m < p.M) ? p.ce_tgt[m] : -1;
   float cm = -INFINITY, cs = 0.f;
 #pragma unroll 1
@@ -399,6 +437,18 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tadd
       __syncwarp();
       release();
     }
+    if (part) {  // acc = acc(first K half) + partial(second K half), in this order
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float4 q;
+        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(q.x), "=f"(q.y), "=f"(q.z), "=f"(q.w)
+                     : "r"(part_addr<BN>(part, row, c * 8 + i)));
+        v[4 * i] += q.x; v[4 * i + 1] += q.y; v[4 * i + 2] += q.z; v[4 * i + 3] += q.w;
+      }
+    }
+    const EpiIn cur = nxt;
+    if (c + 1 < c_first + BN / 64) epi_fetch32(p, z, m, n0 + (c + 1) * 32, nxt);
     if (m < p.M) {
       if (p.epi == EPI_CE) {
         epi_ce32(p, m, n0 + c * 32, v, tgt, cm, cs);
@@ -408,10 +458,11 @@ __device__ __forceinline__ void epilogue_tile(const GemmParams& p, uint32_t tadd
           cs = 0.f;
         }
       } else {
-        epi_row32<bf16>(p, z, m, n0 + c * 32, v);
+        epi_row32<bf16>(p, z, m, n0 + c * 32, v, cur);
       }
     }
   }
+  return true;
 }
 
 // Persistent warp-specialised tcgen05 GEMM. Requirements (checked on the host):
@@ -541,12 +592,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int n0 = (p.m_fast ? r / m_tiles : r % n_tiles) * BN;
       const int acc = lt & 1;
       const uint32_t use = lt >> 1;
-      if (!mbar_wait(&acc_full[acc], use & 1, err, DEV_TIMEOUT_ACC)) break;
-      tc_fence_after();
       const uint32_t taddr = tmem_base + acc * BN + ((uint32_t)(quarter * 32) << 16);
-      epilogue_tile<BN>(p, taddr, z, m0 + row_in_tile, n0, c_first, [&] {
-        if (elect_lane0()) mbar_arrive(&acc_empty[acc]);
-      });
+      if (!epilogue_tile<BN>(
+              p, taddr, z, m0 + row_in_tile, n0, c_first,
+              [&] { return mbar_wait(&acc_full[acc], use & 1, err, DEV_TIMEOUT_ACC); },
+              [&] {
+                if (elect_lane0()) mbar_arrive(&acc_empty[acc]);
+              }))
+        break;
     }
   }
   tc_fence_before();
@@ -554,6 +607,161 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ============================================================== tcgen05 engine, K split over a CTA pair
+// For the thin products of an adaptive step (1024 rows, N = 2048: 64 tiles of 128 x 256
+// for 148 SMs), a cluster of two CTAs computes one 128 x BN tile: CTA r accumulates
+// k blocks [r kb/2, (r+1) kb/2) in its own TMEM. Once CTA 0's MMAs have completed its
+// operand stages are idle; CTA 1 then writes its partial accumulator there over
+// distributed shared memory, and CTA 0 adds it to its own before the epilogue
+// (acc = acc_0 + acc_1, always in this order: deterministic). The tile count doubles
+// at the operand bytes per FLOP of a 128 x BN tile, and no global workspace is used.
+// One tile per cluster: the grid is exactly two CTAs per tile.
+template <int BN, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    gemm_tck_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmB2, const GemmParams p, int* err) {
+  using C = TcCfg<BN>;
+  static_assert(TC_BM * BN * 4 <= C::STAGES * C::STAGE_BYTES, "partial tile must fit the operand stages");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = (uint64_t*)(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = bars;                       // [STAGES]
+  uint64_t* empty = bars + C::STAGES;          // [STAGES]
+  uint64_t* acc_full = bars + 2 * C::STAGES;   // this CTA's MMAs are complete
+  uint64_t* part_free = acc_full + 1;          // CTA 1: CTA 0's stages may be overwritten
+  uint64_t* part_full = acc_full + 2;          // CTA 0: CTA 1's partial is in place (epilogue threads)
+  uint32_t* tmem_slot = (uint32_t*)(acc_full + 3);
+
+  const int warp = threadIdx.x >> 5;
+  const uint32_t rank = cluster_ctarank();
+  const int m_tiles = (p.M + TC_BM - 1) / TC_BM;
+  const int n_tiles = p.N / BN;
+  const int tiles_per_batch = m_tiles * n_tiles;
+  const int tile = (int)cluster_id_x();
+  const int z = tile / tiles_per_batch;
+  const int r = tile % tiles_per_batch;
+  const int m0 = (p.m_fast ? r % m_tiles : r / n_tiles) * TC_BM;
+  const int n0 = (p.m_fast ? r / m_tiles : r % n_tiles) * BN;
+  const int kb_one = p.K / TC_BK;
+  const int k_half = (p.B2 ? 2 * kb_one : kb_one) / 2;
+  const int kb_begin = (int)rank * k_half;
+  const int zb_scale = p.sB ? 1 : 0;
+  const int zb2_scale = p.sB2 ? 1 : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(acc_full, 1);
+    mbar_init(part_free, 1);
+    mbar_init(part_full, TC_EPI_WARPS * 32);
+    fence_mbar_init();
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+    if (p.B2) prefetch_tmap(&tmB2);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  cluster_sync();  // both CTAs' barriers are initialised before either arrives remotely
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+  pdl_trigger();
+
+  if (warp == 0) {
+    if (elect_lane0()) {
+      for (int i = 0; i < k_half; ++i) {
+        const int kb = kb_begin + i;
+        const int s = i % C::STAGES;
+        const uint32_t round = i / C::STAGES;
+        if (!mbar_wait(&empty[s], (round & 1) ^ 1, err, DEV_TIMEOUT_EMPTY)) break;
+        uint8_t* sa = smem + s * C::STAGE_BYTES;
+        uint8_t* sb = sa + C::A_BYTES;
+        mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+        const bool second = kb >= kb_one;
+        const int k0 = (second ? kb - kb_one : kb) * TC_BK;
+        const CUtensorMap* mb = second ? &tmB2 : &tmB;
+        const int zb = z * (second ? zb2_scale : zb_scale);
+        if (A_MN) {
+          tma_load_3d(sa, &tmA, &full[s], m0, k0, z);
+          tma_load_3d(sa + 8192, &tmA, &full[s], m0 + 64, k0, z);
+        } else {
+          tma_load_3d(sa, &tmA, &full[s], k0, m0, z);
+        }
+        if (B_MN) {
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j) tma_load_3d(sb + j * 8192, mb, &full[s], n0 + 64 * j, k0, zb);
+        } else {
+          tma_load_3d(sb, mb, &full[s], k0, n0, zb);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (elect_lane0()) {
+      constexpr uint32_t idesc = idesc_bf16_f32(TC_BM, BN, A_MN, B_MN);
+      bool ok = true;
+      for (int i = 0; i < k_half; ++i) {
+        const int s = i % C::STAGES;
+        const uint32_t round = i / C::STAGES;
+        if (!mbar_wait(&full[s], round & 1, err, DEV_TIMEOUT_FULL)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + s * C::STAGE_BYTES);
+        const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < TC_BK / 16; ++kk) {
+          const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+                                   : smem_desc_sw128(sa + kk * 32, 16, 1024);
+          const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                   : smem_desc_sw128(sb + kk * 32, 16, 1024);
+          tc_mma_f16(tmem_base, ad, bd, idesc, (i | kk) ? 1u : 0u);
+        }
+        tc_commit(&empty[s]);
+      }
+      if (ok) tc_commit(acc_full);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int c_first = (warp >= 6 ? 1 : 0) * (BN / 64);
+    const int row = quarter * 32 + (threadIdx.x & 31);
+    const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t part = smem_u32(smem);
+    if (rank == 1) {
+      // partial accumulator -> CTA 0's stage buffers, once CTA 0 has released them
+      if (mbar_wait(acc_full, 0, err, DEV_TIMEOUT_ACC) && mbar_wait_cluster(part_free, 0, err, DEV_TIMEOUT_ACC)) {
+        tc_fence_after();
+        const uint32_t peer = mapa_shared(part, 0);
+#pragma unroll 1
+        for (int c = c_first; c < c_first + BN / 64; ++c) {
+          float v[32];
+          tmem_ld32(taddr + c * 32, v);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            st_cluster_v4(part_addr<BN>(peer, row, c * 8 + i), v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+        }
+        mbar_arrive_cluster(mapa_shared(smem_u32(part_full), 0));
+      }
+    } else {
+      epilogue_tile<BN>(
+          p, taddr, z, m0 + row, n0, c_first,
+          [&] {
+            if (!mbar_wait(acc_full, 0, err, DEV_TIMEOUT_ACC)) return false;
+            if (warp == 2 && elect_lane0()) mbar_arrive_cluster(mapa_shared(smem_u32(part_free), 1));
+            return mbar_wait_cluster(part_full, 0, err, DEV_TIMEOUT_ACC);
+          },
+          [] {}, part, row);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // neither CTA leaves while the peer may still write to or arrive on it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, BN);
   }
 }
 
@@ -707,12 +915,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int n0 = (p.m_fast ? r / m_tiles : r % n_tiles) * BN;
       const int acc = lt & 1;
       const uint32_t use = lt >> 1;
-      if (!mbar_wait(&acc_full[acc], use & 1, err, DEV_TIMEOUT_ACC)) break;
-      tc_fence_after();
       const uint32_t taddr = tmem_base + acc * BN + ((uint32_t)(quarter * 32) << 16);
-      epilogue_tile<BN>(p, taddr, z, m0 + row_in_tile, n0, c_first, [&] {
-        if (elect_lane0()) mbar_arrive_cluster(acc_empty0 + 8u * acc);
-      });
+      if (!epilogue_tile<BN>(
+              p, taddr, z, m0 + row_in_tile, n0, c_first,
+              [&] { return mbar_wait(&acc_full[acc], use & 1, err, DEV_TIMEOUT_ACC); },
+              [&] {
+                if (elect_lane0()) mbar_arrive_cluster(acc_empty0 + 8u * acc);
+              }))
+        break;
     }
   }
   tc_fence_before();

@@ -177,6 +177,59 @@ template <int BN, bool AM, bool BM> static int pair_capacity() {
   return cap;
 }
 
+// Clusters of the K-split kernel that can be resident at once (0: cannot be placed).
+template <int BN, bool AM, bool BM> static int tck_capacity() {
+  static int cap = -1;
+  if (cap < 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(TC_THREADS);
+    cfg.dynamicSmemBytes = TcCfg<BN>::SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tck_kernel<BN, AM, BM>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    cap = n;
+  }
+  return cap;
+}
+
+// K split over a CTA pair, one 128 x BN tile per cluster (gemm_tck_kernel). The caller
+// has checked that the k-block count (doubled with B2) is even.
+template <int BN, bool AM, bool BM>
+static cudaError_t launch_tck(const GemmParams& p, cudaStream_t st, int* err, bool* ok) {
+  CUtensorMap ta, tb, tb2;
+  *ok = tck_capacity<BN, AM, BM>() > 0 && make_operand_map(&ta, p.A, p.M, p.K, p.lda, p.batch, p.sA, AM, TC_BM) &&
+        make_operand_map(&tb, p.B, p.N, p.K, p.ldb, p.batch, p.sB, BM, BN);
+  if (*ok && p.B2) *ok = make_operand_map(&tb2, p.B2, p.N, p.K, p.ldb, p.batch, p.sB2, BM, BN);
+  else tb2 = tb;
+  if (!*ok) return cudaSuccess;
+  const int tiles = ((p.M + TC_BM - 1) / TC_BM) * (p.N / BN) * p.batch;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * tiles);
+  cfg.blockDim = dim3(TC_THREADS);
+  cfg.dynamicSmemBytes = TcCfg<BN>::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, gemm_tck_kernel<BN, AM, BM>, ta, tb, tb2, p, err);
+}
+
 template <int BN, bool AM, bool BM>
 static cudaError_t launch_tc2(const GemmParams& p, cudaStream_t st, int* err, bool* ok) {
   CUtensorMap ta, tb, tb2;
@@ -291,6 +344,9 @@ template <int BN, bool AM, bool BM> static cudaError_t tc_attr() {
   const cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, AM, BM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              TcCfg<BN>::SMEM);
   if (e != cudaSuccess) return e;
+  const cudaError_t e2 = cudaFuncSetAttribute(gemm_tck_kernel<BN, AM, BM>,
+                                              cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<BN>::SMEM);
+  if (e2 != cudaSuccess) return e2;
   return cudaFuncSetAttribute(gemm_tc2_kernel<BN, AM, BM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               Tc2Cfg<BN>::SMEM);
 }
@@ -319,6 +375,7 @@ int prime_kernel_attributes() {
   // resident-pair counts of the paired GEMMs, queried now rather than at a first launch
   pair_capacity<128, false, false>(); pair_capacity<256, false, false>(); pair_capacity<128, false, true>();
   pair_capacity<256, false, true>();  pair_capacity<128, true, true>();   pair_capacity<256, true, true>();
+  tck_capacity<256, false, false>();  tck_capacity<256, false, true>();   tck_capacity<256, true, true>();
   done = 1;
   return 0;
 }
@@ -351,9 +408,10 @@ bool gemm_uses_tc(const GemmParams& p, int elem_is_bf16) {
   return !skinny_ok(p, elem_is_bf16) && tc_ok(p, elem_is_bf16);
 }
 
-// Returns 0 on success, or a cudaError_t value. engine: GEMM_AUTO (tcgen05 CTA pairs
-// for M > 128, single-CTA tcgen05 otherwise, SIMT where tensor cores do not fit),
-// GEMM_SIMT, or GEMM_TC1 (no CTA pairs).
+// Returns 0 on success, or a cudaError_t value. engine: GEMM_AUTO (tcgen05: CTA pairs
+// for large products, the K split over CTA pairs for thin ones, single-CTA tiles
+// otherwise; SIMT where tensor cores do not fit), GEMM_SIMT, or GEMM_TC1 (single-CTA
+// tiles only).
 int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err, int num_sms, int engine) {
   if (p.M <= 0 || p.N <= 0 || p.K <= 0 || p.batch <= 0) return 0;
   const bool force_simt = engine == GEMM_SIMT;
@@ -410,6 +468,27 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
           e = w256 ? launch_tc2<256, true, true>(pt, st, err, &ok) : launch_tc2<128, true, true>(pt, st, err, &ok);
         if (e != cudaSuccess) return (int)e;
       }
+    }
+    if (ok) {
+      if (p.epi == EPI_QKV_ROPE) {
+        return (int)rope_launch<bf16>((bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd,
+                                      p.rope_lo, p.rope_hi, 0, p.rope_pos_dev, st, p.rope_ring_k, p.rope_ring_v, p.rope_C);
+      }
+      return 0;
+    }
+    // K split over CTA pairs: thin products whose 128 x 256 tiles fill at most half the
+    // SMs (the N = 2048 products of an adaptive step: 64 tiles) run each tile on two SMs
+    // with 256-wide tiles instead of 128-wide tiles on one. The hand-over of the partial
+    // tile costs a few microseconds, so only long K pays: measured on B200 at 1024 x 2048,
+    // K = 8192 (W_init + dW, 4096 each) 47 -> 43 us, K = 6144 36 -> 34 us, K = 32000
+    // 152 -> 113 us, but K = 4096 28 -> 32 us and K = 2048 22 -> 28 us.
+    const int t256 = (p.N % 256 == 0) ? m_tiles * (p.N / 256) * p.batch : 0;
+    const int kbt = (p.K / TC_BK) * (p.B2 ? 2 : 1);
+    if (engine != GEMM_TC1 && p.epi != EPI_CE && t256 > 0 && 2 * t256 <= num_sms && kbt % 2 == 0 && kbt >= 96) {
+      if (!p.a_mn && !p.b_mn) e = launch_tck<256, false, false>(pt, st, err, &ok);
+      else if (!p.a_mn && p.b_mn) e = launch_tck<256, false, true>(pt, st, err, &ok);
+      else e = launch_tck<256, true, true>(pt, st, err, &ok);
+      if (e != cudaSuccess) return (int)e;
     }
     if (ok) {
       if (p.epi == EPI_QKV_ROPE) {

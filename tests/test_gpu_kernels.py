@@ -30,8 +30,9 @@ def _store(x_log, mn):
     return x_log.transpose(1, 2).contiguous() if mn else x_log.contiguous()
 
 
-# engine 0 runs M > 128 on CTA pairs (256-row tiles, ragged M tails and batches included),
-# engine 3 on single-CTA tiles, engine 1 on SIMT
+# engine 0 picks CTA pairs for large products, the K split over CTA pairs where 128 x 256
+# tiles fill at most half the SMs and K is long (test_gemm_k_split_pairs), single-CTA
+# tiles otherwise; engine 3 runs single-CTA tiles only, engine 1 SIMT
 SHAPES = [(256, 256, 128, 1), (200, 384, 192, 2), (1024, 512, 64, 1), (128, 2048, 256, 1), (384, 128, 1024, 3),
           (1024, 2048, 512, 1), (640, 4096, 128, 1), (100, 256, 64, 2)]
 
@@ -124,6 +125,71 @@ def test_gemm_epilogues(T, engine):
     T.ttt_k_status()
     assert (W.double() - (W0 - 0.05 * acc)).abs().max().item() < 1e-5
     assert torch.equal(Sh, W.to(torch.bfloat16))
+
+
+# Thin products that engine 0 runs with K split over a CTA pair (two SMs per 128 x 256
+# tile, the second half's partial added in the first CTA's shared memory): layouts, a
+# ragged M tail with batches, and double-K (B + B2: the first CTA takes the B half, the
+# second the B2 half), with an odd k-block count per operand.
+K_SPLIT_CASES = [(1024, 2048, 8192, 1, 0, 0, False), (1024, 2048, 6144, 1, 0, 1, False),
+                 (1024, 2048, 6144, 1, 1, 1, False), (300, 512, 6400, 2, 0, 0, False),
+                 (1024, 2048, 3136, 1, 0, 0, True), (256, 768, 4160, 1, 0, 1, True)]
+
+
+@pytest.mark.parametrize("M,N,K,batch,a_mn,b_mn,b2", K_SPLIT_CASES)
+def test_gemm_k_split_pairs(T, M, N, K, batch, a_mn, b_mn, b2):
+    A = _rand((batch, M, K), torch.bfloat16, 31, 0.5)
+    B = _rand((batch, N, K), torch.bfloat16, 32, 0.5)
+    B2 = _rand((batch, N, K), torch.bfloat16, 33, 0.05) if b2 else None
+    Bt = B.double() + (B2.double() if b2 else 0)
+    acc = A.double() @ Bt.transpose(1, 2)
+    kw = dict(batch=batch, sA=M * K, a_mn=a_mn, sB=N * K, b_mn=b_mn, sD=M * N)
+    if b2:
+        kw.update(B2=_store(B2, b_mn), sB2=N * K)
+    As, Bs = _store(A, a_mn), _store(B, b_mn)
+    scale = acc.abs().max().item()
+    # fp32 store, twice: the fixed order of the two halves makes the result reproducible
+    D1 = torch.full((batch, M, N), float("nan"), dtype=torch.float32, device="cuda")
+    D2 = torch.full_like(D1, float("nan"))
+    T.ttt_k_gemm(As, Bs, D1, M, N, K, **kw)
+    T.ttt_k_gemm(As, Bs, D2, M, N, K, **kw)
+    T.ttt_k_status()
+    assert (D1.double() - acc).abs().max().item() < 4e-6 * scale
+    assert torch.equal(D1, D2)
+    # residual in place
+    R = _rand((batch, M, N), torch.float32, 34)
+    D = R.clone()
+    T.ttt_k_gemm(As, Bs, D, M, N, K, X=D, ldx=N, sX=M * N, epi=T.EPI_RESID, **kw)
+    T.ttt_k_status()
+    assert (D.double() - (acc + R.double())).abs().max().item() < 4e-6 * scale + 1e-5
+    # GELU pair (bf16)
+    U = torch.empty((batch, M, N), dtype=torch.bfloat16, device="cuda")
+    G = torch.empty_like(U)
+    T.ttt_k_gemm(As, Bs, G, M, N, K, Y=U, ldy=N, sY=M * N, epi=T.EPI_GELU, **kw)
+    T.ttt_k_status()
+    assert torch.allclose(U.double(), acc, rtol=1e-2, atol=1e-2 * scale)
+    assert torch.allclose(G.double(), torch.nn.functional.gelu(acc), rtol=1e-2, atol=1e-2 * scale)
+    # GELU' gate (bf16)
+    Xu = _rand((batch, M, N), torch.bfloat16, 35)
+    Dg = torch.empty_like(U)
+    T.ttt_k_gemm(As, Bs, Dg, M, N, K, X=Xu, ldx=N, sX=M * N, epi=T.EPI_DGELU, **kw)
+    T.ttt_k_status()
+    x = Xu.double()
+    gp = 0.5 * (1 + torch.erf(x / math.sqrt(2))) + x * torch.exp(-0.5 * x * x) / math.sqrt(2 * math.pi)
+    assert torch.allclose(Dg.double(), acc * gp, rtol=2e-2, atol=2e-2 * scale)
+    # fused SGD on fp32 master weights with the bf16 copy
+    W = _rand((batch, M, N), torch.float32, 36)
+    W0 = W.double().clone()
+    Sh = torch.empty_like(U)
+    T.ttt_k_gemm(As, Bs, W, M, N, K, Y=Sh, ldy=N, sY=M * N, alpha=-0.01, epi=T.EPI_SGD, **kw)
+    T.ttt_k_status()
+    assert (W.double() - (W0 - 0.01 * acc)).abs().max().item() < 4e-6 * 0.01 * scale + 1e-6
+    assert torch.equal(Sh, W.to(torch.bfloat16))
+    # the single-CTA engine agrees to fp32 rounding of the two summation orders
+    D3 = torch.empty_like(D1)
+    T.ttt_k_gemm(As, Bs, D3, M, N, K, engine=3, **kw)
+    T.ttt_k_status()
+    assert (D3.double() - D1.double()).abs().max().item() < 4e-6 * scale
 
 
 def _attn_reference(qkv, ring_k, ring_v, B, H, hd, n, q0, window, C):
