@@ -148,20 +148,22 @@ def test_gemm_k_split_pairs(T, M, N, K, batch, a_mn, b_mn, b2):
         kw.update(B2=_store(B2, b_mn), sB2=N * K)
     As, Bs = _store(A, a_mn), _store(B, b_mn)
     scale = acc.abs().max().item()
+    # the tensor cores' fp32 accumulation error grows about linearly with the K steps
+    tol = 2e-6 * max(1.0, K * (2 if b2 else 1) / 1024)
     # fp32 store, twice: the fixed order of the two halves makes the result reproducible
     D1 = torch.full((batch, M, N), float("nan"), dtype=torch.float32, device="cuda")
     D2 = torch.full_like(D1, float("nan"))
     T.ttt_k_gemm(As, Bs, D1, M, N, K, **kw)
     T.ttt_k_gemm(As, Bs, D2, M, N, K, **kw)
     T.ttt_k_status()
-    assert (D1.double() - acc).abs().max().item() < 4e-6 * scale
+    assert (D1.double() - acc).abs().max().item() < tol * scale
     assert torch.equal(D1, D2)
     # residual in place
     R = _rand((batch, M, N), torch.float32, 34)
     D = R.clone()
     T.ttt_k_gemm(As, Bs, D, M, N, K, X=D, ldx=N, sX=M * N, epi=T.EPI_RESID, **kw)
     T.ttt_k_status()
-    assert (D.double() - (acc + R.double())).abs().max().item() < 4e-6 * scale + 1e-5
+    assert (D.double() - (acc + R.double())).abs().max().item() < tol * scale + 1e-5
     # GELU pair (bf16)
     U = torch.empty((batch, M, N), dtype=torch.bfloat16, device="cuda")
     G = torch.empty_like(U)
@@ -183,13 +185,13 @@ def test_gemm_k_split_pairs(T, M, N, K, batch, a_mn, b_mn, b2):
     Sh = torch.empty_like(U)
     T.ttt_k_gemm(As, Bs, W, M, N, K, Y=Sh, ldy=N, sY=M * N, alpha=-0.01, epi=T.EPI_SGD, **kw)
     T.ttt_k_status()
-    assert (W.double() - (W0 - 0.01 * acc)).abs().max().item() < 4e-6 * 0.01 * scale + 1e-6
+    assert (W.double() - (W0 - 0.01 * acc)).abs().max().item() < tol * 0.01 * scale + 1e-6
     assert torch.equal(Sh, W.to(torch.bfloat16))
     # the single-CTA engine agrees to fp32 rounding of the two summation orders
     D3 = torch.empty_like(D1)
     T.ttt_k_gemm(As, Bs, D3, M, N, K, engine=3, **kw)
     T.ttt_k_status()
-    assert (D3.double() - D1.double()).abs().max().item() < 4e-6 * scale
+    assert (D3.double() - D1.double()).abs().max().item() < tol * scale
 
 
 def _attn_reference(qkv, ring_k, ring_v, B, H, hd, n, q0, window, C):
