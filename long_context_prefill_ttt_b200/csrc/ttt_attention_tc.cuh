@@ -17,7 +17,10 @@
 //              row is rescaled in TMEM after the previous P·V has completed.
 //              Exponents stay below 2^8, so bf16 P and fp32 sums stay exact
 //              enough, and O and l always share the same reference maximum.
-// TMEM: S0 columns [0,128), S1 [128,256), O [256, 256+HD); 512 allocated.
+// The softmax warps first copy their rows of Q from shared memory into TMEM, where the
+// S MMAs take them as the A operand (the MMA then reads only the K tile from shared
+// memory).
+// TMEM: S0 columns [0,128), S1 [128,256), O [256, 256+HD), Q [384, 384+HD/2); 512 allocated.
 // Every mbarrier wait is time-bounded and records an error instead of hanging.
 #pragma once
 
@@ -39,6 +42,7 @@ template <int HD> struct AttnTcCfg {
   static constexpr int OFF_BAR = OFF_P0 + 2 * PB;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr uint32_t S_COL = 0, O_COL = 256;
+  static constexpr uint32_t Q_COL = 384;  // Q as the A operand of S, copied once into TMEM
 };
 
 __device__ __forceinline__ bool warp_any(bool v) { return __any_sync(0xffffffffu, v); }
@@ -67,7 +71,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* p_full = bars + 17;    // [2]
   uint64_t* pv_done = bars + 19;   // [2]
   uint64_t* o_done = bars + 21;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 22);
+  uint64_t* qt_full = bars + 22;   // Q is in TMEM (4 warps)
+  uint32_t* tmem_slot = (uint32_t*)(bars + 23);
 
   const int warp = threadIdx.x >> 5;
   const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -90,6 +95,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&p_full[s], 4);  mbar_init(&pv_done[s], 1);
     }
     mbar_init(o_done, 1);
+    mbar_init(qt_full, 4);
     fence_mbar_init();
     prefetch_tmap(&tm_qkv);
     prefetch_tmap(&tm_rk);
@@ -148,8 +154,8 @@ __global__ void __launch_bounds__(192, 1)
     if (elect_lane0()) {
       constexpr uint32_t idS = idesc_bf16_f32(128, Cf::BN, false, false);
       constexpr uint32_t idO = idesc_bf16_f32(128, HD, false, true);
-      const uint32_t sQ = smem_u32(sm);
-      bool ok = mbar_wait(q_full, 0, err, DEV_TIMEOUT_FULL);
+      bool ok = mbar_wait(qt_full, 0, err, DEV_TIMEOUT_FULL);
+      tc_fence_after();
       auto issue_pv = [&](int i) -> bool {
         const int s = i & 1;
         const int vs = i % Cf::VST;
@@ -177,9 +183,8 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t sK = smem_u32(sm + Cf::OFF_K0 + ks * Cf::KVB);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(sQ + (kk >> 2) * (Cf::BM * 128) + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = smem_desc_sw128(sK + (kk >> 2) * (Cf::BN * 128) + (kk & 3) * 32, 16, 1024);
-          tc_mma_f16(tmem + Cf::S_COL + s * Cf::BN, ad, bd, idS, kk ? 1u : 0u);
+          tc_mma_f16_ta(tmem + Cf::S_COL + s * Cf::BN, tmem + Cf::Q_COL + kk * 8, bd, idS, kk ? 1u : 0u);
         }
         tc_commit(&s_full[s]);
         tc_commit(&k_empty[ks]);
@@ -197,8 +202,25 @@ __global__ void __launch_bounds__(192, 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const float sc = p.scale * 1.4426950408889634f;
     float m_used = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
+    bool ok = mbar_wait(q_full, 0, err, DEV_TIMEOUT_FULL);
+    if (ok) {
+      // this row of Q: shared memory (128-byte swizzled) -> TMEM, bf16 pairs in K order
+#pragma unroll
+      for (int kb = 0; kb < KB; ++kb) {
+        float w[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 a = *(const uint4*)(sm + kb * Cf::BM * 128 + r * 128 + ((c ^ (r & 7)) << 4));
+          w[4 * c] = __uint_as_float(a.x); w[4 * c + 1] = __uint_as_float(a.y);
+          w[4 * c + 2] = __uint_as_float(a.z); w[4 * c + 3] = __uint_as_float(a.w);
+        }
+        tmem_st32(tmem + lane_base + Cf::Q_COL + kb * 32, w);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qt_full);
+    }
+    for (int j = 0; j < ntiles && ok; ++j) {
       const int s = j & 1;
       const int64_t j0 = jt0 + (int64_t)j * Cf::BN;
       if (!mbar_wait(&s_full[s], (j >> 1) & 1, err, DEV_TIMEOUT_ACC)) { ok = false; break; }
@@ -317,8 +339,11 @@ __global__ void __launch_bounds__(192, 1)
 // write dS (bf16) to one of two shared-memory buffers; the MMA warp accumulates
 // dQ += dS K in TMEM (the K tile read again as an MN-major operand). With S/dP and
 // dS double-buffered, S_{j+1} and dP_{j+1} run on the tensor cores while the
-// warps form dS_j. dQ is scaled by 1/sqrt(hd) on the way out.
-// TMEM: S0 [0,64), dP0 [64,128), S1 [128,192), dP1 [192,256), dQ [256, 256+HD).
+// warps form dS_j. dQ is scaled by 1/sqrt(hd) on the way out. The four warps first
+// copy their rows of Q and dO from shared memory into TMEM, where the S and dP MMAs
+// take them as the A operand.
+// TMEM: S0 [0,64), dP0 [64,128), S1 [128,192), dP1 [192,256), dQ [256, 256+HD),
+// Q [384, 384+HD/2), dO [448, 448+HD/2).
 template <int HD> struct AttnDqCfg {
   static constexpr int BM = 128, BN = 64;
   static constexpr int KST = 3, VST = 3;
@@ -332,6 +357,9 @@ template <int HD> struct AttnDqCfg {
   static constexpr int OFF_BAR = OFF_DS + 2 * DSB;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr uint32_t DQ_COL = 256;
+  // Q and dO as the A operands of S and dP, copied once into TMEM (bf16 pairs, one row
+  // per lane): the MMAs then read only their 64-key B tile from shared memory
+  static constexpr uint32_t Q_COL = 384, DO_COL = 448;
   static __device__ __forceinline__ uint32_t s_col(int b) { return b * 128; }
   static __device__ __forceinline__ uint32_t dp_col(int b) { return b * 128 + 64; }
 };
@@ -356,7 +384,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* ds_full = bars + 17;   // [2]
   uint64_t* ds_free = bars + 19;   // [2]
   uint64_t* dq_done = bars + 21;
-  uint32_t* tmem_slot = (uint32_t*)(bars + 22);
+  uint64_t* qt_full = bars + 22;   // Q and dO are in TMEM (4 warps)
+  uint32_t* tmem_slot = (uint32_t*)(bars + 23);
 
   const int warp = threadIdx.x >> 5;
   const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -379,6 +408,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&ds_full[s], 4); mbar_init(&ds_free[s], 1);
     }
     mbar_init(dq_done, 1);
+    mbar_init(qt_full, 4);
     fence_mbar_init();
     prefetch_tmap(&tm_q); prefetch_tmap(&tm_kv); prefetch_tmap(&tm_rk); prefetch_tmap(&tm_rv); prefetch_tmap(&tm_do);
   }
@@ -428,8 +458,8 @@ __global__ void __launch_bounds__(192, 1)
     if (elect_lane0()) {
       constexpr uint32_t idS = idesc_bf16_f32(128, Cf::BN, false, false);
       constexpr uint32_t idQ = idesc_bf16_f32(128, HD, false, true);
-      const uint32_t sQ = smem_u32(sm), sdO = smem_u32(sm + Cf::OFF_DO);
-      bool ok = mbar_wait(q_full, 0, err, DEV_TIMEOUT_FULL);
+      bool ok = mbar_wait(qt_full, 0, err, DEV_TIMEOUT_FULL);
+      tc_fence_after();
       auto issue_dq = [&](int i) -> bool {
         const int s = i & 1, ks = i % 3;
         if (!mbar_wait(&ds_full[s], (i >> 1) & 1, err, DEV_TIMEOUT_FULL)) return false;
@@ -459,17 +489,15 @@ __global__ void __launch_bounds__(192, 1)
         const uint32_t sV = smem_u32(sm + Cf::OFF_V0 + vs * Cf::KVB);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t offa = (kk >> 2) * (Cf::BM * 128) + (kk & 3) * 32;
           const uint32_t offb = (kk >> 2) * (Cf::BN * 128) + (kk & 3) * 32;
-          tc_mma_f16(tmem + Cf::s_col(s), smem_desc_sw128(sQ + offa, 16, 1024), smem_desc_sw128(sK + offb, 16, 1024),
-                     idS, kk ? 1u : 0u);
+          tc_mma_f16_ta(tmem + Cf::s_col(s), tmem + Cf::Q_COL + kk * 8, smem_desc_sw128(sK + offb, 16, 1024), idS,
+                        kk ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t offa = (kk >> 2) * (Cf::BM * 128) + (kk & 3) * 32;
           const uint32_t offb = (kk >> 2) * (Cf::BN * 128) + (kk & 3) * 32;
-          tc_mma_f16(tmem + Cf::dp_col(s), smem_desc_sw128(sdO + offa, 16, 1024),
-                     smem_desc_sw128(sV + offb, 16, 1024), idS, kk ? 1u : 0u);
+          tc_mma_f16_ta(tmem + Cf::dp_col(s), tmem + Cf::DO_COL + kk * 8, smem_desc_sw128(sV + offb, 16, 1024), idS,
+                        kk ? 1u : 0u);
         }
         tc_commit(&sp_full[s]);
         tc_commit(&v_empty[vs]);
@@ -489,12 +517,33 @@ __global__ void __launch_bounds__(192, 1)
     const float nL = r < nq ? -p.lse[si] * 1.4426950408889634f : -INFINITY;  // exp2(s*sc - lse*log2e)
     const int64_t lo_key = P - p.window + 1;
     const uint32_t span = (uint32_t)(P - lo_key);
-    bool ok = true;
     float Dr = 0.f;
+    bool ok = mbar_wait(q_full, 0, err, DEV_TIMEOUT_FULL);
+    if (ok) {
+      // this row of Q and of dO: shared memory (128-byte swizzled) -> TMEM, as bf16 pairs in K order
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const uint8_t* src = sm + (t ? Cf::OFF_DO : 0);
+        const uint32_t col = t ? Cf::DO_COL : Cf::Q_COL;
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb) {
+          float w[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 a = *(const uint4*)(src + kb * Cf::BM * 128 + r * 128 + ((c ^ (r & 7)) << 4));
+            w[4 * c] = __uint_as_float(a.x); w[4 * c + 1] = __uint_as_float(a.y);
+            w[4 * c + 2] = __uint_as_float(a.z); w[4 * c + 3] = __uint_as_float(a.w);
+          }
+          tmem_st32(tmem + lane_base + col + kb * 32, w);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(qt_full);
+    }
     if (p.dsum_in_dq) {
       // D = rowsum(dO * O) of this row and head, from the staged dO tile and O; the
       // dK/dV kernel that follows reads it from Dsum
-      ok = mbar_wait(q_full, 0, err, DEV_TIMEOUT_FULL);
       if (ok && r < nq) {
         const bf16* Orow = (const bf16*)p.O + ((int64_t)b * p.n + i0 + r) * p.ldo + h * HD;
         float acc = 0.f;

@@ -230,13 +230,15 @@ constexpr int TC_BK = 64;
 // quarter, each taking half of the tile's columns)
 constexpr int TC_THREADS = 320;
 constexpr int TC_EPI_WARPS = 8;
+constexpr int EPI_STAGE_BYTES = 32 * 32 * 4;  // epilogue staging per warp: 32 rows x 32 fp32
 
 template <int BN> struct TcCfg {
   static constexpr int STAGES = (BN == 256) ? 4 : 6;
   static constexpr int A_BYTES = TC_BM * TC_BK * 2;
   static constexpr int B_BYTES = BN * TC_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ +
+                              TC_EPI_WARPS * EPI_STAGE_BYTES /*epilogue staging*/;
   static constexpr int TMEM_COLS = 2 * BN;
 };
 
@@ -273,15 +275,165 @@ __device__ __forceinline__ float gelu_prime_tc(float u) {
   return 0.5f * (1.0f + erf_as7128(u * 0.70710678118654752f)) + u * e * 0.39894228040143268f;
 }
 
-// Global inputs of the epilogue for 32 columns of one row, as raw 16-byte words: the
-// fp32 residual (EPI_RESID) or fp32 master weights (EPI_SGD) in all eight, the bf16
-// pre-activations (EPI_DGELU) in the first four. They are fetched one 32-column chunk
-// ahead of their use (the first chunk before the accumulator is waited for), so each
-// thread has a whole chunk of loads in flight instead of one load per store.
+// ---------------------------------------------------------------- epilogue staging
+// Each accumulator row belongs to one thread (TMEM lane = row), so a thread's stores of
+// its row are 32 accesses to 32 different 128-byte lines per warp instruction, which the
+// load/store unit serves one line at a time (measured: a 128 x 128 fp32 residual
+// epilogue took 7.3K clocks). Global traffic of the epilogue therefore goes through a
+// per-warp shared-memory buffer of 32 rows x 32 columns: eight lanes cover one row's
+// 128 bytes (fp32) or four lanes its 64 bytes (bf16), so that each warp instruction
+// moves whole lines, and each thread reads or writes its own row in shared memory. The
+// 16-byte word q of row r sits at q ^ (r & 7) (fp32 rows) or q ^ ((r >> 1) & 3) (bf16
+// rows), so neither access pattern has bank conflicts.
+
+__device__ __forceinline__ uint32_t stg_f32(int r, int q) { return (uint32_t)(r * 128 + ((q ^ (r & 7)) << 4)); }
+__device__ __forceinline__ uint32_t stg_b16(int r, int q) { return (uint32_t)(r * 64 + ((q ^ ((r >> 1) & 3)) << 4)); }
+
+// Global inputs of the epilogue for the warp's 32 rows (from mw) and 32 columns (from
+// n): for the staged epilogues, this lane's 16-byte pieces in the coalesced layout of
+// the fp32 residual (EPI_RESID) or fp32 master weights (EPI_SGD), rows 4i + lane/8,
+// piece lane % 8; for EPI_DGELU, the bf16 pre-activations of the lane's own row (first
+// four words). They are fetched one 32-column chunk ahead of their use (the first chunk
+// before the accumulator is waited for).
 struct EpiIn {
   uint4 w[8];
 };
-__device__ __forceinline__ void epi_fetch32(const GemmParams& p, int z, int m, int n, EpiIn& in) {
+__device__ __forceinline__ void epi_fetch32_mixed(const GemmParams& p, int z, int mw, int n, EpiIn& in) {
+  const int lane = threadIdx.x & 31;
+  if (p.epi == EPI_RESID || p.epi == EPI_SGD) {
+    const float* base = p.epi == EPI_RESID ? (const float*)p.X + (int64_t)z * p.sX : (const float*)p.D + (int64_t)z * p.sD;
+    const int64_t ld = p.epi == EPI_RESID ? p.ldx : p.ldd;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int row = mw + 4 * i + (lane >> 3);
+      in.w[i] = row < p.M ? *(const uint4*)(base + (int64_t)row * ld + n + (lane & 7) * 4) : make_uint4(0, 0, 0, 0);
+    }
+  } else if (p.epi == EPI_DGELU) {  // row-wise: the bf16 pre-activations of this thread's own row
+    const int m = mw + lane;
+    if (m < p.M) {
+      const uint4* x = (const uint4*)((const bf16*)p.X + (int64_t)z * p.sX + (int64_t)m * p.ldx + n);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) in.w[i] = x[i];
+    }
+  }
+}
+
+// The coalesced pieces of `in` -> shared memory (put), then this thread's row out of
+// it (get: f(i, x_i) for its 32 values in column order).
+__device__ __forceinline__ void stage_put_f32(uint8_t* stg, const EpiIn& in) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) *(uint4*)(stg + stg_f32(4 * i + (lane >> 3), lane & 7)) = in.w[i];
+}
+template <typename F>
+__device__ __forceinline__ void stage_get_f32(const uint8_t* stg, F f) {
+  const int lane = threadIdx.x & 31;
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 x = *(const float4*)(stg + stg_f32(lane, q));
+    f(4 * q, x.x); f(4 * q + 1, x.y); f(4 * q + 2, x.z); f(4 * q + 3, x.w);
+  }
+  __syncwarp();
+}
+// This thread's row of 32 values -> shared memory -> coalesced global stores of the
+// warp's 32 rows (from mw) at columns [n, n + 32) of dst (leading dimension ld).
+__device__ __forceinline__ void stage_out_f32(uint8_t* stg, const float* v, float* dst, int64_t ld, int mw, int M,
+                                              int n) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    *(float4*)(stg + stg_f32(lane, q)) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int r = 4 * i + (lane >> 3);
+    const uint4 w = *(const uint4*)(stg + stg_f32(r, lane & 7));
+    if (mw + r < M) *(uint4*)(dst + (int64_t)(mw + r) * ld + n + (lane & 7) * 4) = w;
+  }
+  __syncwarp();
+}
+__device__ __forceinline__ void stage_out_b16(uint8_t* stg, const float* v, bf16* dst, int64_t ld, int mw, int M,
+                                              int n) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *(uint4*)(stg + stg_b16(lane, q)) =
+        make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                   pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = 8 * i + (lane >> 2);
+    const uint4 w = *(const uint4*)(stg + stg_b16(r, lane & 3));
+    if (mw + r < M) *(uint4*)(dst + (int64_t)(mw + r) * ld + n + (lane & 3) * 8) = w;
+  }
+  __syncwarp();
+}
+
+// 32 consecutive accumulator columns [n, n + 32) of this thread's row (m = mw + lane)
+// through the epilogue; `in` holds what epi_fetch32 read for the warp's rows (from mw)
+// and these columns. All 32 lanes of the warp call it together (rows past M are not
+// stored). The fp32 read-modify-write epilogues (residual, SGD) go through the staging
+// buffer; the bf16-output epilogues store their rows directly, which measured faster
+// for them (GELU 1024x4096x2048: 21 us direct, 24 us staged; SGD weight gradient
+// 2048x4096x1024: 37.5 us direct, 31.7 us staged).
+// n_next >= 0: once `in` is consumed, it is refilled with the inputs of the chunk at
+// columns [n_next, n_next + 32).
+__device__ __forceinline__ void epi_row32_mixed(const GemmParams& p, int z, int mw, int n, float* v, EpiIn& in,
+                                          uint8_t* stg, int n_next) {
+  const int m = mw + (int)(threadIdx.x & 31);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] *= p.alpha;
+  if (p.epi == EPI_STORE && p.d_f32) {
+    stage_out_f32(stg, v, (float*)p.D + (int64_t)z * p.sD, p.ldd, mw, p.M, n);
+  } else if (p.epi == EPI_RESID) {
+    stage_put_f32(stg, in);
+    if (n_next >= 0) epi_fetch32_mixed(p, z, mw, n_next, in);
+    stage_get_f32(stg, [&](int i, float x) { v[i] += x; });
+    stage_out_f32(stg, v, (float*)p.D + (int64_t)z * p.sD, p.ldd, mw, p.M, n);
+  } else if (p.epi == EPI_SGD) {  // D (fp32 master) += acc, Y = bf16 copy of the new D
+    stage_put_f32(stg, in);
+    if (n_next >= 0) epi_fetch32_mixed(p, z, mw, n_next, in);
+    stage_get_f32(stg, [&](int i, float w) { v[i] += w; });
+    stage_out_f32(stg, v, (float*)p.D + (int64_t)z * p.sD, p.ldd, mw, p.M, n);
+    if (p.Y) stage_out_b16(stg, v, (bf16*)p.Y + (int64_t)z * p.sY, p.ldy, mw, p.M, n);
+  } else if (m < p.M) {
+    const int64_t od = (int64_t)z * p.sD + (int64_t)m * p.ldd + n;
+    uint4* d = (uint4*)((bf16*)p.D + od);
+    if (p.epi == EPI_GELU) {
+      if (p.Y) {
+        uint4* y = (uint4*)((bf16*)p.Y + (int64_t)z * p.sY + (int64_t)m * p.ldy + n);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          y[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                            pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = gelu_tc(v[i]);
+    } else if (p.epi == EPI_DGELU) {  // pre-activations of this row, fetched row-wise by epi_fetch32
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const bf16* u = reinterpret_cast<const bf16*>(&in.w[i]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[8 * i + e] *= gelu_prime_tc(__bfloat162float(u[e]));
+      }
+    }
+    if (p.epi == EPI_DGELU && n_next >= 0) epi_fetch32_mixed(p, z, mw, n_next, in);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      d[i] = make_uint4(pack_bf16x2(v[8 * i], v[8 * i + 1]), pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
+                        pack_bf16x2(v[8 * i + 4], v[8 * i + 5]), pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+  }
+}
+
+// Row-wise epilogue (all layouts but the weight-gradient one): the global inputs of the
+// epilogue for 32 columns of one row, as raw 16-byte words: the fp32 residual
+// (EPI_RESID) or fp32 master weights (EPI_SGD) in all eight, the bf16 pre-activations
+// (EPI_DGELU) in the first four. They are fetched one 32-column chunk ahead of their use
+// (the first chunk before the accumulator is waited for), so each thread has a whole
+// chunk of loads in flight instead of one load per store.
+__device__ __forceinline__ void epi_fetch32_row(const GemmParams& p, int z, int m, int n, EpiIn& in) {
   if (m >= p.M) return;
   if (p.epi == EPI_RESID) {
     const uint4* x = (const uint4*)((const float*)p.X + (int64_t)z * p.sX + (int64_t)m * p.ldx + n);
@@ -301,7 +453,7 @@ __device__ __forceinline__ void epi_fetch32(const GemmParams& p, int z, int m, i
 // 32 consecutive accumulator columns of one row through the epilogue, vectorised;
 // `in` holds what epi_fetch32 read for the same columns.
 template <typename T>
-__device__ __forceinline__ void epi_row32(const GemmParams& p, int z, int m, int n, float* v, const EpiIn& in) {
+__device__ __forceinline__ void epi_row32_direct(const GemmParams& p, int z, int m, int n, float* v, const EpiIn& in) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] *= p.alpha;
   const int64_t od = (int64_t)z * p.sD + (int64_t)m * p.ldd + n;
@@ -404,12 +556,6 @@ __device__ __forceinline__ void epi_ce32(const GemmParams& p, int m, int n, floa
   cm = M;
 }
 
-// Epilogue of one accumulator tile for one epilogue warp: the warp fetches the global
-// inputs of its first 32 columns, waits for the accumulator (wait_acc() false: the
-// wait timed out), then reads its TMEM lane quarter (one output row per thread, row m)
-// over its half of the tile's columns [c_first*32, c_first*32 + BN/2), calls release()
-// once those columns are read (the accumulator may then be overwritten), and applies
-// the epilogue, each chunk's inputs fetched while the previous chunk is stored.
 // Split-K partial tile in shared memory: fp32 [128 rows][BN], the 16-byte word q of a
 // row stored at q ^ (row & 7), so that eight consecutive rows writing or reading the
 // same columns hit distinct banks.
@@ -418,12 +564,72 @@ __device__ __forceinline__ uint32_t part_addr(uint32_t base, int row, int q) {
   return base + (uint32_t)(row * BN + ((q ^ (row & 7)) << 2)) * 4u;
 }
 
+// Epilogue of one accumulator tile for one epilogue warp: the warp fetches the global
+// inputs of its first 32 columns, waits for the accumulator (wait_acc() false: the
+// wait timed out), then reads its TMEM lane quarter (one output row per thread, row m)
+// over its half of the tile's columns [c_first*32, c_first*32 + BN/2), calls release()
+// once those columns are read (the accumulator may then be overwritten), and applies
+// the epilogue through its staging buffer stg, each chunk's inputs fetched while the
+// previous chunk is stored. part: shared address of a split-K partial tile to add to
+// the accumulator (0: none), row: this thread's row in the tile.
+template <int BN, typename Wait, typename Release>
+__device__ __forceinline__ bool epilogue_tile_staged(const GemmParams& p, uint32_t taddr, int z, int m, int n0, int c_first,
+                                              uint8_t* stg, Wait wait_acc, Release release, uint32_t part = 0,
+                                              int row = 0) {
+  const int mw = m - (int)(threadIdx.x & 31);  // first row of this warp
+  EpiIn nxt;
+  epi_fetch32_mixed(p, z, mw, n0 + c_first * 32, nxt);
+  if (!wait_acc()) return false;
+  tc_fence_after();
+  const int tgt = (p.epi == EPI_CE && m < p.M) ? p.ce_tgt[m] : -1;
+  float cm = -INFINITY, cs = 0.f;
+#pragma unroll 1
+  for (int c = c_first; c < c_first + BN / 64; ++c) {
+    float v[32];
+    tmem_ld32(taddr + c * 32, v);
+    if (c == c_first + BN / 64 - 1) {  // this warp's columns are read: its share of the accumulator is free
+      tc_fence_before();
+      __syncwarp();
+      release();
+    }
+    if (part) {  // acc = acc(first K half) + partial(second K half), in this order
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float4 q;
+        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                     : "=f"(q.x), "=f"(q.y), "=f"(q.z), "=f"(q.w)
+                     : "r"(part_addr<BN>(part, row, c * 8 + i)));
+        v[4 * i] += q.x; v[4 * i + 1] += q.y; v[4 * i + 2] += q.z; v[4 * i + 3] += q.w;
+      }
+    }
+    if (p.epi == EPI_CE) {
+      if (m < p.M) {
+        epi_ce32(p, m, n0 + c * 32, v, tgt, cm, cs);
+        if (c & 1) {  // a 64-column vocabulary chunk is complete
+          p.ce_part[(int64_t)m * (p.N / 64) + (n0 + c * 32) / 64] = make_float2(cm, cs);
+          cm = -INFINITY;
+          cs = 0.f;
+        }
+      }
+    } else {
+      epi_row32_mixed(p, z, mw, n0 + c * 32, v, nxt, stg, c + 1 < c_first + BN / 64 ? n0 + (c + 1) * 32 : -1);
+    }
+  }
+  return true;
+}
+
+// Epilogue of one accumulator tile for one epilogue warp: the warp fetches the global
+// inputs of its first 32 columns, waits for the accumulator (wait_acc() false: the
+// wait timed out), then reads its TMEM lane quarter (one output row per thread, row m)
+// over its half of the tile's columns [c_first*32, c_first*32 + BN/2), calls release()
+// once those columns are read (the accumulator may then be overwritten), and applies
+// the epilogue, each chunk's inputs fetched while the previous chunk is stored.
 // part: shared address of a split-K partial tile to add to the accumulator (0: none).
 template <int BN, typename Wait, typename Release>
-__device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint32_t taddr, int z, int m, int n0, int c_first,
+__device__ __forceinline__ bool epilogue_tile_direct(const GemmParams& p, uint32_t taddr, int z, int m, int n0, int c_first,
                                               Wait wait_acc, Release release, uint32_t part = 0, int row = 0) {
   EpiIn nxt;
-  epi_fetch32(p, z, m, n0 + c_first * 32, nxt);
+  epi_fetch32_row(p, z, m, n0 + c_first * 32, nxt);
   if (!wait_acc()) return false;
   tc_fence_after();
   const int tgt = (p.epi == EPI_CE && m < p.M) ? p.ce_tgt[m] : -1;
@@ -448,7 +654,7 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint32_t tadd
       }
     }
     const EpiIn cur = nxt;
-    if (c + 1 < c_first + BN / 64) epi_fetch32(p, z, m, n0 + (c + 1) * 32, nxt);
+    if (c + 1 < c_first + BN / 64) epi_fetch32_row(p, z, m, n0 + (c + 1) * 32, nxt);
     if (m < p.M) {
       if (p.epi == EPI_CE) {
         epi_ce32(p, m, n0 + c * 32, v, tgt, cm, cs);
@@ -458,11 +664,27 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint32_t tadd
           cs = 0.f;
         }
       } else {
-        epi_row32<bf16>(p, z, m, n0 + c * 32, v, cur);
+        epi_row32_direct<bf16>(p, z, m, n0 + c * 32, v, cur);
       }
     }
   }
   return true;
+}
+
+// The epilogue of a tile: staged through shared memory in the weight-gradient layout
+// (A and B MN-major: the fused SGD update, whose fp32 read-modify-write of the master
+// weights is bound by uncoalesced row accesses: 2048x4096x1024 37.5 -> 30 us staged),
+// row-wise everywhere else (the bf16-output and residual epilogues of the other
+// layouts measured 2-7 us slower per launch staged, from the registers the staged path
+// takes at this kernel's 168-register limit).
+template <int BN, bool STAGED, typename Wait, typename Release>
+__device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint32_t taddr, int z, int m, int n0, int c_first,
+                                              uint8_t* stg, Wait wait_acc, Release release, uint32_t part = 0,
+                                              int row = 0) {
+  if constexpr (STAGED)
+    return epilogue_tile_staged<BN>(p, taddr, z, m, n0, c_first, stg, wait_acc, release, part, row);
+  else
+    return epilogue_tile_direct<BN>(p, taddr, z, m, n0, c_first, wait_acc, release, part, row);
 }
 
 // Persistent warp-specialised tcgen05 GEMM. Requirements (checked on the host):
@@ -584,6 +806,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int quarter = warp & 3;
     const int c_first = (warp >= 6 ? 1 : 0) * (BN / 64);
     const int row_in_tile = quarter * 32 + (threadIdx.x & 31);
+    uint8_t* stg = smem + C::STAGES * C::STAGE_BYTES + 256 + (warp - 2) * EPI_STAGE_BYTES;
     int lt = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
       const int z = tile / tiles_per_batch;
@@ -593,8 +816,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int acc = lt & 1;
       const uint32_t use = lt >> 1;
       const uint32_t taddr = tmem_base + acc * BN + ((uint32_t)(quarter * 32) << 16);
-      if (!epilogue_tile<BN>(
-              p, taddr, z, m0 + row_in_tile, n0, c_first,
+      if (!epilogue_tile<BN, A_MN>(
+              p, taddr, z, m0 + row_in_tile, n0, c_first, stg,
               [&] { return mbar_wait(&acc_full[acc], use & 1, err, DEV_TIMEOUT_ACC); },
               [&] {
                 if (elect_lane0()) mbar_arrive(&acc_empty[acc]);
@@ -730,6 +953,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int row = quarter * 32 + (threadIdx.x & 31);
     const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
     const uint32_t part = smem_u32(smem);
+    uint8_t* stg = smem + C::STAGES * C::STAGE_BYTES + 256 + (warp - 2) * EPI_STAGE_BYTES;
     if (rank == 1) {
       // partial accumulator -> CTA 0's stage buffers, once CTA 0 has released them
       if (mbar_wait(acc_full, 0, err, DEV_TIMEOUT_ACC) && mbar_wait_cluster(part_free, 0, err, DEV_TIMEOUT_ACC)) {
@@ -746,8 +970,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         mbar_arrive_cluster(mapa_shared(smem_u32(part_full), 0));
       }
     } else {
-      epilogue_tile<BN>(
-          p, taddr, z, m0 + row, n0, c_first,
+      epilogue_tile<BN, A_MN>(
+          p, taddr, z, m0 + row, n0, c_first, stg,
           [&] {
             if (!mbar_wait(acc_full, 0, err, DEV_TIMEOUT_ACC)) return false;
             if (warp == 2 && elect_lane0()) mbar_arrive_cluster(mapa_shared(smem_u32(part_free), 1));
@@ -783,7 +1007,8 @@ template <int BN> struct Tc2Cfg {
   static constexpr int B_BYTES = BH * TC_BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (BN == 256) ? 6 : 8;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/ +
+                              TC_EPI_WARPS * EPI_STAGE_BYTES /*epilogue staging*/;
   static constexpr int TMEM_COLS = 2 * BN;
 };
 
@@ -907,6 +1132,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const int quarter = warp & 3;
     const int c_first = (warp >= 6 ? 1 : 0) * (BN / 64);
     const int row_in_tile = quarter * 32 + (threadIdx.x & 31);
+    uint8_t* stg = smem + C::STAGES * C::STAGE_BYTES + 256 + (warp - 2) * EPI_STAGE_BYTES;
     int lt = 0;
     for (int tile = pair; tile < num_tiles; tile += npairs, ++lt) {
       const int z = tile / tiles_per_batch;
@@ -916,8 +1142,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int acc = lt & 1;
       const uint32_t use = lt >> 1;
       const uint32_t taddr = tmem_base + acc * BN + ((uint32_t)(quarter * 32) << 16);
-      if (!epilogue_tile<BN>(
-              p, taddr, z, m0 + row_in_tile, n0, c_first,
+      if (!epilogue_tile<BN, A_MN>(
+              p, taddr, z, m0 + row_in_tile, n0, c_first, stg,
               [&] { return mbar_wait(&acc_full[acc], use & 1, err, DEV_TIMEOUT_ACC); },
               [&] {
                 if (elect_lane0()) mbar_arrive_cluster(acc_empty0 + 8u * acc);
