@@ -223,6 +223,87 @@ __global__ void __launch_bounds__(256) gemm_skinny_kernel(GemmParams p) {
   }
 }
 
+// ============================================================== few-row engine (decode)
+// Up to 8 rows per batch slice (one token per sequence in decode, or one row of a
+// sequence against its own fast weights): every weight byte is read once and the
+// product is bound by memory latency and bandwidth, not arithmetic. A CTA of 8 warps
+// owns 32 output columns; the slice's rows of A are staged once in shared memory, each
+// warp streams 4 weight rows (and their dW rows) with 16 bytes per lane and all of a
+// lane's loads of a row in flight, and each lane's 4 x 8 partial sums are reduced across
+// the warp by recursive halving (31 shuffles), after which lane l holds column l / 8,
+// row l % 8. Compared with the two-columns-per-CTA kernel above, A is read once per 32
+// columns instead of once per 2.
+constexpr int RW_COLS = 32;
+constexpr int RW_MAXM = 8;
+constexpr int RW_SMEM_MAX = 96 * 1024;  // staged A: M * K * 2 bytes
+static __global__ void __launch_bounds__(256) gemm_rows_kernel(GemmParams p) {
+  extern __shared__ uint4 xs4[];  // [M][K / 8] 16-byte chunks of this slice's A
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int z = blockIdx.y;
+  const int kc = p.K / 8;
+  pdl_wait();  // A (and the epilogue inputs) come from the previous kernel
+  {
+    const bf16* A = (const bf16*)p.A + (int64_t)z * p.sA;
+    for (int i = threadIdx.x; i < p.M * kc; i += 256) {
+      const int m = i / kc, c = i - m * kc;
+      xs4[i] = *(const uint4*)(A + (int64_t)m * p.lda + c * 8);
+    }
+  }
+  __syncthreads();
+  pdl_trigger();
+  const int n0 = blockIdx.x * RW_COLS + warp * 4;
+  const bf16* Bw = (const bf16*)p.B + (int64_t)z * p.sB;
+  const bf16* B2w = p.B2 ? (const bf16*)p.B2 + (int64_t)z * p.sB2 : nullptr;
+  float v[4 * RW_MAXM];  // [column j][row m]
+#pragma unroll
+  for (int i = 0; i < 4 * RW_MAXM; ++i) v[i] = 0.f;
+#pragma unroll 4
+  for (int c = lane; c < kc; c += 32) {
+    uint4 wu[4], w2[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + j < p.N ? n0 + j : p.N - 1;  // columns past N compute a copy, never stored
+      wu[j] = *(const uint4*)(Bw + (int64_t)n * p.ldb + c * 8);
+      w2[j] = B2w ? *(const uint4*)(B2w + (int64_t)n * p.ldb + c * 8) : make_uint4(0, 0, 0, 0);
+    }
+    float w[4][8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const bf16* e = reinterpret_cast<const bf16*>(&wu[j]);
+      const bf16* e2 = reinterpret_cast<const bf16*>(&w2[j]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[j][i] = __bfloat162float(e[i]) + __bfloat162float(e2[i]);
+    }
+#pragma unroll
+    for (int m = 0; m < RW_MAXM; ++m) {
+      if (m < p.M) {
+        const uint4 xu = xs4[m * kc + c];
+        const bf16* xe = reinterpret_cast<const bf16*>(&xu);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float x = __bfloat162float(xe[i]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) v[j * RW_MAXM + m] = fmaf(x, w[j][i], v[j * RW_MAXM + m]);
+        }
+      }
+    }
+  }
+  // recursive halving: at offset o a lane keeps the half of its values selected by
+  // (lane & o) and adds its partner's copy of that half
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = up ? v[i] : v[i + o];
+      const float keep = up ? v[i + o] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  const int n = n0 + (lane >> 3), m = lane & 7;
+  if (m < p.M && n < p.N) epi_apply<bf16>(p, z, m, n, v[0]);
+}
+
 // ============================================================== tcgen05 engine
 constexpr int TC_BM = 128;
 constexpr int TC_BK = 64;
@@ -571,11 +652,12 @@ __device__ __forceinline__ uint32_t part_addr(uint32_t base, int row, int q) {
 // once those columns are read (the accumulator may then be overwritten), and applies
 // the epilogue through its staging buffer stg, each chunk's inputs fetched while the
 // previous chunk is stored. part: shared address of a split-K partial tile to add to
-// the accumulator (0: none), row: this thread's row in the tile.
+// the accumulator (0: none, [128 rows][BN] from chunk part_c0 on), row: this thread's
+// row in the tile.
 template <int BN, typename Wait, typename Release>
 __device__ __forceinline__ bool epilogue_tile_staged(const GemmParams& p, uint32_t taddr, int z, int m, int n0, int c_first,
                                               uint8_t* stg, Wait wait_acc, Release release, uint32_t part = 0,
-                                              int row = 0) {
+                                              int row = 0, int part_c0 = 0) {
   const int mw = m - (int)(threadIdx.x & 31);  // first row of this warp
   EpiIn nxt;
   epi_fetch32_mixed(p, z, mw, n0 + c_first * 32, nxt);
@@ -598,7 +680,7 @@ __device__ __forceinline__ bool epilogue_tile_staged(const GemmParams& p, uint32
         float4 q;
         asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                      : "=f"(q.x), "=f"(q.y), "=f"(q.z), "=f"(q.w)
-                     : "r"(part_addr<BN>(part, row, c * 8 + i)));
+                     : "r"(part_addr<BN>(part, row, (c - part_c0) * 8 + i)));
         v[4 * i] += q.x; v[4 * i + 1] += q.y; v[4 * i + 2] += q.z; v[4 * i + 3] += q.w;
       }
     }
@@ -624,10 +706,12 @@ __device__ __forceinline__ bool epilogue_tile_staged(const GemmParams& p, uint32
 // over its half of the tile's columns [c_first*32, c_first*32 + BN/2), calls release()
 // once those columns are read (the accumulator may then be overwritten), and applies
 // the epilogue, each chunk's inputs fetched while the previous chunk is stored.
-// part: shared address of a split-K partial tile to add to the accumulator (0: none).
+// part: shared address of a split-K partial tile ([128 rows][BN] from chunk part_c0 on)
+// to add to the accumulator (0: none).
 template <int BN, typename Wait, typename Release>
 __device__ __forceinline__ bool epilogue_tile_direct(const GemmParams& p, uint32_t taddr, int z, int m, int n0, int c_first,
-                                              Wait wait_acc, Release release, uint32_t part = 0, int row = 0) {
+                                              Wait wait_acc, Release release, uint32_t part = 0, int row = 0,
+                                              int part_c0 = 0) {
   EpiIn nxt;
   epi_fetch32_row(p, z, m, n0 + c_first * 32, nxt);
   if (!wait_acc()) return false;
@@ -649,7 +733,7 @@ __device__ __forceinline__ bool epilogue_tile_direct(const GemmParams& p, uint32
         float4 q;
         asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                      : "=f"(q.x), "=f"(q.y), "=f"(q.z), "=f"(q.w)
-                     : "r"(part_addr<BN>(part, row, c * 8 + i)));
+                     : "r"(part_addr<BN>(part, row, (c - part_c0) * 8 + i)));
         v[4 * i] += q.x; v[4 * i + 1] += q.y; v[4 * i + 2] += q.z; v[4 * i + 3] += q.w;
       }
     }
@@ -680,11 +764,11 @@ __device__ __forceinline__ bool epilogue_tile_direct(const GemmParams& p, uint32
 template <int BN, bool STAGED, typename Wait, typename Release>
 __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint32_t taddr, int z, int m, int n0, int c_first,
                                               uint8_t* stg, Wait wait_acc, Release release, uint32_t part = 0,
-                                              int row = 0) {
+                                              int row = 0, int part_c0 = 0) {
   if constexpr (STAGED)
-    return epilogue_tile_staged<BN>(p, taddr, z, m, n0, c_first, stg, wait_acc, release, part, row);
+    return epilogue_tile_staged<BN>(p, taddr, z, m, n0, c_first, stg, wait_acc, release, part, row, part_c0);
   else
-    return epilogue_tile_direct<BN>(p, taddr, z, m, n0, c_first, wait_acc, release, part, row);
+    return epilogue_tile_direct<BN>(p, taddr, z, m, n0, c_first, wait_acc, release, part, row, part_c0);
 }
 
 // Persistent warp-specialised tcgen05 GEMM. Requirements (checked on the host):
@@ -836,12 +920,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 // ============================================================== tcgen05 engine, K split over a CTA pair
 // For the thin products of an adaptive step (1024 rows, N = 2048: 64 tiles of 128 x 256
 // for 148 SMs), a cluster of two CTAs computes one 128 x BN tile: CTA r accumulates
-// k blocks [r kb/2, (r+1) kb/2) in its own TMEM. Once CTA 0's MMAs have completed its
-// operand stages are idle; CTA 1 then writes its partial accumulator there over
-// distributed shared memory, and CTA 0 adds it to its own before the epilogue
-// (acc = acc_0 + acc_1, always in this order: deterministic). The tile count doubles
-// at the operand bytes per FLOP of a 128 x BN tile, and no global workspace is used.
-// One tile per cluster: the grid is exactly two CTAs per tile.
+// k blocks [r kb/2, (r+1) kb/2) in its own TMEM. Once a CTA's MMAs have completed its
+// operand stages are idle; each CTA then writes the half of its partial accumulator
+// that the peer finishes into the peer's stages over distributed shared memory, and
+// both run the epilogue of their own half of the columns (acc_0 + acc_1 = acc_1 + acc_0
+// in fp32: deterministic). The tile count doubles at the operand bytes per FLOP of a
+// 128 x BN tile, every MMA is 256 wide, and no global workspace is used. One tile per
+// cluster: the grid is exactly two CTAs per tile.
 template <int BN, bool A_MN, bool B_MN>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     gemm_tck_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -854,8 +939,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t* full = bars;                       // [STAGES]
   uint64_t* empty = bars + C::STAGES;          // [STAGES]
   uint64_t* acc_full = bars + 2 * C::STAGES;   // this CTA's MMAs are complete
-  uint64_t* part_free = acc_full + 1;          // CTA 1: CTA 0's stages may be overwritten
-  uint64_t* part_full = acc_full + 2;          // CTA 0: CTA 1's partial is in place (epilogue threads)
+  uint64_t* part_free = acc_full + 1;          // the peer's stages may be overwritten
+  uint64_t* part_full = acc_full + 2;          // the peer's partial is in place (its epilogue threads)
   uint32_t* tmem_slot = (uint32_t*)(acc_full + 3);
 
   const int warp = threadIdx.x >> 5;
@@ -948,37 +1033,42 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (ok) tc_commit(acc_full);
     }
   } else {
+    // CTA r finishes the columns [r BN/2, (r+1) BN/2) of the tile: it sends its partial
+    // accumulator of the other half into the peer's idle operand stages and adds the
+    // peer's partial of its own half (a + b = b + a in fp32: the same result on both
+    // sides of the pair). Warps 2-5 and 6-9 each take half of every such half.
+    constexpr int HALF = BN / 64;  // 32-column chunks per half of the tile
     const int quarter = warp & 3;
-    const int c_first = (warp >= 6 ? 1 : 0) * (BN / 64);
+    const int grp = warp >= 6 ? 1 : 0;
     const int row = quarter * 32 + (threadIdx.x & 31);
     const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
-    const uint32_t part = smem_u32(smem);
+    const uint32_t part = smem_u32(smem);  // the peer's partial of this CTA's half: [128][BN/2] fp32
     uint8_t* stg = smem + C::STAGES * C::STAGE_BYTES + 256 + (warp - 2) * EPI_STAGE_BYTES;
-    if (rank == 1) {
-      // partial accumulator -> CTA 0's stage buffers, once CTA 0 has released them
-      if (mbar_wait(acc_full, 0, err, DEV_TIMEOUT_ACC) && mbar_wait_cluster(part_free, 0, err, DEV_TIMEOUT_ACC)) {
-        tc_fence_after();
-        const uint32_t peer = mapa_shared(part, 0);
-#pragma unroll 1
-        for (int c = c_first; c < c_first + BN / 64; ++c) {
-          float v[32];
-          tmem_ld32(taddr + c * 32, v);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            st_cluster_v4(part_addr<BN>(peer, row, c * 8 + i), v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-        }
-        mbar_arrive_cluster(mapa_shared(smem_u32(part_full), 0));
-      }
-    } else {
-      epilogue_tile<BN, A_MN>(
-          p, taddr, z, m0 + row, n0, c_first, stg,
-          [&] {
-            if (!mbar_wait(acc_full, 0, err, DEV_TIMEOUT_ACC)) return false;
-            if (warp == 2 && elect_lane0()) mbar_arrive_cluster(mapa_shared(smem_u32(part_free), 1));
-            return mbar_wait_cluster(part_full, 0, err, DEV_TIMEOUT_ACC);
-          },
-          [] {}, part, row);
+    const int mine0 = (int)rank * HALF, other0 = (1 - (int)rank) * HALF;
+    bool ok = mbar_wait(acc_full, 0, err, DEV_TIMEOUT_ACC);
+    if (ok) {
+      tc_fence_after();
+      // this CTA's MMAs are complete, so its stages are free for the peer's partial
+      if (warp == 2 && elect_lane0()) mbar_arrive_cluster(mapa_shared(smem_u32(part_free), 1 - rank));
+      ok = mbar_wait_cluster(part_free, 0, err, DEV_TIMEOUT_ACC);
     }
+    if (ok) {
+      const uint32_t peer = mapa_shared(part, 1 - rank);
+#pragma unroll 1
+      for (int k = 0; k < HALF / 2; ++k) {
+        const int c = other0 + grp * (HALF / 2) + k;
+        float v[32];
+        tmem_ld32(taddr + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          st_cluster_v4(part_addr<BN / 2>(peer, row, (c - other0) * 8 + i), v[4 * i], v[4 * i + 1], v[4 * i + 2],
+                        v[4 * i + 3]);
+      }
+      mbar_arrive_cluster(mapa_shared(smem_u32(part_full), 1 - rank));
+    }
+    epilogue_tile<BN / 2, A_MN>(
+        p, taddr, z, m0 + row, n0, mine0 + grp * (HALF / 2), stg,
+        [&] { return ok && mbar_wait_cluster(part_full, 0, err, DEV_TIMEOUT_ACC); }, [] {}, part, row, mine0);
   }
   tc_fence_before();
   __syncthreads();

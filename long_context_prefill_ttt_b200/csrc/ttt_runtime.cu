@@ -357,6 +357,8 @@ int prime_kernel_attributes() {
   const cudaError_t r[] = {tc_attr<128, false, false>(), tc_attr<256, false, false>(), tc_attr<128, false, true>(),
                            tc_attr<256, false, true>(),  tc_attr<128, true, true>(),   tc_attr<256, true, true>(),
                            attn_mma_attributes<64>(),    attn_mma_attributes<128>(),
+                           cudaFuncSetAttribute(gemm_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                RW_SMEM_MAX),
                            cudaFuncSetAttribute(attn_fwd_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 AttnTcCfg<64>::SMEM),
                            cudaFuncSetAttribute(attn_fwd_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -419,11 +421,18 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
   if (!force_simt && skinny_ok(p, elem_is_bf16)) {
     GemmParams q = p;
     if (p.epi == EPI_QKV_ROPE) q.epi = EPI_STORE;
-    dim3 grid((p.N + 1) / 2, p.batch);
-    if (elem_is_bf16)
-      gemm_skinny_kernel<bf16><<<grid, 256, 0, st>>>(q);
-    else
-      gemm_skinny_kernel<float><<<grid, 256, 0, st>>>(q);
+    const size_t xbytes = (size_t)p.M * p.K * 2;
+    if (elem_is_bf16 && p.M <= RW_MAXM && xbytes <= (size_t)RW_SMEM_MAX) {
+      const cudaError_t e = launch_pdl(gemm_rows_kernel, dim3((p.N + RW_COLS - 1) / RW_COLS, p.batch), dim3(256),
+                                       xbytes, st, q);
+      if (e != cudaSuccess) return (int)e;
+    } else {
+      dim3 grid((p.N + 1) / 2, p.batch);
+      if (elem_is_bf16)
+        gemm_skinny_kernel<bf16><<<grid, 256, 0, st>>>(q);
+      else
+        gemm_skinny_kernel<float><<<grid, 256, 0, st>>>(q);
+    }
     if (p.epi == EPI_QKV_ROPE) {
       const cudaError_t re =
         elem_is_bf16 ? rope_launch<bf16>((bf16*)p.D, p.ldd, p.rope_cols, p.M, p.rope_n, p.rope_pos0, p.rope_hd,
@@ -478,13 +487,14 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
     }
     // K split over CTA pairs: thin products whose 128 x 256 tiles fill at most half the
     // SMs (the N = 2048 products of an adaptive step: 64 tiles) run each tile on two SMs
-    // with 256-wide tiles instead of 128-wide tiles on one. The hand-over of the partial
-    // tile costs a few microseconds, so only long K pays: measured on B200 at 1024 x 2048,
-    // K = 8192 (W_init + dW, 4096 each) 47 -> 43 us, K = 6144 36 -> 34 us, K = 32000
-    // 152 -> 113 us, but K = 4096 28 -> 32 us and K = 2048 22 -> 28 us.
+    // with 256-wide tiles instead of 128-wide tiles on one (an M = 128 MMA costs about the
+    // same at N = 128 as at N = 256). The exchange of the partial halves costs a few
+    // microseconds, so K >= 4096 pays: measured on B200 at 1024 x 2048, K = 8192
+    // (W_init + dW) 45.6 -> 35.9 us, K = 6144 35.8 -> 27.6 us, K = 4096 26.2 -> 22.6 us,
+    // K = 32000 150 -> 109 us; K = 2048 21.4 -> 22.1 us stays on single CTAs.
     const int t256 = (p.N % 256 == 0) ? m_tiles * (p.N / 256) * p.batch : 0;
     const int kbt = (p.K / TC_BK) * (p.B2 ? 2 : 1);
-    if (engine != GEMM_TC1 && p.epi != EPI_CE && t256 > 0 && 2 * t256 <= num_sms && kbt % 2 == 0 && kbt >= 96) {
+    if (engine != GEMM_TC1 && p.epi != EPI_CE && t256 > 0 && 2 * t256 <= num_sms && kbt % 2 == 0 && kbt >= 64) {
       if (!p.a_mn && !p.b_mn) e = launch_tck<256, false, false>(pt, st, err, &ok);
       else if (!p.a_mn && p.b_mn) e = launch_tck<256, false, true>(pt, st, err, &ok);
       else e = launch_tck<256, true, true>(pt, st, err, &ok);

@@ -128,10 +128,10 @@ def test_gemm_epilogues(T, engine):
 
 
 # Thin products that engine 0 runs with K split over a CTA pair (two SMs per 128 x 256
-# tile, the second half's partial added in the first CTA's shared memory): layouts, a
+# tile, each finishing half of its columns with the peer's partial): layouts, a
 # ragged M tail with batches, and double-K (B + B2: the first CTA takes the B half, the
 # second the B2 half), with an odd k-block count per operand.
-K_SPLIT_CASES = [(1024, 2048, 8192, 1, 0, 0, False), (1024, 2048, 6144, 1, 0, 1, False),
+K_SPLIT_CASES = [(1024, 2048, 8192, 1, 0, 0, False), (1024, 2048, 4096, 1, 0, 1, False),
                  (1024, 2048, 6144, 1, 1, 1, False), (300, 512, 6400, 2, 0, 0, False),
                  (1024, 2048, 3136, 1, 0, 0, True), (256, 768, 4160, 1, 0, 1, True)]
 
@@ -276,9 +276,12 @@ def test_attention_forward_and_backward(T, engine, dtype, B, H, hd, n, q0, windo
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
-@pytest.mark.parametrize("M,N,K,batch", [(1, 768, 768, 8), (8, 2304, 768, 1), (16, 384, 3072, 2), (8, 32000, 768, 1)])
+@pytest.mark.parametrize("M,N,K,batch", [(1, 768, 768, 8), (8, 2304, 768, 1), (16, 384, 3072, 2), (8, 32000, 768, 1),
+                                         (3, 1000, 3072, 2), (8, 776, 6144, 1)])
 def test_skinny_gemm_rows_per_sequence(T, dtype, M, N, K, batch):
-    """Decode-sized products (<= 16 rows per slice): shared W plus per-slice dW, residual and GELU epilogues."""
+    """Decode-sized products (<= 16 rows per slice): shared W plus per-slice dW, residual and GELU epilogues.
+    bf16 with <= 8 rows runs the 32-columns-per-CTA kernel: N off its column grid, and A filling
+    its 96 KB staging buffer (8 x 6144), are among the cases."""
     A = _rand((batch, M, K), dtype, 31)
     Bs = _rand((1, N, K), dtype, 32, 0.05)
     B2 = _rand((batch, N, K), dtype, 33, 1e-3)
