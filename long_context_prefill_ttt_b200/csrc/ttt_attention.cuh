@@ -255,18 +255,28 @@ template <typename T, int HD>
 __global__ void __launch_bounds__(256) attn_decode_kernel(const T* __restrict__ q, int64_t ldq,
                                                           const T* __restrict__ ring_k, const T* __restrict__ ring_v,
                                                           int C, int d, int window, const int64_t* __restrict__ pos,
-                                                          float scale, T* __restrict__ out, int64_t ldo) {
-  // Each lane owns one key per step: its K row gives the score, its V row is
-  // accumulated into the lane's partial output (all row loads independent); the
-  // 32 partial outputs of a warp are summed once at the end.
+                                                          float scale, T* __restrict__ out, int64_t ldo,
+                                                          float* __restrict__ part, int* __restrict__ ticket) {
+  // The window of (head h, sequence b) is split into gridDim.z equal parts, one CTA
+  // each. In a CTA each lane owns one key per step: its K row gives the score, its V row
+  // is accumulated into the lane's partial output (all row loads independent); the 32
+  // partial outputs of a warp are summed once at the end, then the 8 warps'. With more
+  // than one part, each CTA stores its (max, sum, unnormalised output) in `part` and the
+  // last CTA of the (h, b) to finish (a ticket counter, reset by that CTA) merges the
+  // parts in their fixed order, so the result does not depend on which CTA is last.
   constexpr int CH = HD < 32 ? HD : (HD == 128 ? 16 : 32);  // row chunk held in registers
   __shared__ float qs[HD];
   __shared__ float wm[8], wl[8];
   __shared__ float wo[8][HD];
-  const int h = blockIdx.x, b = blockIdx.y;
+  __shared__ int last;
+  const int h = blockIdx.x, b = blockIdx.y, z = blockIdx.z, nz = gridDim.z;
+  const int H = gridDim.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t P = *pos;
   const int64_t lo = P - window + 1 > 0 ? P - window + 1 : 0;
+  const int64_t span = (P - lo + nz) / nz;  // keys per part (the last part may be shorter or empty)
+  const int64_t zlo = lo + z * span;
+  const int64_t zhi = (zlo + span - 1 < P) ? zlo + span - 1 : P;
   for (int c = threadIdx.x; c < HD; c += 256) qs[c] = to_f32(q[(int64_t)b * ldq + h * HD + c]) * scale;
   __syncthreads();
   const T* Kb = ring_k + (int64_t)b * C * d + h * HD;
@@ -275,10 +285,10 @@ __global__ void __launch_bounds__(256) attn_decode_kernel(const T* __restrict__ 
 #pragma unroll
   for (int c = 0; c < HD; ++c) acc[c] = 0.f;
   float m = -INFINITY, l = 0.f;  // warp-uniform running max, lane-partial sum
-  for (int64_t j0 = lo + warp * 32; j0 <= P; j0 += 256) {
+  for (int64_t j0 = zlo + warp * 32; j0 <= zhi; j0 += 256) {
     const int64_t j = j0 + lane;
-    const bool valid = j <= P;
-    const int64_t slot = (valid ? j : P) % C;
+    const bool valid = j <= zhi;
+    const int64_t slot = (valid ? j : zhi) % C;
     float s = 0.f;
 #pragma unroll
     for (int c0 = 0; c0 < HD; c0 += CH) {
@@ -325,12 +335,186 @@ __global__ void __launch_bounds__(256) attn_decode_kernel(const T* __restrict__ 
   for (int w = 0; w < 8; ++w) M = fmaxf(M, wm[w]);
   float Lsum = 0.f;
   for (int w = 0; w < 8; ++w) Lsum += wm[w] == -INFINITY ? 0.f : wl[w] * expf(wm[w] - M);
+  if (nz == 1) {
+    for (int c = threadIdx.x; c < HD; c += 256) {
+      float o = 0.f;
+      for (int w = 0; w < 8; ++w)
+        if (wm[w] != -INFINITY) o += wo[w][c] * expf(wm[w] - M);
+      out[(int64_t)b * ldo + h * HD + c] = from_f32<T>(o / Lsum);
+    }
+    return;
+  }
+  // this part -> part[(b, h, z)] = (M, L, O[HD]); the last CTA of (h, b) merges
+  float* mine = part + (((int64_t)b * H + h) * nz + z) * (HD + 2);
   for (int c = threadIdx.x; c < HD; c += 256) {
     float o = 0.f;
     for (int w = 0; w < 8; ++w)
       if (wm[w] != -INFINITY) o += wo[w][c] * expf(wm[w] - M);
-    out[(int64_t)b * ldo + h * HD + c] = from_f32<T>(o / Lsum);
+    mine[2 + c] = o;
   }
+  if (threadIdx.x == 0) {
+    mine[0] = M;
+    mine[1] = Lsum;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(ticket + (int64_t)b * H + h, 1) == nz - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  const float* base = part + ((int64_t)b * H + h) * nz * (HD + 2);
+  float Mt = -INFINITY;
+  for (int zz = 0; zz < nz; ++zz) Mt = fmaxf(Mt, __ldcg(base + zz * (HD + 2)));
+  float Lt = 0.f;
+  for (int zz = 0; zz < nz; ++zz) {
+    const float mz = __ldcg(base + zz * (HD + 2));
+    if (mz != -INFINITY) Lt += __ldcg(base + zz * (HD + 2) + 1) * expf(mz - Mt);
+  }
+  for (int c = threadIdx.x; c < HD; c += 256) {
+    float o = 0.f;
+    for (int zz = 0; zz < nz; ++zz) {
+      const float mz = __ldcg(base + zz * (HD + 2));
+      if (mz != -INFINITY) o += __ldcg(base + zz * (HD + 2) + 2 + c) * expf(mz - Mt);
+    }
+    out[(int64_t)b * ldo + h * HD + c] = from_f32<T>(o / Lt);
+  }
+  if (threadIdx.x == 0) ticket[(int64_t)b * H + h] = 0;  // ready for the next launch
+}
+
+// Decode attention for bf16 at head dims 64 and 128: one CTA of 4 warps per (head h,
+// sequence b, part z of the window). The HD/8 lanes of a key group read one key row
+// (16 bytes each, so a warp instruction covers whole rows: 4 keys at HD = 64, 2 at
+// HD = 128), form the score by a reduction over the group, and keep a running max, sum
+// and their 8 output elements; the groups of a warp and then the warps are merged at
+// the end. Registers stay few, so the window can be split into many parts; the part
+// results are merged by the last CTA of the (h, b) as in attn_decode_kernel.
+template <int HD>
+__global__ void __launch_bounds__(128) attn_decode_rows_kernel(const bf16* __restrict__ q, int64_t ldq,
+                                                               const bf16* __restrict__ ring_k,
+                                                               const bf16* __restrict__ ring_v, int C, int d,
+                                                               int window, const int64_t* __restrict__ pos,
+                                                               float scale, bf16* __restrict__ out, int64_t ldo,
+                                                               float* __restrict__ part, int* __restrict__ ticket) {
+  constexpr int LPK = HD / 8;    // lanes per key row
+  constexpr int KPW = 32 / LPK;  // keys per warp step
+  constexpr int U = 4;           // steps whose loads are issued together
+  __shared__ float wm[4], wl[4];
+  __shared__ float wo[4][HD];
+  __shared__ int last;
+  const int h = blockIdx.x, b = blockIdx.y, z = blockIdx.z, nz = gridDim.z, H = gridDim.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane / LPK, e = lane % LPK;  // key group within the warp, 16-byte chunk of the row
+  const int64_t P = *pos;
+  const int64_t lo = P - window + 1 > 0 ? P - window + 1 : 0;
+  const int64_t span = (P - lo + nz) / nz;
+  const int64_t zlo = lo + z * span;
+  const int64_t zhi = (zlo + span - 1 < P) ? zlo + span - 1 : P;
+  float qv[8];
+  {
+    const uint4 u = *(const uint4*)(q + (int64_t)b * ldq + h * HD + e * 8);
+    const bf16* qe = reinterpret_cast<const bf16*>(&u);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) qv[i] = __bfloat162float(qe[i]) * scale;
+  }
+  const bf16* Kb = ring_k + (int64_t)b * C * d + h * HD + e * 8;
+  const bf16* Vb = ring_v + (int64_t)b * C * d + h * HD + e * 8;
+  float m = -INFINITY, l = 0.f, acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  // the warp's first key per step is uniform across the warp (every lane runs the same
+  // iterations and shuffles); group g takes key jw + g
+  for (int64_t jw = zlo + warp * KPW; jw <= zhi; jw += (int64_t)4 * KPW * U) {
+    uint4 ku[U], vu[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t j = jw + (int64_t)u * 4 * KPW + g;
+      const int64_t slot = (j <= zhi ? j : zhi) % C;
+      ku[u] = *(const uint4*)(Kb + slot * d);
+      vu[u] = *(const uint4*)(Vb + slot * d);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t j = jw + (int64_t)u * 4 * KPW + g;
+      const bf16* ke = reinterpret_cast<const bf16*>(&ku[u]);
+      float sc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sc = fmaf(qv[i], __bfloat162float(ke[i]), sc);
+#pragma unroll
+      for (int o = 1; o < LPK; o <<= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+      if (j <= zhi) {  // uniform across the key group
+        const float mn = fmaxf(m, sc);
+        const float corr = expf(m - mn);  // 0 while m = -inf
+        const float pj = expf(sc - mn);
+        l = l * corr + pj;
+        const bf16* ve = reinterpret_cast<const bf16*>(&vu[u]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = fmaf(pj, __bfloat162float(ve[i]), acc[i] * corr);
+        m = mn;
+      }
+    }
+  }
+  // merge the key groups of the warp (lanes with the same chunk e)
+#pragma unroll
+  for (int o = LPK; o < 32; o <<= 1) {
+    const float mo = __shfl_xor_sync(0xffffffffu, m, o);
+    const float lo_ = __shfl_xor_sync(0xffffffffu, l, o);
+    const float mn = fmaxf(m, mo);
+    const float fa = m == -INFINITY ? 0.f : expf(m - mn);
+    const float fb = mo == -INFINITY ? 0.f : expf(mo - mn);
+    l = l * fa + lo_ * fb;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = acc[i] * fa + __shfl_xor_sync(0xffffffffu, acc[i], o) * fb;
+    m = mn;
+  }
+  if (g == 0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) wo[warp][e * 8 + i] = acc[i];
+    if (e == 0) { wm[warp] = m; wl[warp] = l; }
+  }
+  __syncthreads();
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w]);
+  float Lsum = 0.f;
+#pragma unroll
+  for (int w = 0; w < 4; ++w) Lsum += wm[w] == -INFINITY ? 0.f : wl[w] * expf(wm[w] - M);
+  float* mine = nz > 1 ? part + (((int64_t)b * H + h) * nz + z) * (HD + 2) : nullptr;
+  for (int c = threadIdx.x; c < HD; c += 128) {
+    float o = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+      if (wm[w] != -INFINITY) o += wo[w][c] * expf(wm[w] - M);
+    if (nz == 1) out[(int64_t)b * ldo + h * HD + c] = __float2bfloat16_rn(o / Lsum);
+    else mine[2 + c] = o;
+  }
+  if (nz == 1) return;
+  if (threadIdx.x == 0) {
+    mine[0] = M;
+    mine[1] = Lsum;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(ticket + (int64_t)b * H + h, 1) == nz - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  const float* base = part + ((int64_t)b * H + h) * nz * (HD + 2);
+  float Mt = -INFINITY;
+  for (int zz = 0; zz < nz; ++zz) Mt = fmaxf(Mt, __ldcg(base + zz * (HD + 2)));
+  float Lt = 0.f;
+  for (int zz = 0; zz < nz; ++zz) {
+    const float mz = __ldcg(base + zz * (HD + 2));
+    if (mz != -INFINITY) Lt += __ldcg(base + zz * (HD + 2) + 1) * expf(mz - Mt);
+  }
+  for (int c = threadIdx.x; c < HD; c += 128) {
+    float o = 0.f;
+    for (int zz = 0; zz < nz; ++zz) {
+      const float mz = __ldcg(base + zz * (HD + 2));
+      if (mz != -INFINITY) o += __ldcg(base + zz * (HD + 2) + 2 + c) * expf(mz - Mt);
+    }
+    out[(int64_t)b * ldo + h * HD + c] = __float2bfloat16_rn(o / Lt);
+  }
+  if (threadIdx.x == 0) ticket[(int64_t)b * H + h] = 0;  // ready for the next launch
 }
 
 }  // namespace ttt

@@ -732,6 +732,9 @@ template <typename T> class Engine : public ttt_handle {
   std::vector<int32_t> pend_tok_host;
   // decode scratch
   int32_t* chosen = nullptr; float* dec_loss = nullptr; float* dec_zmax = nullptr; int32_t* forced_col = nullptr;
+  // decode attention over the window in dec_split parts of ~256 keys: partial results
+  // [B][H][dec_split][hd + 2] and one ticket per (sequence, head)
+  int dec_split = 1; float* dec_part = nullptr; int* dec_ticket = nullptr;
   // per-call growable buffers
   int64_t chunk_pos = 0;                  // absolute position of row 0 of the chunk in the adaptive buffers
   bool decode_mode = false;               // set while a decode token step is being captured
@@ -957,12 +960,19 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
   dec_zmax = arena.get<float>(B);
   forced_col = arena.get<int32_t>(B);
   pos_dev = arena.get<int64_t>(1);
+  {
+    const int64_t w = kwin < C ? kwin : C;
+    dec_split = (int)std::min<int64_t>(16, std::max<int64_t>(1, (w + 255) / 256));
+    dec_part = arena.get<float>((size_t)B * H * dec_split * (hd + 2));
+    dec_ticket = arena.get<int>((size_t)B * H);
+  }
   if (arena.failed) {
     arena.release();
     return fail(this, TTT_ERR_OOM, "device allocation failed");
   }
   dev_bytes = arena.bytes;
   TTT_CUDA(cudaMemsetAsync(dev_err, 0, sizeof(int), st));
+  TTT_CUDA(cudaMemsetAsync(dec_ticket, 0, sizeof(int) * (size_t)B * H, st));
 
   // RoPE tables in double precision: lo[p][i] = angle p*theta_i (p < 1024), hi[q][i] = angle 1024*q*theta_i
   {
@@ -1105,12 +1115,27 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
   }
   if (decode_mode) {
     const float scale = 1.0f / sqrtf((float)hd);
-    const dim3 dg(H, B);
+    const dim3 dg(H, B, dec_split);  // the window in dec_split parts, merged by the last CTA of each (head, sequence)
+    if (is_bf16 && (hd == 64 || hd == 128)) {
+      if (hd == 64)
+        attn_decode_rows_kernel<64><<<dg, 128, 0, st>>>((const bf16*)qkv, 3 * d, (const bf16*)Lw.ring_k,
+                                                        (const bf16*)Lw.ring_v, C, d, kwin, pos_dev, scale,
+                                                        (bf16*)o, d, dec_part, dec_ticket);
+      else
+        attn_decode_rows_kernel<128><<<dg, 128, 0, st>>>((const bf16*)qkv, 3 * d, (const bf16*)Lw.ring_k,
+                                                         (const bf16*)Lw.ring_v, C, d, kwin, pos_dev, scale,
+                                                         (bf16*)o, d, dec_part, dec_ticket);
+      TTT_LAUNCHED();
+      GemmParams pd = gp(rows, d, d, o, d, false, Lw.Wo, d, false, xout, d, true, EPI_RESID);
+      pd.X = xin; pd.ldx = d;
+      return gemm(pd);
+    }
+    const dim3 dg1(H, B, 1);  // one CTA per (head, sequence) for the register-heavy kernel
     switch (hd) {
-      case 16: attn_decode_kernel<T, 16><<<dg, 256, 0, st>>>(qkv, 3 * d, Lw.ring_k, Lw.ring_v, C, d, kwin, pos_dev, scale, o, d); break;
-      case 32: attn_decode_kernel<T, 32><<<dg, 256, 0, st>>>(qkv, 3 * d, Lw.ring_k, Lw.ring_v, C, d, kwin, pos_dev, scale, o, d); break;
-      case 64: attn_decode_kernel<T, 64><<<dg, 256, 0, st>>>(qkv, 3 * d, Lw.ring_k, Lw.ring_v, C, d, kwin, pos_dev, scale, o, d); break;
-      case 128: attn_decode_kernel<T, 128><<<dg, 256, 0, st>>>(qkv, 3 * d, Lw.ring_k, Lw.ring_v, C, d, kwin, pos_dev, scale, o, d); break;
+      case 16: attn_decode_kernel<T, 16><<<dg1, 256, 0, st>>>(qkv, 3 * d, Lw.ring_k, Lw.ring_v, C, d, kwin, pos_dev, scale, o, d, dec_part, dec_ticket); break;
+      case 32: attn_decode_kernel<T, 32><<<dg1, 256, 0, st>>>(qkv, 3 * d, Lw.ring_k, Lw.ring_v, C, d, kwin, pos_dev, scale, o, d, dec_part, dec_ticket); break;
+      case 64: attn_decode_kernel<T, 64><<<dg1, 256, 0, st>>>(qkv, 3 * d, Lw.ring_k, Lw.ring_v, C, d, kwin, pos_dev, scale, o, d, dec_part, dec_ticket); break;
+      case 128: attn_decode_kernel<T, 128><<<dg1, 256, 0, st>>>(qkv, 3 * d, Lw.ring_k, Lw.ring_v, C, d, kwin, pos_dev, scale, o, d, dec_part, dec_ticket); break;
       default: poisoned = true; return fail(this, TTT_ERR_UNSUPPORTED, "decode: head dim must be 16, 32, 64 or 128");
     }
     TTT_LAUNCHED();
