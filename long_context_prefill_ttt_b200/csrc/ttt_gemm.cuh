@@ -227,17 +227,17 @@ __global__ void __launch_bounds__(256) gemm_skinny_kernel(GemmParams p) {
 // Up to 8 rows per batch slice (one token per sequence in decode, or one row of a
 // sequence against its own fast weights): every weight byte is read once and the
 // product is bound by memory latency and bandwidth, not arithmetic. A CTA of 8 warps
-// owns 32 output columns; the slice's rows of A are staged once in shared memory, each
-// warp streams 4 weight rows (and their dW rows) with 16 bytes per lane and all of a
-// lane's loads of a row in flight, and each lane's 4 x 8 partial sums are reduced across
-// the warp by recursive halving (31 shuffles), after which lane l holds column l / 8,
-// row l % 8. Compared with the two-columns-per-CTA kernel above, A is read once per 32
-// columns instead of once per 2.
-constexpr int RW_COLS = 32;
+// owns 8 * CW output columns; the slice's rows of A are staged once in shared memory,
+// each warp streams CW weight rows (and their dW rows) with 16 bytes per lane and all
+// of a lane's loads of a row in flight, and each lane's CW x 8 partial sums are reduced
+// across the warp by recursive halving, after which lane l holds one (column, row) sum.
+// CW is chosen on the host so that narrow products still spread over the SMs.
 constexpr int RW_MAXM = 8;
 constexpr int RW_SMEM_MAX = 96 * 1024;  // staged A: M * K * 2 bytes
-static __global__ void __launch_bounds__(256) gemm_rows_kernel(GemmParams p) {
-  extern __shared__ uint4 xs4[];  // [M][K / 8] 16-byte chunks of this slice's A
+template <int CW>
+__global__ void __launch_bounds__(256) gemm_rows_kernel(GemmParams p) {
+  constexpr int NV = CW * RW_MAXM;  // partial sums per lane: [column j][row m]
+  extern __shared__ uint4 xs4[];    // [M][K / 8] 16-byte chunks of this slice's A
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int z = blockIdx.y;
   const int kc = p.K / 8;
@@ -251,24 +251,24 @@ static __global__ void __launch_bounds__(256) gemm_rows_kernel(GemmParams p) {
   }
   __syncthreads();
   pdl_trigger();
-  const int n0 = blockIdx.x * RW_COLS + warp * 4;
+  const int n0 = (blockIdx.x * 8 + warp) * CW;
   const bf16* Bw = (const bf16*)p.B + (int64_t)z * p.sB;
   const bf16* B2w = p.B2 ? (const bf16*)p.B2 + (int64_t)z * p.sB2 : nullptr;
-  float v[4 * RW_MAXM];  // [column j][row m]
+  float v[NV];
 #pragma unroll
-  for (int i = 0; i < 4 * RW_MAXM; ++i) v[i] = 0.f;
+  for (int i = 0; i < NV; ++i) v[i] = 0.f;
 #pragma unroll 4
   for (int c = lane; c < kc; c += 32) {
-    uint4 wu[4], w2[4];
+    uint4 wu[CW], w2[CW];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < CW; ++j) {
       const int n = n0 + j < p.N ? n0 + j : p.N - 1;  // columns past N compute a copy, never stored
       wu[j] = *(const uint4*)(Bw + (int64_t)n * p.ldb + c * 8);
       w2[j] = B2w ? *(const uint4*)(B2w + (int64_t)n * p.ldb + c * 8) : make_uint4(0, 0, 0, 0);
     }
-    float w[4][8];
+    float w[CW][8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
+    for (int j = 0; j < CW; ++j) {
       const bf16* e = reinterpret_cast<const bf16*>(&wu[j]);
       const bf16* e2 = reinterpret_cast<const bf16*>(&w2[j]);
 #pragma unroll
@@ -283,25 +283,34 @@ static __global__ void __launch_bounds__(256) gemm_rows_kernel(GemmParams p) {
         for (int i = 0; i < 8; ++i) {
           const float x = __bfloat162float(xe[i]);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) v[j * RW_MAXM + m] = fmaf(x, w[j][i], v[j * RW_MAXM + m]);
+          for (int j = 0; j < CW; ++j) v[j * RW_MAXM + m] = fmaf(x, w[j][i], v[j * RW_MAXM + m]);
         }
       }
     }
   }
-  // recursive halving: at offset o a lane keeps the half of its values selected by
-  // (lane & o) and adds its partner's copy of that half
+  // recursive halving over the offsets 16, 8, ...: a lane keeps the half of its values
+  // selected by (lane & o) and adds its partner's copy of that half; once one value is
+  // left, the remaining offsets sum it over the lanes that share its index
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    const bool up = (lane & o) != 0;
+  for (int st = 0; st < 5; ++st) {
+    const int o = 16 >> st;
+    const int cnt = NV >> st;  // values left before this step
+    if (cnt > 1) {
+      const bool up = (lane & o) != 0;
 #pragma unroll
-    for (int i = 0; i < o; ++i) {
-      const float send = up ? v[i] : v[i + o];
-      const float keep = up ? v[i + o] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      for (int i = 0; i < cnt / 2; ++i) {
+        const float send = up ? v[i] : v[i + cnt / 2];
+        const float keep = up ? v[i + cnt / 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
     }
   }
-  const int n = n0 + (lane >> 3), m = lane & 7;
-  if (m < p.M && n < p.N) epi_apply<bf16>(p, z, m, n, v[0]);
+  // lane l holds index (l / (32 / NV)) = column j * 8 + row m
+  const int idx = lane / (32 / NV);
+  const int n = n0 + idx / RW_MAXM, m = idx % RW_MAXM;
+  if (lane % (32 / NV) == 0 && m < p.M && n < p.N) epi_apply<bf16>(p, z, m, n, v[0]);
 }
 
 // ============================================================== tcgen05 engine

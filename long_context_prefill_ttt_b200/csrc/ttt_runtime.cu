@@ -357,7 +357,11 @@ int prime_kernel_attributes() {
   const cudaError_t r[] = {tc_attr<128, false, false>(), tc_attr<256, false, false>(), tc_attr<128, false, true>(),
                            tc_attr<256, false, true>(),  tc_attr<128, true, true>(),   tc_attr<256, true, true>(),
                            attn_mma_attributes<64>(),    attn_mma_attributes<128>(),
-                           cudaFuncSetAttribute(gemm_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           cudaFuncSetAttribute(gemm_rows_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                RW_SMEM_MAX),
+                           cudaFuncSetAttribute(gemm_rows_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                RW_SMEM_MAX),
+                           cudaFuncSetAttribute(gemm_rows_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 RW_SMEM_MAX),
                            cudaFuncSetAttribute(attn_fwd_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 AttnTcCfg<64>::SMEM),
@@ -423,8 +427,16 @@ int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err
     if (p.epi == EPI_QKV_ROPE) q.epi = EPI_STORE;
     const size_t xbytes = (size_t)p.M * p.K * 2;
     if (elem_is_bf16 && p.M <= RW_MAXM && xbytes <= (size_t)RW_SMEM_MAX) {
-      const cudaError_t e = launch_pdl(gemm_rows_kernel, dim3((p.N + RW_COLS - 1) / RW_COLS, p.batch), dim3(256),
-                                       xbytes, st, q);
+      // columns per warp: the most that still gives every SM a CTA (8 warps per CTA)
+      const int64_t slices = p.batch;
+      const int cw = ((int64_t)(p.N + 31) / 32) * slices >= num_sms ? 4 : ((int64_t)(p.N + 15) / 16) * slices >= num_sms ? 2 : 1;
+      cudaError_t e;
+      if (cw == 4)
+        e = launch_pdl(gemm_rows_kernel<4>, dim3((p.N + 31) / 32, p.batch), dim3(256), xbytes, st, q);
+      else if (cw == 2)
+        e = launch_pdl(gemm_rows_kernel<2>, dim3((p.N + 15) / 16, p.batch), dim3(256), xbytes, st, q);
+      else
+        e = launch_pdl(gemm_rows_kernel<1>, dim3((p.N + 7) / 8, p.batch), dim3(256), xbytes, st, q);
       if (e != cudaSuccess) return (int)e;
     } else {
       dim3 grid((p.N + 1) / 2, p.batch);

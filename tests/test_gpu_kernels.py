@@ -277,11 +277,12 @@ def test_attention_forward_and_backward(T, engine, dtype, B, H, hd, n, q0, windo
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("M,N,K,batch", [(1, 768, 768, 8), (8, 2304, 768, 1), (16, 384, 3072, 2), (8, 32000, 768, 1),
-                                         (3, 1000, 3072, 2), (8, 776, 6144, 1)])
+                                         (3, 1000, 3072, 2), (8, 776, 6144, 1), (4, 3072, 1024, 1)])
 def test_skinny_gemm_rows_per_sequence(T, dtype, M, N, K, batch):
     """Decode-sized products (<= 16 rows per slice): shared W plus per-slice dW, residual and GELU epilogues.
-    bf16 with <= 8 rows runs the 32-columns-per-CTA kernel: N off its column grid, and A filling
-    its 96 KB staging buffer (8 x 6144), are among the cases."""
+    bf16 with <= 8 rows runs the few-row kernel with 8, 16 or 32 columns per CTA (all three occur
+    here): N off its column grid, and A filling its 96 KB staging buffer (8 x 6144), are among
+    the cases."""
     A = _rand((batch, M, K), dtype, 31)
     Bs = _rand((1, N, K), dtype, 32, 0.05)
     B2 = _rand((batch, N, K), dtype, 33, 1e-3)
