@@ -60,6 +60,12 @@ struct GemmParams {
   // (consecutive tiles share A rows), 1 = column blocks outer (consecutive tiles share
   // B rows, so a B larger than L2 streams from DRAM once). Set by the host.
   int m_fast;
+  // Optional RMSNorm of the rows of A on the way in: A(m, k) = bf16 of
+  // norm_x(m, k) * rstd_m * norm_g[k] with rstd_m = 1 / sqrt(mean_k norm_x(m, k)^2 + norm_eps),
+  // norm_x fp32 with A's strides (lda, sA). The few-row engine applies it while staging A
+  // (and also writes the normalised rows to A and rstd_m to norm_rstd[z * M + m]); every
+  // other path runs a separate RMSNorm pass into A first.
+  const float* norm_x; const float* norm_g; float norm_eps; float* norm_rstd;
 };
 
 // ============================================================== epilogue (per element)
@@ -242,7 +248,30 @@ __global__ void __launch_bounds__(256) gemm_rows_kernel(GemmParams p) {
   const int z = blockIdx.y;
   const int kc = p.K / 8;
   pdl_wait();  // A (and the epilogue inputs) come from the previous kernel
-  {
+  if (p.norm_x) {  // warp m normalises row m of the slice (RMSNorm) while staging it
+    for (int m = warp; m < p.M; m += 8) {
+      const float* xr = p.norm_x + (int64_t)z * p.sA + (int64_t)m * p.lda;
+      float ss = 0.f;
+      for (int c = lane; c < kc; c += 32) {
+        const float4 a = *(const float4*)(xr + c * 8), b = *(const float4*)(xr + c * 8 + 4);
+        ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w + b.x * b.x + b.y * b.y + b.z * b.z + b.w * b.w;
+      }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      const float rs = rsqrtf(ss / p.K + p.norm_eps);
+      const bool first = blockIdx.x == 0;  // one CTA per slice also writes the normalised rows
+      if (first && lane == 0 && p.norm_rstd) p.norm_rstd[(int64_t)z * p.M + m] = rs;
+      bf16* Ar = (bf16*)p.A + (int64_t)z * p.sA + (int64_t)m * p.lda;
+      for (int c = lane; c < kc; c += 32) {
+        const float4 a = *(const float4*)(xr + c * 8), b = *(const float4*)(xr + c * 8 + 4);
+        const float4 ga = *(const float4*)(p.norm_g + c * 8), gb = *(const float4*)(p.norm_g + c * 8 + 4);
+        const uint4 u = make_uint4(pack_bf16x2(a.x * rs * ga.x, a.y * rs * ga.y), pack_bf16x2(a.z * rs * ga.z, a.w * rs * ga.w),
+                                   pack_bf16x2(b.x * rs * gb.x, b.y * rs * gb.y), pack_bf16x2(b.z * rs * gb.z, b.w * rs * gb.w));
+        xs4[m * kc + c] = u;
+        if (first) *(uint4*)(Ar + c * 8) = u;
+      }
+    }
+  } else {
     const bf16* A = (const bf16*)p.A + (int64_t)z * p.sA;
     for (int i = threadIdx.x; i < p.M * kc; i += 256) {
       const int m = i / kc, c = i - m * kc;

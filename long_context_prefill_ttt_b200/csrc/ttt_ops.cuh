@@ -416,17 +416,64 @@ __global__ void __launch_bounds__(256) ce_kernel(T* __restrict__ z, int V, const
 }
 
 // Greedy choice for decode: argmax (lowest id on ties) unless forced[row] >= 0.
-// Writes chosen id, its loss -log p, and the row's max logit.
+// Writes chosen id, its loss -log p, and the row's max logit. bf16 rows with V % 8 == 0
+// take one pass with 16-byte loads: each thread keeps its (max, lowest index of the
+// max, sum of exp(z - max)) and the block merges them; otherwise two scalar passes.
+__device__ __forceinline__ void amx_merge(float& m, int& i, float& s, float om, int oi, float os) {
+  const float mn = fmaxf(m, om);
+  s = (m == -INFINITY ? 0.f : s * expf(m - mn)) + (om == -INFINITY ? 0.f : os * expf(om - mn));
+  if (om > m || (om == m && oi < i)) i = oi;
+  m = mn;
+}
 template <typename T>
-__global__ void __launch_bounds__(256) argmax_kernel(const T* __restrict__ z, int V,
-                                                     const int32_t* __restrict__ forced, int32_t* chosen,
-                                                     float* loss, float* zmax_out) {
+__global__ void __launch_bounds__(1024) argmax_kernel(const T* __restrict__ z, int V,
+                                                      const int32_t* __restrict__ forced, int32_t* chosen,
+                                                      float* loss, float* zmax_out) {
   const int row = blockIdx.x;
   const T* zr = z + (int64_t)row * V;
   __shared__ float rv[32];
   __shared__ int ri[32];
   __shared__ float rs[32];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
+  if (sizeof(T) == 2 && V % 8 == 0) {
+    float m = -INFINITY, s = 0.f;
+    int bi = 0x7fffffff;
+    for (int c = tid * 8; c < V; c += blockDim.x * 8) {
+      const uint4 u = *(const uint4*)(zr + c);
+      const T* e = reinterpret_cast<const T*>(&u);
+      float x[8], cm = -INFINITY;
+      int ci = 0x7fffffff;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        x[k] = to_f32(e[k]);
+        if (x[k] > cm) { cm = x[k]; ci = c + k; }  // strict: the lowest index of the chunk's max
+      }
+      float cs = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) cs += expf(x[k] - cm);
+      amx_merge(m, bi, s, cm, ci, cs);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      const float om = __shfl_xor_sync(0xffffffffu, m, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      const float os = __shfl_xor_sync(0xffffffffu, s, o);
+      amx_merge(m, bi, s, om, oi, os);
+    }
+    if (lane == 0) { rv[w] = m; ri[w] = bi; rs[w] = s; }
+    __syncthreads();
+    if (tid == 0) {
+      float M = rv[0], S = rs[0];
+      int I = ri[0];
+      for (int i = 1; i < nw; ++i) amx_merge(M, I, S, rv[i], ri[i], rs[i]);
+      const int f = forced ? forced[row] : -1;
+      const int c = (f >= 0 && f < V) ? f : I;
+      chosen[row] = c;
+      loss[row] = M + logf(S) - to_f32(zr[c]);
+      if (zmax_out) zmax_out[row] = M;
+    }
+    return;
+  }
   float best = -INFINITY;
   int bi = 0x7fffffff;
   for (int c = tid; c < V; c += blockDim.x) {

@@ -420,6 +420,24 @@ bool gemm_uses_tc(const GemmParams& p, int elem_is_bf16) {
 // tiles only).
 int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t st, int* err, int num_sms, int engine) {
   if (p.M <= 0 || p.N <= 0 || p.K <= 0 || p.batch <= 0) return 0;
+  if (p.norm_x) {
+    const bool rows_path = engine != GEMM_SIMT && skinny_ok(p, elem_is_bf16) && elem_is_bf16 && p.M <= RW_MAXM &&
+                           (size_t)p.M * p.K * 2 <= (size_t)RW_SMEM_MAX && p.K % 8 == 0 && p.lda % 8 == 0 &&
+                           (p.batch == 1 || p.sA % 8 == 0);
+    if (!rows_path) {  // a separate RMSNorm pass into A, then the product
+      if (p.batch > 1 && p.sA != (int64_t)p.M * p.lda) return (int)cudaErrorInvalidValue;
+      const int rows = p.M * p.batch;
+      const cudaError_t e =
+          elem_is_bf16 ? rmsnorm_fwd_launch<bf16>(p.norm_x, p.lda, p.norm_g, p.norm_eps, rows, p.K, (bf16*)p.A, p.lda,
+                                                  p.norm_rstd, st)
+                       : rmsnorm_fwd_launch<float>(p.norm_x, p.lda, p.norm_g, p.norm_eps, rows, p.K, (float*)p.A,
+                                                   p.lda, p.norm_rstd, st);
+      if (e != cudaSuccess) return (int)e;
+      GemmParams q = p;
+      q.norm_x = nullptr;
+      return gemm_launch(q, elem_is_bf16, st, err, num_sms, engine);
+    }
+  }
   const bool force_simt = engine == GEMM_SIMT;
   if (p.epi == EPI_CE && (force_simt || !gemm_uses_tc(p, elem_is_bf16))) return (int)cudaErrorInvalidValue;
   if (!force_simt && skinny_ok(p, elem_is_bf16)) {
@@ -807,6 +825,19 @@ template <typename T> class Engine : public ttt_handle {
     p.alpha = 1.f; p.epi = epi;
     return p;
   }
+  // r = RMSNorm(x) (gain g) as the A operand of p: in a decode token step the few-row GEMM
+  // normalises while staging its rows (one launch instead of two); elsewhere a separate pass.
+  int norm_into(GemmParams& p, const float* x, const float* g, float* rstd, T* r, int rows) {
+    if (decode_mode) {
+      p.norm_x = x; p.norm_g = g; p.norm_eps = cfg.rms_eps; p.norm_rstd = rstd;
+      return TTT_OK;
+    }
+    ++launches;
+    const cudaError_t e = rmsnorm_fwd_launch<T>(x, d, g, cfg.rms_eps, rows, d, r, d, rstd, st);
+    if (e == cudaSuccess) return TTT_OK;
+    poisoned = true;
+    return fail(this, TTT_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(e));
+  }
   // sum over queries P = q0..q0+n-1 of min(P+1, k): query-key pairs of the window (review eq. (1))
   double attn_pairs(int64_t n, int64_t q0) const {
     double s = 0;
@@ -1108,8 +1139,6 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
                                T* o, float* lse, int n, int64_t q0, bool commit) {
   const int rows = B * n;
   int rc;
-  rmsnorm_fwd_launch<T>((const float*)xin, d, Lw.g_attn, cfg.rms_eps, rows, d, r, d, rstd, st);
-  TTT_LAUNCHED();
   // The chunk's keys and values go to the ring in the RoPE pass when that cannot
   // overwrite a slot this attention still reads: rows of a chunk of n <= b positions
   // and the window before them span n + k - 1 < C positions. (A frozen segment is
@@ -1123,6 +1152,7 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
     pq.rope_pos0 = decode_mode ? 0 : q0;
     pq.rope_pos_dev = decode_mode ? pos_dev : nullptr;
     if (append_in_rope) { pq.rope_ring_k = Lw.ring_k; pq.rope_ring_v = Lw.ring_v; pq.rope_C = C; }
+    if ((rc = norm_into(pq, xin, Lw.g_attn, rstd, r, rows)) != TTT_OK) return rc;
     if ((rc = gemm(pq)) != TTT_OK) return rc;
   }
   if (decode_mode) {
@@ -1196,9 +1226,9 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
 // x += W2 gelu(W1 RMSNorm(x)) (frozen blocks)
 template <typename T> int Engine<T>::frozen_mlp(const LayerDev<T>& Lw, float* x, T* r, T* hid, int rows) {
   int rc;
-  rmsnorm_fwd_launch<T>((const float*)x, d, Lw.g_mlp, cfg.rms_eps, rows, d, r, d, nullptr, st);
-  TTT_LAUNCHED();
-  if ((rc = gemm(gp(rows, h, d, r, d, false, Lw.W1, d, false, hid, h, false, EPI_GELU))) != TTT_OK) return rc;
+  GemmParams p1 = gp(rows, h, d, r, d, false, Lw.W1, d, false, hid, h, false, EPI_GELU);
+  if ((rc = norm_into(p1, x, Lw.g_mlp, nullptr, r, rows)) != TTT_OK) return rc;
+  if ((rc = gemm(p1)) != TTT_OK) return rc;
   GemmParams p = gp(rows, d, h, hid, h, false, Lw.W2, h, false, x, d, true, EPI_RESID);
   p.X = x; p.ldx = d;
   return gemm(p);
@@ -1221,10 +1251,9 @@ template <typename T> int Engine<T>::ttt_forward(int cn, int64_t pos, bool commi
                               commit)) != TTT_OK)
       return rc;
     // TTT-MLP with the fast weights of each sequence (batched over sequences)
-    rmsnorm_fwd_launch<T>((const float*)A.a, d, Lw.g_ttt, cfg.rms_eps, rows, d, A.r2, d, A.rstd2, st);
-    TTT_LAUNCHED();
     GemmParams p = gp(cn, ht, d, A.r2, d, false, Lw.W1t, d, false, A.g, ht, false, EPI_GELU);
     p.batch = B; p.sA = (int64_t)cn * d; p.sD = (int64_t)cn * ht;
+    if ((rc = norm_into(p, A.a, Lw.g_ttt, A.rstd2, A.r2, rows)) != TTT_OK) return rc;
     fast_operand(p, Lw.W1t_init, Lw.W1t, (int64_t)ht * d);
     p.Y = A.u; p.ldy = ht; p.sY = (int64_t)cn * ht;
     if ((rc = gemm(p)) != TTT_OK) return rc;
@@ -1234,11 +1263,9 @@ template <typename T> int Engine<T>::ttt_forward(int cn, int64_t pos, bool commi
     p.X = A.a; p.ldx = d; p.sX = (int64_t)cn * d;
     if ((rc = gemm(p)) != TTT_OK) return rc;
     // static MLP
-    rmsnorm_fwd_launch<T>((const float*)A.m, d, Lw.g_static, cfg.rms_eps, rows, d, A.r3, d,
-                                                         A.rstd3, st);
-    TTT_LAUNCHED();
     p = gp(rows, hs, d, A.r3, d, false, Lw.W1s, d, false, A.gs, hs, false, EPI_GELU);
     p.Y = A.us; p.ldy = hs;
+    if ((rc = norm_into(p, A.m, Lw.g_static, A.rstd3, A.r3, rows)) != TTT_OK) return rc;
     if ((rc = gemm(p)) != TTT_OK) return rc;
     float* xnext = (j + 1 < Lt) ? blk[j + 1].x : y;
     p = gp(rows, d, hs, A.gs, hs, false, Lw.W2s, hs, false, xnext, d, true, EPI_RESID);
@@ -1491,16 +1518,18 @@ template <typename T> int Engine<T>::decode_token_launches(int64_t n, int32_t* o
   TTT_CUDA(cudaMemcpyAsync(tin, xs, (size_t)B * d * 4, cudaMemcpyDeviceToDevice, st));
   gemm_class = PC_GEMM_TTT;
   if ((rc = ttt_forward(1, 0, true)) != TTT_OK) return rc;
-  rmsnorm_fwd_launch<T>((const float*)y, d, g_final, cfg.rms_eps, rows, d, rf, d, rstdf, st);
-  TTT_LAUNCHED();
-  if ((rc = gemm(gp(rows, V, d, rf, d, false, E, d, false, z, V, false, EPI_STORE))) != TTT_OK) return rc;
+  {
+    GemmParams ph = gp(rows, V, d, rf, d, false, E, d, false, z, V, false, EPI_STORE);
+    if ((rc = norm_into(ph, y, g_final, rstdf, rf, rows)) != TTT_OK) return rc;
+    if ((rc = gemm(ph)) != TTT_OK) return rc;
+  }
   const int32_t* fcol = nullptr;
   if (fdev) {
     forced_gather_kernel<<<1, 32 * ((B + 31) / 32), 0, st>>>(fdev, n, B, forced_col, pos_dev, base);
     TTT_LAUNCHED();
     fcol = forced_col;
   }
-  argmax_kernel<T><<<rows, 256, 0, st>>>(z, V, fcol, pend_tok_dev, dec_loss, dec_zmax);
+  argmax_kernel<T><<<rows, 1024, 0, st>>>(z, V, fcol, pend_tok_dev, dec_loss, dec_zmax);
   TTT_LAUNCHED();
   decode_record_kernel<<<1, 32 * ((B + 31) / 32), 0, st>>>(pend_tok_dev, dec_loss, B, n, otok, oloss, pend_tgt, bsz,
                                                            pos_dev, base);
