@@ -387,14 +387,17 @@ __global__ void __launch_bounds__(256) attn_decode_kernel(const T* __restrict__ 
 // HD = 128), form the score by a reduction over the group, and keep a running max, sum
 // and their 8 output elements; the groups of a warp and then the warps are merged at
 // the end. Registers stay few, so the window can be split into many parts; the part
-// results are merged by the last CTA of the (h, b) as in attn_decode_kernel.
+// results are merged by the last CTA of the (h, b) as in attn_decode_kernel. The ring is
+// read through plain (coherent) loads: this kernel may write its newest row itself.
 template <int HD>
 __global__ void __launch_bounds__(128) attn_decode_rows_kernel(const bf16* __restrict__ q, int64_t ldq,
-                                                               const bf16* __restrict__ ring_k,
-                                                               const bf16* __restrict__ ring_v, int C, int d,
+                                                               const bf16* ring_k, const bf16* ring_v, int C, int d,
                                                                int window, const int64_t* __restrict__ pos,
                                                                float scale, bf16* __restrict__ out, int64_t ldo,
-                                                               float* __restrict__ part, int* __restrict__ ticket) {
+                                                               float* __restrict__ part, int* __restrict__ ticket,
+                                                               const float2* __restrict__ rope_lo,
+                                                               const float2* __restrict__ rope_hi,
+                                                               bf16* __restrict__ ring_k_w, bf16* __restrict__ ring_v_w) {
   constexpr int LPK = HD / 8;    // lanes per key row
   constexpr int KPW = 32 / LPK;  // keys per warp step
   constexpr int U = 4;           // steps whose loads are issued together
@@ -409,13 +412,58 @@ __global__ void __launch_bounds__(128) attn_decode_rows_kernel(const bf16* __res
   const int64_t span = (P - lo + nz) / nz;
   const int64_t zlo = lo + z * span;
   const int64_t zhi = (zlo + span - 1 < P) ? zlo + span - 1 : P;
+  // With rope_lo set, q and k of this position arrive unrotated: each lane rotates its
+  // 8 elements of q (pairs (i, i + HD/2), the partner chunk in lane e ^ LPK/2) at position
+  // P from the angle tables, lo[P & 1023] and hi[P >> 10] combined by the angle-addition
+  // formulas; the CTA whose part holds key P also writes the rotated k and the v of this
+  // position to the ring (slot P mod C) before any of its warps reads the ring.
+  const int half_e = e & (LPK / 2 - 1);  // chunk index within its half of the head
+  float cs[8], sn[8];
+  if (rope_lo) {
+    const float2* a2 = rope_lo + (P & 1023) * (HD / 2) + half_e * 8;
+    const float2* b2 = rope_hi + (P >> 10) * (HD / 2) + half_e * 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float2 a = a2[i], bb = b2[i];
+      cs[i] = a.x * bb.x - a.y * bb.y;
+      sn[i] = a.y * bb.x + a.x * bb.y;
+    }
+  }
+  auto rotate = [&](const uint4& own, const uint4& mate, float* outv) {  // this lane's 8 rotated elements
+    const bf16* x = reinterpret_cast<const bf16*>(&own);
+    const bf16* y = reinterpret_cast<const bf16*>(&mate);
+    const bool first_half = e < LPK / 2;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float u = __bfloat162float(x[i]), v = __bfloat162float(y[i]);
+      outv[i] = first_half ? u * cs[i] - v * sn[i] : u * cs[i] + v * sn[i];
+    }
+  };
   float qv[8];
   {
     const uint4 u = *(const uint4*)(q + (int64_t)b * ldq + h * HD + e * 8);
-    const bf16* qe = reinterpret_cast<const bf16*>(&u);
+    if (rope_lo) {
+      const uint4 mate = *(const uint4*)(q + (int64_t)b * ldq + h * HD + (e ^ (LPK / 2)) * 8);
+      rotate(u, mate, qv);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) qv[i] = __bfloat162float(qe[i]) * scale;
+      for (int i = 0; i < 8; ++i) qv[i] *= scale;
+    } else {
+      const bf16* qe = reinterpret_cast<const bf16*>(&u);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) qv[i] = __bfloat162float(qe[i]) * scale;
+    }
   }
+  if (rope_lo && ring_k_w && warp == 0 && g == 0 && P >= zlo && P <= zhi) {
+    const bf16* kq = q + (int64_t)b * ldq + d + h * HD;  // k follows q in the q|k|v row
+    const uint4 ku = *(const uint4*)(kq + e * 8), km = *(const uint4*)(kq + (e ^ (LPK / 2)) * 8);
+    float kr[8];
+    rotate(ku, km, kr);
+    const int64_t off = ((int64_t)b * C + P % C) * d + h * HD + e * 8;
+    *(uint4*)(ring_k_w + off) = make_uint4(pack_bf16x2(kr[0], kr[1]), pack_bf16x2(kr[2], kr[3]),
+                                           pack_bf16x2(kr[4], kr[5]), pack_bf16x2(kr[6], kr[7]));
+    *(uint4*)(ring_v_w + off) = *(const uint4*)(kq + d + e * 8);
+  }
+  if (rope_lo) __syncthreads();  // the ring row of P is in place for every warp of this CTA
   const bf16* Kb = ring_k + (int64_t)b * C * d + h * HD + e * 8;
   const bf16* Vb = ring_v + (int64_t)b * C * d + h * HD + e * 8;
   float m = -INFINITY, l = 0.f, acc[8];

@@ -1145,28 +1145,34 @@ int Engine<T>::attention_block(const LayerDev<T>& Lw, int layer, float* xin, flo
   // longer than the ring and appends after its attention.) Decode appends its one
   // position there too, then attends over the window entirely from the ring.
   const bool append_in_rope = commit && (decode_mode || n <= bsz);
+  // A decode step on the lane-group attention kernel rotates q and k and appends k, v to
+  // the ring inside that kernel: the projection then stores q|k|v as they are.
+  const bool rope_in_attn = decode_mode && is_bf16 && (hd == 64 || hd == 128);
   {  // q|k|v = r Wqkv^T with RoPE applied to q and k in the GEMM epilogue
-    GemmParams pq = gp(rows, 3 * d, d, r, d, false, Lw.Wqkv, d, false, qkv, 3 * d, false, EPI_QKV_ROPE);
+    GemmParams pq = gp(rows, 3 * d, d, r, d, false, Lw.Wqkv, d, false, qkv, 3 * d, false,
+                       rope_in_attn ? EPI_STORE : EPI_QKV_ROPE);
     pq.rope_lo = rope_lo; pq.rope_hi = rope_hi; pq.rope_hd = hd; pq.rope_cols = 2 * d;
     pq.rope_n = decode_mode ? 1 : n;
     pq.rope_pos0 = decode_mode ? 0 : q0;
     pq.rope_pos_dev = decode_mode ? pos_dev : nullptr;
-    if (append_in_rope) { pq.rope_ring_k = Lw.ring_k; pq.rope_ring_v = Lw.ring_v; pq.rope_C = C; }
+    if (append_in_rope && !rope_in_attn) { pq.rope_ring_k = Lw.ring_k; pq.rope_ring_v = Lw.ring_v; pq.rope_C = C; }
     if ((rc = norm_into(pq, xin, Lw.g_attn, rstd, r, rows)) != TTT_OK) return rc;
     if ((rc = gemm(pq)) != TTT_OK) return rc;
   }
   if (decode_mode) {
     const float scale = 1.0f / sqrtf((float)hd);
     const dim3 dg(H, B, dec_split);  // the window in dec_split parts, merged by the last CTA of each (head, sequence)
-    if (is_bf16 && (hd == 64 || hd == 128)) {
+    if (rope_in_attn) {
       if (hd == 64)
         attn_decode_rows_kernel<64><<<dg, 128, 0, st>>>((const bf16*)qkv, 3 * d, (const bf16*)Lw.ring_k,
                                                         (const bf16*)Lw.ring_v, C, d, kwin, pos_dev, scale,
-                                                        (bf16*)o, d, dec_part, dec_ticket);
+                                                        (bf16*)o, d, dec_part, dec_ticket, rope_lo, rope_hi,
+                                                        (bf16*)Lw.ring_k, (bf16*)Lw.ring_v);
       else
         attn_decode_rows_kernel<128><<<dg, 128, 0, st>>>((const bf16*)qkv, 3 * d, (const bf16*)Lw.ring_k,
                                                          (const bf16*)Lw.ring_v, C, d, kwin, pos_dev, scale,
-                                                         (bf16*)o, d, dec_part, dec_ticket);
+                                                         (bf16*)o, d, dec_part, dec_ticket, rope_lo, rope_hi,
+                                                         (bf16*)Lw.ring_k, (bf16*)Lw.ring_v);
       TTT_LAUNCHED();
       GemmParams pd = gp(rows, d, d, o, d, false, Lw.Wo, d, false, xout, d, true, EPI_RESID);
       pd.X = xin; pd.ldx = d;
