@@ -7,12 +7,13 @@
 //   warp 0     TMA: Q once, then K and V tiles into separate rings (a K stage is
 //              freed as soon as its Q K^T is done, a V stage after its P V);
 //   warp 1     MMA issue (one thread): S_j = Q K_j^T into one of two TMEM S
-//              buffers, then O += P_{j-1} V_{j-1} (P from shared memory, V as an
-//              MN-major operand) into the TMEM O accumulator;
+//              buffers, then O += P_{j-1} V_{j-1} (P read from TMEM as the A
+//              operand, V as an MN-major operand) into the TMEM O accumulator;
+//              the completion of P_j V_j frees S buffer j % 2 for S_{j+2};
 //   warps 2-5  softmax, one thread per query row (TMEM lane): read S_j, mask on
 //              diagonal / window-edge tiles, online softmax in the log2 domain,
-//              write P_j (bf16) to shared memory in the 128-byte-swizzled layout
-//              the MMA reads. The running maximum is raised only when a row's
+//              write P_j (bf16 pairs) over the scores in S_j's TMEM columns. The
+//              running maximum is raised only when a row's
 //              maximum grows by more than 8 (a factor 256): then the thread's O
 //              row is rescaled in TMEM after the previous P·V has completed.
 //              Exponents stay below 2^8, so bf16 P and fp32 sums stay exact
@@ -91,7 +92,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);  mbar_init(&s_free[s], 4);
+      mbar_init(&s_full[s], 1);  mbar_init(&s_free[s], 1);
       mbar_init(&p_full[s], 4);  mbar_init(&pv_done[s], 1);
     }
     mbar_init(o_done, 1);
@@ -162,15 +163,14 @@ __global__ void __launch_bounds__(192, 1)
         if (!mbar_wait(&v_full[vs], (i / Cf::VST) & 1, err, DEV_TIMEOUT_FULL)) return false;
         if (!mbar_wait(&p_full[s], (i >> 1) & 1, err, DEV_TIMEOUT_FULL)) return false;
         tc_fence_after();
-        const uint32_t sP = smem_u32(sm + Cf::OFF_P0 + s * Cf::PB);
         const uint32_t sV = smem_u32(sm + Cf::OFF_V0 + vs * Cf::KVB);
 #pragma unroll
-        for (int kk = 0; kk < Cf::BN / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(sP + (kk >> 2) * (128 * 128) + (kk & 3) * 32, 16, 1024);
+        for (int kk = 0; kk < Cf::BN / 16; ++kk) {  // A = P_i from TMEM (in the columns of S_i)
           const uint64_t bd = smem_desc_sw128(sV + kk * 2048, Cf::BN * 128, 1024);
-          tc_mma_f16(tmem + Cf::O_COL, ad, bd, idO, (i | kk) ? 1u : 0u);
+          tc_mma_f16_ta(tmem + Cf::O_COL, tmem + Cf::S_COL + s * Cf::BN + kk * 8, bd, idO, (i | kk) ? 1u : 0u);
         }
         tc_commit(&pv_done[s]);
+        tc_commit(&s_free[s]);  // P_i is consumed: S_{i+2} may overwrite the buffer
         tc_commit(&v_empty[vs]);
         return true;
       };
@@ -233,9 +233,6 @@ __global__ void __launch_bounds__(192, 1)
           tmem_ld32_nowait(tmem + lane_base + Cf::S_COL + s * Cf::BN + c * 32, vr + c * 32);
         tmem_ld_wait();
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[s]);
       const bool need_mask = (j0 + Cf::BN - 1 > P0) || (j0 < Plast - p.window + 1);
       if (need_mask) {  // diagonal / window-edge tile: branch-free per-element mask
         const int64_t lo_key = P - p.window + 1;
@@ -277,13 +274,13 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       l *= factor;
-      // the P buffer s was last read by P_{j-2} V_{j-2}
-      if (j >= 2 && !mbar_wait(&pv_done[s], ((j - 2) >> 1) & 1, err, DEV_TIMEOUT_ACC)) { ok = false; break; }
+      // P_j (bf16 pairs in key order) into the first BN/2 columns of S_j's TMEM buffer,
+      // whose scores are all in registers: the P·V MMA takes it as its A operand
       const float nbase = m_used == -INFINITY ? 0.f : -m_used;
-      uint8_t* prow = sm + Cf::OFF_P0 + s * Cf::PB + r * 128;
       float ls8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int kb = 0; kb < Cf::BN / 64; ++kb) {
+        float pw[32];  // 64 P values of this row as 32 bf16 pairs
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
           float e8[8];
@@ -292,14 +289,13 @@ __global__ void __launch_bounds__(192, 1)
             e8[e] = ex2_tc(fmaf(v[kb * 64 + cc * 8 + e], sc, nbase));  // exp2(s*sc - m): masked -inf -> 0
             ls8[e] += e8[e];
           }
-          const uint4 pk = make_uint4(pack_bf16x2(e8[0], e8[1]), pack_bf16x2(e8[2], e8[3]),
-                                      pack_bf16x2(e8[4], e8[5]), pack_bf16x2(e8[6], e8[7]));
-          *(uint4*)(prow + kb * (Cf::BM * 128) + ((cc ^ (r & 7)) << 4)) = pk;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) pw[cc * 4 + e] = __uint_as_float(pack_bf16x2(e8[2 * e], e8[2 * e + 1]));
         }
+        tmem_st32(tmem + lane_base + Cf::S_COL + s * Cf::BN + kb * 32, pw);
       }
       l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
-      fence_proxy_async();  // P (generic-proxy stores) visible to the tensor core
-      tc_fence_before();
+      tc_fence_before();  // P_j's TMEM stores (waited for) before the MMA warp's P·V
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[s]);
     }
