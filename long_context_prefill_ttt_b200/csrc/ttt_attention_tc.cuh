@@ -332,10 +332,10 @@ __global__ void __launch_bounds__(192, 1)
 // each row's whole window (ring and current rows). Per tile j: S = Q K^T and
 // dP = dO V^T into one of two TMEM buffers (MMA warp); four warps form
 // dS = P (dP - D) with P = exp(S*scale - lse) from the forward's log-sum-exp and
-// write dS (bf16) to one of two shared-memory buffers; the MMA warp accumulates
-// dQ += dS K in TMEM (the K tile read again as an MN-major operand). With S/dP and
-// dS double-buffered, S_{j+1} and dP_{j+1} run on the tensor cores while the
-// warps form dS_j. dQ is scaled by 1/sqrt(hd) on the way out. The four warps first
+// write dS (bf16 pairs) over the scores in the buffer's S columns; the MMA warp
+// accumulates dQ += dS K in TMEM (dS as the A operand from TMEM, the K tile read again
+// as an MN-major operand), and its completion frees the buffer for tile j+2. With two
+// buffers, S_{j+1} and dP_{j+1} run on the tensor cores while the warps form dS_j. dQ is scaled by 1/sqrt(hd) on the way out. The four warps first
 // copy their rows of Q and dO from shared memory into TMEM, where the S and dP MMAs
 // take them as the A operand.
 // TMEM: S0 [0,64), dP0 [64,128), S1 [128,192), dP1 [192,256), dQ [256, 256+HD),
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&sp_full[s], 1); mbar_init(&sp_free[s], 4);
+      mbar_init(&sp_full[s], 1); mbar_init(&sp_free[s], 1);
       mbar_init(&ds_full[s], 4); mbar_init(&ds_free[s], 1);
     }
     mbar_init(dq_done, 1);
@@ -460,15 +460,13 @@ __global__ void __launch_bounds__(192, 1)
         const int s = i & 1, ks = i % 3;
         if (!mbar_wait(&ds_full[s], (i >> 1) & 1, err, DEV_TIMEOUT_FULL)) return false;
         tc_fence_after();
-        const uint32_t sdS = smem_u32(sm + Cf::OFF_DS + s * Cf::DSB);
         const uint32_t sK = smem_u32(sm + Cf::OFF_K0 + ks * Cf::KVB);
 #pragma unroll
-        for (int kk = 0; kk < Cf::BN / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(sdS + kk * 32, 16, 1024);
+        for (int kk = 0; kk < Cf::BN / 16; ++kk) {  // A = dS_i from TMEM (in the columns of S_i)
           const uint64_t bd = smem_desc_sw128(sK + kk * 2048, Cf::BN * 128, 1024);
-          tc_mma_f16(tmem + Cf::DQ_COL, ad, bd, idQ, (i | kk) ? 1u : 0u);
+          tc_mma_f16_ta(tmem + Cf::DQ_COL, tmem + Cf::s_col(s) + kk * 8, bd, idQ, (i | kk) ? 1u : 0u);
         }
-        tc_commit(&ds_free[s]);
+        tc_commit(&sp_free[s]);  // dS_i is consumed: S_{i+2} and dP_{i+2} may overwrite the buffer
         tc_commit(&k_empty[ks]);
         return true;
       };
@@ -565,8 +563,7 @@ __global__ void __launch_bounds__(192, 1)
       const int s = j & 1;
       const int64_t j0 = jt0 + (int64_t)j * Cf::BN;
       const bool need_mask = (j0 + Cf::BN - 1 > P0) || (j0 < Plast - p.window + 1);
-      if (!mbar_wait(&sp_full[s], (j >> 1) & 1, err, DEV_TIMEOUT_ACC) ||
-          !mbar_wait(&ds_free[s], ((j >> 1) & 1) ^ 1, err, DEV_TIMEOUT_ACC)) {
+      if (!mbar_wait(&sp_full[s], (j >> 1) & 1, err, DEV_TIMEOUT_ACC)) {
         ok = false;
         break;
       }
@@ -577,10 +574,8 @@ __global__ void __launch_bounds__(192, 1)
       tmem_ld32_nowait(tmem + lane_base + Cf::dp_col(s), dr);
       tmem_ld32_nowait(tmem + lane_base + Cf::dp_col(s) + 32, dr + 32);
       tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sp_free[s]);  // S/dP buffer s may be overwritten by tile j+2
-      uint8_t* drow = sm + Cf::OFF_DS + s * Cf::DSB + r * 128;
+      // dS_j (bf16 pairs in key order) over the scores in the first BN/2 columns of S_j
+      float dsw[Cf::BN / 2];
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc) {
         float ds[8];
@@ -594,11 +589,11 @@ __global__ void __launch_bounds__(192, 1)
           }
           ds[e] = pr * (__uint_as_float(dr[c]) - Dr);
         }
-        *(uint4*)(drow + ((cc ^ (r & 7)) << 4)) =
-            make_uint4(pack_bf16x2(ds[0], ds[1]), pack_bf16x2(ds[2], ds[3]), pack_bf16x2(ds[4], ds[5]),
-                       pack_bf16x2(ds[6], ds[7]));
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dsw[cc * 4 + e] = __uint_as_float(pack_bf16x2(ds[2 * e], ds[2 * e + 1]));
       }
-      fence_proxy_async();
+      tmem_st32(tmem + lane_base + Cf::s_col(s), dsw);
+      tc_fence_before();  // dS_j's TMEM stores (waited for) before the MMA warp's dQ product
       __syncwarp();
       if (lane == 0) mbar_arrive(&ds_full[s]);
     }
