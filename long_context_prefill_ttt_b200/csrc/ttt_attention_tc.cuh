@@ -32,15 +32,13 @@ namespace ttt {
 
 template <int HD> struct AttnTcCfg {
   static constexpr int BM = 128, BN = 128;
-  static constexpr int KST = HD == 64 ? 3 : 2;  // K stages
+  static constexpr int KST = HD == 64 ? 3 : 2;  // K stages (a third at HD = 128 measured 1% slower)
   static constexpr int VST = HD == 64 ? 3 : 2;  // V stages
   static constexpr int QB = BM * HD * 2;      // Q tile bytes
   static constexpr int KVB = BN * HD * 2;     // K (and V) tile bytes
-  static constexpr int PB = BM * BN * 2;      // P tile bytes
   static constexpr int OFF_K0 = QB;
   static constexpr int OFF_V0 = OFF_K0 + KST * KVB;
-  static constexpr int OFF_P0 = OFF_V0 + VST * KVB;
-  static constexpr int OFF_BAR = OFF_P0 + 2 * PB;
+  static constexpr int OFF_BAR = OFF_V0 + VST * KVB;  // P lives in TMEM
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr uint32_t S_COL = 0, O_COL = 256;
   static constexpr uint32_t Q_COL = 384;  // Q as the A operand of S, copied once into TMEM
@@ -345,12 +343,10 @@ template <int HD> struct AttnDqCfg {
   static constexpr int KST = 3, VST = 3;
   static constexpr int QB = BM * HD * 2;
   static constexpr int KVB = BN * HD * 2;
-  static constexpr int DSB = BM * BN * 2;
   static constexpr int OFF_DO = QB;
   static constexpr int OFF_K0 = 2 * QB;
   static constexpr int OFF_V0 = OFF_K0 + KST * KVB;
-  static constexpr int OFF_DS = OFF_V0 + VST * KVB;
-  static constexpr int OFF_BAR = OFF_DS + 2 * DSB;
+  static constexpr int OFF_BAR = OFF_V0 + VST * KVB;  // dS lives in TMEM
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr uint32_t DQ_COL = 256;
   // Q and dO as the A operands of S and dP, copied once into TMEM (bf16 pairs, one row
@@ -633,9 +629,10 @@ __global__ void __launch_bounds__(192, 1)
 // dimension. Per query block j: S^T = K Q_j^T and dP^T = V dO_j^T into one of two
 // TMEM buffers (MMA warp); four warps (one key row each) form P^T = exp(S^T*scale
 // - lse) and dS^T = P^T (dP^T - D) with the per-query lse and D read from shared
-// memory, and write both (bf16) to one of two shared-memory buffers; the MMA warp
-// accumulates dV += P^T dO_j and dK += dS^T Q_j in TMEM (Q_j and dO_j read again as
-// MN-major operands). Query rows past the sequence end get lse = +inf, so their
+// memory, and write both (bf16 pairs) over S^T and dP^T in TMEM; the MMA warp
+// accumulates dV += P^T dO_j and dK += dS^T Q_j in TMEM (P^T and dS^T as A operands
+// from TMEM, Q_j and dO_j read again as MN-major operands), and its completion frees
+// the buffer for block j+2. Query rows past the sequence end get lse = +inf, so their
 // P and dS vanish. dK is scaled by 1/sqrt(hd) on the way out.
 // TMEM: dV [0,HD), dK [128,128+HD), S^T_b [256+128b, 256+128b+64), dP^T_b next 64.
 template <int HD> struct AttnDkvCfg {
@@ -643,13 +640,10 @@ template <int HD> struct AttnDkvCfg {
   static constexpr int QST = 3;                 // Q / dO stages
   static constexpr int KVB = BK * HD * 2;       // K (and V) tile bytes
   static constexpr int QB = BQ * HD * 2;        // Q (and dO) block bytes
-  static constexpr int PB = BK * BQ * 2;        // P^T (and dS^T) tile bytes
   static constexpr int OFF_V = KVB;
   static constexpr int OFF_Q0 = 2 * KVB;
   static constexpr int OFF_DO0 = OFF_Q0 + QST * QB;
-  static constexpr int OFF_P0 = OFF_DO0 + QST * QB;
-  static constexpr int OFF_DS0 = OFF_P0 + 2 * PB;
-  static constexpr int OFF_LD = OFF_DS0 + 2 * PB;  // [2][ -lse*log2e (64) | D (64) ] floats
+  static constexpr int OFF_LD = OFF_DO0 + QST * QB;  // [2][ -lse*log2e (64) | D (64) ] floats (P^T, dS^T in TMEM)
   static constexpr int OFF_BAR = OFF_LD + 2 * 2 * BQ * 4;
   static constexpr int SMEM = OFF_BAR + 256 + 1024;
   static constexpr uint32_t DV_COL = 0, DK_COL = 128;
@@ -693,7 +687,7 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(kv_full, 1);
     for (int s = 0; s < Cf::QST; ++s) { mbar_init(&q_full[s], 1); mbar_init(&q_empty[s], 1); }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&sp_full[s], 1); mbar_init(&sp_free[s], 4);
+      mbar_init(&sp_full[s], 1); mbar_init(&sp_free[s], 1);
       mbar_init(&pd_full[s], 4); mbar_init(&pd_free[s], 1);
     }
     mbar_init(acc_done, 1);
@@ -741,16 +735,15 @@ __global__ void __launch_bounds__(192, 1)
         const int s = i & 1, qs = i % Cf::QST;
         if (!mbar_wait(&pd_full[s], (i >> 1) & 1, err, DEV_TIMEOUT_FULL)) return false;
         tc_fence_after();
-        const uint32_t sP = smem_u32(sm + Cf::OFF_P0 + s * Cf::PB), sdS = smem_u32(sm + Cf::OFF_DS0 + s * Cf::PB);
         const uint32_t sQ = smem_u32(sm + Cf::OFF_Q0 + qs * Cf::QB), sdO = smem_u32(sm + Cf::OFF_DO0 + qs * Cf::QB);
 #pragma unroll
-        for (int kk = 0; kk < Cf::BQ / 16; ++kk) {
-          tc_mma_f16(tmem + Cf::DV_COL, smem_desc_sw128(sP + kk * 32, 16, 1024),
-                     smem_desc_sw128(sdO + kk * 2048, Cf::BQ * 128, 1024), idA, (i | kk) ? 1u : 0u);
-          tc_mma_f16(tmem + Cf::DK_COL, smem_desc_sw128(sdS + kk * 32, 16, 1024),
-                     smem_desc_sw128(sQ + kk * 2048, Cf::BQ * 128, 1024), idA, (i | kk) ? 1u : 0u);
+        for (int kk = 0; kk < Cf::BQ / 16; ++kk) {  // A = P^T and dS^T from TMEM (over S^T and dP^T)
+          tc_mma_f16_ta(tmem + Cf::DV_COL, tmem + Cf::s_col(s) + kk * 8,
+                        smem_desc_sw128(sdO + kk * 2048, Cf::BQ * 128, 1024), idA, (i | kk) ? 1u : 0u);
+          tc_mma_f16_ta(tmem + Cf::DK_COL, tmem + Cf::dp_col(s) + kk * 8,
+                        smem_desc_sw128(sQ + kk * 2048, Cf::BQ * 128, 1024), idA, (i | kk) ? 1u : 0u);
         }
-        tc_commit(&pd_free[s]);
+        tc_commit(&sp_free[s]);  // P^T and dS^T are consumed: block i+2 may overwrite the buffer
         tc_commit(&q_empty[qs]);
         return true;
       };
@@ -808,8 +801,7 @@ __global__ void __launch_bounds__(192, 1)
       const bool need_mask = (i0 < k0 + Cf::BK - 1) || (i0 + Cf::BQ - 1 - k0 > p.window - 1);
       // after a timed-out wait the loop still runs to its end (without waiting or
       // computing) so that all four warps meet at every named barrier
-      if (ok) ok = mbar_wait(&sp_full[s], (j >> 1) & 1, err, DEV_TIMEOUT_ACC) &&
-                   mbar_wait(&pd_free[s], ((j >> 1) & 1) ^ 1, err, DEV_TIMEOUT_ACC);
+      if (ok) ok = mbar_wait(&sp_full[s], (j >> 1) & 1, err, DEV_TIMEOUT_ACC);
       if (ok) {
         tc_fence_after();
         uint32_t sr[64], dr[64];
@@ -818,13 +810,9 @@ __global__ void __launch_bounds__(192, 1)
         tmem_ld32_nowait(tmem + lane_base + Cf::dp_col(s), dr);
         tmem_ld32_nowait(tmem + lane_base + Cf::dp_col(s) + 32, dr + 32);
         tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sp_free[s]);  // S^T/dP^T buffer s may be overwritten by block j+2
         const float* nl = ldbuf + s * 2 * Cf::BQ;
         const float* dd = nl + Cf::BQ;
-        uint8_t* prow = sm + Cf::OFF_P0 + s * Cf::PB + r * 128;
-        uint8_t* drow = sm + Cf::OFF_DS0 + s * Cf::PB + r * 128;
+        float pw[Cf::BQ / 2], dw[Cf::BQ / 2];  // P^T and dS^T of this key row as bf16 pairs
   #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
           const float4 nl0 = *(const float4*)(nl + cc * 8), nl1 = *(const float4*)(nl + cc * 8 + 4);
@@ -843,13 +831,16 @@ __global__ void __launch_bounds__(192, 1)
             pv[e] = pr;
             ds[e] = pr * (__uint_as_float(dr[c]) - dv[e]);
           }
-          const int sw = (cc ^ (r & 7)) << 4;
-          *(uint4*)(prow + sw) = make_uint4(pack_bf16x2(pv[0], pv[1]), pack_bf16x2(pv[2], pv[3]),
-                                            pack_bf16x2(pv[4], pv[5]), pack_bf16x2(pv[6], pv[7]));
-          *(uint4*)(drow + sw) = make_uint4(pack_bf16x2(ds[0], ds[1]), pack_bf16x2(ds[2], ds[3]),
-                                            pack_bf16x2(ds[4], ds[5]), pack_bf16x2(ds[6], ds[7]));
+  #pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            pw[cc * 4 + e] = __uint_as_float(pack_bf16x2(pv[2 * e], pv[2 * e + 1]));
+            dw[cc * 4 + e] = __uint_as_float(pack_bf16x2(ds[2 * e], ds[2 * e + 1]));
+          }
         }
-        fence_proxy_async();
+        // over the scores in TMEM (both read above): the MMA warp takes them as A operands
+        tmem_st32(tmem + lane_base + Cf::s_col(s), pw);
+        tmem_st32(tmem + lane_base + Cf::dp_col(s), dw);
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&pd_full[s]);
       }
