@@ -51,6 +51,30 @@ int ttt_k_gemm(int32_t elem_dtype, int32_t M, int32_t N, int32_t K, int32_t batc
                int64_t sD, int32_t d_f32, const void* X, int64_t ldx, int64_t sX, void* Y, int64_t ldy, int64_t sY,
                float alpha, int32_t epi, int32_t engine, void* stream);
 
+/* One product of ttt_k_gemm_pair: the arguments of ttt_k_gemm with the same meaning. */
+typedef struct {
+  int32_t M, N, K, batch;
+  const void* A; int64_t lda, sA; int32_t a_mn;
+  const void* B; int64_t ldb, sB; int32_t b_mn;
+  const void* B2; int64_t sB2;
+  void* D; int64_t ldd, sD; int32_t d_f32;
+  const void* X; int64_t ldx, sX;
+  void* Y; int64_t ldy, sY;
+  float alpha; int32_t epi;
+} ttt_gemm_desc;
+
+/* Two independent products (no operand of one is an output of the other; their outputs
+ * do not overlap), enqueued on one stream. Where both are bf16 tcgen05 products with the
+ * same a_mn/b_mn and N % 256 == 0 they share one persistent single-CTA launch of 128 x 256
+ * tiles, the second product's tiles following the first's, so that one product's
+ * epilogues overlap the other's mainloop (the two weight-gradient SGD steps of an adaptive
+ * MLP block); otherwise each runs as ttt_k_gemm(engine 0) would. Each result equals the
+ * single-CTA engine's (engine 3) up to the tile width it picks. The descriptors are read
+ * during the call only (the caller keeps ownership); device pointers as in ttt_k_gemm.
+ * TTT_ERR_INVALID_ARG for a descriptor ttt_k_gemm would reject, TTT_ERR_CUDA on a launch
+ * error. */
+int ttt_k_gemm_pair(int32_t elem_dtype, const ttt_gemm_desc* first, const ttt_gemm_desc* second, void* stream);
+
 /* LM head and softmax cross-entropy, chunked over the vocabulary (summary, loss l_t;
  * technical review §3, eq. (3)), bf16 on tcgen05. r [M][d] (final-norm output rows),
  * E [V][d] (tied embedding), targets [M] int32 in [0, V).

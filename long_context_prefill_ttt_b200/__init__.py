@@ -50,6 +50,18 @@ class ttt_weights(ctypes.Structure):
                 ("values_dtype", ctypes.c_int32), ("ptr_kind", ctypes.c_int32)]
 
 
+class ttt_gemm_desc(ctypes.Structure):
+    """One product of ttt_k_gemm_pair (the arguments of ttt_k_gemm)."""
+    _fields_ = [("M", ctypes.c_int32), ("N", ctypes.c_int32), ("K", ctypes.c_int32), ("batch", ctypes.c_int32),
+                ("A", ctypes.c_void_p), ("lda", ctypes.c_int64), ("sA", ctypes.c_int64), ("a_mn", ctypes.c_int32),
+                ("B", ctypes.c_void_p), ("ldb", ctypes.c_int64), ("sB", ctypes.c_int64), ("b_mn", ctypes.c_int32),
+                ("B2", ctypes.c_void_p), ("sB2", ctypes.c_int64),
+                ("D", ctypes.c_void_p), ("ldd", ctypes.c_int64), ("sD", ctypes.c_int64), ("d_f32", ctypes.c_int32),
+                ("X", ctypes.c_void_p), ("ldx", ctypes.c_int64), ("sX", ctypes.c_int64),
+                ("Y", ctypes.c_void_p), ("ldy", ctypes.c_int64), ("sY", ctypes.c_int64),
+                ("alpha", ctypes.c_float), ("epi", ctypes.c_int32)]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with `python -m long_context_prefill_ttt_b200.build`")
@@ -72,6 +84,7 @@ def _load():
         "ttt_version": (ctypes.c_char_p, []),
         "ttt_k_gemm": (ctypes.c_int, [I32, I32, I32, I32, I32, VP, I64, I64, I32, VP, I64, I64, I32, VP, I64, VP,
                                       I64, I64, I32, VP, I64, I64, VP, I64, I64, F, I32, I32, VP]),
+        "ttt_k_gemm_pair": (ctypes.c_int, [I32, P(ttt_gemm_desc), P(ttt_gemm_desc), VP]),
         "ttt_k_attention_fwd": (ctypes.c_int, [I32, I32, I32, I32, I32, I64, I32, VP, VP, VP, I32, VP, VP, I32, VP]),
         "ttt_k_attention_bwd": (ctypes.c_int, [I32, I32, I32, I32, I32, I64, I32, VP, VP, VP, I32, VP, VP, VP, VP,
                                                VP, I32, VP]),
@@ -386,10 +399,9 @@ def _dtype_code(t):
     return TTT_BF16 if t.dtype == torch.bfloat16 else TTT_FP32
 
 
-def ttt_k_gemm(A, B, D, M, N, K, *, batch=1, lda=None, sA=0, a_mn=False, ldb=None, sB=0, b_mn=False, B2=None,
-               sB2=0, ldd=None, sD=0, X=None, ldx=0, sX=0, Y=None, ldy=0, sY=0, alpha=1.0, epi=EPI_STORE,
-               engine=ENGINE_AUTO, stream=None):
-    """Enqueue one contraction on device tensors (see include/ttt_kernels.h)."""
+def _gemm_desc(A, B, D, M, N, K, *, batch=1, lda=None, sA=0, a_mn=False, ldb=None, sB=0, b_mn=False, B2=None,
+               sB2=0, ldd=None, sD=0, X=None, ldx=0, sX=0, Y=None, ldy=0, sY=0, alpha=1.0, epi=EPI_STORE):
+    """Checks one product's device tensors against its sizes; returns its ttt_gemm_desc."""
     torch = _torch()
     lda = lda if lda is not None else (M if a_mn else K)
     ldb = ldb if ldb is not None else (N if b_mn else K)
@@ -411,14 +423,32 @@ def ttt_k_gemm(A, B, D, M, N, K, *, batch=1, lda=None, sA=0, a_mn=False, ldb=Non
     if Y is not None:
         _check(Y, "Y", el, _extent(M, N, ldy, sY, batch))
     _on_device(A=A, B=B, B2=B2, D=D, X=X, Y=Y)
-    rc = lib.ttt_k_gemm(_dtype_code(A), M, N, K, batch, A.data_ptr(), lda, sA, int(a_mn), B.data_ptr(), ldb, sB,
-                        int(b_mn), B2.data_ptr() if B2 is not None else None, sB2, D.data_ptr(), ldd, sD,
-                        int(D.dtype == torch.float32),
-                        X.data_ptr() if X is not None else None, ldx, sX,
-                        Y.data_ptr() if Y is not None else None, ldy, sY, float(alpha), epi, engine,
-                        _stream_ptr(stream))
+    ptr = lambda x: x.data_ptr() if x is not None else None  # noqa: E731
+    return ttt_gemm_desc(M, N, K, batch, A.data_ptr(), lda, sA, int(a_mn), B.data_ptr(), ldb, sB, int(b_mn),
+                         ptr(B2), sB2, D.data_ptr(), ldd, sD, int(D.dtype == torch.float32), ptr(X), ldx, sX,
+                         ptr(Y), ldy, sY, float(alpha), epi)
+
+
+def ttt_k_gemm(A, B, D, M, N, K, *, engine=ENGINE_AUTO, stream=None, **kw):
+    """Enqueue one contraction on device tensors (see include/ttt_kernels.h); keyword
+    arguments as _gemm_desc."""
+    g = _gemm_desc(A, B, D, M, N, K, **kw)
+    rc = lib.ttt_k_gemm(_dtype_code(A), g.M, g.N, g.K, g.batch, g.A, g.lda, g.sA, g.a_mn, g.B, g.ldb, g.sB, g.b_mn,
+                        g.B2, g.sB2, g.D, g.ldd, g.sD, g.d_f32, g.X, g.ldx, g.sX, g.Y, g.ldy, g.sY, g.alpha, g.epi,
+                        engine, _stream_ptr(stream))
     if rc != TTT_OK:
         raise TTTError(rc, "ttt_k_gemm")
+
+
+def ttt_k_gemm_pair(first, second, stream=None):
+    """Enqueue two independent contractions, one launch where they can share it.
+    first, second: dicts of ttt_k_gemm's arguments (A, B, D, M, N, K and keywords)."""
+    if _elem_name(first["A"]) != _elem_name(second["A"]):
+        raise ValueError("both products must have the same element type")
+    a, b = _gemm_desc(**first), _gemm_desc(**second)
+    rc = lib.ttt_k_gemm_pair(_dtype_code(first["A"]), ctypes.byref(a), ctypes.byref(b), _stream_ptr(stream))
+    if rc != TTT_OK:
+        raise TTTError(rc, "ttt_k_gemm_pair")
 
 
 def _check_attention(qkv, out, lse, B, H, hd, n, q0, ring_k, ring_v, C, dout=None, dqkv=None, dsum=None):

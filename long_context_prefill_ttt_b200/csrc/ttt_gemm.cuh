@@ -809,13 +809,21 @@ __device__ __forceinline__ bool epilogue_tile(const GemmParams& p, uint32_t tadd
     return epilogue_tile_direct<BN>(p, taddr, z, m, n0, c_first, wait_acc, release, part, row, part_c0);
 }
 
+// One or two independent products of the same layout and tile width in one persistent
+// launch (the tile list of the second follows that of the first), with their tensor maps.
+struct TcGroup {
+  CUtensorMap tmA[2], tmB[2], tmB2[2];
+  GemmParams p[2];
+  int nprob;
+};
+
 // Persistent warp-specialised tcgen05 GEMM. Requirements (checked on the host):
 // N % BN == 0, K % 64 == 0, 16-byte aligned rows; M may have a tail (TMA fills
-// out-of-range rows with zeros and the epilogue skips them).
+// out-of-range rows with zeros and the epilogue skips them). With two products
+// (g.nprob = 2) the CTAs walk both tile lists as one, so that the epilogue of one
+// product's tiles overlaps the mainloop of the next tiles.
 template <int BN, bool A_MN, bool B_MN>
-__global__ void __launch_bounds__(TC_THREADS, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmB2, const GemmParams p, int* err) {
+__global__ void __launch_bounds__(TC_THREADS, 1) gemm_tc_kernel(const __grid_constant__ TcGroup g, int* err) {
   using C = TcCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -827,22 +835,33 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint32_t* tmem_slot = (uint32_t*)(bars + 2 * C::STAGES + 4);
 
   const int warp = threadIdx.x >> 5;
-  const int m_tiles = (p.M + TC_BM - 1) / TC_BM;
-  const int n_tiles = p.N / BN;
-  const int tiles_per_batch = m_tiles * n_tiles;
-  const int num_tiles = tiles_per_batch * p.batch;
-  const int kb_one = p.K / TC_BK;
-  const int k_blocks = p.B2 ? 2 * kb_one : kb_one;
-  const int zb_scale = p.sB ? 1 : 0;    // shared B (batch stride 0): always batch slice 0
-  const int zb2_scale = p.sB2 ? 1 : 0;
+  // tile counts of each product; tiles [0, nt0) belong to product 0, the rest to product 1
+  const int mt0 = (g.p[0].M + TC_BM - 1) / TC_BM, ntl0 = g.p[0].N / BN, tpb0 = mt0 * ntl0;
+  const int nt0 = tpb0 * g.p[0].batch;
+  const int mt1 = g.nprob > 1 ? (g.p[1].M + TC_BM - 1) / TC_BM : 1, ntl1 = g.nprob > 1 ? g.p[1].N / BN : 1;
+  const int tpb1 = mt1 * ntl1;
+  const int num_tiles = nt0 + (g.nprob > 1 ? tpb1 * g.p[1].batch : 0);
+  // product, batch slice and tile origin of a tile
+  auto locate = [&](int tile, int& pi, int& z, int& m0, int& n0) {
+    pi = tile >= nt0 ? 1 : 0;
+    const int t = tile - (pi ? nt0 : 0);
+    const int tpb = pi ? tpb1 : tpb0, mt = pi ? mt1 : mt0, ntl = pi ? ntl1 : ntl0;
+    const GemmParams& P = pi ? g.p[1] : g.p[0];
+    z = t / tpb;
+    const int r = t % tpb;
+    m0 = (P.m_fast ? r % mt : r / ntl) * TC_BM;
+    n0 = (P.m_fast ? r / mt : r % ntl) * BN;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int a = 0; a < 2; ++a) { mbar_init(&acc_full[a], 1); mbar_init(&acc_empty[a], TC_EPI_WARPS); }
     fence_mbar_init();
-    prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
-    if (p.B2) prefetch_tmap(&tmB2);
+    for (int i = 0; i < g.nprob; ++i) {
+      prefetch_tmap(&g.tmA[i]);
+      prefetch_tmap(&g.tmB[i]);
+      if (g.p[i].B2) prefetch_tmap(&g.tmB2[i]);
+    }
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -860,10 +879,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int z = tile / tiles_per_batch;
-        const int r = tile % tiles_per_batch;
-        const int m0 = (p.m_fast ? r % m_tiles : r / n_tiles) * TC_BM;
-        const int n0 = (p.m_fast ? r / m_tiles : r % n_tiles) * BN;
+        int pi, z, m0, n0;
+        locate(tile, pi, z, m0, n0);
+        const GemmParams& P = pi ? g.p[1] : g.p[0];
+        const CUtensorMap* mA = &g.tmA[pi];
+        const int kb_one = P.K / TC_BK;
+        const int k_blocks = P.B2 ? 2 * kb_one : kb_one;
+        const int zb_scale = P.sB ? 1 : 0;  // shared B (batch stride 0): always batch slice 0
+        const int zb2_scale = P.sB2 ? 1 : 0;
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
           const int s = it % C::STAGES;
           const uint32_t round = it / C::STAGES;
@@ -873,13 +896,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
           const bool second = kb >= kb_one;
           const int k0 = (second ? kb - kb_one : kb) * TC_BK;
-          const CUtensorMap* mb = second ? &tmB2 : &tmB;
+          const CUtensorMap* mb = second ? &g.tmB2[pi] : &g.tmB[pi];
           const int zb = z * (second ? zb2_scale : zb_scale);
           if (A_MN) {
-            tma_load_3d(sa, &tmA, &full[s], m0, k0, z);
-            tma_load_3d(sa + 8192, &tmA, &full[s], m0 + 64, k0, z);
+            tma_load_3d(sa, mA, &full[s], m0, k0, z);
+            tma_load_3d(sa + 8192, mA, &full[s], m0 + 64, k0, z);
           } else {
-            tma_load_3d(sa, &tmA, &full[s], k0, m0, z);
+            tma_load_3d(sa, mA, &full[s], k0, m0, z);
           }
           if (B_MN) {
 #pragma unroll
@@ -896,6 +919,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       int it = 0, lt = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++lt) {
+        const GemmParams& P = tile >= nt0 ? g.p[1] : g.p[0];
+        const int kb_one = P.K / TC_BK;
+        const int k_blocks = P.B2 ? 2 * kb_one : kb_one;
         const int acc = lt & 1;
         const uint32_t use = lt >> 1;
         if (!mbar_wait(&acc_empty[acc], (use & 1) ^ 1, err, DEV_TIMEOUT_ACC)) break;
@@ -931,15 +957,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     uint8_t* stg = smem + C::STAGES * C::STAGE_BYTES + 256 + (warp - 2) * EPI_STAGE_BYTES;
     int lt = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++lt) {
-      const int z = tile / tiles_per_batch;
-      const int r = tile % tiles_per_batch;
-      const int m0 = (p.m_fast ? r % m_tiles : r / n_tiles) * TC_BM;
-      const int n0 = (p.m_fast ? r / m_tiles : r % n_tiles) * BN;
+      int pi, z, m0, n0;
+      locate(tile, pi, z, m0, n0);
       const int acc = lt & 1;
       const uint32_t use = lt >> 1;
       const uint32_t taddr = tmem_base + acc * BN + ((uint32_t)(quarter * 32) << 16);
       if (!epilogue_tile<BN, A_MN>(
-              p, taddr, z, m0 + row_in_tile, n0, c_first, stg,
+              pi ? g.p[1] : g.p[0], taddr, z, m0 + row_in_tile, n0, c_first, stg,
               [&] { return mbar_wait(&acc_full[acc], use & 1, err, DEV_TIMEOUT_ACC); },
               [&] {
                 if (elect_lane0()) mbar_arrive(&acc_empty[acc]);
@@ -1291,6 +1315,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 // ============================================================== host side
 enum GemmEngine : int { GEMM_AUTO = 0, GEMM_SIMT = 1, GEMM_TC1 = 3 };
 int gemm_launch(const GemmParams& p, int elem_is_bf16, cudaStream_t stream, int* err, int num_sms, int engine);
+// Two independent products, in one launch where they can share it (same engine, operand
+// layouts and tile width); 0 or a cudaError_t.
+int gemm_launch_pair(const GemmParams& a, const GemmParams& b, int elem_is_bf16, cudaStream_t stream, int* err,
+                     int num_sms);
 // Whether gemm_launch would run p on the tcgen05 engine (EPI_CE requires it).
 bool gemm_uses_tc(const GemmParams& p, int elem_is_bf16);
 // Sets the dynamic shared-memory limits of all large-smem kernels; 0 or a cudaError_t.

@@ -142,28 +142,47 @@ using namespace ttt;
 
 extern "C" {
 
+// Validates one product's arguments and fills its parameter block; false = invalid.
+static bool gemm_params_from(const ttt_gemm_desc& g, GemmParams* p) {
+  if (g.M < 0 || g.N < 0 || g.K < 0 || g.batch < 1 || !g.A || !g.B || !g.D || g.epi < 0 || g.epi > 4) return false;
+  if ((g.epi == EPI_RESID || g.epi == EPI_DGELU) && !g.X) return false;
+  if ((g.epi == EPI_RESID || g.epi == EPI_SGD) && !g.d_f32) return false;
+  memset(p, 0, sizeof(*p));
+  p->M = g.M; p->N = g.N; p->K = g.K; p->batch = g.batch;
+  p->A = g.A; p->lda = g.lda; p->sA = g.sA; p->a_mn = g.a_mn;
+  p->B = g.B; p->ldb = g.ldb; p->sB = g.sB; p->b_mn = g.b_mn;
+  p->B2 = g.B2; p->sB2 = g.sB2;
+  p->D = g.D; p->ldd = g.ldd; p->sD = g.sD; p->d_f32 = g.d_f32;
+  p->X = g.X; p->ldx = g.ldx; p->sX = g.sX;
+  p->Y = g.Y; p->ldy = g.ldy; p->sY = g.sY;
+  p->alpha = g.alpha; p->epi = g.epi;
+  return true;
+}
+
 int ttt_k_gemm(int32_t elem_dtype, int32_t M, int32_t N, int32_t K, int32_t batch, const void* A, int64_t lda,
                int64_t sA, int32_t a_mn, const void* B, int64_t ldb, int64_t sB, int32_t b_mn, const void* B2,
                int64_t sB2, void* D, int64_t ldd,
                int64_t sD, int32_t d_f32, const void* X, int64_t ldx, int64_t sX, void* Y, int64_t ldy, int64_t sY,
                float alpha, int32_t epi, int32_t engine, void* stream) {
-  if (M < 0 || N < 0 || K < 0 || batch < 1 || !A || !B || !D || epi < 0 || epi > 4) return TTT_ERR_INVALID_ARG;
-  if ((epi == EPI_RESID || epi == EPI_DGELU) && !X) return TTT_ERR_INVALID_ARG;
-  if ((epi == EPI_RESID || epi == EPI_SGD) && !d_f32) return TTT_ERR_INVALID_ARG;
+  const ttt_gemm_desc g = {M, N, K, batch, A, lda, sA, a_mn, B, ldb, sB, b_mn, B2, sB2, D, ldd, sD, d_f32,
+                           X, ldx, sX, Y, ldy, sY, alpha, epi};
+  GemmParams p;
+  if (!gemm_params_from(g, &p)) return TTT_ERR_INVALID_ARG;
   int* err = status_word();
   if (!err) return TTT_ERR_CUDA;
-  GemmParams p;
-  memset(&p, 0, sizeof(p));
-  p.M = M; p.N = N; p.K = K; p.batch = batch;
-  p.A = A; p.lda = lda; p.sA = sA; p.a_mn = a_mn;
-  p.B = B; p.ldb = ldb; p.sB = sB; p.b_mn = b_mn;
-  p.B2 = B2; p.sB2 = sB2;
-  p.D = D; p.ldd = ldd; p.sD = sD; p.d_f32 = d_f32;
-  p.X = X; p.ldx = ldx; p.sX = sX;
-  p.Y = Y; p.ldy = ldy; p.sY = sY;
-  p.alpha = alpha; p.epi = epi;
   const int e = gemm_launch(p, elem_dtype == TTT_BF16 ? 1 : 0, (cudaStream_t)stream, err, sm_count(),
                             engine == TTT_ENGINE_SIMT ? GEMM_SIMT : engine == TTT_ENGINE_TC1 ? GEMM_TC1 : GEMM_AUTO);
+  return e == 0 ? TTT_OK : TTT_ERR_CUDA;
+}
+
+int ttt_k_gemm_pair(int32_t elem_dtype, const ttt_gemm_desc* first, const ttt_gemm_desc* second, void* stream) {
+  if (!first || !second) return TTT_ERR_INVALID_ARG;
+  GemmParams a, b;
+  if (!gemm_params_from(*first, &a) || !gemm_params_from(*second, &b)) return TTT_ERR_INVALID_ARG;
+  int* err = status_word();
+  if (!err) return TTT_ERR_CUDA;
+  if (prime_kernel_attributes() != 0) return TTT_ERR_CUDA;
+  const int e = gemm_launch_pair(a, b, elem_dtype == TTT_BF16 ? 1 : 0, (cudaStream_t)stream, err, sm_count());
   return e == 0 ? TTT_OK : TTT_ERR_CUDA;
 }
 

@@ -137,18 +137,29 @@ static bool make_operand_map(CUtensorMap* map, const void* base, int64_t rows, i
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
+// Single-CTA tcgen05 launch of one product, or of two (p2) in one persistent grid.
 template <int BN, bool AM, bool BM>
-static cudaError_t launch_tc(const GemmParams& p, cudaStream_t st, int* err, int num_sms, bool* ok) {
-  CUtensorMap ta, tb, tb2;
-  *ok = make_operand_map(&ta, p.A, p.M, p.K, p.lda, p.batch, p.sA, AM, TC_BM) &&
-        make_operand_map(&tb, p.B, p.N, p.K, p.ldb, p.batch, p.sB, BM, BN);
-  if (*ok && p.B2) *ok = make_operand_map(&tb2, p.B2, p.N, p.K, p.ldb, p.batch, p.sB2, BM, BN);
-  else tb2 = tb;
+static cudaError_t launch_tc(const GemmParams& p, cudaStream_t st, int* err, int num_sms, bool* ok,
+                             const GemmParams* p2 = nullptr) {
+  TcGroup g;
+  memset(&g, 0, sizeof(g));
+  g.nprob = p2 ? 2 : 1;
+  const GemmParams* ps[2] = {&p, p2};
+  *ok = true;
+  int tiles = 0;
+  for (int i = 0; i < g.nprob && *ok; ++i) {
+    const GemmParams& q = *ps[i];
+    *ok = make_operand_map(&g.tmA[i], q.A, q.M, q.K, q.lda, q.batch, q.sA, AM, TC_BM) &&
+          make_operand_map(&g.tmB[i], q.B, q.N, q.K, q.ldb, q.batch, q.sB, BM, BN);
+    if (*ok && q.B2) *ok = make_operand_map(&g.tmB2[i], q.B2, q.N, q.K, q.ldb, q.batch, q.sB2, BM, BN);
+    else g.tmB2[i] = g.tmB[i];
+    g.p[i] = q;
+    tiles += ((q.M + TC_BM - 1) / TC_BM) * (q.N / BN) * q.batch;
+  }
   if (!*ok) return cudaSuccess;
   using C = TcCfg<BN>;
-  const int tiles = ((p.M + TC_BM - 1) / TC_BM) * (p.N / BN) * p.batch;
   const int grid = tiles < num_sms ? tiles : num_sms;
-  return launch_pdl(gemm_tc_kernel<BN, AM, BM>, dim3(grid), dim3(TC_THREADS), C::SMEM, st, ta, tb, tb2, p, err);
+  return launch_pdl(gemm_tc_kernel<BN, AM, BM>, dim3(grid), dim3(TC_THREADS), C::SMEM, st, g, err);
 }
 
 // Pairs of CTAs that can be resident at once for one paired-GEMM variant (0 = the
@@ -407,6 +418,32 @@ static bool tc_ok(const GemmParams& p, int elem_is_bf16) {
   if (ok && p.Y && !(aligned16(p.Y) && p.ldy % 8 == 0 && (p.batch == 1 || p.sY % 8 == 0))) ok = false;
   if (ok && p.epi == EPI_CE && !(p.batch == 1 && !p.d_f32 && p.ce_tgt && p.ce_part && p.ce_zt)) ok = false;
   return ok;
+}
+
+// Two independent products on one stream: one grouped single-CTA tcgen05 launch where
+// both fit it with the same operand layouts and 256-wide tiles (the CTAs then overlap
+// one product's epilogues with the other's mainloop), else two launches.
+int gemm_launch_pair(const GemmParams& a, const GemmParams& b, int elem_is_bf16, cudaStream_t st, int* err,
+                     int num_sms) {
+  const bool grp = elem_is_bf16 && a.epi != EPI_CE && b.epi != EPI_CE && a.epi != EPI_QKV_ROPE &&
+                   b.epi != EPI_QKV_ROPE && !a.norm_x && !b.norm_x && a.a_mn == b.a_mn && a.b_mn == b.b_mn &&
+                   a.N % 256 == 0 && b.N % 256 == 0 && a.M > 0 && b.M > 0 && a.batch > 0 && b.batch > 0 &&
+                   gemm_uses_tc(a, 1) && gemm_uses_tc(b, 1);
+  if (grp) {
+    GemmParams x = a, y = b;  // walk the larger operand of each once (as gemm_launch does)
+    x.m_fast = x.N > x.M ? 1 : 0;
+    y.m_fast = y.N > y.M ? 1 : 0;
+    bool ok = false;
+    cudaError_t e;
+    if (!a.a_mn && !a.b_mn) e = launch_tc<256, false, false>(x, st, err, num_sms, &ok, &y);
+    else if (!a.a_mn && a.b_mn) e = launch_tc<256, false, true>(x, st, err, num_sms, &ok, &y);
+    else e = launch_tc<256, true, true>(x, st, err, num_sms, &ok, &y);
+    if (e != cudaSuccess) return (int)e;
+    if (ok) return 0;
+  }
+  const int e = gemm_launch(a, elem_is_bf16, st, err, num_sms, GEMM_AUTO);
+  if (e != 0) return e;
+  return gemm_launch(b, elem_is_bf16, st, err, num_sms, GEMM_AUTO);
 }
 
 bool gemm_uses_tc(const GemmParams& p, int elem_is_bf16) {
@@ -808,6 +845,23 @@ template <typename T> class Engine : public ttt_handle {
     const int e = gemm_launch(p, is_bf16 ? 1 : 0, st, dev_err, num_sms, GEMM_AUTO);
     prof.end(st);
     ++launches;
+    if (e != 0) {
+      poisoned = true;
+      return fail(this, TTT_ERR_CUDA, std::string("gemm: ") + cudaGetErrorString((cudaError_t)e));
+    }
+    return TTT_OK;
+  }
+  // Two independent products (gemm_launch_pair): one launch where they can share it.
+  int gemm2(const GemmParams& a, const GemmParams& b) {
+    const size_t es = is_bf16 ? 2 : 4;
+    auto bytes = [&](const GemmParams& p) {
+      return (double)p.batch * ((double)p.M * p.K * es + (double)p.N * p.K * es + (double)p.M * p.N * (p.d_f32 ? 4 : es));
+    };
+    prof.begin(st, gemm_class, 2.0 * a.M * a.N * (double)a.K * a.batch + 2.0 * b.M * b.N * (double)b.K * b.batch,
+               bytes(a) + bytes(b));
+    const int e = gemm_launch_pair(a, b, is_bf16 ? 1 : 0, st, dev_err, num_sms);
+    prof.end(st);
+    launches += 2;
     if (e != 0) {
       poisoned = true;
       return fail(this, TTT_ERR_CUDA, std::string("gemm: ") + cudaGetErrorString((cudaError_t)e));
@@ -1315,17 +1369,16 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
     }
     // dW2t[o][i] = sum_t dm[t][o] g[t][i]  -> W2t32 += -eta * dW2t ; bf16 copy refreshed
     // (bf16 path: W2t32 holds the accumulated update dW, so the copy keeps its precision)
-    p = gp(d, ht, cn, GT, d, true, A.g, ht, true, Lw.W2t32, ht, true, EPI_SGD);
-    p.batch = B; p.sA = (int64_t)cn * d; p.sB = (int64_t)cn * ht; p.sD = (int64_t)d * ht;
-    p.alpha = -cfg.eta;
-    if (is_bf16) { p.Y = Lw.W2t; p.ldy = ht; p.sY = (int64_t)d * ht; }
-    if ((rc = gemm(p)) != TTT_OK) return rc;
-    // dW1t[o][i] = sum_t du[t][o] r2[t][i]
-    p = gp(ht, d, cn, dhid, ht, true, A.r2, d, true, Lw.W1t32, d, true, EPI_SGD);
-    p.batch = B; p.sA = (int64_t)cn * ht; p.sB = (int64_t)cn * d; p.sD = (int64_t)ht * d;
-    p.alpha = -cfg.eta;
-    if (is_bf16) { p.Y = Lw.W1t; p.ldy = d; p.sY = (int64_t)ht * d; }
-    if ((rc = gemm(p)) != TTT_OK) return rc;
+    GemmParams p2w = gp(d, ht, cn, GT, d, true, A.g, ht, true, Lw.W2t32, ht, true, EPI_SGD);
+    p2w.batch = B; p2w.sA = (int64_t)cn * d; p2w.sB = (int64_t)cn * ht; p2w.sD = (int64_t)d * ht;
+    p2w.alpha = -cfg.eta;
+    if (is_bf16) { p2w.Y = Lw.W2t; p2w.ldy = ht; p2w.sY = (int64_t)d * ht; }
+    // dW1t[o][i] = sum_t du[t][o] r2[t][i]; independent of dW2t: both in one launch
+    GemmParams p1w = gp(ht, d, cn, dhid, ht, true, A.r2, d, true, Lw.W1t32, d, true, EPI_SGD);
+    p1w.batch = B; p1w.sA = (int64_t)cn * ht; p1w.sB = (int64_t)cn * d; p1w.sD = (int64_t)ht * d;
+    p1w.alpha = -cfg.eta;
+    if (is_bf16) { p1w.Y = Lw.W1t; p1w.ldy = d; p1w.sY = (int64_t)ht * d; }
+    if ((rc = gemm2(p2w, p1w)) != TTT_OK) return rc;
     if (j == 0) break;  // upstream of the first adaptive MLP does not depend on the fast weights
     rmsnorm_bwd_launch<T>((const float*)A.a, Lw.g_ttt, A.rstd2, dr, G, rows, d, G, GT, st);
     TTT_LAUNCHED();

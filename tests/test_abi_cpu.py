@@ -28,7 +28,7 @@ def declared_functions():
 def test_headers_declare_the_boundary():
     names = declared_functions()
     for n in ("ttt_create", "ttt_prefill", "ttt_decode", "ttt_get_weights", "ttt_reset", "ttt_destroy",
-              "ttt_last_error", "ttt_k_gemm", "ttt_k_attention_fwd", "ttt_k_attention_bwd"):
+              "ttt_last_error", "ttt_k_gemm", "ttt_k_gemm_pair", "ttt_k_attention_fwd", "ttt_k_attention_bwd"):
         assert n in names
 
 
@@ -69,6 +69,9 @@ def test_null_handle_calls_return_invalid_arg():
     assert T.lib.ttt_prefill(None, None, 4, None, 0) == T.TTT_ERR_INVALID_ARG
     assert T.lib.ttt_decode(None, 1, None, None, None, 0) == T.TTT_ERR_INVALID_ARG
     assert T.lib.ttt_reset(None) == T.TTT_ERR_INVALID_ARG
+    assert T.lib.ttt_k_gemm_pair(T.TTT_BF16, None, None, None) == T.TTT_ERR_INVALID_ARG
+    empty = T.ttt_gemm_desc()          # null operands: rejected before any CUDA call
+    assert T.lib.ttt_k_gemm_pair(T.TTT_BF16, ctypes.byref(empty), ctypes.byref(empty), None) == T.TTT_ERR_INVALID_ARG
     assert T.lib.ttt_position(None) == -1
     T.lib.ttt_destroy(None)
 
@@ -90,6 +93,13 @@ def test_binding_refuses_buffers_that_do_not_cover_the_call():
         T.ttt_k_gemm(A, B, D, M, N, K, batch=2, sA=0, sB=0, B2=B, sB2=N * K, sD=0)
     with pytest.raises(ValueError, match="must be a device buffer"):
         T.ttt_k_gemm(A, B, D, M, N, K)       # right sizes, but host memory
+    one = dict(A=A, B=B, D=D, M=M, N=N, K=K)
+    with pytest.raises(ValueError, match="D: .* elements"):
+        T.ttt_k_gemm_pair(dict(one, D=D[:5]), one)
+    with pytest.raises(ValueError, match="same element type"):
+        T.ttt_k_gemm_pair(one, dict(one, A=A.float(), B=B.float()))
+    with pytest.raises(ValueError, match="must be a device buffer"):
+        T.ttt_k_gemm_pair(one, one)
     qkv, out, lse = torch.zeros(4 * 3 * 64, dtype=bf), torch.zeros(4 * 64, dtype=bf), torch.zeros(4)
     with pytest.raises(ValueError, match="ring_k"):
         T.ttt_k_attention_fwd(qkv, out, lse, 1, 1, 64, 4, 128, 64, None, None, 256)

@@ -194,6 +194,53 @@ def test_gemm_k_split_pairs(T, M, N, K, batch, a_mn, b_mn, b2):
     assert (D3.double() - D1.double()).abs().max().item() < tol * scale
 
 
+# Two independent products through ttt_k_gemm_pair: (M, N) of each, shared K, batch,
+# layout, epilogue. The first case is the adaptive MLP's two weight-gradient SGD steps at
+# the ~1B workload's sizes (d 2048, hidden 8192, 1024-position mini-batch: 1024 tiles, so
+# CTAs cross from the first product's tiles into the second's); the others span ragged M
+# tails, batches and the forward / data-gradient layouts; the last has N % 256 != 0 and
+# takes two separate launches.
+PAIR_CASES = [((2048, 8192), (8192, 2048), 1024, 1, 1, 1, "sgd"), ((520, 1024), (1000, 512), 256, 2, 1, 1, "sgd"),
+              ((300, 512), (200, 768), 192, 1, 0, 0, "gelu"), ((128, 256), (640, 256), 128, 3, 0, 1, "store"),
+              ((256, 384), (256, 256), 128, 1, 0, 0, "store")]
+
+
+@pytest.mark.parametrize("mn1,mn2,K,batch,a_mn,b_mn,epi", PAIR_CASES)
+def test_gemm_pair(T, mn1, mn2, K, batch, a_mn, b_mn, epi):
+    cases = []
+    for i, (M, N) in enumerate((mn1, mn2)):
+        A = _rand((batch, M, K), torch.bfloat16, 41 + 10 * i, 0.5)
+        B = _rand((batch, N, K), torch.bfloat16, 42 + 10 * i, 0.5)
+        acc = A.double() @ B.double().transpose(1, 2)
+        kw = dict(A=_store(A, a_mn), B=_store(B, b_mn), M=M, N=N, K=K, batch=batch, sA=M * K, a_mn=a_mn,
+                  sB=N * K, b_mn=b_mn, sD=M * N)
+        if epi == "sgd":
+            W = _rand((batch, M, N), torch.float32, 43 + 10 * i)
+            Y = torch.empty((batch, M, N), dtype=torch.bfloat16, device="cuda")
+            kw.update(D=W, Y=Y, ldy=N, sY=M * N, alpha=-0.01, epi=T.EPI_SGD)
+            want = W.double() - 0.01 * acc
+        elif epi == "gelu":
+            U = torch.empty((batch, M, N), dtype=torch.bfloat16, device="cuda")
+            kw.update(D=torch.empty_like(U), Y=U, ldy=N, sY=M * N, epi=T.EPI_GELU)
+            want = acc
+        else:
+            kw.update(D=torch.full((batch, M, N), float("nan"), dtype=torch.float32, device="cuda"))
+            want = acc
+        cases.append((kw, want, acc.abs().max().item()))
+    T.ttt_k_gemm_pair(cases[0][0], cases[1][0])
+    T.ttt_k_status()
+    tol = 2e-6 * max(1.0, K / 1024)
+    for kw, want, scale in cases:
+        if epi == "sgd":
+            assert (kw["D"].double() - want).abs().max().item() < tol * 0.01 * scale + 1e-6
+            assert torch.equal(kw["Y"], kw["D"].to(torch.bfloat16))
+        elif epi == "gelu":
+            assert torch.allclose(kw["Y"].double(), want, rtol=1e-2, atol=1e-2 * scale)
+            assert torch.allclose(kw["D"].double(), torch.nn.functional.gelu(want), rtol=1e-2, atol=1e-2 * scale)
+        else:
+            assert (kw["D"].double() - want).abs().max().item() < tol * scale
+
+
 def _attn_reference(qkv, ring_k, ring_v, B, H, hd, n, q0, window, C):
     """float64 keys/values at absolute positions, explicit window mask."""
     d = H * hd
