@@ -42,6 +42,21 @@ Readings taken where the pages are silent:
   R11 greedy decode takes the lowest id among equal maxima; decode's loss
      output is -log p(chosen token) under the weights in force.
 
+Variant with the layer-wise key-value-binding inner loss (cfg.inner_loss ==
+"kvb"; technical review §8, eq. (10); summary, "Alternative Derivation
+(Connection to TTT-KVB)"): each adaptive block's fast weights W = (W1t, W2t)
+fit g(theta_K x_t; W) to theta_V x_t instead of descending the next-token loss.
+Readings taken:
+  K1 x_t is the adaptive MLP's own input (the block's RMSNorm output r2), and
+     g(k; W) = W2t gelu(W1t k) is the same two-layer MLP the block applies to r2
+     on its output path; theta_K, theta_V are frozen d x d matrices of the block.
+  K2 the chunk's inner loss is (1/b) sum_t ||g(theta_K x_t; W) - theta_V x_t||^2
+     (squared Euclidean norm, mean over the b positions as in R9); each block
+     descends its own loss w.r.t. its own W only (layer-wise: no gradient passes
+     between blocks), with the same eta, schedule and per-sequence state.
+  K3 the recorded per-token losses are still the next-token losses of the
+     model with the weights in force (the inner loss only drives the update).
+
 Arithmetic is float64 throughout. Matrix products use numpy's matmul as the
 library primitive. Queries are processed in groups only to bound memory; each
 row is the plain definition. This oracle is pinned by the tests in
@@ -288,6 +303,8 @@ class Oracle:
         losses = lse - z[np.arange(n), t]
         if not need_grad:
             return losses, None
+        if getattr(cfg, "inner_loss", "e2e") == "kvb":
+            return losses, self._kvb_losses_and_grads(seq, caches)[1]
         # mean over the b positions of the chunk (reading R9)
         pz = np.exp(z - lse[:, None])
         pz[np.arange(n), t] -= 1.0
@@ -319,6 +336,26 @@ class Oracle:
             dv = dv_all[nc:].reshape(n, -1)
             dr1 = dq @ w[p + "Wq"] + dk @ w[p + "Wk"] + dv @ w[p + "Wv"]
             dy = da + rms_norm_backward(c["x"], w[p + "attn_norm"], c["rstd1"], dr1)
+        return losses, grads
+
+    def _kvb_losses_and_grads(self, seq, caches):
+        """Layer-wise key-value-binding inner loss of every adaptive block and its
+        gradient w.r.t. that block's fast weights (review §8, eq. (10); readings K1-K2)."""
+        cfg, w = self.cfg, self.w
+        losses, grads = [], []
+        for j in range(cfg.n_ttt):
+            p = f"layers.{cfg.first_ttt + j}."
+            fw = seq.fast[j]
+            x = caches[j]["r2"]
+            k = x @ w[p + "theta_K"].T
+            v = x @ w[p + "theta_V"].T
+            u = k @ fw["W1t"].T
+            g = gelu(u)
+            e = g @ fw["W2t"].T - v
+            losses.append(float(np.sum(e * e)) / cfg.minibatch_b)
+            de = (2.0 / cfg.minibatch_b) * e
+            du = (de @ fw["W2t"]) * gelu_prime(u)
+            grads.append({"W1t": du.T @ k, "W2t": de.T @ g})
         return losses, grads
 
     def _sgd(self, seq, grads):
@@ -413,3 +450,16 @@ class Oracle:
         h = self._frozen_forward(st, tokens_chunk[:-1], st.n_pos, commit=False)
         losses, grads = self._chunk(st, h, st.n_pos, tokens_chunk[1:], need_grad=True, commit=False)
         return float(np.mean(losses)), grads
+
+    def chunk_inner_losses_and_grads(self, seq, tokens_chunk):
+        """Key-value-binding variant: each adaptive block's inner loss on the next full
+        chunk and its gradient, without changing any state (tokens_chunk as above)."""
+        st = self.seqs[seq]
+        cfg = self.cfg
+        assert len(tokens_chunk) == cfg.minibatch_b + 1 and not st.pend_inputs
+        y = self._frozen_forward(st, tokens_chunk[:-1], st.n_pos, commit=False)
+        caches = []
+        for j in range(cfg.n_ttt):
+            y, c = self._ttt_block(st, j, y, st.n_pos, commit=False, keep=True)
+            caches.append(c)
+        return self._kvb_losses_and_grads(st, caches)

@@ -58,6 +58,10 @@ class TTTConfig:
     decode_n: int = 0            # tokens generated after the prefill (decode workload)
     weight_seed: int = 0
     token_seed: int = 0
+    # inner loss of the adaptive blocks: "e2e" (next-token cross-entropy at the output)
+    # or "kvb" (each block's layer-wise key-value-binding reconstruction loss, which
+    # adds the frozen projections theta_K, theta_V to every adaptive block)
+    inner_loss: str = "e2e"
 
     @property
     def head_dim(self) -> int:
@@ -153,6 +157,8 @@ def weight_shapes(cfg: TTTConfig):
             out += [(p + "ttt_norm", (d,)), (p + "W1t", (cfg.ttt_hidden, d)),
                     (p + "W2t", (d, cfg.ttt_hidden)), (p + "static_norm", (d,)),
                     (p + "W1s", (cfg.static_hidden, d)), (p + "W2s", (d, cfg.static_hidden))]
+            if cfg.inner_loss == "kvb":
+                out += [(p + "theta_K", (d, d)), (p + "theta_V", (d, d))]
         else:
             out += [(p + "mlp_norm", (d,)), (p + "W1", (cfg.mlp_hidden, d)),
                     (p + "W2", (d, cfg.mlp_hidden))]

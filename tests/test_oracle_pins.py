@@ -405,3 +405,93 @@ def test_chunkwise_autograd_reduces_to_the_static_loop_with_one_adaptive_block()
         got, fast = TS.mini_batch_ttt_chunked(cfg, w, toks[0], rule)
         np.testing.assert_allclose(got.numpy(), ref_losses.numpy(), rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(fast[0]["W1t"].numpy(), ref_fast[0]["W1t"].numpy(), rtol=1e-10, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- key-value-binding inner loss (variant)
+
+def tiny_kvb(n_ttt=2, **kw):
+    # a smaller step than the next-token pins: with these weights (std 0.5) the
+    # reconstruction errors are O(1) per component and eta = 0.5 diverges
+    kw.setdefault("eta", 0.02)
+    return tiny(n_ttt=n_ttt, inner_loss="kvb", **kw)
+
+
+@pytest.mark.parametrize("n_ttt", [1, 2])
+def test_kvb_gradient_matches_finite_differences(n_ttt):
+    """Hand-written gradient of each block's reconstruction loss (technical review §8,
+    eq. (10)) w.r.t. that block's fast weights, on chunk 3 (window cache non-empty)."""
+    cfg = tiny_kvb(n_ttt=n_ttt, T=8)
+    w = weights(cfg)
+    toks = tokens(cfg, n=cfg.T + 1 + cfg.minibatch_b)
+    orc = Oracle(cfg, w)
+    orc.prefill(toks[:, :cfg.T + 1])
+    chunk = toks[0, cfg.T:cfg.T + cfg.minibatch_b + 1]
+    losses, grads = orc.chunk_inner_losses_and_grads(0, chunk)
+    assert all(v > 0 for v in losses)
+    for j in range(cfg.n_ttt):
+        for name in ("W1t", "W2t"):
+            W = orc.seqs[0].fast[j][name]
+            num = _fd(lambda: orc.chunk_inner_losses_and_grads(0, chunk)[0][j], W)
+            # central differences of losses of size ~100 carry ~1e-8 of rounding
+            np.testing.assert_allclose(grads[j][name], num, rtol=1e-5, atol=1e-7)
+
+
+@pytest.mark.parametrize("n_ttt,b,k,T", [(2, 4, 6, 16), (3, 4, 9, 18), (1, 3, 5, 14)])
+def test_kvb_trajectory_matches_chunkwise_autograd(n_ttt, b, k, T):
+    """The whole prefill with the reconstruction inner loss against an independent
+    chunk-wise loop (library mse_loss, SDPA and autograd, tests/torch_static.py): losses
+    and final fast weights. Negative controls: letting each block's loss reach the
+    earlier blocks' weights (not layer-wise) and the next-token inner loss both move the
+    first adaptive block's weights far outside the tolerance."""
+    cfg = tiny_kvb(n_ttt=n_ttt, minibatch_b=b, window_k=k, T=T)
+    w = weights(cfg)
+    toks = tokens(cfg)
+    orc = Oracle(cfg, w)
+    losses = orc.prefill(toks)
+    ref_losses, ref_fast = TS.mini_batch_ttt_kvb_chunked(cfg, w, toks[0])
+    np.testing.assert_allclose(losses[0], ref_losses.numpy(), rtol=1e-10, atol=1e-12)
+    for j in range(n_ttt):
+        W1, W2 = orc.fast_weights(0, j)
+        np.testing.assert_allclose(W1, ref_fast[j]["W1t"].numpy(), rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(W2, ref_fast[j]["W2t"].numpy(), rtol=1e-10, atol=1e-12)
+    W1_0 = orc.fast_weights(0, 0)[0]
+    if n_ttt > 1:
+        _, joint = TS.mini_batch_ttt_kvb_chunked(cfg, w, toks[0], layerwise=False)
+        assert np.max(np.abs(joint[0]["W1t"].numpy() - W1_0)) > 1e-6
+    e2e = Oracle(cfg.replace(inner_loss="e2e"), w)
+    e2e.prefill(toks)
+    assert np.max(np.abs(e2e.fast_weights(0, 0)[0] - W1_0)) > 1e-6
+
+
+def test_kvb_zero_key_projection_never_moves_the_weights():
+    """theta_K = 0: every key is 0, so gelu(W1t k) = 0 and both weight gradients vanish
+    (dW2t pairs the error with gelu(0) = 0, dW1t pairs it with k = 0): the prefill is
+    the static model's and the fast weights stay W_init."""
+    cfg = tiny_kvb(n_ttt=2, T=16)
+    w = weights(cfg)
+    for l in range(cfg.first_ttt, cfg.n_layers):
+        w[f"layers.{l}.theta_K"] = np.zeros_like(w[f"layers.{l}.theta_K"])
+    toks = tokens(cfg)
+    orc = Oracle(cfg, w)
+    losses = orc.prefill(toks)
+    np.testing.assert_allclose(losses[0], TS.static_forward(cfg, w, toks[0]).numpy(), rtol=1e-10, atol=1e-12)
+    for j in range(cfg.n_ttt):
+        l = cfg.first_ttt + j
+        assert np.array_equal(orc.fast_weights(0, j)[0], w[f"layers.{l}.W1t"].astype(np.float64))
+        assert np.array_equal(orc.fast_weights(0, j)[1], w[f"layers.{l}.W2t"].astype(np.float64))
+
+
+def test_kvb_teacher_forced_decode_equals_prefill():
+    """Decode's update after a full chunk of generated tokens uses the same inner loss
+    (review §7, Algorithm 3)."""
+    cfg = tiny_kvb(n_ttt=2, T=8)
+    w = weights(cfg)
+    toks = tokens(cfg, n=8 + 1 + 10)
+    full = Oracle(cfg, w)
+    lf = full.prefill(toks)
+    dec = Oracle(cfg, w)
+    lp = dec.prefill(toks[:, :9])
+    r = dec.decode(10, forced=toks[:, 9:])
+    np.testing.assert_allclose(np.concatenate([lp, r["losses"]], axis=1), lf, rtol=1e-10, atol=1e-12)
+    for j in range(cfg.n_ttt):
+        np.testing.assert_allclose(dec.fast_weights(0, j)[0], full.fast_weights(0, j)[0], rtol=1e-10, atol=1e-12)

@@ -118,7 +118,8 @@ def _attend(q, keys, vals, q_pos, k_pos, window):
 def _adaptive_layer(cfg, w, l, fast_j, x, pos, k_hist, v_hist, hist_pos):
     """One adaptive block over rows x at positions pos; attention sees the given
     earlier keys/values (constants) and the rows' own keys/values.
-    Returns (output, post-RoPE keys of the rows, values of the rows)."""
+    Returns (output, post-RoPE keys of the rows, values of the rows, the rows that enter
+    the adaptive MLP)."""
     d, H = cfg.d, cfg.n_heads
     hd = d // H
     n = x.shape[0]
@@ -135,7 +136,7 @@ def _adaptive_layer(cfg, w, l, fast_j, x, pos, k_hist, v_hist, hist_pos):
     x = x + F.gelu(r2 @ fast_j["W1t"].T, approximate="none") @ fast_j["W2t"].T
     r3 = F.rms_norm(x, (d,), weight=w[p + "static_norm"], eps=cfg.rms_eps)
     x = x + F.gelu(r3 @ w[p + "W1s"].T, approximate="none") @ w[p + "W2s"].T
-    return x, k, v
+    return x, k, v, r2
 
 
 def _frozen_stack(cfg, w, tok_in, pos):
@@ -166,7 +167,7 @@ def _static_adaptive_kv(cfg, w, x, pos, fast):
     with torch.no_grad():
         for j in range(cfg.n_ttt):
             l = cfg.n_layers - cfg.n_ttt + j
-            x, k, v = _adaptive_layer(cfg, w, l, fast[j], x, pos, empty, empty, none)
+            x, k, v, _ = _adaptive_layer(cfg, w, l, fast[j], x, pos, empty, empty, none)
             ks.append(k)
             vs.append(v)
     return ks, vs
@@ -218,14 +219,68 @@ def mini_batch_ttt_chunked(cfg, weights, tokens, cache_rule="as_computed"):
         pos = torch.arange(c0, c1)
         new = []
         for j in range(cfg.n_ttt):
-            x, k, v = _adaptive_layer(cfg, w, first + j, cur[j], x, pos, ks[j][lo:c0], vs[j][lo:c0],
-                                      torch.arange(lo, c0))
+            x, k, v, _ = _adaptive_layer(cfg, w, first + j, cur[j], x, pos, ks[j][lo:c0], vs[j][lo:c0],
+                                         torch.arange(lo, c0))
             new.append((k.detach(), v.detach()))
         rf = F.rms_norm(x, (cfg.d,), weight=w["final_norm"], eps=cfg.rms_eps)
         ell = F.cross_entropy(rf @ w["E"].T, tok[c0 + 1:c1 + 1], reduction="none")
         losses[c0:c1] = ell.detach()
         if c1 - c0 == b:
             (ell.sum() / b).backward()
+            fast = [{n: (t - cfg.eta * t.grad).detach() for n, t in f.items()} for f in cur]
+        for j in range(cfg.n_ttt):
+            k_cache[j] = torch.cat([k_cache[j], new[j][0]])
+            v_cache[j] = torch.cat([v_cache[j], new[j][1]])
+    return losses, fast
+
+
+# ----------------------------------------------------------------------------- key-value-binding inner loss
+
+def mini_batch_ttt_kvb_chunked(cfg, weights, tokens, layerwise=True):
+    """Mini-batch TTT with the key-value-binding inner loss, by autograd, chunk by chunk.
+
+    Each adaptive block j maps keys theta_K x to values theta_V x through its own MLP
+    W2t gelu(W1t .), x being the rows that enter that MLP; the chunk's inner loss of the
+    block is the summed squared error (library mse_loss) divided by b, and
+    W_i = W_{i-1} - eta * its gradient. With layerwise=True the rows x are taken as
+    given, so block j's loss moves only W_j; layerwise=False lets every block's loss
+    reach the earlier blocks' weights through x (a misreading, for negative controls).
+    Keys/values of earlier chunks are cached as computed. The recorded losses are the
+    next-token losses with W_{i-1}. Returns (losses [T], fast weights).
+    """
+    w = {k: _t(v) for k, v in weights.items()}
+    tok = torch.as_tensor(tokens, dtype=torch.long)
+    T = tok.shape[0] - 1
+    H, hd = cfg.n_heads, cfg.d // cfg.n_heads
+    b, first = cfg.minibatch_b, cfg.n_layers - cfg.n_ttt
+    x0 = _frozen_stack(cfg, w, tok[:T], torch.arange(T))
+    fast = initial_fast(cfg, weights)
+    k_cache = [torch.zeros(0, H, hd, dtype=torch.float64) for _ in range(cfg.n_ttt)]
+    v_cache = [torch.zeros(0, H, hd, dtype=torch.float64) for _ in range(cfg.n_ttt)]
+    losses = torch.zeros(T, dtype=torch.float64)
+    for c0 in range(0, T, b):
+        c1 = min(T, c0 + b)
+        cur = [{n: t.detach().clone().requires_grad_(True) for n, t in f.items()} for f in fast]
+        lo = max(0, c0 - cfg.window_k + 1)
+        x = x0[c0:c1]
+        pos = torch.arange(c0, c1)
+        new, inner = [], []
+        for j in range(cfg.n_ttt):
+            l = first + j
+            x, k, v, xin = _adaptive_layer(cfg, w, l, cur[j], x, pos, k_cache[j][lo:c0], v_cache[j][lo:c0],
+                                           torch.arange(lo, c0))
+            new.append((k.detach(), v.detach()))
+            if layerwise:
+                xin = xin.detach()
+            keys = xin @ w[f"layers.{l}.theta_K"].T
+            vals = xin @ w[f"layers.{l}.theta_V"].T
+            pred = F.gelu(keys @ cur[j]["W1t"].T, approximate="none") @ cur[j]["W2t"].T
+            inner.append(F.mse_loss(pred, vals, reduction="sum") / b)
+        with torch.no_grad():
+            rf = F.rms_norm(x, (cfg.d,), weight=w["final_norm"], eps=cfg.rms_eps)
+            losses[c0:c1] = F.cross_entropy(rf @ w["E"].T, tok[c0 + 1:c1 + 1], reduction="none")
+        if c1 - c0 == b:
+            sum(inner).backward()
             fast = [{n: (t - cfg.eta * t.grad).detach() for n, t in f.items()} for f in cur]
         for j in range(cfg.n_ttt):
             k_cache[j] = torch.cat([k_cache[j], new[j][0]])
