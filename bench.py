@@ -43,7 +43,11 @@ WORKLOAD = "b1_128k_bf16"
 def model_flops(cfg, T=None, B=None):
     """Algorithmic FLOPs of one prefill (forward of all blocks, LM head, backward
     into the adaptive MLPs); recompute, norms and elementwise work not counted.
-    Attention pairs P = sum_p min(p+1, k) (review eq. (1)); P_in = pairs inside chunks."""
+    Attention pairs P = sum_p min(p+1, k) (review eq. (1)); P_in = pairs inside chunks.
+    With the key-value-binding inner loss (review §8, eq. (10)) the update needs no
+    LM-head or cross-block backward: per adaptive block, the k and v projections
+    (2 x 2Td^2), the binding MLP forward (2 x 2Td h_t) and its backward into W1t, W2t
+    (3 x 2Td h_t)."""
     T = cfg.T if T is None else T
     B = cfg.batch if B is None else B
     d, V, L, Lt, h, ht, hs, k, b = (cfg.d, cfg.vocab, cfg.n_layers, cfg.n_ttt, cfg.mlp_hidden, cfg.ttt_hidden,
@@ -54,6 +58,8 @@ def model_flops(cfg, T=None, B=None):
     P_in = n_full * b * (b + 1) / 2 + (T % b) * ((T % b) + 1) / 2
     fwd = (L - Lt) * (8 * T * d * d + 4 * T * d * h + 4 * d * P) + \
         Lt * (8 * T * d * d + 4 * T * d * (ht + hs) + 4 * d * P) + 2 * T * d * V
+    if getattr(cfg, "inner_loss", "e2e") == "kvb":
+        return B * (fwd + Lt * (4 * T * d * d + 10 * T * d * ht))
     bwd = 2 * T * d * V
     for j in range(Lt):
         bwd += 4 * T * d * hs + 2 * T * d * ht * (3 if j == 0 else 4)
@@ -326,6 +332,32 @@ def run_full_attention(cfg, tok_dev, args, device):
             "model_tflop_per_step": model_flops(fcfg) / 1e12}
 
 
+def run_kvb_variant(cfg, tok_dev, args, device, peaks):
+    """The key-value-binding variant (technical review §8, eq. (10); summary,
+    "Alternative Derivation"): the same model and tokens, each adaptive block updated
+    by its own layer-wise reconstruction loss with frozen theta_K, theta_V instead of
+    the next-token loss. The pages give no step size for it; eta = 1e-3 keeps its
+    squared-error descent stable at this width. Reported beside the metric."""
+    import torch
+    import long_context_prefill_ttt_b200 as T
+    kcfg = cfg.replace(inner_loss="kvb", eta=1e-3)
+    w = syn.make_weights(kcfg)
+    wd = {k: torch.from_numpy(v).to(device) for k, v in w.items()}
+    del w
+    loss = torch.empty((kcfg.batch, kcfg.T), dtype=torch.float32, device=device)
+    h = T.ttt_create(kcfg, wd, max_segment=args.segment)
+    del wd
+    ms = _time_prefill(T, h, tok_dev, loss, args.kvb_steps, 1)
+    del h
+    torch.cuda.empty_cache()
+    fl = model_flops(kcfg)
+    tokens = kcfg.batch * kcfg.T
+    return {"workload": f"{kcfg.name} with the key-value-binding inner loss (eta {kcfg.eta})",
+            "tokens_per_s": tokens / (ms / 1e3), "ms_per_step": ms, "s_per_1k_tokens": ms / 1e3 / (tokens / 1e3),
+            "steps": args.kvb_steps, "warmup": 1, "model_tflop_per_step": fl / 1e12,
+            "frac_of_peak": fl / (ms / 1e3) / 1e12 / peaks["bf16"]}
+
+
 def run_ours(args):
     import torch
 
@@ -443,6 +475,17 @@ def run_ours(args):
         h = None
         comparator = run_full_attention(cfg, tok_dev, args, device)
         comparator["ttt_e2e_speedup"] = value / comparator["tokens_per_s"]
+    kvb = None
+    if args.kvb and rank == 0 and ws == 1 and cfg.n_ttt > 0:
+        if h is not None:
+            del h
+            torch.cuda.empty_cache()
+            h = None
+        try:
+            kvb = run_kvb_variant(cfg, tok_dev, args, device, peaks)
+            kvb["ttt_e2e_s_per_1k_tokens"] = (ms_max / args.steps) / 1e3 / (cfg.batch * cfg.T / 1e3)
+        except Exception as ex:  # the metric above stands without it
+            kvb = {"error": f"{type(ex).__name__}: {ex}"}
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -478,6 +521,8 @@ def run_ours(args):
         line["fixed_128k_tokens_sweep"] = sweep
     if comparator is not None:
         line["full_attention_comparator"] = comparator
+    if kvb is not None:
+        line["kvb_variant"] = kvb
     if rank == 0 and ws == 1 and args.cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(cfg, n_tokens=args.ref_tokens)
     if rank == 0:
@@ -507,6 +552,9 @@ def main():
     ap.add_argument("--no-comparator", dest="comparator", action="store_false",
                     help="skip the full-attention comparator (same architecture, no adaptive blocks, k >= T)")
     ap.add_argument("--comparator-steps", type=int, default=2)
+    ap.add_argument("--no-kvb", dest="kvb", action="store_false",
+                    help="skip the key-value-binding variant beside the metric")
+    ap.add_argument("--kvb-steps", type=int, default=2)
     ap.add_argument("--profile-steps", type=int, default=1,
                     help="steps of the separate instrumented pass that gives the per-class profile")
     ap.add_argument("--no-batched", dest="batched", action="store_false",

@@ -47,6 +47,19 @@ enum {
 };
 
 enum { TTT_FP32 = 0, TTT_BF16 = 1 };
+
+/* Inner loss that drives the fast-weight update (ttt_config.inner_loss).
+ *   TTT_LOSS_E2E: the next-token cross-entropy at the model's output, back-propagated
+ *     into every adaptive MLP (summary, "Test-Time Training (Inner Loop)"; technical
+ *     review §5 eq. (9)).
+ *   TTT_LOSS_KVB: the layer-wise key-value-binding variant (technical review §8,
+ *     eq. (10); summary, "Alternative Derivation (Connection to TTT-KVB)"): each
+ *     adaptive block fits its MLP g(k; W) = W2t gelu(W1t k) from k = theta_K x to
+ *     v = theta_V x, x the MLP's own normalised input, minimising
+ *     (1/b) sum_t ||g(theta_K x_t; W) - theta_V x_t||^2 over the chunk with respect
+ *     to its own W only. theta_K, theta_V are frozen [d][d] matrices of the block.
+ *     The recorded per-token losses stay the next-token losses under W_{i-1}. */
+enum { TTT_LOSS_E2E = 0, TTT_LOSS_KVB = 1 };
 enum { TTT_PTR_HOST = 0, TTT_PTR_DEVICE = 1 };
 
 typedef struct ttt_handle ttt_handle;
@@ -70,6 +83,7 @@ typedef struct {
   float rope_base;        /* RoPE base */
   int32_t dtype;          /* TTT_FP32 (fp32 everywhere) or TTT_BF16 (bf16 operands, fp32 accumulation and master fast weights) */
   int32_t max_segment;    /* positions per sequence processed per frozen-phase segment (0 = default 32768; rounded to b) */
+  int32_t inner_loss;     /* TTT_LOSS_E2E (default, 0) or TTT_LOSS_KVB */
   void* cuda_stream;      /* cudaStream_t to run on (NULL = legacy default stream) */
 } ttt_config;
 
@@ -80,7 +94,9 @@ typedef struct {
  *     attn_norm [d], Wq [d][d], Wk [d][d], Wv [d][d], Wo [d][d],
  *     frozen layer (l < L - L_t): mlp_norm [d], W1 [h][d], W2 [d][h]
  *     TTT layer    (l >= L - L_t): ttt_norm [d], W1t [h_t][d], W2t [d][h_t],
- *                                  static_norm [d], W1s [h_s][d], W2s [d][h_s]
+ *                                  static_norm [d], W1s [h_s][d], W2s [d][h_s],
+ *                                  and with inner_loss == TTT_LOSS_KVB also
+ *                                  theta_K [d][d], theta_V [d][d]
  * values_dtype: element type of the given arrays (TTT_FP32 float32, or TTT_BF16 raw bf16 bits);
  * norm gains are always float32. The library copies everything; the caller keeps its buffers. */
 typedef struct {

@@ -24,6 +24,7 @@ LIB_PATH = os.path.join(_PKG, "libttt_b200.so")
 TTT_OK, TTT_ERR_INVALID_ARG, TTT_ERR_OOM, TTT_ERR_CUDA = 0, -1, -2, -3
 TTT_ERR_TIMEOUT, TTT_ERR_STREAM, TTT_ERR_POISONED, TTT_ERR_UNSUPPORTED = -4, -5, -6, -7
 TTT_FP32, TTT_BF16 = 0, 1
+TTT_LOSS_E2E, TTT_LOSS_KVB = 0, 1
 TTT_PTR_HOST, TTT_PTR_DEVICE = 0, 1
 EPI_STORE, EPI_RESID, EPI_GELU, EPI_DGELU, EPI_SGD = 0, 1, 2, 3, 4
 ENGINE_AUTO, ENGINE_SIMT, ENGINE_MMA, ENGINE_TC1 = 0, 1, 2, 3
@@ -42,7 +43,8 @@ class ttt_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("vocab", "d", "n_layers", "n_heads", "n_ttt", "mlp_hidden",
                                               "ttt_hidden", "static_hidden", "window_k", "minibatch_b", "batch")] + \
                [("eta", ctypes.c_float), ("rms_eps", ctypes.c_float), ("rope_base", ctypes.c_float),
-                ("dtype", ctypes.c_int32), ("max_segment", ctypes.c_int32), ("cuda_stream", ctypes.c_void_p)]
+                ("dtype", ctypes.c_int32), ("max_segment", ctypes.c_int32), ("inner_loss", ctypes.c_int32),
+                ("cuda_stream", ctypes.c_void_p)]
 
 
 class ttt_weights(ctypes.Structure):
@@ -199,6 +201,8 @@ def make_config(cfg, stream=None, max_segment=0) -> ttt_config:
     dt = _get(cfg, "dtype", "bf16")
     c.dtype = TTT_BF16 if dt in ("bf16", TTT_BF16) else TTT_FP32
     c.max_segment = int(max_segment or _get(cfg, "max_segment", 0) or 0)
+    loss = _get(cfg, "inner_loss", "e2e")
+    c.inner_loss = TTT_LOSS_KVB if loss in ("kvb", TTT_LOSS_KVB) else TTT_LOSS_E2E
     c.cuda_stream = _stream_ptr(stream).value
     return c
 
@@ -212,6 +216,8 @@ def weight_names(cfg):
         names += [p + n for n in ("attn_norm", "Wq", "Wk", "Wv", "Wo")]
         if l >= L - Lt:
             names += [p + n for n in ("ttt_norm", "W1t", "W2t", "static_norm", "W1s", "W2s")]
+            if _get(cfg, "inner_loss", "e2e") in ("kvb", TTT_LOSS_KVB):
+                names += [p + "theta_K", p + "theta_V"]
         else:
             names += [p + n for n in ("mlp_norm", "W1", "W2")]
     return names
@@ -255,6 +261,8 @@ def weight_shapes(cfg):
         out += [d, d * d, d * d, d * d, d * d]
         if l >= L - Lt:
             out += [d, ht * d, d * ht, d, hs * d, d * hs]
+            if _get(cfg, "inner_loss", "e2e") in ("kvb", TTT_LOSS_KVB):
+                out += [d * d, d * d]
         else:
             out += [d, h * d, d * h]
     return out

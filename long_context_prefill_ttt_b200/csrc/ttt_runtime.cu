@@ -759,6 +759,7 @@ template <typename T> struct LayerDev {
   float* W1t32 = nullptr; float* W2t32 = nullptr;                      // [B][ht][d], [B][d][ht]
   T* W1t = nullptr; T* W2t = nullptr;
   T* W1t_init = nullptr; T* W2t_init = nullptr;                        // [ht][d], [d][ht]
+  T* theta_kv = nullptr;  // key-value-binding inner loss: theta_K [d][d] then theta_V [d][d]
   T* ring_k = nullptr; T* ring_v = nullptr;                            // [B][C][d]
 };
 
@@ -776,6 +777,7 @@ template <typename T> class Engine : public ttt_handle {
   int B, d, V, L, Lt, H, hd, h, ht, hs, kwin, bsz, C, S;
   int first_ttt;
   bool is_bf16;
+  bool kvb = false;  // inner loss: layer-wise key-value binding instead of the next-token loss
   Arena arena;
   int* dev_err = nullptr;
   T* E = nullptr;
@@ -918,6 +920,7 @@ template <typename T> class Engine : public ttt_handle {
   int frozen_mlp(const LayerDev<T>& Lw, float* x, T* r, T* hid, int rows);
   int ttt_forward(int cn, int64_t pos, bool commit);
   int ttt_backward(int cn);
+  int kvb_update(int cn);
   int decode_token_launches(int64_t n, int32_t* otok, float* oloss, const int32_t* fdev, int64_t base);
   int ttt_step(const float* in, const int32_t* targets, int cn, int64_t pos, float* loss_out, int64_t loss_ld,
                int64_t loss_off, bool grad, bool commit);
@@ -961,6 +964,7 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
   bsz = cfg.minibatch_b;
   first_ttt = L - Lt;
   is_bf16 = cfg.dtype == TTT_BF16;
+  kvb = cfg.inner_loss == TTT_LOSS_KVB;
   C = ((kwin + bsz + 127) / 128) * 128;
   int seg = cfg.max_segment > 0 ? cfg.max_segment : 32768;
   S = ((seg + bsz - 1) / bsz) * bsz;
@@ -997,6 +1001,7 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
       Lw.W2t32 = arena.get<float>((size_t)B * d * ht);
       Lw.W1t_init = arena.get<T>((size_t)ht * d);
       Lw.W2t_init = arena.get<T>((size_t)d * ht);
+      if (kvb) Lw.theta_kv = arena.get<T>((size_t)2 * d * d);
       if (is_bf16) {
         Lw.W1t = arena.get<T>((size_t)B * ht * d);
         Lw.W2t = arena.get<T>((size_t)B * d * ht);
@@ -1151,6 +1156,10 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
       UP(Lw.g_static, true, d, true);
       UP(Lw.W1s, false, (int64_t)hs * d, false);
       UP(Lw.W2s, false, (int64_t)d * hs, false);
+      if (kvb) {
+        UP(Lw.theta_kv, false, dd, false);
+        UP(Lw.theta_kv + dd, false, dd, false);
+      }
     }
   }
 #undef UP
@@ -1438,6 +1447,64 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
   return TTT_OK;
 }
 
+// Key-value-binding variant of the update (technical review §8, eq. (10); summary,
+// "Alternative Derivation"): every adaptive block j descends its own chunk loss
+// (1/b) sum_t ||W2t gelu(W1t k_t) - v_t||^2 with k = theta_K r2, v = theta_V r2 and r2
+// the normalised input of its MLP from this chunk's forward (W_{i-1}). Layer-wise: no
+// gradient passes between blocks, so each block's update reads only its own forward
+// rows and fast weights, and the order of the blocks does not matter. With e the
+// residual, de = (2/b) e, du = (de W2t) * gelu'(u), dW2t = de^T gelu(u), dW1t = du^T k.
+// The forward's MLP activations of the block are dead once its forward ran (no backward
+// reads them in this mode), so u and gelu(u) of the binding loss reuse them; k goes to
+// the attention-gradient buffer dob and the fp32 residual to G.
+template <typename T> int Engine<T>::kvb_update(int cn) {
+  const int rows = B * cn;
+  int rc;
+  const float two_over_b = 2.0f / (float)bsz;
+  for (int j = 0; j < Lt; ++j) {
+    const LayerDev<T>& Lw = layers[first_ttt + j];
+    BlockAct<T>& A = blk[j];
+    T* kb = dob;  // k = r2 theta_K^T  [rows][d]
+    // k (element type) and G = -(2/b) v (fp32): two products over the same rows
+    GemmParams pk = gp(rows, d, d, A.r2, d, false, Lw.theta_kv, d, false, kb, d, false, EPI_STORE);
+    GemmParams pv = gp(rows, d, d, A.r2, d, false, Lw.theta_kv + (size_t)d * d, d, false, G, d, true, EPI_STORE);
+    pv.alpha = -two_over_b;
+    if ((rc = gemm2(pk, pv)) != TTT_OK) return rc;
+    // u = k W1t^T (kept in A.u), gelu(u) (in A.g), per sequence with W_{i-1}
+    GemmParams p = gp(cn, ht, d, kb, d, false, Lw.W1t, d, false, A.g, ht, false, EPI_GELU);
+    p.batch = B; p.sA = (int64_t)cn * d; p.sD = (int64_t)cn * ht;
+    fast_operand(p, Lw.W1t_init, Lw.W1t, (int64_t)ht * d);
+    p.Y = A.u; p.ldy = ht; p.sY = (int64_t)cn * ht;
+    if ((rc = gemm(p)) != TTT_OK) return rc;
+    // G = (2/b) (gelu(u) W2t^T - v) = de, in place over -(2/b) v
+    p = gp(cn, d, ht, A.g, ht, false, Lw.W2t, ht, false, G, d, true, EPI_RESID);
+    p.batch = B; p.sA = (int64_t)cn * ht; p.sD = (int64_t)cn * d;
+    fast_operand(p, Lw.W2t_init, Lw.W2t, (int64_t)d * ht);
+    p.X = G; p.ldx = d; p.sX = (int64_t)cn * d;
+    p.alpha = two_over_b;
+    if ((rc = gemm(p)) != TTT_OK) return rc;
+    convert_kernel<float, T><<<nblk((int64_t)rows * d, 256), 256, 0, st>>>(G, GT, (int64_t)rows * d);
+    TTT_LAUNCHED();
+    // du = (de W2t) * gelu'(u)
+    p = gp(cn, ht, d, GT, d, false, Lw.W2t, ht, true, dhid, ht, false, EPI_DGELU);
+    p.batch = B; p.sA = (int64_t)cn * d; p.sD = (int64_t)cn * ht;
+    fast_operand(p, Lw.W2t_init, Lw.W2t, (int64_t)d * ht);
+    p.X = A.u; p.ldx = ht; p.sX = (int64_t)cn * ht;
+    if ((rc = gemm(p)) != TTT_OK) return rc;
+    // W2t -= eta de^T gelu(u), W1t -= eta du^T k: one launch, SGD fused into the epilogue
+    GemmParams p2w = gp(d, ht, cn, GT, d, true, A.g, ht, true, Lw.W2t32, ht, true, EPI_SGD);
+    p2w.batch = B; p2w.sA = (int64_t)cn * d; p2w.sB = (int64_t)cn * ht; p2w.sD = (int64_t)d * ht;
+    p2w.alpha = -cfg.eta;
+    if (is_bf16) { p2w.Y = Lw.W2t; p2w.ldy = ht; p2w.sY = (int64_t)d * ht; }
+    GemmParams p1w = gp(ht, d, cn, dhid, ht, true, kb, d, true, Lw.W1t32, d, true, EPI_SGD);
+    p1w.batch = B; p1w.sA = (int64_t)cn * ht; p1w.sB = (int64_t)cn * d; p1w.sD = (int64_t)ht * d;
+    p1w.alpha = -cfg.eta;
+    if (is_bf16) { p1w.Y = Lw.W1t; p1w.ldy = d; p1w.sY = (int64_t)ht * d; }
+    if ((rc = gemm2(p2w, p1w)) != TTT_OK) return rc;
+  }
+  return TTT_OK;
+}
+
 }  // namespace ttt
 
 namespace ttt {
@@ -1467,7 +1534,8 @@ int Engine<T>::ttt_step(const float* in, const int32_t* targets, int cn, int64_t
   // the logits. The gradient is the mean over the b positions of the chunk
   // (summary: mini-batch GD with 1/b).
   GemmParams ph = gp(rows, V, d, rf, d, false, E, d, false, z, V, false, EPI_STORE);
-  const float gscale = grad ? 1.0f / bsz : 0.f;
+  // the key-value-binding variant needs no dz: its update never reads the head's gradient
+  const float gscale = (grad && !kvb) ? 1.0f / bsz : 0.f;
   bool fused = false;
   if (ce_part) {
     GemmParams pc = ph;
@@ -1483,7 +1551,7 @@ int Engine<T>::ttt_step(const float* in, const int32_t* targets, int cn, int64_t
   }
   TTT_LAUNCHED();
   if (grad) {
-    if ((rc = ttt_backward(cn)) != TTT_OK) return rc;
+    if ((rc = kvb ? kvb_update(cn) : ttt_backward(cn)) != TTT_OK) return rc;
   }
   return TTT_OK;
 }
@@ -1731,6 +1799,8 @@ static int validate(const ttt_config* c, std::string* why) {
     return bad("widths and vocab must be multiples of 8");
   if (c->mlp_hidden <= 0 || c->ttt_hidden <= 0 || c->static_hidden <= 0) return bad("non-positive hidden width");
   if (c->dtype != TTT_FP32 && c->dtype != TTT_BF16) return bad("dtype must be TTT_FP32 or TTT_BF16");
+  if (c->inner_loss != TTT_LOSS_E2E && c->inner_loss != TTT_LOSS_KVB)
+    return bad("inner_loss must be TTT_LOSS_E2E or TTT_LOSS_KVB");
   if (!(c->rms_eps > 0.f) || !(c->rope_base > 1.f) || !std::isfinite(c->eta)) return bad("bad eps, rope base or eta");
   return TTT_OK;
 }
@@ -1744,7 +1814,7 @@ extern "C" {
 
 int32_t ttt_num_weight_tensors(const ttt_config* c) {
   if (!c) return -1;
-  return 2 + (c->n_layers - c->n_ttt) * 8 + c->n_ttt * 11;
+  return 2 + (c->n_layers - c->n_ttt) * 8 + c->n_ttt * (c->inner_loss == TTT_LOSS_KVB ? 13 : 11);
 }
 
 int ttt_create(const ttt_config* cfg, const ttt_weights* w, ttt_handle** out) {

@@ -42,9 +42,11 @@ def test_library_exports_every_declared_symbol():
 
 def test_weight_tensor_count_and_order_match_the_generator():
     import long_context_prefill_ttt_b200 as T
-    for name in ("tiny_fp32", "small_bf16", "b1_128k_bf16"):
-        cfg = syn.config(name)
+    for name, loss in (("tiny_fp32", "e2e"), ("small_bf16", "e2e"), ("b1_128k_bf16", "e2e"),
+                       ("tiny_fp32", "kvb"), ("small_bf16", "kvb")):
+        cfg = syn.config(name, inner_loss=loss)
         c = T.make_config(cfg)
+        assert c.inner_loss == (T.TTT_LOSS_KVB if loss == "kvb" else T.TTT_LOSS_E2E)
         assert T.lib.ttt_num_weight_tensors(ctypes.byref(c)) == len(syn.weight_shapes(cfg))
         assert T.weight_names(cfg) == [n for n, _ in syn.weight_shapes(cfg)]
 
@@ -61,6 +63,16 @@ def test_create_rejects_invalid_configs_without_touching_the_device(field, value
     w = T.ttt_weights()
     rc = T.lib.ttt_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(out))
     assert rc == T.TTT_ERR_INVALID_ARG
+    assert not out.value
+
+
+def test_create_rejects_an_unknown_inner_loss():
+    import long_context_prefill_ttt_b200 as T
+    c = T.make_config(syn.config("tiny_fp32"))
+    c.inner_loss = 2
+    out = ctypes.c_void_p()
+    w = T.ttt_weights()
+    assert T.lib.ttt_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(out)) == T.TTT_ERR_INVALID_ARG
     assert not out.value
 
 

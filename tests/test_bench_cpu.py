@@ -40,6 +40,14 @@ def _direct_model_flops(cfg):
             fwd += mm(T, cfg.ttt_hidden, d) + mm(T, d, cfg.ttt_hidden)
             fwd += mm(T, cfg.static_hidden, d) + mm(T, d, cfg.static_hidden)
     fwd += mm(T, V, d)
+    if cfg.inner_loss == "kvb":                        # each block's binding loss only
+        upd = 0.0
+        for j in range(Lt):
+            upd += mm(T, d, d) + mm(T, d, d)                                   # k, v projections
+            upd += mm(T, cfg.ttt_hidden, d) + mm(T, d, cfg.ttt_hidden)         # g(k; W)
+            upd += mm(T, cfg.ttt_hidden, d)                                    # du = de W2t
+            upd += mm(cfg.ttt_hidden, d, T) + mm(d, cfg.ttt_hidden, T)         # dW1t, dW2t
+        return (fwd + upd) * cfg.batch
     bwd = mm(T, d, V)                                  # dh = dz E
     for j in range(Lt):
         bwd += mm(T, cfg.static_hidden, d) + mm(T, d, cfg.static_hidden)   # static MLP data gradient
@@ -54,7 +62,8 @@ def _direct_model_flops(cfg):
 
 @pytest.mark.parametrize("name,overrides", [("tiny_fp32", {}), ("small_bf16", {"T": 4096}),
                                             ("tiny_fp32", {"n_ttt": 0, "window_k": 256}),
-                                            ("tiny_fp32", {"n_ttt": 3, "T": 200})])
+                                            ("tiny_fp32", {"n_ttt": 3, "T": 200}),
+                                            ("small_bf16", {"T": 4096, "inner_loss": "kvb"})])
 def test_model_flops_equals_the_product_by_product_count(name, overrides):
     cfg = syn.config(name, **overrides)
     assert bench.model_flops(cfg) == pytest.approx(_direct_model_flops(cfg), rel=1e-12)
