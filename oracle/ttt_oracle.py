@@ -47,9 +47,13 @@ Variant with the layer-wise key-value-binding inner loss (cfg.inner_loss ==
 (Connection to TTT-KVB)"): each adaptive block's fast weights W = (W1t, W2t)
 fit g(theta_K x_t; W) to theta_V x_t instead of descending the next-token loss.
 Readings taken:
-  K1 x_t is the adaptive MLP's own input (the block's RMSNorm output r2), and
-     g(k; W) = W2t gelu(W1t k) is the same two-layer MLP the block applies to r2
-     on its output path; theta_K, theta_V are frozen d x d matrices of the block.
+  K1 x_t is the block's RMSNorm output r2 ahead of its adaptive MLP, and
+     g(k; W) = W2t gelu(W1t k) is the adaptive two-layer MLP; theta_K, theta_V are
+     frozen d x d matrices of the block. Output rule: the sub-layer's output is the
+     binding prediction itself, m = a + g(theta_K r2; W_{i-1}), i.e. the pre-update
+     weights and the key projection (technical review §8: the simplified
+     construction; summary, "Alternative Derivation", step 3, Simplified Output
+     Rule: the prediction of g is reused as the output embedding).
   K2 the chunk's inner loss is (1/b) sum_t ||g(theta_K x_t; W) - theta_V x_t||^2
      (squared Euclidean norm, mean over the b positions as in R9); each block
      descends its own loss w.r.t. its own W only (layer-wise: no gradient passes
@@ -262,14 +266,16 @@ class Oracle:
         fw = seq.fast[j]
         a, c = self._attn(seq, l, x, s, commit, keep)
         r2, rstd2 = rms_norm(a, w[p + "ttt_norm"], cfg.rms_eps)
-        u = r2 @ fw["W1t"].T
+        # key-value binding (reading K1): the MLP reads the key projection of r2
+        xin = r2 @ w[p + "theta_K"].T if getattr(cfg, "inner_loss", "e2e") == "kvb" else r2
+        u = xin @ fw["W1t"].T
         g = gelu(u)
         m = a + g @ fw["W2t"].T
         r3, rstd3 = rms_norm(m, w[p + "static_norm"], cfg.rms_eps)
         us = r3 @ w[p + "W1s"].T
         y = m + gelu(us) @ w[p + "W2s"].T
         if keep:
-            c.update(a=a, rstd2=rstd2, r2=r2, u=u, g=g, m=m, rstd3=rstd3, us=us)
+            c.update(a=a, rstd2=rstd2, r2=r2, xin=xin, u=u, g=g, m=m, rstd3=rstd3, us=us)
         return y, c
 
     def _head(self, y):
@@ -346,11 +352,10 @@ class Oracle:
         for j in range(cfg.n_ttt):
             p = f"layers.{cfg.first_ttt + j}."
             fw = seq.fast[j]
-            x = caches[j]["r2"]
-            k = x @ w[p + "theta_K"].T
-            v = x @ w[p + "theta_V"].T
-            u = k @ fw["W1t"].T
-            g = gelu(u)
+            c = caches[j]
+            k = c["xin"]                      # theta_K r2: the MLP's input (reading K1)
+            v = c["r2"] @ w[p + "theta_V"].T
+            u, g = c["u"], c["g"]             # the forward's prediction g(k; W_{i-1})
             e = g @ fw["W2t"].T - v
             losses.append(float(np.sum(e * e)) / cfg.minibatch_b)
             de = (2.0 / cfg.minibatch_b) * e

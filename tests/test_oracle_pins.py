@@ -442,7 +442,10 @@ def test_kvb_trajectory_matches_chunkwise_autograd(n_ttt, b, k, T):
     chunk-wise loop (library mse_loss, SDPA and autograd, tests/torch_static.py): losses
     and final fast weights. Negative controls: letting each block's loss reach the
     earlier blocks' weights (not layer-wise) and the next-token inner loss both move the
-    first adaptive block's weights far outside the tolerance."""
+    first adaptive block's weights far outside the tolerance, and applying the MLP to
+    the normalised rows themselves on the output path (instead of reusing the
+    prediction from the key projection, technical review §8 / summary step 3) moves
+    the recorded losses far outside it."""
     cfg = tiny_kvb(n_ttt=n_ttt, minibatch_b=b, window_k=k, T=T)
     w = weights(cfg)
     toks = tokens(cfg)
@@ -461,12 +464,15 @@ def test_kvb_trajectory_matches_chunkwise_autograd(n_ttt, b, k, T):
     e2e = Oracle(cfg.replace(inner_loss="e2e"), w)
     e2e.prefill(toks)
     assert np.max(np.abs(e2e.fast_weights(0, 0)[0] - W1_0)) > 1e-6
+    other, _ = TS.mini_batch_ttt_kvb_chunked(cfg, w, toks[0], output_from_keys=False)
+    assert np.max(np.abs(other.numpy() - losses[0])) > 1e-6
 
 
 def test_kvb_zero_key_projection_never_moves_the_weights():
-    """theta_K = 0: every key is 0, so gelu(W1t k) = 0 and both weight gradients vanish
-    (dW2t pairs the error with gelu(0) = 0, dW1t pairs it with k = 0): the prefill is
-    the static model's and the fast weights stay W_init."""
+    """theta_K = 0: every key is 0, so the MLP's prediction gelu(W1t k) W2t, which is
+    also the sub-layer's output, is 0, and both weight gradients vanish (dW2t pairs the
+    error with gelu(0) = 0, dW1t pairs it with k = 0): the prefill is the static model
+    without the adaptive MLPs (their W2t zeroed) and the fast weights stay W_init."""
     cfg = tiny_kvb(n_ttt=2, T=16)
     w = weights(cfg)
     for l in range(cfg.first_ttt, cfg.n_layers):
@@ -474,7 +480,11 @@ def test_kvb_zero_key_projection_never_moves_the_weights():
     toks = tokens(cfg)
     orc = Oracle(cfg, w)
     losses = orc.prefill(toks)
-    np.testing.assert_allclose(losses[0], TS.static_forward(cfg, w, toks[0]).numpy(), rtol=1e-10, atol=1e-12)
+    w_off = dict(w)
+    for l in range(cfg.first_ttt, cfg.n_layers):
+        w_off[f"layers.{l}.W2t"] = np.zeros_like(w[f"layers.{l}.W2t"])
+    np.testing.assert_allclose(losses[0], TS.static_forward(cfg, w_off, toks[0]).numpy(), rtol=1e-10, atol=1e-12)
+    assert np.max(np.abs(losses[0] - TS.static_forward(cfg, w, toks[0]).numpy())) > 1e-6
     for j in range(cfg.n_ttt):
         l = cfg.first_ttt + j
         assert np.array_equal(orc.fast_weights(0, j)[0], w[f"layers.{l}.W1t"].astype(np.float64))

@@ -115,11 +115,12 @@ def _attend(q, keys, vals, q_pos, k_pos, window):
     return o.transpose(0, 1)
 
 
-def _adaptive_layer(cfg, w, l, fast_j, x, pos, k_hist, v_hist, hist_pos):
+def _adaptive_layer(cfg, w, l, fast_j, x, pos, k_hist, v_hist, hist_pos, mlp_in=None):
     """One adaptive block over rows x at positions pos; attention sees the given
-    earlier keys/values (constants) and the rows' own keys/values.
-    Returns (output, post-RoPE keys of the rows, values of the rows, the rows that enter
-    the adaptive MLP)."""
+    earlier keys/values (constants) and the rows' own keys/values. mlp_in, when given,
+    maps the normalised rows to the adaptive MLP's input (the key projection of the
+    key-value-binding variant). Returns (output, post-RoPE keys of the rows, values of
+    the rows, the normalised rows ahead of the adaptive MLP)."""
     d, H = cfg.d, cfg.n_heads
     hd = d // H
     n = x.shape[0]
@@ -133,7 +134,8 @@ def _adaptive_layer(cfg, w, l, fast_j, x, pos, k_hist, v_hist, hist_pos):
     o = _attend(q, keys, vals, pos, torch.cat([hist_pos, pos]), cfg.window_k)
     x = x + o.reshape(n, d) @ w[p + "Wo"].T
     r2 = F.rms_norm(x, (d,), weight=w[p + "ttt_norm"], eps=cfg.rms_eps)
-    x = x + F.gelu(r2 @ fast_j["W1t"].T, approximate="none") @ fast_j["W2t"].T
+    xin = r2 if mlp_in is None else mlp_in(r2)
+    x = x + F.gelu(xin @ fast_j["W1t"].T, approximate="none") @ fast_j["W2t"].T
     r3 = F.rms_norm(x, (d,), weight=w[p + "static_norm"], eps=cfg.rms_eps)
     x = x + F.gelu(r3 @ w[p + "W1s"].T, approximate="none") @ w[p + "W2s"].T
     return x, k, v, r2
@@ -236,17 +238,20 @@ def mini_batch_ttt_chunked(cfg, weights, tokens, cache_rule="as_computed"):
 
 # ----------------------------------------------------------------------------- key-value-binding inner loss
 
-def mini_batch_ttt_kvb_chunked(cfg, weights, tokens, layerwise=True):
+def mini_batch_ttt_kvb_chunked(cfg, weights, tokens, layerwise=True, output_from_keys=True):
     """Mini-batch TTT with the key-value-binding inner loss, by autograd, chunk by chunk.
 
     Each adaptive block j maps keys theta_K x to values theta_V x through its own MLP
-    W2t gelu(W1t .), x being the rows that enter that MLP; the chunk's inner loss of the
-    block is the summed squared error (library mse_loss) divided by b, and
-    W_i = W_{i-1} - eta * its gradient. With layerwise=True the rows x are taken as
-    given, so block j's loss moves only W_j; layerwise=False lets every block's loss
-    reach the earlier blocks' weights through x (a misreading, for negative controls).
-    Keys/values of earlier chunks are cached as computed. The recorded losses are the
-    next-token losses with W_{i-1}. Returns (losses [T], fast weights).
+    W2t gelu(W1t .), x being the block's normalised rows ahead of that MLP; the chunk's
+    inner loss of the block is the summed squared error (library mse_loss) divided by
+    b, and W_i = W_{i-1} - eta * its gradient. The block's MLP output is the same
+    prediction, g(theta_K x; W_{i-1}) (output_from_keys=False applies g to x itself on
+    the output path instead: a misreading, for negative controls). With layerwise=True
+    the rows x are taken as given, so block j's loss moves only W_j; layerwise=False
+    lets every block's loss reach the earlier blocks' weights through x (a misreading,
+    for negative controls). Keys/values of earlier chunks are cached as computed. The
+    recorded losses are the next-token losses with W_{i-1}. Returns (losses [T], fast
+    weights).
     """
     w = {k: _t(v) for k, v in weights.items()}
     tok = torch.as_tensor(tokens, dtype=torch.long)
@@ -267,8 +272,10 @@ def mini_batch_ttt_kvb_chunked(cfg, weights, tokens, layerwise=True):
         new, inner = [], []
         for j in range(cfg.n_ttt):
             l = first + j
+            theta_k = w[f"layers.{l}.theta_K"]
+            proj = (lambda r, th=theta_k: r @ th.T) if output_from_keys else None
             x, k, v, xin = _adaptive_layer(cfg, w, l, cur[j], x, pos, k_cache[j][lo:c0], v_cache[j][lo:c0],
-                                           torch.arange(lo, c0))
+                                           torch.arange(lo, c0), mlp_in=proj)
             new.append((k.detach(), v.detach()))
             if layerwise:
                 xin = xin.detach()
