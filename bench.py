@@ -44,10 +44,10 @@ def model_flops(cfg, T=None, B=None):
     """Algorithmic FLOPs of one prefill (forward of all blocks, LM head, backward
     into the adaptive MLPs); recompute, norms and elementwise work not counted.
     Attention pairs P = sum_p min(p+1, k) (review eq. (1)); P_in = pairs inside chunks.
-    With the key-value-binding inner loss (review §8, eq. (10)) the update needs no
-    LM-head or cross-block backward: per adaptive block, the k and v projections
-    (2 x 2Td^2), the binding MLP forward (2 x 2Td h_t) and its backward into W1t, W2t
-    (3 x 2Td h_t)."""
+    With the key-value-binding inner loss (review §8, eq. (10)) the adaptive MLP reads
+    the key projection (2Td^2 more forward per block), and the update needs no LM-head
+    or cross-block backward: per adaptive block, the value projection (2Td^2) and the
+    binding MLP's backward into W1t, W2t (3 x 2Td h_t); its forward is the block's."""
     T = cfg.T if T is None else T
     B = cfg.batch if B is None else B
     d, V, L, Lt, h, ht, hs, k, b = (cfg.d, cfg.vocab, cfg.n_layers, cfg.n_ttt, cfg.mlp_hidden, cfg.ttt_hidden,
@@ -59,7 +59,7 @@ def model_flops(cfg, T=None, B=None):
     fwd = (L - Lt) * (8 * T * d * d + 4 * T * d * h + 4 * d * P) + \
         Lt * (8 * T * d * d + 4 * T * d * (ht + hs) + 4 * d * P) + 2 * T * d * V
     if getattr(cfg, "inner_loss", "e2e") == "kvb":
-        return B * (fwd + Lt * (4 * T * d * d + 10 * T * d * ht))
+        return B * (fwd + Lt * (4 * T * d * d + 6 * T * d * ht))
     bwd = 2 * T * d * V
     for j in range(Lt):
         bwd += 4 * T * d * hs + 2 * T * d * ht * (3 if j == 0 else 4)
@@ -224,7 +224,7 @@ def run_decode(T, args, device):
             "gpu_launches": launches}
 
 
-def _time_prefill(T, h, tok, loss, steps, warmup):
+def _time_prefill(T, h, tok, loss, steps, warmup, check=True):
     """Device time (ms) of `steps` reset+prefill calls after `warmup` untimed ones."""
     import torch
     for _ in range(warmup):
@@ -238,7 +238,8 @@ def _time_prefill(T, h, tok, loss, steps, warmup):
         T.ttt_prefill(h, tok, loss)
     e1.record()
     torch.cuda.synchronize()
-    assert torch.isfinite(loss).all().item(), "non-finite loss"
+    if check:
+        assert torch.isfinite(loss).all().item(), "non-finite loss"
     return e0.elapsed_time(e1) / steps
 
 
@@ -336,20 +337,26 @@ def run_kvb_variant(cfg, tok_dev, args, device, peaks):
     """The key-value-binding variant (technical review §8, eq. (10); summary,
     "Alternative Derivation"): the same model and tokens, each adaptive block updated
     by its own layer-wise reconstruction loss with frozen theta_K, theta_V instead of
-    the next-token loss. The pages give no step size for it; eta = 1e-3 keeps its
-    squared-error descent stable at this width. Reported beside the metric."""
+    the next-token loss. The pages give no step size for it; its squared error sums
+    over d outputs, so the step that suits the next-token loss diverges at this width,
+    and --kvb-eta (default 1e-4) sets it. The cost does not depend on it. Reported
+    beside the metric."""
     import torch
     import long_context_prefill_ttt_b200 as T
-    kcfg = cfg.replace(inner_loss="kvb", eta=1e-3)
+    kcfg = cfg.replace(inner_loss="kvb", eta=args.kvb_eta)
     w = syn.make_weights(kcfg)
     wd = {k: torch.from_numpy(v).to(device) for k, v in w.items()}
     del w
     loss = torch.empty((kcfg.batch, kcfg.T), dtype=torch.float32, device=device)
     h = T.ttt_create(kcfg, wd, max_segment=args.segment)
     del wd
-    ms = _time_prefill(T, h, tok_dev, loss, args.kvb_steps, 1)
+    ms = _time_prefill(T, h, tok_dev, loss, args.kvb_steps, 1, check=False)
     del h
     torch.cuda.empty_cache()
+    bad = (~torch.isfinite(loss)).nonzero()
+    if bad.numel():
+        raise FloatingPointError(f"non-finite loss from position {int(bad[0, 1])} "
+                                 f"(chunk {int(bad[0, 1]) // kcfg.minibatch_b})")
     fl = model_flops(kcfg)
     tokens = kcfg.batch * kcfg.T
     return {"workload": f"{kcfg.name} with the key-value-binding inner loss (eta {kcfg.eta})",
@@ -555,6 +562,7 @@ def main():
     ap.add_argument("--no-kvb", dest="kvb", action="store_false",
                     help="skip the key-value-binding variant beside the metric")
     ap.add_argument("--kvb-steps", type=int, default=2)
+    ap.add_argument("--kvb-eta", type=float, default=1e-4)
     ap.add_argument("--profile-steps", type=int, default=1,
                     help="steps of the separate instrumented pass that gives the per-class profile")
     ap.add_argument("--no-batched", dest="batched", action="store_false",

@@ -518,6 +518,33 @@ __global__ void convert_kernel(const S* __restrict__ src, D* __restrict__ dst, i
   if (i < n) dst[i] = from_f32<D>(to_f32(src[i]));
 }
 
+// Residual of the key-value-binding loss of one adaptive block, scaled to its gradient:
+// G = s (m - a) + G, where m - a is the MLP's prediction (its sub-layer output) and G
+// holds -s v on entry (s = 2/b); GT receives G in the element type. n4 = elements / 4;
+// all pointers 16-byte aligned (rows of d % 8 == 0 elements in 256-byte aligned buffers).
+template <typename T>
+__global__ void __launch_bounds__(256) kvb_residual_kernel(const float* __restrict__ m, const float* __restrict__ a,
+                                                           float* __restrict__ G, T* __restrict__ GT, float s,
+                                                           int64_t n4) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  const float4 mv = reinterpret_cast<const float4*>(m)[i];
+  const float4 av = reinterpret_cast<const float4*>(a)[i];
+  float4 g = reinterpret_cast<float4*>(G)[i];
+  g.x += s * (mv.x - av.x);
+  g.y += s * (mv.y - av.y);
+  g.z += s * (mv.z - av.z);
+  g.w += s * (mv.w - av.w);
+  reinterpret_cast<float4*>(G)[i] = g;
+  T* o = GT + 4 * i;
+  o[0] = from_f32<T>(g.x);
+  o[1] = from_f32<T>(g.y);
+  o[2] = from_f32<T>(g.z);
+  o[3] = from_f32<T>(g.w);
+}
+
 // out = init + delta (fast weights W_init + dW exported in fp32)
 template <typename T>
 __global__ void add_init_kernel(const T* __restrict__ init, const float* __restrict__ delta, float* __restrict__ out,

@@ -767,6 +767,7 @@ template <typename T> struct LayerDev {
 template <typename T> struct BlockAct {
   float* x; float* rstd1; T* qkv; T* o; float* lse; float* a; float* rstd2; T* r2; T* u; T* g;
   float* m; float* rstd3; T* r3; T* us; T* gs;
+  T* k;  // key-value-binding variant: the adaptive MLP's input theta_K r2 (else unused)
 };
 
 template <typename T> class Engine : public ttt_handle {
@@ -1035,6 +1036,7 @@ template <typename T> int Engine<T>::create(const ttt_config* c, const ttt_weigh
     A.r3 = arena.get<T>((size_t)Mc * d);
     A.us = arena.get<T>((size_t)Mc * hs);
     A.gs = arena.get<T>((size_t)Mc * hs);
+    A.k = kvb ? arena.get<T>((size_t)Mc * d) : nullptr;
   }
   // chunk input: the first adaptive block's input buffer, or its own buffer without adaptive blocks
   tin = blk.empty() ? arena.get<float>((size_t)Mc * d) : blk[0].x;
@@ -1319,10 +1321,17 @@ template <typename T> int Engine<T>::ttt_forward(int cn, int64_t pos, bool commi
     if ((rc = attention_block(Lw, l, A.x, A.a, A.r3 /*scratch for r1*/, A.rstd1, A.qkv, A.o, A.lse, cn, pos,
                               commit)) != TTT_OK)
       return rc;
-    // TTT-MLP with the fast weights of each sequence (batched over sequences)
-    GemmParams p = gp(cn, ht, d, A.r2, d, false, Lw.W1t, d, false, A.g, ht, false, EPI_GELU);
+    // TTT-MLP with the fast weights of each sequence (batched over sequences). In the
+    // key-value-binding variant it reads the key projection k = theta_K r2, and its
+    // output is that binding prediction (the pre-update weights, the key projection).
+    if (kvb) {
+      GemmParams pk = gp(rows, d, d, A.r2, d, false, Lw.theta_kv, d, false, A.k, d, false, EPI_STORE);
+      if ((rc = norm_into(pk, A.a, Lw.g_ttt, A.rstd2, A.r2, rows)) != TTT_OK) return rc;
+      if ((rc = gemm(pk)) != TTT_OK) return rc;
+    }
+    GemmParams p = gp(cn, ht, d, kvb ? A.k : A.r2, d, false, Lw.W1t, d, false, A.g, ht, false, EPI_GELU);
     p.batch = B; p.sA = (int64_t)cn * d; p.sD = (int64_t)cn * ht;
-    if ((rc = norm_into(p, A.a, Lw.g_ttt, A.rstd2, A.r2, rows)) != TTT_OK) return rc;
+    if (!kvb && (rc = norm_into(p, A.a, Lw.g_ttt, A.rstd2, A.r2, rows)) != TTT_OK) return rc;
     fast_operand(p, Lw.W1t_init, Lw.W1t, (int64_t)ht * d);
     p.Y = A.u; p.ldy = ht; p.sY = (int64_t)cn * ht;
     if ((rc = gemm(p)) != TTT_OK) return rc;
@@ -1449,14 +1458,12 @@ template <typename T> int Engine<T>::ttt_backward(int cn) {
 
 // Key-value-binding variant of the update (technical review §8, eq. (10); summary,
 // "Alternative Derivation"): every adaptive block j descends its own chunk loss
-// (1/b) sum_t ||W2t gelu(W1t k_t) - v_t||^2 with k = theta_K r2, v = theta_V r2 and r2
-// the normalised input of its MLP from this chunk's forward (W_{i-1}). Layer-wise: no
-// gradient passes between blocks, so each block's update reads only its own forward
-// rows and fast weights, and the order of the blocks does not matter. With e the
-// residual, de = (2/b) e, du = (de W2t) * gelu'(u), dW2t = de^T gelu(u), dW1t = du^T k.
-// The forward's MLP activations of the block are dead once its forward ran (no backward
-// reads them in this mode), so u and gelu(u) of the binding loss reuse them; k goes to
-// the attention-gradient buffer dob and the fp32 residual to G.
+// (1/b) sum_t ||g(k_t; W) - v_t||^2, g(k; W) = W2t gelu(W1t k), with k = theta_K r2 and
+// v = theta_V r2, r2 the block's normalised rows ahead of its MLP. The forward with
+// W_{i-1} already made the prediction: it is the MLP sub-layer's output m - a, with
+// u = W1t k and gelu(u) kept in the block's buffers. Layer-wise: no gradient passes
+// between blocks, so each block's update reads only its own rows and fast weights.
+// de = (2/b)(m - a - v), du = (de W2t) * gelu'(u), dW2t = de^T gelu(u), dW1t = du^T k.
 template <typename T> int Engine<T>::kvb_update(int cn) {
   const int rows = B * cn;
   int rc;
@@ -1464,29 +1471,21 @@ template <typename T> int Engine<T>::kvb_update(int cn) {
   for (int j = 0; j < Lt; ++j) {
     const LayerDev<T>& Lw = layers[first_ttt + j];
     BlockAct<T>& A = blk[j];
-    T* kb = dob;  // k = r2 theta_K^T  [rows][d]
-    // k (element type) and G = -(2/b) v (fp32): two products over the same rows
-    GemmParams pk = gp(rows, d, d, A.r2, d, false, Lw.theta_kv, d, false, kb, d, false, EPI_STORE);
+    // G = -(2/b) v
     GemmParams pv = gp(rows, d, d, A.r2, d, false, Lw.theta_kv + (size_t)d * d, d, false, G, d, true, EPI_STORE);
     pv.alpha = -two_over_b;
-    if ((rc = gemm2(pk, pv)) != TTT_OK) return rc;
-    // u = k W1t^T (kept in A.u), gelu(u) (in A.g), per sequence with W_{i-1}
-    GemmParams p = gp(cn, ht, d, kb, d, false, Lw.W1t, d, false, A.g, ht, false, EPI_GELU);
-    p.batch = B; p.sA = (int64_t)cn * d; p.sD = (int64_t)cn * ht;
-    fast_operand(p, Lw.W1t_init, Lw.W1t, (int64_t)ht * d);
-    p.Y = A.u; p.ldy = ht; p.sY = (int64_t)cn * ht;
-    if ((rc = gemm(p)) != TTT_OK) return rc;
-    // G = (2/b) (gelu(u) W2t^T - v) = de, in place over -(2/b) v
-    p = gp(cn, d, ht, A.g, ht, false, Lw.W2t, ht, false, G, d, true, EPI_RESID);
-    p.batch = B; p.sA = (int64_t)cn * ht; p.sD = (int64_t)cn * d;
-    fast_operand(p, Lw.W2t_init, Lw.W2t, (int64_t)d * ht);
-    p.X = G; p.ldx = d; p.sX = (int64_t)cn * d;
-    p.alpha = two_over_b;
-    if ((rc = gemm(p)) != TTT_OK) return rc;
-    convert_kernel<float, T><<<nblk((int64_t)rows * d, 256), 256, 0, st>>>(G, GT, (int64_t)rows * d);
+    if ((rc = gemm(pv)) != TTT_OK) return rc;
+    // G = (2/b)(m - a) + G = de (fp32), GT its element-type copy for the products below
+    const cudaError_t e = launch_pdl(kvb_residual_kernel<T>, dim3(nblk((int64_t)rows * d / 4, 256)), dim3(256), 0,
+                                     st, (const float*)A.m, (const float*)A.a, G, GT, two_over_b,
+                                     (int64_t)rows * d / 4);
+    if (e != cudaSuccess) {
+      poisoned = true;
+      return fail(this, TTT_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(e));
+    }
     TTT_LAUNCHED();
     // du = (de W2t) * gelu'(u)
-    p = gp(cn, ht, d, GT, d, false, Lw.W2t, ht, true, dhid, ht, false, EPI_DGELU);
+    GemmParams p = gp(cn, ht, d, GT, d, false, Lw.W2t, ht, true, dhid, ht, false, EPI_DGELU);
     p.batch = B; p.sA = (int64_t)cn * d; p.sD = (int64_t)cn * ht;
     fast_operand(p, Lw.W2t_init, Lw.W2t, (int64_t)d * ht);
     p.X = A.u; p.ldx = ht; p.sX = (int64_t)cn * ht;
@@ -1496,7 +1495,7 @@ template <typename T> int Engine<T>::kvb_update(int cn) {
     p2w.batch = B; p2w.sA = (int64_t)cn * d; p2w.sB = (int64_t)cn * ht; p2w.sD = (int64_t)d * ht;
     p2w.alpha = -cfg.eta;
     if (is_bf16) { p2w.Y = Lw.W2t; p2w.ldy = ht; p2w.sY = (int64_t)d * ht; }
-    GemmParams p1w = gp(ht, d, cn, dhid, ht, true, kb, d, true, Lw.W1t32, d, true, EPI_SGD);
+    GemmParams p1w = gp(ht, d, cn, dhid, ht, true, A.k, d, true, Lw.W1t32, d, true, EPI_SGD);
     p1w.batch = B; p1w.sA = (int64_t)cn * ht; p1w.sB = (int64_t)cn * d; p1w.sD = (int64_t)ht * d;
     p1w.alpha = -cfg.eta;
     if (is_bf16) { p1w.Y = Lw.W1t; p1w.ldy = d; p1w.sY = (int64_t)ht * d; }

@@ -43,8 +43,7 @@ def _direct_model_flops(cfg):
     if cfg.inner_loss == "kvb":                        # each block's binding loss only
         upd = 0.0
         for j in range(Lt):
-            upd += mm(T, d, d) + mm(T, d, d)                                   # k, v projections
-            upd += mm(T, cfg.ttt_hidden, d) + mm(T, d, cfg.ttt_hidden)         # g(k; W)
+            upd += mm(T, d, d) + mm(T, d, d)                                   # k (MLP input), v projections
             upd += mm(T, cfg.ttt_hidden, d)                                    # du = de W2t
             upd += mm(cfg.ttt_hidden, d, T) + mm(d, cfg.ttt_hidden, T)         # dW1t, dW2t
         return (fwd + upd) * cfg.batch
