@@ -61,6 +61,20 @@ Readings taken:
   K3 the recorded per-token losses are still the next-token losses of the
      model with the weights in force (the inner loss only drives the update).
 
+Outer-loop meta-gradient (technical review §4, eqs. (5)-(7) and §7 Algorithm 2;
+summary, "Outer Loop"): meta_gradient() differentiates the mean of the scored
+losses, L(W_0; X) = (1/N) sum_i A_i(W_{i-1}), with respect to the initial fast
+weights W_0 through the whole update trajectory, by eq. (7) as written. Reading:
+  M1 A_i and its Hessian are those the inner loop defines: the window cache of
+     earlier chunks is a constant (R3) in the outer derivative too, and the
+     static parameters phi stay fixed (eq. (7) suppresses their paths).
+  M2 T is a multiple of b (every scored loss belongs to a chunk that updates).
+The Hessian-vector products come from the complex-step derivative of the
+hand-written chunk gradient (Squire and Trapp, SIAM Review 40(1), 1998):
+H v = Im grad A(W + i h v) / h, exact up to rounding because that gradient is
+a real-analytic function of W. This is the only place where the oracle runs on
+complex arrays.
+
 Arithmetic is float64 throughout. Matrix products use numpy's matmul as the
 library primitive. Queries are processed in groups only to bound memory; each
 row is the plain definition. This oracle is pinned by the tests in
@@ -145,7 +159,7 @@ def window_attention(q, keys, vals, q_pos, k_pos, window, keep_probs=False, grou
     n, H, hd = q.shape
     scale = 1.0 / math.sqrt(hd)
     o = np.empty_like(q)
-    probs = np.empty((H, n, keys.shape[0])) if keep_probs else None
+    probs = np.empty((H, n, keys.shape[0]), dtype=np.result_type(q, keys)) if keep_probs else None
     k_pos = np.asarray(k_pos)
     for g0 in range(0, n, group):
         g1 = min(n, g0 + group)
@@ -436,6 +450,63 @@ class Oracle:
                     self._sgd(seq, grads)
                     seq.pend_inputs, seq.pend_targets = [], []
         return res
+
+    # --------------------------------------------------------------- outer loop (Algorithm 2)
+    def meta_gradient(self, tokens, step=1e-30):
+        """Outer-loop gradient for one sequence (tokens [T+1], T = N b; readings M1-M2).
+
+        Forward: Algorithm 1 from W_0 with the chunk gradients g_i = grad A_i(W_{i-1})
+        and the states W_{i-1} kept. Backward, eq. (7) accumulated from the last chunk:
+        lambda_N = g_N, lambda_i = g_i + (I - eta H_{A_i}(W_{i-1})) lambda_{i+1}
+        (H symmetric, so J^T products become this recursion); grad = lambda_1 / N.
+        The oracle's own state is not used or changed. Returns (L, grads) with grads
+        a list of {"W1t", "W2t"} per adaptive block.
+        """
+        cfg = self.cfg
+        assert getattr(cfg, "inner_loss", "e2e") == "e2e", "eq. (7) is written for the next-token inner loss"
+        tok = np.asarray(tokens)
+        T = tok.shape[0] - 1
+        b, eta = cfg.minibatch_b, cfg.eta
+        assert T > 0 and T % b == 0, "reading M2: T must be a multiple of b"
+        N = T // b
+        st = _Seq(cfg, self.w)
+        h = self._frozen_forward(st, tok[:T], 0, commit=True)
+        Ws, gs, means = [], [], []
+        for i in range(N):
+            c0 = i * b
+            Ws.append([{n: W.copy() for n, W in f.items()} for f in st.fast])
+            losses, grads = self._chunk(st, h[c0:c0 + b], c0, tok[c0 + 1:c0 + b + 1], need_grad=True, commit=True)
+            means.append(float(np.mean(losses)))
+            gs.append(grads)
+            self._sgd(st, grads)
+
+        def hvp(i, v):
+            # H_{A_i}(W_{i-1}) v by the complex step; chunk i reads the cache of positions < i b
+            c0 = i * b
+            st.fast = [{n: Ws[i][j][n] + 1j * step * v[j][n] for n in ("W1t", "W2t")} for j in range(cfg.n_ttt)]
+            _, gc = self._chunk(st, h[c0:c0 + b], c0, tok[c0 + 1:c0 + b + 1], need_grad=True, commit=False)
+            return [{n: np.imag(gc[j][n]) / step for n in ("W1t", "W2t")} for j in range(cfg.n_ttt)]
+
+        lam = [{n: G.copy() for n, G in g.items()} for g in gs[N - 1]]
+        for i in range(N - 2, -1, -1):
+            hv = hvp(i, lam)
+            lam = [{n: gs[i][j][n] + lam[j][n] - eta * hv[j][n] for n in ("W1t", "W2t")} for j in range(cfg.n_ttt)]
+        return float(np.mean(means)), [{n: G / N for n, G in g.items()} for g in lam]
+
+    def chunk_hvp(self, seq, tokens_chunk, v, step=1e-30):
+        """H v of the next full chunk's mean loss at the current fast weights (the
+        complex-step product used by meta_gradient), without changing any state."""
+        st = self.seqs[seq]
+        cfg = self.cfg
+        assert len(tokens_chunk) == cfg.minibatch_b + 1 and not st.pend_inputs
+        h = self._frozen_forward(st, tokens_chunk[:-1], st.n_pos, commit=False)
+        saved = st.fast
+        st.fast = [{n: saved[j][n] + 1j * step * v[j][n] for n in ("W1t", "W2t")} for j in range(cfg.n_ttt)]
+        try:
+            _, gc = self._chunk(st, h, st.n_pos, tokens_chunk[1:], need_grad=True, commit=False)
+        finally:
+            st.fast = saved
+        return [{n: np.imag(gc[j][n]) / step for n in ("W1t", "W2t")} for j in range(cfg.n_ttt)]
 
     # --------------------------------------------------------------- inspection
     def fast_weights(self, seq, j):

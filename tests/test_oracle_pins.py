@@ -505,3 +505,116 @@ def test_kvb_teacher_forced_decode_equals_prefill():
     np.testing.assert_allclose(np.concatenate([lp, r["losses"]], axis=1), lf, rtol=1e-10, atol=1e-12)
     for j in range(cfg.n_ttt):
         np.testing.assert_allclose(dec.fast_weights(0, j)[0], full.fast_weights(0, j)[0], rtol=1e-10, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- outer-loop meta-gradient
+
+def _outer_loss(cfg, w, toks):
+    return float(np.mean(Oracle(cfg, w).prefill(toks)[0]))
+
+
+def _with_initial_fast(cfg, w, delta, scale):
+    w2 = dict(w)
+    for j in range(cfg.n_ttt):
+        l = cfg.first_ttt + j
+        for n in ("W1t", "W2t"):
+            w2[f"layers.{l}.{n}"] = w[f"layers.{l}.{n}"].astype(np.float64) + scale * delta[j][n]
+    return w2
+
+
+def test_meta_gradient_matches_finite_differences_of_the_outer_loss():
+    """Eq. (7) of the technical review (§4) against central differences of the scored
+    mean loss L(W_0) = mean of Algorithm 1's losses, along random directions. One
+    adaptive block: its keys/values do not depend on W, so eq. (7) is the whole
+    derivative. Negative control: dropping the -eta H term (the first-order
+    approximation eq. (6) warns against) misses far outside the tolerance."""
+    cfg = tiny(n_ttt=1, T=16)
+    w = weights(cfg)
+    toks = tokens(cfg)
+    orc = Oracle(cfg, w)
+    L, grad = orc.meta_gradient(toks[0])
+    assert L == pytest.approx(_outer_loss(cfg, w, toks), rel=1e-12)
+    first_order = [{n: np.zeros_like(g[n]) for n in g} for g in grad]
+    st = Oracle(cfg, w)
+    b, N = cfg.minibatch_b, cfg.T // cfg.minibatch_b
+    for i in range(N):                    # (1/N) sum_i grad A_i(W_{i-1}) along the same trajectory
+        _, g = st.chunk_loss_and_grad(0, toks[0, i * b:(i + 1) * b + 1])
+        for j in range(cfg.n_ttt):
+            for n in g[j]:
+                first_order[j][n] += g[j][n] / N
+        st.prefill(toks[:, i * b:(i + 1) * b + 1])
+    rng = np.random.default_rng(3)
+    eps = 1e-5
+    for _ in range(3):
+        v = [{n: rng.standard_normal(grad[j][n].shape) for n in grad[j]} for j in range(cfg.n_ttt)]
+        fd = (_outer_loss(cfg, _with_initial_fast(cfg, w, v, eps), toks)
+              - _outer_loss(cfg, _with_initial_fast(cfg, w, v, -eps), toks)) / (2 * eps)
+        dot = sum(float(np.sum(grad[j][n] * v[j][n])) for j in range(cfg.n_ttt) for n in v[j])
+        fo = sum(float(np.sum(first_order[j][n] * v[j][n])) for j in range(cfg.n_ttt) for n in v[j])
+        assert dot == pytest.approx(fd, rel=1e-6, abs=1e-8)
+        assert abs(fo - fd) > 1e-3 * abs(fd)
+
+
+@pytest.mark.parametrize("n_ttt,b,k,T", [(1, 4, 4, 16), (2, 4, 6, 16), (3, 3, 5, 12)])
+def test_meta_gradient_matches_autograd_through_the_unrolled_updates(n_ttt, b, k, T):
+    """Eq. (7) against the library's reverse-over-reverse (tests/torch_static.py:
+    create_graph through every inner gradient, earlier keys/values detached as the
+    inner loop holds them, reading M1), for 1-3 adaptive blocks and 4 chunks."""
+    cfg = tiny(n_ttt=n_ttt, minibatch_b=b, window_k=k, T=T)
+    w = weights(cfg)
+    toks = tokens(cfg)
+    L, grad = Oracle(cfg, w).meta_gradient(toks[0])
+    Lr, ref = TS.outer_gradient_chunked(cfg, w, toks[0])
+    assert L == pytest.approx(Lr, rel=1e-12)
+    for j in range(n_ttt):
+        for n in ("W1t", "W2t"):
+            np.testing.assert_allclose(grad[j][n], ref[j][n].numpy(), rtol=1e-9, atol=1e-12)
+
+
+def test_meta_gradient_with_eta_zero_is_the_static_model_gradient():
+    """eta = 0: every J_i is the identity and every W_i = W_0, so eq. (7) reduces to the
+    gradient of the static model's mean loss (autograd of the whole-sequence forward).
+    One adaptive block, so that no key or value the whole-sequence autograd
+    differentiates depends on W (with two, it would also follow the second block's
+    earlier keys, which reading M1 holds constant)."""
+    cfg = tiny(n_ttt=1, T=16, eta=0.0)
+    w = weights(cfg)
+    toks = tokens(cfg)
+    _, grad = Oracle(cfg, w).meta_gradient(toks[0])
+    fast = TS.initial_fast(cfg, w, requires_grad=True)
+    TS.static_forward(cfg, w, toks[0], fast=fast).mean().backward()
+    for j in range(cfg.n_ttt):
+        for n in ("W1t", "W2t"):
+            np.testing.assert_allclose(grad[j][n], fast[j][n].grad.numpy(), rtol=1e-10, atol=1e-13)
+
+
+@pytest.mark.parametrize("n_ttt", [1, 2])
+def test_complex_step_hessian_vector_product_matches_finite_differences(n_ttt):
+    """The Hessian-vector product used by eq. (7), on chunk 3 (window cache non-empty),
+    against central differences of the hand-written chunk gradient."""
+    cfg = tiny(n_ttt=n_ttt, T=8)
+    w = weights(cfg)
+    toks = tokens(cfg, n=cfg.T + 1 + cfg.minibatch_b)
+    orc = Oracle(cfg, w)
+    orc.prefill(toks[:, :cfg.T + 1])
+    chunk = toks[0, cfg.T:cfg.T + cfg.minibatch_b + 1]
+    rng = np.random.default_rng(5)
+    fast = orc.seqs[0].fast
+    v = [{n: rng.standard_normal(fast[j][n].shape) for n in ("W1t", "W2t")} for j in range(n_ttt)]
+    hv = orc.chunk_hvp(0, chunk, v)
+    eps = 1e-5
+
+    def grad_at(scale):
+        saved = [{n: W.copy() for n, W in f.items()} for f in fast]
+        for j in range(n_ttt):
+            for n in ("W1t", "W2t"):
+                fast[j][n] = saved[j][n] + scale * v[j][n]
+        g = orc.chunk_loss_and_grad(0, chunk)[1]
+        for j in range(n_ttt):
+            fast[j].update(saved[j])
+        return g
+
+    gp, gm = grad_at(eps), grad_at(-eps)
+    for j in range(n_ttt):
+        for n in ("W1t", "W2t"):
+            np.testing.assert_allclose(hv[j][n], (gp[j][n] - gm[j][n]) / (2 * eps), rtol=1e-5, atol=1e-7)

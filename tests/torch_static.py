@@ -293,3 +293,51 @@ def mini_batch_ttt_kvb_chunked(cfg, weights, tokens, layerwise=True, output_from
             k_cache[j] = torch.cat([k_cache[j], new[j][0]])
             v_cache[j] = torch.cat([v_cache[j], new[j][1]])
     return losses, fast
+
+
+# ----------------------------------------------------------------------------- outer loop (meta-gradient)
+
+def outer_gradient_chunked(cfg, weights, tokens):
+    """The outer objective L(W_0) = (1/N) sum_i A_i(W_{i-1}) and its gradient w.r.t. the
+    initial fast weights, by autograd through the unrolled inner updates.
+
+    Chunk by chunk as mini_batch_ttt_chunked (earlier chunks' keys/values detached, as
+    the inner loop holds them), but the update keeps the graph: each inner gradient is
+    taken with create_graph=True, W_i = W_{i-1} - eta * grad, and the final backward
+    differentiates through every step (the library's reverse-over-reverse).
+    Returns (L, [{"W1t", "W2t"} per adaptive block]).
+    """
+    w = {k: _t(v) for k, v in weights.items()}
+    tok = torch.as_tensor(tokens, dtype=torch.long)
+    T = tok.shape[0] - 1
+    H, hd = cfg.n_heads, cfg.d // cfg.n_heads
+    b, first = cfg.minibatch_b, cfg.n_layers - cfg.n_ttt
+    assert T % b == 0
+    x0 = _frozen_stack(cfg, w, tok[:T], torch.arange(T))
+    w0 = initial_fast(cfg, weights, requires_grad=True)
+    fast = w0
+    k_cache = [torch.zeros(0, H, hd, dtype=torch.float64) for _ in range(cfg.n_ttt)]
+    v_cache = [torch.zeros(0, H, hd, dtype=torch.float64) for _ in range(cfg.n_ttt)]
+    total = torch.zeros((), dtype=torch.float64)
+    for c0 in range(0, T, b):
+        c1 = c0 + b
+        lo = max(0, c0 - cfg.window_k + 1)
+        x = x0[c0:c1]
+        pos = torch.arange(c0, c1)
+        new = []
+        for j in range(cfg.n_ttt):
+            x, k, v, _ = _adaptive_layer(cfg, w, first + j, fast[j], x, pos, k_cache[j][lo:c0], v_cache[j][lo:c0],
+                                         torch.arange(lo, c0))
+            new.append((k.detach(), v.detach()))
+        rf = F.rms_norm(x, (cfg.d,), weight=w["final_norm"], eps=cfg.rms_eps)
+        A = F.cross_entropy(rf @ w["E"].T, tok[c0 + 1:c1 + 1], reduction="mean")
+        total = total + A
+        params = [f[n] for f in fast for n in ("W1t", "W2t")]
+        grads = iter(torch.autograd.grad(A, params, create_graph=True))
+        fast = [{n: f[n] - cfg.eta * next(grads) for n in ("W1t", "W2t")} for f in fast]
+        for j in range(cfg.n_ttt):
+            k_cache[j] = torch.cat([k_cache[j], new[j][0]])
+            v_cache[j] = torch.cat([v_cache[j], new[j][1]])
+    L = total / (T // b)
+    g = iter(torch.autograd.grad(L, [f[n] for f in w0 for n in ("W1t", "W2t")]))
+    return float(L.detach()), [{n: next(g) for n in ("W1t", "W2t")} for _ in w0]
