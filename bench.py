@@ -376,7 +376,10 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600), device_id=device)
     import long_context_prefill_ttt_b200 as T
 
-    cfg = syn.config(args.workload, **({"T": args.T} if args.T else {}))
+    over = {"T": args.T} if args.T else {}
+    if args.inner_loss == "kvb":  # the variant as the measured workload (e.g. for its launch list)
+        over.update(inner_loss="kvb", eta=args.kvb_eta)
+    cfg = syn.config(args.workload, **over)
     w = syn.make_weights(cfg)
     wd = {k: torch.from_numpy(v).to(device) for k, v in w.items()}
     del w
@@ -483,7 +486,7 @@ def run_ours(args):
         comparator = run_full_attention(cfg, tok_dev, args, device)
         comparator["ttt_e2e_speedup"] = value / comparator["tokens_per_s"]
     kvb = None
-    if args.kvb and rank == 0 and ws == 1 and cfg.n_ttt > 0:
+    if args.kvb and rank == 0 and ws == 1 and cfg.n_ttt > 0 and cfg.inner_loss == "e2e":
         if h is not None:
             del h
             torch.cuda.empty_cache()
@@ -499,7 +502,8 @@ def run_ours(args):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"{cfg.name}: V{cfg.vocab} d{cfg.d} L{cfg.n_layers} (last {cfg.n_ttt} adaptive) "
                                f"H{cfg.n_heads} h{cfg.mlp_hidden} ({cfg.ttt_hidden}+{cfg.static_hidden}) "
-                               f"k{cfg.window_k} b{cfg.minibatch_b} T{cfg.T} B{cfg.batch}",
+                               f"k{cfg.window_k} b{cfg.minibatch_b} T{cfg.T} B{cfg.batch}"
+                               + (f", key-value-binding inner loss (eta {cfg.eta})" if cfg.inner_loss == "kvb" else ""),
                    "tokens_per_step_per_gpu": cfg.batch * cfg.T, "parallelism": f"replicas x{ws}",
                    "device_bytes": dev_bytes,
                    "l2": "no flush: every step streams > 2.5 GB of weights and GBs of activations (L2 126 MB)"},
@@ -563,6 +567,8 @@ def main():
                     help="skip the key-value-binding variant beside the metric")
     ap.add_argument("--kvb-steps", type=int, default=2)
     ap.add_argument("--kvb-eta", type=float, default=1e-4)
+    ap.add_argument("--inner-loss", default="e2e", choices=["e2e", "kvb"],
+                    help="inner loss of the measured workload (kvb: the key-value-binding variant)")
     ap.add_argument("--profile-steps", type=int, default=1,
                     help="steps of the separate instrumented pass that gives the per-class profile")
     ap.add_argument("--no-batched", dest="batched", action="store_false",
