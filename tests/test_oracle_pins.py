@@ -618,3 +618,35 @@ def test_complex_step_hessian_vector_product_matches_finite_differences(n_ttt):
     for j in range(n_ttt):
         for n in ("W1t", "W2t"):
             np.testing.assert_allclose(hv[j][n], (gp[j][n] - gm[j][n]) / (2 * eps), rtol=1e-5, atol=1e-7)
+
+
+def test_meta_gradient_of_a_single_chunk_is_its_inner_gradient():
+    """b = T: one chunk, scored with W_0 and never followed by a loss of W_1, so eq. (7)
+    is grad A_1(W_0), the chunk gradient of the inner loop."""
+    cfg = tiny(n_ttt=2, T=8, minibatch_b=8, window_k=8)
+    w = weights(cfg)
+    toks = tokens(cfg)
+    L, grad = Oracle(cfg, w).meta_gradient(toks[0])
+    mean, g = Oracle(cfg, w).chunk_loss_and_grad(0, toks[0])
+    assert L == pytest.approx(mean, rel=1e-14)
+    for j in range(cfg.n_ttt):
+        for n in ("W1t", "W2t"):
+            np.testing.assert_allclose(grad[j][n], g[j][n], rtol=1e-12, atol=1e-15)
+
+
+def test_reading_m1_differs_from_the_total_derivative_with_two_adaptive_blocks():
+    """With two adaptive blocks the second block's cached keys/values depend on W_0
+    through the first block, so the total derivative of L (central differences)
+    differs from eq. (7) under reading M1, where the cache is a constant as in the
+    inner gradient: the reading is a real choice, not a restatement."""
+    cfg = tiny(n_ttt=2, T=16)
+    w = weights(cfg)
+    toks = tokens(cfg)
+    _, grad = Oracle(cfg, w).meta_gradient(toks[0])
+    v = [{n: np.random.default_rng(3 + j).standard_normal(grad[j][n].shape) for n in grad[j]}
+         for j in range(cfg.n_ttt)]
+    eps = 1e-5
+    fd = (_outer_loss(cfg, _with_initial_fast(cfg, w, v, eps), toks)
+          - _outer_loss(cfg, _with_initial_fast(cfg, w, v, -eps), toks)) / (2 * eps)
+    dot = sum(float(np.sum(grad[j][n] * v[j][n])) for j in range(cfg.n_ttt) for n in v[j])
+    assert abs(dot - fd) > 1e-3 * abs(fd)
