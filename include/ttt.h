@@ -133,8 +133,9 @@ int ttt_prefill(ttt_handle* h, const int32_t* tokens, int64_t T, float* out_loss
  * token, takes the argmax of the logits (lowest id on ties) — or, when forced
  * is non-NULL, the id forced[b][t] — writes it to out_tokens[b][t] and
  * -log p(chosen) to out_losses[b][t] (may be NULL). When a chunk of b
- * positions completes, its mean loss is differentiated and W updated
- * (summary, "Decoding Multiple Tokens"). forced/out_* use ptr_kind. */
+ * positions completes, its inner loss (the chunk's mean next-token loss, or
+ * with TTT_LOSS_KVB each adaptive block's binding loss) is differentiated and
+ * W updated (summary, "Decoding Multiple Tokens"). forced/out_* use ptr_kind. */
 int ttt_decode(ttt_handle* h, int64_t n, const int32_t* forced, int32_t* out_tokens, float* out_losses,
                int32_t ptr_kind);
 

@@ -89,3 +89,32 @@ def test_kvb_bf16_matches_oracle(T, name, overrides):
     P.compare(cfg, r["w"], r["gpu_losses"], r["orc_losses"], r["gpu_w"], r["orc_w"], report=rep)
     print(name, "kvb", rep)
     assert rep["dw"] <= 5e-2
+
+
+def test_kvb_m125_decode_bf16_greedy_matches_oracle(T):
+    """bf16 decode of the variant on the ~125M architecture (chunks of 256, window 512, so
+    that the oracle finishes in about half a minute): each token step normalises the
+    block's rows inside the few-row key-projection product; 300 tokens after a
+    256-position prefix complete a chunk, whose binding update runs from the decoded
+    tokens. The oracle is teacher-forced on the GPU's tokens (near-ties may flip under
+    bf16); each GPU token must be within delta of the oracle's best logit, then losses
+    and weights are compared at the bf16 tolerances."""
+    cfg = syn.config("m125_decode_bf16", T=256, batch=1, minibatch_b=256, window_k=512, inner_loss="kvb",
+                     eta=3e-3)
+    w = syn.make_weights(cfg)
+    toks = syn.make_token_batch(cfg)
+    h = T.ttt_create(cfg, w)
+    T.ttt_prefill(h, toks)
+    n = 300
+    gtok, gloss = T.ttt_decode(h, n)
+    orc = Oracle(cfg, w)
+    orc.prefill(toks)
+    r = orc.decode(n, forced=gtok)
+    delta = 2e-2 * np.maximum(1.0, np.abs(r["z_max"]))
+    assert np.all(r["z_chosen"] >= r["z_max"] - delta)
+    assert float(np.max(np.abs(gloss - r["losses"]) / np.abs(r["losses"]))) <= 2e-2
+    for s in range(cfg.batch):
+        for j in range(cfg.n_ttt):
+            g1, g2 = T.ttt_get_weights(h, s, j)
+            o1, o2 = orc.fast_weights(s, j)
+            assert P.rel_fro(g1, o1) <= 5e-3 and P.rel_fro(g2, o2) <= 5e-3
