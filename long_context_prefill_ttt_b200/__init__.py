@@ -202,6 +202,8 @@ def make_config(cfg, stream=None, max_segment=0) -> ttt_config:
     c.dtype = TTT_BF16 if dt in ("bf16", TTT_BF16) else TTT_FP32
     c.max_segment = int(max_segment or _get(cfg, "max_segment", 0) or 0)
     loss = _get(cfg, "inner_loss", "e2e")
+    if loss not in ("e2e", "kvb", TTT_LOSS_E2E, TTT_LOSS_KVB):
+        raise ValueError(f"inner_loss must be 'e2e' or 'kvb', not {loss!r}")
     c.inner_loss = TTT_LOSS_KVB if loss in ("kvb", TTT_LOSS_KVB) else TTT_LOSS_E2E
     c.cuda_stream = _stream_ptr(stream).value
     return c

@@ -70,6 +70,8 @@ def test_create_rejects_an_unknown_inner_loss():
     import long_context_prefill_ttt_b200 as T
     c = T.make_config(syn.config("tiny_fp32"))
     c.inner_loss = 2
+    with pytest.raises(ValueError):
+        T.make_config(syn.config("tiny_fp32", inner_loss="KVB"))
     out = ctypes.c_void_p()
     w = T.ttt_weights()
     assert T.lib.ttt_create(ctypes.byref(c), ctypes.byref(w), ctypes.byref(out)) == T.TTT_ERR_INVALID_ARG
