@@ -180,7 +180,10 @@ def run_reference(args):
     dist, rank, local, ws = _dist()
     if rank != 0:
         return 0
-    cfg = syn.config(args.workload, **({"T": args.T} if args.T else {}))
+    over = {"T": args.T} if args.T else {}
+    if args.inner_loss == "kvb":
+        over.update(inner_loss="kvb", eta=args.kvb_eta)
+    cfg = syn.config(args.workload, **over)
     per_step = []
     for _ in range(args.warmup):
         pass  # the oracle has no warm-up state; each step is a fresh bounded sample
@@ -494,6 +497,9 @@ def run_ours(args):
         try:
             kvb = run_kvb_variant(cfg, tok_dev, args, device, peaks)
             kvb["ttt_e2e_s_per_1k_tokens"] = (ms_max / args.steps) / 1e3 / (cfg.batch * cfg.T / 1e3)
+            if args.cpu_baseline:  # the oracle of the variant on a bounded sample, beside it
+                kvb["cpu_baseline"] = cpu_baseline(cfg.replace(inner_loss="kvb", eta=args.kvb_eta),
+                                                   n_tokens=args.ref_tokens)
         except Exception as ex:  # the metric above stands without it
             kvb = {"error": f"{type(ex).__name__}: {ex}"}
     line = {
