@@ -68,6 +68,19 @@ def model_flops(cfg, T=None, B=None):
     return B * (fwd + bwd)
 
 
+def decode_bytes_per_step(cfg, pos):
+    """Least HBM bytes one decode token step reads at position pos (bf16): every frozen
+    weight once (E, attention, frozen and static MLPs, the shared W_init), each
+    sequence's bf16 fast-weight update copies, and each sequence's window of keys and
+    values in every layer (min(pos + 1, k) positions)."""
+    d, V, L, Lt = cfg.d, cfg.vocab, cfg.n_layers, cfg.n_ttt
+    h, ht, hs, B = cfg.mlp_hidden, cfg.ttt_hidden, cfg.static_hidden, cfg.batch
+    frozen = V * d + L * 4 * d * d + (L - Lt) * 2 * d * h + Lt * 2 * d * (hs + ht)
+    fast = B * Lt * 2 * d * ht
+    kv = B * L * 2 * min(pos + 1, cfg.window_k) * d
+    return 2 * (frozen + fast + kv)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -202,9 +215,12 @@ def run_reference(args):
     return 0
 
 
-def run_decode(T, args, device):
+def run_decode(T, args, device, peaks):
     """Decode on the ~125M architecture: prefill a prefix, then greedy tokens with an
-    update after every b decoded tokens (review Alg. 3). Reported beside the metric."""
+    update after every b decoded tokens (review Alg. 3). Reported beside the metric, as
+    tokens/s, as a fraction of the bf16 peak in model FLOPs (the forward of every decoded
+    position and the update of every completed chunk: the prefill count of the decoded
+    positions) and as a fraction of HBM bandwidth (decode_bytes_per_step)."""
     import torch
     cfg = syn.config("m125_decode_bf16", **({"T": args.decode_prefix} if args.decode_prefix else {}))
     n = args.decode_n or cfg.decode_n
@@ -222,9 +238,16 @@ def run_decode(T, args, device):
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1)
     launches = T.ttt_last_launch_count(h)
+    flops = model_flops(cfg, T=cfg.T + n) - model_flops(cfg, T=cfg.T)
+    nbytes = float(sum(decode_bytes_per_step(cfg, cfg.T + i) for i in range(n)))
     return {"tokens_per_s": cfg.batch * n / (ms / 1e3), "ms_per_token_step": ms / n, "batch": cfg.batch,
             "prefix": cfg.T, "n": n, "updates": (cfg.T + n) // cfg.minibatch_b - cfg.T // cfg.minibatch_b,
-            "gpu_launches": launches}
+            "gpu_launches": launches,
+            "model_flops": {"tflop": flops / 1e12, "achieved_tflops": flops / (ms / 1e3) / 1e12,
+                            "frac_of_peak": flops / (ms / 1e3) / 1e12 / peaks["bf16"]},
+            "hbm": {"bytes_per_token_step": nbytes / n, "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
+                    "peak_gbs": peaks["hbm"], "frac": nbytes / (ms / 1e3) / 1e9 / peaks["hbm"],
+                    "floor_ms_per_token_step": nbytes / n / (peaks["hbm"] * 1e9) * 1e3}}
 
 
 def _time_prefill(T, h, tok, loss, steps, warmup, check=True):
@@ -471,7 +494,7 @@ def run_ours(args):
     dev_bytes = T.ttt_device_bytes(h)
     decode = None
     if args.decode and rank == 0 and ws == 1:
-        decode = run_decode(T, args, device)
+        decode = run_decode(T, args, device, peaks)
     batched = None
     if args.batched and rank == 0 and ws == 1:
         batched = run_batched_prefill(T, args, device, peaks)

@@ -118,3 +118,20 @@ def test_reference_arm_prints_once_from_rank_zero(rank):
         assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
     else:
         assert lines == []
+
+
+def test_decode_accounting_of_the_125m_decode_workload():
+    """Decode's model FLOPs per decoded token (forward of the position plus its share of
+    the chunk update) and its least HBM bytes per token step, assembled tensor by tensor:
+    weights once, each sequence's bf16 fast-weight copies, each sequence's windows."""
+    cfg = syn.config("m125_decode_bf16")
+    n = cfg.decode_n
+    per_token = (bench.model_flops(cfg, T=cfg.T + n) - bench.model_flops(cfg, T=cfg.T)) / (cfg.batch * n)
+    assert per_token / 1e9 == pytest.approx(0.295 + 0.114, rel=5e-3)
+    d, L, Lt, B = cfg.d, cfg.n_layers, cfg.n_ttt, cfg.batch
+    tensors = [cfg.vocab * d] + [d * d] * 4 * L + [cfg.mlp_hidden * d] * 2 * (L - Lt) + \
+        [cfg.static_hidden * d] * 2 * Lt + [cfg.ttt_hidden * d] * 2 * Lt
+    fast = [cfg.ttt_hidden * d] * 2 * Lt * B
+    windows = [cfg.window_k * d] * 2 * L * B
+    assert bench.decode_bytes_per_step(cfg, cfg.T) == 2 * (sum(tensors) + sum(fast) + sum(windows))
+    assert bench.decode_bytes_per_step(cfg, 9) == 2 * (sum(tensors) + sum(fast) + 10 * d * 2 * L * B)
