@@ -511,6 +511,9 @@ def run_ours(args):
         h = None
         comparator = run_full_attention(cfg, tok_dev, args, device)
         comparator["ttt_e2e_speedup"] = value / comparator["tokens_per_s"]
+        # the pages' own figure, for context only (another model on another GPU)
+        comparator["pages_figure"] = {"ttt_e2e_speedup": 2.7, "context": "128K", "hardware": "1x H100",
+                                      "model": "3B", "source": "b-lab.team summary, Results; abstract"}
     kvb = None
     if args.kvb and rank == 0 and ws == 1 and cfg.n_ttt > 0 and cfg.inner_loss == "e2e":
         if h is not None:
