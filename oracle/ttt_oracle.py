@@ -46,7 +46,9 @@ Variant with the layer-wise key-value-binding inner loss (cfg.inner_loss ==
 "kvb"; technical review §8, eq. (10); summary, "Alternative Derivation
 (Connection to TTT-KVB)"): each adaptive block's fast weights W = (W1t, W2t)
 fit g(theta_K x_t; W) to theta_V x_t instead of descending the next-token loss.
-Readings taken:
+The model is otherwise the one above (adaptive MLPs in the last quarter of the
+blocks); the pages' own TTT-KVB models used multi-head LoRA MLPs in every layer,
+whose shapes they do not give. Readings taken:
   K1 x_t is the block's RMSNorm output r2 ahead of its adaptive MLP, and
      g(k; W) = W2t gelu(W1t k) is the adaptive two-layer MLP; theta_K, theta_V are
      frozen d x d matrices of the block. Output rule: the sub-layer's output is the
