@@ -12,6 +12,11 @@ span-copy tokens, N(0, 0.02) weights), resident in HBM for `value`; `e2e`
 passes pinned host buffers through the same C-ABI call (H2D of the tokens and
 D2H of the losses inside the timed region).
 
+Beside the metric (rank 0, one GPU): decode on the ~125M architecture with its
+model-FLOP and HBM fractions, the batched ~125M prefill, the fixed-128K-tokens
+sweep, the full-attention comparator, and the key-value-binding variant of the
+same workload with its own bounded oracle sample (--no-* flags skip each).
+
 Multi-GPU: replicas only (each rank runs its own independent sequence batch,
 no data-path collective; the path's chain W_{i-1} -> W_i is serial), time =
 max over ranks; value = tokens of all ranks / that time.
